@@ -1,0 +1,337 @@
+"""Pins of the fp64 oracle against facts fixed by the definitions and the mathematics (CPU only).
+
+Each test names what it pins and which plausible mistake it would catch.  Sources: RoLA
+("3 Preliminary" 3D RoPE and eq. (1) relative property; "4.1" block-sparse + low-rank branches;
+"4.2" rank-truncated rotary schedule; "4.3"/"B.1" RoPE outside the activation, one query-independent
+sum; "B.2" geometric rotary schedule) and RoPeSLR's appendix on 3D RoPE (base 10000).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from tests import brute
+from sparse_rank_hybrid_b200 import inputs as I
+from sparse_rank_hybrid_b200 import workloads as W
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(path):
+    with open(path) as f:
+        return [l.split() for l in f if l.strip() and not l.startswith("#")]
+
+
+# ----------------------------------------------------------------------------------------- RoPE
+def test_rope_split_golden(oracle_mod):
+    """Pairs per axis match the Wan 44/42/42 split (D=128) and the same rule at D=64."""
+    for D, pt, ph, pw in _rows(os.path.join(GOLD, "rope_split.txt")):
+        axis, _ = oracle_mod.rope_pairs(int(D))
+        assert [int((axis == a).sum()) for a in range(3)] == [int(pt), int(ph), int(pw)]
+        # native order: all t pairs, then h, then w
+        assert np.all(np.diff(axis) >= 0)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_rope_frequencies_geometric_base(oracle_mod, D):
+    """Per axis: first frequency 1, constant ratio (geometric, RoLA B.2), and p_a steps of the ratio
+    divide by exactly the base 10000 (RoFormer schedule theta^(-2m/d_a)).  Catches a wrong exponent
+    width (D instead of d_a), an off-by-one in m, or a wrong base."""
+    axis, omega = oracle_mod.rope_pairs(D, theta=1e4)
+    for a in range(3):
+        w = omega[axis == a]
+        p = w.size
+        assert w[0] == 1.0
+        ratio = w[1:] / w[:-1]
+        assert np.allclose(ratio, ratio[0], rtol=1e-13)
+        assert math.isclose(ratio[0] ** p, 1e-4, rel_tol=1e-12)
+
+
+def test_rope_axis_isolation(oracle_mod):
+    """With a grid that is 1 long on an axis, that axis' pairs are untouched; with the other two axes
+    flat, only that axis' pairs move.  Catches a wrong pair->axis assignment or a wrong token->(t,h,w)
+    decomposition."""
+    rng = np.random.default_rng(0)
+    D = 128
+    axis, _ = oracle_mod.rope_pairs(D)
+    for a, grid in enumerate([(1, 5, 7), (5, 1, 7), (5, 7, 1)]):
+        L = grid[0] * grid[1] * grid[2]
+        x = rng.standard_normal((L, D))
+        y = oracle_mod.rope_rows(x, grid, D // 2)
+        pairs = np.where(axis == a)[0]
+        cols = np.sort(np.concatenate([2 * pairs, 2 * pairs + 1]))
+        assert np.array_equal(y[:, cols], x[:, cols])
+    for a, grid in enumerate([(9, 1, 1), (1, 9, 1), (1, 1, 9)]):
+        x = rng.standard_normal((9, D))
+        y = oracle_mod.rope_rows(x, grid, D // 2)
+        moved = np.where(np.any(y != x, axis=0))[0] // 2
+        assert set(np.unique(moved)) <= set(np.where(axis == a)[0])
+
+
+def test_rope_position_closed_form(oracle_mod):
+    """A unit vector in the first pair of an axis (frequency 1) at token (t, h, w) ends at angle
+    t (resp. h, w): cos/sin of the integer position, counter-clockwise.  Catches a sign flip of sin,
+    a swapped pair layout, or a wrong row-major decomposition."""
+    D = 64
+    grid = (3, 4, 5)
+    axis, _ = oracle_mod.rope_pairs(D)
+    first = [int(np.where(axis == a)[0][0]) for a in range(3)]
+    L = 60
+    x = np.zeros((L, D))
+    for j in first:
+        x[:, 2 * j] = 1.0
+    y = oracle_mod.rope_rows(x, grid, D // 2)
+    for n in range(L):
+        t, h, w = n // 20, (n // 5) % 4, n % 5
+        for a, p in zip(range(3), (t, h, w)):
+            j = first[a]
+            assert math.isclose(y[n, 2 * j], math.cos(p), abs_tol=1e-15)
+            assert math.isclose(y[n, 2 * j + 1], math.sin(p), abs_tol=1e-15)
+
+
+def test_rope_matches_complex_rotation(oracle_mod):
+    """2x2 rotation == complex multiplication by exp(i angle) (independent formulation), including a
+    position offset and a truncated rotation (npairs < D/2)."""
+    rng = np.random.default_rng(1)
+    D, grid, off = 128, (3, 6, 7), (2, -3, 5)
+    L = 126
+    x = rng.standard_normal((L, D))
+    axis, omega = oracle_mod.rope_pairs(D)
+    pos = brute.grid_positions(grid, off)
+    for npairs in (D // 2, 16, 32):
+        y = oracle_mod.rope_rows(x, grid, npairs, offset=off)
+        yb = brute.rope_complex(x, pos, axis, omega, npairs)
+        assert np.allclose(y, yb, rtol=0, atol=1e-13)
+
+
+def test_rope_orthogonal_and_relative(oracle_mod):
+    """Rotations preserve norms, and q^(p) . k^(p') depends only on p - p' (RoLA eq. (1))."""
+    rng = np.random.default_rng(2)
+    D, grid = 128, (4, 5, 6)
+    L = 120
+    q = rng.standard_normal((L, D))
+    k = rng.standard_normal((L, D))
+    qh = oracle_mod.rope_rows(q, grid, D // 2)
+    assert np.allclose(np.linalg.norm(qh, axis=1), np.linalg.norm(q, axis=1), rtol=1e-13)
+    s0 = oracle_mod.rope_rows(q, grid, D // 2) @ oracle_mod.rope_rows(k, grid, D // 2).T
+    s1 = oracle_mod.rope_rows(q, grid, D // 2, offset=(7, -2, 11)) @ \
+        oracle_mod.rope_rows(k, grid, D // 2, offset=(7, -2, 11)).T
+    assert np.allclose(s0, s1, rtol=0, atol=1e-10)
+
+
+# ------------------------------------------------------------------------------ pooling, top-k
+def test_block_means_ragged(oracle_mod):
+    """Block means == numpy reshape-mean, with a partial last block averaged over its real tokens."""
+    rng = np.random.default_rng(3)
+    L, D, b = 300, 16, 64
+    x = rng.standard_normal((L, D))
+    m = oracle_mod.block_means(x, b)
+    assert m.shape == (5, D)
+    ref = [x[i * b:min(L, (i + 1) * b)].mean(axis=0) for i in range(5)]
+    assert np.allclose(m, np.stack(ref), rtol=0, atol=1e-14)
+    s = oracle_mod.block_scores(m, m[::-1].copy())
+    assert np.allclose(s, m @ m[::-1].T, rtol=0, atol=1e-13)
+
+
+def test_keep_count_golden(oracle_mod):
+    for nb, kf, k in _rows(os.path.join(GOLD, "keep_counts.txt")):
+        assert oracle_mod.keep_count(float(kf), int(nb)) == int(k)
+
+
+@pytest.mark.parametrize("nb,k", [(37, 4), (64, 1), (20, 20), (100, 13)])
+def test_topk_matches_full_sort(oracle_mod, nb, k):
+    """Top-k by comparator sort == full lexicographic sort, with many exact ties (quantised scores)
+    so the lower-index tie-break is exercised; tie flags follow their definition."""
+    rng = np.random.default_rng(nb * 7 + k)
+    s = np.round(rng.standard_normal((nb, nb)) * 3) / 3  # heavy exact ties
+    idx, tie = oracle_mod.topk(s, k)
+    assert np.array_equal(idx, brute.topk_lexsort(s, k))
+    for a in range(nb):
+        srt = np.sort(s[a])[::-1]
+        exp = k < nb and (srt[k - 1] - srt[k]) <= 1e-6 * max(1.0, abs(srt[k - 1]))
+        assert bool(tie[a]) == bool(exp)
+
+
+def test_topk_tie_break_prefers_lower_index(oracle_mod):
+    s = np.zeros((6, 6))
+    s[0] = [1.0, 5.0, 5.0, 2.0, 5.0, 0.5]
+    idx, tie = oracle_mod.topk(s, 2)
+    assert idx[0].tolist() == [1, 2] and tie[0] == 1
+    idx, tie = oracle_mod.topk(s, 3)
+    assert idx[0].tolist() == [1, 2, 4] and tie[0] == 0
+
+
+# --------------------------------------------------------------------------------- sparse branch
+def _head(oracle_mod, w, b=0, h=0, **kw):
+    x = I.make_inputs(w)
+    dec = oracle_mod.decode_bf16
+    return oracle_mod.head_forward(dec(x["q"][b, :, h]), dec(x["k"][b, :, h]), dec(x["v"][b, :, h]),
+                                   dec(x["A"]), (w.T, w.H, w.W), w.block, w.keep_frac, w.rank, **kw), x
+
+
+def test_sparse_keep_all_equals_dense_sdpa(oracle_mod):
+    """keep_frac = 1: the sparse branch is dense softmax attention (torch fp64 SDPA)."""
+    w = W.TINY.with_(keep_frac=1.0)
+    r, x = _head(oracle_mod, w, branches=1)
+    v = oracle_mod.decode_bf16(x["v"][0, :, 0])
+    allowed = np.ones((w.L, w.L), dtype=bool)
+    ref = brute.masked_dense_attention(r["qh"], r["kh"], v, allowed)
+    assert r["keep"] == 4
+    assert np.allclose(r["out_sparse"], ref, rtol=0, atol=1e-12)
+
+
+def test_sparse_equals_masked_dense_ragged(oracle_mod):
+    """keep < 1 on a grid whose L is not a multiple of the block (ragged last block): the gathered-key
+    attention equals a dense masked SDPA built from the kept-block mask."""
+    grid = (3, 5, 7)  # L = 105, block 32 -> 4 blocks, last has 9 tokens
+    x = I.make_custom(11, 1, grid, 1, 64, 16)
+    dec = oracle_mod.decode_bf16
+    q, k, v, A = dec(x["q"][0, :, 0]), dec(x["k"][0, :, 0]), dec(x["v"][0, :, 0]), dec(x["A"])
+    r = oracle_mod.head_forward(q, k, v, A, grid, 32, 0.5, 16, branches=1)
+    allowed = brute.block_mask(r["idx"], 105, 32)
+    ref = brute.masked_dense_attention(r["qh"], r["kh"], v, allowed)
+    assert np.allclose(r["out_sparse"], ref, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------- low-rank branch
+def test_features_relu_matmul(oracle_mod):
+    import torch
+    rng = np.random.default_rng(4)
+    x, A = rng.standard_normal((50, 64)), rng.standard_normal((64, 16))
+    ref = torch.relu(torch.from_numpy(x) @ torch.from_numpy(A)).numpy()
+    assert np.allclose(oracle_mod.features(x, A), ref, rtol=0, atol=1e-13)
+
+
+def test_lowrank_summary_equals_quadratic(oracle_mod):
+    """The query-independent summary form (RoLA B.1) equals the explicit L x L quadratic form."""
+    w = W.TINY
+    r, x = _head(oracle_mod, w, branches=2)
+    v = oracle_mod.decode_bf16(x["v"][0, :, 0])
+    ref = brute.lowrank_quadratic(r["psiq"], r["phiq"], r["psik"], r["phik"], v)
+    assert np.allclose(r["out_lowrank"], ref, rtol=1e-11, atol=1e-13)
+    # the truncated rotation touches only the first r coordinates
+    assert np.array_equal(r["psik"][:, w.rank:], r["phik"][:, w.rank:]) or r["psik"].shape[1] == w.rank
+
+
+def test_lowrank_kernel_is_relative(oracle_mod):
+    """psi(q_i) . psi(k_j) equals the relative-angle form (depends on p_i - p_j only), for the
+    rank-truncated schedule (first r/2 pairs of the D-wide table) with r = 64 < D = 128 (spans the
+    t and h axes)."""
+    rng = np.random.default_rng(5)
+    D, R, grid = 128, 64, (3, 4, 5)
+    L = 60
+    phiq = np.maximum(rng.standard_normal((L, R)), 0)
+    phik = np.maximum(rng.standard_normal((L, R)), 0)
+    psiq = oracle_mod.rope_rows(phiq, grid, R // 2, schedule_dim=D)
+    psik = oracle_mod.rope_rows(phik, grid, R // 2, schedule_dim=D)
+    axis, omega = oracle_mod.rope_pairs(D)
+    pos = brute.grid_positions(grid)
+    ref = brute.relative_kernel(phiq, phik, pos, pos, axis, omega, R // 2)
+    assert np.allclose(psiq @ psik.T, ref, rtol=0, atol=1e-12)
+    assert set(axis[:R // 2]) == {0, 1}  # 22 temporal pairs, then 10 height pairs
+
+
+def test_lowrank_identity_projection_full_rank(oracle_mod):
+    """r = D, A = I: features are relu(x) and the readout weight is relu(q)^T R(p_j - p_i) relu(k)."""
+    rng = np.random.default_rng(6)
+    D, grid = 64, (2, 3, 4)
+    L = 24
+    q, k, v = (rng.standard_normal((L, D)) for _ in range(3))
+    r = oracle_mod.head_forward(q, k, v, np.eye(D), grid, 8, 1.0, D, branches=2)
+    axis, omega = oracle_mod.rope_pairs(D)
+    pos = brute.grid_positions(grid)
+    wgt = brute.relative_kernel(np.maximum(q, 0), np.maximum(k, 0), pos, pos, axis, omega, D // 2)
+    den = (np.maximum(q, 0) @ np.maximum(k, 0).T).sum(1, keepdims=True) + 1e-6
+    assert np.allclose(r["out_lowrank"], (wgt @ v) / den, rtol=1e-10, atol=1e-12)
+
+
+def test_lowrank_r32_rotates_temporal_pairs_only(oracle_mod):
+    """r = 32 < 2 * 22: the truncated rotation uses temporal pairs only, so with one frame (T = 1)
+    psi = phi exactly."""
+    rng = np.random.default_rng(7)
+    phi = np.maximum(rng.standard_normal((40, 32)), 0)
+    psi = oracle_mod.rope_rows(phi, (1, 5, 8), 16, schedule_dim=128)
+    assert np.array_equal(psi, phi)
+
+
+# ------------------------------------------------------------------------------- whole forward
+def test_forward_shift_invariant(oracle_mod):
+    """Shifting all (t, h, w) positions by a constant leaves masks and both branches unchanged
+    (RoPE relative invariance, RoLA eq. (1) and B.1)."""
+    w = W.TINY
+    x = I.make_inputs(w)
+    g = (w.T, w.H, w.W)
+    o0, p0 = oracle_mod.forward(x, g, w.block, w.keep_frac, w.rank)
+    o1, p1 = oracle_mod.forward(x, g, w.block, w.keep_frac, w.rank, offset=(5, -3, 17))
+    for key in p0:
+        assert np.array_equal(p0[key]["idx"], p1[key]["idx"])
+    assert np.allclose(o0, o1, rtol=0, atol=1e-11)
+
+
+def test_forward_single_block_degenerate(oracle_mod):
+    """L smaller than one block: one block, k = 1, the sparse branch is dense attention."""
+    grid = (1, 3, 5)
+    x = I.make_custom(12, 1, grid, 1, 64, 16)
+    dec = oracle_mod.decode_bf16
+    q, k, v, A = dec(x["q"][0, :, 0]), dec(x["k"][0, :, 0]), dec(x["v"][0, :, 0]), dec(x["A"])
+    r = oracle_mod.head_forward(q, k, v, A, grid, 64, 0.1, 16)
+    assert r["keep"] == 1 and r["idx"].tolist() == [[0]] and r["tie"][0] == 0
+    ref = brute.masked_dense_attention(r["qh"], r["kh"], v, np.ones((15, 15), bool))
+    assert np.allclose(r["out_sparse"], ref, rtol=0, atol=1e-12)
+    assert np.allclose(r["out"], r["out_sparse"] + r["out_lowrank"], rtol=0, atol=0)
+
+
+def test_forward_thread_count_independent(oracle_mod):
+    """The oracle's results do not depend on the OpenMP thread count (fixed summation order)."""
+    import subprocess, sys, json
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys, hashlib; sys.path.insert(0, %r); import oracle;"
+            "from sparse_rank_hybrid_b200 import workloads as W, inputs as I;"
+            "w = W.TINY; x = I.make_inputs(w);"
+            "o, _ = oracle.forward(x, (w.T, w.H, w.W), w.block, w.keep_frac, w.rank);"
+            "print(hashlib.sha256(o.tobytes()).hexdigest())") % root
+    outs = []
+    for n in ("1", "4"):
+        env = dict(os.environ, OMP_NUM_THREADS=n, PYTHONHASHSEED="0")
+        outs.append(subprocess.check_output([sys.executable, "-c", code], env=env).strip())
+    assert outs[0] == outs[1]
+
+
+# --------------------------------------------------------------- pins catch planted mistakes
+def test_pins_catch_planted_mistakes(oracle_mod):
+    """Plant plausible mistakes into oracle outputs on the CPU and check the pins reject them."""
+    rng = np.random.default_rng(8)
+    D, grid = 64, (3, 4, 5)
+    L = 60
+    x = rng.standard_normal((L, D))
+    axis, omega = oracle_mod.rope_pairs(D)
+    pos = brute.grid_positions(grid)
+    good = oracle_mod.rope_rows(x, grid, D // 2)
+    assert np.allclose(good, brute.rope_complex(x, pos, axis, omega, D // 2), atol=1e-13)
+    # (a) sin sign flipped (clockwise rotation)
+    xs = x.copy(); xs[:, 1::2] *= -1
+    bad = oracle_mod.rope_rows(xs, grid, D // 2); bad[:, 1::2] *= -1
+    assert not np.allclose(bad, brute.rope_complex(x, pos, axis, omega, D // 2), atol=1e-6)
+    # (b) axes swapped (h positions used for t pairs)
+    pos_bad = pos[:, [1, 0, 2]]
+    assert not np.allclose(good, brute.rope_complex(x, pos_bad, axis, omega, D // 2), atol=1e-6)
+    # (c) normaliser with rotated instead of unrotated features
+    phiq = np.maximum(rng.standard_normal((L, 16)), 0)
+    phik = np.maximum(rng.standard_normal((L, 16)), 0)
+    v = rng.standard_normal((L, D))
+    psiq = oracle_mod.rope_rows(phiq, grid, 8, schedule_dim=D)
+    psik = oracle_mod.rope_rows(phik, grid, 8, schedule_dim=D)
+    S, z = oracle_mod.summary(psik, phik, v)
+    good = oracle_mod.lowrank_apply(psiq, phiq, S, z)
+    assert np.allclose(good, brute.lowrank_quadratic(psiq, phiq, psik, phik, v), rtol=1e-10)
+    bad = oracle_mod.lowrank_apply(psiq, psiq, S, psik.sum(0))
+    assert not np.allclose(bad, brute.lowrank_quadratic(psiq, phiq, psik, phik, v), rtol=1e-4)
+    # (d) softmax scale dropped
+    qh, kh = rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    idx = np.arange(1)[None].repeat(1, 0)
+    full = oracle_mod.sparse_attn(qh, kh, v, 64, idx)
+    assert np.allclose(full, brute.masked_dense_attention(qh, kh, v, np.ones((L, L), bool)), atol=1e-12)
+    unscaled = oracle_mod.sparse_attn(qh * math.sqrt(D), kh, v, 64, idx)
+    assert not np.allclose(unscaled, brute.masked_dense_attention(qh, kh, v, np.ones((L, L), bool)),
+                           atol=1e-4)
