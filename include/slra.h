@@ -1,0 +1,198 @@
+/*
+ * slra.h - C ABI of libslra.so: the forward pass of 3D-RoPE sparse + low-rank hybrid attention for
+ * video diffusion transformers, as hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (page titles and sections of the method's sources):
+ *   RoLA: Rotary-Positioned Low-Rank Linear Attention for Efficient Diffusion Transformers
+ *     - "3 Preliminary": a video latent T x H x W is flattened to L = T*H*W tokens (row-major t,h,w);
+ *       3D RoPE splits each head across the t, h, w axes and makes q.k depend on relative offsets
+ *       (eq. (1)).
+ *     - "4.1": a block-sparse softmax branch for the high-energy "spikes" plus a low-rank branch whose
+ *       global context is computed once per head at O(L r d_h) cost.
+ *     - "4.2": the low-rank branch reuses the first r rotary coordinates (r/2 complete pairs) of the
+ *       backbone's own schedule; "4.3": that rotation is applied OUTSIDE the nonlinearity, so the
+ *       summary stays query-independent ("B.1").
+ *   RoPeSLR: 3D RoPE-driven Sparse-LowRank Attention for Efficient Diffusion Transformers
+ *     - appendix on 3D RoPE: rotary base 10000, head dimension partitioned over (t, x, y).
+ *
+ *   qh, kh      = 3D RoPE of q, k (pairs (2j, 2j+1); pairs split t/h/w = c-2*floor(c/3), floor(c/3),
+ *                 floor(c/3) with c = D/2, i.e. 44/42/42 dims at D = 128; omega = theta^(-2m/d_axis))
+ *   qbar, kbar  = mean of qh, kh over each block of `block` tokens (last block: its real tokens)
+ *   K(alpha)    = the k = clamp(round(keep_frac * nb), 1, nb) key blocks with the largest
+ *                 qbar_alpha . kbar_beta, ties to the lower block index
+ *   O_sparse_i  = softmax_j(qh_i . kh_j / sqrt(D)) v_j over the keys of K(alpha(i))
+ *   phi(x)      = relu(x A) on raw q, k;   psi = phi with its first r coordinates rotated like RoPE
+ *   S = sum_j psi(k_j) v_j^T (r x D),  z = sum_j phi(k_j)   (all L keys, per head)
+ *   O_lowrank_i = psi(q_i)^T S / (phi(q_i) . z + 1e-6)
+ *   out         = O_sparse + O_lowrank
+ *
+ * Conventions for every entry point:
+ *   - Device pointers unless stated otherwise.  The caller owns every buffer; nothing is retained
+ *     after a call returns.  Calls are asynchronous on `stream` (NULL = the legacy default stream)
+ *     and never synchronize, except slra_device_status and slra_attn_fwd_host.
+ *   - All arguments are validated before anything is launched; an invalid call returns a status and
+ *     launches nothing.  Launch failures return SLRA_ERR_CUDA.
+ *   - Problems detected on the device (an input too large for the fp16 operands, a bounded wait that
+ *     ran out) are recorded in a status word inside the workspace and reported by
+ *     slra_device_status.
+ *   - A workspace may be used by one call at a time (calls on one stream are ordered; calls on
+ *     different streams need different workspaces).
+ */
+#ifndef SLRA_H
+#define SLRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SLRA_ABI_VERSION 1
+
+/* Exported symbols (the library is built with hidden visibility for everything else). */
+#if defined(__GNUC__)
+#define SLRA_API __attribute__((visibility("default")))
+#else
+#define SLRA_API
+#endif
+
+/* cudaStream_t without including the CUDA headers. */
+typedef struct CUstream_st* slra_stream_t;
+
+typedef enum slra_status {
+    SLRA_OK = 0,
+    SLRA_ERR_INVALID_ARG = 1,     /* NULL pointer, non-positive size, L overflow, keep_frac outside (0,1] */
+    SLRA_ERR_UNSUPPORTED = 2,     /* valid but not implemented: head_dim, block, rank, too many blocks  */
+    SLRA_ERR_ALIGNMENT = 3,       /* a pointer is not 16-byte aligned                                   */
+    SLRA_ERR_WORKSPACE = 4,       /* workspace NULL, misaligned (256 B) or smaller than required         */
+    SLRA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or a kernel launch failed                */
+    SLRA_ERR_DEVICE_TIMEOUT = 6,  /* (device status) a bounded wait inside a kernel ran out              */
+    SLRA_ERR_RANGE = 7,           /* (device status) |value| >= 65504 after RoPE: does not fit fp16      */
+    SLRA_ERR_NO_DEVICE = 8        /* no sm_100 device is current                                         */
+} slra_status;
+
+typedef enum slra_out_dtype { SLRA_OUT_F32 = 0, SLRA_OUT_BF16 = 1 } slra_out_dtype;
+
+/* Which branches contribute to `out` (default both). */
+enum { SLRA_BRANCH_SPARSE = 1, SLRA_BRANCH_LOWRANK = 2, SLRA_BRANCH_BOTH = 3 };
+
+/*
+ * Problem description.  Fill it with slra_problem_init, then adjust optional fields.
+ *   batch, heads, head_dim  B, Hh, D.  D in {64, 128}.
+ *   T, H, W                 latent grid; L = T*H*W tokens (row-major t, h, w).
+ *   block                   tokens per block for both queries and keys; 64 or 128.
+ *   keep_frac               kept fraction of key blocks per query block, in (0, 1].
+ *   rank                    r: multiple of 16 with 16 <= r <= D.
+ *   theta                   rotary base (default 10000).
+ *   out_dtype               SLRA_OUT_F32 (default) or SLRA_OUT_BF16.
+ *   branches                SLRA_BRANCH_* mask (default both).
+ *   pos_offset              constant added to every (t, h, w) position (default 0; RoPE makes the
+ *                           result independent of it, which the tests use).
+ *   rope_split              rotary pairs per (t, h, w); all zero = default split described above.
+ *   wait_timeout_ns         bound of every wait inside the kernels (default 2e9 ns = 2 s).
+ *   attn_events             optional pair of cudaEvent_t (NULL = none): recorded on `stream` right
+ *                           before and right after the attention kernel, so a caller can time the
+ *                           dominant kernel alone.  The caller creates and owns them.
+ */
+typedef struct slra_problem {
+    int64_t batch, heads, head_dim;
+    int64_t T, H, W;
+    int64_t block;
+    double keep_frac;
+    int64_t rank;
+    double theta;
+    int32_t out_dtype;
+    int32_t branches;
+    int64_t pos_offset[3];
+    int64_t rope_split[3];
+    uint64_t wait_timeout_ns;
+    void* attn_events[2];
+} slra_problem;
+
+/*
+ * Where the intermediates live inside a workspace (byte offsets from its start; all 256-B aligned).
+ * They are valid after a forward call and may be read for inspection:
+ *   qh, kh, vh   fp16 [B*Hh][nb*block][D]  rotated q, k and fp16 copy of v, head-major, zero padded
+ *   qbar, kbar   fp64 [B*Hh][nb][D]        block means of qh, kh (computed in fp64)
+ *   idx          int32 [B*Hh][nb][keep]    kept key blocks per query block, ascending
+ *   tie          uint8 [B*Hh][nb]          1 where the k-th and (k+1)-th block scores are within
+ *                                          1e-6 * max(1, |s_k|) (a numerically fragile selection)
+ *   S            fp32 [B*Hh][rank][D]      low-rank summary
+ *   z            fp32 [B*Hh][rank]         sum of the unrotated key features
+ *   status       int32                     device status word (see slra_device_status)
+ */
+typedef struct slra_ws_layout {
+    size_t total_bytes;
+    int64_t L, nb, keep, nsplit;
+    size_t status, rope_table, qh, kh, vh, qbar, kbar, idx, tie, s_part, z_part, S, z;
+} slra_ws_layout;
+
+/* ABI version (SLRA_ABI_VERSION).  Never fails. */
+SLRA_API int slra_abi_version(void);
+
+/* Static, human-readable name of a status code.  Never returns NULL. */
+SLRA_API const char* slra_status_string(int status);
+
+/* Fill *p with the given sizes and the defaults above.  Returns SLRA_ERR_INVALID_ARG if p is NULL. */
+SLRA_API slra_status slra_problem_init(slra_problem* p, int64_t batch, int64_t heads, int64_t head_dim, int64_t T,
+                              int64_t H, int64_t W, int64_t block, double keep_frac, int64_t rank);
+
+/* Check a problem description without touching the GPU.  SLRA_OK or the reason it is rejected. */
+SLRA_API slra_status slra_validate(const slra_problem* p);
+
+/* Kept key blocks per query block, k = clamp(floor(keep_frac * nb + 0.5), 1, nb); -1 if invalid. */
+SLRA_API int64_t slra_keep_count(const slra_problem* p);
+
+/* Workspace size and the offsets of the intermediates in it.  No GPU access. */
+SLRA_API slra_status slra_workspace_layout(const slra_problem* p, slra_ws_layout* layout);
+
+/*
+ * Full forward pass (RoLA "4.1" sparse + low-rank hybrid; all steps listed at the top of this file).
+ *   q, k, v    bf16 [B][L][Hh][D] contiguous (token-major), 16-B aligned.
+ *   A          bf16 [D][rank] contiguous, the feature projection shared by all heads and by q and k.
+ *   out        [B][L][Hh][D] contiguous, fp32 or bf16 as p->out_dtype; must not alias q, k, v.
+ *   workspace  device buffer of at least layout.total_bytes bytes, 256-B aligned.
+ * Launches 6 kernels on `stream` (tables, RoPE + pooling, selection, low-rank partial sums and their
+ * reduction, attention with the fused low-rank readout) and returns without synchronizing.
+ */
+SLRA_API slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
+                          void* out, void* workspace, size_t workspace_bytes, slra_stream_t stream);
+
+/*
+ * The same forward pass on HOST buffers: copies q, k, v, A from host memory into `io` (a device
+ * buffer of at least slra_host_io_bytes(p) bytes), runs slra_attn_fwd and copies `out` back to host
+ * memory, all on `stream`, then synchronizes the stream.  Host buffers should be pinned for speed.
+ */
+SLRA_API size_t slra_host_io_bytes(const slra_problem* p);
+SLRA_API slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const void* k_host,
+                               const void* v_host, const void* A_host, void* out_host, void* io,
+                               size_t io_bytes, void* workspace, size_t workspace_bytes, slra_stream_t stream);
+
+/*
+ * Block selection only (3D RoPE, block means, scores, top-k): fills the qh/kh/vh, qbar/kbar, idx and
+ * tie sections of the workspace.  Same argument rules as slra_attn_fwd.
+ */
+SLRA_API slra_status slra_select_blocks(const slra_problem* p, const void* q, const void* k, const void* v,
+                               void* workspace, size_t workspace_bytes, slra_stream_t stream);
+
+/*
+ * Low-rank summary only (RoLA "4.1", "B.1"): fills the S and z sections of the workspace from raw k,
+ * v and A.  Same argument rules as slra_attn_fwd.
+ */
+SLRA_API slra_status slra_lowrank_summary(const slra_problem* p, const void* k, const void* v, const void* A,
+                                 void* workspace, size_t workspace_bytes, slra_stream_t stream);
+
+/*
+ * Synchronize `stream`, then read and clear the device status word of `workspace`.  *status receives
+ * SLRA_OK, SLRA_ERR_DEVICE_TIMEOUT or SLRA_ERR_RANGE.  Every compute entry point clears the word when it
+ * starts, so this reports the calls made since the last compute call began (a timeout wins over a
+ * range problem).
+ */
+SLRA_API slra_status slra_device_status(void* workspace, slra_stream_t stream, int32_t* status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLRA_H */

@@ -1,0 +1,443 @@
+// C ABI of libslra.so (declared in include/slra.h): argument validation, workspace layout, TMA
+// descriptors and the launch sequence of the hybrid attention forward.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/slra.h"
+#include "common.cuh"
+
+using namespace slra;
+
+namespace {
+
+constexpr int kTargetCtas = 2 * 148;  // low-rank split count aims at two CTAs per B200 SM
+constexpr int kLrTileTokens = 32;
+constexpr int64_t kMaxBlocks = 2048;  // selection keeps a row of scores in shared memory
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool default_split(int64_t D, const int64_t* s, int64_t out[3]) {
+    const int64_t c = D / 2;
+    if (s[0] == 0 && s[1] == 0 && s[2] == 0) {
+        out[1] = c / 3;
+        out[2] = c / 3;
+        out[0] = c - 2 * (c / 3);
+        return true;
+    }
+    if (s[0] < 0 || s[1] < 0 || s[2] < 0 || s[0] + s[1] + s[2] != c) return false;
+    out[0] = s[0]; out[1] = s[1]; out[2] = s[2];
+    return true;
+}
+
+struct Derived {
+    Geom g;
+    RopeMeta meta;
+    int table_entries;
+    int nsplit;
+    slra_ws_layout lay;
+};
+
+slra_status derive(const slra_problem* p, Derived* d) {
+    if (!p) return SLRA_ERR_INVALID_ARG;
+    if (p->batch < 1 || p->heads < 1 || p->T < 1 || p->H < 1 || p->W < 1) return SLRA_ERR_INVALID_ARG;
+    if (!(p->keep_frac > 0.0 && p->keep_frac <= 1.0)) return SLRA_ERR_INVALID_ARG;
+    if (p->theta < 0.0 || std::isnan(p->theta)) return SLRA_ERR_INVALID_ARG;
+    if (p->out_dtype != SLRA_OUT_F32 && p->out_dtype != SLRA_OUT_BF16) return SLRA_ERR_INVALID_ARG;
+    if (p->branches < 0 || p->branches > 3) return SLRA_ERR_INVALID_ARG;
+    if (p->head_dim != 64 && p->head_dim != 128) return SLRA_ERR_UNSUPPORTED;
+    if (p->block != 64 && p->block != 128) return SLRA_ERR_UNSUPPORTED;
+    if (p->rank < 16 || p->rank > p->head_dim || p->rank % 16 != 0) return SLRA_ERR_UNSUPPORTED;
+    const int64_t L = p->T * p->H * p->W;
+    if (p->T > (1 << 20) || p->H > (1 << 20) || p->W > (1 << 20) || L > (int64_t(1) << 28))
+        return SLRA_ERR_INVALID_ARG;
+    const int64_t nb = (L + p->block - 1) / p->block;
+    if (nb > kMaxBlocks) return SLRA_ERR_UNSUPPORTED;
+    const int64_t BH = p->batch * p->heads;
+    if (BH * nb * p->block >= (int64_t(1) << 31)) return SLRA_ERR_UNSUPPORTED;  // TMA row coordinate
+    int64_t split[3];
+    if (!default_split(p->head_dim, p->rope_split, split)) return SLRA_ERR_INVALID_ARG;
+    int64_t keep = static_cast<int64_t>(std::floor(p->keep_frac * static_cast<double>(nb) + 0.5));
+    keep = keep < 1 ? 1 : (keep > nb ? nb : keep);
+
+    Geom& g = d->g;
+    g.B = static_cast<int>(p->batch);
+    g.Hh = static_cast<int>(p->heads);
+    g.D = static_cast<int>(p->head_dim);
+    g.T = static_cast<int>(p->T);
+    g.H = static_cast<int>(p->H);
+    g.W = static_cast<int>(p->W);
+    g.L = static_cast<int>(L);
+    g.block = static_cast<int>(p->block);
+    g.nb = static_cast<int>(nb);
+    g.keep = static_cast<int>(keep);
+    g.R = static_cast<int>(p->rank);
+    g.Lp = static_cast<int>(nb * p->block);
+
+    RopeMeta& m = d->meta;
+    std::memset(&m, 0, sizeof m);
+    m.npairs = g.D / 2;
+    m.theta = p->theta > 0.0 ? p->theta : 10000.0;
+    const int lens[3] = {g.T, g.H, g.W};
+    int j = 0, off = 0;
+    for (int a = 0; a < 3; ++a) {
+        m.apairs[a] = static_cast<int>(split[a]);
+        m.axis_len[a] = lens[a];
+        m.off[a] = p->pos_offset[a];
+        for (int mm = 0; mm < split[a]; ++mm, ++j) {
+            m.axis[j] = a;
+            m.mloc[j] = mm;
+            m.tab_off[j] = off;
+            off += lens[a];
+        }
+    }
+    d->table_entries = off;
+    const int64_t ntiles = (L + kLrTileTokens - 1) / kLrTileTokens;
+    int64_t ns = (kTargetCtas + BH - 1) / BH;
+    ns = ns < 1 ? 1 : (ns > ntiles ? ntiles : ns);
+    d->nsplit = static_cast<int>(ns);
+
+    slra_ws_layout& w = d->lay;
+    std::memset(&w, 0, sizeof w);
+    w.L = L;
+    w.nb = nb;
+    w.keep = keep;
+    w.nsplit = ns;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align_up(o + bytes, 256);
+        return at;
+    };
+    const size_t rows = static_cast<size_t>(BH) * nb * p->block;
+    w.status = take(256);
+    w.rope_table = take(sizeof(double2) * static_cast<size_t>(off) + sizeof(int2) * kMaxPairs);
+    w.qh = take(rows * p->head_dim * 2);
+    w.kh = take(rows * p->head_dim * 2);
+    w.vh = take(rows * p->head_dim * 2);
+    w.qbar = take(static_cast<size_t>(BH) * nb * p->head_dim * 8);
+    w.kbar = take(static_cast<size_t>(BH) * nb * p->head_dim * 8);
+    w.idx = take(static_cast<size_t>(BH) * nb * keep * 4);
+    w.tie = take(static_cast<size_t>(BH) * nb);
+    w.s_part = take(static_cast<size_t>(BH) * ns * p->rank * p->head_dim * 4);
+    w.z_part = take(static_cast<size_t>(BH) * ns * p->rank * 4);
+    w.S = take(static_cast<size_t>(BH) * p->rank * p->head_dim * 4);
+    w.z = take(static_cast<size_t>(BH) * p->rank * 4);
+    w.total_bytes = o;
+    return SLRA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+// The current device must be an sm_100 part (the kernels are built for sm_100a only).
+slra_status check_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return SLRA_ERR_NO_DEVICE; }
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SLRA_ERR_NO_DEVICE;
+    }
+    return (major == 10 && minor == 0) ? SLRA_OK : SLRA_ERR_NO_DEVICE;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2D fp16 map over a head-major [rows][D] buffer, box 64 columns x box_rows rows, 128-B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int D, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct Ptrs {
+    uint8_t* base;
+    int* status;
+    double2* tab;
+    int2* pairs;
+    __half *qh, *kh, *vh;
+    double *qbar, *kbar;
+    int32_t* idx;
+    uint8_t* tie;
+    float *s_part, *z_part, *S, *z;
+};
+
+Ptrs carve(void* ws, const Derived& d) {
+    Ptrs p;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    const slra_ws_layout& w = d.lay;
+    p.base = b;
+    p.status = reinterpret_cast<int*>(b + w.status);
+    p.tab = reinterpret_cast<double2*>(b + w.rope_table);
+    p.pairs = reinterpret_cast<int2*>(b + w.rope_table + sizeof(double2) * d.table_entries);
+    p.qh = reinterpret_cast<__half*>(b + w.qh);
+    p.kh = reinterpret_cast<__half*>(b + w.kh);
+    p.vh = reinterpret_cast<__half*>(b + w.vh);
+    p.qbar = reinterpret_cast<double*>(b + w.qbar);
+    p.kbar = reinterpret_cast<double*>(b + w.kbar);
+    p.idx = reinterpret_cast<int32_t*>(b + w.idx);
+    p.tie = b + w.tie;
+    p.s_part = reinterpret_cast<float*>(b + w.s_part);
+    p.z_part = reinterpret_cast<float*>(b + w.z_part);
+    p.S = reinterpret_cast<float*>(b + w.S);
+    p.z = reinterpret_cast<float*>(b + w.z);
+    return p;
+}
+
+slra_status check_ws(const Derived& d, void* ws, size_t bytes) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < d.lay.total_bytes) return SLRA_ERR_WORKSPACE;
+    return SLRA_OK;
+}
+
+slra_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SLRA_OK : SLRA_ERR_CUDA; }
+
+// Tables + RoPE/pooling + selection.
+slra_status run_select(const Derived& d, const Ptrs& w, const void* q, const void* k, const void* v,
+                       cudaStream_t st) {
+    const Geom& g = d.g;
+    cudaError_t e = launch_rope_pool(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                     static_cast<const __nv_bfloat16*>(v), w.tab, w.pairs, g, w.qh, w.kh, w.vh,
+                                     w.qbar, w.kbar, w.status, st);
+    if (e != cudaSuccess) return SLRA_ERR_CUDA;
+    return cuda_status(launch_select(w.qbar, w.kbar, g, w.idx, w.tie, st));
+}
+
+slra_status run_lowrank(const Derived& d, const Ptrs& w, const void* k, const void* v, const void* A,
+                        cudaStream_t st) {
+    const Geom& g = d.g;
+    cudaError_t e = launch_lowrank_partial(static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                                           static_cast<const __nv_bfloat16*>(A), w.tab, w.pairs, g, d.nsplit,
+                                           w.s_part, w.z_part, st);
+    if (e != cudaSuccess) return SLRA_ERR_CUDA;
+    return cuda_status(launch_lowrank_reduce(w.s_part, w.z_part, g, d.nsplit, w.S, w.z, st));
+}
+
+slra_status begin(const Derived& d, const Ptrs& w, cudaStream_t st) {
+    if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return SLRA_ERR_CUDA;
+    return cuda_status(launch_rope_table(w.tab, w.pairs, d.meta, d.table_entries, st));
+}
+
+size_t qkv_bytes(const Derived& d) {
+    return static_cast<size_t>(d.g.B) * d.g.L * d.g.Hh * d.g.D * 2;
+}
+
+}  // namespace
+
+extern "C" {
+
+int slra_abi_version(void) { return SLRA_ABI_VERSION; }
+
+const char* slra_status_string(int s) {
+    switch (s) {
+        case SLRA_OK: return "ok";
+        case SLRA_ERR_INVALID_ARG: return "invalid argument";
+        case SLRA_ERR_UNSUPPORTED: return "unsupported size or option";
+        case SLRA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case SLRA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case SLRA_ERR_CUDA: return "CUDA call or kernel launch failed";
+        case SLRA_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel ran out";
+        case SLRA_ERR_RANGE: return "input value out of fp16 range after RoPE";
+        case SLRA_ERR_NO_DEVICE: return "no sm_100 device is current";
+        default: return "unknown status";
+    }
+}
+
+slra_status slra_problem_init(slra_problem* p, int64_t batch, int64_t heads, int64_t head_dim, int64_t T, int64_t H,
+                              int64_t W, int64_t block, double keep_frac, int64_t rank) {
+    if (!p) return SLRA_ERR_INVALID_ARG;
+    std::memset(p, 0, sizeof *p);
+    p->batch = batch;
+    p->heads = heads;
+    p->head_dim = head_dim;
+    p->T = T;
+    p->H = H;
+    p->W = W;
+    p->block = block;
+    p->keep_frac = keep_frac;
+    p->rank = rank;
+    p->theta = 10000.0;
+    p->out_dtype = SLRA_OUT_F32;
+    p->branches = SLRA_BRANCH_BOTH;
+    p->wait_timeout_ns = 2000000000ull;
+    return SLRA_OK;
+}
+
+slra_status slra_validate(const slra_problem* p) {
+    Derived d;
+    return derive(p, &d);
+}
+
+int64_t slra_keep_count(const slra_problem* p) {
+    Derived d;
+    return derive(p, &d) == SLRA_OK ? d.g.keep : -1;
+}
+
+slra_status slra_workspace_layout(const slra_problem* p, slra_ws_layout* layout) {
+    if (!layout) return SLRA_ERR_INVALID_ARG;
+    Derived d;
+    slra_status s = derive(p, &d);
+    if (s != SLRA_OK) return s;
+    *layout = d.lay;
+    return SLRA_OK;
+}
+
+slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
+                          void* out, void* workspace, size_t workspace_bytes, slra_stream_t stream) {
+    Derived d;
+    slra_status s = derive(p, &d);
+    if (s != SLRA_OK) return s;
+    if (!q || !k || !v || !A || !out) return SLRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(A) || !aligned16(out)) return SLRA_ERR_ALIGNMENT;
+    if ((s = check_ws(d, workspace, workspace_bytes)) != SLRA_OK) return s;
+    const size_t in_b = qkv_bytes(d);
+    const size_t out_b = in_b / 2 * (p->out_dtype == SLRA_OUT_F32 ? 4 : 2);
+    if (overlaps(out, out_b, q, in_b) || overlaps(out, out_b, k, in_b) || overlaps(out, out_b, v, in_b) ||
+        overlaps(out, out_b, workspace, workspace_bytes))
+        return SLRA_ERR_INVALID_ARG;
+    if ((s = check_device()) != SLRA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const Ptrs w = carve(workspace, d);
+    const int branches = p->branches == 0 ? SLRA_BRANCH_BOTH : p->branches;
+    const Geom& g = d.g;
+
+    AttnMaps maps;
+    const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
+    if (!make_map(&maps.q, w.qh, rows, g.D, 128) || !make_map(&maps.k, w.kh, rows, g.D, g.block) ||
+        !make_map(&maps.v, w.vh, rows, g.D, g.block))
+        return SLRA_ERR_CUDA;
+
+    if ((s = begin(d, w, st)) != SLRA_OK) return s;
+    if (branches & SLRA_BRANCH_SPARSE)
+        if ((s = run_select(d, w, q, k, v, st)) != SLRA_OK) return s;
+    if (branches & SLRA_BRANCH_LOWRANK)
+        if ((s = run_lowrank(d, w, k, v, A, st)) != SLRA_OK) return s;
+
+    AttnArgs a;
+    a.idx = w.idx;
+    a.keep = (branches & SLRA_BRANCH_SPARSE) ? g.keep : 0;
+    a.q_raw = static_cast<const __nv_bfloat16*>(q);
+    a.A = static_cast<const __nv_bfloat16*>(A);
+    a.S = w.S;
+    a.z = w.z;
+    a.tab = w.tab;
+    a.pairs = w.pairs;
+    a.lowrank = (branches & SLRA_BRANCH_LOWRANK) ? 1 : 0;
+    a.out = out;
+    a.out_bf16 = p->out_dtype == SLRA_OUT_BF16 ? 1 : 0;
+    a.status = w.status;
+    a.timeout_ns = p->wait_timeout_ns ? p->wait_timeout_ns : 2000000000ull;
+    if (p->attn_events[0] && cudaEventRecord(static_cast<cudaEvent_t>(p->attn_events[0]), st) != cudaSuccess)
+        return SLRA_ERR_CUDA;
+    if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
+    if (p->attn_events[1] && cudaEventRecord(static_cast<cudaEvent_t>(p->attn_events[1]), st) != cudaSuccess)
+        return SLRA_ERR_CUDA;
+    return SLRA_OK;
+}
+
+size_t slra_host_io_bytes(const slra_problem* p) {
+    Derived d;
+    if (derive(p, &d) != SLRA_OK) return 0;
+    const size_t in_b = align_up(qkv_bytes(d), 256);
+    const size_t a_b = align_up(static_cast<size_t>(d.g.D) * d.g.R * 2, 256);
+    const size_t out_b = align_up(qkv_bytes(d) / 2 * (p->out_dtype == SLRA_OUT_F32 ? 4 : 2), 256);
+    return 3 * in_b + a_b + out_b;
+}
+
+slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const void* k_host, const void* v_host,
+                               const void* A_host, void* out_host, void* io, size_t io_bytes, void* workspace,
+                               size_t workspace_bytes, slra_stream_t stream) {
+    Derived d;
+    slra_status s = derive(p, &d);
+    if (s != SLRA_OK) return s;
+    if (!q_host || !k_host || !v_host || !A_host || !out_host || !io) return SLRA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(io) & 255u) != 0 || io_bytes < slra_host_io_bytes(p)) return SLRA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t raw = qkv_bytes(d);
+    const size_t in_b = align_up(raw, 256);
+    const size_t a_raw = static_cast<size_t>(d.g.D) * d.g.R * 2;
+    const size_t out_raw = raw / 2 * (p->out_dtype == SLRA_OUT_F32 ? 4 : 2);
+    uint8_t* b = static_cast<uint8_t*>(io);
+    void *dq = b, *dk = b + in_b, *dv = b + 2 * in_b, *dA = b + 3 * in_b;
+    void* dout = b + 3 * in_b + align_up(a_raw, 256);
+    if (cudaMemcpyAsync(dq, q_host, raw, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k_host, raw, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v_host, raw, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dA, A_host, a_raw, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return SLRA_ERR_CUDA;
+    s = slra_attn_fwd(p, dq, dk, dv, dA, dout, workspace, workspace_bytes, stream);
+    if (s != SLRA_OK) return s;
+    if (cudaMemcpyAsync(out_host, dout, out_raw, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SLRA_ERR_CUDA;
+    return cuda_status(cudaStreamSynchronize(st));
+}
+
+slra_status slra_select_blocks(const slra_problem* p, const void* q, const void* k, const void* v, void* workspace,
+                               size_t workspace_bytes, slra_stream_t stream) {
+    Derived d;
+    slra_status s = derive(p, &d);
+    if (s != SLRA_OK) return s;
+    if (!q || !k || !v) return SLRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SLRA_ERR_ALIGNMENT;
+    if ((s = check_ws(d, workspace, workspace_bytes)) != SLRA_OK) return s;
+    if ((s = check_device()) != SLRA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const Ptrs w = carve(workspace, d);
+    if ((s = begin(d, w, st)) != SLRA_OK) return s;
+    return run_select(d, w, q, k, v, st);
+}
+
+slra_status slra_lowrank_summary(const slra_problem* p, const void* k, const void* v, const void* A, void* workspace,
+                                 size_t workspace_bytes, slra_stream_t stream) {
+    Derived d;
+    slra_status s = derive(p, &d);
+    if (s != SLRA_OK) return s;
+    if (!k || !v || !A) return SLRA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(A)) return SLRA_ERR_ALIGNMENT;
+    if ((s = check_ws(d, workspace, workspace_bytes)) != SLRA_OK) return s;
+    if ((s = check_device()) != SLRA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const Ptrs w = carve(workspace, d);
+    if ((s = begin(d, w, st)) != SLRA_OK) return s;
+    return run_lowrank(d, w, k, v, A, st);
+}
+
+slra_status slra_device_status(void* workspace, slra_stream_t stream, int32_t* status) {
+    if (!workspace || !status) return SLRA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int v = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SLRA_ERR_CUDA;
+    if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return SLRA_ERR_CUDA;
+    if (cudaMemset(workspace, 0, sizeof v) != cudaSuccess) return SLRA_ERR_CUDA;
+    *status = (v & kDevTimeout) ? SLRA_ERR_DEVICE_TIMEOUT : ((v & kDevRange) ? SLRA_ERR_RANGE : SLRA_OK);
+    return SLRA_OK;
+}
+
+}  // extern "C"

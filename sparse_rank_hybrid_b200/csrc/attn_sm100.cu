@@ -1,0 +1,420 @@
+// Block-sparse softmax attention over the kept key blocks, on the sm_100a tensor cores, with the
+// low-rank branch's query-side readout fused into the epilogue.
+//
+// Method (RoLA, "4.1"): for each query block alpha, exact softmax attention of its queries over the
+// union of the kept key blocks K(alpha); plus O_lr,i = psi(q_i)^T S / (phi(q_i) . z + 1e-6) with
+// phi = relu(q A) on the raw query and psi its first r coordinates rotated by 3D RoPE ("4.2", "4.3").
+//
+// One CTA (128 threads = 4 warps) per (query block, batch*head); two CTAs share an SM, so one CTA's
+// softmax overlaps the other's matrix products.  Per kept key block:
+//   TMA   k^ tile [block][D] and v tile [block][D] (fp16, 128-B swizzle) into shared memory;
+//   MMA   S = q^ k^T      (tcgen05.mma kind::f16, M=128, N=block, K=D; fp32 accumulator in TMEM);
+//   softmax: thread i owns row i (TMEM lane i): row max, lazy rescale of O (only when the max grows
+//         by more than 2^8), P = 2^(s*log2e/sqrt(D) - m) rounded to fp16 and written back into the
+//         TMEM columns of S;
+//   MMA   O += P v        (A operand = P from TMEM, B = v tile MN-major; M=128, N=D, K=block).
+// Epilogue: O / l plus the low-rank readout (CUDA cores, fp32), stored as fp32 or bf16.
+//
+// All waits are bounded (see sm100.cuh); a wait that runs out records a timeout in the status word
+// and the CTA leaves the loop, releases its tensor memory and returns.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace slra {
+
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kTmemCols = 256;   // S/P at columns [0, 128), O at [128, 128 + D)
+constexpr int kColO = 128;
+
+template <int D>
+struct AttnLayout {
+    static constexpr int kQBytes = 128 * D * 2;
+    static constexpr int kKVBytes = 128 * D * 2;  // sized for block 128
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + kKVBytes;
+    static constexpr int kOffBar = kOffV + kKVBytes;  // 5 mbarriers
+    static constexpr int kOffMisc = kOffBar + 64;     // tmem base, abort flag
+    static constexpr int kBytes = kOffMisc + 64;
+};
+
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+    attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, AttnArgs a, Geom g) {
+    using Lay = AttnLayout<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __half* sq = reinterpret_cast<__half*>(smem + Lay::kOffQ);
+    __half* sk = reinterpret_cast<__half*>(smem + Lay::kOffK);
+    __half* sv = reinterpret_cast<__half*>(smem + Lay::kOffV);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
+    uint64_t* bar_q = bars + 0;
+    uint64_t* bar_k = bars + 1;
+    uint64_t* bar_v = bars + 2;
+    uint64_t* bar_s = bars + 3;
+    uint64_t* bar_o = bars + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int alpha = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int blk = g.block;
+    const int keep = a.keep;
+    const uint64_t tmo = a.timeout_ns;
+    const int32_t* my_idx = a.idx + (static_cast<size_t>(bh) * g.nb + alpha) * (keep > 0 ? g.keep : 0);
+
+    if (tid == 0) {
+        for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem;               // S (fp32) and P (fp16 packed) columns
+    const uint32_t tO = tmem + kColO;       // O accumulator
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+
+    const uint32_t idesc_s = idesc_f16_f32(128, blk, false, false);
+    const uint32_t idesc_o = idesc_f16_f32(128, D, false, true);
+    const uint32_t q_addr = smem_addr(sq), k_addr = smem_addr(sk), v_addr = smem_addr(sv);
+    const uint32_t kv_bytes = static_cast<uint32_t>(blk) * D * 2;
+    const int row0 = bh * g.Lp;  // first row of this head in the head-major buffers
+
+    auto fail = [&]() {
+        *abort_flag = 1;
+        atomicOr(a.status, kDevTimeout);
+    };
+    auto issue_s = [&]() {  // S = q^ k^T over the D/16 k-steps
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(q_addr + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * (blk * 128) + (kk & 3) * 32, 16, 1024);
+            umma_ss(tS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_s);
+    };
+    auto load_kv = [&](uint64_t* bar, __half* dst, const CUtensorMap* tm, int beta) {
+        mbar_expect_tx(bar, kv_bytes);
+#pragma unroll
+        for (int s = 0; s < D / 64; ++s)
+            tma_load_2d(reinterpret_cast<uint8_t*>(dst) + s * (blk * 128), tm, bar, s * 64, row0 + beta * blk);
+    };
+
+    // Operations issued / observed complete per barrier (thread 0 only), so an aborted CTA can drain
+    // what is still in flight before it releases shared and tensor memory.
+    int n_q_issued = 0, n_q_done = 0, n_k_issued = 0, n_k_done = 0, n_v_issued = 0, n_v_done = 0;
+    int n_s_issued = 0, n_s_done = 0, n_o_issued = 0, n_o_done = 0;
+
+    // ------------------------------------------------------------------ prologue: Q, K0, V0, S0
+    if (keep > 0 && tid == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        mbar_expect_tx(bar_q, 128 * D * 2);
+#pragma unroll
+        for (int s = 0; s < D / 64; ++s)
+            tma_load_2d(reinterpret_cast<uint8_t*>(sq) + s * (128 * 128), &tm_q, bar_q, s * 64, row0 + alpha * blk);
+        const int beta0 = my_idx[0];
+        load_kv(bar_k, sk, &tm_k, beta0);
+        load_kv(bar_v, sv, &tm_v, beta0);
+        n_q_issued = 1; n_k_issued = 1; n_v_issued = 1;
+        if (mbar_wait(bar_q, 0, tmo, abort_flag)) n_q_done = 1;
+        if (n_q_done && mbar_wait(bar_k, 0, tmo, abort_flag)) {
+            n_k_done = 1;
+            tc_fence_after();
+            issue_s();
+            n_s_issued = 1;
+        } else {
+            fail();
+        }
+    }
+
+    const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+    float m_run = 0.f, l_run = 0.f;
+    int next_beta = 0;
+    for (int j = 0; j < keep; ++j) {
+        const bool ok = mbar_wait(bar_s, j & 1, tmo, abort_flag);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) fail();
+            break;
+        }
+        tc_fence_after();
+        if (tid == 0) ++n_s_done;
+        if (tid == 0 && j + 1 < keep) {  // S_j done reading the k tile: fetch the next one
+            next_beta = my_idx[j + 1];
+            load_kv(bar_k, sk, &tm_k, next_beta);
+            ++n_k_issued;
+        }
+        // ---- softmax on row (warp*32 + lane)
+        const int beta_row = __ldg(my_idx + j);
+        const int valid = min(blk, g.L - beta_row * blk);  // keys of this block that exist
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (c * 32 < blk) tmem_ld32(tS + lane_base + c * 32, sr[c]);
+        tmem_ld_wait(sr[0]);
+#pragma unroll
+        for (int c = 1; c < 4; ++c)
+            if (c * 32 < blk) reg_fence(sr[c]);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (c * 32 >= blk) continue;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                float t = __uint_as_float(sr[c][i]) * scale_log2;
+                if (c * 32 + i >= valid) t = -INFINITY;
+                sr[c][i] = __float_as_uint(t);
+                mx = fmaxf(mx, t);
+            }
+        }
+        if (j == 0) {
+            m_run = mx;
+        } else {
+            const bool need = mx > m_run + 8.0f;
+            if (__any_sync(0xffffffffu, need)) {  // warp-uniform: TMEM access is warp-collective
+                const float m_new = fmaxf(m_run, mx);
+                const float alpha_r = ex2_approx(m_run - m_new);
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + lane_base + c * 32, o);
+                    tmem_ld_wait(o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha_r);
+                    tmem_st32(tO + lane_base + c * 32, o);
+                }
+                tmem_st_wait();
+                l_run *= alpha_r;
+                m_run = m_new;
+            }
+        }
+        float lsum = 0.f;
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {  // 64 keys -> 32 packed fp16x2 columns
+            if (c2 * 64 >= blk) continue;
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int key = c2 * 64 + 2 * i;
+                const float p0 = ex2_approx(__uint_as_float(sr[key >> 5][key & 31]) - m_run);
+                const float p1 = ex2_approx(__uint_as_float(sr[(key + 1) >> 5][(key + 1) & 31]) - m_run);
+                const __half2 hp = __floats2half2_rn(p0, p1);
+                lsum += __low2float(hp) + __high2float(hp);
+                pk[i] = *reinterpret_cast<const uint32_t*>(&hp);
+            }
+            tmem_st32(tS + lane_base + c2 * 32, pk);
+        }
+        tmem_st_wait();
+        l_run += lsum;
+        tc_fence_before();
+        __syncthreads();
+        // ---- issue O += P v, then (after it completes) the next S
+        if (warp == 0) {
+            if (lane == 0 && !*abort_flag) {
+                tc_fence_after();
+                if (!mbar_wait(bar_v, j & 1, tmo, abort_flag)) {
+                    fail();
+                } else {
+                    ++n_v_done;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        if (kk * 16 >= blk) break;
+                        const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, static_cast<uint32_t>(blk) * 128, 1024);
+                        umma_ts(tO, tS + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_o);
+                    ++n_o_issued;
+                    if (!mbar_wait(bar_o, j & 1, tmo, abort_flag)) {
+                        fail();
+                    } else {
+                        ++n_o_done;
+                        if (j + 1 < keep) {
+                            load_kv(bar_v, sv, &tm_v, next_beta);
+                            ++n_v_issued;
+                            if (mbar_wait(bar_k, (j + 1) & 1, tmo, abort_flag)) {
+                                ++n_k_done;
+                                tc_fence_after();
+                                issue_s();
+                                ++n_s_issued;
+                            } else {
+                                fail();
+                            }
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    tc_fence_after();
+    const bool aborted = *abort_flag != 0;
+
+    // ------------------------------------------------------------------ epilogue
+    const int i_row = warp * 32 + lane;
+    const int n = alpha * blk + i_row;
+    const bool row_valid = (i_row < blk) && (n < g.L) && !aborted;
+    float acc[D];
+#pragma unroll
+    for (int e = 0; e < D; ++e) acc[e] = 0.f;
+    float inv_den = 0.f;
+    if (a.lowrank && !aborted) {
+        float* As = reinterpret_cast<float*>(smem);  // [D][R] fp32, reuses the tile buffers
+        for (int e = tid; e < D * g.R; e += kThreads) As[e] = __bfloat162float(a.A[e]);
+        __syncthreads();
+        if (row_valid) {
+            const __nv_bfloat16* qrow = a.q_raw + ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;
+            const float* Sh = a.S + static_cast<size_t>(bh) * g.R * D;
+            const float* zh = a.z + static_cast<size_t>(bh) * g.R;
+            float den = 0.f;
+            for (int c0 = 0; c0 < g.R; c0 += 16) {
+                float phi[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) phi[c] = 0.f;
+                for (int d0 = 0; d0 < D; d0 += 8) {
+                    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow + d0));
+                    const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 qf = __bfloat1622float2(q2[u]);
+                        const float* a0 = As + (d0 + 2 * u) * g.R + c0;
+                        const float* a1 = a0 + g.R;
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) phi[c] = fmaf(qf.y, a1[c], fmaf(qf.x, a0[c], phi[c]));
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    phi[c] = fmaxf(phi[c], 0.f);
+                    den = fmaf(phi[c], __ldg(zh + c0 + c), den);
+                }
+#pragma unroll
+                for (int pp = 0; pp < 8; ++pp) {
+                    const int2 pi = __ldg(a.pairs + (c0 >> 1) + pp);  // (axis, table offset)
+                    const double2 cs = __ldg(a.tab + pi.y + token_axis_pos(n, pi.x, g.H, g.W));
+                    const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+                    const float x0 = phi[2 * pp], x1 = phi[2 * pp + 1];
+                    phi[2 * pp] = x0 * cf - x1 * sf;
+                    phi[2 * pp + 1] = x0 * sf + x1 * cf;
+                }
+#pragma unroll 4
+                for (int c = 0; c < 16; ++c) {
+                    const float4* s4 = reinterpret_cast<const float4*>(Sh + (c0 + c) * D);
+#pragma unroll
+                    for (int e4 = 0; e4 < D / 4; ++e4) {
+                        const float4 sv4 = __ldg(s4 + e4);
+                        acc[4 * e4 + 0] = fmaf(phi[c], sv4.x, acc[4 * e4 + 0]);
+                        acc[4 * e4 + 1] = fmaf(phi[c], sv4.y, acc[4 * e4 + 1]);
+                        acc[4 * e4 + 2] = fmaf(phi[c], sv4.z, acc[4 * e4 + 2]);
+                        acc[4 * e4 + 3] = fmaf(phi[c], sv4.w, acc[4 * e4 + 3]);
+                    }
+                }
+            }
+            inv_den = 1.f / (den + 1e-6f);
+        }
+    }
+    const float inv_l = (keep > 0 && l_run > 0.f) ? 1.f / l_run : 0.f;
+    const bool warp_has_rows = (warp * 32 < blk) && (alpha * blk + warp * 32 < g.L) && !aborted;
+    if (warp_has_rows) {
+        const size_t obase = ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            if (keep > 0) {
+                tmem_ld32(tO + lane_base + c * 32, o);
+                tmem_ld_wait(o);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = 0u;
+            }
+            if (row_valid) {
+                float r[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(o[i]) * inv_l + acc[c * 32 + i] * inv_den;
+                if (a.out_bf16) {
+                    __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(a.out) + obase + c * 32;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 pk;
+                        __nv_bfloat162 t0 = __floats2bfloat162_rn(r[i], r[i + 1]);
+                        __nv_bfloat162 t1 = __floats2bfloat162_rn(r[i + 2], r[i + 3]);
+                        __nv_bfloat162 t2 = __floats2bfloat162_rn(r[i + 4], r[i + 5]);
+                        __nv_bfloat162 t3 = __floats2bfloat162_rn(r[i + 6], r[i + 7]);
+                        pk.x = *reinterpret_cast<uint32_t*>(&t0);
+                        pk.y = *reinterpret_cast<uint32_t*>(&t1);
+                        pk.z = *reinterpret_cast<uint32_t*>(&t2);
+                        pk.w = *reinterpret_cast<uint32_t*>(&t3);
+                        *reinterpret_cast<uint4*>(op + i) = pk;
+                    }
+                } else {
+                    float* op = reinterpret_cast<float*>(a.out) + obase + c * 32;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(op + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                }
+            }
+        }
+    }
+    // ------------------------------------------------------------------ teardown
+    if (aborted && tid == 0) {
+        // Let copies and products still in flight land before the memory is released.  Each wait is
+        // bounded (10 ms) and ignores the abort flag.
+        volatile int no_abort = 0;
+        const uint64_t drain = 10000000ull;
+        if (n_q_issued > n_q_done) mbar_wait(bar_q, 0, drain, &no_abort);
+        if (n_k_issued > n_k_done) mbar_wait(bar_k, n_k_done & 1, drain, &no_abort);
+        if (n_v_issued > n_v_done) mbar_wait(bar_v, n_v_done & 1, drain, &no_abort);
+        if (n_s_issued > n_s_done) mbar_wait(bar_s, n_s_done & 1, drain, &no_abort);
+        if (n_o_issued > n_o_done) mbar_wait(bar_o, n_o_done & 1, drain, &no_abort);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+size_t attn_smem_bytes(const Geom& g) {
+    return (g.D == 128 ? AttnLayout<128>::kBytes : AttnLayout<64>::kBytes) + 1024;
+}
+
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st) {
+    dim3 grid(g.nb, g.BH());
+    const size_t sm = attn_smem_bytes(g);
+    cudaError_t e;
+    if (g.D == 128) {
+        e = cudaFuncSetAttribute(attn_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        attn_sm100_kernel<128><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, a, g);
+    } else {
+        e = cudaFuncSetAttribute(attn_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        attn_sm100_kernel<64><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, a, g);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace slra

@@ -1,0 +1,77 @@
+// Internal parameter blocks shared by the kernels and the C-ABI layer of libslra.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace slra {
+
+constexpr int kMaxPairs = 64;  // head_dim <= 128
+
+// Bits of the device status word.
+constexpr int kDevTimeout = 1;
+constexpr int kDevRange = 2;
+
+// Sizes of one call.  L = T*H*W; Lp = nb*block (rows of the padded head-major buffers).
+struct Geom {
+    int B, Hh, D, T, H, W, L, block, nb, keep, R, Lp;
+    int BH() const { return B * Hh; }
+};
+
+// 3D RoPE schedule: pair j rotates with the position along axis[j]; its cos/sin for position p
+// (0-based grid coordinate; the constant offset is folded into the table) is tab[tab_off[j] + p].
+struct RopeMeta {
+    int npairs;
+    int axis[kMaxPairs];
+    int mloc[kMaxPairs];   // index of the pair within its axis
+    int apairs[3];         // pairs per axis
+    int tab_off[kMaxPairs];
+    int axis_len[3];       // T, H, W
+    long long off[3];      // position offsets
+    double theta;
+};
+
+__host__ __device__ inline int token_axis_pos(int n, int axis, int H, int W) {
+    return axis == 0 ? n / (H * W) : (axis == 1 ? (n / W) % H : n % W);
+}
+
+// ---- launchers (defined in prep_kernels.cu and attn_sm100.cu) --------------------------------
+cudaError_t launch_rope_table(double2* tab, int2* pairs, const RopeMeta& meta, int entries, cudaStream_t st);
+cudaError_t launch_rope_pool(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                             const double2* tab, const int2* pairs, const Geom& g, __half* qh, __half* kh,
+                             __half* vh, double* qbar, double* kbar, int* status, cudaStream_t st);
+cudaError_t launch_select(const double* qbar, const double* kbar, const Geom& g, int32_t* idx, uint8_t* tie,
+                          cudaStream_t st);
+cudaError_t launch_lowrank_partial(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,
+                                   const double2* tab, const int2* pairs, const Geom& g, int nsplit,
+                                   float* s_part, float* z_part, cudaStream_t st);
+cudaError_t launch_lowrank_reduce(const float* s_part, const float* z_part, const Geom& g, int nsplit, float* S,
+                                  float* z, cudaStream_t st);
+
+// fp16 head-major [BH*Lp][D] tensor maps; q box 64 x 128 rows, k/v box 64 x `block` rows, 128-B swizzle.
+struct AttnMaps {
+    CUtensorMap q, k, v;
+};
+
+struct AttnArgs {
+    const int32_t* idx;
+    int keep;  // 0: no sparse branch
+    const __nv_bfloat16* q_raw;
+    const __nv_bfloat16* A;
+    const float* S;
+    const float* z;
+    const double2* tab;
+    const int2* pairs;  // per rotary pair: (axis, offset of its cos/sin table)
+    int lowrank;  // add the low-rank readout
+    void* out;
+    int out_bf16;
+    int* status;
+    unsigned long long timeout_ns;
+};
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st);
+size_t attn_smem_bytes(const Geom& g);
+
+}  // namespace slra

@@ -1,0 +1,431 @@
+// Preparation kernels of the hybrid attention forward (all HBM- or latency-bound, CUDA cores):
+//   rope_table      cos/sin of every (rotary pair, grid position), fp64
+//   rope_pool       3D RoPE of q and k, fp16 head-major copies of q^, k^ and v for the tensor-core
+//                   kernel, fp64 block means of q^ and k^
+//   select          fp64 block scores qbar . kbar and per-row top-k (radix select, lower index wins ties)
+//   lowrank_partial phi = relu(k A), rank-truncated RoPE outside the activation, split-L partial sums
+//                   of S = sum_j psi(k_j) v_j^T and z = sum_j phi(k_j)
+//   lowrank_reduce  fixed-order sum of the partials (deterministic)
+// Method: RoLA ("3 Preliminary" 3D RoPE; "4.1" block-sparse + low-rank branches; "4.2" first r rotary
+// coordinates; "4.3" RoPE outside the activation; "B.1" one query-independent sum per head).
+#include "common.cuh"
+
+namespace slra {
+
+// ------------------------------------------------------------------------------ rope_table
+__global__ void rope_table_kernel(double2* tab, int2* pairs, RopeMeta meta, int entries) {
+    int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e < meta.npairs) pairs[e] = make_int2(meta.axis[e], meta.tab_off[e]);
+    if (e >= entries) return;
+    int j = 0;
+    while (j + 1 < meta.npairs && meta.tab_off[j + 1] <= e) ++j;
+    int a = meta.axis[j];
+    int p = e - meta.tab_off[j];
+    double da = 2.0 * static_cast<double>(meta.apairs[a]);
+    double omega = pow(meta.theta, -2.0 * static_cast<double>(meta.mloc[j]) / da);
+    double ang = static_cast<double>(p + meta.off[a]) * omega;
+    double s, c;
+    sincos(ang, &s, &c);
+    tab[e] = make_double2(c, s);
+}
+
+cudaError_t launch_rope_table(double2* tab, int2* pairs, const RopeMeta& meta, int entries, cudaStream_t st) {
+    const int n = entries > meta.npairs ? entries : meta.npairs;
+    rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(tab, pairs, meta, entries);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------ rope_pool
+// One CTA per (query/key block, batch*head).  Thread t owns rotary pair j = t % (D/2) and walks the
+// block's tokens with stride 256/(D/2).  A warp touches 32 consecutive pairs (128 contiguous bytes)
+// of one token per load.  The rotation and the block sums are fp64 so the selection scores are
+// exact to ~1e-15 relative (the top-k decision is made on them).
+template <int D>
+__global__ void __launch_bounds__(256) rope_pool_kernel(const __nv_bfloat16* __restrict__ q,
+                                                        const __nv_bfloat16* __restrict__ k,
+                                                        const __nv_bfloat16* __restrict__ v,
+                                                        const double2* __restrict__ tab,
+                                                        const int2* __restrict__ pairs, Geom g,
+                                                        __half* __restrict__ qh, __half* __restrict__ kh,
+                                                        __half* __restrict__ vh, double* __restrict__ qbar,
+                                                        double* __restrict__ kbar, int* status) {
+    constexpr int P = D / 2;
+    constexpr int G = 256 / P;
+    __shared__ double red[G][4][P];
+    const int j = threadIdx.x % P, grp = threadIdx.x / P;
+    const int alpha = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int n0 = alpha * g.block;
+    const int2 pinfo = pairs[j];
+    const int axis = pinfo.x;
+    const int toff = pinfo.y;
+    double sq0 = 0.0, sq1 = 0.0, sk0 = 0.0, sk1 = 0.0;
+    bool bad = false;
+    for (int i = grp; i < g.block; i += G) {
+        const int n = n0 + i;
+        const size_t dst = (static_cast<size_t>(bh) * g.Lp + n) * D + 2 * j;
+        if (n < g.L) {
+            const double2 cs = tab[toff + token_axis_pos(n, axis, g.H, g.W)];
+            const size_t src = ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D + 2 * j;
+            const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + src));
+            const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + src));
+            const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + src));
+            const double qy0 = static_cast<double>(qf.x) * cs.x - static_cast<double>(qf.y) * cs.y;
+            const double qy1 = static_cast<double>(qf.x) * cs.y + static_cast<double>(qf.y) * cs.x;
+            const double ky0 = static_cast<double>(kf.x) * cs.x - static_cast<double>(kf.y) * cs.y;
+            const double ky1 = static_cast<double>(kf.x) * cs.y + static_cast<double>(kf.y) * cs.x;
+            sq0 += qy0; sq1 += qy1; sk0 += ky0; sk1 += ky1;
+            const float m = fmaxf(fmaxf(fabsf(static_cast<float>(qy0)), fabsf(static_cast<float>(qy1))),
+                                  fmaxf(fmaxf(fabsf(static_cast<float>(ky0)), fabsf(static_cast<float>(ky1))),
+                                        fmaxf(fabsf(vf.x), fabsf(vf.y))));
+            bad |= !(m <= 65504.0f);
+            *reinterpret_cast<__half2*>(qh + dst) = __floats2half2_rn(static_cast<float>(qy0), static_cast<float>(qy1));
+            *reinterpret_cast<__half2*>(kh + dst) = __floats2half2_rn(static_cast<float>(ky0), static_cast<float>(ky1));
+            *reinterpret_cast<__half2*>(vh + dst) = __floats2half2_rn(vf.x, vf.y);
+        } else {
+            const __half2 z2 = __floats2half2_rn(0.f, 0.f);
+            *reinterpret_cast<__half2*>(qh + dst) = z2;
+            *reinterpret_cast<__half2*>(kh + dst) = z2;
+            *reinterpret_cast<__half2*>(vh + dst) = z2;
+        }
+    }
+    red[grp][0][j] = sq0; red[grp][1][j] = sq1; red[grp][2][j] = sk0; red[grp][3][j] = sk1;
+    __syncthreads();
+    if (grp == 0) {
+        double a0 = 0.0, a1 = 0.0, c0 = 0.0, c1 = 0.0;
+        for (int u = 0; u < G; ++u) { a0 += red[u][0][j]; a1 += red[u][1][j]; c0 += red[u][2][j]; c1 += red[u][3][j]; }
+        const int cnt = min(g.block, g.L - n0);
+        const size_t o = (static_cast<size_t>(bh) * g.nb + alpha) * D + 2 * j;
+        qbar[o] = a0 / cnt; qbar[o + 1] = a1 / cnt;
+        kbar[o] = c0 / cnt; kbar[o + 1] = c1 / cnt;
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, kDevRange);
+}
+
+cudaError_t launch_rope_pool(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                             const double2* tab, const int2* pairs, const Geom& g, __half* qh, __half* kh,
+                             __half* vh, double* qbar, double* kbar, int* status, cudaStream_t st) {
+    dim3 grid(g.nb, g.BH());
+    if (g.D == 128)
+        rope_pool_kernel<128><<<grid, 256, 0, st>>>(q, k, v, tab, pairs, g, qh, kh, vh, qbar, kbar, status);
+    else
+        rope_pool_kernel<64><<<grid, 256, 0, st>>>(q, k, v, tab, pairs, g, qh, kh, vh, qbar, kbar, status);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------ select
+// Order-preserving map of a double to uint64 (-0.0 folded into +0.0 first).
+__device__ __forceinline__ uint64_t ordered_key(double x) {
+    x = x + 0.0;
+    const uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+__device__ __forceinline__ double key_value(uint64_t k) {
+    const uint64_t u = (k >> 63) ? (k & 0x7FFFFFFFFFFFFFFFull) : ~k;
+    return __longlong_as_double(static_cast<long long>(u));
+}
+
+constexpr int kSelRows = 8;  // query blocks per CTA (one warp each in the selection phase)
+
+// One CTA per (8 query blocks, batch*head).  Phase 1: fp64 dot products of the 8 qbar rows with all
+// kbar rows, staged 32 key blocks at a time through shared memory.  Phase 2: warp w selects row w's
+// top-k by an 8-pass radix select on the order-preserving 64-bit keys, then writes the selected block
+// indices in ascending order (ties at the threshold resolved to the lowest indices) and the tie flag.
+template <int D>
+__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ qbar,
+                                                     const double* __restrict__ kbar, Geom g,
+                                                     int32_t* __restrict__ idx, uint8_t* __restrict__ tie) {
+    extern __shared__ __align__(16) unsigned char sm_raw[];
+    double* qrow = reinterpret_cast<double*>(sm_raw);          // [8][D]
+    double* kch = qrow + kSelRows * D;                          // [32][D+1]
+    double* scores = kch + 32 * (D + 1);                        // [8][nb]
+    int* hist = reinterpret_cast<int*>(scores + kSelRows * g.nb);  // [8][256]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bh = blockIdx.y;
+    const int a0 = blockIdx.x * kSelRows;
+    const int nb = g.nb;
+    const double* qb = qbar + static_cast<size_t>(bh) * nb * D;
+    const double* kb = kbar + static_cast<size_t>(bh) * nb * D;
+
+    for (int e = tid; e < kSelRows * D; e += 256) {
+        const int r = e / D;
+        qrow[e] = (a0 + r < nb) ? qb[static_cast<size_t>(a0 + r) * D + (e % D)] : 0.0;
+    }
+    for (int c0 = 0; c0 < nb; c0 += 32) {
+        __syncthreads();
+        for (int e = tid; e < 32 * D; e += 256) {
+            const int i = e / D, d = e % D;
+            kch[i * (D + 1) + d] = (c0 + i < nb) ? kb[static_cast<size_t>(c0 + i) * D + d] : 0.0;
+        }
+        __syncthreads();
+        const int r = tid >> 5, c = tid & 31;
+        if (c0 + c < nb) {
+            const double* qr = qrow + r * D;
+            const double* kr = kch + c * (D + 1);
+            double acc = 0.0;
+#pragma unroll 8
+            for (int d = 0; d < D; ++d) acc = fma(qr[d], kr[d], acc);
+            scores[r * nb + c0 + c] = acc;
+        }
+    }
+    __syncthreads();
+
+    const int alpha = a0 + warp;
+    if (alpha >= nb) return;
+    const double* srow = scores + warp * nb;
+    int* hw = hist + warp * 256;
+    const int keep = g.keep;
+    uint64_t prefix = 0, pmask = 0;
+    int rem = keep;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int i = lane; i < 256; i += 32) hw[i] = 0;
+        __syncwarp();
+        for (int i = lane; i < nb; i += 32) {
+            const uint64_t u = ordered_key(srow[i]);
+            if ((u & pmask) == prefix) atomicAdd(&hw[(u >> shift) & 255], 1);
+        }
+        __syncwarp();
+        // lane owns bins 255-8*lane .. 248-8*lane (descending)
+        int cnt[8], local = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) { cnt[t] = hw[255 - (lane * 8 + t)]; local += cnt[t]; }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int nbv = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += nbv;
+        }
+        const int excl = incl - local;
+        const unsigned owner = __ballot_sync(0xffffffffu, excl < rem && rem <= incl);
+        const int src = __ffs(owner) - 1;
+        int binsel = 0, above = 0;
+        if (lane == src) {
+            int acc = excl;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                if (acc + cnt[t] >= rem) { binsel = 255 - (lane * 8 + t); above = acc; break; }
+                acc += cnt[t];
+            }
+        }
+        binsel = __shfl_sync(0xffffffffu, binsel, src);
+        above = __shfl_sync(0xffffffffu, above, src);
+        rem -= above;
+        prefix |= static_cast<uint64_t>(binsel) << shift;
+        pmask |= 0xFFull << shift;
+        __syncwarp();
+    }
+    // prefix = key of the k-th largest score; take every larger key and the first `rem` equal ones.
+    int32_t* out = idx + (static_cast<size_t>(bh) * nb + alpha) * keep;
+    int written = 0, eq_seen = 0;
+    uint64_t next_best = 0;
+    bool has_next = false;
+    for (int base = 0; base < nb; base += 32) {
+        const int i = base + lane;
+        const bool valid = i < nb;
+        const uint64_t u = valid ? ordered_key(srow[i]) : 0;
+        const bool gt = valid && u > prefix;
+        const bool eq = valid && u == prefix;
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        const unsigned below = (1u << lane) - 1u;
+        const bool sel = gt || (eq && (eq_seen + __popc(eqm & below)) < rem);
+        const unsigned selm = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[written + __popc(selm & below)] = i;
+        written += __popc(selm);
+        eq_seen += __popc(eqm);
+        if (valid && !sel && (!has_next || u > next_best)) { next_best = u; has_next = true; }
+    }
+    // (k+1)-th largest = max over the unselected keys
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t ob = __shfl_xor_sync(0xffffffffu, next_best, o);
+        const int oh = __shfl_xor_sync(0xffffffffu, has_next ? 1 : 0, o);
+        if (oh && (!has_next || ob > next_best)) { next_best = ob; has_next = true; }
+    }
+    if (lane == 0) {
+        uint8_t t = 0;
+        if (keep < nb && has_next) {
+            const double sk = key_value(prefix), sk1 = key_value(next_best);
+            t = (sk - sk1) <= 1e-6 * fmax(1.0, fabs(sk));
+        }
+        tie[static_cast<size_t>(bh) * nb + alpha] = t;
+    }
+}
+
+static size_t select_smem(const Geom& g) {
+    return sizeof(double) * (kSelRows * g.D + 32 * (g.D + 1) + static_cast<size_t>(kSelRows) * g.nb) +
+           sizeof(int) * kSelRows * 256;
+}
+
+cudaError_t launch_select(const double* qbar, const double* kbar, const Geom& g, int32_t* idx, uint8_t* tie,
+                          cudaStream_t st) {
+    dim3 grid((g.nb + kSelRows - 1) / kSelRows, g.BH());
+    const size_t sm = select_smem(g);
+    cudaError_t e;
+    if (g.D == 128) {
+        e = cudaFuncSetAttribute(select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        select_kernel<128><<<grid, 256, sm, st>>>(qbar, kbar, g, idx, tie);
+    } else {
+        e = cudaFuncSetAttribute(select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        select_kernel<64><<<grid, 256, sm, st>>>(qbar, kbar, g, idx, tie);
+    }
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------ low-rank summary
+constexpr int kLrTile = 32;  // tokens per step
+
+// One CTA per (split of the sequence, batch*head).  Per 32-token step: stage raw k and v (fp32) in
+// shared memory, phi = relu(k A) (thread per (token, feature)), rotate the first R coordinates with
+// the token's 3D RoPE angles (psi), then accumulate S[c][e] += sum_t psi[t][c] v[t][e] in registers
+// (thread owns one e and R/(256/D) features) and z[c] += sum_t phi[t][c].
+template <int D, int R>
+__global__ void __launch_bounds__(256) lowrank_partial_kernel(const __nv_bfloat16* __restrict__ k,
+                                                              const __nv_bfloat16* __restrict__ v,
+                                                              const __nv_bfloat16* __restrict__ A,
+                                                              const double2* __restrict__ tab,
+                                                              const int2* __restrict__ pairs, Geom g, int nsplit, float* __restrict__ s_part,
+                                                              float* __restrict__ z_part) {
+    extern __shared__ __align__(16) float smf[];
+    float* As = smf;                        // [D][R]
+    float* ks = As + D * R;                 // [32][D+1]
+    float* vs = ks + kLrTile * (D + 1);     // [32][D]
+    float* ph = vs + kLrTile * D;           // [32][R+1]
+    float* ps = ph + kLrTile * (R + 1);     // [32][R]
+    constexpr int G = 256 / D;              // feature groups
+    constexpr int NA = R / G;               // accumulators per thread
+    const int tid = threadIdx.x;
+    const int split = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int ntiles = (g.L + kLrTile - 1) / kLrTile;
+    const int per = (ntiles + nsplit - 1) / nsplit;
+    const int t0 = split * per, t1 = min(ntiles, t0 + per);
+
+    for (int e = tid; e < D * R; e += 256) As[e] = __bfloat162float(A[e]);
+    const int e_own = tid % D, cg = tid / D;
+    float acc[NA];
+#pragma unroll
+    for (int i = 0; i < NA; ++i) acc[i] = 0.f;
+    float zacc = 0.f;
+
+    for (int tile = t0; tile < t1; ++tile) {
+        const int n0 = tile * kLrTile;
+        __syncthreads();
+        for (int e = tid; e < kLrTile * (D / 2); e += 256) {
+            const int tt = e / (D / 2), dp = e % (D / 2);
+            const int n = n0 + tt;
+            float2 kf = make_float2(0.f, 0.f), vf = make_float2(0.f, 0.f);
+            if (n < g.L) {
+                const size_t src = ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D + 2 * dp;
+                kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + src));
+                vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + src));
+            }
+            ks[tt * (D + 1) + 2 * dp] = kf.x; ks[tt * (D + 1) + 2 * dp + 1] = kf.y;
+            vs[tt * D + 2 * dp] = vf.x; vs[tt * D + 2 * dp + 1] = vf.y;
+        }
+        __syncthreads();
+        for (int o = tid; o < kLrTile * R; o += 256) {
+            const int tt = o / R, c = o % R;
+            const float* kr = ks + tt * (D + 1);
+            float a = 0.f;
+#pragma unroll 16
+            for (int d = 0; d < D; ++d) a = fmaf(kr[d], As[d * R + c], a);
+            ph[tt * (R + 1) + c] = fmaxf(a, 0.f);
+        }
+        __syncthreads();
+        for (int o = tid; o < kLrTile * (R / 2); o += 256) {
+            const int tt = o / (R / 2), p = o % (R / 2);
+            const int n = n0 + tt;
+            const float x0 = ph[tt * (R + 1) + 2 * p], x1 = ph[tt * (R + 1) + 2 * p + 1];
+            float c = 1.f, s = 0.f;
+            if (n < g.L) {
+                const int2 pi = pairs[p];
+                const double2 cs = tab[pi.y + token_axis_pos(n, pi.x, g.H, g.W)];
+                c = static_cast<float>(cs.x);
+                s = static_cast<float>(cs.y);
+            }
+            ps[tt * R + 2 * p] = x0 * c - x1 * s;
+            ps[tt * R + 2 * p + 1] = x0 * s + x1 * c;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int tt = 0; tt < kLrTile; ++tt) {
+            const float vv = vs[tt * D + e_own];
+            const float* pr = ps + tt * R + cg;
+#pragma unroll
+            for (int i = 0; i < NA; ++i) acc[i] = fmaf(pr[G * i], vv, acc[i]);
+        }
+        if (tid < R)
+            for (int tt = 0; tt < kLrTile; ++tt) zacc += ph[tt * (R + 1) + tid];
+    }
+    float* sp = s_part + (static_cast<size_t>(bh) * nsplit + split) * R * D;
+#pragma unroll
+    for (int i = 0; i < NA; ++i) sp[(cg + G * i) * D + e_own] = acc[i];
+    if (tid < R) z_part[(static_cast<size_t>(bh) * nsplit + split) * R + tid] = zacc;
+}
+
+template <int D, int R>
+static cudaError_t lr_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,
+                             const double2* tab, const int2* pairs, const Geom& g, int nsplit, float* s_part,
+                             float* z_part, cudaStream_t st) {
+    const size_t sm = sizeof(float) * (D * R + kLrTile * (D + 1) + kLrTile * D + kLrTile * (R + 1) + kLrTile * R);
+    cudaError_t e = cudaFuncSetAttribute(lowrank_partial_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sm);
+    if (e != cudaSuccess) return e;
+    lowrank_partial_kernel<D, R><<<dim3(nsplit, g.BH()), 256, sm, st>>>(k, v, A, tab, pairs, g, nsplit, s_part, z_part);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lowrank_partial(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,
+                                   const double2* tab, const int2* pairs, const Geom& g, int nsplit,
+                                   float* s_part, float* z_part, cudaStream_t st) {
+    if (g.D == 128) {
+        switch (g.R) {
+            case 16: return lr_launch<128, 16>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 32: return lr_launch<128, 32>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 48: return lr_launch<128, 48>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 64: return lr_launch<128, 64>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 80: return lr_launch<128, 80>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 96: return lr_launch<128, 96>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 112: return lr_launch<128, 112>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 128: return lr_launch<128, 128>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+        }
+    } else if (g.D == 64) {
+        switch (g.R) {
+            case 16: return lr_launch<64, 16>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 32: return lr_launch<64, 32>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 48: return lr_launch<64, 48>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+            case 64: return lr_launch<64, 64>(k, v, A, tab, pairs, g, nsplit, s_part, z_part, st);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+__global__ void lowrank_reduce_kernel(const float* __restrict__ s_part, const float* __restrict__ z_part, int RD,
+                                      int R, int nsplit, float* __restrict__ S, float* __restrict__ z) {
+    const int bh = blockIdx.y;
+    const int o = blockIdx.x * blockDim.x + threadIdx.x;
+    if (o < RD) {
+        const float* p = s_part + static_cast<size_t>(bh) * nsplit * RD + o;
+        float a = 0.f;
+        for (int s = 0; s < nsplit; ++s) a += p[static_cast<size_t>(s) * RD];
+        S[static_cast<size_t>(bh) * RD + o] = a;
+    } else if (o < RD + R) {
+        const int c = o - RD;
+        const float* p = z_part + static_cast<size_t>(bh) * nsplit * R + c;
+        float a = 0.f;
+        for (int s = 0; s < nsplit; ++s) a += p[static_cast<size_t>(s) * R];
+        z[static_cast<size_t>(bh) * R + c] = a;
+    }
+}
+
+cudaError_t launch_lowrank_reduce(const float* s_part, const float* z_part, const Geom& g, int nsplit, float* S,
+                                  float* z, cudaStream_t st) {
+    const int RD = g.R * g.D;
+    dim3 grid((RD + g.R + 255) / 256, g.BH());
+    lowrank_reduce_kernel<<<grid, 256, 0, st>>>(s_part, z_part, RD, g.R, nsplit, S, z);
+    return cudaGetLastError();
+}
+
+}  // namespace slra

@@ -1,0 +1,257 @@
+"""Python binding of libslra.so (the C ABI in include/slra.h): argument marshalling only.
+
+Every step of the forward pass runs in the library's CUDA kernels; this module only fills the
+problem struct, hands device pointers (torch tensors' storage) and the current torch stream to the
+C entry points, and raises on a non-zero status.  If the library cannot be loaded the calls raise:
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libslra.so")
+
+OK = 0
+ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_RANGE, \
+    ERR_NO_DEVICE = range(1, 9)
+OUT_F32, OUT_BF16 = 0, 1
+BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
+
+# Every symbol include/slra.h declares.
+EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_validate", "slra_keep_count",
+           "slra_workspace_layout", "slra_attn_fwd", "slra_host_io_bytes", "slra_attn_fwd_host",
+           "slra_select_blocks", "slra_lowrank_summary", "slra_device_status")
+
+
+class SlraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("heads", ctypes.c_int64), ("head_dim", ctypes.c_int64),
+                ("T", ctypes.c_int64), ("H", ctypes.c_int64), ("W", ctypes.c_int64),
+                ("block", ctypes.c_int64), ("keep_frac", ctypes.c_double), ("rank", ctypes.c_int64),
+                ("theta", ctypes.c_double), ("out_dtype", ctypes.c_int32), ("branches", ctypes.c_int32),
+                ("pos_offset", ctypes.c_int64 * 3), ("rope_split", ctypes.c_int64 * 3),
+                ("wait_timeout_ns", ctypes.c_uint64), ("attn_events", ctypes.c_void_p * 2)]
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [("total_bytes", ctypes.c_size_t), ("L", ctypes.c_int64), ("nb", ctypes.c_int64),
+                ("keep", ctypes.c_int64), ("nsplit", ctypes.c_int64)] + \
+               [(n, ctypes.c_size_t) for n in ("status", "rope_table", "qh", "kh", "vh", "qbar", "kbar", "idx",
+                                               "tie", "s_part", "z_part", "S", "z")]
+
+
+_lib = None
+
+
+def lib():
+    """Load libslra.so (raises if it is missing: the CUDA path has no substitute)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m sparse_rank_hybrid_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S = ctypes.c_void_p, ctypes.c_size_t
+        PP = ctypes.POINTER(_Problem)
+        L.slra_abi_version.restype = ctypes.c_int
+        L.slra_status_string.restype = ctypes.c_char_p
+        L.slra_status_string.argtypes = [ctypes.c_int]
+        L.slra_problem_init.argtypes = [PP] + [ctypes.c_int64] * 7 + [ctypes.c_double, ctypes.c_int64]
+        L.slra_validate.argtypes = [PP]
+        L.slra_keep_count.restype = ctypes.c_int64
+        L.slra_keep_count.argtypes = [PP]
+        L.slra_workspace_layout.argtypes = [PP, ctypes.POINTER(_Layout)]
+        L.slra_attn_fwd.argtypes = [PP, P, P, P, P, P, P, S, P]
+        L.slra_host_io_bytes.restype = S
+        L.slra_host_io_bytes.argtypes = [PP]
+        L.slra_attn_fwd_host.argtypes = [PP, P, P, P, P, P, P, S, P, S, P]
+        L.slra_select_blocks.argtypes = [PP, P, P, P, P, S, P]
+        L.slra_lowrank_summary.argtypes = [PP, P, P, P, P, S, P]
+        L.slra_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+        for name in ("slra_problem_init", "slra_validate", "slra_workspace_layout", "slra_attn_fwd",
+                     "slra_attn_fwd_host", "slra_select_blocks", "slra_lowrank_summary", "slra_device_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().slra_status_string(int(s)).decode()
+
+
+def _check(s: int, where: str):
+    if s != OK:
+        raise SlraError(s, where)
+
+
+@dataclass
+class Problem:
+    batch: int
+    heads: int
+    head_dim: int
+    T: int
+    H: int
+    W: int
+    block: int
+    keep_frac: float
+    rank: int
+    theta: float = 1e4
+    out_dtype: int = OUT_F32
+    branches: int = BRANCH_BOTH
+    pos_offset: tuple = (0, 0, 0)
+    rope_split: tuple = (0, 0, 0)
+    wait_timeout_ns: int = 2_000_000_000
+    attn_events: tuple = (None, None)  # raw cudaEvent_t handles (ints) or None
+
+    @property
+    def L(self) -> int:
+        return self.T * self.H * self.W
+
+    @classmethod
+    def from_workload(cls, w, **kw) -> "Problem":
+        return cls(w.batch, w.heads, w.head_dim, w.T, w.H, w.W, w.block, w.keep_frac, w.rank, **kw)
+
+    def c(self) -> _Problem:
+        p = _Problem()
+        _check(lib().slra_problem_init(ctypes.byref(p), self.batch, self.heads, self.head_dim, self.T, self.H,
+                                       self.W, self.block, float(self.keep_frac), self.rank), "slra_problem_init")
+        p.theta = float(self.theta)
+        p.out_dtype = int(self.out_dtype)
+        p.branches = int(self.branches)
+        p.pos_offset[:] = [int(x) for x in self.pos_offset]
+        p.rope_split[:] = [int(x) for x in self.rope_split]
+        p.wait_timeout_ns = int(self.wait_timeout_ns)
+        p.attn_events[0] = self.attn_events[0]
+        p.attn_events[1] = self.attn_events[1]
+        return p
+
+
+@dataclass
+class Layout:
+    total_bytes: int
+    L: int
+    nb: int
+    keep: int
+    nsplit: int
+    offsets: dict = field(default_factory=dict)
+
+
+def validate(prob: Problem) -> int:
+    return int(lib().slra_validate(ctypes.byref(prob.c())))
+
+
+def keep_count(prob: Problem) -> int:
+    return int(lib().slra_keep_count(ctypes.byref(prob.c())))
+
+
+def layout(prob: Problem) -> Layout:
+    lay = _Layout()
+    _check(lib().slra_workspace_layout(ctypes.byref(prob.c()), ctypes.byref(lay)), "slra_workspace_layout")
+    offs = {n: int(getattr(lay, n)) for n, _ in _Layout._fields_[5:]}
+    return Layout(int(lay.total_bytes), int(lay.L), int(lay.nb), int(lay.keep), int(lay.nsplit), offs)
+
+
+# ------------------------------------------------------------------------------- torch helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> int:
+    return int(t.data_ptr())
+
+
+def _stream_handle(stream) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def alloc_workspace(prob: Problem, device="cuda"):
+    torch = _torch()
+    return torch.empty(layout(prob).total_bytes, dtype=torch.uint8, device=device)
+
+
+def _check_bf16(name, t, shape):
+    torch = _torch()
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected contiguous CUDA bf16 tensor of shape {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def attn_fwd(prob: Problem, q, k, v, A, out=None, workspace=None, stream=None):
+    """Full forward pass.  q, k, v: CUDA bf16 [B, L, Hh, D]; A: CUDA bf16 [D, rank].
+    Returns (out, workspace); out is fp32 or bf16 [B, L, Hh, D] as prob.out_dtype."""
+    torch = _torch()
+    shp = (prob.batch, prob.L, prob.heads, prob.head_dim)
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_bf16(n, t, shp)
+    _check_bf16("A", A, (prob.head_dim, prob.rank))
+    if out is None:
+        out = torch.empty(shp, dtype=torch.float32 if prob.out_dtype == OUT_F32 else torch.bfloat16,
+                          device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(prob, q.device)
+    _check(lib().slra_attn_fwd(ctypes.byref(prob.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(A), _ptr(out),
+                               _ptr(workspace), workspace.numel(), _stream_handle(stream)), "slra_attn_fwd")
+    return out, workspace
+
+
+def host_io_bytes(prob: Problem) -> int:
+    return int(lib().slra_host_io_bytes(ctypes.byref(prob.c())))
+
+
+def attn_fwd_host(prob: Problem, q_host, k_host, v_host, A_host, out_host, io, workspace, stream=None):
+    """Forward pass on host buffers (pinned CPU tensors): copies in, computes, copies out, synchronizes."""
+    _check(lib().slra_attn_fwd_host(ctypes.byref(prob.c()), _ptr(q_host), _ptr(k_host), _ptr(v_host),
+                                    _ptr(A_host), _ptr(out_host), _ptr(io), io.numel(), _ptr(workspace),
+                                    workspace.numel(), _stream_handle(stream)), "slra_attn_fwd_host")
+    return out_host
+
+
+def select_blocks(prob: Problem, q, k, v, workspace=None, stream=None):
+    if workspace is None:
+        workspace = alloc_workspace(prob, q.device)
+    _check(lib().slra_select_blocks(ctypes.byref(prob.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(workspace),
+                                    workspace.numel(), _stream_handle(stream)), "slra_select_blocks")
+    return workspace
+
+
+def lowrank_summary(prob: Problem, k, v, A, workspace=None, stream=None):
+    if workspace is None:
+        workspace = alloc_workspace(prob, k.device)
+    _check(lib().slra_lowrank_summary(ctypes.byref(prob.c()), _ptr(k), _ptr(v), _ptr(A), _ptr(workspace),
+                                      workspace.numel(), _stream_handle(stream)), "slra_lowrank_summary")
+    return workspace
+
+
+def device_status(workspace, stream=None) -> int:
+    st = ctypes.c_int32(-1)
+    _check(lib().slra_device_status(_ptr(workspace), _stream_handle(stream), ctypes.byref(st)),
+           "slra_device_status")
+    return int(st.value)
+
+
+def ws_view(prob: Problem, workspace, name: str):
+    """A typed view of one intermediate inside a workspace (see slra_ws_layout)."""
+    torch = _torch()
+    lay = layout(prob)
+    BH, nb, D, R, k = prob.batch * prob.heads, lay.nb, prob.head_dim, prob.rank, lay.keep
+    spec = {"qh": (torch.float16, (BH, nb * prob.block, D)), "kh": (torch.float16, (BH, nb * prob.block, D)),
+            "vh": (torch.float16, (BH, nb * prob.block, D)), "qbar": (torch.float64, (BH, nb, D)),
+            "kbar": (torch.float64, (BH, nb, D)), "idx": (torch.int32, (BH, nb, k)),
+            "tie": (torch.uint8, (BH, nb)), "S": (torch.float32, (BH, R, D)), "z": (torch.float32, (BH, R))}
+    dt, shape = spec[name]
+    off = lay.offsets[name]
+    n = 1
+    for s in shape:
+        n *= s
+    nbytes = n * torch.empty(0, dtype=dt).element_size()
+    return workspace[off:off + nbytes].view(dt).view(shape)

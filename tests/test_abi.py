@@ -1,0 +1,81 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol that
+include/slra.h declares, and validates problems / sizes workspaces without touching a device."""
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_rank_hybrid_b200 import build as B
+from sparse_rank_hybrid_b200 import slra
+from sparse_rank_hybrid_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "slra.h")).read()
+    return sorted(set(re.findall(r"\b(slra_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    out = subprocess.check_output(["nm", "-D", "--defined-only", B.LIB], text=True)
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    declared = _declared()
+    assert set(declared) == set(slra.EXPORTS)
+    missing = [s for s in declared if s not in exported]
+    assert not missing, missing
+    # nothing else leaks out of the library (internal C++ symbols are hidden)
+    assert {s for s in exported if s.startswith("slra_")} == set(declared)
+
+
+def test_abi_version_and_status_strings():
+    assert slra.lib().slra_abi_version() == 1
+    for s in range(0, 9):
+        assert slra.status_string(s) and slra.status_string(s) != "unknown status"
+    assert slra.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("w", list(W.MAIN.values()), ids=lambda w: w.name)
+def test_keep_count_and_layout(w, oracle_mod):
+    p = slra.Problem.from_workload(w)
+    assert slra.validate(p) == slra.OK
+    assert slra.keep_count(p) == oracle_mod.keep_count(w.keep_frac, w.nb)
+    lay = slra.layout(p)
+    assert lay.nb == w.nb and lay.L == w.L
+    offs = sorted(lay.offsets.values())
+    assert all(o % 256 == 0 for o in offs) and offs[0] == 0 and lay.total_bytes >= offs[-1]
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 96, slra.ERR_UNSUPPORTED), ("block", 32, slra.ERR_UNSUPPORTED),
+    ("rank", 24, slra.ERR_UNSUPPORTED), ("rank", 256, slra.ERR_UNSUPPORTED), ("rank", 0, slra.ERR_UNSUPPORTED),
+    ("keep_frac", 0.0, slra.ERR_INVALID_ARG), ("keep_frac", 1.5, slra.ERR_INVALID_ARG),
+    ("T", 0, slra.ERR_INVALID_ARG), ("heads", 0, slra.ERR_INVALID_ARG), ("out_dtype", 7, slra.ERR_INVALID_ARG),
+    ("rope_split", (10, 10, 10), slra.ERR_INVALID_ARG), ("branches", 9, slra.ERR_INVALID_ARG),
+    ("T", 5000, slra.ERR_UNSUPPORTED),  # 5000*45*80 tokens -> more than 2048 blocks
+])
+def test_validation_rejects(field, value, status):
+    p = slra.Problem.from_workload(W.WAN_14B)
+    setattr(p, field, value)
+    assert slra.validate(p) == status
+
+
+def test_calls_without_device_fail_cleanly():
+    """On a machine without a GPU every compute entry point returns an error status (never crashes)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("has a GPU")
+    p = slra.Problem.from_workload(W.TINY)
+    lay = slra.layout(p)
+    import ctypes
+    buf = ctypes.create_string_buffer(lay.total_bytes + 512)
+    base = (ctypes.addressof(buf) + 255) // 256 * 256
+    s = slra.lib().slra_attn_fwd(ctypes.byref(p.c()), base, base, base, base, base + 256, base, lay.total_bytes,
+                                 None)
+    assert s != slra.OK

@@ -1,0 +1,154 @@
+"""GPU parity: the C-ABI CUDA path against the fp64 oracle on the same seeded inputs.
+
+Small cases are compared element by element over every output; the large workloads (the
+configurations the benchmark times) on every mask row and S/z of sampled heads and on the outputs of
+sampled query blocks (first, last = ragged, and random ones).  Tolerances are in tests/parity.py.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from sparse_rank_hybrid_b200 import inputs as I
+from sparse_rank_hybrid_b200 import slra
+from sparse_rank_hybrid_b200 import workloads as W
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+REPORT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "gpurun_out", "parity_stats.jsonl")
+
+
+def _log(stats):
+    try:
+        os.makedirs(os.path.dirname(REPORT), exist_ok=True)
+        with open(REPORT, "a") as f:
+            f.write(json.dumps({k: (float(v) if isinstance(v, (np.floating,)) else v) for k, v in stats.items()}) + "\n")
+    except OSError:
+        pass
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_rank_hybrid_b200 import build
+    build.build()
+    import oracle
+    oracle.build()
+
+
+def _case(w, label=None, heads=None, qblocks=None, **kw):
+    p = slra.Problem.from_workload(w, **kw)
+    x = I.make_inputs(w)
+    gpu = parity.run_gpu(p, x)
+    st = parity.compare(p, x, gpu, heads=heads, qblocks=qblocks, label=label or w.name)
+    _log(st)
+    return st, gpu
+
+
+def test_tiny_full():
+    _case(W.TINY)
+
+
+def test_tiny_branches_separately():
+    _case(W.TINY, "tiny-sparse-only", branches=slra.BRANCH_SPARSE)
+    _case(W.TINY, "tiny-lowrank-only", branches=slra.BRANCH_LOWRANK)
+
+
+@pytest.mark.parametrize("grid,D,R,block,keep,B,heads", [
+    ((3, 10, 13), 128, 32, 128, 0.3, 1, 2),    # L = 390: ragged last block (6 tokens)
+    ((2, 9, 11), 64, 64, 64, 0.25, 2, 3),      # batch 2, D = 64, r = D, ragged (6 tokens)
+    ((1, 5, 7), 128, 16, 128, 0.1, 1, 1),      # L < block: one block, k = 1
+    ((4, 12, 16), 128, 128, 128, 1.0, 1, 2),   # keep everything: dense attention, r = D
+    ((4, 12, 16), 128, 64, 64, 0.05, 1, 2),    # block 64 with D = 128, keep = 1 of 12
+    ((5, 16, 20), 128, 48, 128, 0.2, 1, 3),    # r = 48 (not a power of two)
+])
+def test_edge_shapes(grid, D, R, block, keep, B, heads):
+    w = W.Workload(f"edge-{grid}-{D}-{R}-{block}-{keep}", B, heads, D, *grid, R, block, keep, 7000 + D + R)
+    _case(w)
+
+
+def test_shift_invariance_on_gpu():
+    """Shifting all positions leaves masks and outputs unchanged (within fp rounding)."""
+    w = W.TINY.with_(T=4, H=16, W=16, heads=2, block=64, keep_frac=0.25)
+    x = I.make_inputs(w)
+    p0 = slra.Problem.from_workload(w)
+    p1 = slra.Problem.from_workload(w, pos_offset=(3, -7, 11))
+    g0, g1 = parity.run_gpu(p0, x), parity.run_gpu(p1, x)
+    assert np.array_equal(g0["idx"], g1["idx"])
+    assert np.abs(g0["out"] - g1["out"]).max() < 1e-3
+
+
+def test_deterministic_and_bf16_out():
+    w = W.TINY.with_(T=4, H=16, W=16, heads=2, block=64, keep_frac=0.25)
+    x = I.make_inputs(w)
+    p = slra.Problem.from_workload(w)
+    a, b = parity.run_gpu(p, x), parity.run_gpu(p, x)
+    assert np.array_equal(a["out"], b["out"]) and np.array_equal(a["idx"], b["idx"])
+    pb = slra.Problem.from_workload(w, out_dtype=slra.OUT_BF16)
+    c = parity.run_gpu(pb, x)
+    # bf16 rounding of the output: at most half an ulp of bf16 (2^-9 relative) plus the fp32 error
+    assert np.all(np.abs(c["out"] - a["out"]) <= np.abs(a["out"]) * 2.0 ** -8 + 1e-6)
+
+
+def test_host_entry_point_matches_device():
+    import torch
+    w = W.TINY
+    x = I.make_inputs(w)
+    p = slra.Problem.from_workload(w)
+    dev = parity.run_gpu(p, x)["out"]
+    host = {n: torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v", "A")}
+    out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32).pin_memory()
+    io = torch.empty(slra.host_io_bytes(p), dtype=torch.uint8, device="cuda")
+    ws = slra.alloc_workspace(p)
+    slra.attn_fwd_host(p, host["q"], host["k"], host["v"], host["A"], out, io, ws)
+    assert np.array_equal(out.numpy().astype(np.float64), dev)
+
+
+def test_range_error_reported():
+    """An input too large for the fp16 operands is reported through the device status word."""
+    import torch
+    w = W.TINY
+    x = I.make_inputs(w)
+    q = parity.to_gpu(x["q"]).clone()
+    q[0, 5, 0, 3] = 1e6
+    k, v, A = (parity.to_gpu(x[n]) for n in ("k", "v", "A"))
+    p = slra.Problem.from_workload(w)
+    _, ws = slra.attn_fwd(p, q, k, v, A)
+    assert slra.device_status(ws) == slra.ERR_RANGE
+    assert slra.device_status(ws) == slra.OK  # reading clears it
+
+
+def _sample_blocks(nb, seed, n=3):
+    rng = np.random.default_rng(seed)
+    return sorted({0, nb - 1, *rng.choice(nb, size=n, replace=False).tolist()})
+
+
+def test_wan_1_3b_full_size():
+    w = W.WAN_1_3B
+    heads = [(0, 0), (0, 5), (0, 11)]
+    _case(w, heads=heads, qblocks=_sample_blocks(w.nb, 1))
+
+
+def test_wan_14b_bench_config():
+    """The configuration the benchmark times (Wan2.1-14B 720p, 75,600 tokens, 40 heads, keep 10%)."""
+    w = W.WAN_14B
+    heads = [(0, 0), (0, 17), (0, 39)]
+    _case(w, heads=heads, qblocks=_sample_blocks(w.nb, 2))
+
+
+@pytest.mark.slow
+def test_hunyuan_long():
+    w = W.HUNYUAN
+    heads = [(0, 0), (0, 23)]
+    _case(w, heads=heads, qblocks=_sample_blocks(w.nb, 3, n=2))
+
+
+@pytest.mark.parametrize("name", ["sweep-keep5-r16", "sweep-keep100-r128", "sweep-keep50-r64"])
+def test_sweep_points(name):
+    w = W.by_name(name)
+    heads = [(0, 3)]
+    _case(w, heads=heads, qblocks=[0, w.nb - 1])
