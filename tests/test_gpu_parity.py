@@ -72,14 +72,18 @@ def test_edge_shapes(grid, D, R, block, keep, B, heads):
 
 
 def test_shift_invariance_on_gpu():
-    """Shifting all positions leaves masks and outputs unchanged (within fp rounding)."""
+    """Shifting all positions leaves the masks unchanged exactly (fp64 selection) and the outputs
+    unchanged up to the fp16 rounding of the rotated operands, which differs between the two runs:
+    both stay within the parity tolerance of the (exactly invariant) oracle."""
     w = W.TINY.with_(T=4, H=16, W=16, heads=2, block=64, keep_frac=0.25)
     x = I.make_inputs(w)
     p0 = slra.Problem.from_workload(w)
     p1 = slra.Problem.from_workload(w, pos_offset=(3, -7, 11))
     g0, g1 = parity.run_gpu(p0, x), parity.run_gpu(p1, x)
     assert np.array_equal(g0["idx"], g1["idx"])
-    assert np.abs(g0["out"] - g1["out"]).max() < 1e-3
+    d = np.abs(g0["out"] - g1["out"])
+    assert d.max() <= parity.MAX_ABS and d.sum() / np.abs(g0["out"]).sum() <= parity.MEAN_REL
+    parity.compare(p1, x, g1, label="tiny-shifted")
 
 
 def test_deterministic_and_bf16_out():
