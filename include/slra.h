@@ -69,7 +69,8 @@ typedef enum slra_status {
     SLRA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or a kernel launch failed                */
     SLRA_ERR_DEVICE_TIMEOUT = 6,  /* (device status) a bounded wait inside a kernel ran out              */
     SLRA_ERR_RANGE = 7,           /* (device status) |value| >= 65504 after RoPE: does not fit fp16      */
-    SLRA_ERR_NO_DEVICE = 8        /* no sm_100 device is current                                         */
+    SLRA_ERR_NO_DEVICE = 8,       /* no sm_100 device is current                                         */
+    SLRA_ERR_SCRATCH_LIMIT = 9    /* slra_lowrank_summary_noalloc: problem exceeds its fixed scratch area */
 } slra_status;
 
 typedef enum slra_out_dtype { SLRA_OUT_F32 = 0, SLRA_OUT_BF16 = 1 } slra_out_dtype;
@@ -190,6 +191,37 @@ SLRA_API slra_status slra_lowrank_summary(const slra_problem* p, const void* k, 
  * range problem).
  */
 SLRA_API slra_status slra_device_status(void* workspace, slra_stream_t stream, int32_t* status);
+
+/*
+ * Low-rank summary without any allocation: S = sum_j psi(k_j) v_j^T and z = sum_j phi(k_j), the same
+ * result as slra_lowrank_summary (up to the order of the fp32 partial sums), written straight into
+ * caller buffers and using no workspace.  The method's sources have no counterpart to this entry
+ * point; it exists for callers that cannot allocate device memory at the point of the call: code
+ * running inside a framework that hands out device memory only through its own pool and forbids side
+ * allocations, plugin-style execute hooks that must not allocate, and latency-critical serving loops
+ * where cudaMalloc/cudaFree would synchronize the device and stall other streams.
+ *
+ *   k, v     bf16 [B][L][Hh][D] contiguous, 16-B aligned (device).
+ *   A        bf16 [D][rank] contiguous, 16-B aligned (device).
+ *   S        fp32 [B*Hh][rank][D] output (device, 16-B aligned).
+ *   z        fp32 [B*Hh][rank]    output (device, 16-B aligned).
+ *
+ * Scratch (the rotary tables and the split-L partial sums) lives in one fixed array of
+ * SLRA_NOALLOC_SCRATCH_BYTES (16 MiB) compiled into the library: every GPU that loads the library
+ * holds that array until the process exits.  The number of sequence splits is reduced until the
+ * partial sums fit; a problem whose partial sums do not fit even unsplit
+ * (B*Hh*rank*(D+1)*4 bytes plus the tables over the limit) is rejected with SLRA_ERR_SCRATCH_LIMIT
+ * before anything is launched.  The call performs no cudaMalloc, cudaFree or other allocation.
+ *
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current) and caches it; make that first call before any stream capture.  All calls
+ * share the one array: every scratch byte a call reads it has first written itself, so nothing left
+ * by an earlier call is used, but calls that overlap on the GPU (on different streams, or from
+ * different host threads without ordering) race on the array and must be serialized by the caller.
+ */
+#define SLRA_NOALLOC_SCRATCH_BYTES (16u << 20)
+SLRA_API slra_status slra_lowrank_summary_noalloc(const slra_problem* p, const void* k, const void* v,
+                                                  const void* A, float* S, float* z, slra_stream_t stream);
 
 #ifdef __cplusplus
 }

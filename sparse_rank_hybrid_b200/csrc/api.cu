@@ -267,6 +267,7 @@ const char* slra_status_string(int s) {
         case SLRA_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel ran out";
         case SLRA_ERR_RANGE: return "input value out of fp16 range after RoPE";
         case SLRA_ERR_NO_DEVICE: return "no sm_100 device is current";
+        case SLRA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the fixed no-allocation area holds";
         default: return "unknown status";
     }
 }
@@ -441,3 +442,72 @@ slra_status slra_device_status(void* workspace, slra_stream_t stream, int32_t* s
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free low-rank summary.  Its scratch (rotary tables + split-L partial sums) is this
+// file-scope device array; host code must not pass the array's name to a kernel (on the host it is
+// only a stand-in), so its device address is looked up once per device and cached.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SLRA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up on first use).
+slra_status scratch_address(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return SLRA_ERR_NO_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return SLRA_ERR_CUDA;
+        }
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return SLRA_OK;
+}
+
+}  // namespace
+
+extern "C" slra_status slra_lowrank_summary_noalloc(const slra_problem* p, const void* k, const void* v,
+                                                    const void* A, float* S, float* z, slra_stream_t stream) {
+    Derived d;
+    slra_status s = derive(p, &d);
+    if (s != SLRA_OK) return s;
+    if (!k || !v || !A || !S || !z) return SLRA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(A) || !aligned16(S) || !aligned16(z)) return SLRA_ERR_ALIGNMENT;
+    const Geom& g = d.g;
+    // scratch: [cos/sin table | pair info] [partial S] [partial z], each 256-B aligned
+    const size_t tab_bytes = align_up(sizeof(double2) * static_cast<size_t>(d.table_entries) + sizeof(int2) * kMaxPairs, 256);
+    const size_t per_split = static_cast<size_t>(g.BH()) * g.R * (g.D + 1) * sizeof(float) + 512;
+    if (tab_bytes + per_split > SLRA_NOALLOC_SCRATCH_BYTES) return SLRA_ERR_SCRATCH_LIMIT;
+    int nsplit = d.nsplit;
+    const size_t fit = (SLRA_NOALLOC_SCRATCH_BYTES - tab_bytes) / per_split;
+    if (static_cast<size_t>(nsplit) > fit) nsplit = static_cast<int>(fit);
+    if ((s = check_device()) != SLRA_OK) return s;
+    void* scratch = nullptr;
+    if ((s = scratch_address(&scratch)) != SLRA_OK) return s;
+    uint8_t* base = static_cast<uint8_t*>(scratch);
+    double2* tab = reinterpret_cast<double2*>(base);
+    int2* pairs = reinterpret_cast<int2*>(base + sizeof(double2) * d.table_entries);
+    float* s_part = reinterpret_cast<float*>(base + tab_bytes);
+    float* z_part = reinterpret_cast<float*>(
+        base + tab_bytes + align_up(static_cast<size_t>(g.BH()) * nsplit * g.R * g.D * sizeof(float), 256));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // Every kernel below writes all the scratch it later reads (the whole table, every partial slot of
+    // every split), so nothing needs clearing between calls.
+    if (launch_rope_table(tab, pairs, d.meta, d.table_entries, st) != cudaSuccess) return SLRA_ERR_CUDA;
+    if (launch_lowrank_partial(static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                               static_cast<const __nv_bfloat16*>(A), tab, pairs, g, nsplit, s_part, z_part,
+                               st) != cudaSuccess)
+        return SLRA_ERR_CUDA;
+    return cuda_status(launch_lowrank_reduce(s_part, z_part, g, nsplit, S, z, st));
+}

@@ -16,14 +16,14 @@ LIB_PATH = os.path.join(_HERE, "libslra.so")
 
 OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_RANGE, \
-    ERR_NO_DEVICE = range(1, 9)
+    ERR_NO_DEVICE, ERR_SCRATCH_LIMIT = range(1, 10)
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
 
 # Every symbol include/slra.h declares.
 EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_validate", "slra_keep_count",
            "slra_workspace_layout", "slra_attn_fwd", "slra_host_io_bytes", "slra_attn_fwd_host",
-           "slra_select_blocks", "slra_lowrank_summary", "slra_device_status")
+           "slra_select_blocks", "slra_lowrank_summary", "slra_device_status", "slra_lowrank_summary_noalloc")
 
 
 class SlraError(RuntimeError):
@@ -75,8 +75,10 @@ def lib():
         L.slra_select_blocks.argtypes = [PP, P, P, P, P, S, P]
         L.slra_lowrank_summary.argtypes = [PP, P, P, P, P, S, P]
         L.slra_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+        L.slra_lowrank_summary_noalloc.argtypes = [PP, P, P, P, P, P, P]
         for name in ("slra_problem_init", "slra_validate", "slra_workspace_layout", "slra_attn_fwd",
-                     "slra_attn_fwd_host", "slra_select_blocks", "slra_lowrank_summary", "slra_device_status"):
+                     "slra_attn_fwd_host", "slra_select_blocks", "slra_lowrank_summary", "slra_device_status",
+                     "slra_lowrank_summary_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -230,6 +232,14 @@ def lowrank_summary(prob: Problem, k, v, A, workspace=None, stream=None):
     _check(lib().slra_lowrank_summary(ctypes.byref(prob.c()), _ptr(k), _ptr(v), _ptr(A), _ptr(workspace),
                                       workspace.numel(), _stream_handle(stream)), "slra_lowrank_summary")
     return workspace
+
+
+def lowrank_summary_noalloc(prob: Problem, k, v, A, S, z, stream=None):
+    """Low-rank summary into caller tensors S [B*Hh, rank, D] and z [B*Hh, rank] (fp32, CUDA) without
+    any allocation: the library's fixed scratch array is used instead of a workspace."""
+    _check(lib().slra_lowrank_summary_noalloc(ctypes.byref(prob.c()), _ptr(k), _ptr(v), _ptr(A), _ptr(S), _ptr(z),
+                                              _stream_handle(stream)), "slra_lowrank_summary_noalloc")
+    return S, z
 
 
 def device_status(workspace, stream=None) -> int:
