@@ -18,6 +18,7 @@
 // All waits are bounded (see sm100.cuh); a wait that runs out records a timeout in the status word
 // and the CTA leaves the loop, releases its tensor memory and returns.
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "sm100.cuh"
 
 namespace slra {
@@ -47,6 +48,52 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
                    "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
                    "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
                    "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1) as one packed fp32x2 FMA.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// (s0, s1) += (a0, a1) as one packed fp32x2 add.
+__device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+        "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(s0), "+f"(s1)
+        : "f"(a0), "f"(a1));
+}
+
+// fp16x2 with lo in the low half (the lower key index sits in the lower 16 bits of a TMEM column).
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// 2^x without the MUFU unit, for x <= 128: n = floor(x) via a round-down add of 1.5 * 2^23, f = x - n,
+// 2^f from the degree-3 minimax polynomial of exp2_poly.cuh (max relative error 7.5e-5), and 2^n
+// added into the exponent field.  Inputs below -126 (and -inf) are clamped to -126: p(0) is just
+// below 1 (exponent field 126), so n must stay >= -126 for the exponent field to stay >= 0; the result
+// there is < 2^-125, which rounds to zero in the fp16 P operand anyway.
+__device__ __forceinline__ float exp2_soft(float x) {
+    x = fmaxf(x, -126.0f);
+    float t;
+    asm("add.rm.f32 %0, %1, 0f4B400000;" : "=f"(t) : "f"(x));
+    const float f = x - (t - 12582912.0f);
+    const float p = fmaf(fmaf(fmaf(SLRA_EXP2_C3, f, SLRA_EXP2_C2), f, SLRA_EXP2_C1), f, SLRA_EXP2_C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 }  // namespace
@@ -151,8 +198,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+    // The kept list is ascending, so the only block that can be partial (the sequence's last) can only
+    // be the last one visited.
+    const int last_valid = keep > 0 ? min(blk, g.L - __ldg(my_idx + keep - 1) * blk) : blk;
     float m_run = 0.f, l_run = 0.f;
-    int next_beta = 0;
     for (int j = 0; j < keep; ++j) {
         const bool ok = mbar_wait(bar_s, j & 1, tmo, abort_flag);
         if (__syncthreads_or(!ok)) {
@@ -160,15 +209,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             break;
         }
         tc_fence_after();
-        if (tid == 0) ++n_s_done;
-        if (tid == 0 && j + 1 < keep) {  // S_j done reading the k tile: fetch the next one
-            next_beta = my_idx[j + 1];
-            load_kv(bar_k, sk, &tm_k, next_beta);
-            ++n_k_issued;
+        if (tid == 0) {
+            ++n_s_done;
+            // S_j has finished reading the k tile and (issued before it) P.V_{j-1} the v tile.
+            if (j + 1 < keep) { load_kv(bar_k, sk, &tm_k, my_idx[j + 1]); ++n_k_issued; }
+            if (j > 0) { load_kv(bar_v, sv, &tm_v, my_idx[j]); ++n_v_issued; }
         }
-        // ---- softmax on row (warp*32 + lane)
-        const int beta_row = __ldg(my_idx + j);
-        const int valid = min(blk, g.L - beta_row * blk);  // keys of this block that exist
+        // ---- softmax of row (warp*32 + lane); O is stable (P.V_{j-1} completed before S_j)
         uint32_t sr[4][32];
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -177,60 +224,70 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int c = 1; c < 4; ++c)
             if (c * 32 < blk) reg_fence(sr[c]);
+        if (j == keep - 1 && last_valid < blk) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (c * 32 + i >= last_valid) sr[c][i] = __float_as_uint(-INFINITY);
+        }
         float mx = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             if (c * 32 >= blk) continue;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float t = __uint_as_float(sr[c][i]) * scale_log2;
-                if (c * 32 + i >= valid) t = -INFINITY;
-                sr[c][i] = __float_as_uint(t);
-                mx = fmaxf(mx, t);
-            }
+            for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
         }
+        mx *= scale_log2;
         if (j == 0) {
             m_run = mx;
-        } else {
-            const bool need = mx > m_run + 8.0f;
-            if (__any_sync(0xffffffffu, need)) {  // warp-uniform: TMEM access is warp-collective
-                const float m_new = fmaxf(m_run, mx);
-                const float alpha_r = ex2_approx(m_run - m_new);
+        } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {  // warp-uniform: TMEM access is collective
+            const float m_new = fmaxf(m_run, mx);
+            const float alpha_r = ex2_approx(m_run - m_new);
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + lane_base + c * 32, o);
-                    tmem_ld_wait(o);
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + lane_base + c * 32, o);
+                tmem_ld_wait(o);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha_r);
-                    tmem_st32(tO + lane_base + c * 32, o);
-                }
-                tmem_st_wait();
-                l_run *= alpha_r;
-                m_run = m_new;
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha_r);
+                tmem_st32(tO + lane_base + c * 32, o);
             }
+            tmem_st_wait();
+            l_run *= alpha_r;
+            m_run = m_new;
         }
-        float lsum = 0.f;
+        const float neg_m = -m_run;
+        float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {  // 64 keys -> 32 packed fp16x2 columns
+        for (int c2 = 0; c2 < 2; ++c2) {  // 64 keys -> 32 packed fp16x2 TMEM columns
             if (c2 * 64 >= blk) continue;
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const int key = c2 * 64 + 2 * i;
-                const float p0 = ex2_approx(__uint_as_float(sr[key >> 5][key & 31]) - m_run);
-                const float p1 = ex2_approx(__uint_as_float(sr[(key + 1) >> 5][(key + 1) & 31]) - m_run);
-                const __half2 hp = __floats2half2_rn(p0, p1);
-                lsum += __low2float(hp) + __high2float(hp);
-                pk[i] = *reinterpret_cast<const uint32_t*>(&hp);
+                float t0, t1;
+                ffma2(t0, t1, __uint_as_float(sr[key >> 5][key & 31]), __uint_as_float(sr[key >> 5][(key & 31) + 1]),
+                      scale_log2, scale_log2, neg_m, neg_m);
+                float p0, p1;
+                if ((i & 3) == 0) {  // a quarter of the exponentials on the FMA/ALU pipes
+                    p0 = exp2_soft(t0);
+                    p1 = exp2_soft(t1);
+                } else {
+                    p0 = ex2_approx(t0);
+                    p1 = ex2_approx(t1);
+                }
+                fadd2(sum0, sum1, p0, p1);
+                pk[i] = pack_half2(p0, p1);
             }
             tmem_st32(tS + lane_base + c2 * 32, pk);
         }
         tmem_st_wait();
-        l_run += lsum;
+        l_run += sum0 + sum1;
         tc_fence_before();
         __syncthreads();
-        // ---- issue O += P v, then (after it completes) the next S
+        // ---- issue O += P v, then immediately the next S (tensor-core operations issued by one thread
+        //      run in order, so S_{j+1} overwrites the P columns only after P.V_j has read them)
         if (warp == 0) {
             if (lane == 0 && !*abort_flag) {
                 tc_fence_after();
@@ -244,29 +301,29 @@ __global__ void __launch_bounds__(kThreads, 2)
                         const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, static_cast<uint32_t>(blk) * 128, 1024);
                         umma_ts(tO, tS + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit(bar_o);
-                    ++n_o_issued;
-                    if (!mbar_wait(bar_o, j & 1, tmo, abort_flag)) {
-                        fail();
-                    } else {
-                        ++n_o_done;
-                        if (j + 1 < keep) {
-                            load_kv(bar_v, sv, &tm_v, next_beta);
-                            ++n_v_issued;
-                            if (mbar_wait(bar_k, (j + 1) & 1, tmo, abort_flag)) {
-                                ++n_k_done;
-                                tc_fence_after();
-                                issue_s();
-                                ++n_s_issued;
-                            } else {
-                                fail();
-                            }
+                    if (j + 1 < keep) {
+                        if (mbar_wait(bar_k, (j + 1) & 1, tmo, abort_flag)) {
+                            ++n_k_done;
+                            issue_s();  // commits bar_s, which also covers this P.V
+                            ++n_s_issued;
+                        } else {
+                            umma_commit(bar_o);
+                            ++n_o_issued;
+                            fail();
                         }
+                    } else {
+                        umma_commit(bar_o);
+                        ++n_o_issued;
                     }
                 }
             }
             __syncwarp();
         }
+    }
+    if (keep > 0) {  // the last P.V has landed in O
+        const bool ok = !*abort_flag && mbar_wait(bar_o, 0, tmo, abort_flag);
+        if (__syncthreads_or(!ok) && tid == 0) fail();
+        if (tid == 0 && ok) ++n_o_done;
     }
     __syncthreads();
     tc_fence_after();
