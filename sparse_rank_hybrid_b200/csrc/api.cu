@@ -13,8 +13,6 @@ using namespace slra;
 
 namespace {
 
-constexpr int kTargetCtas = 2 * 148;  // low-rank split count aims at two CTAs per B200 SM
-constexpr int kLrTileTokens = 32;
 constexpr int64_t kMaxBlocks = 2048;  // selection keeps a row of scores in shared memory
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -94,9 +92,7 @@ slra_status derive(const slra_problem* p, Derived* d) {
         }
     }
     d->table_entries = off;
-    const int64_t ntiles = (L + kLrTileTokens - 1) / kLrTileTokens;
-    int64_t ns = (kTargetCtas + BH - 1) / BH;
-    ns = ns < 1 ? 1 : (ns > ntiles ? ntiles : ns);
+    const int64_t ns = lowrank_nsplit(g);
     d->nsplit = static_cast<int>(ns);
 
     slra_ws_layout& w = d->lay;
@@ -147,36 +143,6 @@ slra_status check_device() {
         return SLRA_ERR_NO_DEVICE;
     }
     return (major == 10 && minor == 0) ? SLRA_OK : SLRA_ERR_NO_DEVICE;
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-        else
-            cudaGetLastError();
-    });
-    return fn;
-}
-
-// 2D fp16 map over a head-major [rows][D] buffer, box 64 columns x box_rows rows, 128-B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int D, int box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 struct Ptrs {
@@ -231,12 +197,22 @@ slra_status run_select(const Derived& d, const Ptrs& w, const void* q, const voi
     return cuda_status(launch_select(w.qbar, w.kbar, g, w.idx, w.tie, st));
 }
 
+// Low-rank partial sums: tensor-core kernel for head_dim 128, CUDA-core kernel otherwise.
+cudaError_t lowrank_partial(const Derived& d, const void* k, const void* v, const void* A, const double2* tab,
+                            const int2* pairs, int nsplit, float* s_part, float* z_part, int* status,
+                            unsigned long long timeout_ns, cudaStream_t st) {
+    const auto* kb = static_cast<const __nv_bfloat16*>(k);
+    const auto* vb = static_cast<const __nv_bfloat16*>(v);
+    const auto* Ab = static_cast<const __nv_bfloat16*>(A);
+    if (d.g.D == 128)
+        return launch_lowrank_tc(kb, vb, Ab, tab, pairs, d.g, nsplit, s_part, z_part, status, timeout_ns, st);
+    return launch_lowrank_partial(kb, vb, Ab, tab, pairs, d.g, nsplit, s_part, z_part, st);
+}
+
 slra_status run_lowrank(const Derived& d, const Ptrs& w, const void* k, const void* v, const void* A,
-                        cudaStream_t st) {
+                        unsigned long long timeout_ns, cudaStream_t st) {
     const Geom& g = d.g;
-    cudaError_t e = launch_lowrank_partial(static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-                                           static_cast<const __nv_bfloat16*>(A), w.tab, w.pairs, g, d.nsplit,
-                                           w.s_part, w.z_part, st);
+    cudaError_t e = lowrank_partial(d, k, v, A, w.tab, w.pairs, d.nsplit, w.s_part, w.z_part, w.status, timeout_ns, st);
     if (e != cudaSuccess) return SLRA_ERR_CUDA;
     return cuda_status(launch_lowrank_reduce(w.s_part, w.z_part, g, d.nsplit, w.S, w.z, st));
 }
@@ -244,6 +220,10 @@ slra_status run_lowrank(const Derived& d, const Ptrs& w, const void* k, const vo
 slra_status begin(const Derived& d, const Ptrs& w, cudaStream_t st) {
     if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return SLRA_ERR_CUDA;
     return cuda_status(launch_rope_table(w.tab, w.pairs, d.meta, d.table_entries, st));
+}
+
+unsigned long long timeout_of(const slra_problem* p) {
+    return p->wait_timeout_ns ? p->wait_timeout_ns : 2000000000ull;
 }
 
 size_t qkv_bytes(const Derived& d) {
@@ -332,15 +312,15 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
 
     AttnMaps maps;
     const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
-    if (!make_map(&maps.q, w.qh, rows, g.D, 128) || !make_map(&maps.k, w.kh, rows, g.D, g.block) ||
-        !make_map(&maps.v, w.vh, rows, g.D, g.block))
+    if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) || !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
+        !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block))
         return SLRA_ERR_CUDA;
 
     if ((s = begin(d, w, st)) != SLRA_OK) return s;
     if (branches & SLRA_BRANCH_SPARSE)
         if ((s = run_select(d, w, q, k, v, st)) != SLRA_OK) return s;
     if (branches & SLRA_BRANCH_LOWRANK)
-        if ((s = run_lowrank(d, w, k, v, A, st)) != SLRA_OK) return s;
+        if ((s = run_lowrank(d, w, k, v, A, timeout_of(p), st)) != SLRA_OK) return s;
 
     AttnArgs a;
     a.idx = w.idx;
@@ -427,7 +407,7 @@ slra_status slra_lowrank_summary(const slra_problem* p, const void* k, const voi
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const Ptrs w = carve(workspace, d);
     if ((s = begin(d, w, st)) != SLRA_OK) return s;
-    return run_lowrank(d, w, k, v, A, st);
+    return run_lowrank(d, w, k, v, A, timeout_of(p), st);
 }
 
 slra_status slra_device_status(void* workspace, slra_stream_t stream, int32_t* status) {
@@ -475,6 +455,13 @@ slra_status scratch_address(void** out) {
     return SLRA_OK;
 }
 
+// A status word for the kernels' bounded waits, placed after the partial sums inside the scratch.
+int* noalloc_status(uint8_t* base, size_t tab_bytes, const Geom& g, int nsplit) {
+    const size_t s_bytes = align_up(static_cast<size_t>(g.BH()) * nsplit * g.R * g.D * sizeof(float), 256);
+    const size_t z_bytes = align_up(static_cast<size_t>(g.BH()) * nsplit * g.R * sizeof(float), 256);
+    return reinterpret_cast<int*>(base + tab_bytes + s_bytes + z_bytes);
+}
+
 }  // namespace
 
 extern "C" slra_status slra_lowrank_summary_noalloc(const slra_problem* p, const void* k, const void* v,
@@ -505,9 +492,9 @@ extern "C" slra_status slra_lowrank_summary_noalloc(const slra_problem* p, const
     // Every kernel below writes all the scratch it later reads (the whole table, every partial slot of
     // every split), so nothing needs clearing between calls.
     if (launch_rope_table(tab, pairs, d.meta, d.table_entries, st) != cudaSuccess) return SLRA_ERR_CUDA;
-    if (launch_lowrank_partial(static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-                               static_cast<const __nv_bfloat16*>(A), tab, pairs, g, nsplit, s_part, z_part,
-                               st) != cudaSuccess)
+    // the device status word of this entry point is the scratch's first word after the partial sums
+    if (lowrank_partial(d, k, v, A, tab, pairs, nsplit, s_part, z_part, noalloc_status(base, tab_bytes, g, nsplit),
+                        timeout_of(p), st) != cudaSuccess)
         return SLRA_ERR_CUDA;
     return cuda_status(launch_lowrank_reduce(s_part, z_part, g, nsplit, S, z, st));
 }

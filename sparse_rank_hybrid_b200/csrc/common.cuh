@@ -18,7 +18,7 @@ constexpr int kDevRange = 2;
 // Sizes of one call.  L = T*H*W; Lp = nb*block (rows of the padded head-major buffers).
 struct Geom {
     int B, Hh, D, T, H, W, L, block, nb, keep, R, Lp;
-    int BH() const { return B * Hh; }
+    __host__ __device__ int BH() const { return B * Hh; }
 };
 
 // 3D RoPE schedule: pair j rotates with the position along axis[j]; its cos/sin for position p
@@ -48,6 +48,13 @@ cudaError_t launch_select(const double* qbar, const double* kbar, const Geom& g,
 cudaError_t launch_lowrank_partial(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,
                                    const double2* tab, const int2* pairs, const Geom& g, int nsplit,
                                    float* s_part, float* z_part, cudaStream_t st);
+// Tensor-core low-rank partial sums (head_dim 128), see lowrank_sm100.cu.
+cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,
+                              const double2* tab, const int2* pairs, const Geom& g, int nsplit, float* s_part,
+                              float* z_part, int* status, unsigned long long timeout_ns, cudaStream_t st);
+int lowrank_nsplit(const Geom& g);
+bool make_map_headmajor(CUtensorMap* m, const void* base, uint64_t rows, int D, int box_rows);
+bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int D, int box_tokens);
 cudaError_t launch_lowrank_reduce(const float* s_part, const float* z_part, const Geom& g, int nsplit, float* S,
                                   float* z, cudaStream_t st);
 

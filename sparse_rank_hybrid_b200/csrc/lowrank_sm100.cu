@@ -1,0 +1,401 @@
+// Low-rank summary on the sm_100a tensor cores (head_dim 128): per head, over all L keys,
+//   S = sum_j psi(k_j) v_j^T,   z = sum_j phi(k_j),   phi(k) = relu(k A),   psi = phi with its first
+// r coordinates rotated by the token's 3D RoPE angles (RoLA "4.1", "4.2", "4.3", "B.1").
+//
+// Persistent CTAs (one per SM, 128 threads) walk work items = (head, range of 128-token tiles).  Per
+// tile:
+//   TMA    raw k and v tiles [128 tokens][128] bf16 straight from the [B][L][Hh][D] inputs (4D tensor
+//          maps, 128-B swizzle, two stages so the next tiles stream in while this one is processed);
+//   MMA    phi = k A  (M = 128 tokens, N = r, K = 128; A^T staged once per CTA as the B operand);
+//   threads (thread = token = TMEM lane) relu, accumulate z in registers, rotate the first r
+//          coordinates and write psi as bf16 hi + lo halves (psi = hi + lo to ~2^-16) into shared
+//          memory, token-major;
+//   MMA    S^T += v^T [psi_hi | psi_lo]  (M = 128 = D, N = 2*Rp, K = 128 tokens), accumulated in TMEM
+//          over the whole work item; v is exact in bf16, so S is exact to the fp32 accumulation.
+// At the end of an item its S and z partial sums go to the split-L partial buffers, which a
+// fixed-order reduction sums per head.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace slra {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kTok = 128;                      // tokens per tile
+constexpr int kTileBytes = kTok * kD * 2;      // 32 KB (two 64-column slabs of 16 KB)
+constexpr int kStages = 2;
+
+struct LrLayout {
+    int rp;           // padded psi width per half (64 or 128)
+    int off_k[kStages], off_v[kStages];
+    int off_at;       // A^T [r][128] bf16, K-major swizzled
+    int off_psi;      // [128 tokens][2*rp] bf16, 64-column slabs
+    int off_zred;     // [4 warps][R/2] fp32 (z is reduced in two halves)
+    int off_bar;
+    int off_misc;
+    int bytes;
+};
+
+__host__ __device__ inline LrLayout lr_layout(int R) {
+    LrLayout l;
+    l.rp = R <= 64 ? 64 : 128;
+    int o = 0;
+    for (int s = 0; s < kStages; ++s) { l.off_k[s] = o; o += kTileBytes; l.off_v[s] = o; o += kTileBytes; }
+    l.off_at = o;
+    o += ((R * 256 + 1023) / 1024) * 1024;
+    l.off_psi = o;
+    o += kTok * 2 * l.rp * 2;
+    l.off_zred = o;
+    o += 4 * (R / 2) * 4;
+    l.off_bar = o;
+    o += 128;
+    l.off_misc = o;
+    o += 64;
+    l.bytes = o;
+    return l;
+}
+
+// bf16 bits of x rounded to nearest even.
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<const uint16_t*>(&h);
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+        "[%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+// Byte offset of element (row, col) in a tile of 64-column slabs of [rows][128 B] with the 128-B swizzle
+// (16-byte chunk index XOR row % 8): the layout TMA writes and the tensor-core descriptors read.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows_per_slab) {
+    const int slab = col >> 6, c = col & 63;
+    return static_cast<uint32_t>(slab * rows_per_slab * 128 + row * 128 + ((((c >> 3) ^ (row & 7)) << 4) | ((c & 7) << 1)));
+}
+
+}  // namespace
+
+struct LrArgs {
+    const __nv_bfloat16* A;
+    const double2* tab;
+    const int2* pairs;
+    float* s_part;   // [BH][nsplit][R][D]
+    float* z_part;   // [BH][nsplit][R]
+    int nsplit;
+    int tiles_per_split;
+    int* status;
+    unsigned long long timeout_ns;
+};
+
+template <int R>
+__global__ void __launch_bounds__(128, 1)
+    lowrank_sm100_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                         LrArgs a, Geom g) {
+    const LrLayout lay = lr_layout(R);
+    constexpr int RP = R <= 64 ? 64 : 128;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.off_bar);
+    uint64_t* bar_kv = bars;         // [kStages]: k and v tile of a stage landed
+    uint64_t* bar_phi = bars + 2;    // phi MMA done
+    uint64_t* bar_s = bars + 3;      // S MMA done (covers every earlier MMA)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + lay.off_misc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + lay.off_misc + 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t tmo = a.timeout_ns;
+
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    // A^T as the K-major B operand of phi = k A: row n = feature, 128 dims in two swizzled slabs.
+    for (int e = tid; e < R * kD; e += 128) {
+        const int d = e / R, c = e % R;  // coalesced read of A [D][R]
+        *reinterpret_cast<uint16_t*>(smem + lay.off_at + sw128_offset(c, d, R)) =
+            *reinterpret_cast<const uint16_t*>(a.A + e);
+    }
+    // zero the padding columns of both psi halves once; tiles only ever write the first R of each half
+    for (int e = tid; e < kTok * 2 * RP; e += 128) {
+        const int t = e / (2 * RP), col = e % (2 * RP);
+        if ((col % RP) >= R) *reinterpret_cast<uint16_t*>(smem + lay.off_psi + sw128_offset(t, col, kTok)) = 0;
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_phi = tmem;          // R columns
+    const uint32_t t_s = tmem + 128;      // 2*RP columns: S^T hi | lo
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t idesc_phi = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(R) >> 3) << 17) | ((128u >> 4) << 24);
+    const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                             ((uint32_t(2 * RP) >> 3) << 17) | ((128u >> 4) << 24);
+    const uint32_t at_addr = smem_addr(smem + lay.off_at), psi_addr = smem_addr(smem + lay.off_psi);
+
+    const int ntiles = (g.L + kTok - 1) / kTok;
+    const int n_items = g.BH() * a.nsplit;
+    // The sequence of (item, tile) this CTA processes, flattened, so loads can run two tiles ahead.
+    auto tile_of = [&](int q, int& item, int& tile) -> bool {  // q-th tile of this CTA
+        int it = blockIdx.x;
+        while (it < n_items) {
+            const int split = it % a.nsplit;
+            const int t0 = split * a.tiles_per_split, t1 = min(ntiles, t0 + a.tiles_per_split);
+            const int cnt = max(0, t1 - t0);
+            if (q < cnt) { item = it; tile = t0 + q; return true; }
+            q -= cnt;
+            it += gridDim.x;
+        }
+        return false;
+    };
+    // thread 0's bookkeeping of issued / observed operations (for the bounded drain on abort)
+    int n_load[kStages] = {0, 0}, n_wait[kStages] = {0, 0};
+    int n_s_issued = 0, n_s_done = 0, n_phi_issued = 0;
+    auto issue_load = [&](int q) {
+        int item, tile;
+        if (!tile_of(q, item, tile)) return;
+        const int s = q % kStages;
+        const int bh = item / a.nsplit, b = bh / g.Hh, h = bh % g.Hh;
+        mbar_expect_tx(bar_kv + s, 2 * kTileBytes);
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(smem + lay.off_k[s] + x * (kTileBytes / 2), &tm_k, bar_kv + s, x * 64, h, tile * kTok, b);
+            tma_load_4d(smem + lay.off_v[s] + x * (kTileBytes / 2), &tm_v, bar_kv + s, x * 64, h, tile * kTok, b);
+        }
+        ++n_load[s];
+    };
+    auto fail = [&]() {
+        *abort_flag = 1;
+        atomicOr(a.status, kDevTimeout);
+    };
+    if (tid == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        issue_load(0);
+        issue_load(1);
+    }
+
+    int q = 0;      // running tile count of this CTA (same in every thread)
+    int n_phi = 0;  // phi MMAs completed (same in every thread)
+    int n_s = 0;    // S MMAs issued (same in every thread)
+    bool aborted = false;
+    for (int item = blockIdx.x; item < n_items && !aborted; item += gridDim.x) {
+        const int bh = item / a.nsplit, split = item % a.nsplit;
+        const int t0 = split * a.tiles_per_split, t1 = min(ntiles, t0 + a.tiles_per_split);
+        if (t1 <= t0) {  // empty split (never produced by the host plan): contributes zeros
+            float* sp0 = a.s_part + (static_cast<size_t>(bh) * a.nsplit + split) * R * kD;
+            for (int c = 0; c < R; ++c) sp0[c * kD + tid] = 0.f;
+            if (tid < R) a.z_part[(static_cast<size_t>(bh) * a.nsplit + split) * R + tid] = 0.f;
+            continue;
+        }
+        float zacc[R];
+#pragma unroll
+        for (int c = 0; c < R; ++c) zacc[c] = 0.f;
+        for (int tile = t0; tile < t1; ++tile, ++q) {
+            const int s = q % kStages;
+            // ---- phi = k A
+            if (tid == 0) {
+                if (!mbar_wait(bar_kv + s, n_wait[s] & 1, tmo, abort_flag)) {
+                    fail();
+                } else {
+                    ++n_wait[s];
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {
+                        const uint64_t ad = sdesc_sw128(smem_addr(smem + lay.off_k[s]) + (kk >> 2) * (kTok * 128) + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(at_addr + (kk >> 2) * (R * 128) + (kk & 3) * 32, 16, 1024);
+                        umma_ss(t_phi, ad, bd, idesc_phi, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar_phi);
+                    ++n_phi_issued;
+                }
+            }
+            // (the previous tile's S MMA already completed: thread 0 waited for it before reloading)
+            const bool ok = mbar_wait(bar_phi, n_phi & 1, tmo, abort_flag);
+            if (__syncthreads_or(!ok)) {
+                if (tid == 0) fail();
+                aborted = true;
+                break;
+            }
+            ++n_phi;
+            tc_fence_after();
+            // ---- relu, z, rotation, psi hi/lo into shared memory (thread = token row)
+            const int n = tile * kTok + tid;
+            const bool real = n < g.L;
+            uint32_t raw[R];
+#pragma unroll
+            for (int c0 = 0; c0 < R; c0 += 32) {
+                uint32_t r32[32];  // for R % 32 == 16 the last window also reads 16 unused columns
+                tmem_ld32(t_phi + lane_base + c0, r32);
+                tmem_ld_wait(r32);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (c0 + i < R) raw[c0 + i] = r32[i];
+            }
+#pragma unroll
+            for (int p = 0; p < R / 2; ++p) {
+                float x0 = real ? fmaxf(__uint_as_float(raw[2 * p]), 0.f) : 0.f;
+                float x1 = real ? fmaxf(__uint_as_float(raw[2 * p + 1]), 0.f) : 0.f;
+                zacc[2 * p] += x0;
+                zacc[2 * p + 1] += x1;
+                float cf = 1.f, sf = 0.f;
+                if (real) {
+                    const int2 pi = __ldg(a.pairs + p);
+                    const double2 cs = __ldg(a.tab + pi.y + token_axis_pos(n, pi.x, g.H, g.W));
+                    cf = static_cast<float>(cs.x);
+                    sf = static_cast<float>(cs.y);
+                }
+                const float y0 = x0 * cf - x1 * sf, y1 = x0 * sf + x1 * cf;
+                const uint16_t h0 = bf16_bits(y0), h1 = bf16_bits(y1);
+                const float r0 = y0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
+                const float r1 = y1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
+                const uint32_t hi = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+                const uint32_t lo = static_cast<uint32_t>(bf16_bits(r0)) | (static_cast<uint32_t>(bf16_bits(r1)) << 16);
+                *reinterpret_cast<uint32_t*>(smem + lay.off_psi + sw128_offset(tid, 2 * p, kTok)) = hi;
+                *reinterpret_cast<uint32_t*>(smem + lay.off_psi + sw128_offset(tid, RP + 2 * p, kTok)) = lo;
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            // ---- S^T += v^T [psi_hi | psi_lo]; once it has completed, stage s takes the tile two ahead
+            if (tid == 0 && !*abort_flag) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTok / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(smem_addr(smem + lay.off_v[s]) + kk * 2048, kTileBytes / 2, 1024);
+                    const uint64_t bd = sdesc_sw128(psi_addr + kk * 2048, kTok * 128, 1024);
+                    umma_ss(t_s, ad, bd, idesc_s, (tile > t0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bar_s);
+                ++n_s_issued;
+                if (mbar_wait(bar_s, n_s_done & 1, tmo, abort_flag)) {
+                    ++n_s_done;
+                    issue_load(q + kStages);
+                } else {
+                    fail();
+                }
+            }
+            ++n_s;
+        }
+        if (aborted) break;
+        // ---- item done: S^T (lane = e, columns = c for hi and lo) and z to the partial buffers
+        const bool ok = mbar_wait(bar_s, (n_s - 1) & 1, tmo, abort_flag);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) fail();
+            aborted = true;
+            break;
+        }
+        tc_fence_after();
+        float* sp = a.s_part + (static_cast<size_t>(bh) * a.nsplit + split) * R * kD;
+#pragma unroll
+        for (int c0 = 0; c0 < R; c0 += 16) {
+            uint32_t hi[32], lo[32];
+            tmem_ld32(t_s + lane_base + c0, hi);
+            tmem_ld_wait(hi);
+            tmem_ld32(t_s + lane_base + RP + c0, lo);
+            tmem_ld_wait(lo);
+            const int cn = min(16, R - c0);
+            for (int i = 0; i < cn; ++i) sp[(c0 + i) * kD + tid] = __uint_as_float(hi[i]) + __uint_as_float(lo[i]);
+        }
+        // z: sum the per-thread partials over the 128 threads (warp shuffles, then the 4 warp sums)
+#pragma unroll
+        for (int c = 0; c < R; ++c) {
+            float v = zacc[c];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            zacc[c] = v;  // every lane of the warp holds the warp's sum
+        }
+        float* zslots = reinterpret_cast<float*>(smem + lay.off_zred);  // [4][R/2]
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            if (lane == 0) {
+#pragma unroll
+                for (int c = 0; c < R / 2; ++c) zslots[warp * (R / 2) + c] = zacc[half * (R / 2) + c];
+            }
+            __syncthreads();
+            if (tid < R / 2)
+                a.z_part[(static_cast<size_t>(bh) * a.nsplit + split) * R + half * (R / 2) + tid] =
+                    ((zslots[tid] + zslots[R / 2 + tid]) + zslots[R + tid]) + zslots[3 * (R / 2) + tid];
+            __syncthreads();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    if (aborted && tid == 0) {
+        // let loads still in flight land before the shared memory is released (bounded, 10 ms each)
+        volatile int no_abort = 0;
+        for (int st = 0; st < kStages; ++st)
+            if (n_load[st] > n_wait[st]) mbar_wait(bar_kv + st, n_wait[st] & 1, 10000000ull, &no_abort);
+        if (n_phi_issued > n_phi) mbar_wait(bar_phi, n_phi & 1, 10000000ull, &no_abort);
+        if (n_s_issued > n_s_done) mbar_wait(bar_s, n_s_done & 1, 10000000ull, &no_abort);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace slra
+
+namespace slra {
+
+int lowrank_tc_tiles_per_split(const Geom& g, int nsplit) {
+    const int ntiles = (g.L + kTok - 1) / kTok;
+    return (ntiles + nsplit - 1) / nsplit;
+}
+
+template <int R>
+static cudaError_t lr_tc_launch(const CUtensorMap& tk, const CUtensorMap& tv, const LrArgs& a, const Geom& g,
+                                cudaStream_t st) {
+    const size_t sm = static_cast<size_t>(lr_layout(R).bytes) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(lowrank_sm100_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int items = g.BH() * a.nsplit;
+    lowrank_sm100_kernel<R><<<items < sms ? items : sms, 128, sm, st>>>(tk, tv, a, g);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,
+                              const double2* tab, const int2* pairs, const Geom& g, int nsplit, float* s_part,
+                              float* z_part, int* status, unsigned long long timeout_ns, cudaStream_t st) {
+    CUtensorMap tk, tv;
+    if (!make_map_tokens(&tk, k, g.B, g.L, g.Hh, g.D, kTok) || !make_map_tokens(&tv, v, g.B, g.L, g.Hh, g.D, kTok))
+        return cudaErrorInvalidValue;
+    LrArgs a;
+    a.A = A;
+    a.tab = tab;
+    a.pairs = pairs;
+    a.s_part = s_part;
+    a.z_part = z_part;
+    a.nsplit = nsplit;
+    a.tiles_per_split = lowrank_tc_tiles_per_split(g, nsplit);
+    a.status = status;
+    a.timeout_ns = timeout_ns;
+    switch (g.R) {
+        case 16: return lr_tc_launch<16>(tk, tv, a, g, st);
+        case 32: return lr_tc_launch<32>(tk, tv, a, g, st);
+        case 48: return lr_tc_launch<48>(tk, tv, a, g, st);
+        case 64: return lr_tc_launch<64>(tk, tv, a, g, st);
+        case 80: return lr_tc_launch<80>(tk, tv, a, g, st);
+        case 96: return lr_tc_launch<96>(tk, tv, a, g, st);
+        case 112: return lr_tc_launch<112>(tk, tv, a, g, st);
+        case 128: return lr_tc_launch<128>(tk, tv, a, g, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace slra
