@@ -231,13 +231,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int i = 0; i < 32; ++i)
                     if (c * 32 + i >= last_valid) sr[c][i] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        // row max: four independent chains of 3-input max (short dependency chains)
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             if (c * 32 >= blk) continue;
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+            for (int i = 0; i < 32; i += 8) {
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    mx4[t] = fmax3(mx4[t], __uint_as_float(sr[c][i + 2 * t]), __uint_as_float(sr[c][i + 2 * t + 1]));
+            }
         }
+        float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
         mx *= scale_log2;
         if (j == 0) {
             m_run = mx;
@@ -258,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             m_run = m_new;
         }
         const float neg_m = -m_run;
-        float sum0 = 0.f, sum1 = 0.f;
+        float sums[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};  // independent accumulators
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {  // 64 keys -> 32 packed fp16x2 TMEM columns
             if (c2 * 64 >= blk) continue;
@@ -277,13 +283,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                     p0 = ex2_approx(t0);
                     p1 = ex2_approx(t1);
                 }
-                fadd2(sum0, sum1, p0, p1);
+                fadd2(sums[i & 3][0], sums[i & 3][1], p0, p1);
                 pk[i] = pack_half2(p0, p1);
             }
             tmem_st32(tS + lane_base + c2 * 32, pk);
         }
         tmem_st_wait();
-        l_run += sum0 + sum1;
+        l_run += ((sums[0][0] + sums[0][1]) + (sums[1][0] + sums[1][1])) +
+                 ((sums[2][0] + sums[2][1]) + (sums[3][0] + sums[3][1]));
         tc_fence_before();
         __syncthreads();
         // ---- issue O += P v, then immediately the next S (tensor-core operations issued by one thread
