@@ -36,6 +36,7 @@ struct Derived {
     int table_entries;
     int nsplit;
     slra_ws_layout lay;
+    size_t at_img, sb_img;  // operand images of the tensor-core readout (offsets; head_dim 128 only)
 };
 
 slra_status derive(const slra_problem* p, Derived* d) {
@@ -121,6 +122,12 @@ slra_status derive(const slra_problem* p, Derived* d) {
     w.z_part = take(static_cast<size_t>(BH) * ns * p->rank * 4);
     w.S = take(static_cast<size_t>(BH) * p->rank * p->head_dim * 4);
     w.z = take(static_cast<size_t>(BH) * p->rank * 4);
+    if (p->head_dim == 128) {
+        d->at_img = take(static_cast<size_t>(p->rank) * 256);
+        d->sb_img = take(static_cast<size_t>(BH) * ((p->rank + 63) / 64) * kSbChunkBytes);
+    } else {
+        d->at_img = d->sb_img = 0;
+    }
     w.total_bytes = o;
     return SLRA_OK;
 }
@@ -155,6 +162,7 @@ struct Ptrs {
     int32_t* idx;
     uint8_t* tie;
     float *s_part, *z_part, *S, *z;
+    uint8_t *at_img, *sb_img;  // nullptr unless head_dim 128
 };
 
 Ptrs carve(void* ws, const Derived& d) {
@@ -176,6 +184,8 @@ Ptrs carve(void* ws, const Derived& d) {
     p.z_part = reinterpret_cast<float*>(b + w.z_part);
     p.S = reinterpret_cast<float*>(b + w.S);
     p.z = reinterpret_cast<float*>(b + w.z);
+    p.at_img = d.at_img ? b + d.at_img : nullptr;
+    p.sb_img = d.sb_img ? b + d.sb_img : nullptr;
     return p;
 }
 
@@ -214,7 +224,8 @@ slra_status run_lowrank(const Derived& d, const Ptrs& w, const void* k, const vo
     const Geom& g = d.g;
     cudaError_t e = lowrank_partial(d, k, v, A, w.tab, w.pairs, d.nsplit, w.s_part, w.z_part, w.status, timeout_ns, st);
     if (e != cudaSuccess) return SLRA_ERR_CUDA;
-    return cuda_status(launch_lowrank_reduce(w.s_part, w.z_part, g, d.nsplit, w.S, w.z, st));
+    return cuda_status(launch_lowrank_reduce(w.s_part, w.z_part, g, d.nsplit, w.S, w.z,
+                                             static_cast<const __nv_bfloat16*>(A), w.at_img, w.sb_img, st));
 }
 
 slra_status begin(const Derived& d, const Ptrs& w, cudaStream_t st) {
@@ -313,7 +324,8 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
     AttnMaps maps;
     const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
     if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) || !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
-        !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block))
+        !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
+        !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, 128))
         return SLRA_ERR_CUDA;
 
     if ((s = begin(d, w, st)) != SLRA_OK) return s;
@@ -331,6 +343,8 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
     a.z = w.z;
     a.tab = w.tab;
     a.pairs = w.pairs;
+    a.at_img = w.at_img;
+    a.sb_img = w.sb_img;
     a.lowrank = (branches & SLRA_BRANCH_LOWRANK) ? 1 : 0;
     a.out = out;
     a.out_bf16 = p->out_dtype == SLRA_OUT_BF16 ? 1 : 0;
@@ -496,5 +510,5 @@ extern "C" slra_status slra_lowrank_summary_noalloc(const slra_problem* p, const
     if (lowrank_partial(d, k, v, A, tab, pairs, nsplit, s_part, z_part, noalloc_status(base, tab_bytes, g, nsplit),
                         timeout_of(p), st) != cudaSuccess)
         return SLRA_ERR_CUDA;
-    return cuda_status(launch_lowrank_reduce(s_part, z_part, g, nsplit, S, z, st));
+    return cuda_status(launch_lowrank_reduce(s_part, z_part, g, nsplit, S, z, nullptr, nullptr, nullptr, st));
 }

@@ -13,7 +13,8 @@
 //         by more than 2^8), P = 2^(s*log2e/sqrt(D) - m) rounded to fp16 and written back into the
 //         TMEM columns of S;
 //   MMA   O += P v        (A operand = P from TMEM, B = v tile MN-major; M=128, N=D, K=block).
-// Epilogue: O / l plus the low-rank readout (CUDA cores, fp32), stored as fp32 or bf16.
+// Epilogue: the low-rank readout (head_dim 128: on the tensor cores, accumulated into O; head_dim 64: on
+// the CUDA cores in fp32), then O / l stored as fp32 or bf16.
 //
 // All waits are bounded (see sm100.cuh); a wait that runs out records a timeout in the status word
 // and the CTA leaves the loop, releases its tensor memory and returns.
@@ -36,7 +37,7 @@ struct AttnLayout {
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kKVBytes;
-    static constexpr int kOffBar = kOffV + kKVBytes;  // 5 mbarriers
+    static constexpr int kOffBar = kOffV + kKVBytes;  // 7 mbarriers
     static constexpr int kOffMisc = kOffBar + 64;     // tmem base, abort flag
     static constexpr int kBytes = kOffMisc + 64;
 };
@@ -101,7 +102,8 @@ __device__ __forceinline__ float exp2_soft(float x) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, AttnArgs a, Geom g) {
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qraw,
+                      AttnArgs a, Geom g) {
     using Lay = AttnLayout<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int32_t* my_idx = a.idx + (static_cast<size_t>(bh) * g.nb + alpha) * (keep > 0 ? g.keep : 0);
 
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -340,73 +342,225 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int i_row = warp * 32 + lane;
     const int n = alpha * blk + i_row;
     const bool row_valid = (i_row < blk) && (n < g.L) && !aborted;
-    float acc[D];
+    float inv_l = (keep > 0 && l_run > 0.f) ? 1.f / l_run : 0.f;
+    bool o_live = keep > 0;  // O holds the sparse branch (and, below, the low-rank readout)
+    int n_eld_issued = 0, n_eld = 0, n_emm_issued = 0, n_emm = 0;  // epilogue barrier bookkeeping
+    uint64_t* bar_eld = bars + 5;  // epilogue loads
+    uint64_t* bar_emm = bars + 6;  // epilogue products
+    if constexpr (D == 128) {
+        if (a.lowrank && !aborted) {
+            // Low-rank readout on the tensor cores, accumulated straight into O (so out = O / l):
+            //   phi = q A        raw bf16 query tile (TMA) x A^T image, into the free S columns;
+            //   psi = R_r(p) relu(phi) * l / (relu(phi) . z + 1e-6), split into bf16 hi + lo;
+            //   O  += psi S      as psi_hi S_hi + psi_hi S_lo + psi_lo S_hi, one 64-feature chunk at a time.
+            const int R = g.R;
+            const int nch = (R + 63) / 64;
+            uint8_t* X = smem;           // raw query tile, then each chunk's psi operand [128][3*rc]
+            uint8_t* Y = smem + 32768;   // A^T image [R][128]
+            uint8_t* Z = smem + 49152;   // S image of the current chunk [128][3*rc]
+            const bool z_early = R <= 64;  // Y and Z do not overlap: load chunk 0's S image up front
+            auto sb_bytes = [&](int ch) -> uint32_t {
+                const int rc = min(64, R - 64 * ch);
+                return static_cast<uint32_t>((3 * rc + 63) / 64) * (D * 128);
+            };
+            const uint8_t* sb_head = a.sb_img + static_cast<size_t>(bh) * nch * kSbChunkBytes;
+            if (tid == 0) {
+                mbar_expect_tx(bar_eld, 32768 + R * 256 + (z_early ? sb_bytes(0) : 0));
+                tma_load_4d(X, &tm_qraw, bar_eld, 0, h, alpha * blk, b);
+                tma_load_4d(X + 16384, &tm_qraw, bar_eld, 64, h, alpha * blk, b);
+                bulk_load(Y, a.at_img, R * 256, bar_eld);
+                if (z_early) bulk_load(Z, sb_head, sb_bytes(0), bar_eld);
+                ++n_eld_issued;
+                if (mbar_wait(bar_eld, n_eld & 1, tmo, abort_flag)) {
+                    ++n_eld;
+                    tc_fence_after();
+                    const uint32_t idesc_phi = idesc_bf16_f32(128, R);
 #pragma unroll
-    for (int e = 0; e < D; ++e) acc[e] = 0.f;
-    float inv_den = 0.f;
-    if (a.lowrank && !aborted) {
-        float* As = reinterpret_cast<float*>(smem);  // [D][R] fp32, reuses the tile buffers
-        for (int e = tid; e < D * g.R; e += kThreads) As[e] = __bfloat162float(a.A[e]);
-        __syncthreads();
-        if (row_valid) {
-            const __nv_bfloat16* qrow = a.q_raw + ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;
-            const float* Sh = a.S + static_cast<size_t>(bh) * g.R * D;
-            const float* zh = a.z + static_cast<size_t>(bh) * g.R;
-            float den = 0.f;
-            for (int c0 = 0; c0 < g.R; c0 += 16) {
-                float phi[16];
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t ad = sdesc_sw128(smem_addr(X) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(smem_addr(Y) + (kk >> 2) * (R * 128) + (kk & 3) * 32, 16, 1024);
+                        umma_ss(tS, ad, bd, idesc_phi, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar_emm);
+                    ++n_emm_issued;
+                } else {
+                    fail();
+                }
+            }
+            bool ok = mbar_wait(bar_emm, n_emm & 1, tmo, abort_flag);
+            if (__syncthreads_or(!ok)) {
+                if (tid == 0) fail();
+            } else {
+                ++n_emm;
+                tc_fence_after();
+                if (!z_early && tid == 0) {  // the feature product has finished with Y
+                    mbar_expect_tx(bar_eld, sb_bytes(0));
+                    bulk_load(Z, sb_head, sb_bytes(0), bar_eld);
+                    ++n_eld_issued;
+                }
+                // phi . z over all R features (unrotated features in the denominator)
+                const float* zh = a.z + static_cast<size_t>(bh) * R;
+                float den = 0.f;
 #pragma unroll
-                for (int c = 0; c < 16; ++c) phi[c] = 0.f;
-                for (int d0 = 0; d0 < D; d0 += 8) {
-                    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow + d0));
-                    const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    if (c0 < R) {
+                        uint32_t v[32];
+                        tmem_ld32(tS + lane_base + c0, v);
+                        tmem_ld_wait(v);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 qf = __bfloat1622float2(q2[u]);
-                        const float* a0 = As + (d0 + 2 * u) * g.R + c0;
-                        const float* a1 = a0 + g.R;
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) phi[c] = fmaf(qf.y, a1[c], fmaf(qf.x, a0[c], phi[c]));
+                        for (int i = 0; i < 32; ++i)
+                            if (c0 + i < R) den = fmaf(fmaxf(__uint_as_float(v[i]), 0.f), __ldg(zh + c0 + i), den);
                     }
                 }
+                const float l_eff = keep > 0 ? l_run : 1.f;
+                const float scale = l_eff / (den + 1e-6f);
+                const int n_tab = n < g.L ? n : g.L - 1;  // rows past the sequence: any valid table entry
+                for (int ch = 0; ch < nch && ok; ++ch) {
+                    const int rc = min(64, R - 64 * ch);
+                    if (ch > 0) {  // the previous chunk's product must have finished with X and Z
+                        ok = mbar_wait(bar_emm, n_emm & 1, tmo, abort_flag);
+                        if (__syncthreads_or(!ok)) {
+                            if (tid == 0) fail();
+                            ok = false;
+                            break;
+                        }
+                        ++n_emm;
+                        tc_fence_after();
+                        if (tid == 0) {
+                            mbar_expect_tx(bar_eld, sb_bytes(ch));
+                            bulk_load(Z, sb_head + static_cast<size_t>(ch) * kSbChunkBytes, sb_bytes(ch), bar_eld);
+                            ++n_eld_issued;
+                        }
+                    }
+                    uint32_t v[2][32];
+                    tmem_ld32(tS + lane_base + 64 * ch, v[0]);
+                    tmem_ld32(tS + lane_base + 64 * ch + 32, v[1]);
+                    tmem_ld_wait(v[0]);
+                    reg_fence(v[1]);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    phi[c] = fmaxf(phi[c], 0.f);
-                    den = fmaf(phi[c], __ldg(zh + c0 + c), den);
+                    for (int pp = 0; pp < 32; ++pp) {
+                        if (2 * pp < rc) {
+                            const float x0 = fmaxf(__uint_as_float(v[pp >> 4][(2 * pp) & 31]), 0.f);
+                            const float x1 = fmaxf(__uint_as_float(v[pp >> 4][(2 * pp + 1) & 31]), 0.f);
+                            const int2 pi = __ldg(a.pairs + 32 * ch + pp);
+                            const double2 cs = __ldg(a.tab + pi.y + token_axis_pos(n_tab, pi.x, g.H, g.W));
+                            const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+                            const float y0 = (x0 * cf - x1 * sf) * scale, y1 = (x0 * sf + x1 * cf) * scale;
+                            const __nv_bfloat162 hi = __floats2bfloat162_rn(y0, y1);
+                            const float2 hf = __bfloat1622float2(hi);
+                            const __nv_bfloat162 lo = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
+                            const uint32_t hb = *reinterpret_cast<const uint32_t*>(&hi);
+                            const uint32_t lb = *reinterpret_cast<const uint32_t*>(&lo);
+                            *reinterpret_cast<uint32_t*>(X + sw128_offset(i_row, 2 * pp, 128)) = hb;
+                            *reinterpret_cast<uint32_t*>(X + sw128_offset(i_row, rc + 2 * pp, 128)) = hb;
+                            *reinterpret_cast<uint32_t*>(X + sw128_offset(i_row, 2 * rc + 2 * pp, 128)) = lb;
+                        }
+                    }
+                    fence_async_smem();
+                    tc_fence_before();
+                    __syncthreads();
+                    if (tid == 0 && !*abort_flag) {
+                        // chunk 0's S image came with the first load phase when it was loaded up front
+                        const bool z_landed = (ch == 0 && z_early);
+                        if (z_landed || mbar_wait(bar_eld, n_eld & 1, tmo, abort_flag)) {
+                            if (!z_landed) ++n_eld;
+                            tc_fence_after();
+                            const uint32_t idesc_lr = idesc_bf16_f32(128, D);
+                            for (int kk = 0; kk < (3 * rc) / 16; ++kk) {
+                                const uint64_t ad = sdesc_sw128(smem_addr(X) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                                const uint64_t bd = sdesc_sw128(smem_addr(Z) + (kk >> 2) * (D * 128) + (kk & 3) * 32, 16, 1024);
+                                umma_ss(tO, ad, bd, idesc_lr, (keep > 0 || ch > 0 || kk > 0) ? 1u : 0u);
+                            }
+                            umma_commit(bar_emm);
+                            ++n_emm_issued;
+                        } else {
+                            fail();
+                        }
+                    }
                 }
-#pragma unroll
-                for (int pp = 0; pp < 8; ++pp) {
-                    const int2 pi = __ldg(a.pairs + (c0 >> 1) + pp);  // (axis, table offset)
-                    const double2 cs = __ldg(a.tab + pi.y + token_axis_pos(n, pi.x, g.H, g.W));
-                    const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
-                    const float x0 = phi[2 * pp], x1 = phi[2 * pp + 1];
-                    phi[2 * pp] = x0 * cf - x1 * sf;
-                    phi[2 * pp + 1] = x0 * sf + x1 * cf;
-                }
-#pragma unroll 4
-                for (int c = 0; c < 16; ++c) {
-                    const float4* s4 = reinterpret_cast<const float4*>(Sh + (c0 + c) * D);
-#pragma unroll
-                    for (int e4 = 0; e4 < D / 4; ++e4) {
-                        const float4 sv4 = __ldg(s4 + e4);
-                        acc[4 * e4 + 0] = fmaf(phi[c], sv4.x, acc[4 * e4 + 0]);
-                        acc[4 * e4 + 1] = fmaf(phi[c], sv4.y, acc[4 * e4 + 1]);
-                        acc[4 * e4 + 2] = fmaf(phi[c], sv4.z, acc[4 * e4 + 2]);
-                        acc[4 * e4 + 3] = fmaf(phi[c], sv4.w, acc[4 * e4 + 3]);
+                if (ok) {
+                    ok = !*abort_flag && mbar_wait(bar_emm, n_emm & 1, tmo, abort_flag);
+                    if (__syncthreads_or(!ok)) {
+                        if (tid == 0) fail();
+                    } else {
+                        ++n_emm;
+                        tc_fence_after();
+                        inv_l = 1.f / l_eff;
+                        o_live = true;
                     }
                 }
             }
-            inv_den = 1.f / (den + 1e-6f);
         }
     }
-    const float inv_l = (keep > 0 && l_run > 0.f) ? 1.f / l_run : 0.f;
-    const bool warp_has_rows = (warp * 32 < blk) && (alpha * blk + warp * 32 < g.L) && !aborted;
+    float acc[D == 128 ? 1 : D];
+    float inv_den = 0.f;
+    if constexpr (D != 128) {
+#pragma unroll
+        for (int e = 0; e < D; ++e) acc[e] = 0.f;
+        if (a.lowrank && !aborted) {
+            float* As = reinterpret_cast<float*>(smem);  // [D][R] fp32, reuses the tile buffers
+            for (int e = tid; e < D * g.R; e += kThreads) As[e] = __bfloat162float(a.A[e]);
+            __syncthreads();
+            if (row_valid) {
+                const __nv_bfloat16* qrow = a.q_raw + ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;
+                const float* Sh = a.S + static_cast<size_t>(bh) * g.R * D;
+                const float* zh = a.z + static_cast<size_t>(bh) * g.R;
+                float den = 0.f;
+                for (int c0 = 0; c0 < g.R; c0 += 16) {
+                    float phi[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) phi[c] = 0.f;
+                    for (int d0 = 0; d0 < D; d0 += 8) {
+                        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow + d0));
+                        const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float2 qf = __bfloat1622float2(q2[u]);
+                            const float* a0 = As + (d0 + 2 * u) * g.R + c0;
+                            const float* a1 = a0 + g.R;
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) phi[c] = fmaf(qf.y, a1[c], fmaf(qf.x, a0[c], phi[c]));
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        phi[c] = fmaxf(phi[c], 0.f);
+                        den = fmaf(phi[c], __ldg(zh + c0 + c), den);
+                    }
+#pragma unroll
+                    for (int pp = 0; pp < 8; ++pp) {
+                        const int2 pi = __ldg(a.pairs + (c0 >> 1) + pp);  // (axis, table offset)
+                        const double2 cs = __ldg(a.tab + pi.y + token_axis_pos(n, pi.x, g.H, g.W));
+                        const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+                        const float x0 = phi[2 * pp], x1 = phi[2 * pp + 1];
+                        phi[2 * pp] = x0 * cf - x1 * sf;
+                        phi[2 * pp + 1] = x0 * sf + x1 * cf;
+                    }
+#pragma unroll 4
+                    for (int c = 0; c < 16; ++c) {
+                        const float4* s4 = reinterpret_cast<const float4*>(Sh + (c0 + c) * D);
+#pragma unroll
+                        for (int e4 = 0; e4 < D / 4; ++e4) {
+                            const float4 sv4 = __ldg(s4 + e4);
+                            acc[4 * e4 + 0] = fmaf(phi[c], sv4.x, acc[4 * e4 + 0]);
+                            acc[4 * e4 + 1] = fmaf(phi[c], sv4.y, acc[4 * e4 + 1]);
+                            acc[4 * e4 + 2] = fmaf(phi[c], sv4.z, acc[4 * e4 + 2]);
+                            acc[4 * e4 + 3] = fmaf(phi[c], sv4.w, acc[4 * e4 + 3]);
+                        }
+                    }
+                }
+                inv_den = 1.f / (den + 1e-6f);
+            }
+        }
+    }
+    const bool aborted2 = *abort_flag != 0;
+    const bool warp_has_rows = (warp * 32 < blk) && (alpha * blk + warp * 32 < g.L) && !aborted2;
     if (warp_has_rows) {
         const size_t obase = ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            if (keep > 0) {
+            if (o_live) {
                 tmem_ld32(tO + lane_base + c * 32, o);
                 tmem_ld_wait(o);
             } else {
@@ -416,7 +570,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (row_valid) {
                 float r[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(o[i]) * inv_l + acc[c * 32 + i] * inv_den;
+                for (int i = 0; i < 32; ++i) {
+                    float x = __uint_as_float(o[i]) * inv_l;
+                    if constexpr (D != 128) x += acc[c * 32 + i] * inv_den;
+                    r[i] = x;
+                }
                 if (a.out_bf16) {
                     __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(a.out) + obase + c * 32;
 #pragma unroll
@@ -442,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     }
     // ------------------------------------------------------------------ teardown
-    if (aborted && tid == 0) {
+    if (*abort_flag && tid == 0) {
         // Let copies and products still in flight land before the memory is released.  Each wait is
         // bounded (10 ms) and ignores the abort flag.
         volatile int no_abort = 0;
@@ -452,6 +610,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (n_v_issued > n_v_done) mbar_wait(bar_v, n_v_done & 1, drain, &no_abort);
         if (n_s_issued > n_s_done) mbar_wait(bar_s, n_s_done & 1, drain, &no_abort);
         if (n_o_issued > n_o_done) mbar_wait(bar_o, n_o_done & 1, drain, &no_abort);
+        if (n_eld_issued > n_eld) mbar_wait(bar_eld, n_eld & 1, drain, &no_abort);
+        if (n_emm_issued > n_emm) mbar_wait(bar_emm, n_emm & 1, drain, &no_abort);
     }
     tc_fence_before();
     __syncthreads();
@@ -472,11 +632,11 @@ cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, const Geom& g, cud
     if (g.D == 128) {
         e = cudaFuncSetAttribute(attn_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        attn_sm100_kernel<128><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, a, g);
+        attn_sm100_kernel<128><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, a, g);
     } else {
         e = cudaFuncSetAttribute(attn_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        attn_sm100_kernel<64><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, a, g);
+        attn_sm100_kernel<64><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, a, g);
     }
     return cudaGetLastError();
 }

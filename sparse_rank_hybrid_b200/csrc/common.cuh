@@ -56,12 +56,19 @@ int lowrank_nsplit(const Geom& g);
 bool make_map_headmajor(CUtensorMap* m, const void* base, uint64_t rows, int D, int box_rows);
 bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int D, int box_tokens);
 cudaError_t launch_lowrank_reduce(const float* s_part, const float* z_part, const Geom& g, int nsplit, float* S,
-                                  float* z, cudaStream_t st);
+                                  float* z, const __nv_bfloat16* A, uint8_t* at_img, uint8_t* sb_img, cudaStream_t st);
 
 // fp16 head-major [BH*Lp][D] tensor maps; q box 64 x 128 rows, k/v box 64 x `block` rows, 128-B swizzle.
 struct AttnMaps {
     CUtensorMap q, k, v;
+    CUtensorMap q_raw;  // 4D map over the raw bf16 queries [B][L][Hh][D], box 64 x 1 x 128 x 1
 };
+
+// Operand images for the tensor-core low-rank readout (head_dim 128), built by the reduction:
+//   A^T image: [R rows][128] bf16 K-major, 128-B swizzled (R*256 bytes);
+//   S image per (batch*head, 64-feature chunk): [D rows][3*rc] bf16 K-major swizzled, the K columns
+//   holding (S_hi, S_lo, S_hi) of the chunk's rc features (kSbChunkBytes apart).
+constexpr int kSbChunkBytes = 3 * 128 * 128;
 
 struct AttnArgs {
     const int32_t* idx;
@@ -72,6 +79,8 @@ struct AttnArgs {
     const float* z;
     const double2* tab;
     const int2* pairs;  // per rotary pair: (axis, offset of its cos/sin table)
+    const uint8_t* at_img;  // A^T operand image (head_dim 128)
+    const uint8_t* sb_img;  // S operand images (head_dim 128)
     int lowrank;  // add the low-rank readout
     void* out;
     int out_bf16;

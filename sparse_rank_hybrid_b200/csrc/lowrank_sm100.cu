@@ -62,22 +62,6 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
     return *reinterpret_cast<const uint16_t*>(&h);
 }
 
-__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
-                                            int c3) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
-        "[%2];" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-        : "memory");
-}
-
-// Byte offset of element (row, col) in a tile of 64-column slabs of [rows][128 B] with the 128-B swizzle
-// (16-byte chunk index XOR row % 8): the layout TMA writes and the tensor-core descriptors read.
-__device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows_per_slab) {
-    const int slab = col >> 6, c = col & 63;
-    return static_cast<uint32_t>(slab * rows_per_slab * 128 + row * 128 + ((((c >> 3) ^ (row & 7)) << 4) | ((c & 7) << 1)));
-}
-
 }  // namespace
 
 struct LrArgs {

@@ -9,6 +9,7 @@
 // Method: RoLA ("3 Preliminary" 3D RoPE; "4.1" block-sparse + low-rank branches; "4.2" first r rotary
 // coordinates; "4.3" RoPE outside the activation; "B.1" one query-independent sum per head).
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace slra {
 
@@ -402,8 +403,19 @@ cudaError_t launch_lowrank_partial(const __nv_bfloat16* k, const __nv_bfloat16* 
     return cudaErrorInvalidValue;
 }
 
+__device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<const uint16_t*>(&h);
+}
+
+// Fixed-order sum of the split-L partials -> S [R][D] and z [R] per head.  With images requested
+// (head_dim 128) it also writes, per head and 64-feature chunk, the S operand image of the attention
+// epilogue's readout product (K columns S_hi | S_lo | S_hi, bf16 split so that hi + lo = S to ~2^-16),
+// and (blocks of head 0) the A^T operand image of its feature product.
 __global__ void lowrank_reduce_kernel(const float* __restrict__ s_part, const float* __restrict__ z_part, int RD,
-                                      int R, int nsplit, float* __restrict__ S, float* __restrict__ z) {
+                                      int R, int D, int nsplit, float* __restrict__ S, float* __restrict__ z,
+                                      const __nv_bfloat16* __restrict__ A, uint8_t* __restrict__ at_img,
+                                      uint8_t* __restrict__ sb_img) {
     const int bh = blockIdx.y;
     const int o = blockIdx.x * blockDim.x + threadIdx.x;
     if (o < RD) {
@@ -411,6 +423,21 @@ __global__ void lowrank_reduce_kernel(const float* __restrict__ s_part, const fl
         float a = 0.f;
         for (int s = 0; s < nsplit; ++s) a += p[static_cast<size_t>(s) * RD];
         S[static_cast<size_t>(bh) * RD + o] = a;
+        if (sb_img) {
+            const int c = o / D, e = o % D;
+            const int nch = (R + 63) / 64, ch = c / 64, cc = c % 64, rc = min(64, R - 64 * ch);
+            const uint16_t hi = bf16_rn_bits(a);
+            const uint16_t lo = bf16_rn_bits(a - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+            uint8_t* img = sb_img + (static_cast<size_t>(bh) * nch + ch) * kSbChunkBytes;
+            *reinterpret_cast<uint16_t*>(img + sw128_offset(e, cc, D)) = hi;
+            *reinterpret_cast<uint16_t*>(img + sw128_offset(e, rc + cc, D)) = lo;
+            *reinterpret_cast<uint16_t*>(img + sw128_offset(e, 2 * rc + cc, D)) = hi;
+        }
+        if (at_img && bh == 0) {  // element (c, d) of A^T = A[d][c]
+            const int c = o / D, d = o % D;
+            *reinterpret_cast<uint16_t*>(at_img + sw128_offset(c, d, R)) =
+                *reinterpret_cast<const uint16_t*>(A + static_cast<size_t>(d) * R + c);
+        }
     } else if (o < RD + R) {
         const int c = o - RD;
         const float* p = z_part + static_cast<size_t>(bh) * nsplit * R + c;
@@ -421,10 +448,11 @@ __global__ void lowrank_reduce_kernel(const float* __restrict__ s_part, const fl
 }
 
 cudaError_t launch_lowrank_reduce(const float* s_part, const float* z_part, const Geom& g, int nsplit, float* S,
-                                  float* z, cudaStream_t st) {
+                                  float* z, const __nv_bfloat16* A, uint8_t* at_img, uint8_t* sb_img,
+                                  cudaStream_t st) {
     const int RD = g.R * g.D;
     dim3 grid((RD + g.R + 255) / 256, g.BH());
-    lowrank_reduce_kernel<<<grid, 256, 0, st>>>(s_part, z_part, RD, g.R, nsplit, S, z);
+    lowrank_reduce_kernel<<<grid, 256, 0, st>>>(s_part, z_part, RD, g.R, g.D, nsplit, S, z, A, at_img, sb_img);
     return cudaGetLastError();
 }
 

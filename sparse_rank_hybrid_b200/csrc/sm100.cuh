@@ -77,6 +77,39 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// 4D tiled load (no multicast), coordinates innermost first.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+        "[%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+// Plain bulk copy global -> shared (no multicast); both addresses 16-B aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+// Byte offset of element (row, col) of a 16-bit tile stored as 64-column slabs of [rows][128 B] with the
+// 128-B swizzle (16-byte chunk index XOR row % 8): the layout TMA writes and the K-major / MN-major
+// SW128 matrix descriptors read (the tile base must be 1024-B aligned).
+__host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows_per_slab) {
+    const int slab = col >> 6, c = col & 63;
+    return static_cast<uint32_t>(slab * rows_per_slab * 128 + row * 128 +
+                                 ((((c >> 3) ^ (row & 7)) << 4) | ((c & 7) << 1)));
+}
+
+// Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulation, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(N) >> 3) << 17) |
+           ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+
 // ------------------------------------------------------------------------------- tcgen05 / TMEM
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {  // whole warp
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
