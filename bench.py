@@ -195,12 +195,11 @@ def run_ours(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     x = I.make_inputs(w)
     q, k, v, A = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v", "A"))
-    ev_a = torch.cuda.Event(enable_timing=True)
-    ev_b = torch.cuda.Event(enable_timing=True)
-    ev_a.record()
-    ev_b.record()
+    stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+    for e in stage_ev:
+        e.record()
     torch.cuda.synchronize()
-    prob = slra.Problem.from_workload(w, attn_events=(ev_a.cuda_event, ev_b.cuda_event))
+    prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev))
     ws = slra.alloc_workspace(prob, dev)
     out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
@@ -226,7 +225,7 @@ def run_ours(args, w, rank, world, local_rank):
     f_attn = f_sparse + 4.0 * w.L * w.rank * w.head_dim * BH
 
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    attn_ms = []
+    stage_ms = []
     clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
     barrier()
@@ -239,7 +238,7 @@ def run_ours(args, w, rank, world, local_rank):
         slra.attn_fwd(prob, q, k, v, A, out=out, workspace=ws)
         step_ev[i][1].record(stream)
         torch.cuda.synchronize()
-        attn_ms.append(ev_a.elapsed_time(ev_b))
+        stage_ms.append([stage_ev[i].elapsed_time(stage_ev[i + 1]) for i in range(6)])
     barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -279,7 +278,8 @@ def run_ours(args, w, rank, world, local_rank):
     if rank != 0:
         return
     hbm, tf_burst, tf_sust, src = peaks()
-    attn_avg = statistics.mean(attn_ms)
+    stage_avg = [statistics.mean(x[i] for x in stage_ms) for i in range(6)]
+    attn_avg = stage_avg[5]
     achieved = f_attn / (attn_avg * 1e-3) / 1e12
     traffic = load_traffic(w.name)
     bytes_min = F.io_bytes(w.batch, w.L, w.heads, w.head_dim, w.rank, 4)
@@ -302,6 +302,8 @@ def run_ours(args, w, rank, world, local_rank):
                           "note": "max(kept FLOPs / sustained tensor peak, min bytes / HBM peak) vs ms_per_step"},
         "e2e": {"value": f_total * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "kernel_ms": dict(zip(("rope_table", "rope_pool", "select", "lowrank_partial", "lowrank_reduce",
+                               "attention"), (round(x, 4) for x in stage_avg))),
         "gpu_launches": 6 * args.steps,
         "clocks": clk,
         "cpu_baseline": {"value": cpu_v, "unit": "TFLOP/s", "cores": cpu_threads, "kind": "oracle",

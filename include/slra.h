@@ -92,9 +92,13 @@ enum { SLRA_BRANCH_SPARSE = 1, SLRA_BRANCH_LOWRANK = 2, SLRA_BRANCH_BOTH = 3 };
  *                           result independent of it, which the tests use).
  *   rope_split              rotary pairs per (t, h, w); all zero = default split described above.
  *   wait_timeout_ns         bound of every wait inside the kernels (default 2e9 ns = 2 s).
- *   attn_events             optional pair of cudaEvent_t (NULL = none): recorded on `stream` right
- *                           before and right after the attention kernel, so a caller can time the
- *                           dominant kernel alone.  The caller creates and owns them.
+ *   stage_events            optional cudaEvent_t handles (NULL entries are skipped), recorded on
+ *                           `stream` between the library's launches so a caller can time each
+ *                           kernel alone: [0] before the first launch, [1] after the rotary tables,
+ *                           [2] after RoPE + pooling, [3] after block selection, [4] after the low-rank
+ *                           partial sums, [5] after their reduction, [6] after the attention kernel
+ *                           (the branch entry points record the boundaries of the stages they run).
+ *                           The caller creates and owns them.
  */
 typedef struct slra_problem {
     int64_t batch, heads, head_dim;
@@ -108,7 +112,7 @@ typedef struct slra_problem {
     int64_t pos_offset[3];
     int64_t rope_split[3];
     uint64_t wait_timeout_ns;
-    void* attn_events[2];
+    void* stage_events[7];
 } slra_problem;
 
 /*

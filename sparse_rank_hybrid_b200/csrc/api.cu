@@ -196,15 +196,30 @@ slra_status check_ws(const Derived& d, void* ws, size_t bytes) {
 
 slra_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SLRA_OK : SLRA_ERR_CUDA; }
 
+// Record the caller's timing event for stage boundary i, if one was given.
+slra_status mark(const slra_problem* p, int i, cudaStream_t st) {
+    void* e = p->stage_events[i];
+    if (e && cudaEventRecord(static_cast<cudaEvent_t>(e), st) != cudaSuccess) return SLRA_ERR_CUDA;
+    return SLRA_OK;
+}
+
+unsigned long long timeout_of(const slra_problem* p) {
+    return p->wait_timeout_ns ? p->wait_timeout_ns : 2000000000ull;
+}
+
+
 // Tables + RoPE/pooling + selection.
-slra_status run_select(const Derived& d, const Ptrs& w, const void* q, const void* k, const void* v,
-                       cudaStream_t st) {
+slra_status run_select(const slra_problem* p, const Derived& d, const Ptrs& w, const void* q, const void* k,
+                       const void* v, cudaStream_t st) {
     const Geom& g = d.g;
     cudaError_t e = launch_rope_pool(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                      static_cast<const __nv_bfloat16*>(v), w.tab, w.pairs, g, w.qh, w.kh, w.vh,
                                      w.qbar, w.kbar, w.status, st);
     if (e != cudaSuccess) return SLRA_ERR_CUDA;
-    return cuda_status(launch_select(w.qbar, w.kbar, g, w.idx, w.tie, st));
+    slra_status s = mark(p, 2, st);
+    if (s != SLRA_OK) return s;
+    if ((s = cuda_status(launch_select(w.qbar, w.kbar, g, w.idx, w.tie, st))) != SLRA_OK) return s;
+    return mark(p, 3, st);
 }
 
 // Low-rank partial sums: tensor-core kernel for head_dim 128, CUDA-core kernel otherwise.
@@ -219,22 +234,27 @@ cudaError_t lowrank_partial(const Derived& d, const void* k, const void* v, cons
     return launch_lowrank_partial(kb, vb, Ab, tab, pairs, d.g, nsplit, s_part, z_part, st);
 }
 
-slra_status run_lowrank(const Derived& d, const Ptrs& w, const void* k, const void* v, const void* A,
-                        unsigned long long timeout_ns, cudaStream_t st) {
+slra_status run_lowrank(const slra_problem* p, const Derived& d, const Ptrs& w, const void* k, const void* v,
+                        const void* A, cudaStream_t st) {
     const Geom& g = d.g;
-    cudaError_t e = lowrank_partial(d, k, v, A, w.tab, w.pairs, d.nsplit, w.s_part, w.z_part, w.status, timeout_ns, st);
+    cudaError_t e = lowrank_partial(d, k, v, A, w.tab, w.pairs, d.nsplit, w.s_part, w.z_part, w.status,
+                                    timeout_of(p), st);
     if (e != cudaSuccess) return SLRA_ERR_CUDA;
-    return cuda_status(launch_lowrank_reduce(w.s_part, w.z_part, g, d.nsplit, w.S, w.z,
-                                             static_cast<const __nv_bfloat16*>(A), w.at_img, w.sb_img, st));
+    slra_status s = mark(p, 4, st);
+    if (s != SLRA_OK) return s;
+    if ((s = cuda_status(launch_lowrank_reduce(w.s_part, w.z_part, g, d.nsplit, w.S, w.z,
+                                               static_cast<const __nv_bfloat16*>(A), w.at_img, w.sb_img, st))) !=
+        SLRA_OK)
+        return s;
+    return mark(p, 5, st);
 }
 
-slra_status begin(const Derived& d, const Ptrs& w, cudaStream_t st) {
+slra_status begin(const slra_problem* p, const Derived& d, const Ptrs& w, cudaStream_t st) {
+    slra_status s = mark(p, 0, st);
+    if (s != SLRA_OK) return s;
     if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return SLRA_ERR_CUDA;
-    return cuda_status(launch_rope_table(w.tab, w.pairs, d.meta, d.table_entries, st));
-}
-
-unsigned long long timeout_of(const slra_problem* p) {
-    return p->wait_timeout_ns ? p->wait_timeout_ns : 2000000000ull;
+    if ((s = cuda_status(launch_rope_table(w.tab, w.pairs, d.meta, d.table_entries, st))) != SLRA_OK) return s;
+    return mark(p, 1, st);
 }
 
 size_t qkv_bytes(const Derived& d) {
@@ -328,11 +348,11 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
         !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, 128))
         return SLRA_ERR_CUDA;
 
-    if ((s = begin(d, w, st)) != SLRA_OK) return s;
+    if ((s = begin(p, d, w, st)) != SLRA_OK) return s;
     if (branches & SLRA_BRANCH_SPARSE)
-        if ((s = run_select(d, w, q, k, v, st)) != SLRA_OK) return s;
+        if ((s = run_select(p, d, w, q, k, v, st)) != SLRA_OK) return s;
     if (branches & SLRA_BRANCH_LOWRANK)
-        if ((s = run_lowrank(d, w, k, v, A, timeout_of(p), st)) != SLRA_OK) return s;
+        if ((s = run_lowrank(p, d, w, k, v, A, st)) != SLRA_OK) return s;
 
     AttnArgs a;
     a.idx = w.idx;
@@ -350,12 +370,8 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
     a.out_bf16 = p->out_dtype == SLRA_OUT_BF16 ? 1 : 0;
     a.status = w.status;
     a.timeout_ns = p->wait_timeout_ns ? p->wait_timeout_ns : 2000000000ull;
-    if (p->attn_events[0] && cudaEventRecord(static_cast<cudaEvent_t>(p->attn_events[0]), st) != cudaSuccess)
-        return SLRA_ERR_CUDA;
     if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
-    if (p->attn_events[1] && cudaEventRecord(static_cast<cudaEvent_t>(p->attn_events[1]), st) != cudaSuccess)
-        return SLRA_ERR_CUDA;
-    return SLRA_OK;
+    return mark(p, 6, st);
 }
 
 size_t slra_host_io_bytes(const slra_problem* p) {
@@ -405,8 +421,8 @@ slra_status slra_select_blocks(const slra_problem* p, const void* q, const void*
     if ((s = check_device()) != SLRA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const Ptrs w = carve(workspace, d);
-    if ((s = begin(d, w, st)) != SLRA_OK) return s;
-    return run_select(d, w, q, k, v, st);
+    if ((s = begin(p, d, w, st)) != SLRA_OK) return s;
+    return run_select(p, d, w, q, k, v, st);
 }
 
 slra_status slra_lowrank_summary(const slra_problem* p, const void* k, const void* v, const void* A, void* workspace,
@@ -420,8 +436,8 @@ slra_status slra_lowrank_summary(const slra_problem* p, const void* k, const voi
     if ((s = check_device()) != SLRA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const Ptrs w = carve(workspace, d);
-    if ((s = begin(d, w, st)) != SLRA_OK) return s;
-    return run_lowrank(d, w, k, v, A, timeout_of(p), st);
+    if ((s = begin(p, d, w, st)) != SLRA_OK) return s;
+    return run_lowrank(p, d, w, k, v, A, st);
 }
 
 slra_status slra_device_status(void* workspace, slra_stream_t stream, int32_t* status) {

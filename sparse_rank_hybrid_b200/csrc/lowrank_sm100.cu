@@ -2,8 +2,8 @@
 //   S = sum_j psi(k_j) v_j^T,   z = sum_j phi(k_j),   phi(k) = relu(k A),   psi = phi with its first
 // r coordinates rotated by the token's 3D RoPE angles (RoLA "4.1", "4.2", "4.3", "B.1").
 //
-// Persistent CTAs (one per SM, 128 threads) walk work items = (head, range of 128-token tiles).  Per
-// tile:
+// Persistent CTAs (one per SM, 256 threads: two threads per token row, each taking half of the
+// features) walk work items = (head, range of 128-token tiles).  Per tile:
 //   TMA    raw k and v tiles [128 tokens][128] bf16 straight from the [B][L][Hh][D] inputs (4D tensor
 //          maps, 128-B swizzle, two stages so the next tiles stream in while this one is processed);
 //   MMA    phi = k A  (M = 128 tokens, N = r, K = 128; A^T staged once per CTA as the B operand);
@@ -31,7 +31,7 @@ struct LrLayout {
     int off_k[kStages], off_v[kStages];
     int off_at;       // A^T [r][128] bf16, K-major swizzled
     int off_psi;      // [128 tokens][2*rp] bf16, 64-column slabs
-    int off_zred;     // [4 warps][R/2] fp32 (z is reduced in two halves)
+    int off_zred;     // [8 warps][R/2] fp32
     int off_bar;
     int off_misc;
     int bytes;
@@ -46,8 +46,9 @@ __host__ __device__ inline LrLayout lr_layout(int R) {
     o += ((R * 256 + 1023) / 1024) * 1024;
     l.off_psi = o;
     o += kTok * 2 * l.rp * 2;
-    l.off_zred = o;
-    o += 4 * (R / 2) * 4;
+    // R = 128 has no psi padding to preserve, so its z slots reuse the psi buffer (free at item end)
+    l.off_zred = R == 128 ? l.off_psi : o;
+    if (R != 128) o += 8 * (R / 2) * 4;
     l.off_bar = o;
     o += 128;
     l.off_misc = o;
@@ -77,20 +78,23 @@ struct LrArgs {
 };
 
 template <int R>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     lowrank_sm100_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          LrArgs a, Geom g) {
     const LrLayout lay = lr_layout(R);
     constexpr int RP = R <= 64 ? 64 : 128;
+    constexpr int RH = R / 2;           // features per thread: two threads share a token row
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.off_bar);
     uint64_t* bar_kv = bars;         // [kStages]: k and v tile of a stage landed
-    uint64_t* bar_phi = bars + 2;    // phi MMA done
+    uint64_t* bar_phi = bars + 2;    // phi MMA done (covers every earlier MMA)
     uint64_t* bar_s = bars + 3;      // S MMA done (covers every earlier MMA)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + lay.off_misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + lay.off_misc + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int row = tid & 127;          // token row = TMEM lane
+    const int half = tid >> 7;          // features [half*RH, half*RH + RH)
     const uint64_t tmo = a.timeout_ns;
 
     if (tid == 0) {
@@ -103,13 +107,13 @@ __global__ void __launch_bounds__(128, 1)
         tmem_relinquish();
     }
     // A^T as the K-major B operand of phi = k A: row n = feature, 128 dims in two swizzled slabs.
-    for (int e = tid; e < R * kD; e += 128) {
+    for (int e = tid; e < R * kD; e += 256) {
         const int d = e / R, c = e % R;  // coalesced read of A [D][R]
         *reinterpret_cast<uint16_t*>(smem + lay.off_at + sw128_offset(c, d, R)) =
             *reinterpret_cast<const uint16_t*>(a.A + e);
     }
     // zero the padding columns of both psi halves once; tiles only ever write the first R of each half
-    for (int e = tid; e < kTok * 2 * RP; e += 128) {
+    for (int e = tid; e < kTok * 2 * RP; e += 256) {
         const int t = e / (2 * RP), col = e % (2 * RP);
         if ((col % RP) >= R) *reinterpret_cast<uint16_t*>(smem + lay.off_psi + sw128_offset(t, col, kTok)) = 0;
     }
@@ -120,15 +124,15 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t t_phi = tmem;          // R columns
     const uint32_t t_s = tmem + 128;      // 2*RP columns: S^T hi | lo
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t idesc_phi = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(R) >> 3) << 17) | ((128u >> 4) << 24);
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t idesc_phi = idesc_bf16_f32(128, R);
     const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                              ((uint32_t(2 * RP) >> 3) << 17) | ((128u >> 4) << 24);
     const uint32_t at_addr = smem_addr(smem + lay.off_at), psi_addr = smem_addr(smem + lay.off_psi);
 
     const int ntiles = (g.L + kTok - 1) / kTok;
     const int n_items = g.BH() * a.nsplit;
-    // The sequence of (item, tile) this CTA processes, flattened, so loads can run two tiles ahead.
+    // The sequence of (item, tile) this CTA processes, flattened, so loads can run ahead.
     auto tile_of = [&](int q, int& item, int& tile) -> bool {  // q-th tile of this CTA
         int it = blockIdx.x;
         while (it < n_items) {
@@ -144,6 +148,11 @@ __global__ void __launch_bounds__(128, 1)
     // thread 0's bookkeeping of issued / observed operations (for the bounded drain on abort)
     int n_load[kStages] = {0, 0}, n_wait[kStages] = {0, 0};
     int n_s_issued = 0, n_s_done = 0, n_phi_issued = 0;
+    int q_total = 0;  // tiles this CTA will process
+    {
+        int it2, t2;
+        while (tile_of(q_total, it2, t2)) ++q_total;
+    }
     auto issue_load = [&](int q) {
         int item, tile;
         if (!tile_of(q, item, tile)) return;
@@ -160,15 +169,32 @@ __global__ void __launch_bounds__(128, 1)
         *abort_flag = 1;
         atomicOr(a.status, kDevTimeout);
     };
+    // phi_q = k_q A for the q-th tile (thread 0): wait for its k tile, issue, commit
+    auto issue_phi = [&](int q) -> bool {
+        const int s = q % kStages;
+        if (!mbar_wait(bar_kv + s, n_wait[s] & 1, tmo, abort_flag)) return false;
+        ++n_wait[s];
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(smem_addr(smem + lay.off_k[s]) + (kk >> 2) * (kTok * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(at_addr + (kk >> 2) * (R * 128) + (kk & 3) * 32, 16, 1024);
+            umma_ss(t_phi, ad, bd, idesc_phi, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_phi);
+        ++n_phi_issued;
+        return true;
+    };
     if (tid == 0) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
         issue_load(0);
         issue_load(1);
+        if (q_total > 0 && !issue_phi(0)) fail();
     }
 
     int q = 0;      // running tile count of this CTA (same in every thread)
-    int n_phi = 0;  // phi MMAs completed (same in every thread)
+    int n_phi = 0;  // phi MMAs observed complete (same in every thread)
     int n_s = 0;    // S MMAs issued (same in every thread)
     bool aborted = false;
     for (int item = blockIdx.x; item < n_items && !aborted; item += gridDim.x) {
@@ -176,33 +202,17 @@ __global__ void __launch_bounds__(128, 1)
         const int t0 = split * a.tiles_per_split, t1 = min(ntiles, t0 + a.tiles_per_split);
         if (t1 <= t0) {  // empty split (never produced by the host plan): contributes zeros
             float* sp0 = a.s_part + (static_cast<size_t>(bh) * a.nsplit + split) * R * kD;
-            for (int c = 0; c < R; ++c) sp0[c * kD + tid] = 0.f;
+            for (int e = tid; e < R * kD; e += 256) sp0[e] = 0.f;
             if (tid < R) a.z_part[(static_cast<size_t>(bh) * a.nsplit + split) * R + tid] = 0.f;
             continue;
         }
-        float zacc[R];
+        float zacc[RH];
 #pragma unroll
-        for (int c = 0; c < R; ++c) zacc[c] = 0.f;
+        for (int c = 0; c < RH; ++c) zacc[c] = 0.f;
         for (int tile = t0; tile < t1; ++tile, ++q) {
             const int s = q % kStages;
-            // ---- phi = k A
-            if (tid == 0) {
-                if (!mbar_wait(bar_kv + s, n_wait[s] & 1, tmo, abort_flag)) {
-                    fail();
-                } else {
-                    ++n_wait[s];
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint64_t ad = sdesc_sw128(smem_addr(smem + lay.off_k[s]) + (kk >> 2) * (kTok * 128) + (kk & 3) * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(at_addr + (kk >> 2) * (R * 128) + (kk & 3) * 32, 16, 1024);
-                        umma_ss(t_phi, ad, bd, idesc_phi, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(bar_phi);
-                    ++n_phi_issued;
-                }
-            }
-            // (the previous tile's S MMA already completed: thread 0 waited for it before reloading)
+            // phi_q was issued by thread 0 (at the end of the previous tile, or before the loop); its
+            // completion also means every earlier S product has finished with the psi buffer
             const bool ok = mbar_wait(bar_phi, n_phi & 1, tmo, abort_flag);
             if (__syncthreads_or(!ok)) {
                 if (tid == 0) fail();
@@ -211,45 +221,46 @@ __global__ void __launch_bounds__(128, 1)
             }
             ++n_phi;
             tc_fence_after();
-            // ---- relu, z, rotation, psi hi/lo into shared memory (thread = token row)
-            const int n = tile * kTok + tid;
+            // ---- relu, z, rotation, psi hi/lo into shared memory (two threads per token row)
+            const int n = tile * kTok + row;
             const bool real = n < g.L;
-            uint32_t raw[R];
+            uint32_t raw[RH];
 #pragma unroll
-            for (int c0 = 0; c0 < R; c0 += 32) {
-                uint32_t r32[32];  // for R % 32 == 16 the last window also reads 16 unused columns
-                tmem_ld32(t_phi + lane_base + c0, r32);
+            for (int c0 = 0; c0 < RH; c0 += 32) {
+                uint32_t r32[32];  // a window past RH reads unused (in-range) TMEM columns
+                tmem_ld32(t_phi + lane_base + half * RH + c0, r32);
                 tmem_ld_wait(r32);
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (c0 + i < R) raw[c0 + i] = r32[i];
+                    if (c0 + i < RH) raw[c0 + i] = r32[i];
             }
+            const int HW = g.H * g.W;
+            const int pos3[3] = {n / HW, (n / g.W) % g.H, n % g.W};
 #pragma unroll
-            for (int p = 0; p < R / 2; ++p) {
-                float x0 = real ? fmaxf(__uint_as_float(raw[2 * p]), 0.f) : 0.f;
-                float x1 = real ? fmaxf(__uint_as_float(raw[2 * p + 1]), 0.f) : 0.f;
-                zacc[2 * p] += x0;
-                zacc[2 * p + 1] += x1;
+            for (int pp = 0; pp < RH / 2; ++pp) {
+                const int p = half * (RH / 2) + pp;  // global rotary pair
+                float x0 = real ? fmaxf(__uint_as_float(raw[2 * pp]), 0.f) : 0.f;
+                float x1 = real ? fmaxf(__uint_as_float(raw[2 * pp + 1]), 0.f) : 0.f;
+                zacc[2 * pp] += x0;
+                zacc[2 * pp + 1] += x1;
                 float cf = 1.f, sf = 0.f;
                 if (real) {
                     const int2 pi = __ldg(a.pairs + p);
-                    const double2 cs = __ldg(a.tab + pi.y + token_axis_pos(n, pi.x, g.H, g.W));
+                    const double2 cs = __ldg(a.tab + pi.y + pos3[pi.x]);
                     cf = static_cast<float>(cs.x);
                     sf = static_cast<float>(cs.y);
                 }
                 const float y0 = x0 * cf - x1 * sf, y1 = x0 * sf + x1 * cf;
-                const uint16_t h0 = bf16_bits(y0), h1 = bf16_bits(y1);
-                const float r0 = y0 - __uint_as_float(static_cast<uint32_t>(h0) << 16);
-                const float r1 = y1 - __uint_as_float(static_cast<uint32_t>(h1) << 16);
-                const uint32_t hi = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-                const uint32_t lo = static_cast<uint32_t>(bf16_bits(r0)) | (static_cast<uint32_t>(bf16_bits(r1)) << 16);
-                *reinterpret_cast<uint32_t*>(smem + lay.off_psi + sw128_offset(tid, 2 * p, kTok)) = hi;
-                *reinterpret_cast<uint32_t*>(smem + lay.off_psi + sw128_offset(tid, RP + 2 * p, kTok)) = lo;
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(y0, y1);
+                const float2 hf = __bfloat1622float2(hi);
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
+                *reinterpret_cast<__nv_bfloat162*>(smem + lay.off_psi + sw128_offset(row, 2 * p, kTok)) = hi;
+                *reinterpret_cast<__nv_bfloat162*>(smem + lay.off_psi + sw128_offset(row, RP + 2 * p, kTok)) = lo;
             }
             fence_async_smem();
             tc_fence_before();
             __syncthreads();
-            // ---- S^T += v^T [psi_hi | psi_lo]; once it has completed, stage s takes the tile two ahead
+            // ---- S^T += v^T [psi_hi | psi_lo]; then phi of the next tile; then reload stage s
             if (tid == 0 && !*abort_flag) {
                 tc_fence_after();
 #pragma unroll
@@ -260,7 +271,11 @@ __global__ void __launch_bounds__(128, 1)
                 }
                 umma_commit(bar_s);
                 ++n_s_issued;
-                if (mbar_wait(bar_s, n_s_done & 1, tmo, abort_flag)) {
+                bool good = true;
+                // the next tile's phi product goes in right behind (its k tile is already loading)
+                if (q + 1 < q_total) good = issue_phi(q + 1);
+                // stage s is free once this S product is done: refill it with the tile two ahead
+                if (good && mbar_wait(bar_s, n_s_done & 1, tmo, abort_flag)) {
                     ++n_s_done;
                     issue_load(q + kStages);
                 } else {
@@ -280,42 +295,42 @@ __global__ void __launch_bounds__(128, 1)
         tc_fence_after();
         float* sp = a.s_part + (static_cast<size_t>(bh) * a.nsplit + split) * R * kD;
 #pragma unroll
-        for (int c0 = 0; c0 < R; c0 += 16) {
+        for (int c0 = 0; c0 < RH; c0 += 16) {
             uint32_t hi[32], lo[32];
-            tmem_ld32(t_s + lane_base + c0, hi);
+            tmem_ld32(t_s + lane_base + half * RH + c0, hi);
             tmem_ld_wait(hi);
-            tmem_ld32(t_s + lane_base + RP + c0, lo);
+            tmem_ld32(t_s + lane_base + RP + half * RH + c0, lo);
             tmem_ld_wait(lo);
-            const int cn = min(16, R - c0);
-            for (int i = 0; i < cn; ++i) sp[(c0 + i) * kD + tid] = __uint_as_float(hi[i]) + __uint_as_float(lo[i]);
+            const int cn = min(16, RH - c0);
+            for (int i = 0; i < cn; ++i)
+                sp[(half * RH + c0 + i) * kD + row] = __uint_as_float(hi[i]) + __uint_as_float(lo[i]);
         }
-        // z: sum the per-thread partials over the 128 threads (warp shuffles, then the 4 warp sums)
+        // z: sum the per-thread partials over the token rows (warp shuffles, then the 4 warps of a half)
 #pragma unroll
-        for (int c = 0; c < R; ++c) {
+        for (int c = 0; c < RH; ++c) {
             float v = zacc[c];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            zacc[c] = v;  // every lane of the warp holds the warp's sum
+            zacc[c] = v;
         }
-        float* zslots = reinterpret_cast<float*>(smem + lay.off_zred);  // [4][R/2]
+        float* zslots = reinterpret_cast<float*>(smem + lay.off_zred);  // [8 warps][RH]
+        if (lane == 0) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            if (lane == 0) {
-#pragma unroll
-                for (int c = 0; c < R / 2; ++c) zslots[warp * (R / 2) + c] = zacc[half * (R / 2) + c];
-            }
-            __syncthreads();
-            if (tid < R / 2)
-                a.z_part[(static_cast<size_t>(bh) * a.nsplit + split) * R + half * (R / 2) + tid] =
-                    ((zslots[tid] + zslots[R / 2 + tid]) + zslots[R + tid]) + zslots[3 * (R / 2) + tid];
-            __syncthreads();
+            for (int c = 0; c < RH; ++c) zslots[warp * RH + c] = zacc[c];
+        }
+        __syncthreads();
+        if (tid < R) {
+            const int hh = tid / RH, c = tid % RH;  // warps 4*hh .. 4*hh+3 hold half hh
+            const float* zs = zslots + (4 * hh) * RH + c;
+            a.z_part[(static_cast<size_t>(bh) * a.nsplit + split) * R + tid] =
+                ((zs[0] + zs[RH]) + zs[2 * RH]) + zs[3 * RH];
         }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
     }
     if (aborted && tid == 0) {
-        // let loads still in flight land before the shared memory is released (bounded, 10 ms each)
+        // let loads and products still in flight land before the memory is released (bounded, 10 ms each)
         volatile int no_abort = 0;
         for (int st = 0; st < kStages; ++st)
             if (n_load[st] > n_wait[st]) mbar_wait(bar_kv + st, n_wait[st] & 1, 10000000ull, &no_abort);
@@ -349,7 +364,7 @@ static cudaError_t lr_tc_launch(const CUtensorMap& tk, const CUtensorMap& tv, co
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int items = g.BH() * a.nsplit;
-    lowrank_sm100_kernel<R><<<items < sms ? items : sms, 128, sm, st>>>(tk, tv, a, g);
+    lowrank_sm100_kernel<R><<<items < sms ? items : sms, 256, sm, st>>>(tk, tv, a, g);
     return cudaGetLastError();
 }
 

@@ -36,11 +36,21 @@ cudaError_t launch_rope_table(double2* tab, int2* pairs, const RopeMeta& meta, i
     return cudaGetLastError();
 }
 
+// 16-byte read-once load that does not allocate in L1 (keeps L1 for the rotary table).
+__device__ __forceinline__ uint4 ldg_stream(const __nv_bfloat16* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
 // ------------------------------------------------------------------------------ rope_pool
-// One CTA per (query/key block, batch*head).  Thread t owns rotary pair j = t % (D/2) and walks the
-// block's tokens with stride 256/(D/2).  A warp touches 32 consecutive pairs (128 contiguous bytes)
-// of one token per load.  The rotation and the block sums are fp64 so the selection scores are
-// exact to ~1e-15 relative (the top-k decision is made on them).
+// One CTA per (query/key block, batch*head).  Thread t owns four consecutive rotary pairs (8 elements,
+// 16 bytes) j = 4*(t % (D/8)) .. +3 and walks the block's tokens with stride 256/(D/8); each access of
+// q, k, v and of the fp16 outputs is one 16-byte load or store, and the D/8 threads of a token cover
+// its 256-byte row.  The rotation and the block sums are fp64 so the selection scores are exact to
+// ~1e-15 relative (the top-k decision is made on them); the fp16 copies come from the same values.
 template <int D>
 __global__ void __launch_bounds__(256) rope_pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                         const __nv_bfloat16* __restrict__ k,
@@ -50,49 +60,93 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const __nv_bfloat16* __r
                                                         __half* __restrict__ qh, __half* __restrict__ kh,
                                                         __half* __restrict__ vh, double* __restrict__ qbar,
                                                         double* __restrict__ kbar, int* status) {
-    constexpr int P = D / 2;
-    constexpr int G = 256 / P;
-    __shared__ double red[G][4][P];
-    const int j = threadIdx.x % P, grp = threadIdx.x / P;
+    constexpr int Q4 = D / 8;          // threads per token row
+    constexpr int G = 256 / Q4;        // tokens in flight
+    __shared__ double red[G][4][4 * Q4];  // [group][q0,q1,k0,k1][pair]
+    const int quad = threadIdx.x % Q4, grp = threadIdx.x / Q4;
     const int alpha = blockIdx.x, bh = blockIdx.y;
     const int b = bh / g.Hh, h = bh % g.Hh;
     const int n0 = alpha * g.block;
-    const int2 pinfo = pairs[j];
-    const int axis = pinfo.x;
-    const int toff = pinfo.y;
-    double sq0 = 0.0, sq1 = 0.0, sk0 = 0.0, sk1 = 0.0;
+    int axis[4], toff[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int2 pi = pairs[4 * quad + u];
+        axis[u] = pi.x;
+        toff[u] = pi.y;
+    }
+    double sq[4][2], sk[4][2];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) sq[u][0] = sq[u][1] = sk[u][0] = sk[u][1] = 0.0;
     bool bad = false;
+    const int HW = g.H * g.W;
+    const size_t row_stride = static_cast<size_t>(g.Hh) * D;  // elements between consecutive tokens
+    const size_t src0 = ((static_cast<size_t>(b) * g.L + n0) * g.Hh + h) * D + 8 * quad;
+    // software pipeline: the next token's q, k, v are in flight while this one is rotated
+    uint4 qn = make_uint4(0u, 0u, 0u, 0u), kn = qn, vn = qn;
+    if (grp < g.block && n0 + grp < g.L) {
+        const size_t src = src0 + static_cast<size_t>(grp) * row_stride;
+        qn = ldg_stream(q + src); kn = ldg_stream(k + src); vn = ldg_stream(v + src);
+    }
     for (int i = grp; i < g.block; i += G) {
         const int n = n0 + i;
-        const size_t dst = (static_cast<size_t>(bh) * g.Lp + n) * D + 2 * j;
+        const uint4 qr = qn, kr = kn, vr = vn;
+        if (i + G < g.block && n + G < g.L) {
+            const size_t src = src0 + static_cast<size_t>(i + G) * row_stride;
+            qn = ldg_stream(q + src); kn = ldg_stream(k + src); vn = ldg_stream(v + src);
+        }
+        const size_t dst = (static_cast<size_t>(bh) * g.Lp + n) * D + 8 * quad;
         if (n < g.L) {
-            const double2 cs = tab[toff + token_axis_pos(n, axis, g.H, g.W)];
-            const size_t src = ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D + 2 * j;
-            const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + src));
-            const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + src));
-            const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + src));
-            const double qy0 = static_cast<double>(qf.x) * cs.x - static_cast<double>(qf.y) * cs.y;
-            const double qy1 = static_cast<double>(qf.x) * cs.y + static_cast<double>(qf.y) * cs.x;
-            const double ky0 = static_cast<double>(kf.x) * cs.x - static_cast<double>(kf.y) * cs.y;
-            const double ky1 = static_cast<double>(kf.x) * cs.y + static_cast<double>(kf.y) * cs.x;
-            sq0 += qy0; sq1 += qy1; sk0 += ky0; sk1 += ky1;
-            const float m = fmaxf(fmaxf(fabsf(static_cast<float>(qy0)), fabsf(static_cast<float>(qy1))),
-                                  fmaxf(fmaxf(fabsf(static_cast<float>(ky0)), fabsf(static_cast<float>(ky1))),
-                                        fmaxf(fabsf(vf.x), fabsf(vf.y))));
+            const int pos3[3] = {n / HW, (n / g.W) % g.H, n % g.W};
+            const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qr);
+            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
+            uint4 qo, ko, vo;
+            uint32_t* qo2 = reinterpret_cast<uint32_t*>(&qo);
+            uint32_t* ko2 = reinterpret_cast<uint32_t*>(&ko);
+            uint32_t* vo2 = reinterpret_cast<uint32_t*>(&vo);
+            float m = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const double2 cs = __ldg(tab + toff[u] + pos3[axis[u]]);
+                const float2 qf = __bfloat1622float2(q2[u]);
+                const float2 kf = __bfloat1622float2(k2[u]);
+                const float2 vf = __bfloat1622float2(v2[u]);
+                const double qy0 = static_cast<double>(qf.x) * cs.x - static_cast<double>(qf.y) * cs.y;
+                const double qy1 = static_cast<double>(qf.x) * cs.y + static_cast<double>(qf.y) * cs.x;
+                const double ky0 = static_cast<double>(kf.x) * cs.x - static_cast<double>(kf.y) * cs.y;
+                const double ky1 = static_cast<double>(kf.x) * cs.y + static_cast<double>(kf.y) * cs.x;
+                sq[u][0] += qy0; sq[u][1] += qy1; sk[u][0] += ky0; sk[u][1] += ky1;
+                const float a0 = static_cast<float>(qy0), a1 = static_cast<float>(qy1);
+                const float c0 = static_cast<float>(ky0), c1 = static_cast<float>(ky1);
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(a0), fabsf(a1)), fmaxf(fmaxf(fabsf(c0), fabsf(c1)),
+                                                                     fmaxf(fabsf(vf.x), fabsf(vf.y)))));
+                const __half2 hq = __floats2half2_rn(a0, a1), hk = __floats2half2_rn(c0, c1),
+                              hv = __floats2half2_rn(vf.x, vf.y);
+                qo2[u] = *reinterpret_cast<const uint32_t*>(&hq);
+                ko2[u] = *reinterpret_cast<const uint32_t*>(&hk);
+                vo2[u] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
             bad |= !(m <= 65504.0f);
-            *reinterpret_cast<__half2*>(qh + dst) = __floats2half2_rn(static_cast<float>(qy0), static_cast<float>(qy1));
-            *reinterpret_cast<__half2*>(kh + dst) = __floats2half2_rn(static_cast<float>(ky0), static_cast<float>(ky1));
-            *reinterpret_cast<__half2*>(vh + dst) = __floats2half2_rn(vf.x, vf.y);
+            *reinterpret_cast<uint4*>(qh + dst) = qo;
+            *reinterpret_cast<uint4*>(kh + dst) = ko;
+            *reinterpret_cast<uint4*>(vh + dst) = vo;
         } else {
-            const __half2 z2 = __floats2half2_rn(0.f, 0.f);
-            *reinterpret_cast<__half2*>(qh + dst) = z2;
-            *reinterpret_cast<__half2*>(kh + dst) = z2;
-            *reinterpret_cast<__half2*>(vh + dst) = z2;
+            const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(qh + dst) = z4;
+            *reinterpret_cast<uint4*>(kh + dst) = z4;
+            *reinterpret_cast<uint4*>(vh + dst) = z4;
         }
     }
-    red[grp][0][j] = sq0; red[grp][1][j] = sq1; red[grp][2][j] = sk0; red[grp][3][j] = sk1;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int j = 4 * quad + u;
+        red[grp][0][j] = sq[u][0]; red[grp][1][j] = sq[u][1];
+        red[grp][2][j] = sk[u][0]; red[grp][3][j] = sk[u][1];
+    }
     __syncthreads();
-    if (grp == 0) {
+    // thread t < D/2 finishes pair t: fixed-order sum over the token groups
+    if (threadIdx.x < D / 2) {
+        const int j = threadIdx.x;
         double a0 = 0.0, a1 = 0.0, c0 = 0.0, c1 = 0.0;
         for (int u = 0; u < G; ++u) { a0 += red[u][0][j]; a1 += red[u][1][j]; c0 += red[u][2][j]; c1 += red[u][3][j]; }
         const int cnt = min(g.block, g.L - n0);
@@ -126,21 +180,29 @@ __device__ __forceinline__ double key_value(uint64_t k) {
     return __longlong_as_double(static_cast<long long>(u));
 }
 
-constexpr int kSelRows = 8;  // query blocks per CTA (one warp each in the selection phase)
+constexpr int kSelRows = 8;   // query blocks per CTA (one warp each in the selection phase)
 
-// One CTA per (8 query blocks, batch*head).  Phase 1: fp64 dot products of the 8 qbar rows with all
-// kbar rows, staged 32 key blocks at a time through shared memory.  Phase 2: warp w selects row w's
-// top-k by an 8-pass radix select on the order-preserving 64-bit keys, then writes the selected block
-// indices in ascending order (ties at the threshold resolved to the lowest indices) and the tie flag.
+// D (8x8, fp64) += A (8x4, row-major) * B (4x8, col-major) on the fp64 tensor pipe.  Fragments: lane l
+// holds A[l/4][l%4], B[l%4][l/4], and D[l/4][2(l%4)], D[l/4][2(l%4)+1].
+__device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d0), "+d"(d1)
+                 : "d"(a), "d"(b));
+}
+
+// One CTA per (8 query blocks, batch*head).  Phase 1: the 8 x nb block of fp64 scores qbar kbar^T on
+// the fp64 tensor pipe (m8n8k4): every warp keeps the 8 qbar rows as A fragments in registers and
+// sweeps its share of 8-key tiles, streaming the kbar fragments from L2.  Phase 2: warp w selects row
+// w's top-k by an 8-pass radix select on the order-preserving 64-bit keys, then writes the selected
+// block indices in ascending order (ties at the threshold resolved to the lowest indices) and the tie
+// flag.
 template <int D>
 __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ qbar,
                                                      const double* __restrict__ kbar, Geom g,
                                                      int32_t* __restrict__ idx, uint8_t* __restrict__ tie) {
     extern __shared__ __align__(16) unsigned char sm_raw[];
-    double* qrow = reinterpret_cast<double*>(sm_raw);          // [8][D]
-    double* kch = qrow + kSelRows * D;                          // [32][D+1]
-    double* scores = kch + 32 * (D + 1);                        // [8][nb]
-    int* hist = reinterpret_cast<int*>(scores + kSelRows * g.nb);  // [8][256]
+    double* scores = reinterpret_cast<double*>(sm_raw);                 // [8][nb]
+    int* hist = reinterpret_cast<int*>(scores + kSelRows * g.nb);      // [8][256]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bh = blockIdx.y;
     const int a0 = blockIdx.x * kSelRows;
@@ -148,26 +210,24 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
     const double* qb = qbar + static_cast<size_t>(bh) * nb * D;
     const double* kb = kbar + static_cast<size_t>(bh) * nb * D;
 
-    for (int e = tid; e < kSelRows * D; e += 256) {
-        const int r = e / D;
-        qrow[e] = (a0 + r < nb) ? qb[static_cast<size_t>(a0 + r) * D + (e % D)] : 0.0;
+    // A fragments: row l/4 of the 8 query blocks, dims 4*kk + l%4 for the D/4 k-steps
+    double af[D / 4];
+    {
+        const int ar = a0 + (lane >> 2);
+#pragma unroll
+        for (int kk = 0; kk < D / 4; ++kk)
+            af[kk] = ar < nb ? __ldg(qb + static_cast<size_t>(ar) * D + 4 * kk + (lane & 3)) : 0.0;
     }
-    for (int c0 = 0; c0 < nb; c0 += 32) {
-        __syncthreads();
-        for (int e = tid; e < 32 * D; e += 256) {
-            const int i = e / D, d = e % D;
-            kch[i * (D + 1) + d] = (c0 + i < nb) ? kb[static_cast<size_t>(c0 + i) * D + d] : 0.0;
-        }
-        __syncthreads();
-        const int r = tid >> 5, c = tid & 31;
-        if (c0 + c < nb) {
-            const double* qr = qrow + r * D;
-            const double* kr = kch + c * (D + 1);
-            double acc = 0.0;
-#pragma unroll 8
-            for (int d = 0; d < D; ++d) acc = fma(qr[d], kr[d], acc);
-            scores[r * nb + c0 + c] = acc;
-        }
+    const int ntile = (nb + 7) / 8;
+    for (int t = warp; t < ntile; t += 8) {
+        const int key = 8 * t + (lane >> 2);  // B fragment: key l/4 of the tile, dims 4*kk + l%4
+        const double* kr = kb + static_cast<size_t>(key < nb ? key : nb - 1) * D + (lane & 3);
+        double d0 = 0.0, d1 = 0.0;
+#pragma unroll
+        for (int kk = 0; kk < D / 4; ++kk) dmma_8x8x4(d0, d1, af[kk], __ldg(kr + 4 * kk));
+        const int r = lane >> 2, c = 8 * t + 2 * (lane & 3);
+        if (c < nb) scores[r * nb + c] = d0;
+        if (c + 1 < nb) scores[r * nb + c + 1] = d1;
     }
     __syncthreads();
 
@@ -253,8 +313,7 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
 }
 
 static size_t select_smem(const Geom& g) {
-    return sizeof(double) * (kSelRows * g.D + 32 * (g.D + 1) + static_cast<size_t>(kSelRows) * g.nb) +
-           sizeof(int) * kSelRows * 256;
+    return sizeof(double) * static_cast<size_t>(kSelRows) * g.nb + sizeof(int) * kSelRows * 256;
 }
 
 cudaError_t launch_select(const double* qbar, const double* kbar, const Geom& g, int32_t* idx, uint8_t* tie,

@@ -38,7 +38,7 @@ class _Problem(ctypes.Structure):
                 ("block", ctypes.c_int64), ("keep_frac", ctypes.c_double), ("rank", ctypes.c_int64),
                 ("theta", ctypes.c_double), ("out_dtype", ctypes.c_int32), ("branches", ctypes.c_int32),
                 ("pos_offset", ctypes.c_int64 * 3), ("rope_split", ctypes.c_int64 * 3),
-                ("wait_timeout_ns", ctypes.c_uint64), ("attn_events", ctypes.c_void_p * 2)]
+                ("wait_timeout_ns", ctypes.c_uint64), ("stage_events", ctypes.c_void_p * 7)]
 
 
 class _Layout(ctypes.Structure):
@@ -110,7 +110,7 @@ class Problem:
     pos_offset: tuple = (0, 0, 0)
     rope_split: tuple = (0, 0, 0)
     wait_timeout_ns: int = 2_000_000_000
-    attn_events: tuple = (None, None)  # raw cudaEvent_t handles (ints) or None
+    stage_events: tuple = (None,) * 7  # raw cudaEvent_t handles (ints) or None, see slra_problem
 
     @property
     def L(self) -> int:
@@ -130,8 +130,8 @@ class Problem:
         p.pos_offset[:] = [int(x) for x in self.pos_offset]
         p.rope_split[:] = [int(x) for x in self.rope_split]
         p.wait_timeout_ns = int(self.wait_timeout_ns)
-        p.attn_events[0] = self.attn_events[0]
-        p.attn_events[1] = self.attn_events[1]
+        for i, e in enumerate(self.stage_events):
+            p.stage_events[i] = e
         return p
 
 
