@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 
 from sparse_rank_hybrid_b200 import flops as F  # noqa: E402
 from sparse_rank_hybrid_b200 import inputs as I  # noqa: E402
+from sparse_rank_hybrid_b200 import replicas  # noqa: E402
 from sparse_rank_hybrid_b200 import workloads as WL  # noqa: E402
 
 METRIC = "ms/attn call & effective TFLOP/s at L=75600, 40 heads, 90% sparsity; %roofline"
@@ -172,7 +173,7 @@ def run_reference(args, w, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded clustered-Gaussian bf16 q/k/v, A ~ N(0, 1/d_h))",
-            "config": {"workload": w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
+            "config": {"workload": base_w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
                        "block": w.block, "keep_frac": w.keep_frac},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
@@ -193,6 +194,8 @@ def run_ours(args, w, rank, world, local_rank):
         oracle.build()  # compile the CPU baseline before any GPU work
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    base_w = w
+    w = replicas.replica_workload(base_w, rank)  # each rank: its own independent problem
     x = I.make_inputs(w)
     q, k, v, A = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v", "A"))
     stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
@@ -243,12 +246,9 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    tot_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([tot_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = replicas.max_over_ranks(sum(step_ms), dev)
     ms_per_step = tot_ms / args.steps
+    job_flops = replicas.sum_over_ranks(f_total, dev)
     status = slra.device_status(ws)
     if status != slra.OK:
         raise RuntimeError(f"device status after timing: {slra.status_string(status)}")
@@ -267,11 +267,7 @@ def run_ours(args, w, rank, world, local_rank):
         slra.attn_fwd_host(prob, host["q"], host["k"], host["v"], host["A"], out_h, io, ws)
         e_ev[i][1].record(stream)
         torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e_ev) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = replicas.max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev) / e2e_steps, dev)
     h2d = sum(int(host[n].numel()) * 2 for n in ("q", "k", "v", "A"))
     d2h = int(out_h.numel()) * 4
 
@@ -284,13 +280,13 @@ def run_ours(args, w, rank, world, local_rank):
     traffic = load_traffic(w.name)
     bytes_min = F.io_bytes(w.batch, w.L, w.heads, w.head_dim, w.rank, 4)
     t_roof = max(f_sparse / (tf_sust * 1e12), bytes_min / (hbm * 1e9))
-    cpu_v, cpu_desc, cpu_threads, _ = oracle_sample(w, x)
+    cpu_v, cpu_desc, cpu_threads, _ = oracle_sample(w, x)  # rank 0 runs the workload itself
     line = {
-        "metric": METRIC, "value": f_total * world / (ms_per_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "metric": METRIC, "value": replicas.job_throughput(job_flops, ms_per_step), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16 tensor-core operands, fp32 accumulate, fp64 selection",
         "data": "synthetic (seeded clustered-Gaussian bf16 q/k/v, A ~ N(0, 1/d_h)); inputs resident in HBM",
-        "config": {"workload": w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
+        "config": {"workload": base_w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
                    "block": w.block, "keep_frac": w.keep_frac, "keep_blocks": int(idx.shape[-1]),
                    "out_dtype": "f32", "l2": "flushed between timed steps (512 MB write)",
                    "parallelism": f"replica x{world} (independent problems, no collective)"},
@@ -300,7 +296,7 @@ def run_ours(args, w, rank, world, local_rank):
                      "peak_source": f"{src} sustained bf16 (same rate as f16)", "attn_ms": attn_avg},
         "call_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_per_step,
                           "note": "max(kept FLOPs / sustained tensor peak, min bytes / HBM peak) vs ms_per_step"},
-        "e2e": {"value": f_total * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": replicas.job_throughput(job_flops, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "kernel_ms": dict(zip(("rope_table", "rope_pool", "select", "lowrank_partial", "lowrank_reduce",
                                "attention"), (round(x, 4) for x in stage_avg))),
@@ -313,13 +309,17 @@ def run_ours(args, w, rank, world, local_rank):
 
 
 def load_traffic(workload: str):
-    """DRAM bytes per launch of the attention kernel from the committed ncu summary, if current."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of the attention kernel from the committed ncu capture, or None when there
+    is none for this workload or the kernel source has changed since it was taken."""
+    import hashlib
     try:
-        with open(path) as f:
-            t = json.load(f)
-        return t.get(workload)
-    except (OSError, ValueError):
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f).get(workload)
+        src = os.path.join(ROOT, "sparse_rank_hybrid_b200", "csrc", "attn_sm100.cu")
+        with open(src, "rb") as f:
+            current = hashlib.sha256(f.read()).hexdigest()
+        return t["bytes"] if t and t.get("source_sha256") == current else None
+    except (OSError, ValueError, KeyError, TypeError):
         return None
 
 

@@ -78,6 +78,12 @@ typedef enum slra_out_dtype { SLRA_OUT_F32 = 0, SLRA_OUT_BF16 = 1 } slra_out_dty
 /* Which branches contribute to `out` (default both). */
 enum { SLRA_BRANCH_SPARSE = 1, SLRA_BRANCH_LOWRANK = 2, SLRA_BRANCH_BOTH = 3 };
 
+/* Test hooks (slra_problem.debug_flags).  SLRA_DEBUG_UNSATISFIED_WAIT makes every CTA of the attention
+ * kernel first wait on a barrier that nothing signals, so the bounded-wait path (timeout recorded in
+ * the status word, the CTA returns without issuing work) can be exercised without faulting or hanging
+ * the GPU.  Use a small wait_timeout_ns with it. */
+enum { SLRA_DEBUG_UNSATISFIED_WAIT = 1 };
+
 /*
  * Problem description.  Fill it with slra_problem_init, then adjust optional fields.
  *   batch, heads, head_dim  B, Hh, D.  D in {64, 128}.
@@ -92,6 +98,7 @@ enum { SLRA_BRANCH_SPARSE = 1, SLRA_BRANCH_LOWRANK = 2, SLRA_BRANCH_BOTH = 3 };
  *                           result independent of it, which the tests use).
  *   rope_split              rotary pairs per (t, h, w); all zero = default split described above.
  *   wait_timeout_ns         bound of every wait inside the kernels (default 2e9 ns = 2 s).
+ *   debug_flags             SLRA_DEBUG_* test hooks (default 0).
  *   stage_events            optional cudaEvent_t handles (NULL entries are skipped), recorded on
  *                           `stream` between the library's launches so a caller can time each
  *                           kernel alone: [0] before the first launch, [1] after the rotary tables,
@@ -112,6 +119,7 @@ typedef struct slra_problem {
     int64_t pos_offset[3];
     int64_t rope_split[3];
     uint64_t wait_timeout_ns;
+    uint32_t debug_flags;
     void* stage_events[7];
 } slra_problem;
 

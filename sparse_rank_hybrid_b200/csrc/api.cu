@@ -370,6 +370,7 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
     a.out_bf16 = p->out_dtype == SLRA_OUT_BF16 ? 1 : 0;
     a.status = w.status;
     a.timeout_ns = p->wait_timeout_ns ? p->wait_timeout_ns : 2000000000ull;
+    a.debug_unsatisfied_wait = (p->debug_flags & SLRA_DEBUG_UNSATISFIED_WAIT) ? 1 : 0;
     if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
     return mark(p, 6, st);
 }

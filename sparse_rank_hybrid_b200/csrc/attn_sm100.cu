@@ -37,7 +37,7 @@ struct AttnLayout {
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kKVBytes;
-    static constexpr int kOffBar = kOffV + kKVBytes;  // 7 mbarriers
+    static constexpr int kOffBar = kOffV + kKVBytes;  // 8 mbarriers
     static constexpr int kOffMisc = kOffBar + 64;     // tmem base, abort flag
     static constexpr int kBytes = kOffMisc + 64;
 };
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int32_t* my_idx = a.idx + (static_cast<size_t>(bh) * g.nb + alpha) * (keep > 0 ? g.keep : 0);
 
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -175,8 +175,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     int n_q_issued = 0, n_q_done = 0, n_k_issued = 0, n_k_done = 0, n_v_issued = 0, n_v_done = 0;
     int n_s_issued = 0, n_s_done = 0, n_o_issued = 0, n_o_done = 0;
 
+    // Test hook: wait on a barrier that nothing arrives at (bars[7]); the bounded wait runs out, records
+    // a timeout and every thread sees the abort flag before any copy or product has been issued.
+    if (a.debug_unsatisfied_wait && tid == 0 && !mbar_wait(bars + 7, 0, tmo, abort_flag)) fail();
+    __syncthreads();
+
     // ------------------------------------------------------------------ prologue: Q, K0, V0, S0
-    if (keep > 0 && tid == 0) {
+    if (keep > 0 && tid == 0 && !*abort_flag) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);

@@ -86,6 +86,7 @@ struct AttnArgs {
     int out_bf16;
     int* status;
     unsigned long long timeout_ns;
+    int debug_unsatisfied_wait;  // test hook: wait on a barrier nothing signals before any work
 };
 cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st);
 size_t attn_smem_bytes(const Geom& g);

@@ -19,6 +19,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DE
     ERR_NO_DEVICE, ERR_SCRATCH_LIMIT = range(1, 10)
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
+DEBUG_UNSATISFIED_WAIT = 1
 
 # Every symbol include/slra.h declares.
 EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_validate", "slra_keep_count",
@@ -38,7 +39,8 @@ class _Problem(ctypes.Structure):
                 ("block", ctypes.c_int64), ("keep_frac", ctypes.c_double), ("rank", ctypes.c_int64),
                 ("theta", ctypes.c_double), ("out_dtype", ctypes.c_int32), ("branches", ctypes.c_int32),
                 ("pos_offset", ctypes.c_int64 * 3), ("rope_split", ctypes.c_int64 * 3),
-                ("wait_timeout_ns", ctypes.c_uint64), ("stage_events", ctypes.c_void_p * 7)]
+                ("wait_timeout_ns", ctypes.c_uint64), ("debug_flags", ctypes.c_uint32),
+                ("stage_events", ctypes.c_void_p * 7)]
 
 
 class _Layout(ctypes.Structure):
@@ -110,6 +112,7 @@ class Problem:
     pos_offset: tuple = (0, 0, 0)
     rope_split: tuple = (0, 0, 0)
     wait_timeout_ns: int = 2_000_000_000
+    debug_flags: int = 0
     stage_events: tuple = (None,) * 7  # raw cudaEvent_t handles (ints) or None, see slra_problem
 
     @property
@@ -130,6 +133,7 @@ class Problem:
         p.pos_offset[:] = [int(x) for x in self.pos_offset]
         p.rope_split[:] = [int(x) for x in self.rope_split]
         p.wait_timeout_ns = int(self.wait_timeout_ns)
+        p.debug_flags = int(self.debug_flags)
         for i, e in enumerate(self.stage_events):
             p.stage_events[i] = e
         return p

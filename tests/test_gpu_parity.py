@@ -156,3 +156,18 @@ def test_sweep_points(name):
     w = W.by_name(name)
     heads = [(0, 3)]
     _case(w, heads=heads, qblocks=[0, w.nb - 1])
+
+
+def test_bounded_wait_timeout_is_reported_and_context_stays_usable():
+    """A wait on a barrier that nothing signals runs out after its bound, the kernel records a timeout
+    in the status word and returns without issuing work; the next call on the same context is exact."""
+    w = W.TINY
+    x = I.make_inputs(w)
+    q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
+    p = slra.Problem.from_workload(w, debug_flags=slra.DEBUG_UNSATISFIED_WAIT, wait_timeout_ns=1_000_000)
+    _, ws = slra.attn_fwd(p, q, k, v, A)
+    assert slra.device_status(ws) == slra.ERR_DEVICE_TIMEOUT
+    assert slra.device_status(ws) == slra.OK
+    st = parity.compare(slra.Problem.from_workload(w), x, parity.run_gpu(slra.Problem.from_workload(w), x),
+                        label="tiny-after-timeout")
+    _log(st)
