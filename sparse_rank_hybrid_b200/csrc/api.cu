@@ -345,7 +345,8 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
     const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
     if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) || !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
         !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
-        !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, 128))
+        !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, 128) ||
+        !make_map_out(&maps.out, out, g.B, g.L, g.Hh, g.D, p->out_dtype == SLRA_OUT_F32))
         return SLRA_ERR_CUDA;
 
     if ((s = begin(p, d, w, st)) != SLRA_OK) return s;

@@ -14,7 +14,7 @@
 //         TMEM columns of S;
 //   MMA   O += P v        (A operand = P from TMEM, B = v tile MN-major; M=128, N=D, K=block).
 // Epilogue: the low-rank readout (head_dim 128: on the tensor cores, accumulated into O; head_dim 64: on
-// the CUDA cores in fp32), then O / l stored as fp32 or bf16.
+// the CUDA cores in fp32), then O / l staged in shared memory and written by TMA stores (fp32 or bf16).
 //
 // All waits are bounded (see sm100.cuh); a wait that runs out records a timeout in the status word
 // and the CTA leaves the loop, releases its tensor memory and returns.
@@ -37,8 +37,8 @@ struct AttnLayout {
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kKVBytes;
-    static constexpr int kOffBar = kOffV + kKVBytes;  // 8 mbarriers
-    static constexpr int kOffMisc = kOffBar + 64;     // tmem base, abort flag
+    static constexpr int kOffBar = kOffV + kKVBytes;  // 16 mbarriers
+    static constexpr int kOffMisc = kOffBar + 128;    // tmem base, abort flag
     static constexpr int kBytes = kOffMisc + 64;
 };
 
@@ -103,7 +103,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qraw,
-                      AttnArgs a, Geom g) {
+                      const __grid_constant__ CUtensorMap tm_out, AttnArgs a, Geom g) {
     using Lay = AttnLayout<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t* bar_v = bars + 2;
     uint64_t* bar_s = bars + 3;
     uint64_t* bar_o = bars + 4;
+    uint64_t* bar_pv = bars + 8;   // P.V done (frees the v tile early)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
 
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int32_t* my_idx = a.idx + (static_cast<size_t>(bh) * g.nb + alpha) * (keep > 0 ? g.keep : 0);
 
     if (tid == 0) {
-        for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 10; ++i) mbar_init(bars + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -174,6 +175,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     // what is still in flight before it releases shared and tensor memory.
     int n_q_issued = 0, n_q_done = 0, n_k_issued = 0, n_k_done = 0, n_v_issued = 0, n_v_done = 0;
     int n_s_issued = 0, n_s_done = 0, n_o_issued = 0, n_o_done = 0;
+    int n_pv_issued = 0, n_pv_done = 0;
+    // epilogue barrier bookkeeping (thread 0 for the loads; every thread for the products)
+    int n_eld_issued = 0, n_eld = 0, n_emm_issued = 0, n_emm = 0, n_ez_issued = 0, n_ez = 0;
+    uint64_t* bar_eld = bars + 5;  // epilogue: raw query tile + A^T image (one phase)
+    uint64_t* bar_ez = bars + 9;   // epilogue: S image of each 64-feature chunk (one phase per chunk)
+    uint64_t* bar_emm = bars + 6;  // epilogue products
+    // The low-rank readout's raw query tile and A^T image are loaded during the last key block, into
+    // the q and k tiles (free once the last S product is done).
+    const bool prefetch_epi = (D == 128) && a.lowrank && keep > 0;
+    auto issue_epilogue_prefetch = [&]() {
+        mbar_expect_tx(bar_eld, 32768 + g.R * 256);
+        tma_load_4d(smem, &tm_qraw, bar_eld, 0, h, alpha * blk, b);
+        tma_load_4d(smem + 16384, &tm_qraw, bar_eld, 64, h, alpha * blk, b);
+        bulk_load(smem + 32768, a.at_img, g.R * 256, bar_eld);
+        ++n_eld_issued;
+    };
 
     // Test hook: wait on a barrier that nothing arrives at (bars[7]); the bounded wait runs out, records
     // a timeout and every thread sees the abort flag before any copy or product has been issued.
@@ -220,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             ++n_s_done;
             // S_j has finished reading the k tile and (issued before it) P.V_{j-1} the v tile.
             if (j + 1 < keep) { load_kv(bar_k, sk, &tm_k, my_idx[j + 1]); ++n_k_issued; }
-            if (j > 0) { load_kv(bar_v, sv, &tm_v, my_idx[j]); ++n_v_issued; }
+            if (j == keep - 1 && prefetch_epi) issue_epilogue_prefetch();  // q and k tiles are free now
         }
         // ---- softmax of row (warp*32 + lane); O is stable (P.V_{j-1} completed before S_j)
         uint32_t sr[4][32];
@@ -315,11 +332,20 @@ __global__ void __launch_bounds__(kThreads, 2)
                         const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, static_cast<uint32_t>(blk) * 128, 1024);
                         umma_ts(tO, tS + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                     }
+                    umma_commit(bar_pv);  // lets the next v tile load as soon as this product is done
+                    ++n_pv_issued;
                     if (j + 1 < keep) {
                         if (mbar_wait(bar_k, (j + 1) & 1, tmo, abort_flag)) {
                             ++n_k_done;
                             issue_s();  // commits bar_s, which also covers this P.V
                             ++n_s_issued;
+                            if (mbar_wait(bar_pv, n_pv_done & 1, tmo, abort_flag)) {
+                                ++n_pv_done;
+                                load_kv(bar_v, sv, &tm_v, my_idx[j + 1]);
+                                ++n_v_issued;
+                            } else {
+                                fail();
+                            }
                         } else {
                             umma_commit(bar_o);
                             ++n_o_issued;
@@ -349,9 +375,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     const bool row_valid = (i_row < blk) && (n < g.L) && !aborted;
     float inv_l = (keep > 0 && l_run > 0.f) ? 1.f / l_run : 0.f;
     bool o_live = keep > 0;  // O holds the sparse branch (and, below, the low-rank readout)
-    int n_eld_issued = 0, n_eld = 0, n_emm_issued = 0, n_emm = 0;  // epilogue barrier bookkeeping
-    uint64_t* bar_eld = bars + 5;  // epilogue loads
-    uint64_t* bar_emm = bars + 6;  // epilogue products
     if constexpr (D == 128) {
         if (a.lowrank && !aborted) {
             // Low-rank readout on the tensor cores, accumulated straight into O (so out = O / l):
@@ -363,19 +386,21 @@ __global__ void __launch_bounds__(kThreads, 2)
             uint8_t* X = smem;           // raw query tile, then each chunk's psi operand [128][3*rc]
             uint8_t* Y = smem + 32768;   // A^T image [R][128]
             uint8_t* Z = smem + 49152;   // S image of the current chunk [128][3*rc]
-            const bool z_early = R <= 64;  // Y and Z do not overlap: load chunk 0's S image up front
+            const bool z_early = R <= 64;  // Y and Z do not overlap: chunk 0's S image loads right away
             auto sb_bytes = [&](int ch) -> uint32_t {
                 const int rc = min(64, R - 64 * ch);
                 return static_cast<uint32_t>((3 * rc + 63) / 64) * (D * 128);
             };
             const uint8_t* sb_head = a.sb_img + static_cast<size_t>(bh) * nch * kSbChunkBytes;
+            // bar_eld: raw query tile + A^T image (prefetched during the last key block when there is
+            // one); bar_ez: the S image of each chunk in turn
             if (tid == 0) {
-                mbar_expect_tx(bar_eld, 32768 + R * 256 + (z_early ? sb_bytes(0) : 0));
-                tma_load_4d(X, &tm_qraw, bar_eld, 0, h, alpha * blk, b);
-                tma_load_4d(X + 16384, &tm_qraw, bar_eld, 64, h, alpha * blk, b);
-                bulk_load(Y, a.at_img, R * 256, bar_eld);
-                if (z_early) bulk_load(Z, sb_head, sb_bytes(0), bar_eld);
-                ++n_eld_issued;
+                if (!prefetch_epi) issue_epilogue_prefetch();
+                if (z_early) {  // the v tile is free (the last P.V is done)
+                    mbar_expect_tx(bar_ez, sb_bytes(0));
+                    bulk_load(Z, sb_head, sb_bytes(0), bar_ez);
+                    ++n_ez_issued;
+                }
                 if (mbar_wait(bar_eld, n_eld & 1, tmo, abort_flag)) {
                     ++n_eld;
                     tc_fence_after();
@@ -399,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ++n_emm;
                 tc_fence_after();
                 if (!z_early && tid == 0) {  // the feature product has finished with Y
-                    mbar_expect_tx(bar_eld, sb_bytes(0));
-                    bulk_load(Z, sb_head, sb_bytes(0), bar_eld);
-                    ++n_eld_issued;
+                    mbar_expect_tx(bar_ez, sb_bytes(0));
+                    bulk_load(Z, sb_head, sb_bytes(0), bar_ez);
+                    ++n_ez_issued;
                 }
                 // phi . z over all R features (unrotated features in the denominator)
                 const float* zh = a.z + static_cast<size_t>(bh) * R;
@@ -432,9 +457,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                         ++n_emm;
                         tc_fence_after();
                         if (tid == 0) {
-                            mbar_expect_tx(bar_eld, sb_bytes(ch));
-                            bulk_load(Z, sb_head + static_cast<size_t>(ch) * kSbChunkBytes, sb_bytes(ch), bar_eld);
-                            ++n_eld_issued;
+                            mbar_expect_tx(bar_ez, sb_bytes(ch));
+                            bulk_load(Z, sb_head + static_cast<size_t>(ch) * kSbChunkBytes, sb_bytes(ch), bar_ez);
+                            ++n_ez_issued;
                         }
                     }
                     uint32_t v[2][32];
@@ -465,10 +490,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tc_fence_before();
                     __syncthreads();
                     if (tid == 0 && !*abort_flag) {
-                        // chunk 0's S image came with the first load phase when it was loaded up front
-                        const bool z_landed = (ch == 0 && z_early);
-                        if (z_landed || mbar_wait(bar_eld, n_eld & 1, tmo, abort_flag)) {
-                            if (!z_landed) ++n_eld;
+                        if (mbar_wait(bar_ez, n_ez & 1, tmo, abort_flag)) {
+                            ++n_ez;
                             tc_fence_after();
                             const uint32_t idesc_lr = idesc_bf16_f32(128, D);
                             for (int kk = 0; kk < (3 * rc) / 16; ++kk) {
@@ -558,10 +581,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
     }
+    // ---- out = O / l (+ the CUDA-core readout for head_dim 64): each thread writes its row into a
+    //      128-B-swizzled staging tile (conflict-free 16-byte stores), then 64-row TMA stores write it
+    //      out; tokens past L are clipped by the tensor map and a 64-token block's second half is skipped.
     const bool aborted2 = *abort_flag != 0;
-    const bool warp_has_rows = (warp * 32 < blk) && (alpha * blk + warp * 32 < g.L) && !aborted2;
-    if (warp_has_rows) {
-        const size_t obase = ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;
+    if (!aborted2) {
+        __syncthreads();  // every product that read the tile buffers has completed
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -572,36 +597,48 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = 0u;
             }
-            if (row_valid) {
-                float r[32];
+            float r[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    float x = __uint_as_float(o[i]) * inv_l;
-                    if constexpr (D != 128) x += acc[c * 32 + i] * inv_den;
-                    r[i] = x;
+            for (int i = 0; i < 32; ++i) {
+                float x = __uint_as_float(o[i]) * inv_l;
+                if constexpr (D != 128) x += acc[c * 32 + i] * inv_den;
+                r[i] = x;
+            }
+            if (a.out_bf16) {  // boxes of 64 columns
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int col = c * 32 + 8 * u;
+                    uint4 pk;
+                    __nv_bfloat162 t0 = __floats2bfloat162_rn(r[8 * u], r[8 * u + 1]);
+                    __nv_bfloat162 t1 = __floats2bfloat162_rn(r[8 * u + 2], r[8 * u + 3]);
+                    __nv_bfloat162 t2 = __floats2bfloat162_rn(r[8 * u + 4], r[8 * u + 5]);
+                    __nv_bfloat162 t3 = __floats2bfloat162_rn(r[8 * u + 6], r[8 * u + 7]);
+                    pk.x = *reinterpret_cast<uint32_t*>(&t0);
+                    pk.y = *reinterpret_cast<uint32_t*>(&t1);
+                    pk.z = *reinterpret_cast<uint32_t*>(&t2);
+                    pk.w = *reinterpret_cast<uint32_t*>(&t3);
+                    *reinterpret_cast<uint4*>(smem + sw128_offset(i_row, col, 128)) = pk;
                 }
-                if (a.out_bf16) {
-                    __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(a.out) + obase + c * 32;
+            } else {  // boxes of 32 columns: box c holds columns [32c, 32c + 32)
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint4 pk;
-                        __nv_bfloat162 t0 = __floats2bfloat162_rn(r[i], r[i + 1]);
-                        __nv_bfloat162 t1 = __floats2bfloat162_rn(r[i + 2], r[i + 3]);
-                        __nv_bfloat162 t2 = __floats2bfloat162_rn(r[i + 4], r[i + 5]);
-                        __nv_bfloat162 t3 = __floats2bfloat162_rn(r[i + 6], r[i + 7]);
-                        pk.x = *reinterpret_cast<uint32_t*>(&t0);
-                        pk.y = *reinterpret_cast<uint32_t*>(&t1);
-                        pk.z = *reinterpret_cast<uint32_t*>(&t2);
-                        pk.w = *reinterpret_cast<uint32_t*>(&t3);
-                        *reinterpret_cast<uint4*>(op + i) = pk;
-                    }
-                } else {
-                    float* op = reinterpret_cast<float*>(a.out) + obase + c * 32;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4*>(op + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t off = c * 16384 + i_row * 128 + (((u ^ (i_row & 7))) << 4);
+                    *reinterpret_cast<float4*>(smem + off) = make_float4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
                 }
             }
+        }
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            const int cols_per_box = a.out_bf16 ? 64 : 32;
+            const int boxes = D / cols_per_box;
+            for (int bx = 0; bx < boxes; ++bx)
+                for (int rh = 0; rh * 64 < blk; ++rh) {
+                    if (alpha * blk + rh * 64 >= g.L) break;
+                    tma_store_4d(&tm_out, smem + bx * 16384 + rh * 64 * 128, bx * cols_per_box, h,
+                                 alpha * blk + rh * 64, b);
+                }
+            tma_store_commit_and_wait();
         }
     }
     // ------------------------------------------------------------------ teardown
@@ -613,9 +650,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (n_q_issued > n_q_done) mbar_wait(bar_q, 0, drain, &no_abort);
         if (n_k_issued > n_k_done) mbar_wait(bar_k, n_k_done & 1, drain, &no_abort);
         if (n_v_issued > n_v_done) mbar_wait(bar_v, n_v_done & 1, drain, &no_abort);
+        if (n_pv_issued > n_pv_done) mbar_wait(bar_pv, n_pv_done & 1, drain, &no_abort);
         if (n_s_issued > n_s_done) mbar_wait(bar_s, n_s_done & 1, drain, &no_abort);
         if (n_o_issued > n_o_done) mbar_wait(bar_o, n_o_done & 1, drain, &no_abort);
         if (n_eld_issued > n_eld) mbar_wait(bar_eld, n_eld & 1, drain, &no_abort);
+        if (n_ez_issued > n_ez) mbar_wait(bar_ez, n_ez & 1, drain, &no_abort);
         if (n_emm_issued > n_emm) mbar_wait(bar_emm, n_emm & 1, drain, &no_abort);
     }
     tc_fence_before();
@@ -637,11 +676,11 @@ cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, const Geom& g, cud
     if (g.D == 128) {
         e = cudaFuncSetAttribute(attn_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        attn_sm100_kernel<128><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, a, g);
+        attn_sm100_kernel<128><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, m.out, a, g);
     } else {
         e = cudaFuncSetAttribute(attn_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        attn_sm100_kernel<64><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, a, g);
+        attn_sm100_kernel<64><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, m.out, a, g);
     }
     return cudaGetLastError();
 }

@@ -55,6 +55,7 @@ cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, co
 int lowrank_nsplit(const Geom& g);
 bool make_map_headmajor(CUtensorMap* m, const void* base, uint64_t rows, int D, int box_rows);
 bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int D, int box_tokens);
+bool make_map_out(CUtensorMap* m, void* base, int B, int L, int Hh, int D, bool f32);
 cudaError_t launch_lowrank_reduce(const float* s_part, const float* z_part, const Geom& g, int nsplit, float* S,
                                   float* z, const __nv_bfloat16* A, uint8_t* at_img, uint8_t* sb_img, cudaStream_t st);
 
@@ -62,6 +63,7 @@ cudaError_t launch_lowrank_reduce(const float* s_part, const float* z_part, cons
 struct AttnMaps {
     CUtensorMap q, k, v;
     CUtensorMap q_raw;  // 4D map over the raw bf16 queries [B][L][Hh][D], box 64 x 1 x 128 x 1
+    CUtensorMap out;    // 4D map over out [B][L][Hh][D] (fp32: box 32 x 1 x 64 x 1; bf16: 64 x 1 x 64 x 1)
 };
 
 // Operand images for the tensor-core low-rank readout (head_dim 128), built by the reduction:

@@ -57,12 +57,6 @@ __host__ __device__ inline LrLayout lr_layout(int R) {
     return l;
 }
 
-// bf16 bits of x rounded to nearest even.
-__device__ __forceinline__ uint16_t bf16_bits(float x) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    return *reinterpret_cast<const uint16_t*>(&h);
-}
-
 }  // namespace
 
 struct LrArgs {

@@ -57,6 +57,23 @@ bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4D map over the output [B][L][Hh][D] for 64-token TMA stores of 128-byte column boxes (32 fp32 or 64
+// bf16 columns), 128-B swizzle on the shared-memory side; tokens past L are not written.
+bool make_map_out(CUtensorMap* m, void* base, int B, int L, int Hh, int D, bool f32) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t es = f32 ? 4 : 2;
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hh), static_cast<cuuint64_t>(L),
+                          static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * es, static_cast<cuuint64_t>(Hh) * D * es,
+                             static_cast<cuuint64_t>(L) * Hh * D * es};
+    cuuint32_t box[4] = {f32 ? 32u : 64u, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Split count of the low-rank partial sums.  head_dim 128 (tensor-core kernel): ranges of 128-token
 // tiles sized so a persistent grid of 148 CTAs gets about eight work items each; otherwise (CUDA-core
 // kernel, 32-token steps) about two CTAs per SM.
