@@ -5,13 +5,14 @@
 // union of the kept key blocks K(alpha); plus O_lr,i = psi(q_i)^T S / (phi(q_i) . z + 1e-6) with
 // phi = relu(q A) on the raw query and psi its first r coordinates rotated by 3D RoPE ("4.2", "4.3").
 //
-// One CTA (128 threads = 4 warps) per (query block, batch*head); two CTAs share an SM, so one CTA's
+// One CTA (256 threads = 8 warps) per (query block, batch*head); two CTAs share an SM, so one CTA's
 // softmax overlaps the other's matrix products.  Per kept key block:
 //   TMA   k^ tile [block][D] and v tile [block][D] (fp16, 128-B swizzle) into shared memory;
 //   MMA   S = q^ k^T      (tcgen05.mma kind::f16, M=128, N=block, K=D; fp32 accumulator in TMEM);
-//   softmax: thread i owns row i (TMEM lane i): row max, lazy rescale of O (only when the max grows
-//         by more than 2^8), P = 2^(s*log2e/sqrt(D) - m) rounded to fp16 and written back into the
-//         TMEM columns of S;
+//   softmax: row i lives in TMEM lane i; warps w and w+4 both reach lanes 32(w%4).. and split the
+//         key block in halves, exchanging their row maxima (and at the end their row sums) through
+//         shared memory: row max, lazy rescale of O (only when the max grows by more than 2^8),
+//         P = 2^(s*log2e/sqrt(D) - m) rounded to fp16 and written back into the TMEM columns of S;
 //   MMA   O += P v        (A operand = P from TMEM, B = v tile MN-major; M=128, N=D, K=block).
 // Epilogue: the low-rank readout (head_dim 128: on the tensor cores, accumulated into O; head_dim 64: on
 // the CUDA cores in fp32), then O / l staged in shared memory and written by TMA stores (fp32 or bf16).
@@ -19,14 +20,13 @@
 // All waits are bounded (see sm100.cuh); a wait that runs out records a timeout in the status word
 // and the CTA leaves the loop, releases its tensor memory and returns.
 #include "common.cuh"
-#include "exp2_poly.cuh"
 #include "sm100.cuh"
 
 namespace slra {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kTmemCols = 256;   // S/P at columns [0, 128), O at [128, 128 + D)
 constexpr int kColO = 128;
 
@@ -39,7 +39,8 @@ struct AttnLayout {
     static constexpr int kOffV = kOffK + kKVBytes;
     static constexpr int kOffBar = kOffV + kKVBytes;  // 16 mbarriers
     static constexpr int kOffMisc = kOffBar + 128;    // tmem base, abort flag
-    static constexpr int kBytes = kOffMisc + 64;
+    static constexpr int kOffXch = kOffMisc + 64;     // [2][128] fp32 row partials of the two key halves
+    static constexpr int kBytes = kOffXch + 1024;
 };
 
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
@@ -83,28 +84,16 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     return r;
 }
 
-// 2^x without the MUFU unit, for x <= 128: n = floor(x) via a round-down add of 1.5 * 2^23, f = x - n,
-// 2^f from the degree-3 minimax polynomial of exp2_poly.cuh (max relative error 7.5e-5), and 2^n
-// added into the exponent field.  Inputs below -126 (and -inf) are clamped to -126: p(0) is just
-// below 1 (exponent field 126), so n must stay >= -126 for the exponent field to stay >= 0; the result
-// there is < 2^-125, which rounds to zero in the fp16 P operand anyway.
-__device__ __forceinline__ float exp2_soft(float x) {
-    x = fmaxf(x, -126.0f);
-    float t;
-    asm("add.rm.f32 %0, %1, 0f4B400000;" : "=f"(t) : "f"(x));
-    const float f = x - (t - 12582912.0f);
-    const float p = fmaf(fmaf(fmaf(SLRA_EXP2_C3, f, SLRA_EXP2_C2), f, SLRA_EXP2_C1), f, SLRA_EXP2_C0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 }  // namespace
 
-template <int D>
+template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qraw,
                       const __grid_constant__ CUtensorMap tm_out, AttnArgs a, Geom g) {
     using Lay = AttnLayout<D>;
+    constexpr int HW = BLK / 2;   // keys per thread: the two warps of a lane group split the key block
+    constexpr int NC = HW / 32;   // 32-column TMEM loads per thread
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __half* sq = reinterpret_cast<__half*>(smem + Lay::kOffQ);
@@ -119,11 +108,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t* bar_pv = bars + 8;   // P.V done (frees the v tile early)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
+    float* xch = reinterpret_cast<float*>(smem + Lay::kOffXch);  // [2][128]: per-half row partials
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lg = warp & 3;    // TMEM lane group (rows 32*lg ..), fixed by the warp's rank in its warpgroup
+    const int hf = warp >> 2;   // which half of the key block (and of O's columns) this warp handles
+    const int i_row = lg * 32 + lane;
     const int alpha = blockIdx.x, bh = blockIdx.y;
     const int b = bh / g.Hh, h = bh % g.Hh;
-    const int blk = g.block;
+    const int blk = BLK;
     const int keep = a.keep;
     const uint64_t tmo = a.timeout_ns;
     const int32_t* my_idx = a.idx + (static_cast<size_t>(bh) * g.nb + alpha) * (keep > 0 ? g.keep : 0);
@@ -143,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem;               // S (fp32) and P (fp16 packed) columns
     const uint32_t tO = tmem + kColO;       // O accumulator
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>(lg * 32) << 16;
 
     const uint32_t idesc_s = idesc_f16_f32(128, blk, false, false);
     const uint32_t idesc_o = idesc_f16_f32(128, D, false, true);
@@ -225,63 +218,71 @@ __global__ void __launch_bounds__(kThreads, 2)
     // The kept list is ascending, so the only block that can be partial (the sequence's last) can only
     // be the last one visited.
     const int last_valid = keep > 0 ? min(blk, g.L - __ldg(my_idx + keep - 1) * blk) : blk;
+    const int key0 = hf * HW;  // first key of this thread's half of the block
+    // m_run is the row's running max (identical in both halves); l_run sums this half's keys only.
     float m_run = 0.f, l_run = 0.f;
     for (int j = 0; j < keep; ++j) {
-        const bool ok = mbar_wait(bar_s, j & 1, tmo, abort_flag);
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) fail();
-            break;
-        }
+        // warp-uniform, since the TMEM loads below are warp-collective
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, tmo, abort_flag));
         tc_fence_after();
-        if (tid == 0) {
+        if (tid == 0 && ok) {
             ++n_s_done;
             // S_j has finished reading the k tile and (issued before it) P.V_{j-1} the v tile.
             if (j + 1 < keep) { load_kv(bar_k, sk, &tm_k, my_idx[j + 1]); ++n_k_issued; }
             if (j == keep - 1 && prefetch_epi) issue_epilogue_prefetch();  // q and k tiles are free now
         }
-        // ---- softmax of row (warp*32 + lane); O is stable (P.V_{j-1} completed before S_j)
-        uint32_t sr[4][32];
+        // ---- softmax of row i_row over keys [key0, key0 + HW); O is stable (P.V_{j-1} completed
+        //      before S_j)
+        uint32_t sr[NC][32];
+        if (ok) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-            if (c * 32 < blk) tmem_ld32(tS + lane_base + c * 32, sr[c]);
-        tmem_ld_wait(sr[0]);
+            for (int c = 0; c < NC; ++c) tmem_ld32(tS + lane_base + key0 + c * 32, sr[c]);
+            tmem_ld_wait(sr[0]);
 #pragma unroll
-        for (int c = 1; c < 4; ++c)
-            if (c * 32 < blk) reg_fence(sr[c]);
+            for (int c = 1; c < NC; ++c) reg_fence(sr[c]);
+        }
+        constexpr int NE = HW;  // elements this thread owns
+        auto el = [&](int e) -> uint32_t& { return sr[e >> 5][e & 31]; };
         if (j == keep - 1 && last_valid < blk) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (c * 32 + i >= last_valid) sr[c][i] = __float_as_uint(-INFINITY);
+            for (int e = 0; e < NE; ++e)
+                if (key0 + e >= last_valid) el(e) = __float_as_uint(-INFINITY);
         }
-        // row max: four independent chains of 3-input max (short dependency chains)
+        // row max over this half: four independent chains of 3-input max
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            if (c * 32 >= blk) continue;
+        for (int e = 0; e < NE; e += 8) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-                    mx4[t] = fmax3(mx4[t], __uint_as_float(sr[c][i + 2 * t]), __uint_as_float(sr[c][i + 2 * t + 1]));
-            }
+            for (int t = 0; t < 4; ++t)
+                mx4[t] = fmax3(mx4[t], __uint_as_float(el(e + 2 * t)), __uint_as_float(el(e + 2 * t + 1)));
         }
-        float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+        const float mx_half = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+        xch[hf * 128 + i_row] = mx_half;
+        // One barrier exchanges the two halves' maxima, makes the abort decision uniform, and orders
+        // every thread's S loads before the P stores below (half 1's P columns overlap half 0's S).
+        tc_fence_before();
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) fail();
+            break;
+        }
+        tc_fence_after();
+        float mx = fmaxf(mx_half, xch[(hf ^ 1) * 128 + i_row]);  // same value in both halves
         mx *= scale_log2;
         if (j == 0) {
             m_run = mx;
         } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {  // warp-uniform: TMEM access is collective
+            // Both warps of the lane group see the same maxima, so they take the same branch; each
+            // rescales its half of O's columns.
             const float m_new = fmaxf(m_run, mx);
             const float alpha_r = ex2_approx(m_run - m_new);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tO + lane_base + c * 32, o);
+            for (int c = 0; c < D / 32; ++c) {  // 16 columns at a time (the scores stay in registers)
+                uint32_t o[16];
+                tmem_ld16(tO + lane_base + hf * (D / 2) + c * 16, o);
                 tmem_ld_wait(o);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha_r);
-                tmem_st32(tO + lane_base + c * 32, o);
+                for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha_r);
+                tmem_st16(tO + lane_base + hf * (D / 2) + c * 16, o);
             }
             tmem_st_wait();
             l_run *= alpha_r;
@@ -289,28 +290,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const float neg_m = -m_run;
         float sums[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};  // independent accumulators
+        // keys (2i, 2i+1) of this half -> packed fp16x2 TMEM column key0/2 + i, 16 columns at a time
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {  // 64 keys -> 32 packed fp16x2 TMEM columns
-            if (c2 * 64 >= blk) continue;
-            uint32_t pk[32];
+        for (int c16 = 0; c16 < NE / 32; ++c16) {
+            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int key = c2 * 64 + 2 * i;
+            for (int u = 0; u < 16; ++u) {
+                const int i = c16 * 16 + u;
                 float t0, t1;
-                ffma2(t0, t1, __uint_as_float(sr[key >> 5][key & 31]), __uint_as_float(sr[key >> 5][(key & 31) + 1]),
-                      scale_log2, scale_log2, neg_m, neg_m);
-                float p0, p1;
-                if ((i & 3) == 0) {  // a quarter of the exponentials on the FMA/ALU pipes
-                    p0 = exp2_soft(t0);
-                    p1 = exp2_soft(t1);
-                } else {
-                    p0 = ex2_approx(t0);
-                    p1 = ex2_approx(t1);
-                }
-                fadd2(sums[i & 3][0], sums[i & 3][1], p0, p1);
-                pk[i] = pack_half2(p0, p1);
+                ffma2(t0, t1, __uint_as_float(el(2 * i)), __uint_as_float(el(2 * i + 1)), scale_log2, scale_log2,
+                      neg_m, neg_m);
+                const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                fadd2(sums[u & 3][0], sums[u & 3][1], p0, p1);
+                pk[u] = pack_half2(p0, p1);
             }
-            tmem_st32(tS + lane_base + c2 * 32, pk);
+            tmem_st16(tS + lane_base + key0 / 2 + c16 * 16, pk);
         }
         tmem_st_wait();
         l_run += ((sums[0][0] + sums[0][1]) + (sums[1][0] + sums[1][1])) +
@@ -327,8 +321,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 } else {
                     ++n_v_done;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        if (kk * 16 >= blk) break;
+                    for (int kk = 0; kk < BLK / 16; ++kk) {
                         const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, static_cast<uint32_t>(blk) * 128, 1024);
                         umma_ts(tO, tS + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                     }
@@ -365,12 +358,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (__syncthreads_or(!ok) && tid == 0) fail();
         if (tid == 0 && ok) ++n_o_done;
     }
+    // Row sum: the two halves' partial sums (fp32 addition commutes, so both get the same total).
+    xch[hf * 128 + i_row] = l_run;
     __syncthreads();
+    l_run += xch[(hf ^ 1) * 128 + i_row];
     tc_fence_after();
     const bool aborted = *abort_flag != 0;
 
     // ------------------------------------------------------------------ epilogue
-    const int i_row = warp * 32 + lane;
     const int n = alpha * blk + i_row;
     const bool row_valid = (i_row < blk) && (n < g.L) && !aborted;
     float inv_l = (keep > 0 && l_run > 0.f) ? 1.f / l_run : 0.f;
@@ -381,6 +376,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             //   phi = q A        raw bf16 query tile (TMA) x A^T image, into the free S columns;
             //   psi = R_r(p) relu(phi) * l / (relu(phi) . z + 1e-6), split into bf16 hi + lo;
             //   O  += psi S      as psi_hi S_hi + psi_hi S_lo + psi_lo S_hi, one 64-feature chunk at a time.
+            // The two warps of a lane group share each row: 32-feature column groups of the
+            // denominator alternate between them, and so do the rotation pairs.
             const int R = g.R;
             const int nch = (R + 63) / 64;
             uint8_t* X = smem;           // raw query tile, then each chunk's psi operand [128][3*rc]
@@ -432,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float* zh = a.z + static_cast<size_t>(bh) * R;
                 float den = 0.f;
 #pragma unroll
-                for (int c0 = 0; c0 < 128; c0 += 32) {
+                for (int c0 = hf * 32; c0 < 128; c0 += 64) {
                     if (c0 < R) {
                         uint32_t v[32];
                         tmem_ld32(tS + lane_base + c0, v);
@@ -442,6 +439,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                             if (c0 + i < R) den = fmaf(fmaxf(__uint_as_float(v[i]), 0.f), __ldg(zh + c0 + i), den);
                     }
                 }
+                xch[hf * 128 + i_row] = den;
+                __syncthreads();
+                den += xch[(hf ^ 1) * 128 + i_row];  // same total in both halves
                 const float l_eff = keep > 0 ? l_run : 1.f;
                 const float scale = l_eff / (den + 1e-6f);
                 const int n_tab = n < g.L ? n : g.L - 1;  // rows past the sequence: any valid table entry
@@ -468,17 +468,22 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tmem_ld_wait(v[0]);
                     reg_fence(v[1]);
 #pragma unroll
-                    for (int pp = 0; pp < 32; ++pp) {
+                    for (int t = 0; t < 16; ++t) {
+                        const int pp = 2 * t + hf;  // rotation pairs alternate between the two warps
                         if (2 * pp < rc) {
-                            const float x0 = fmaxf(__uint_as_float(v[pp >> 4][(2 * pp) & 31]), 0.f);
-                            const float x1 = fmaxf(__uint_as_float(v[pp >> 4][(2 * pp + 1) & 31]), 0.f);
+                            // features 4t + 2hf and 4t + 2hf + 1 (static register indices, then a select)
+                            const int f0 = 4 * t;
+                            const uint32_t u0 = hf ? v[(f0 + 2) >> 5][(f0 + 2) & 31] : v[f0 >> 5][f0 & 31];
+                            const uint32_t u1 = hf ? v[(f0 + 3) >> 5][(f0 + 3) & 31] : v[f0 >> 5][(f0 + 1) & 31];
+                            const float x0 = fmaxf(__uint_as_float(u0), 0.f);
+                            const float x1 = fmaxf(__uint_as_float(u1), 0.f);
                             const int2 pi = __ldg(a.pairs + 32 * ch + pp);
                             const double2 cs = __ldg(a.tab + pi.y + token_axis_pos(n_tab, pi.x, g.H, g.W));
                             const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
                             const float y0 = (x0 * cf - x1 * sf) * scale, y1 = (x0 * sf + x1 * cf) * scale;
                             const __nv_bfloat162 hi = __floats2bfloat162_rn(y0, y1);
-                            const float2 hf = __bfloat1622float2(hi);
-                            const __nv_bfloat162 lo = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
+                            const float2 hf2 = __bfloat1622float2(hi);
+                            const __nv_bfloat162 lo = __floats2bfloat162_rn(y0 - hf2.x, y1 - hf2.y);
                             const uint32_t hb = *reinterpret_cast<const uint32_t*>(&hi);
                             const uint32_t lb = *reinterpret_cast<const uint32_t*>(&lo);
                             *reinterpret_cast<uint32_t*>(X + sw128_offset(i_row, 2 * pp, 128)) = hb;
@@ -520,18 +525,21 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
     }
-    float acc[D == 128 ? 1 : D];
+    // head_dim 64: CUDA-core readout; both warps of a lane group compute the row's features and each
+    // accumulates its half of the output columns.
+    constexpr int DH = D / 2;
+    float acc[D == 128 ? 1 : DH];
     float inv_den = 0.f;
     if constexpr (D != 128) {
 #pragma unroll
-        for (int e = 0; e < D; ++e) acc[e] = 0.f;
+        for (int e = 0; e < DH; ++e) acc[e] = 0.f;
         if (a.lowrank && !aborted) {
             float* As = reinterpret_cast<float*>(smem);  // [D][R] fp32, reuses the tile buffers
             for (int e = tid; e < D * g.R; e += kThreads) As[e] = __bfloat162float(a.A[e]);
             __syncthreads();
             if (row_valid) {
                 const __nv_bfloat16* qrow = a.q_raw + ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;
-                const float* Sh = a.S + static_cast<size_t>(bh) * g.R * D;
+                const float* Sh = a.S + static_cast<size_t>(bh) * g.R * D + hf * DH;
                 const float* zh = a.z + static_cast<size_t>(bh) * g.R;
                 float den = 0.f;
                 for (int c0 = 0; c0 < g.R; c0 += 16) {
@@ -568,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     for (int c = 0; c < 16; ++c) {
                         const float4* s4 = reinterpret_cast<const float4*>(Sh + (c0 + c) * D);
 #pragma unroll
-                        for (int e4 = 0; e4 < D / 4; ++e4) {
+                        for (int e4 = 0; e4 < DH / 4; ++e4) {
                             const float4 sv4 = __ldg(s4 + e4);
                             acc[4 * e4 + 0] = fmaf(phi[c], sv4.x, acc[4 * e4 + 0]);
                             acc[4 * e4 + 1] = fmaf(phi[c], sv4.y, acc[4 * e4 + 1]);
@@ -581,14 +589,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
     }
-    // ---- out = O / l (+ the CUDA-core readout for head_dim 64): each thread writes its row into a
-    //      128-B-swizzled staging tile (conflict-free 16-byte stores), then 64-row TMA stores write it
-    //      out; tokens past L are clipped by the tensor map and a 64-token block's second half is skipped.
+    // ---- out = O / l (+ the CUDA-core readout for head_dim 64): each thread writes its half of its
+    //      row into a 128-B-swizzled staging tile (conflict-free 16-byte stores), then 64-row TMA stores
+    //      write it out; tokens past L are clipped by the tensor map and a 64-token block's second half
+    //      is skipped.
     const bool aborted2 = *abort_flag != 0;
     if (!aborted2) {
         __syncthreads();  // every product that read the tile buffers has completed
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int cc = 0; cc < D / 64; ++cc) {
+            const int c = hf * (D / 64) + cc;  // 32-column group of O
             uint32_t o[32];
             if (o_live) {
                 tmem_ld32(tO + lane_base + c * 32, o);
@@ -601,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 float x = __uint_as_float(o[i]) * inv_l;
-                if constexpr (D != 128) x += acc[c * 32 + i] * inv_den;
+                if constexpr (D != 128) x += acc[cc * 32 + i] * inv_den;
                 r[i] = x;
             }
             if (a.out_bf16) {  // boxes of 64 columns
@@ -669,20 +679,21 @@ size_t attn_smem_bytes(const Geom& g) {
     return (g.D == 128 ? AttnLayout<128>::kBytes : AttnLayout<64>::kBytes) + 1024;
 }
 
-cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st) {
-    dim3 grid(g.nb, g.BH());
+namespace {
+template <int D, int BLK>
+cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st) {
     const size_t sm = attn_smem_bytes(g);
-    cudaError_t e;
-    if (g.D == 128) {
-        e = cudaFuncSetAttribute(attn_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
-        attn_sm100_kernel<128><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, m.out, a, g);
-    } else {
-        e = cudaFuncSetAttribute(attn_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
-        attn_sm100_kernel<64><<<grid, kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, m.out, a, g);
-    }
+    cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sm));
+    if (e != cudaSuccess) return e;
+    attn_sm100_kernel<D, BLK><<<dim3(g.nb, g.BH()), kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, m.out, a, g);
     return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st) {
+    if (g.D == 128) return g.block == 128 ? launch_attn_t<128, 128>(m, a, g, st) : launch_attn_t<128, 64>(m, a, g, st);
+    return g.block == 128 ? launch_attn_t<64, 128>(m, a, g, st) : launch_attn_t<64, 64>(m, a, g, st);
 }
 
 }  // namespace slra
