@@ -356,6 +356,9 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
         if ((s = run_lowrank(p, d, w, k, v, A, st)) != SLRA_OK) return s;
 
     AttnArgs a;
+    a.qh = w.qh;
+    a.kh = w.kh;
+    a.vh = w.vh;
     a.idx = w.idx;
     a.keep = (branches & SLRA_BRANCH_SPARSE) ? g.keep : 0;
     a.q_raw = static_cast<const __nv_bfloat16*>(q);
@@ -364,6 +367,8 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
     a.z = w.z;
     a.tab = w.tab;
     a.pairs = w.pairs;
+    for (int e = 0; e < kMaxPairs; ++e)
+        a.pair_info[e] = e < d.meta.npairs ? make_int2(d.meta.axis[e], d.meta.tab_off[e]) : make_int2(0, 0);
     a.at_img = w.at_img;
     a.sb_img = w.sb_img;
     a.lowrank = (branches & SLRA_BRANCH_LOWRANK) ? 1 : 0;

@@ -14,6 +14,8 @@
 //         shared memory: row max, lazy rescale of O (only when the max grows by more than 2^8),
 //         P = 2^(s*log2e/sqrt(D) - m) rounded to fp16 and written back into the TMEM columns of S;
 //   MMA   O += P v        (A operand = P from TMEM, B = v tile MN-major; M=128, N=D, K=block).
+// P.V_j and S_{j+1} are issued back to back; when S_{j+1} completes, so has P.V_j, and both the next
+// k tile and the next v tile are loaded right then (one tile buffer each).
 // Epilogue: the low-rank readout (head_dim 128: on the tensor cores, accumulated into O; head_dim 64: on
 // the CUDA cores in fp32), then O / l staged in shared memory and written by TMA stores (fp32 or bf16).
 //
@@ -105,7 +107,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t* bar_v = bars + 2;
     uint64_t* bar_s = bars + 3;
     uint64_t* bar_o = bars + 4;
-    uint64_t* bar_pv = bars + 8;   // P.V done (frees the v tile early)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
     float* xch = reinterpret_cast<float*>(smem + Lay::kOffXch);  // [2][128]: per-half row partials
@@ -168,7 +169,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     // what is still in flight before it releases shared and tensor memory.
     int n_q_issued = 0, n_q_done = 0, n_k_issued = 0, n_k_done = 0, n_v_issued = 0, n_v_done = 0;
     int n_s_issued = 0, n_s_done = 0, n_o_issued = 0, n_o_done = 0;
-    int n_pv_issued = 0, n_pv_done = 0;
+    // Thread 0 keeps the kept-block indices one iteration ahead in registers (the loads stay off the
+    // softmax's critical path): beta_cur = block of the next v tile to load, beta_next = of the next k tile.
+    int beta_cur = 0, beta_next = 0;
     // epilogue barrier bookkeeping (thread 0 for the loads; every thread for the products)
     int n_eld_issued = 0, n_eld = 0, n_emm_issued = 0, n_emm = 0, n_ez_issued = 0, n_ez = 0;
     uint64_t* bar_eld = bars + 5;  // epilogue: raw query tile + A^T image (one phase)
@@ -200,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int s = 0; s < D / 64; ++s)
             tma_load_2d(reinterpret_cast<uint8_t*>(sq) + s * (128 * 128), &tm_q, bar_q, s * 64, row0 + alpha * blk);
         const int beta0 = my_idx[0];
+        beta_next = keep > 1 ? __ldg(my_idx + 1) : 0;
         load_kv(bar_k, sk, &tm_k, beta0);
         load_kv(bar_v, sv, &tm_v, beta0);
         n_q_issued = 1; n_k_issued = 1; n_v_issued = 1;
@@ -227,8 +231,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         if (tid == 0 && ok) {
             ++n_s_done;
-            // S_j has finished reading the k tile and (issued before it) P.V_{j-1} the v tile.
-            if (j + 1 < keep) { load_kv(bar_k, sk, &tm_k, my_idx[j + 1]); ++n_k_issued; }
+            // S_j has finished reading the k tile and (issued before it) P.V_{j-1} the v tile: load v_j
+            // and k_{j+1}.
+            if (j > 0) { load_kv(bar_v, sv, &tm_v, beta_cur); ++n_v_issued; }
+            if (j + 1 < keep) { load_kv(bar_k, sk, &tm_k, beta_next); ++n_k_issued; }
+            beta_cur = beta_next;
+            if (j + 2 < keep) beta_next = __ldg(my_idx + j + 2);
             if (j == keep - 1 && prefetch_epi) issue_epilogue_prefetch();  // q and k tiles are free now
         }
         // ---- softmax of row i_row over keys [key0, key0 + HW); O is stable (P.V_{j-1} completed
@@ -325,20 +333,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                         const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, static_cast<uint32_t>(blk) * 128, 1024);
                         umma_ts(tO, tS + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit(bar_pv);  // lets the next v tile load as soon as this product is done
-                    ++n_pv_issued;
                     if (j + 1 < keep) {
                         if (mbar_wait(bar_k, (j + 1) & 1, tmo, abort_flag)) {
                             ++n_k_done;
                             issue_s();  // commits bar_s, which also covers this P.V
                             ++n_s_issued;
-                            if (mbar_wait(bar_pv, n_pv_done & 1, tmo, abort_flag)) {
-                                ++n_pv_done;
-                                load_kv(bar_v, sv, &tm_v, my_idx[j + 1]);
-                                ++n_v_issued;
-                            } else {
-                                fail();
-                            }
                         } else {
                             umma_commit(bar_o);
                             ++n_o_issued;
@@ -445,6 +444,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float l_eff = keep > 0 ? l_run : 1.f;
                 const float scale = l_eff / (den + 1e-6f);
                 const int n_tab = n < g.L ? n : g.L - 1;  // rows past the sequence: any valid table entry
+                const int axis_t = token_axis_pos(n_tab, 0, g.H, g.W), axis_h = token_axis_pos(n_tab, 1, g.H, g.W),
+                          axis_w = token_axis_pos(n_tab, 2, g.H, g.W);
                 for (int ch = 0; ch < nch && ok; ++ch) {
                     const int rc = min(64, R - 64 * ch);
                     if (ch > 0) {  // the previous chunk's product must have finished with X and Z
@@ -462,24 +463,46 @@ __global__ void __launch_bounds__(kThreads, 2)
                             ++n_ez_issued;
                         }
                     }
-                    uint32_t v[2][32];
-                    tmem_ld32(tS + lane_base + 64 * ch, v[0]);
-                    tmem_ld32(tS + lane_base + 64 * ch + 32, v[1]);
-                    tmem_ld_wait(v[0]);
-                    reg_fence(v[1]);
+                    // This thread's 16 rotation pairs of the chunk: features [16hf, 16hf + 16) and
+                    // [32 + 16hf, 48 + 16hf) (so both warps of a lane group have work when rc <= 32).
+                    // Their (cos, sin) are fetched eight at a time, every load issued before any is used;
+                    // the pair table holds all D/2 rotary pairs, so pairs past the rank are still valid
+                    // entries (their results are not stored).  The pair -> (axis, table offset) map comes
+                    // from the launch parameters.
+                    auto feat = [&](int t) { return t < 8 ? 16 * hf + 2 * t : 32 + 16 * hf + 2 * (t - 8); };
+                    float2 rot[16];
+#pragma unroll
+                    for (int b8 = 0; b8 < 2; ++b8) {
+                        int2 pi[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) pi[t] = a.pair_info[32 * ch + feat(b8 * 8 + t) / 2];
+                        double2 cs[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            const int ap = pi[t].x == 0 ? axis_t : (pi[t].x == 1 ? axis_h : axis_w);
+                            cs[t] = __ldg(a.tab + pi[t].y + ap);
+                        }
+#pragma unroll
+                        for (int t = 0; t < 8; ++t)
+                            rot[b8 * 8 + t] = make_float2(static_cast<float>(cs[t].x), static_cast<float>(cs[t].y));
+                    }
+                    uint32_t va[16], vb[16];
+                    tmem_ld16(tS + lane_base + 64 * ch + 16 * hf, va);
+                    tmem_ld16(tS + lane_base + 64 * ch + 32 + 16 * hf, vb);
+                    tmem_ld_wait(va);
+                    asm volatile("" : "+r"(vb[0]), "+r"(vb[1]), "+r"(vb[2]), "+r"(vb[3]), "+r"(vb[4]), "+r"(vb[5]),
+                                 "+r"(vb[6]), "+r"(vb[7]), "+r"(vb[8]), "+r"(vb[9]), "+r"(vb[10]), "+r"(vb[11]),
+                                 "+r"(vb[12]), "+r"(vb[13]), "+r"(vb[14]), "+r"(vb[15]));
 #pragma unroll
                     for (int t = 0; t < 16; ++t) {
-                        const int pp = 2 * t + hf;  // rotation pairs alternate between the two warps
-                        if (2 * pp < rc) {
-                            // features 4t + 2hf and 4t + 2hf + 1 (static register indices, then a select)
-                            const int f0 = 4 * t;
-                            const uint32_t u0 = hf ? v[(f0 + 2) >> 5][(f0 + 2) & 31] : v[f0 >> 5][f0 & 31];
-                            const uint32_t u1 = hf ? v[(f0 + 3) >> 5][(f0 + 3) & 31] : v[f0 >> 5][(f0 + 1) & 31];
+                        const int f = feat(t);
+                        const int pp = f / 2;
+                        if (f < rc) {
+                            const uint32_t u0 = t < 8 ? va[2 * t] : vb[2 * (t - 8)];
+                            const uint32_t u1 = t < 8 ? va[2 * t + 1] : vb[2 * (t - 8) + 1];
                             const float x0 = fmaxf(__uint_as_float(u0), 0.f);
                             const float x1 = fmaxf(__uint_as_float(u1), 0.f);
-                            const int2 pi = __ldg(a.pairs + 32 * ch + pp);
-                            const double2 cs = __ldg(a.tab + pi.y + token_axis_pos(n_tab, pi.x, g.H, g.W));
-                            const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+                            const float cf = rot[t].x, sf = rot[t].y;
                             const float y0 = (x0 * cf - x1 * sf) * scale, y1 = (x0 * sf + x1 * cf) * scale;
                             const __nv_bfloat162 hi = __floats2bfloat162_rn(y0, y1);
                             const float2 hf2 = __bfloat1622float2(hi);
@@ -660,7 +683,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (n_q_issued > n_q_done) mbar_wait(bar_q, 0, drain, &no_abort);
         if (n_k_issued > n_k_done) mbar_wait(bar_k, n_k_done & 1, drain, &no_abort);
         if (n_v_issued > n_v_done) mbar_wait(bar_v, n_v_done & 1, drain, &no_abort);
-        if (n_pv_issued > n_pv_done) mbar_wait(bar_pv, n_pv_done & 1, drain, &no_abort);
         if (n_s_issued > n_s_done) mbar_wait(bar_s, n_s_done & 1, drain, &no_abort);
         if (n_o_issued > n_o_done) mbar_wait(bar_o, n_o_done & 1, drain, &no_abort);
         if (n_eld_issued > n_eld) mbar_wait(bar_eld, n_eld & 1, drain, &no_abort);

@@ -73,6 +73,9 @@ struct AttnMaps {
 constexpr int kSbChunkBytes = 3 * 128 * 128;
 
 struct AttnArgs {
+    const __half* qh;   // head-major fp16 q^, k^, v rows [B*Hh][Lp][D]
+    const __half* kh;
+    const __half* vh;
     const int32_t* idx;
     int keep;  // 0: no sparse branch
     const __nv_bfloat16* q_raw;
@@ -81,6 +84,7 @@ struct AttnArgs {
     const float* z;
     const double2* tab;
     const int2* pairs;  // per rotary pair: (axis, offset of its cos/sin table)
+    int2 pair_info[kMaxPairs];  // the same, as a launch parameter (read through the constant cache)
     const uint8_t* at_img;  // A^T operand image (head_dim 128)
     const uint8_t* sb_img;  // S operand images (head_dim 128)
     int lowrank;  // add the low-rank readout
