@@ -5,22 +5,30 @@
 // union of the kept key blocks K(alpha); plus O_lr,i = psi(q_i)^T S / (phi(q_i) . z + 1e-6) with
 // phi = relu(q A) on the raw query and psi its first r coordinates rotated by 3D RoPE ("4.2", "4.3").
 //
-// One CTA (256 threads = 8 warps) per (query block, batch*head); two CTAs share an SM, so one CTA's
-// softmax overlaps the other's matrix products.  Per kept key block:
-//   TMA   k^ tile [block][D] and v tile [block][D] (fp16, 128-B swizzle) into shared memory;
-//   MMA   S = q^ k^T      (tcgen05.mma kind::f16, M=128, N=block, K=D; fp32 accumulator in TMEM);
-//   softmax: row i lives in TMEM lane i; warps w and w+4 both reach lanes 32(w%4).. and split the
-//         key block in halves, exchanging their row maxima (and at the end their row sums) through
-//         shared memory: row max, lazy rescale of O (only when the max grows by more than 2^8),
-//         P = 2^(s*log2e/sqrt(D) - m) rounded to fp16 and written back into the TMEM columns of S;
-//   MMA   O += P v        (A operand = P from TMEM, B = v tile MN-major; M=128, N=D, K=block).
-// P.V_j and S_{j+1} are issued back to back; when S_{j+1} completes, so has P.V_j, and both the next
-// k tile and the next v tile are loaded right then (one tile buffer each).
-// Epilogue: the low-rank readout (head_dim 128: on the tensor cores, accumulated into O; head_dim 64: on
-// the CUDA cores in fp32), then O / l staged in shared memory and written by TMA stores (fp32 or bf16).
+// One CTA per (query block, batch*head), one CTA per SM, warp-specialised (320 threads):
+//   warps 0-7  softmax: row i lives in TMEM lane i; warps w and w+4 both reach lanes 32(w%4).. and
+//              split the key block in halves, exchanging their row maxima (and at the end their row
+//              sums) through shared memory: row max, lazy rescale of O (only when the max grows by
+//              more than 2^8), P = 2^(s*log2e/sqrt(D) - m) rounded to fp16 and written back into the
+//              TMEM columns of that S buffer;
+//   warp 8     TMA producer: q^ tile, then k^ and v tiles into two slots each (fp16, 128-B swizzle),
+//              each slot refilled as soon as the product that read it has completed;
+//   warp 9     MMA issuer: once the softmax has released P_j, O += P_j v_j (A operand P_j from TMEM,
+//              B = v tile MN-major) and S_{j+2} = q^ k^T_{j+2} into the S buffer P_{j-1} occupied
+//              (tcgen05.mma kind::f16, M=128, N=block, K=D, fp32 in TMEM), their k-steps issued
+//              alternately.
+// With three S buffers S_{j+1} is already in TMEM when the softmax finishes S_j, so a key block
+// costs about the longer of the softmax and the two products instead of their sum.  The two
+// products' k-steps are interleaved one by one: the tensor pipe runs a run of four or more
+// products of one kind followed by a run of the other at about half rate, strictly alternating
+// ones at full rate.
+// TMEM (512 columns): S0 | S1 | S2 | O; the epilogue's phi = q A reuses S0.
+// Epilogue (softmax warps): the low-rank readout (head_dim 128: on the tensor cores, accumulated into
+// O; head_dim 64: on the CUDA cores in fp32), then O / l staged in shared memory and written by TMA
+// stores (fp32 or bf16).
 //
-// All waits are bounded (see sm100.cuh); a wait that runs out records a timeout in the status word
-// and the CTA leaves the loop, releases its tensor memory and returns.
+// All waits are bounded (see sm100.cuh); a wait that runs out records a timeout in the status word,
+// every role leaves its loop, lets what it issued land, and the CTA releases its tensor memory.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -28,22 +36,64 @@ namespace slra {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTmemCols = 256;   // S/P at columns [0, 128), O at [128, 128 + D)
-constexpr int kColO = 128;
+constexpr int kSoftWarps = 8;
+constexpr int kSoftThreads = kSoftWarps * 32;
+constexpr int kWarpLoad = 8;   // TMA producer
+constexpr int kWarpMma = 9;    // tcgen05.mma issuer
+constexpr int kThreads = 320;
+constexpr int kNumS = 3;        // S buffers
+constexpr int kTmemCols = 512;  // S buffers at [128 b, 128 b + 128), O at [384, 384 + D)
+constexpr int kColO = 384;
+constexpr int kColPhi = 0;      // epilogue: phi in S0 (free once the last P.V has completed)
 
+// Shared memory: q^ tile, two k^ slots, two v slots (each sized for a 128-row block), barriers,
+// the row-partial exchange buffer.  The epilogue reuses the tile area.
 template <int D>
 struct AttnLayout {
-    static constexpr int kQBytes = 128 * D * 2;
-    static constexpr int kKVBytes = 128 * D * 2;  // sized for block 128
+    static constexpr int kTile = 128 * D * 2;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kQBytes;
-    static constexpr int kOffV = kOffK + kKVBytes;
-    static constexpr int kOffBar = kOffV + kKVBytes;  // 16 mbarriers
-    static constexpr int kOffMisc = kOffBar + 128;    // tmem base, abort flag
-    static constexpr int kOffXch = kOffMisc + 64;     // [2][128] fp32 row partials of the two key halves
-    static constexpr int kBytes = kOffXch + 1024;
+    static constexpr int kOffK = kOffQ + kTile;      // slots s at kOffK + s * kTile
+    static constexpr int kOffV = kOffK + 2 * kTile;  // slots s at kOffV + s * kTile
+    static constexpr int kOffBar = kOffV + 2 * kTile;  // 32 mbarriers
+    static constexpr int kOffMisc = kOffBar + 256;     // tmem base, abort flag
+    static constexpr int kOffXch = kOffMisc + 64;      // [2 parities][2 halves][128] fp32 row partials
+    static constexpr int kBytes = kOffXch + 2048;
 };
+
+// mbarrier indices
+enum : int {
+    kBarQ = 0,
+    kBarKFull = 1,    // +slot
+    kBarKEmpty = 3,   // +slot: S that read the slot has completed
+    kBarVFull = 5,    // +slot
+    kBarVEmpty = 7,   // +slot: P.V that read the slot has completed
+    kBarSFull = 9,    // +buffer: S_j in TMEM
+    kBarPFull = 12,   // +buffer: P_j in TMEM (one arrival per softmax thread)
+    kBarODone = 15,   // +buffer: P.V_j (reading P from that buffer) has completed
+    kBarEld = 18,     // epilogue: raw query tile + A^T image
+    kBarEz = 19,      // epilogue: S image of each 64-feature chunk
+    kBarEmm = 20,     // epilogue products
+    kBarDebug = 21,   // test hook: nothing arrives here
+    kBarDrain = 22,   // MMA issuer's final commit on the abort path
+    kBarOFinal = 23,  // the last P.V has completed (one phase)
+    kNumBars = 24
+};
+
+// Named barrier 1 over the softmax warps only (the producer and MMA warps never take part).
+__device__ __forceinline__ void group_sync() { asm volatile("barrier.cta.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ bool group_sync_or(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, 1, 256, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred))
+        : "memory");
+    return r != 0;
+}
 
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
     asm volatile(""
@@ -89,7 +139,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 }  // namespace
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qraw,
                       const __grid_constant__ CUtensorMap tm_out, AttnArgs a, Geom g) {
@@ -98,22 +148,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     constexpr int NC = HW / 32;   // 32-column TMEM loads per thread
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __half* sq = reinterpret_cast<__half*>(smem + Lay::kOffQ);
-    __half* sk = reinterpret_cast<__half*>(smem + Lay::kOffK);
-    __half* sv = reinterpret_cast<__half*>(smem + Lay::kOffV);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
-    uint64_t* bar_q = bars + 0;
-    uint64_t* bar_k = bars + 1;
-    uint64_t* bar_v = bars + 2;
-    uint64_t* bar_s = bars + 3;
-    uint64_t* bar_o = bars + 4;
+    uint64_t* bar_q = bars + kBarQ;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
-    float* xch = reinterpret_cast<float*>(smem + Lay::kOffXch);  // [2][128]: per-half row partials
+    float* xch = reinterpret_cast<float*>(smem + Lay::kOffXch);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int lg = warp & 3;    // TMEM lane group (rows 32*lg ..), fixed by the warp's rank in its warpgroup
-    const int hf = warp >> 2;   // which half of the key block (and of O's columns) this warp handles
+    const int hf = (warp >> 2) & 1;   // softmax warps: which half of the key block (and of O's columns)
     const int i_row = lg * 32 + lane;
     const int alpha = blockIdx.x, bh = blockIdx.y;
     const int b = bh / g.Hh, h = bh % g.Hh;
@@ -123,7 +166,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int32_t* my_idx = a.idx + (static_cast<size_t>(bh) * g.nb + alpha) * (keep > 0 ? g.keep : 0);
 
     if (tid == 0) {
-        for (int i = 0; i < 10; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < kNumBars; ++i)
+            mbar_init(bars + i, (i >= kBarPFull && i < kBarPFull + kNumS) ? kSoftThreads : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -135,234 +179,300 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem;               // S (fp32) and P (fp16 packed) columns
     const uint32_t tO = tmem + kColO;       // O accumulator
+    const uint32_t tPhi = tmem + kColPhi;   // epilogue: phi = q A
     const uint32_t lane_base = static_cast<uint32_t>(lg * 32) << 16;
-
-    const uint32_t idesc_s = idesc_f16_f32(128, blk, false, false);
-    const uint32_t idesc_o = idesc_f16_f32(128, D, false, true);
-    const uint32_t q_addr = smem_addr(sq), k_addr = smem_addr(sk), v_addr = smem_addr(sv);
-    const uint32_t kv_bytes = static_cast<uint32_t>(blk) * D * 2;
     const int row0 = bh * g.Lp;  // first row of this head in the head-major buffers
 
     auto fail = [&]() {
         *abort_flag = 1;
         atomicOr(a.status, kDevTimeout);
     };
-    auto issue_s = [&]() {  // S = q^ k^T over the D/16 k-steps
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(q_addr + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * (blk * 128) + (kk & 3) * 32, 16, 1024);
-            umma_ss(tS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_s);
-    };
-    auto load_kv = [&](uint64_t* bar, __half* dst, const CUtensorMap* tm, int beta) {
-        mbar_expect_tx(bar, kv_bytes);
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s)
-            tma_load_2d(reinterpret_cast<uint8_t*>(dst) + s * (blk * 128), tm, bar, s * 64, row0 + beta * blk);
-    };
+    // Test hook: wait on a barrier that nothing arrives at; the bounded wait runs out, records a timeout
+    // and every role sees the abort flag before any copy or product has been issued.
+    if (a.debug_unsatisfied_wait && tid == 0 && !mbar_wait(bars + kBarDebug, 0, tmo, abort_flag)) fail();
+    __syncthreads();
 
-    // Operations issued / observed complete per barrier (thread 0 only), so an aborted CTA can drain
-    // what is still in flight before it releases shared and tensor memory.
-    int n_q_issued = 0, n_q_done = 0, n_k_issued = 0, n_k_done = 0, n_v_issued = 0, n_v_done = 0;
-    int n_s_issued = 0, n_s_done = 0, n_o_issued = 0, n_o_done = 0;
-    // Thread 0 keeps the kept-block indices one iteration ahead in registers (the loads stay off the
-    // softmax's critical path): beta_cur = block of the next v tile to load, beta_next = of the next k tile.
-    int beta_cur = 0, beta_next = 0;
-    // epilogue barrier bookkeeping (thread 0 for the loads; every thread for the products)
-    int n_eld_issued = 0, n_eld = 0, n_emm_issued = 0, n_emm = 0, n_ez_issued = 0, n_ez = 0;
-    uint64_t* bar_eld = bars + 5;  // epilogue: raw query tile + A^T image (one phase)
-    uint64_t* bar_ez = bars + 9;   // epilogue: S image of each 64-feature chunk (one phase per chunk)
-    uint64_t* bar_emm = bars + 6;  // epilogue products
-    // The low-rank readout's raw query tile and A^T image are loaded during the last key block, into
-    // the q and k tiles (free once the last S product is done).
     const bool prefetch_epi = (D == 128) && a.lowrank && keep > 0;
+    // epilogue barrier bookkeeping (softmax thread 0 for the loads; every softmax thread for the products)
+    int n_eld_issued = 0, n_eld = 0, n_emm_issued = 0, n_emm = 0, n_ez_issued = 0, n_ez = 0;
+    uint64_t* bar_eld = bars + kBarEld;
+    uint64_t* bar_ez = bars + kBarEz;
+    uint64_t* bar_emm = bars + kBarEmm;
+    // The low-rank readout's raw query tile and A^T image go to the q tile and k slot 0, the first
+    // chunk's S image (rank <= 64) right after them; all are free once the last S has completed.
     auto issue_epilogue_prefetch = [&]() {
         mbar_expect_tx(bar_eld, 32768 + g.R * 256);
         tma_load_4d(smem, &tm_qraw, bar_eld, 0, h, alpha * blk, b);
         tma_load_4d(smem + 16384, &tm_qraw, bar_eld, 64, h, alpha * blk, b);
         bulk_load(smem + 32768, a.at_img, g.R * 256, bar_eld);
         ++n_eld_issued;
+        if (g.R <= 64) {
+            const uint32_t zb = static_cast<uint32_t>((3 * g.R + 63) / 64) * (D * 128);
+            mbar_expect_tx(bar_ez, zb);
+            bulk_load(smem + 49152, a.sb_img + static_cast<size_t>(bh) * ((g.R + 63) / 64) * kSbChunkBytes, zb,
+                      bar_ez);
+            ++n_ez_issued;
+        }
     };
 
-    // Test hook: wait on a barrier that nothing arrives at (bars[7]); the bounded wait runs out, records
-    // a timeout and every thread sees the abort flag before any copy or product has been issued.
-    if (a.debug_unsatisfied_wait && tid == 0 && !mbar_wait(bars + 7, 0, tmo, abort_flag)) fail();
-    __syncthreads();
-
-    // ------------------------------------------------------------------ prologue: Q, K0, V0, S0
-    if (keep > 0 && tid == 0 && !*abort_flag) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-        mbar_expect_tx(bar_q, 128 * D * 2);
+    float l_run = 0.f;
+    if (warp == kWarpLoad) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0 && keep > 0 && !*abort_flag) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            auto load_tile = [&](uint64_t* bar, uint8_t* dst, const CUtensorMap* tm, int row, int rows) {
+                mbar_expect_tx(bar, static_cast<uint32_t>(rows) * D * 2);
 #pragma unroll
-        for (int s = 0; s < D / 64; ++s)
-            tma_load_2d(reinterpret_cast<uint8_t*>(sq) + s * (128 * 128), &tm_q, bar_q, s * 64, row0 + alpha * blk);
-        const int beta0 = my_idx[0];
-        beta_next = keep > 1 ? __ldg(my_idx + 1) : 0;
-        load_kv(bar_k, sk, &tm_k, beta0);
-        load_kv(bar_v, sv, &tm_v, beta0);
-        n_q_issued = 1; n_k_issued = 1; n_v_issued = 1;
-        if (mbar_wait(bar_q, 0, tmo, abort_flag)) n_q_done = 1;
-        if (n_q_done && mbar_wait(bar_k, 0, tmo, abort_flag)) {
-            n_k_done = 1;
-            tc_fence_after();
-            issue_s();
-            n_s_issued = 1;
-        } else {
-            fail();
-        }
-    }
-
-    const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-    // The kept list is ascending, so the only block that can be partial (the sequence's last) can only
-    // be the last one visited.
-    const int last_valid = keep > 0 ? min(blk, g.L - __ldg(my_idx + keep - 1) * blk) : blk;
-    const int key0 = hf * HW;  // first key of this thread's half of the block
-    // m_run is the row's running max (identical in both halves); l_run sums this half's keys only.
-    float m_run = 0.f, l_run = 0.f;
-    for (int j = 0; j < keep; ++j) {
-        // warp-uniform, since the TMEM loads below are warp-collective
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, tmo, abort_flag));
-        tc_fence_after();
-        if (tid == 0 && ok) {
-            ++n_s_done;
-            // S_j has finished reading the k tile and (issued before it) P.V_{j-1} the v tile: load v_j
-            // and k_{j+1}.
-            if (j > 0) { load_kv(bar_v, sv, &tm_v, beta_cur); ++n_v_issued; }
-            if (j + 1 < keep) { load_kv(bar_k, sk, &tm_k, beta_next); ++n_k_issued; }
-            beta_cur = beta_next;
-            if (j + 2 < keep) beta_next = __ldg(my_idx + j + 2);
-            if (j == keep - 1 && prefetch_epi) issue_epilogue_prefetch();  // q and k tiles are free now
-        }
-        // ---- softmax of row i_row over keys [key0, key0 + HW); O is stable (P.V_{j-1} completed
-        //      before S_j)
-        uint32_t sr[NC][32];
-        if (ok) {
-#pragma unroll
-            for (int c = 0; c < NC; ++c) tmem_ld32(tS + lane_base + key0 + c * 32, sr[c]);
-            tmem_ld_wait(sr[0]);
-#pragma unroll
-            for (int c = 1; c < NC; ++c) reg_fence(sr[c]);
-        }
-        constexpr int NE = HW;  // elements this thread owns
-        auto el = [&](int e) -> uint32_t& { return sr[e >> 5][e & 31]; };
-        if (j == keep - 1 && last_valid < blk) {
-#pragma unroll
-            for (int e = 0; e < NE; ++e)
-                if (key0 + e >= last_valid) el(e) = __float_as_uint(-INFINITY);
-        }
-        // row max over this half: four independent chains of 3-input max
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int e = 0; e < NE; e += 8) {
-#pragma unroll
-            for (int t = 0; t < 4; ++t)
-                mx4[t] = fmax3(mx4[t], __uint_as_float(el(e + 2 * t)), __uint_as_float(el(e + 2 * t + 1)));
-        }
-        const float mx_half = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
-        xch[hf * 128 + i_row] = mx_half;
-        // One barrier exchanges the two halves' maxima, makes the abort decision uniform, and orders
-        // every thread's S loads before the P stores below (half 1's P columns overlap half 0's S).
-        tc_fence_before();
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) fail();
-            break;
-        }
-        tc_fence_after();
-        float mx = fmaxf(mx_half, xch[(hf ^ 1) * 128 + i_row]);  // same value in both halves
-        mx *= scale_log2;
-        if (j == 0) {
-            m_run = mx;
-        } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {  // warp-uniform: TMEM access is collective
-            // Both warps of the lane group see the same maxima, so they take the same branch; each
-            // rescales its half of O's columns.
-            const float m_new = fmaxf(m_run, mx);
-            const float alpha_r = ex2_approx(m_run - m_new);
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {  // 16 columns at a time (the scores stay in registers)
-                uint32_t o[16];
-                tmem_ld16(tO + lane_base + hf * (D / 2) + c * 16, o);
-                tmem_ld_wait(o);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha_r);
-                tmem_st16(tO + lane_base + hf * (D / 2) + c * 16, o);
+                for (int s = 0; s < D / 64; ++s) tma_load_2d(dst + s * (rows * 128), tm, bar, s * 64, row);
+            };
+            auto kslot = [&](int s) { return smem + Lay::kOffK + s * Lay::kTile; };
+            auto vslot = [&](int s) { return smem + Lay::kOffV + s * Lay::kTile; };
+            int nk = 0, nv = 0;  // tiles issued
+            bool ok = true;
+            load_tile(bar_q, smem + Lay::kOffQ, &tm_q, row0 + alpha * blk, 128);
+            load_tile(bars + kBarKFull, kslot(0), &tm_k, row0 + __ldg(my_idx) * blk, blk);
+            nk = 1;
+            if (keep > 1) {
+                load_tile(bars + kBarKFull + 1, kslot(1), &tm_k, row0 + __ldg(my_idx + 1) * blk, blk);
+                nk = 2;
             }
-            tmem_st_wait();
-            l_run *= alpha_r;
-            m_run = m_new;
-        }
-        const float neg_m = -m_run;
-        float sums[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};  // independent accumulators
-        // keys (2i, 2i+1) of this half -> packed fp16x2 TMEM column key0/2 + i, 16 columns at a time
-#pragma unroll
-        for (int c16 = 0; c16 < NE / 32; ++c16) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int i = c16 * 16 + u;
-                float t0, t1;
-                ffma2(t0, t1, __uint_as_float(el(2 * i)), __uint_as_float(el(2 * i + 1)), scale_log2, scale_log2,
-                      neg_m, neg_m);
-                const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-                fadd2(sums[u & 3][0], sums[u & 3][1], p0, p1);
-                pk[u] = pack_half2(p0, p1);
-            }
-            tmem_st16(tS + lane_base + key0 / 2 + c16 * 16, pk);
-        }
-        tmem_st_wait();
-        l_run += ((sums[0][0] + sums[0][1]) + (sums[1][0] + sums[1][1])) +
-                 ((sums[2][0] + sums[2][1]) + (sums[3][0] + sums[3][1]));
-        tc_fence_before();
-        __syncthreads();
-        // ---- issue O += P v, then immediately the next S (tensor-core operations issued by one thread
-        //      run in order, so S_{j+1} overwrites the P columns only after P.V_j has read them)
-        if (warp == 0) {
-            if (lane == 0 && !*abort_flag) {
-                tc_fence_after();
-                if (!mbar_wait(bar_v, j & 1, tmo, abort_flag)) {
-                    fail();
-                } else {
-                    ++n_v_done;
-#pragma unroll
-                    for (int kk = 0; kk < BLK / 16; ++kk) {
-                        const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, static_cast<uint32_t>(blk) * 128, 1024);
-                        umma_ts(tO, tS + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int j = 0; j < keep && ok; ++j) {
+                const int s = j & 1;
+                // v_j into slot s once P.V_{j-2} (the slot's previous reader) has completed
+                if (j >= 2 && !mbar_wait(bars + kBarVEmpty + s, ((j - 2) >> 1) & 1, tmo, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                load_tile(bars + kBarVFull + s, vslot(s), &tm_v, row0 + __ldg(my_idx + j) * blk, blk);
+                ++nv;
+                // k_{j+2} into slot s once S_j has completed
+                if (j + 2 < keep) {
+                    if (!mbar_wait(bars + kBarKEmpty + s, (j >> 1) & 1, tmo, abort_flag)) {
+                        ok = false;
+                        break;
                     }
-                    if (j + 1 < keep) {
-                        if (mbar_wait(bar_k, (j + 1) & 1, tmo, abort_flag)) {
-                            ++n_k_done;
-                            issue_s();  // commits bar_s, which also covers this P.V
-                            ++n_s_issued;
-                        } else {
-                            umma_commit(bar_o);
-                            ++n_o_issued;
-                            fail();
-                        }
-                    } else {
-                        umma_commit(bar_o);
-                        ++n_o_issued;
-                    }
+                    load_tile(bars + kBarKFull + s, kslot(s), &tm_k, row0 + __ldg(my_idx + j + 2) * blk, blk);
+                    ++nk;
                 }
             }
-            __syncwarp();
+            if (!ok) {
+                fail();
+                // let every issued copy land (bounded, ignoring the abort flag)
+                volatile int no_abort = 0;
+                const uint64_t drain = 10000000ull;
+                mbar_wait(bar_q, 0, drain, &no_abort);
+                for (int n = nk - 2 < 0 ? 0 : nk - 2; n < nk; ++n)
+                    mbar_wait(bars + kBarKFull + (n & 1), (n >> 1) & 1, drain, &no_abort);
+                for (int n = nv - 2 < 0 ? 0 : nv - 2; n < nv; ++n)
+                    mbar_wait(bars + kBarVFull + (n & 1), (n >> 1) & 1, drain, &no_abort);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kWarpMma) {
+        // ---------------------------------------------------------------- tcgen05.mma issuer
+        if (lane == 0 && keep > 0 && !*abort_flag) {
+            const uint32_t idesc_s = idesc_f16_f32(128, blk, false, false);
+            const uint32_t idesc_o = idesc_f16_f32(128, D, false, true);
+            const uint32_t q_addr = smem_addr(smem + Lay::kOffQ);
+            // Operand descriptors per slot, computed once; a k-step adds a compile-time offset to the
+            // 14-bit address field (shared-memory addresses stay below 2^18, so it cannot carry out).
+            // The issuing warp shares its sub-partition with two busy softmax warps, so every issue
+            // slot it saves shows up as tensor-pipe throughput.
+            const uint64_t dq = sdesc_sw128(q_addr, 16, 1024);
+            const uint64_t dk0 = sdesc_sw128(smem_addr(smem + Lay::kOffK), 16, 1024);
+            const uint64_t dk1 = sdesc_sw128(smem_addr(smem + Lay::kOffK + Lay::kTile), 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(smem_addr(smem + Lay::kOffV), static_cast<uint32_t>(blk) * 128, 1024);
+            const uint64_t dv1 = sdesc_sw128(smem_addr(smem + Lay::kOffV + Lay::kTile), static_cast<uint32_t>(blk) * 128, 1024);
+            auto s_step = [&](uint32_t dst, uint64_t dkj, int kk) {  // k-step kk of S = q^ k^T
+                const uint32_t qo = static_cast<uint32_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+                const uint32_t ko = static_cast<uint32_t>(((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4);
+                umma_ss(dst, dq + qo, dkj + ko, idesc_s, kk > 0 ? 1u : 0u);
+            };
+            auto s_done = [&](int j) {
+                umma_commit(bars + kBarSFull + j % kNumS);
+                umma_commit(bars + kBarKEmpty + (j & 1));
+            };
+            auto pv_step = [&](uint32_t p, uint64_t dvj, int kk, uint32_t acc) {  // k-step kk of O += P v
+                umma_ts(tO, p + kk * 8, dvj + static_cast<uint32_t>((kk * 2048) >> 4), idesc_o, acc);
+            };
+            auto pv_done = [&](int j) {
+                umma_commit(bars + kBarVEmpty + (j & 1));
+                umma_commit(bars + kBarODone + j % kNumS);
+                if (j == keep - 1) umma_commit(bars + kBarOFinal);
+            };
+            constexpr int kSSteps = D / 16, kPvSteps = BLK / 16;
+            bool ok = mbar_wait(bar_q, 0, tmo, abort_flag);
+            for (int j = 0; j < 2 && j < keep && ok; ++j) {  // S_0, S_1 have no P.V to pair with
+                ok = mbar_wait(bars + kBarKFull + j, 0, tmo, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t dst = tmem + j * 128;
+#pragma unroll
+                    for (int kk = 0; kk < kSSteps; ++kk) s_step(dst, j ? dk1 : dk0, kk);
+                    s_done(j);
+                }
+            }
+            for (int j = 0; j < keep && ok; ++j) {
+                // P.V_j paired with S_{j+2}, whose buffer held P_{j-1} (read by P.V_{j-1}, issued earlier
+                // from this thread: products run in order)
+                const bool has_s = j + 2 < keep;
+                if (!mbar_wait(bars + kBarPFull + j % kNumS, (j / kNumS) & 1, tmo, abort_flag) ||
+                    !mbar_wait(bars + kBarVFull + (j & 1), (j >> 1) & 1, tmo, abort_flag) ||
+                    (has_s && !mbar_wait(bars + kBarKFull + (j & 1), ((j + 2) >> 1) & 1, tmo, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t pj = tmem + (j % kNumS) * 128, s2 = tmem + ((j + 2) % kNumS) * 128;
+                const uint64_t dvj = (j & 1) ? dv1 : dv0, dkj = (j & 1) ? dk1 : dk0;
+                const uint32_t acc0 = j > 0 ? 1u : 0u;
+                if (has_s) {
+#pragma unroll
+                    for (int t = 0; t < (kSSteps > kPvSteps ? kSSteps : kPvSteps); ++t) {
+                        if (t < kPvSteps) pv_step(pj, dvj, t, t > 0 ? 1u : acc0);
+                        if (t < kSSteps) s_step(s2, dkj, t);
+                    }
+                } else {
+#pragma unroll
+                    for (int t = 0; t < kPvSteps; ++t) pv_step(pj, dvj, t, t > 0 ? 1u : acc0);
+                }
+                pv_done(j);
+                if (has_s) s_done(j + 2);
+            }
+            if (!ok) {
+                fail();
+                // one more commit tracks every product issued so far (they complete in order)
+                umma_commit(bars + kBarDrain);
+                volatile int no_abort = 0;
+                mbar_wait(bars + kBarDrain, 0, 10000000ull, &no_abort);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- softmax warps
+        const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+        // The kept list is ascending, so the only block that can be partial (the sequence's last) can
+        // only be the last one visited.
+        const int last_valid = keep > 0 ? min(blk, g.L - __ldg(my_idx + keep - 1) * blk) : blk;
+        const int key0 = hf * HW;  // first key of this thread's half of the block
+        // m_run is the row's running max (identical in both halves); l_run sums this half's keys only.
+        float m_run = 0.f;
+        for (int j = 0; j < keep; ++j) {
+            const int sb = j % kNumS;
+            const uint32_t tSj = tmem + sb * 128;
+            // warp-uniform, since the TMEM loads below are warp-collective
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(bars + kBarSFull + sb, (j / kNumS) & 1, tmo, abort_flag));
+            tc_fence_after();
+            if (tid == 0 && ok && j == keep - 1 && prefetch_epi) issue_epilogue_prefetch();  // all S done
+            // ---- softmax of row i_row over keys [key0, key0 + HW)
+            uint32_t sr[NC][32];
+            if (ok) {
+#pragma unroll
+                for (int c = 0; c < NC; ++c) tmem_ld32(tSj + lane_base + key0 + c * 32, sr[c]);
+                tmem_ld_wait(sr[0]);
+#pragma unroll
+                for (int c = 1; c < NC; ++c) reg_fence(sr[c]);
+            }
+            constexpr int NE = HW;  // elements this thread owns
+            auto el = [&](int e) -> uint32_t& { return sr[e >> 5][e & 31]; };
+            if (j == keep - 1 && last_valid < blk) {
+#pragma unroll
+                for (int e = 0; e < NE; ++e)
+                    if (key0 + e >= last_valid) el(e) = __float_as_uint(-INFINITY);
+            }
+            // row max over this half: four independent chains of 3-input max
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int e = 0; e < NE; e += 8) {
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    mx4[t] = fmax3(mx4[t], __uint_as_float(el(e + 2 * t)), __uint_as_float(el(e + 2 * t + 1)));
+            }
+            const float mx_half = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+            float* xj = xch + (j & 1) * 256;  // by parity, so a fast thread's next write cannot meet this read
+            xj[hf * 128 + i_row] = mx_half;
+            // One barrier exchanges the two halves' maxima, makes the abort decision uniform, and orders
+            // every thread's S loads before the P stores below (half 1's P columns overlap half 0's S).
+            tc_fence_before();
+            if (group_sync_or(!ok)) {
+                if (tid == 0) fail();
+                break;
+            }
+            tc_fence_after();
+            float mx = fmaxf(mx_half, xj[(hf ^ 1) * 128 + i_row]);  // same value in both halves
+            mx *= scale_log2;
+            if (j == 0) {
+                m_run = mx;
+            } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {  // warp-uniform: TMEM access is collective
+                // Both warps of the lane group see the same maxima, so they take the same branch; each
+                // rescales its half of O's columns once P.V_{j-1} has landed in O.
+                // (per-buffer barriers: when S_j has completed, P.V_{j-2} may or may not have, so one
+                // shared counter could be three phases from here)
+                const bool landed = __all_sync(0xffffffffu, mbar_wait(bars + kBarODone + (j - 1) % kNumS,
+                                                                      ((j - 1) / kNumS) & 1, tmo, abort_flag));
+                tc_fence_after();
+                const float m_new = fmaxf(m_run, mx);
+                const float alpha_r = ex2_approx(m_run - m_new);
+                if (landed) {
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {  // 16 columns at a time (the scores stay in registers)
+                        uint32_t o[16];
+                        tmem_ld16(tO + lane_base + hf * (D / 2) + c * 16, o);
+                        tmem_ld_wait(o);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha_r);
+                        tmem_st16(tO + lane_base + hf * (D / 2) + c * 16, o);
+                    }
+                    tmem_st_wait();
+                } else if (lane == 0) {
+                    fail();
+                }
+                l_run *= alpha_r;
+                m_run = m_new;
+            }
+            const float neg_m = -m_run;
+            float sums[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};  // independent accumulators
+            // keys (2i, 2i+1) of this half -> packed fp16x2 TMEM column key0/2 + i, 16 columns at a time
+#pragma unroll
+            for (int c16 = 0; c16 < NE / 32; ++c16) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int i = c16 * 16 + u;
+                    float t0, t1;
+                    ffma2(t0, t1, __uint_as_float(el(2 * i)), __uint_as_float(el(2 * i + 1)), scale_log2, scale_log2,
+                          neg_m, neg_m);
+                    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                    fadd2(sums[u & 3][0], sums[u & 3][1], p0, p1);
+                    pk[u] = pack_half2(p0, p1);
+                }
+                tmem_st16(tSj + lane_base + key0 / 2 + c16 * 16, pk);
+            }
+            tmem_st_wait();
+            l_run += ((sums[0][0] + sums[0][1]) + (sums[1][0] + sums[1][1])) +
+                     ((sums[2][0] + sums[2][1]) + (sums[3][0] + sums[3][1]));
+            tc_fence_before();
+            mbar_arrive(bars + kBarPFull + sb);  // P_j of this thread's row half is in TMEM
         }
     }
+
+    // ==================================================================== softmax warps: epilogue
+    if (warp < kSoftWarps) {
     if (keep > 0) {  // the last P.V has landed in O
-        const bool ok = !*abort_flag && mbar_wait(bar_o, 0, tmo, abort_flag);
-        if (__syncthreads_or(!ok) && tid == 0) fail();
-        if (tid == 0 && ok) ++n_o_done;
+        const bool ok = !*abort_flag && mbar_wait(bars + kBarOFinal, 0, tmo, abort_flag);
+        if (group_sync_or(!ok) && tid == 0) fail();
     }
     // Row sum: the two halves' partial sums (fp32 addition commutes, so both get the same total).
     xch[hf * 128 + i_row] = l_run;
-    __syncthreads();
+    group_sync();
     l_run += xch[(hf ^ 1) * 128 + i_row];
+    // The producer and MMA warps may raise the abort flag at any time, so every decision that picks a
+    // path through the group barriers is taken from one reduction.
+    const bool aborted = group_sync_or(*abort_flag != 0);  // also: the exchange buffer is reused below
     tc_fence_after();
-    const bool aborted = *abort_flag != 0;
 
     // ------------------------------------------------------------------ epilogue
     const int n = alpha * blk + i_row;
@@ -372,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if constexpr (D == 128) {
         if (a.lowrank && !aborted) {
             // Low-rank readout on the tensor cores, accumulated straight into O (so out = O / l):
-            //   phi = q A        raw bf16 query tile (TMA) x A^T image, into the free S columns;
+            //   phi = q A        raw bf16 query tile (TMA) x A^T image, into TMEM columns of its own;
             //   psi = R_r(p) relu(phi) * l / (relu(phi) . z + 1e-6), split into bf16 hi + lo;
             //   O  += psi S      as psi_hi S_hi + psi_hi S_lo + psi_lo S_hi, one 64-feature chunk at a time.
             // The two warps of a lane group share each row: 32-feature column groups of the
@@ -391,12 +501,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             // bar_eld: raw query tile + A^T image (prefetched during the last key block when there is
             // one); bar_ez: the S image of each chunk in turn
             if (tid == 0) {
-                if (!prefetch_epi) issue_epilogue_prefetch();
-                if (z_early) {  // the v tile is free (the last P.V is done)
-                    mbar_expect_tx(bar_ez, sb_bytes(0));
-                    bulk_load(Z, sb_head, sb_bytes(0), bar_ez);
-                    ++n_ez_issued;
-                }
+                if (!prefetch_epi) issue_epilogue_prefetch();  // also chunk 0's S image when rank <= 64
                 if (mbar_wait(bar_eld, n_eld & 1, tmo, abort_flag)) {
                     ++n_eld;
                     tc_fence_after();
@@ -405,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t ad = sdesc_sw128(smem_addr(X) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
                         const uint64_t bd = sdesc_sw128(smem_addr(Y) + (kk >> 2) * (R * 128) + (kk & 3) * 32, 16, 1024);
-                        umma_ss(tS, ad, bd, idesc_phi, kk > 0 ? 1u : 0u);
+                        umma_ss(tPhi, ad, bd, idesc_phi, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(bar_emm);
                     ++n_emm_issued;
@@ -414,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
             bool ok = mbar_wait(bar_emm, n_emm & 1, tmo, abort_flag);
-            if (__syncthreads_or(!ok)) {
+            if (group_sync_or(!ok)) {
                 if (tid == 0) fail();
             } else {
                 ++n_emm;
@@ -431,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int c0 = hf * 32; c0 < 128; c0 += 64) {
                     if (c0 < R) {
                         uint32_t v[32];
-                        tmem_ld32(tS + lane_base + c0, v);
+                        tmem_ld32(tPhi + lane_base + c0, v);
                         tmem_ld_wait(v);
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
@@ -439,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
                 xch[hf * 128 + i_row] = den;
-                __syncthreads();
+                group_sync();
                 den += xch[(hf ^ 1) * 128 + i_row];  // same total in both halves
                 const float l_eff = keep > 0 ? l_run : 1.f;
                 const float scale = l_eff / (den + 1e-6f);
@@ -450,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const int rc = min(64, R - 64 * ch);
                     if (ch > 0) {  // the previous chunk's product must have finished with X and Z
                         ok = mbar_wait(bar_emm, n_emm & 1, tmo, abort_flag);
-                        if (__syncthreads_or(!ok)) {
+                        if (group_sync_or(!ok)) {
                             if (tid == 0) fail();
                             ok = false;
                             break;
@@ -487,8 +592,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                             rot[b8 * 8 + t] = make_float2(static_cast<float>(cs[t].x), static_cast<float>(cs[t].y));
                     }
                     uint32_t va[16], vb[16];
-                    tmem_ld16(tS + lane_base + 64 * ch + 16 * hf, va);
-                    tmem_ld16(tS + lane_base + 64 * ch + 32 + 16 * hf, vb);
+                    tmem_ld16(tPhi + lane_base + 64 * ch + 16 * hf, va);
+                    tmem_ld16(tPhi + lane_base + 64 * ch + 32 + 16 * hf, vb);
                     tmem_ld_wait(va);
                     asm volatile("" : "+r"(vb[0]), "+r"(vb[1]), "+r"(vb[2]), "+r"(vb[3]), "+r"(vb[4]), "+r"(vb[5]),
                                  "+r"(vb[6]), "+r"(vb[7]), "+r"(vb[8]), "+r"(vb[9]), "+r"(vb[10]), "+r"(vb[11]),
@@ -516,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                     fence_async_smem();
                     tc_fence_before();
-                    __syncthreads();
+                    group_sync();
                     if (tid == 0 && !*abort_flag) {
                         if (mbar_wait(bar_ez, n_ez & 1, tmo, abort_flag)) {
                             ++n_ez;
@@ -536,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 if (ok) {
                     ok = !*abort_flag && mbar_wait(bar_emm, n_emm & 1, tmo, abort_flag);
-                    if (__syncthreads_or(!ok)) {
+                    if (group_sync_or(!ok)) {
                         if (tid == 0) fail();
                     } else {
                         ++n_emm;
@@ -558,8 +663,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int e = 0; e < DH; ++e) acc[e] = 0.f;
         if (a.lowrank && !aborted) {
             float* As = reinterpret_cast<float*>(smem);  // [D][R] fp32, reuses the tile buffers
-            for (int e = tid; e < D * g.R; e += kThreads) As[e] = __bfloat162float(a.A[e]);
-            __syncthreads();
+            for (int e = tid; e < D * g.R; e += kSoftThreads) As[e] = __bfloat162float(a.A[e]);
+            group_sync();
             if (row_valid) {
                 const __nv_bfloat16* qrow = a.q_raw + ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;
                 const float* Sh = a.S + static_cast<size_t>(bh) * g.R * D + hf * DH;
@@ -616,9 +721,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     //      row into a 128-B-swizzled staging tile (conflict-free 16-byte stores), then 64-row TMA stores
     //      write it out; tokens past L are clipped by the tensor map and a 64-token block's second half
     //      is skipped.
-    const bool aborted2 = *abort_flag != 0;
+    const bool aborted2 = group_sync_or(*abort_flag != 0);  // every product that read the tile buffers has completed
     if (!aborted2) {
-        __syncthreads();  // every product that read the tile buffers has completed
 #pragma unroll
         for (int cc = 0; cc < D / 64; ++cc) {
             const int c = hf * (D / 64) + cc;  // 32-column group of O
@@ -661,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         fence_async_smem();
-        __syncthreads();
+        group_sync();
         if (tid == 0) {
             const int cols_per_box = a.out_bf16 ? 64 : 32;
             const int boxes = D / cols_per_box;
@@ -674,21 +778,18 @@ __global__ void __launch_bounds__(kThreads, 2)
             tma_store_commit_and_wait();
         }
     }
-    // ------------------------------------------------------------------ teardown
+    // ------------------------------------------------------------------ teardown (softmax warps)
     if (*abort_flag && tid == 0) {
-        // Let copies and products still in flight land before the memory is released.  Each wait is
-        // bounded (10 ms) and ignores the abort flag.
+        // Let the epilogue's copies and products still in flight land before the memory is released.
+        // Each wait is bounded (10 ms) and ignores the abort flag.
         volatile int no_abort = 0;
         const uint64_t drain = 10000000ull;
-        if (n_q_issued > n_q_done) mbar_wait(bar_q, 0, drain, &no_abort);
-        if (n_k_issued > n_k_done) mbar_wait(bar_k, n_k_done & 1, drain, &no_abort);
-        if (n_v_issued > n_v_done) mbar_wait(bar_v, n_v_done & 1, drain, &no_abort);
-        if (n_s_issued > n_s_done) mbar_wait(bar_s, n_s_done & 1, drain, &no_abort);
-        if (n_o_issued > n_o_done) mbar_wait(bar_o, n_o_done & 1, drain, &no_abort);
         if (n_eld_issued > n_eld) mbar_wait(bar_eld, n_eld & 1, drain, &no_abort);
         if (n_ez_issued > n_ez) mbar_wait(bar_ez, n_ez & 1, drain, &no_abort);
         if (n_emm_issued > n_emm) mbar_wait(bar_emm, n_emm & 1, drain, &no_abort);
     }
+    }  // softmax warps
+    // ------------------------------------------------------------------ teardown (all warps)
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
