@@ -63,7 +63,8 @@ typedef struct CUstream_st* slra_stream_t;
 typedef enum slra_status {
     SLRA_OK = 0,
     SLRA_ERR_INVALID_ARG = 1,     /* NULL pointer, non-positive size, L overflow, keep_frac outside (0,1] */
-    SLRA_ERR_UNSUPPORTED = 2,     /* valid but not implemented: head_dim, block, rank, too many blocks  */
+    SLRA_ERR_UNSUPPORTED = 2,     /* valid but not implemented: head_dim, block, rank, more than 2048
+                                     blocks, more than 65535 batch x heads                               */
     SLRA_ERR_ALIGNMENT = 3,       /* a pointer is not 16-byte aligned                                   */
     SLRA_ERR_WORKSPACE = 4,       /* workspace NULL, misaligned (256 B) or smaller than required         */
     SLRA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or a kernel launch failed                */

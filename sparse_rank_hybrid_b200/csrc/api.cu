@@ -55,6 +55,7 @@ slra_status derive(const slra_problem* p, Derived* d) {
     const int64_t nb = (L + p->block - 1) / p->block;
     if (nb > kMaxBlocks) return SLRA_ERR_UNSUPPORTED;
     const int64_t BH = p->batch * p->heads;
+    if (BH > 65535) return SLRA_ERR_UNSUPPORTED;  // a launch grid dimension
     if (BH * nb * p->block >= (int64_t(1) << 31)) return SLRA_ERR_UNSUPPORTED;  // TMA row coordinate
     int64_t split[3];
     if (!default_split(p->head_dim, p->rope_split, split)) return SLRA_ERR_INVALID_ARG;
@@ -212,9 +213,12 @@ unsigned long long timeout_of(const slra_problem* p) {
 slra_status run_select(const slra_problem* p, const Derived& d, const Ptrs& w, const void* q, const void* k,
                        const void* v, cudaStream_t st) {
     const Geom& g = d.g;
-    cudaError_t e = launch_rope_pool(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                                     static_cast<const __nv_bfloat16*>(v), w.tab, w.pairs, g, w.qh, w.kh, w.vh,
-                                     w.qbar, w.kbar, w.status, st);
+    CUtensorMap mq, mk, mv;  // token-major inputs, boxes of 64 columns x one key block of tokens
+    if (!make_map_tokens(&mq, q, g.B, g.L, g.Hh, g.D, g.block) || !make_map_tokens(&mk, k, g.B, g.L, g.Hh, g.D, g.block) ||
+        !make_map_tokens(&mv, v, g.B, g.L, g.Hh, g.D, g.block))
+        return SLRA_ERR_CUDA;
+    cudaError_t e = launch_rope_pool(mq, mk, mv, w.tab, w.pairs, g, w.qh, w.kh, w.vh, w.qbar, w.kbar, w.status,
+                                     timeout_of(p), st);
     if (e != cudaSuccess) return SLRA_ERR_CUDA;
     slra_status s = mark(p, 2, st);
     if (s != SLRA_OK) return s;

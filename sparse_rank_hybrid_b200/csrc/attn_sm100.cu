@@ -570,26 +570,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     // This thread's 16 rotation pairs of the chunk: features [16hf, 16hf + 16) and
                     // [32 + 16hf, 48 + 16hf) (so both warps of a lane group have work when rc <= 32).
-                    // Their (cos, sin) are fetched eight at a time, every load issued before any is used;
-                    // the pair table holds all D/2 rotary pairs, so pairs past the rank are still valid
-                    // entries (their results are not stored).  The pair -> (axis, table offset) map comes
-                    // from the launch parameters.
+                    // Their (cos, sin) loads are all issued before any is used; the pair table holds all
+                    // D/2 rotary pairs, so pairs past the rank are still valid entries (their results are
+                    // not stored).  The pair -> (axis, table offset) map comes from the launch parameters.
                     auto feat = [&](int t) { return t < 8 ? 16 * hf + 2 * t : 32 + 16 * hf + 2 * (t - 8); };
                     float2 rot[16];
 #pragma unroll
-                    for (int b8 = 0; b8 < 2; ++b8) {
-                        int2 pi[8];
+                    const int nrot = rc > 32 ? 16 : 8;  // the second eight lie past the rank when rc <= 32
+                    {
+                        double2 cs[16];
 #pragma unroll
-                        for (int t = 0; t < 8; ++t) pi[t] = a.pair_info[32 * ch + feat(b8 * 8 + t) / 2];
-                        double2 cs[8];
-#pragma unroll
-                        for (int t = 0; t < 8; ++t) {
-                            const int ap = pi[t].x == 0 ? axis_t : (pi[t].x == 1 ? axis_h : axis_w);
-                            cs[t] = __ldg(a.tab + pi[t].y + ap);
+                        for (int t = 0; t < 16; ++t) {
+                            if (t < nrot) {
+                                const int2 pi = a.pair_info[32 * ch + feat(t) / 2];
+                                const int ap = pi.x == 0 ? axis_t : (pi.x == 1 ? axis_h : axis_w);
+                                cs[t] = __ldg(a.tab + pi.y + ap);
+                            }
                         }
 #pragma unroll
-                        for (int t = 0; t < 8; ++t)
-                            rot[b8 * 8 + t] = make_float2(static_cast<float>(cs[t].x), static_cast<float>(cs[t].y));
+                        for (int t = 0; t < 16; ++t)
+                            if (t < nrot) rot[t] = make_float2(static_cast<float>(cs[t].x), static_cast<float>(cs[t].y));
                     }
                     uint32_t va[16], vb[16];
                     tmem_ld16(tPhi + lane_base + 64 * ch + 16 * hf, va);

@@ -36,37 +36,56 @@ cudaError_t launch_rope_table(double2* tab, int2* pairs, const RopeMeta& meta, i
     return cudaGetLastError();
 }
 
-// 16-byte read-once load that does not allocate in L1 (keeps L1 for the rotary table).
-__device__ __forceinline__ uint4 ldg_stream(const __nv_bfloat16* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
 // ------------------------------------------------------------------------------ rope_pool
-// One CTA per (query/key block, batch*head).  Thread t owns four consecutive rotary pairs (8 elements,
-// 16 bytes) j = 4*(t % (D/8)) .. +3 and walks the block's tokens with stride 256/(D/8); each access of
-// q, k, v and of the fp16 outputs is one 16-byte load or store, and the D/8 threads of a token cover
-// its 256-byte row.  The rotation and the block sums are fp64 so the selection scores are exact to
-// ~1e-15 relative (the top-k decision is made on them); the fp16 copies come from the same values.
+// One CTA per (query/key block, batch*head), two CTAs per SM.  Thread 0 brings the block's q, k and v
+// rows of this head into shared memory with TMA (token-major 4D maps, 64-column boxes, 128-B swizzle;
+// tokens past L read as zero), so a whole block's 3 x block x 2D bytes are in flight at once.  Then
+// thread t owns four consecutive rotary pairs (8 elements, 16 bytes) j = 4*(t % (D/8)) .. +3 and walks
+// the block's tokens with stride 256/(D/8); each fp16 output access is one 16-byte store, and the D/8
+// threads of a token cover its row, so a block's rows go out as one contiguous stretch per tensor.
+// The rotation and the block sums are fp64 so the selection scores are exact to ~1e-15 relative (the
+// top-k decision is made on them); the fp16 copies come from the same values.
 template <int D>
-__global__ void __launch_bounds__(256) rope_pool_kernel(const __nv_bfloat16* __restrict__ q,
-                                                        const __nv_bfloat16* __restrict__ k,
-                                                        const __nv_bfloat16* __restrict__ v,
-                                                        const double2* __restrict__ tab,
-                                                        const int2* __restrict__ pairs, Geom g,
-                                                        __half* __restrict__ qh, __half* __restrict__ kh,
-                                                        __half* __restrict__ vh, double* __restrict__ qbar,
-                                                        double* __restrict__ kbar, int* status) {
+__global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                           const __grid_constant__ CUtensorMap tm_k,
+                                                           const __grid_constant__ CUtensorMap tm_v,
+                                                           const double2* __restrict__ tab,
+                                                           const int2* __restrict__ pairs, Geom g,
+                                                           __half* __restrict__ qh, __half* __restrict__ kh,
+                                                           __half* __restrict__ vh, double* __restrict__ qbar,
+                                                           double* __restrict__ kbar, int* status,
+                                                           unsigned long long timeout_ns) {
     constexpr int Q4 = D / 8;          // threads per token row
     constexpr int G = 256 / Q4;        // tokens in flight
-    __shared__ double red[G][4][4 * Q4];  // [group][q0,q1,k0,k1][pair]
+    constexpr int NS = D / 64;         // 64-column slabs per row
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
     const int quad = threadIdx.x % Q4, grp = threadIdx.x / Q4;
-    const int alpha = blockIdx.x, bh = blockIdx.y;
+    // heads vary fastest across the grid: the CTAs in flight read all heads of the same tokens, which
+    // are contiguous in the token-major inputs
+    const int bh = blockIdx.x, alpha = blockIdx.y;
     const int b = bh / g.Hh, h = bh % g.Hh;
-    const int n0 = alpha * g.block;
+    const int blk = g.block;
+    const int n0 = alpha * blk;
+    const uint32_t slab = static_cast<uint32_t>(blk) * 128;  // bytes of one 64-column slab of a tile
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&tm_q);
+        mbar_expect_tx(&bar, 3 * NS * slab);
+#pragma unroll
+        for (int s = 0; s < NS; ++s) {
+            tma_load_4d(smem + (0 * NS + s) * slab, &tm_q, &bar, 64 * s, h, n0, b);
+            tma_load_4d(smem + (1 * NS + s) * slab, &tm_k, &bar, 64 * s, h, n0, b);
+            tma_load_4d(smem + (2 * NS + s) * slab, &tm_v, &bar, 64 * s, h, n0, b);
+        }
+    }
     int axis[4], toff[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -79,23 +98,24 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const __nv_bfloat16* __r
     for (int u = 0; u < 4; ++u) sq[u][0] = sq[u][1] = sk[u][0] = sk[u][1] = 0.0;
     bool bad = false;
     const int HW = g.H * g.W;
-    const size_t row_stride = static_cast<size_t>(g.Hh) * D;  // elements between consecutive tokens
-    const size_t src0 = ((static_cast<size_t>(b) * g.L + n0) * g.Hh + h) * D + 8 * quad;
-    // software pipeline: the next token's q, k, v are in flight while this one is rotated
-    uint4 qn = make_uint4(0u, 0u, 0u, 0u), kn = qn, vn = qn;
-    if (grp < g.block && n0 + grp < g.L) {
-        const size_t src = src0 + static_cast<size_t>(grp) * row_stride;
-        qn = ldg_stream(q + src); kn = ldg_stream(k + src); vn = ldg_stream(v + src);
-    }
-    for (int i = grp; i < g.block; i += G) {
-        const int n = n0 + i;
-        const uint4 qr = qn, kr = kn, vr = vn;
-        if (i + G < g.block && n + G < g.L) {
-            const size_t src = src0 + static_cast<size_t>(i + G) * row_stride;
-            qn = ldg_stream(q + src); kn = ldg_stream(k + src); vn = ldg_stream(v + src);
+    const bool landed = mbar_wait(&bar, 0, timeout_ns, &abort_flag);
+    if (__syncthreads_or(!landed)) {
+        if (threadIdx.x == 0) {
+            atomicOr(status, kDevTimeout);
+            volatile int no_abort = 0;
+            mbar_wait(&bar, 0, 10000000ull, &no_abort);  // let the copies land before the CTA leaves
         }
+        return;
+    }
+    const uint32_t c16 = quad & 7, sl = quad >> 3;  // 16-byte chunk within its slab, slab
+    for (int i = grp; i < blk; i += G) {
+        const int n = n0 + i;
         const size_t dst = (static_cast<size_t>(bh) * g.Lp + n) * D + 8 * quad;
         if (n < g.L) {
+            const uint32_t off = sl * slab + i * 128 + ((c16 ^ (i & 7)) << 4);
+            const uint4 qr = *reinterpret_cast<const uint4*>(smem + 0 * NS * slab + off);
+            const uint4 kr = *reinterpret_cast<const uint4*>(smem + 1 * NS * slab + off);
+            const uint4 vr = *reinterpret_cast<const uint4*>(smem + 2 * NS * slab + off);
             const int pos3[3] = {n / HW, (n / g.W) % g.H, n % g.W};
             const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qr);
             const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
@@ -137,18 +157,25 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const __nv_bfloat16* __r
             *reinterpret_cast<uint4*>(vh + dst) = z4;
         }
     }
+    __syncthreads();  // the tiles are consumed; the reduction reuses their space
+    double* red = reinterpret_cast<double*>(smem);  // [G][q0,q1,k0,k1][D/2]
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
         const int j = 4 * quad + u;
-        red[grp][0][j] = sq[u][0]; red[grp][1][j] = sq[u][1];
-        red[grp][2][j] = sk[u][0]; red[grp][3][j] = sk[u][1];
+        red[(grp * 4 + 0) * (D / 2) + j] = sq[u][0];
+        red[(grp * 4 + 1) * (D / 2) + j] = sq[u][1];
+        red[(grp * 4 + 2) * (D / 2) + j] = sk[u][0];
+        red[(grp * 4 + 3) * (D / 2) + j] = sk[u][1];
     }
     __syncthreads();
     // thread t < D/2 finishes pair t: fixed-order sum over the token groups
     if (threadIdx.x < D / 2) {
         const int j = threadIdx.x;
         double a0 = 0.0, a1 = 0.0, c0 = 0.0, c1 = 0.0;
-        for (int u = 0; u < G; ++u) { a0 += red[u][0][j]; a1 += red[u][1][j]; c0 += red[u][2][j]; c1 += red[u][3][j]; }
+        for (int u = 0; u < G; ++u) {
+            a0 += red[(u * 4 + 0) * (D / 2) + j]; a1 += red[(u * 4 + 1) * (D / 2) + j];
+            c0 += red[(u * 4 + 2) * (D / 2) + j]; c1 += red[(u * 4 + 3) * (D / 2) + j];
+        }
         const int cnt = min(g.block, g.L - n0);
         const size_t o = (static_cast<size_t>(bh) * g.nb + alpha) * D + 2 * j;
         qbar[o] = a0 / cnt; qbar[o + 1] = a1 / cnt;
@@ -157,14 +184,32 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const __nv_bfloat16* __r
     if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, kDevRange);
 }
 
-cudaError_t launch_rope_pool(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+// The q, k, v tiles, or the block-sum exchange that later reuses them ([256/(D/8)][4][D/2] fp64 =
+// 32 KB for any D), whichever is larger.
+size_t rope_pool_smem_bytes(const Geom& g) {
+    const size_t tiles = static_cast<size_t>(3) * g.block * g.D * 2;
+    const size_t red = static_cast<size_t>(256 / (g.D / 8)) * 4 * (g.D / 2) * 8;
+    return (tiles > red ? tiles : red) + 1024;
+}
+
+cudaError_t launch_rope_pool(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                              const double2* tab, const int2* pairs, const Geom& g, __half* qh, __half* kh,
-                             __half* vh, double* qbar, double* kbar, int* status, cudaStream_t st) {
-    dim3 grid(g.nb, g.BH());
-    if (g.D == 128)
-        rope_pool_kernel<128><<<grid, 256, 0, st>>>(q, k, v, tab, pairs, g, qh, kh, vh, qbar, kbar, status);
-    else
-        rope_pool_kernel<64><<<grid, 256, 0, st>>>(q, k, v, tab, pairs, g, qh, kh, vh, qbar, kbar, status);
+                             __half* vh, double* qbar, double* kbar, int* status, unsigned long long timeout_ns,
+                             cudaStream_t st) {
+    dim3 grid(g.BH(), g.nb);
+    const int sm = static_cast<int>(rope_pool_smem_bytes(g));
+    cudaError_t e;
+    if (g.D == 128) {
+        e = cudaFuncSetAttribute(rope_pool_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        if (e != cudaSuccess) return e;
+        rope_pool_kernel<128><<<grid, 256, sm, st>>>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar, status,
+                                                     timeout_ns);
+    } else {
+        e = cudaFuncSetAttribute(rope_pool_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        if (e != cudaSuccess) return e;
+        rope_pool_kernel<64><<<grid, 256, sm, st>>>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar, status,
+                                                    timeout_ns);
+    }
     return cudaGetLastError();
 }
 

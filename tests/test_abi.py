@@ -66,6 +66,16 @@ def test_validation_rejects(field, value, status):
     assert slra.validate(p) == status
 
 
+def test_validation_grid_limit():
+    """batch x heads is a launch grid dimension (at most 65535); a tiny sequence keeps every other
+    limit far away, so only that one decides."""
+    p = slra.Problem.from_workload(W.TINY)
+    p.heads = 65535
+    assert slra.validate(p) == slra.OK
+    p.heads = 65536
+    assert slra.validate(p) == slra.ERR_UNSUPPORTED
+
+
 def test_calls_without_device_fail_cleanly():
     """On a machine without a GPU every compute entry point returns an error status (never crashes)."""
     import torch
