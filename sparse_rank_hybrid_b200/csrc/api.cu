@@ -234,7 +234,7 @@ cudaError_t lowrank_partial(const Derived& d, const void* k, const void* v, cons
     const auto* vb = static_cast<const __nv_bfloat16*>(v);
     const auto* Ab = static_cast<const __nv_bfloat16*>(A);
     if (d.g.D == 128)
-        return launch_lowrank_tc(kb, vb, Ab, tab, pairs, d.g, nsplit, s_part, z_part, status, timeout_ns, st);
+        return launch_lowrank_tc(kb, vb, Ab, tab, d.meta, d.g, nsplit, s_part, z_part, status, timeout_ns, st);
     return launch_lowrank_partial(kb, vb, Ab, tab, pairs, d.g, nsplit, s_part, z_part, st);
 }
 

@@ -575,7 +575,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // not stored).  The pair -> (axis, table offset) map comes from the launch parameters.
                     auto feat = [&](int t) { return t < 8 ? 16 * hf + 2 * t : 32 + 16 * hf + 2 * (t - 8); };
                     float2 rot[16];
-#pragma unroll
                     const int nrot = rc > 32 ? 16 : 8;  // the second eight lie past the rank when rc <= 32
                     {
                         double2 cs[16];

@@ -62,7 +62,8 @@ __host__ __device__ inline LrLayout lr_layout(int R) {
 struct LrArgs {
     const __nv_bfloat16* A;
     const double2* tab;
-    const int2* pairs;
+    int2 pair_info[kMaxPairs];  // per rotary pair: (axis, offset of its cos/sin table), read through the
+                                // constant cache
     float* s_part;   // [BH][nsplit][R][D]
     float* z_part;   // [BH][nsplit][R]
     int nsplit;
@@ -229,27 +230,36 @@ __global__ void __launch_bounds__(256, 1)
                     if (c0 + i < RH) raw[c0 + i] = r32[i];
             }
             const int HW = g.H * g.W;
-            const int pos3[3] = {n / HW, (n / g.W) % g.H, n % g.W};
+            const int nt = real ? n : 0;  // rows past the sequence: any valid table entry (unused)
+            const int pos_t = nt / HW, pos_h = (nt / g.W) % g.H, pos_w = nt % g.W;
 #pragma unroll
-            for (int pp = 0; pp < RH / 2; ++pp) {
+            for (int p0 = 0; p0 < RH / 2; p0 += 8) {
+                // (cos, sin) of eight pairs, every load issued before any is used
+                double2 cs[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (p0 + u < RH / 2) {
+                        const int2 pi = a.pair_info[half * (RH / 2) + p0 + u];
+                        cs[u] = __ldg(a.tab + pi.y + (pi.x == 0 ? pos_t : (pi.x == 1 ? pos_h : pos_w)));
+                    }
+                }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int pp = p0 + u;
+                if (pp >= RH / 2) break;
                 const int p = half * (RH / 2) + pp;  // global rotary pair
                 float x0 = real ? fmaxf(__uint_as_float(raw[2 * pp]), 0.f) : 0.f;
                 float x1 = real ? fmaxf(__uint_as_float(raw[2 * pp + 1]), 0.f) : 0.f;
                 zacc[2 * pp] += x0;
                 zacc[2 * pp + 1] += x1;
-                float cf = 1.f, sf = 0.f;
-                if (real) {
-                    const int2 pi = __ldg(a.pairs + p);
-                    const double2 cs = __ldg(a.tab + pi.y + pos3[pi.x]);
-                    cf = static_cast<float>(cs.x);
-                    sf = static_cast<float>(cs.y);
-                }
+                const float cf = static_cast<float>(cs[u].x), sf = static_cast<float>(cs[u].y);
                 const float y0 = x0 * cf - x1 * sf, y1 = x0 * sf + x1 * cf;
                 const __nv_bfloat162 hi = __floats2bfloat162_rn(y0, y1);
                 const float2 hf = __bfloat1622float2(hi);
                 const __nv_bfloat162 lo = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
                 *reinterpret_cast<__nv_bfloat162*>(smem + lay.off_psi + sw128_offset(row, 2 * p, kTok)) = hi;
                 *reinterpret_cast<__nv_bfloat162*>(smem + lay.off_psi + sw128_offset(row, RP + 2 * p, kTok)) = lo;
+            }
             }
             fence_async_smem();
             tc_fence_before();
@@ -363,7 +373,7 @@ static cudaError_t lr_tc_launch(const CUtensorMap& tk, const CUtensorMap& tv, co
 }
 
 cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,
-                              const double2* tab, const int2* pairs, const Geom& g, int nsplit, float* s_part,
+                              const double2* tab, const RopeMeta& meta, const Geom& g, int nsplit, float* s_part,
                               float* z_part, int* status, unsigned long long timeout_ns, cudaStream_t st) {
     CUtensorMap tk, tv;
     if (!make_map_tokens(&tk, k, g.B, g.L, g.Hh, g.D, kTok) || !make_map_tokens(&tv, v, g.B, g.L, g.Hh, g.D, kTok))
@@ -371,7 +381,8 @@ cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, co
     LrArgs a;
     a.A = A;
     a.tab = tab;
-    a.pairs = pairs;
+    for (int e = 0; e < kMaxPairs; ++e)
+        a.pair_info[e] = e < meta.npairs ? make_int2(meta.axis[e], meta.tab_off[e]) : make_int2(0, 0);
     a.s_part = s_part;
     a.z_part = z_part;
     a.nsplit = nsplit;
