@@ -59,7 +59,7 @@ def _load():
         _lib.orc_block_scores.argtypes = [P, P, I, I, P]
         _lib.orc_topk.argtypes = [P, I, I, P, P]
         _lib.orc_sparse_attn.argtypes = [P, P, P, I, I, I, P, I, P, I, P]
-        _lib.orc_features.argtypes = [P, I, I, P, I, P]
+        _lib.orc_features.argtypes = [P, I, I, P, I, ctypes.c_int, P]
         _lib.orc_summary.argtypes = [P, P, P, I, I, I, P, P]
         _lib.orc_lowrank_apply.argtypes = [P, P, P, P, I, I, P, I, P]
     return _lib
@@ -152,13 +152,17 @@ def sparse_attn(qh, kh, v, block: int, idx: np.ndarray, qblocks=None) -> np.ndar
     return out
 
 
-def features(x: np.ndarray, A: np.ndarray) -> np.ndarray:
+ACT_RELU, ACT_SILU, ACT_IDENTITY, ACT_TANH = 0, 1, 2, 3
+
+
+def features(x: np.ndarray, A: np.ndarray, act: int = ACT_RELU) -> np.ndarray:
+    """phi = act(x A): relu (default), SiLU, identity or tanh (RoLA 5.3, Table 6)."""
     x = np.ascontiguousarray(x, dtype=np.float64)
     A = np.ascontiguousarray(A, dtype=np.float64)
     L, D = x.shape
     R = A.shape[1]
     phi = np.empty((L, R), dtype=np.float64)
-    _load().orc_features(_p(x), L, D, _p(A), R, _p(phi))
+    _load().orc_features(_p(x), L, D, _p(A), R, int(act), _p(phi))
     return phi
 
 
@@ -188,8 +192,12 @@ def lowrank_apply(psiq, phiq, S, z, rows=None) -> np.ndarray:
 
 
 def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, theta=1e4,
-                 offset=(0, 0, 0), split=None, qblocks=None, branches=3, idx_override=None):
+                 offset=(0, 0, 0), split=None, qblocks=None, branches=3, idx_override=None,
+                 activation=ACT_RELU, lowrank_rope=True):
     """Forward pass of one (batch, head): q, k, v fp64 [L, D]; A fp64 [D, R].
+
+    `activation` picks the feature map's nonlinearity; `lowrank_rope=False` drops the truncated RoPE
+    from the low-rank branch (psi = phi), the no-RoPE setting of RoLA's ablation (5.3).
 
     Returns a dict with out (rows of the computed query blocks; NaN elsewhere), the sparse and
     low-rank branch outputs, the rotated q/k, block means, scores, idx, tie flags, S and z.
@@ -218,10 +226,13 @@ def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, t
         o_s = sparse_attn(qh, kh, v, block, use_idx, qb)
         res["out_sparse"] = o_s
         out[rows] += o_s[rows]
-    phiq = features(q, A)
-    phik = features(k, A)
-    psiq = rope_rows(phiq, grid, R // 2, theta, offset, split, schedule_dim=D)
-    psik = rope_rows(phik, grid, R // 2, theta, offset, split, schedule_dim=D)
+    phiq = features(q, A, activation)
+    phik = features(k, A, activation)
+    if lowrank_rope:
+        psiq = rope_rows(phiq, grid, R // 2, theta, offset, split, schedule_dim=D)
+        psik = rope_rows(phik, grid, R // 2, theta, offset, split, schedule_dim=D)
+    else:
+        psiq, psik = phiq.copy(), phik.copy()
     S, z = summary(psik, phik, v)
     res.update(S=S, z=z, phiq=phiq, phik=phik, psiq=psiq, psik=psik)
     if branches & 2:
@@ -233,7 +244,8 @@ def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, t
 
 
 def forward(inp: dict, grid, block: int, keep_frac: float, rank: int, *, theta=1e4, offset=(0, 0, 0),
-            split=None, heads=None, qblocks=None, branches=3, idx_override=None, keep_intermediates=False):
+            split=None, heads=None, qblocks=None, branches=3, idx_override=None, keep_intermediates=False,
+            activation=ACT_RELU, lowrank_rope=True):
     """Full forward over all (batch, head) pairs of bf16 inputs q, k, v [B, L, Hh, D] and A [D, R].
 
     heads: optional list of (b, h) to compute (default all).  qblocks: dict {(b, h): [alpha...]} or a
@@ -251,7 +263,8 @@ def forward(inp: dict, grid, block: int, keep_frac: float, rank: int, *, theta=1
         ov = None if idx_override is None else idx_override[b, h]
         r = head_forward(decode_bf16(q[b, :, h, :]), decode_bf16(k[b, :, h, :]), decode_bf16(v[b, :, h, :]),
                          Af, grid, block, keep_frac, rank, theta=theta, offset=offset, split=split,
-                         qblocks=qb, branches=branches, idx_override=ov)
+                         qblocks=qb, branches=branches, idx_override=ov, activation=activation,
+                         lowrank_rope=lowrank_rope)
         out[b, :, h, :] = r["out"]
         if not keep_intermediates:
             for key in ("qh", "kh", "phiq", "phik", "psiq", "psik", "out_sparse", "out_lowrank", "out"):

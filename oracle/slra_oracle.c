@@ -24,7 +24,8 @@
  * The block-mean-pooled selection score, relu feature map phi(x) = relu(x A) with one A of shape
  * [D][R], the normaliser phi(q).sum_j phi(k_j) + 1e-6 and the plain sum of the two branches are the
  * construction this implementation targets; readings of points the pages leave open are listed in
- * the design notes and repeated at each function below.
+ * the design notes and repeated at each function below.  RoLA's ablation ("5.3", Table 6) adds two
+ * options: SiLU, identity or tanh in place of relu, and the low-rank branch without its RoPE.
  */
 #include <math.h>
 #include <stdint.h>
@@ -241,14 +242,28 @@ ORC_EXPORT void orc_sparse_attn(const double* qh, const double* kh, const double
     }
 }
 
-/* Feature map phi(x) = relu(x A) on the raw (pre-RoPE) rows: x [L][D], A [D][R] -> phi [L][R]. */
-ORC_EXPORT void orc_features(const double* x, int64_t L, int64_t D, const double* A, int64_t R, double* phi) {
+/*
+ * Feature map phi(x) = act(x A) on the raw (pre-RoPE) rows: x [L][D], A [D][R] -> phi [L][R].
+ * act: 0 relu (the benchmark's map), 1 SiLU u / (1 + e^-u), 2 identity, 3 tanh -- the activations
+ * RoLA's ablation compares (RoLA "5.3", Table 6).
+ */
+static double orc_act(double u, int act) {
+    switch (act) {
+        case 1: return u / (1.0 + exp(-u));
+        case 2: return u;
+        case 3: return tanh(u);
+        default: return u > 0.0 ? u : 0.0;
+    }
+}
+
+ORC_EXPORT void orc_features(const double* x, int64_t L, int64_t D, const double* A, int64_t R, int act,
+                             double* phi) {
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < L; ++n)
         for (int64_t c = 0; c < R; ++c) {
             double acc = 0.0;
             for (int64_t d = 0; d < D; ++d) acc += x[n * D + d] * A[d * R + c];
-            phi[n * R + c] = acc > 0.0 ? acc : 0.0;
+            phi[n * R + c] = orc_act(acc, act);
         }
 }
 

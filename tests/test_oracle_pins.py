@@ -203,6 +203,63 @@ def test_features_relu_matmul(oracle_mod):
     assert np.allclose(oracle_mod.features(x, A), ref, rtol=0, atol=1e-13)
 
 
+def test_features_activation_variants(oracle_mod):
+    """The ablation's activations (RoLA 5.3, Table 6) against torch's own SiLU / tanh and a plain
+    matmul for identity, plus two closed-form facts of SiLU (catches a sigmoid in place of SiLU, a
+    sign flip in the exponent, or an activation applied before the projection)."""
+    import torch
+    rng = np.random.default_rng(14)
+    x, A = rng.standard_normal((40, 64)), rng.standard_normal((64, 16))
+    u = torch.from_numpy(x) @ torch.from_numpy(A)
+    assert np.allclose(oracle_mod.features(x, A, oracle_mod.ACT_SILU), torch.nn.functional.silu(u).numpy(),
+                       rtol=1e-14, atol=1e-14)
+    assert np.allclose(oracle_mod.features(x, A, oracle_mod.ACT_TANH), torch.tanh(u).numpy(), rtol=1e-14, atol=1e-14)
+    assert np.allclose(oracle_mod.features(x, A, oracle_mod.ACT_IDENTITY), u.numpy(), rtol=1e-14, atol=1e-14)
+    # SiLU(0) = 0; its minimum sits where sigma(u)(1 + u(1 - sigma(u))) = 0, u* = -1.27846454...,
+    # value -0.27846454... (u* = -(1 + e^u*)); probe it through a 1x1 projection
+    one = np.ones((1, 1))
+    assert oracle_mod.features(np.zeros((1, 1)), one, oracle_mod.ACT_SILU)[0, 0] == 0.0
+    us = -1.2784645427610738
+    assert abs(us + 1.0 + math.exp(us)) < 1e-15
+    val = oracle_mod.features(np.full((1, 1), us), one, oracle_mod.ACT_SILU)[0, 0]
+    assert abs(val - (1.0 + us)) < 1e-14  # at the minimum SiLU(u*) = 1 + u*
+    grid = np.linspace(us - 0.5, us + 0.5, 101)[:, None]
+    assert oracle_mod.features(grid, one, oracle_mod.ACT_SILU).min() >= val - 1e-15
+
+
+@pytest.mark.parametrize("act", [1, 2, 3])
+def test_lowrank_summary_equals_quadratic_other_activations(oracle_mod, act):
+    """The summary form equals the explicit quadratic form for every activation (the summary's
+    factorisation does not depend on the map).  Non-negative q, k and A keep the normaliser away
+    from zero for identity and tanh."""
+    w = W.TINY
+    x = I.make_inputs(w)
+    dec = oracle_mod.decode_bf16
+    q, k, v = np.abs(dec(x["q"][0, :, 0])), np.abs(dec(x["k"][0, :, 0])), dec(x["v"][0, :, 0])
+    A = np.abs(dec(x["A"]))
+    r = oracle_mod.head_forward(q, k, v, A, (w.T, w.H, w.W), w.block, w.keep_frac, w.rank, branches=2,
+                                activation=act)
+    ref = brute.lowrank_quadratic(r["psiq"], r["phiq"], r["psik"], r["phik"], v)
+    assert np.allclose(r["out_lowrank"], ref, rtol=1e-11, atol=1e-13)
+
+
+def test_lowrank_without_rope(oracle_mod):
+    """lowrank_rope=False (the no-RoPE ablation): psi = phi, so the branch is plain linear attention
+    phi(q)^T sum_j phi(k_j) v_j / (phi(q) . sum_j phi(k_j) + 1e-6); it is then independent of the
+    rotary base and of any position offset, and differs from the rotated branch."""
+    w = W.TINY
+    r0, x = _head(oracle_mod, w, branches=2, lowrank_rope=False)
+    v = oracle_mod.decode_bf16(x["v"][0, :, 0])
+    assert np.array_equal(r0["psiq"], r0["phiq"]) and np.array_equal(r0["psik"], r0["phik"])
+    num = r0["phiq"] @ (r0["phik"].T @ v)
+    den = r0["phiq"] @ r0["phik"].sum(0) + 1e-6
+    assert np.allclose(r0["out_lowrank"], num / den[:, None], rtol=1e-11, atol=1e-13)
+    r1, _ = _head(oracle_mod, w, branches=2, lowrank_rope=False, theta=500.0, offset=(3, 1, 2))
+    assert np.allclose(r1["out_lowrank"], r0["out_lowrank"], rtol=1e-13, atol=1e-15)
+    r2, _ = _head(oracle_mod, w, branches=2)
+    assert not np.allclose(r2["out_lowrank"], r0["out_lowrank"], rtol=1e-3)
+
+
 def test_lowrank_summary_equals_quadratic(oracle_mod):
     """The query-independent summary form (RoLA B.1) equals the explicit L x L quadratic form."""
     w = W.TINY
