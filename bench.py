@@ -101,7 +101,15 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------- CPU oracle
-def oracle_sample(w, x, seconds_hint: float = 15.0):
+ACTS = {"relu": 0, "silu": 1, "identity": 2, "tanh": 3}
+
+
+def variant_of(args) -> dict:
+    """Low-rank branch options of the run (the oracle's keyword names)."""
+    return {"activation": ACTS[args.activation], "lowrank_rope": not args.lowrank_norope}
+
+
+def oracle_sample(w, x, variant: dict, seconds_hint: float = 15.0):
     """Time the fp64 oracle on a bounded sample: one head's full selection and low-rank summary plus as
     many query blocks (attention + readout) as fit the hint.  Returns (tflops, desc, threads, secs)."""
     import oracle
@@ -111,7 +119,7 @@ def oracle_sample(w, x, seconds_hint: float = 15.0):
     threads = int(os.environ.get("OMP_NUM_THREADS", 0)) or len(os.sched_getaffinity(0))
     # a first call with one query block measures the per-block cost
     t0 = time.perf_counter()
-    _, per = oracle.forward(x, grid, w.block, w.keep_frac, w.rank, heads=[(0, 0)], qblocks=[0])
+    _, per = oracle.forward(x, grid, w.block, w.keep_frac, w.rank, heads=[(0, 0)], qblocks=[0], **variant)
     t1 = time.perf_counter()
     base = t1 - t0
     nq = 1
@@ -121,7 +129,7 @@ def oracle_sample(w, x, seconds_hint: float = 15.0):
         nq = int(min(nb, max(2, (seconds_hint - base) / per_block)))
         qbs = list(np.linspace(0, nb - 1, nq).astype(int))
         t0 = time.perf_counter()
-        _, per = oracle.forward(x, grid, w.block, w.keep_frac, w.rank, heads=[(0, 0)], qblocks=qbs)
+        _, per = oracle.forward(x, grid, w.block, w.keep_frac, w.rank, heads=[(0, 0)], qblocks=qbs, **variant)
         t1 = time.perf_counter()
     else:
         qbs = [0]
@@ -151,7 +159,8 @@ def run_reference(args, w, rank, world):
 
     def step():
         t0 = time.perf_counter()
-        _, per = oracle.forward(x, grid, w.block, w.keep_frac, w.rank, heads=[(0, 0)], qblocks=qbs)
+        _, per = oracle.forward(x, grid, w.block, w.keep_frac, w.rank, heads=[(0, 0)], qblocks=qbs,
+                                **variant_of(args))
         return time.perf_counter() - t0, per[(0, 0)]
 
     for _ in range(args.warmup):
@@ -174,7 +183,8 @@ def run_reference(args, w, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded clustered-Gaussian bf16 q/k/v, A ~ N(0, 1/d_h))",
             "config": {"workload": base_w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
-                       "block": w.block, "keep_frac": w.keep_frac},
+                       "block": w.block, "keep_frac": w.keep_frac, "activation": args.activation,
+                       "lowrank_rope": not args.lowrank_norope},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -202,7 +212,9 @@ def run_ours(args, w, rank, world, local_rank):
     for e in stage_ev:
         e.record()
     torch.cuda.synchronize()
-    prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev))
+    var = variant_of(args)
+    prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev),
+                                      activation=var["activation"], lowrank_norope=int(not var["lowrank_rope"]))
     ws = slra.alloc_workspace(prob, dev)
     out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
@@ -280,7 +292,7 @@ def run_ours(args, w, rank, world, local_rank):
     traffic = load_traffic(w.name)
     bytes_min = F.io_bytes(w.batch, w.L, w.heads, w.head_dim, w.rank, 4)
     t_roof = max(f_sparse / (tf_sust * 1e12), bytes_min / (hbm * 1e9))
-    cpu_v, cpu_desc, cpu_threads, _ = oracle_sample(w, x)  # rank 0 runs the workload itself
+    cpu_v, cpu_desc, cpu_threads, _ = oracle_sample(w, x, var)  # rank 0 runs the workload itself
     line = {
         "metric": METRIC, "value": replicas.job_throughput(job_flops, ms_per_step), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
@@ -289,7 +301,8 @@ def run_ours(args, w, rank, world, local_rank):
         "config": {"workload": base_w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
                    "block": w.block, "keep_frac": w.keep_frac, "keep_blocks": int(idx.shape[-1]),
                    "out_dtype": "f32", "l2": "flushed between timed steps (512 MB write)",
-                   "parallelism": f"replica x{world} (independent problems, no collective)"},
+                   "parallelism": f"replica x{world} (independent problems, no collective)",
+                   "activation": args.activation, "lowrank_rope": not args.lowrank_norope},
         "flops_per_step": {"sparse_kept": f_sparse, "lowrank": f_lr, "scores": f_sc},
         "roofline": {"kernel": "attn_sm100_kernel", "bound": "tensor", "achieved": achieved, "peak": tf_sust,
                      "unit": "TFLOP/s", "frac": achieved / tf_sust, "traffic": traffic,
@@ -330,6 +343,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--activation", default="relu", choices=sorted(ACTS), help="low-rank feature map")
+    ap.add_argument("--lowrank-norope", action="store_true", help="low-rank branch without its RoPE")
     args = ap.parse_args()
     w = WL.by_name(args.workload)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -21,7 +21,8 @@
  *   K(alpha)    = the k = clamp(round(keep_frac * nb), 1, nb) key blocks with the largest
  *                 qbar_alpha . kbar_beta, ties to the lower block index
  *   O_sparse_i  = softmax_j(qh_i . kh_j / sqrt(D)) v_j over the keys of K(alpha(i))
- *   phi(x)      = relu(x A) on raw q, k;   psi = phi with its first r coordinates rotated like RoPE
+ *   phi(x)      = relu(x A) on raw q, k (or SiLU / identity / tanh, slra_problem.activation);
+ *               psi = phi with its first r coordinates rotated like RoPE (unless lowrank_norope)
  *   S = sum_j psi(k_j) v_j^T (r x D),  z = sum_j phi(k_j)   (all L keys, per head)
  *   O_lowrank_i = psi(q_i)^T S / (phi(q_i) . z + 1e-6)
  *   out         = O_sparse + O_lowrank
@@ -48,7 +49,7 @@
 extern "C" {
 #endif
 
-#define SLRA_ABI_VERSION 1
+#define SLRA_ABI_VERSION 2
 
 /* Exported symbols (the library is built with hidden visibility for everything else). */
 #if defined(__GNUC__)
@@ -85,6 +86,17 @@ enum { SLRA_BRANCH_SPARSE = 1, SLRA_BRANCH_LOWRANK = 2, SLRA_BRANCH_BOTH = 3 };
  * the GPU.  Use a small wait_timeout_ns with it. */
 enum { SLRA_DEBUG_UNSATISFIED_WAIT = 1 };
 
+/* Nonlinearity of the low-rank feature map phi = act(x A) (slra_problem.activation).  RELU is the
+ * benchmark's map; SILU (u / (1 + e^-u)), IDENTITY and TANH are the alternatives RoLA's ablation
+ * compares ("5.3", Table 6).  With IDENTITY or TANH the normaliser phi(q) . sum_j phi(k_j) + 1e-6 can
+ * come close to zero; the library computes it as defined and does not guard it. */
+typedef enum slra_activation {
+    SLRA_ACT_RELU = 0,
+    SLRA_ACT_SILU = 1,
+    SLRA_ACT_IDENTITY = 2,
+    SLRA_ACT_TANH = 3
+} slra_activation;
+
 /*
  * Problem description.  Fill it with slra_problem_init, then adjust optional fields.
  *   batch, heads, head_dim  B, Hh, D.  D in {64, 128}.
@@ -107,6 +119,10 @@ enum { SLRA_DEBUG_UNSATISFIED_WAIT = 1 };
  *                           partial sums, [5] after their reduction, [6] after the attention kernel
  *                           (the branch entry points record the boundaries of the stages they run).
  *                           The caller creates and owns them.
+ *   activation              SLRA_ACT_* map of the low-rank features (default SLRA_ACT_RELU).
+ *   lowrank_norope          0 (default): the low-rank branch rotates the first r feature coordinates
+ *                           with the truncated 3D RoPE after the activation (RoLA "4.2", "4.3");
+ *                           1: no rotation, psi = phi (the no-RoPE setting of RoLA "5.3").
  */
 typedef struct slra_problem {
     int64_t batch, heads, head_dim;
@@ -122,6 +138,8 @@ typedef struct slra_problem {
     uint64_t wait_timeout_ns;
     uint32_t debug_flags;
     void* stage_events[7];
+    int32_t activation;
+    int32_t lowrank_norope;
 } slra_problem;
 
 /*

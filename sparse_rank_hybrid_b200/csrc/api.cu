@@ -46,6 +46,8 @@ slra_status derive(const slra_problem* p, Derived* d) {
     if (p->theta < 0.0 || std::isnan(p->theta)) return SLRA_ERR_INVALID_ARG;
     if (p->out_dtype != SLRA_OUT_F32 && p->out_dtype != SLRA_OUT_BF16) return SLRA_ERR_INVALID_ARG;
     if (p->branches < 0 || p->branches > 3) return SLRA_ERR_INVALID_ARG;
+    if (p->activation < SLRA_ACT_RELU || p->activation > SLRA_ACT_TANH) return SLRA_ERR_INVALID_ARG;
+    if (p->lowrank_norope != 0 && p->lowrank_norope != 1) return SLRA_ERR_INVALID_ARG;
     if (p->head_dim != 64 && p->head_dim != 128) return SLRA_ERR_UNSUPPORTED;
     if (p->block != 64 && p->block != 128) return SLRA_ERR_UNSUPPORTED;
     if (p->rank < 16 || p->rank > p->head_dim || p->rank % 16 != 0) return SLRA_ERR_UNSUPPORTED;
@@ -75,6 +77,8 @@ slra_status derive(const slra_problem* p, Derived* d) {
     g.keep = static_cast<int>(keep);
     g.R = static_cast<int>(p->rank);
     g.Lp = static_cast<int>(nb * p->block);
+    g.act = static_cast<int>(p->activation);
+    g.norope = static_cast<int>(p->lowrank_norope);
 
     RopeMeta& m = d->meta;
     std::memset(&m, 0, sizeof m);
@@ -304,6 +308,8 @@ slra_status slra_problem_init(slra_problem* p, int64_t batch, int64_t heads, int
     p->out_dtype = SLRA_OUT_F32;
     p->branches = SLRA_BRANCH_BOTH;
     p->wait_timeout_ns = 2000000000ull;
+    p->activation = SLRA_ACT_RELU;
+    p->lowrank_norope = 0;
     return SLRA_OK;
 }
 

@@ -3,7 +3,9 @@
 //
 // Method (RoLA, "4.1"): for each query block alpha, exact softmax attention of its queries over the
 // union of the kept key blocks K(alpha); plus O_lr,i = psi(q_i)^T S / (phi(q_i) . z + 1e-6) with
-// phi = relu(q A) on the raw query and psi its first r coordinates rotated by 3D RoPE ("4.2", "4.3").
+// phi = relu(q A) on the raw query and psi its first r coordinates rotated by 3D RoPE ("4.2", "4.3");
+// SiLU, identity or tanh in place of relu, and psi = phi without the rotation, are the options of the
+// ablation ("5.3").
 //
 // One CTA per (query block, batch*head), one CTA per SM, warp-specialised (320 threads):
 //   warps 0-7  softmax: row i lives in TMEM lane i; warps w and w+4 both reach lanes 32(w%4).. and
@@ -138,12 +140,16 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 
 }  // namespace
 
-template <int D, int BLK>
+// kDefault: relu features with the low-rank RoPE (the benchmark's configuration); the activation and
+// no-RoPE branches then fold away at compile time.
+template <int D, int BLK, bool kDefault>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qraw,
                       const __grid_constant__ CUtensorMap tm_out, AttnArgs a, Geom g) {
     using Lay = AttnLayout<D>;
+    const int act = kDefault ? 0 : g.act;        // low-rank feature map
+    const int norope = kDefault ? 0 : g.norope;  // 1: no rotation in the low-rank branch
     constexpr int HW = BLK / 2;   // keys per thread: the two warps of a lane group split the key block
     constexpr int NC = HW / 32;   // 32-column TMEM loads per thread
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -483,7 +489,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (a.lowrank && !aborted) {
             // Low-rank readout on the tensor cores, accumulated straight into O (so out = O / l):
             //   phi = q A        raw bf16 query tile (TMA) x A^T image, into TMEM columns of its own;
-            //   psi = R_r(p) relu(phi) * l / (relu(phi) . z + 1e-6), split into bf16 hi + lo;
+            //   psi = R_r(p) act(phi) * l / (act(phi) . z + 1e-6), split into bf16 hi + lo (no R_r
+            //         when the low-rank RoPE is off);
             //   O  += psi S      as psi_hi S_hi + psi_hi S_lo + psi_lo S_hi, one 64-feature chunk at a time.
             // The two warps of a lane group share each row: 32-feature column groups of the
             // denominator alternate between them, and so do the rotation pairs.
@@ -540,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_ld_wait(v);
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
-                            if (c0 + i < R) den = fmaf(fmaxf(__uint_as_float(v[i]), 0.f), __ldg(zh + c0 + i), den);
+                            if (c0 + i < R) den = fmaf(phi_act(__uint_as_float(v[i]), act), __ldg(zh + c0 + i), den);
                     }
                 }
                 xch[hf * 128 + i_row] = den;
@@ -575,7 +582,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // not stored).  The pair -> (axis, table offset) map comes from the launch parameters.
                     auto feat = [&](int t) { return t < 8 ? 16 * hf + 2 * t : 32 + 16 * hf + 2 * (t - 8); };
                     float2 rot[16];
-                    const int nrot = rc > 32 ? 16 : 8;  // the second eight lie past the rank when rc <= 32
+                    // the second eight lie past the rank when rc <= 32; no rotation without the low-rank RoPE
+                    const int nrot = norope ? 0 : (rc > 32 ? 16 : 8);
                     {
                         double2 cs[16];
 #pragma unroll
@@ -604,9 +612,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (f < rc) {
                             const uint32_t u0 = t < 8 ? va[2 * t] : vb[2 * (t - 8)];
                             const uint32_t u1 = t < 8 ? va[2 * t + 1] : vb[2 * (t - 8) + 1];
-                            const float x0 = fmaxf(__uint_as_float(u0), 0.f);
-                            const float x1 = fmaxf(__uint_as_float(u1), 0.f);
-                            const float cf = rot[t].x, sf = rot[t].y;
+                            const float x0 = phi_act(__uint_as_float(u0), act);
+                            const float x1 = phi_act(__uint_as_float(u1), act);
+                            const float cf = norope ? 1.f : rot[t].x, sf = norope ? 0.f : rot[t].y;
                             const float y0 = (x0 * cf - x1 * sf) * scale, y1 = (x0 * sf + x1 * cf) * scale;
                             const __nv_bfloat162 hi = __floats2bfloat162_rn(y0, y1);
                             const float2 hf2 = __bfloat1622float2(hi);
@@ -687,11 +695,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        phi[c] = fmaxf(phi[c], 0.f);
+                        phi[c] = phi_act(phi[c], act);
                         den = fmaf(phi[c], __ldg(zh + c0 + c), den);
                     }
 #pragma unroll
                     for (int pp = 0; pp < 8; ++pp) {
+                        if (norope) break;
                         const int2 pi = __ldg(a.pairs + (c0 >> 1) + pp);  // (axis, table offset)
                         const double2 cs = __ldg(a.tab + pi.y + token_axis_pos(n, pi.x, g.H, g.W));
                         const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
@@ -802,14 +811,20 @@ size_t attn_smem_bytes(const Geom& g) {
 }
 
 namespace {
+template <int D, int BLK, bool kDefault>
+cudaError_t launch_attn_v(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st) {
+    const size_t sm = attn_smem_bytes(g);
+    cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D, BLK, kDefault>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+    if (e != cudaSuccess) return e;
+    attn_sm100_kernel<D, BLK, kDefault><<<dim3(g.nb, g.BH()), kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, m.out,
+                                                                                    a, g);
+    return cudaGetLastError();
+}
 template <int D, int BLK>
 cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st) {
-    const size_t sm = attn_smem_bytes(g);
-    cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sm));
-    if (e != cudaSuccess) return e;
-    attn_sm100_kernel<D, BLK><<<dim3(g.nb, g.BH()), kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, m.out, a, g);
-    return cudaGetLastError();
+    return (g.act == 0 && g.norope == 0) ? launch_attn_v<D, BLK, true>(m, a, g, st)
+                                         : launch_attn_v<D, BLK, false>(m, a, g, st);
 }
 }  // namespace
 

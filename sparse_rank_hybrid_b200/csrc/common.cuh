@@ -18,8 +18,24 @@ constexpr int kDevRange = 2;
 // Sizes of one call.  L = T*H*W; Lp = nb*block (rows of the padded head-major buffers).
 struct Geom {
     int B, Hh, D, T, H, W, L, block, nb, keep, R, Lp;
+    int act;     // SLRA_ACT_* of the low-rank feature map
+    int norope;  // 1: no rotation in the low-rank branch (psi = phi)
     __host__ __device__ int BH() const { return B * Hh; }
 };
+
+// phi = act(u) for the low-rank feature map: relu (0), SiLU u / (1 + e^-u) (1), identity (2), tanh (3).
+// relu stays inline; the other maps go through one out-of-line function, so the fully unrolled feature
+// loops do not carry inlined copies of expf / tanhf (the choice is uniform over a launch).
+static __device__ __noinline__ float phi_act_other(float u, int act) {
+    switch (act) {
+        case 1: return u / (1.0f + expf(-u));
+        case 2: return u;
+        default: return tanhf(u);
+    }
+}
+__device__ __forceinline__ float phi_act(float u, int act) {
+    return act == 0 ? fmaxf(u, 0.f) : phi_act_other(u, act);
+}
 
 // 3D RoPE schedule: pair j rotates with the position along axis[j]; its cos/sin for position p
 // (0-based grid coordinate; the constant offset is folded into the table) is tab[tab_off[j] + p].

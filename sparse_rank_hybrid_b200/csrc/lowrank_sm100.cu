@@ -1,5 +1,5 @@
 // Low-rank summary on the sm_100a tensor cores (head_dim 128): per head, over all L keys,
-//   S = sum_j psi(k_j) v_j^T,   z = sum_j phi(k_j),   phi(k) = relu(k A),   psi = phi with its first
+//   S = sum_j psi(k_j) v_j^T,   z = sum_j phi(k_j),   phi(k) = act(k A) (relu by default), psi = phi with its first
 // r coordinates rotated by the token's 3D RoPE angles (RoLA "4.1", "4.2", "4.3", "B.1").
 //
 // Persistent CTAs (one per SM, 256 threads: two threads per token row, each taking half of the
@@ -7,9 +7,10 @@
 //   TMA    raw k and v tiles [128 tokens][128] bf16 straight from the [B][L][Hh][D] inputs (4D tensor
 //          maps, 128-B swizzle, two stages so the next tiles stream in while this one is processed);
 //   MMA    phi = k A  (M = 128 tokens, N = r, K = 128; A^T staged once per CTA as the B operand);
-//   threads (thread = token = TMEM lane) relu, accumulate z in registers, rotate the first r
-//          coordinates and write psi as bf16 hi + lo halves (psi = hi + lo to ~2^-16) into shared
-//          memory, token-major;
+//   threads (thread = token = TMEM lane) apply the activation (relu unless another is chosen),
+//          accumulate z in registers, rotate the first r coordinates (unless the low-rank RoPE is
+//          off) and write psi as bf16 hi + lo halves (psi = hi + lo to ~2^-16) into shared memory,
+//          token-major;
 //   MMA    S^T += v^T [psi_hi | psi_lo]  (M = 128 = D, N = 2*Rp, K = 128 tokens), accumulated in TMEM
 //          over the whole work item; v is exact in bf16, so S is exact to the fp32 accumulation.
 // At the end of an item its S and z partial sums go to the split-L partial buffers, which a
@@ -72,11 +73,15 @@ struct LrArgs {
     unsigned long long timeout_ns;
 };
 
-template <int R>
+// kDefault: relu features with the RoPE (the benchmark's configuration); the activation and no-RoPE
+// branches then fold away at compile time.
+template <int R, bool kDefault>
 __global__ void __launch_bounds__(256, 1)
     lowrank_sm100_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          LrArgs a, Geom g) {
     const LrLayout lay = lr_layout(R);
+    const int act = kDefault ? 0 : g.act;
+    const int norope = kDefault ? 0 : g.norope;
     constexpr int RP = R <= 64 ? 64 : 128;
     constexpr int RH = R / 2;           // features per thread: two threads share a token row
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(256, 1)
             }
             ++n_phi;
             tc_fence_after();
-            // ---- relu, z, rotation, psi hi/lo into shared memory (two threads per token row)
+            // ---- activation, z, rotation, psi hi/lo into shared memory (two threads per token row)
             const int n = tile * kTok + row;
             const bool real = n < g.L;
             uint32_t raw[RH];
@@ -240,7 +245,8 @@ __global__ void __launch_bounds__(256, 1)
                 for (int u = 0; u < 8; ++u) {
                     if (p0 + u < RH / 2) {
                         const int2 pi = a.pair_info[half * (RH / 2) + p0 + u];
-                        cs[u] = __ldg(a.tab + pi.y + (pi.x == 0 ? pos_t : (pi.x == 1 ? pos_h : pos_w)));
+                        cs[u] = norope ? make_double2(1.0, 0.0)
+                                         : __ldg(a.tab + pi.y + (pi.x == 0 ? pos_t : (pi.x == 1 ? pos_h : pos_w)));
                     }
                 }
 #pragma unroll
@@ -248,8 +254,8 @@ __global__ void __launch_bounds__(256, 1)
                 const int pp = p0 + u;
                 if (pp >= RH / 2) break;
                 const int p = half * (RH / 2) + pp;  // global rotary pair
-                float x0 = real ? fmaxf(__uint_as_float(raw[2 * pp]), 0.f) : 0.f;
-                float x1 = real ? fmaxf(__uint_as_float(raw[2 * pp + 1]), 0.f) : 0.f;
+                float x0 = real ? phi_act(__uint_as_float(raw[2 * pp]), act) : 0.f;
+                float x1 = real ? phi_act(__uint_as_float(raw[2 * pp + 1]), act) : 0.f;
                 zacc[2 * pp] += x0;
                 zacc[2 * pp + 1] += x1;
                 const float cf = static_cast<float>(cs[u].x), sf = static_cast<float>(cs[u].y);
@@ -358,18 +364,25 @@ int lowrank_tc_tiles_per_split(const Geom& g, int nsplit) {
     return (ntiles + nsplit - 1) / nsplit;
 }
 
-template <int R>
-static cudaError_t lr_tc_launch(const CUtensorMap& tk, const CUtensorMap& tv, const LrArgs& a, const Geom& g,
-                                cudaStream_t st) {
+template <int R, bool kDefault>
+static cudaError_t lr_tc_launch_v(const CUtensorMap& tk, const CUtensorMap& tv, const LrArgs& a, const Geom& g,
+                                  cudaStream_t st) {
     const size_t sm = static_cast<size_t>(lr_layout(R).bytes) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(lowrank_sm100_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    cudaError_t e = cudaFuncSetAttribute(lowrank_sm100_kernel<R, kDefault>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int items = g.BH() * a.nsplit;
-    lowrank_sm100_kernel<R><<<items < sms ? items : sms, 256, sm, st>>>(tk, tv, a, g);
+    lowrank_sm100_kernel<R, kDefault><<<items < sms ? items : sms, 256, sm, st>>>(tk, tv, a, g);
     return cudaGetLastError();
+}
+template <int R>
+static cudaError_t lr_tc_launch(const CUtensorMap& tk, const CUtensorMap& tv, const LrArgs& a, const Geom& g,
+                                cudaStream_t st) {
+    return (g.act == 0 && g.norope == 0) ? lr_tc_launch_v<R, true>(tk, tv, a, g, st)
+                                         : lr_tc_launch_v<R, false>(tk, tv, a, g, st);
 }
 
 cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,

@@ -3,7 +3,7 @@
 //   rope_pool       3D RoPE of q and k, fp16 head-major copies of q^, k^ and v for the tensor-core
 //                   kernel, fp64 block means of q^ and k^
 //   select          fp64 block scores qbar . kbar and per-row top-k (radix select, lower index wins ties)
-//   lowrank_partial phi = relu(k A), rank-truncated RoPE outside the activation, split-L partial sums
+//   lowrank_partial phi = act(k A), rank-truncated RoPE outside the activation, split-L partial sums
 //                   of S = sum_j psi(k_j) v_j^T and z = sum_j phi(k_j)
 //   lowrank_reduce  fixed-order sum of the partials (deterministic)
 // Method: RoLA ("3 Preliminary" 3D RoPE; "4.1" block-sparse + low-rank branches; "4.2" first r rotary
@@ -382,7 +382,7 @@ cudaError_t launch_select(const double* qbar, const double* kbar, const Geom& g,
 constexpr int kLrTile = 32;  // tokens per step
 
 // One CTA per (split of the sequence, batch*head).  Per 32-token step: stage raw k and v (fp32) in
-// shared memory, phi = relu(k A) (thread per (token, feature)), rotate the first R coordinates with
+// shared memory, phi = act(k A) (thread per (token, feature)), rotate the first R coordinates with
 // the token's 3D RoPE angles (psi), then accumulate S[c][e] += sum_t psi[t][c] v[t][e] in registers
 // (thread owns one e and R/(256/D) features) and z[c] += sum_t phi[t][c].
 template <int D, int R>
@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(256) lowrank_partial_kernel(const __nv_bfloat1
             float a = 0.f;
 #pragma unroll 16
             for (int d = 0; d < D; ++d) a = fmaf(kr[d], As[d * R + c], a);
-            ph[tt * (R + 1) + c] = fmaxf(a, 0.f);
+            ph[tt * (R + 1) + c] = phi_act(a, g.act);
         }
         __syncthreads();
         for (int o = tid; o < kLrTile * (R / 2); o += 256) {
@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(256) lowrank_partial_kernel(const __nv_bfloat1
             const int n = n0 + tt;
             const float x0 = ph[tt * (R + 1) + 2 * p], x1 = ph[tt * (R + 1) + 2 * p + 1];
             float c = 1.f, s = 0.f;
-            if (n < g.L) {
+            if (n < g.L && !g.norope) {
                 const int2 pi = pairs[p];
                 const double2 cs = tab[pi.y + token_axis_pos(n, pi.x, g.H, g.W)];
                 c = static_cast<float>(cs.x);

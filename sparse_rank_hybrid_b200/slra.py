@@ -20,6 +20,8 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DE
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
 DEBUG_UNSATISFIED_WAIT = 1
+ABI_VERSION = 2
+ACT_RELU, ACT_SILU, ACT_IDENTITY, ACT_TANH = 0, 1, 2, 3
 
 # Every symbol include/slra.h declares.
 EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_validate", "slra_keep_count",
@@ -40,7 +42,8 @@ class _Problem(ctypes.Structure):
                 ("theta", ctypes.c_double), ("out_dtype", ctypes.c_int32), ("branches", ctypes.c_int32),
                 ("pos_offset", ctypes.c_int64 * 3), ("rope_split", ctypes.c_int64 * 3),
                 ("wait_timeout_ns", ctypes.c_uint64), ("debug_flags", ctypes.c_uint32),
-                ("stage_events", ctypes.c_void_p * 7)]
+                ("stage_events", ctypes.c_void_p * 7), ("activation", ctypes.c_int32),
+                ("lowrank_norope", ctypes.c_int32)]
 
 
 class _Layout(ctypes.Structure):
@@ -60,6 +63,9 @@ def lib():
         if not os.path.exists(LIB_PATH):
             raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m sparse_rank_hybrid_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
+        L.slra_abi_version.restype = ctypes.c_int
+        if L.slra_abi_version() != ABI_VERSION:  # the structs below mirror this version of include/slra.h
+            raise RuntimeError(f"{LIB_PATH} has ABI {L.slra_abi_version()}, this binding expects {ABI_VERSION}")
         P, S = ctypes.c_void_p, ctypes.c_size_t
         PP = ctypes.POINTER(_Problem)
         L.slra_abi_version.restype = ctypes.c_int
@@ -114,6 +120,8 @@ class Problem:
     wait_timeout_ns: int = 2_000_000_000
     debug_flags: int = 0
     stage_events: tuple = (None,) * 7  # raw cudaEvent_t handles (ints) or None, see slra_problem
+    activation: int = 0                # ACT_* map of the low-rank features
+    lowrank_norope: int = 0            # 1: no RoPE in the low-rank branch
 
     @property
     def L(self) -> int:
@@ -136,6 +144,8 @@ class Problem:
         p.debug_flags = int(self.debug_flags)
         for i, e in enumerate(self.stage_events):
             p.stage_events[i] = e
+        p.activation = int(self.activation)
+        p.lowrank_norope = int(self.lowrank_norope)
         return p
 
 

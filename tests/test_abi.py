@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_abi_version_and_status_strings():
-    assert slra.lib().slra_abi_version() == 1
+    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 2
     for s in range(0, 9):
         assert slra.status_string(s) and slra.status_string(s) != "unknown status"
     assert slra.status_string(99) == "unknown status"
@@ -59,6 +59,8 @@ def test_keep_count_and_layout(w, oracle_mod):
     ("T", 0, slra.ERR_INVALID_ARG), ("heads", 0, slra.ERR_INVALID_ARG), ("out_dtype", 7, slra.ERR_INVALID_ARG),
     ("rope_split", (10, 10, 10), slra.ERR_INVALID_ARG), ("branches", 9, slra.ERR_INVALID_ARG),
     ("T", 5000, slra.ERR_UNSUPPORTED),  # 5000*45*80 tokens -> more than 2048 blocks
+    ("activation", 4, slra.ERR_INVALID_ARG), ("activation", -1, slra.ERR_INVALID_ARG),
+    ("lowrank_norope", 2, slra.ERR_INVALID_ARG),
 ])
 def test_validation_rejects(field, value, status):
     p = slra.Problem.from_workload(W.WAN_14B)

@@ -40,9 +40,11 @@ def _build():
     oracle.build()
 
 
-def _case(w, label=None, heads=None, qblocks=None, **kw):
+def _case(w, label=None, heads=None, qblocks=None, transform=None, **kw):
     p = slra.Problem.from_workload(w, **kw)
     x = I.make_inputs(w)
+    if transform is not None:
+        x = transform(x)
     gpu = parity.run_gpu(p, x)
     st = parity.compare(p, x, gpu, heads=heads, qblocks=qblocks, label=label or w.name)
     _log(st)
@@ -69,6 +71,41 @@ def test_tiny_branches_separately():
 def test_edge_shapes(grid, D, R, block, keep, B, heads):
     w = W.Workload(f"edge-{grid}-{D}-{R}-{block}-{keep}", B, heads, D, *grid, R, block, keep, 7000 + D + R)
     _case(w)
+
+
+def _nonneg(x):
+    """q, k and A with the bf16 sign bit cleared: every feature x A is then >= 0, which keeps the
+    normaliser phi(q) . z + 1e-6 away from zero for the identity and tanh maps."""
+    y = dict(x)
+    for n in ("q", "k", "A"):
+        y[n] = np.bitwise_and(x[n], np.uint16(0x7FFF))
+    return y
+
+
+EDGE_128 = W.Workload("edge-act-128", 1, 2, 128, 3, 10, 13, 32, 128, 0.3, 7160)   # L = 390, ragged
+EDGE_128_R64 = W.Workload("edge-act-128-r64", 1, 2, 128, 2, 9, 11, 64, 64, 0.25, 7192)
+
+
+@pytest.mark.parametrize("act", [slra.ACT_SILU, slra.ACT_IDENTITY, slra.ACT_TANH])
+def test_activation_variants(act):
+    """The feature map's alternatives (RoLA 5.3, Table 6) on both readout paths: head_dim 64 (CUDA
+    cores) and head_dim 128 (tensor cores; r = 32, and r = 64 with block 64).  Features that can be
+    negative let the normaliser come close to zero on Gaussian inputs (SiLU on the tiny case: 0.13
+    against a median of 159, low-rank outputs up to ~590, where fp32 rounding alone exceeds the 1e-2
+    absolute bound), so these cases use non-negative q, k and A."""
+    _case(W.TINY, f"tiny-act{act}", activation=act, transform=_nonneg)
+    _case(EDGE_128, f"edge128-act{act}", activation=act, transform=_nonneg)
+    _case(EDGE_128_R64, f"edge128r64-act{act}", activation=act, transform=_nonneg)
+
+
+def test_lowrank_without_rope():
+    """The low-rank branch without its RoPE (psi = phi) on both readout paths, and with SiLU on a
+    sampled head of the Wan2.1-1.3B shape."""
+    _case(W.TINY, "tiny-norope", lowrank_norope=1)
+    _case(EDGE_128, "edge128-norope", lowrank_norope=1)
+    w = W.WAN_1_3B
+    _case(w, "wan1.3b-silu-norope", heads=[(0, 5)], qblocks=_sample_blocks(w.nb, 4, n=2),
+          activation=slra.ACT_SILU, lowrank_norope=1, transform=_nonneg)
 
 
 def test_shift_invariance_on_gpu():
