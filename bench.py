@@ -102,11 +102,20 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------------- CPU oracle
 ACTS = {"relu": 0, "silu": 1, "identity": 2, "tanh": 3}
+BRANCHES = {"both": 3, "sparse": 1, "lowrank": 2}
+
+
+def identity_bits(D: int) -> np.ndarray:
+    """A = I as bf16 bits (1.0 = 0x3F80): the full-width linear-attention baseline's projection."""
+    a = np.zeros((D, D), dtype=np.uint16)
+    a[np.arange(D), np.arange(D)] = 0x3F80
+    return a
 
 
 def variant_of(args) -> dict:
     """Low-rank branch options of the run (the oracle's keyword names)."""
-    return {"activation": ACTS[args.activation], "lowrank_rope": not args.lowrank_norope}
+    return {"activation": ACTS[args.activation], "lowrank_rope": not args.lowrank_norope,
+            "branches": BRANCHES[args.branches]}
 
 
 def oracle_sample(w, x, variant: dict, seconds_hint: float = 15.0):
@@ -136,10 +145,11 @@ def oracle_sample(w, x, variant: dict, seconds_hint: float = 15.0):
     secs = t1 - t0
     r = per[(0, 0)]
     sz = F.block_sizes(w.L, w.block)
-    kept = float(4.0 * w.head_dim * sum(sz[r["idx"][a]].sum() * sz[a] for a in qbs))
+    br = variant.get("branches", 3)
+    kept = float(4.0 * w.head_dim * sum(sz[r["idx"][a]].sum() * sz[a] for a in qbs)) if br & 1 else 0.0
     rows = int(sum(sz[a] for a in qbs))
-    work = (kept + F.score_flops(nb, w.head_dim, 1) + 4.0 * w.L * w.rank * w.head_dim
-            + 4.0 * rows * w.rank * w.head_dim)
+    work = kept + (F.score_flops(nb, w.head_dim, 1) if br & 1 else 0.0) + \
+        ((4.0 * w.L * w.rank * w.head_dim + 4.0 * rows * w.rank * w.head_dim) if br & 2 else 0.0)
     desc = (f"fp64 C oracle, head (0,0) of {w.name}: full 3D RoPE, pooling, scores, top-k and low-rank "
             f"summary over all {w.L} tokens, plus attention + low-rank readout for {len(qbs)} of {nb} query "
             f"blocks; value = that work's effective FLOPs / wall time")
@@ -151,6 +161,8 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return
     x = I.make_inputs(w)
+    if args.linear_baseline:
+        x["A"] = identity_bits(w.head_dim)
     import oracle
     oracle.build()
     grid = (w.T, w.H, w.W)
@@ -170,10 +182,11 @@ def run_reference(args, w, rank, world):
         t, r = step()
         times.append(t)
     sz = F.block_sizes(w.L, w.block)
-    kept = float(4.0 * w.head_dim * sum(sz[r["idx"][a]].sum() * sz[a] for a in qbs))
+    br = BRANCHES[args.branches]
+    kept = float(4.0 * w.head_dim * sum(sz[r["idx"][a]].sum() * sz[a] for a in qbs)) if br & 1 else 0.0
     rows = int(sum(sz[a] for a in qbs))
-    work = (kept + F.score_flops(w.nb, w.head_dim, 1) + 4.0 * w.L * w.rank * w.head_dim
-            + 4.0 * rows * w.rank * w.head_dim)
+    work = kept + (F.score_flops(w.nb, w.head_dim, 1) if br & 1 else 0.0) + \
+        ((4.0 * w.L * w.rank * w.head_dim + 4.0 * rows * w.rank * w.head_dim) if br & 2 else 0.0)
     tot = sum(times)
     value = work * args.steps / tot / 1e12
     sample = (f"one step = head (0,0) of {w.name}: full selection and low-rank summary over {w.L} tokens "
@@ -207,13 +220,16 @@ def run_ours(args, w, rank, world, local_rank):
     base_w = w
     w = replicas.replica_workload(base_w, rank)  # each rank: its own independent problem
     x = I.make_inputs(w)
+    if args.linear_baseline:
+        x["A"] = identity_bits(w.head_dim)
     q, k, v, A = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v", "A"))
     stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
     for e in stage_ev:
         e.record()
     torch.cuda.synchronize()
     var = variant_of(args)
-    prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev),
+    br = BRANCHES[args.branches]
+    prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev), branches=br,
                                       activation=var["activation"], lowrank_norope=int(not var["lowrank_rope"]))
     ws = slra.alloc_workspace(prob, dev)
     out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
@@ -230,14 +246,19 @@ def run_ours(args, w, rank, world, local_rank):
     status = slra.device_status(ws)
     if status != slra.OK:
         raise RuntimeError(f"device status after warm-up: {slra.status_string(status)}")
-    idx = slra.ws_view(prob, ws, "idx").cpu().numpy()
     BH = w.batch * w.heads
-    f_sparse = F.sparse_flops(idx, w.L, w.block, w.head_dim)
-    f_lr = F.lowrank_flops(w.L, w.rank, w.head_dim, BH)
-    f_sc = F.score_flops(w.nb, w.head_dim, BH)
+    if br & 1:
+        idx = slra.ws_view(prob, ws, "idx").cpu().numpy()
+        f_sparse = F.sparse_flops(idx, w.L, w.block, w.head_dim)
+        f_sc = F.score_flops(w.nb, w.head_dim, BH)
+        keep_blocks = int(idx.shape[-1])
+    else:
+        f_sparse = f_sc = 0.0
+        keep_blocks = 0
+    f_lr = F.lowrank_flops(w.L, w.rank, w.head_dim, BH) if br & 2 else 0.0
     f_total = f_sparse + f_lr + f_sc
     # attention kernel's own algorithmic work: kept products + the fused readout (q A and psi S)
-    f_attn = f_sparse + 4.0 * w.L * w.rank * w.head_dim * BH
+    f_attn = f_sparse + (4.0 * w.L * w.rank * w.head_dim * BH if br & 2 else 0.0)
 
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     stage_ms = []
@@ -299,10 +320,11 @@ def run_ours(args, w, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16 tensor-core operands, fp32 accumulate, fp64 selection",
         "data": "synthetic (seeded clustered-Gaussian bf16 q/k/v, A ~ N(0, 1/d_h)); inputs resident in HBM",
         "config": {"workload": base_w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
-                   "block": w.block, "keep_frac": w.keep_frac, "keep_blocks": int(idx.shape[-1]),
+                   "block": w.block, "keep_frac": w.keep_frac, "keep_blocks": keep_blocks,
                    "out_dtype": "f32", "l2": "flushed between timed steps (512 MB write)",
                    "parallelism": f"replica x{world} (independent problems, no collective)",
-                   "activation": args.activation, "lowrank_rope": not args.lowrank_norope},
+                   "activation": args.activation, "lowrank_rope": not args.lowrank_norope,
+                   "branches": args.branches, "linear_baseline": bool(args.linear_baseline)},
         "flops_per_step": {"sparse_kept": f_sparse, "lowrank": f_lr, "scores": f_sc},
         "roofline": {"kernel": "attn_sm100_kernel", "bound": "tensor", "achieved": achieved, "peak": tf_sust,
                      "unit": "TFLOP/s", "frac": achieved / tf_sust, "traffic": traffic,
@@ -345,8 +367,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--activation", default="relu", choices=sorted(ACTS), help="low-rank feature map")
     ap.add_argument("--lowrank-norope", action="store_true", help="low-rank branch without its RoPE")
+    ap.add_argument("--linear-baseline", action="store_true",
+                    help="full-width linear-attention branch: rank = head_dim, A = I, relu, no low-rank RoPE")
+    ap.add_argument("--branches", default="both", choices=["both", "sparse", "lowrank"])
     args = ap.parse_args()
     w = WL.by_name(args.workload)
+    if args.linear_baseline:
+        args.lowrank_norope = True
+        args.activation = "relu"
+        w = w.with_(name=w.name + "-linear", rank=w.head_dim)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -360,10 +360,17 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
         return SLRA_ERR_CUDA;
 
     if ((s = begin(p, d, w, st)) != SLRA_OK) return s;
-    if (branches & SLRA_BRANCH_SPARSE)
+    // a branch that is off still records its stage boundaries, so its stages time as zero
+    if (branches & SLRA_BRANCH_SPARSE) {
         if ((s = run_select(p, d, w, q, k, v, st)) != SLRA_OK) return s;
-    if (branches & SLRA_BRANCH_LOWRANK)
+    } else if ((s = mark(p, 2, st)) != SLRA_OK || (s = mark(p, 3, st)) != SLRA_OK) {
+        return s;
+    }
+    if (branches & SLRA_BRANCH_LOWRANK) {
         if ((s = run_lowrank(p, d, w, k, v, A, st)) != SLRA_OK) return s;
+    } else if ((s = mark(p, 4, st)) != SLRA_OK || (s = mark(p, 5, st)) != SLRA_OK) {
+        return s;
+    }
 
     AttnArgs a;
     a.qh = w.qh;

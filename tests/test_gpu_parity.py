@@ -108,6 +108,23 @@ def test_lowrank_without_rope():
           activation=slra.ACT_SILU, lowrank_norope=1, transform=_nonneg)
 
 
+def _identity_A(x):
+    """A = I (bf16 1.0 on the diagonal) for a rank equal to head_dim."""
+    y = dict(x)
+    D = x["A"].shape[0]
+    a = np.zeros((D, D), dtype=np.uint16)
+    a[np.arange(D), np.arange(D)] = 0x3F80
+    y["A"] = a
+    return y
+
+
+def test_full_width_linear_baseline():
+    """r = D, A = I, relu, no low-rank RoPE: ReLU linear attention with a D x D context (the
+    pages' full-width linear branch), on both readout paths."""
+    _case(W.TINY.with_(rank=64), "tiny-linear", lowrank_norope=1, transform=_identity_A)
+    _case(EDGE_128.with_(rank=128), "edge128-linear", lowrank_norope=1, transform=_identity_A)
+
+
 def test_shift_invariance_on_gpu():
     """Shifting all positions leaves the masks unchanged exactly (fp64 selection) and the outputs
     unchanged up to the fp16 rounding of the rotated operands, which differs between the two runs:

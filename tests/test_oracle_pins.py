@@ -260,6 +260,22 @@ def test_lowrank_without_rope(oracle_mod):
     assert not np.allclose(r2["out_lowrank"], r0["out_lowrank"], rtol=1e-3)
 
 
+def test_full_width_linear_attention_baseline(oracle_mod):
+    """r = D, A = I, relu, no low-rank RoPE: the branch is ReLU linear attention with a D x D
+    context, out_i = relu(q_i) (relu(K)^T V) / (relu(q_i) . sum_j relu(k_j) + 1e-6) -- the full-width
+    linear branch the pages compare against (RoPeSLR appendix FLOP analysis, RoLA App. F)."""
+    w = W.TINY.with_(rank=64)
+    x = I.make_inputs(w)
+    dec = oracle_mod.decode_bf16
+    q, k, v = dec(x["q"][0, :, 1]), dec(x["k"][0, :, 1]), dec(x["v"][0, :, 1])
+    r = oracle_mod.head_forward(q, k, v, np.eye(64), (w.T, w.H, w.W), w.block, w.keep_frac, 64, branches=2,
+                                lowrank_rope=False)
+    fq, fk = np.maximum(q, 0), np.maximum(k, 0)
+    ctx = fk.T @ v                      # D x D context, computed once per head
+    ref = (fq @ ctx) / (fq @ fk.sum(0) + 1e-6)[:, None]
+    assert np.allclose(r["out_lowrank"], ref, rtol=1e-12, atol=1e-14)
+
+
 def test_lowrank_summary_equals_quadratic(oracle_mod):
     """The query-independent summary form (RoLA B.1) equals the explicit L x L quadratic form."""
     w = W.TINY
