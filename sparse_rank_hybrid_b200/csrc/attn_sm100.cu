@@ -348,13 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pv_done(j);
                 if (has_s) s_done(j + 2);
             }
-            if (!ok) {
-                fail();
-                // one more commit tracks every product issued so far (they complete in order)
-                umma_commit(bars + kBarDrain);
-                volatile int no_abort = 0;
-                mbar_wait(bars + kBarDrain, 0, 10000000ull, &no_abort);
-            }
+            if (!ok) fail();
+            // One more commit tracks every product this thread issued; waiting for it (bounded, whatever
+            // the abort flag says) means none of them outlives the CTA, however the other roles end.
+            umma_commit(bars + kBarDrain);
+            volatile int no_abort = 0;
+            mbar_wait(bars + kBarDrain, 0, 10000000ull, &no_abort);
         }
         __syncwarp();
     } else {
