@@ -193,11 +193,13 @@ def lowrank_apply(psiq, phiq, S, z, rows=None) -> np.ndarray:
 
 def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, theta=1e4,
                  offset=(0, 0, 0), split=None, qblocks=None, branches=3, idx_override=None,
-                 activation=ACT_RELU, lowrank_rope=True):
+                 activation=ACT_RELU, lowrank_rope=True, A_k=None):
     """Forward pass of one (batch, head): q, k, v fp64 [L, D]; A fp64 [D, R].
 
     `activation` picks the feature map's nonlinearity; `lowrank_rope=False` drops the truncated RoPE
-    from the low-rank branch (psi = phi), the no-RoPE setting of RoLA's ablation (5.3).
+    from the low-rank branch (psi = phi), the no-RoPE setting of RoLA's ablation (5.3).  `A_k`, when
+    given, is a separate key projection Pk (RoLA E.2 lists Pq and Pk as the branch's parameters):
+    query features use A, key features use A_k.
 
     Returns a dict with out (rows of the computed query blocks; NaN elsewhere), the sparse and
     low-rank branch outputs, the rotated q/k, block means, scores, idx, tie flags, S and z.
@@ -227,7 +229,7 @@ def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, t
         res["out_sparse"] = o_s
         out[rows] += o_s[rows]
     phiq = features(q, A, activation)
-    phik = features(k, A, activation)
+    phik = features(k, A if A_k is None else A_k, activation)
     if lowrank_rope:
         psiq = rope_rows(phiq, grid, R // 2, theta, offset, split, schedule_dim=D)
         psik = rope_rows(phik, grid, R // 2, theta, offset, split, schedule_dim=D)
@@ -245,8 +247,12 @@ def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, t
 
 def forward(inp: dict, grid, block: int, keep_frac: float, rank: int, *, theta=1e4, offset=(0, 0, 0),
             split=None, heads=None, qblocks=None, branches=3, idx_override=None, keep_intermediates=False,
-            activation=ACT_RELU, lowrank_rope=True):
+            activation=ACT_RELU, lowrank_rope=True, proj_separate=False, proj_per_head=False):
     """Full forward over all (batch, head) pairs of bf16 inputs q, k, v [B, L, Hh, D] and A [D, R].
+
+    With `proj_separate` and/or `proj_per_head`, A holds [1 + separate][per_head ? Hh : 1][D][R]
+    bf16 values: the query projection(s) first, then the key projection(s) (RoLA E.2's Pq, Pk;
+    RoPeSLR's head-wise low-rank parameterization); head h uses entry h of each.
 
     heads: optional list of (b, h) to compute (default all).  qblocks: dict {(b, h): [alpha...]} or a
     list applied to every head (default all query blocks).  Returns per-(b, h) dicts of results plus
@@ -254,7 +260,7 @@ def forward(inp: dict, grid, block: int, keep_frac: float, rank: int, *, theta=1
     """
     q, k, v, A = inp["q"], inp["k"], inp["v"], inp["A"]
     B, L, Hh, D = q.shape
-    Af = decode_bf16(A)
+    Af = decode_bf16(A).reshape(2 if proj_separate else 1, Hh if proj_per_head else 1, D, rank)
     pairs = [(b, h) for b in range(B) for h in range(Hh)] if heads is None else list(heads)
     out = np.full((B, L, Hh, D), np.nan)
     per = {}
@@ -262,9 +268,10 @@ def forward(inp: dict, grid, block: int, keep_frac: float, rank: int, *, theta=1
         qb = qblocks.get((b, h), []) if isinstance(qblocks, dict) else qblocks
         ov = None if idx_override is None else idx_override[b, h]
         r = head_forward(decode_bf16(q[b, :, h, :]), decode_bf16(k[b, :, h, :]), decode_bf16(v[b, :, h, :]),
-                         Af, grid, block, keep_frac, rank, theta=theta, offset=offset, split=split,
-                         qblocks=qb, branches=branches, idx_override=ov, activation=activation,
-                         lowrank_rope=lowrank_rope)
+                         Af[0, h if proj_per_head else 0], grid, block, keep_frac, rank, theta=theta,
+                         offset=offset, split=split, qblocks=qb, branches=branches, idx_override=ov,
+                         activation=activation, lowrank_rope=lowrank_rope,
+                         A_k=Af[-1, h if proj_per_head else 0])
         out[b, :, h, :] = r["out"]
         if not keep_intermediates:
             for key in ("qh", "kh", "phiq", "phik", "psiq", "psik", "out_sparse", "out_lowrank", "out"):

@@ -5,7 +5,9 @@ method's arithmetic.  The recipe stands in for real DiT activations (which are n
 for each of q, k, v in that order, one N(0,1) centroid per (batch, head, frame, 4x4 spatial tile)
 and per-token N(0,1) noise, X = 0.5*noise + centroid, rounded to bf16 (round-to-nearest-even).
 The feature projection A ~ N(0, 1/head_dim) of shape [head_dim, rank] is drawn after v (or from its
-own seed for the sweep workloads), also rounded to bf16.
+own seed for the sweep workloads), also rounded to bf16.  Separate and/or per-head projections
+(make_projections) come from a stream of their own, seeded with the workload seed + 5000, so the
+q/k/v draws stay the same.
 
 Arrays are returned as uint16 numpy arrays holding bf16 bit patterns, laid out [B, L, heads, D]
 (token-major, as a DiT QKV projection emits them) and [D, rank] for A.
@@ -61,3 +63,11 @@ def make_custom(seed: int, B: int, L_or_grid, heads: int, D: int, R: int, scale:
            for n in ("q", "k", "v")}
     out["A"] = f32_to_bf16_bits(rng.standard_normal((D, R), dtype=np.float32) * np.float32(1.0 / np.sqrt(D)))
     return out
+
+
+def make_projections(seed: int, heads: int, D: int, R: int, separate: bool, per_head: bool) -> np.ndarray:
+    """Projection argument for separate (Pq, Pk) and/or per-head projections: bf16 bits of shape
+    [1 + separate, heads if per_head else 1, D, R], query projections first, each entry ~ N(0, 1/D)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    shape = (2 if separate else 1, heads if per_head else 1, D, R)
+    return f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32) * np.float32(1.0 / np.sqrt(D)))

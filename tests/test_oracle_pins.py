@@ -408,3 +408,53 @@ def test_pins_catch_planted_mistakes(oracle_mod):
     unscaled = oracle_mod.sparse_attn(qh * math.sqrt(D), kh, v, 64, idx)
     assert not np.allclose(unscaled, brute.masked_dense_attention(qh, kh, v, np.ones((L, L), bool)),
                            atol=1e-4)
+
+
+# ------------------------------------------------------------------- separate / per-head projections
+def test_separate_projections_relative_form(oracle_mod):
+    """Separate query and key projections Pq != Pk (RoLA E.2): the readout weight of query i on key j
+    is relu(q_i Pq)^T R(p_j - p_i) relu(k_j Pk) over the first r coordinates, and the normaliser uses
+    the unrotated features.  Both are written out here from numpy features and the brute relative
+    kernel, so an oracle that swapped the projections or used one for both sides fails."""
+    rng = np.random.default_rng(11)
+    D, R, grid = 64, 32, (2, 3, 4)
+    L = 24
+    q, k, v = (rng.standard_normal((L, D)) for _ in range(3))
+    Pq, Pk = rng.standard_normal((D, R)) / 8, rng.standard_normal((D, R)) / 8
+    r = oracle_mod.head_forward(q, k, v, Pq, grid, 8, 1.0, R, branches=2, A_k=Pk)
+    fq, fk = np.maximum(q @ Pq, 0), np.maximum(k @ Pk, 0)
+    axis, omega = oracle_mod.rope_pairs(D)
+    pos = brute.grid_positions(grid)
+    wgt = brute.relative_kernel(fq, fk, pos, pos, axis, omega, R // 2)
+    den = fq @ fk.sum(0) + 1e-6
+    assert np.allclose(r["out_lowrank"], (wgt @ v) / den[:, None], rtol=1e-10, atol=1e-12)
+    swapped = oracle_mod.head_forward(q, k, v, Pk, grid, 8, 1.0, R, branches=2, A_k=Pq)
+    assert not np.allclose(swapped["out_lowrank"], r["out_lowrank"], rtol=1e-3)
+
+
+def test_projection_layout_per_head_and_separate(oracle_mod):
+    """forward() with per-head and/or separate projections reads head h's matrices from entry h,
+    query side first: entries equal to the shared matrix reproduce the shared run exactly, a head whose
+    entry is another matrix reproduces a shared run with that matrix, and Pq = A, Pk = B differs from
+    both shared runs."""
+    w = W.TINY
+    x = I.make_inputs(w)
+    grid = (w.T, w.H, w.W)
+    other = I.make_projections(4242, 1, w.head_dim, w.rank, False, False)[0, 0]
+
+    def run(A, **kw):
+        y = dict(x)
+        y["A"] = A
+        return oracle_mod.forward(y, grid, w.block, w.keep_frac, w.rank, branches=2, **kw)[0]
+
+    shared, shared_o = run(x["A"]), run(other)
+    per_head = run(np.stack([x["A"], other])[None], proj_per_head=True)   # head 0: A, head 1: other
+    assert np.array_equal(per_head[:, :, 0], shared[:, :, 0])
+    assert np.array_equal(per_head[:, :, 1], shared_o[:, :, 1])
+    same = run(np.stack([x["A"], x["A"]])[:, None], proj_separate=True)
+    assert np.array_equal(same, shared)
+    mixed = run(np.stack([x["A"], other])[:, None], proj_separate=True)  # Pq = A, Pk = other
+    assert not np.allclose(mixed, shared, rtol=1e-3) and not np.allclose(mixed, shared_o, rtol=1e-3)
+    both = run(np.stack([np.stack([x["A"], other]), np.stack([x["A"], other])]), proj_separate=True,
+               proj_per_head=True)
+    assert np.array_equal(both[:, :, 0], shared[:, :, 0]) and np.array_equal(both[:, :, 1], shared_o[:, :, 1])
