@@ -103,6 +103,8 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------- CPU oracle
 ACTS = {"relu": 0, "silu": 1, "identity": 2, "tanh": 3}
 BRANCHES = {"both": 3, "sparse": 1, "lowrank": 2}
+# projection layouts: (separate Pq / Pk, one per head)
+PROJS = {"shared": (0, 0), "separate": (1, 0), "per-head": (0, 1), "separate-per-head": (1, 1)}
 
 
 def identity_bits(D: int) -> np.ndarray:
@@ -114,8 +116,21 @@ def identity_bits(D: int) -> np.ndarray:
 
 def variant_of(args) -> dict:
     """Low-rank branch options of the run (the oracle's keyword names)."""
+    sep, ph = PROJS[args.proj]
     return {"activation": ACTS[args.activation], "lowrank_rope": not args.lowrank_norope,
-            "branches": BRANCHES[args.branches]}
+            "branches": BRANCHES[args.branches], "proj_separate": bool(sep), "proj_per_head": bool(ph)}
+
+
+def make_run_inputs(args, w) -> dict:
+    """The run's seeded inputs: the workload's q, k, v and A, with A replaced for the linear baseline
+    (A = I) or a separate / per-head projection layout."""
+    x = I.make_inputs(w)
+    if args.linear_baseline:
+        x["A"] = identity_bits(w.head_dim)
+    elif args.proj != "shared":
+        sep, ph = PROJS[args.proj]
+        x["A"] = I.make_projections(w.seed + 5000, w.heads, w.head_dim, w.rank, bool(sep), bool(ph))
+    return x
 
 
 def oracle_sample(w, x, variant: dict, seconds_hint: float = 15.0):
@@ -160,9 +175,7 @@ def run_reference(args, w, rank, world):
     """Reference arm: the CPU oracle timed step by step on a bounded sample of the workload."""
     if rank != 0:
         return
-    x = I.make_inputs(w)
-    if args.linear_baseline:
-        x["A"] = identity_bits(w.head_dim)
+    x = make_run_inputs(args, w)
     import oracle
     oracle.build()
     grid = (w.T, w.H, w.W)
@@ -195,9 +208,10 @@ def run_reference(args, w, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded clustered-Gaussian bf16 q/k/v, A ~ N(0, 1/d_h))",
-            "config": {"workload": base_w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
+            "config": {"workload": w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
                        "block": w.block, "keep_frac": w.keep_frac, "activation": args.activation,
-                       "lowrank_rope": not args.lowrank_norope},
+                       "lowrank_rope": not args.lowrank_norope, "branches": args.branches,
+                       "linear_baseline": bool(args.linear_baseline), "projection": args.proj},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -219,10 +233,8 @@ def run_ours(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     base_w = w
     w = replicas.replica_workload(base_w, rank)  # each rank: its own independent problem
-    x = I.make_inputs(w)
-    if args.linear_baseline:
-        x["A"] = identity_bits(w.head_dim)
-    q, k, v, A = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v", "A"))
+    x = make_run_inputs(args, w)
+    q, k, v = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v"))
     stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
     for e in stage_ev:
         e.record()
@@ -230,7 +242,9 @@ def run_ours(args, w, rank, world, local_rank):
     var = variant_of(args)
     br = BRANCHES[args.branches]
     prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev), branches=br,
-                                      activation=var["activation"], lowrank_norope=int(not var["lowrank_rope"]))
+                                      activation=var["activation"], lowrank_norope=int(not var["lowrank_rope"]),
+                                      proj_separate=int(var["proj_separate"]), proj_per_head=int(var["proj_per_head"]))
+    A = torch.from_numpy(x["A"].view(np.int16)).view(torch.bfloat16).to(dev).reshape(prob.projection_shape)
     ws = slra.alloc_workspace(prob, dev)
     out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
@@ -324,7 +338,8 @@ def run_ours(args, w, rank, world, local_rank):
                    "out_dtype": "f32", "l2": "flushed between timed steps (512 MB write)",
                    "parallelism": f"replica x{world} (independent problems, no collective)",
                    "activation": args.activation, "lowrank_rope": not args.lowrank_norope,
-                   "branches": args.branches, "linear_baseline": bool(args.linear_baseline)},
+                   "branches": args.branches, "linear_baseline": bool(args.linear_baseline),
+                   "projection": args.proj},
         "flops_per_step": {"sparse_kept": f_sparse, "lowrank": f_lr, "scores": f_sc},
         "roofline": {"kernel": "attn_sm100_kernel", "bound": "tensor", "achieved": achieved, "peak": tf_sust,
                      "unit": "TFLOP/s", "frac": achieved / tf_sust, "traffic": traffic,
@@ -370,7 +385,11 @@ def main():
     ap.add_argument("--linear-baseline", action="store_true",
                     help="full-width linear-attention branch: rank = head_dim, A = I, relu, no low-rank RoPE")
     ap.add_argument("--branches", default="both", choices=["both", "sparse", "lowrank"])
+    ap.add_argument("--proj", default="shared", choices=list(PROJS),
+                    help="query/key projection layout: one shared A, separate Pq/Pk, per head, or both")
     args = ap.parse_args()
+    if args.linear_baseline and args.proj != "shared":
+        ap.error("--linear-baseline uses A = I (one shared projection)")
     w = WL.by_name(args.workload)
     if args.linear_baseline:
         args.lowrank_norope = True

@@ -21,7 +21,9 @@
  *   K(alpha)    = the k = clamp(round(keep_frac * nb), 1, nb) key blocks with the largest
  *                 qbar_alpha . kbar_beta, ties to the lower block index
  *   O_sparse_i  = softmax_j(qh_i . kh_j / sqrt(D)) v_j over the keys of K(alpha(i))
- *   phi(x)      = relu(x A) on raw q, k (or SiLU / identity / tanh, slra_problem.activation);
+ *   phi(x)      = relu(x P) on raw q, k (or SiLU / identity / tanh, slra_problem.activation), with
+ *                 P = Pq for queries and Pk for keys (one shared matrix A by default; separate and
+ *                 per-head projections are options, see slra_problem.proj_separate / proj_per_head);
  *               psi = phi with its first r coordinates rotated like RoPE (unless lowrank_norope)
  *   S = sum_j psi(k_j) v_j^T (r x D),  z = sum_j phi(k_j)   (all L keys, per head)
  *   O_lowrank_i = psi(q_i)^T S / (phi(q_i) . z + 1e-6)
@@ -49,7 +51,7 @@
 extern "C" {
 #endif
 
-#define SLRA_ABI_VERSION 2
+#define SLRA_ABI_VERSION 3
 
 /* Exported symbols (the library is built with hidden visibility for everything else). */
 #if defined(__GNUC__)
@@ -123,6 +125,13 @@ typedef enum slra_activation {
  *   lowrank_norope          0 (default): the low-rank branch rotates the first r feature coordinates
  *                           with the truncated 3D RoPE after the activation (RoLA "4.2", "4.3");
  *                           1: no rotation, psi = phi (the no-RoPE setting of RoLA "5.3").
+ *   proj_separate           0 (default): one projection serves queries and keys; 1: separate query and
+ *                           key projections Pq, Pk (the parameters RoLA "E.2" lists).
+ *   proj_per_head           0 (default): one projection (or pair) for all heads; 1: one per head (the
+ *                           head-wise low-rank parameterization of RoPeSLR's abstract).
+ *                           Both flags only change how the A argument is laid out:
+ *                           bf16 [1 + proj_separate][proj_per_head ? heads : 1][D][rank], the query
+ *                           projection(s) first; slra_projection_elems gives its element count.
  */
 typedef struct slra_problem {
     int64_t batch, heads, head_dim;
@@ -140,6 +149,8 @@ typedef struct slra_problem {
     void* stage_events[7];
     int32_t activation;
     int32_t lowrank_norope;
+    int32_t proj_separate;
+    int32_t proj_per_head;
 } slra_problem;
 
 /*
@@ -176,13 +187,19 @@ SLRA_API slra_status slra_validate(const slra_problem* p);
 /* Kept key blocks per query block, k = clamp(floor(keep_frac * nb + 0.5), 1, nb); -1 if invalid. */
 SLRA_API int64_t slra_keep_count(const slra_problem* p);
 
+/* Number of bf16 elements the projection argument A holds:
+ * (1 + proj_separate) * (proj_per_head ? heads : 1) * head_dim * rank; -1 if the problem is invalid. */
+SLRA_API int64_t slra_projection_elems(const slra_problem* p);
+
 /* Workspace size and the offsets of the intermediates in it.  No GPU access. */
 SLRA_API slra_status slra_workspace_layout(const slra_problem* p, slra_ws_layout* layout);
 
 /*
  * Full forward pass (RoLA "4.1" sparse + low-rank hybrid; all steps listed at the top of this file).
  *   q, k, v    bf16 [B][L][Hh][D] contiguous (token-major), 16-B aligned.
- *   A          bf16 [D][rank] contiguous, the feature projection shared by all heads and by q and k.
+ *   A          bf16 projection(s), contiguous, 16-B aligned: [D][rank] shared by q, k and all heads by
+ *              default; [1 + proj_separate][proj_per_head ? Hh : 1][D][rank] in general (query
+ *              projections first, then key projections).
  *   out        [B][L][Hh][D] contiguous, fp32 or bf16 as p->out_dtype; must not alias q, k, v.
  *   workspace  device buffer of at least layout.total_bytes bytes, 256-B aligned.
  * Launches 6 kernels on `stream` (tables, RoPE + pooling, selection, low-rank partial sums and their
@@ -192,9 +209,10 @@ SLRA_API slra_status slra_attn_fwd(const slra_problem* p, const void* q, const v
                           void* out, void* workspace, size_t workspace_bytes, slra_stream_t stream);
 
 /*
- * The same forward pass on HOST buffers: copies q, k, v, A from host memory into `io` (a device
- * buffer of at least slra_host_io_bytes(p) bytes), runs slra_attn_fwd and copies `out` back to host
- * memory, all on `stream`, then synchronizes the stream.  Host buffers should be pinned for speed.
+ * The same forward pass on HOST buffers: copies q, k, v and A (slra_projection_elems(p) elements)
+ * from host memory into `io` (a device buffer of at least slra_host_io_bytes(p) bytes), runs
+ * slra_attn_fwd and copies `out` back to host memory, all on `stream`, then synchronizes the stream.
+ * Host buffers should be pinned for speed.
  */
 SLRA_API size_t slra_host_io_bytes(const slra_problem* p);
 SLRA_API slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const void* k_host,
@@ -233,7 +251,8 @@ SLRA_API slra_status slra_device_status(void* workspace, slra_stream_t stream, i
  * where cudaMalloc/cudaFree would synchronize the device and stall other streams.
  *
  *   k, v     bf16 [B][L][Hh][D] contiguous, 16-B aligned (device).
- *   A        bf16 [D][rank] contiguous, 16-B aligned (device).
+ *   A        bf16 projection(s) laid out as for slra_attn_fwd, 16-B aligned (device); the summary
+ *            uses the key projection(s).
  *   S        fp32 [B*Hh][rank][D] output (device, 16-B aligned).
  *   z        fp32 [B*Hh][rank]    output (device, 16-B aligned).
  *

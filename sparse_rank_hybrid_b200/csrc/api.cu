@@ -37,6 +37,8 @@ struct Derived {
     int nsplit;
     slra_ws_layout lay;
     size_t at_img, sb_img;  // operand images of the tensor-core readout (offsets; head_dim 128 only)
+    size_t a_elems;         // bf16 elements of the projection argument
+    size_t ak_off;          // elements from its start to the key projection(s)
 };
 
 slra_status derive(const slra_problem* p, Derived* d) {
@@ -48,6 +50,8 @@ slra_status derive(const slra_problem* p, Derived* d) {
     if (p->branches < 0 || p->branches > 3) return SLRA_ERR_INVALID_ARG;
     if (p->activation < SLRA_ACT_RELU || p->activation > SLRA_ACT_TANH) return SLRA_ERR_INVALID_ARG;
     if (p->lowrank_norope != 0 && p->lowrank_norope != 1) return SLRA_ERR_INVALID_ARG;
+    if (p->proj_separate != 0 && p->proj_separate != 1) return SLRA_ERR_INVALID_ARG;
+    if (p->proj_per_head != 0 && p->proj_per_head != 1) return SLRA_ERR_INVALID_ARG;
     if (p->head_dim != 64 && p->head_dim != 128) return SLRA_ERR_UNSUPPORTED;
     if (p->block != 64 && p->block != 128) return SLRA_ERR_UNSUPPORTED;
     if (p->rank < 16 || p->rank > p->head_dim || p->rank % 16 != 0) return SLRA_ERR_UNSUPPORTED;
@@ -79,6 +83,11 @@ slra_status derive(const slra_problem* p, Derived* d) {
     g.Lp = static_cast<int>(nb * p->block);
     g.act = static_cast<int>(p->activation);
     g.norope = static_cast<int>(p->lowrank_norope);
+    g.a_stride = p->proj_per_head ? g.D * g.R : 0;
+    // projection argument: [1 + separate][per_head ? Hh : 1][D][R], query projection(s) first
+    const size_t one_side = static_cast<size_t>(p->proj_per_head ? p->heads : 1) * p->head_dim * p->rank;
+    d->a_elems = one_side * (p->proj_separate ? 2 : 1);
+    d->ak_off = p->proj_separate ? one_side : 0;
 
     RopeMeta& m = d->meta;
     std::memset(&m, 0, sizeof m);
@@ -128,7 +137,7 @@ slra_status derive(const slra_problem* p, Derived* d) {
     w.S = take(static_cast<size_t>(BH) * p->rank * p->head_dim * 4);
     w.z = take(static_cast<size_t>(BH) * p->rank * 4);
     if (p->head_dim == 128) {
-        d->at_img = take(static_cast<size_t>(p->rank) * 256);
+        d->at_img = take(static_cast<size_t>(p->proj_per_head ? p->heads : 1) * p->rank * 256);
         d->sb_img = take(static_cast<size_t>(BH) * ((p->rank + 63) / 64) * kSbChunkBytes);
     } else {
         d->at_img = d->sb_img = 0;
@@ -230,13 +239,14 @@ slra_status run_select(const slra_problem* p, const Derived& d, const Ptrs& w, c
     return mark(p, 3, st);
 }
 
-// Low-rank partial sums: tensor-core kernel for head_dim 128, CUDA-core kernel otherwise.
+// Low-rank partial sums: tensor-core kernel for head_dim 128, CUDA-core kernel otherwise.  A is the
+// whole projection argument; the kernels get the key projection(s).
 cudaError_t lowrank_partial(const Derived& d, const void* k, const void* v, const void* A, const double2* tab,
                             const int2* pairs, int nsplit, float* s_part, float* z_part, int* status,
                             unsigned long long timeout_ns, cudaStream_t st) {
     const auto* kb = static_cast<const __nv_bfloat16*>(k);
     const auto* vb = static_cast<const __nv_bfloat16*>(v);
-    const auto* Ab = static_cast<const __nv_bfloat16*>(A);
+    const auto* Ab = static_cast<const __nv_bfloat16*>(A) + d.ak_off;  // the key projection(s)
     if (d.g.D == 128)
         return launch_lowrank_tc(kb, vb, Ab, tab, d.meta, d.g, nsplit, s_part, z_part, status, timeout_ns, st);
     return launch_lowrank_partial(kb, vb, Ab, tab, pairs, d.g, nsplit, s_part, z_part, st);
@@ -250,6 +260,7 @@ slra_status run_lowrank(const slra_problem* p, const Derived& d, const Ptrs& w, 
     if (e != cudaSuccess) return SLRA_ERR_CUDA;
     slra_status s = mark(p, 4, st);
     if (s != SLRA_OK) return s;
+    // the readout's A^T image comes from the query projection(s), at the start of A
     if ((s = cuda_status(launch_lowrank_reduce(w.s_part, w.z_part, g, d.nsplit, w.S, w.z,
                                                static_cast<const __nv_bfloat16*>(A), w.at_img, w.sb_img, st))) !=
         SLRA_OK)
@@ -310,6 +321,8 @@ slra_status slra_problem_init(slra_problem* p, int64_t batch, int64_t heads, int
     p->wait_timeout_ns = 2000000000ull;
     p->activation = SLRA_ACT_RELU;
     p->lowrank_norope = 0;
+    p->proj_separate = 0;
+    p->proj_per_head = 0;
     return SLRA_OK;
 }
 
@@ -321,6 +334,11 @@ slra_status slra_validate(const slra_problem* p) {
 int64_t slra_keep_count(const slra_problem* p) {
     Derived d;
     return derive(p, &d) == SLRA_OK ? d.g.keep : -1;
+}
+
+int64_t slra_projection_elems(const slra_problem* p) {
+    Derived d;
+    return derive(p, &d) == SLRA_OK ? static_cast<int64_t>(d.a_elems) : -1;
 }
 
 slra_status slra_workspace_layout(const slra_problem* p, slra_ws_layout* layout) {
@@ -343,7 +361,7 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
     const size_t in_b = qkv_bytes(d);
     const size_t out_b = in_b / 2 * (p->out_dtype == SLRA_OUT_F32 ? 4 : 2);
     if (overlaps(out, out_b, q, in_b) || overlaps(out, out_b, k, in_b) || overlaps(out, out_b, v, in_b) ||
-        overlaps(out, out_b, workspace, workspace_bytes))
+        overlaps(out, out_b, A, d.a_elems * 2) || overlaps(out, out_b, workspace, workspace_bytes))
         return SLRA_ERR_INVALID_ARG;
     if ((s = check_device()) != SLRA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -379,7 +397,7 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
     a.idx = w.idx;
     a.keep = (branches & SLRA_BRANCH_SPARSE) ? g.keep : 0;
     a.q_raw = static_cast<const __nv_bfloat16*>(q);
-    a.A = static_cast<const __nv_bfloat16*>(A);
+    a.A = static_cast<const __nv_bfloat16*>(A);  // query projection(s)
     a.S = w.S;
     a.z = w.z;
     a.tab = w.tab;
@@ -402,7 +420,7 @@ size_t slra_host_io_bytes(const slra_problem* p) {
     Derived d;
     if (derive(p, &d) != SLRA_OK) return 0;
     const size_t in_b = align_up(qkv_bytes(d), 256);
-    const size_t a_b = align_up(static_cast<size_t>(d.g.D) * d.g.R * 2, 256);
+    const size_t a_b = align_up(d.a_elems * 2, 256);
     const size_t out_b = align_up(qkv_bytes(d) / 2 * (p->out_dtype == SLRA_OUT_F32 ? 4 : 2), 256);
     return 3 * in_b + a_b + out_b;
 }
@@ -418,7 +436,7 @@ slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t raw = qkv_bytes(d);
     const size_t in_b = align_up(raw, 256);
-    const size_t a_raw = static_cast<size_t>(d.g.D) * d.g.R * 2;
+    const size_t a_raw = d.a_elems * 2;
     const size_t out_raw = raw / 2 * (p->out_dtype == SLRA_OUT_F32 ? 4 : 2);
     uint8_t* b = static_cast<uint8_t*>(io);
     void *dq = b, *dk = b + in_b, *dv = b + 2 * in_b, *dA = b + 3 * in_b;

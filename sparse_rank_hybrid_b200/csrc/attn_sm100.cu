@@ -211,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(bar_eld, 32768 + g.R * 256);
         tma_load_4d(smem, &tm_qraw, bar_eld, 0, h, alpha * blk, b);
         tma_load_4d(smem + 16384, &tm_qraw, bar_eld, 64, h, alpha * blk, b);
-        bulk_load(smem + 32768, a.at_img, g.R * 256, bar_eld);
+        // this head's image when the projections are per head
+        bulk_load(smem + 32768, a.at_img + (g.a_stride ? static_cast<size_t>(h) * g.R * 256 : 0), g.R * 256, bar_eld);
         ++n_eld_issued;
         if (g.R <= 64) {
             const uint32_t zb = static_cast<uint32_t>((3 * g.R + 63) / 64) * (D * 128);
@@ -669,7 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < DH; ++e) acc[e] = 0.f;
         if (a.lowrank && !aborted) {
             float* As = reinterpret_cast<float*>(smem);  // [D][R] fp32, reuses the tile buffers
-            for (int e = tid; e < D * g.R; e += kSoftThreads) As[e] = __bfloat162float(a.A[e]);
+            const __nv_bfloat16* Ah = a.A + static_cast<size_t>(h) * g.a_stride;  // this head's query projection
+            for (int e = tid; e < D * g.R; e += kSoftThreads) As[e] = __bfloat162float(Ah[e]);
             group_sync();
             if (row_valid) {
                 const __nv_bfloat16* qrow = a.q_raw + ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;

@@ -20,6 +20,7 @@ struct Geom {
     int B, Hh, D, T, H, W, L, block, nb, keep, R, Lp;
     int act;     // SLRA_ACT_* of the low-rank feature map
     int norope;  // 1: no rotation in the low-rank branch (psi = phi)
+    int a_stride;  // elements between consecutive heads' projections (D * R when per head, else 0)
     __host__ __device__ int BH() const { return B * Hh; }
 };
 

@@ -6,7 +6,8 @@
 // features) walk work items = (head, range of 128-token tiles).  Per tile:
 //   TMA    raw k and v tiles [128 tokens][128] bf16 straight from the [B][L][Hh][D] inputs (4D tensor
 //          maps, 128-B swizzle, two stages so the next tiles stream in while this one is processed);
-//   MMA    phi = k A  (M = 128 tokens, N = r, K = 128; A^T staged once per CTA as the B operand);
+//   MMA    phi = k A  (M = 128 tokens, N = r, K = 128; A^T staged in shared memory as the B operand:
+//          once per CTA when the projection is shared, again at each change of head when it is per head);
 //   threads (thread = token = TMEM lane) apply the activation (relu unless another is chosen),
 //          accumulate z in registers, rotate the first r coordinates (unless the low-rank RoPE is
 //          off) and write psi as bf16 hi + lo halves (psi = hi + lo to ~2^-16) into shared memory,
@@ -106,12 +107,37 @@ __global__ void __launch_bounds__(256, 1)
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    // A^T as the K-major B operand of phi = k A: row n = feature, 128 dims in two swizzled slabs.
-    for (int e = tid; e < R * kD; e += 256) {
-        const int d = e / R, c = e % R;  // coalesced read of A [D][R]
-        *reinterpret_cast<uint16_t*>(smem + lay.off_at + sw128_offset(c, d, R)) =
-            *reinterpret_cast<const uint16_t*>(a.A + e);
-    }
+    const int ntiles = (g.L + kTok - 1) / kTok;
+    const int n_items = g.BH() * a.nsplit;
+    // The sequence of (item, tile) this CTA processes, flattened, so loads can run ahead.
+    auto tile_of = [&](int q, int& item, int& tile) -> bool {  // q-th tile of this CTA
+        int it = blockIdx.x;
+        while (it < n_items) {
+            const int split = it % a.nsplit;
+            const int t0 = split * a.tiles_per_split, t1 = min(ntiles, t0 + a.tiles_per_split);
+            const int cnt = max(0, t1 - t0);
+            if (q < cnt) { item = it; tile = t0 + q; return true; }
+            q -= cnt;
+            it += gridDim.x;
+        }
+        return false;
+    };
+    auto head_of_tile = [&](int q) -> int {  // head of this CTA's q-th tile (-1 past the end)
+        int item, tile;
+        return tile_of(q, item, tile) ? (item / a.nsplit) % g.Hh : -1;
+    };
+    // A^T as the K-major B operand of phi = k A: row n = feature, 128 dims in two swizzled slabs; with
+    // per-head projections, the matrix of head hd.
+    auto build_at = [&](int hd) {
+        const __nv_bfloat16* Ah = a.A + static_cast<size_t>(hd) * g.a_stride;
+        for (int e = tid; e < R * kD; e += 256) {
+            const int d = e / R, c = e % R;  // coalesced read of A [D][R]
+            *reinterpret_cast<uint16_t*>(smem + lay.off_at + sw128_offset(c, d, R)) =
+                *reinterpret_cast<const uint16_t*>(Ah + e);
+        }
+    };
+    int h_loaded = g.a_stride ? max(0, head_of_tile(0)) : 0;  // head whose projection is staged
+    build_at(h_loaded);
     // zero the padding columns of both psi halves once; tiles only ever write the first R of each half
     for (int e = tid; e < kTok * 2 * RP; e += 256) {
         const int t = e / (2 * RP), col = e % (2 * RP);
@@ -130,21 +156,6 @@ __global__ void __launch_bounds__(256, 1)
                              ((uint32_t(2 * RP) >> 3) << 17) | ((128u >> 4) << 24);
     const uint32_t at_addr = smem_addr(smem + lay.off_at), psi_addr = smem_addr(smem + lay.off_psi);
 
-    const int ntiles = (g.L + kTok - 1) / kTok;
-    const int n_items = g.BH() * a.nsplit;
-    // The sequence of (item, tile) this CTA processes, flattened, so loads can run ahead.
-    auto tile_of = [&](int q, int& item, int& tile) -> bool {  // q-th tile of this CTA
-        int it = blockIdx.x;
-        while (it < n_items) {
-            const int split = it % a.nsplit;
-            const int t0 = split * a.tiles_per_split, t1 = min(ntiles, t0 + a.tiles_per_split);
-            const int cnt = max(0, t1 - t0);
-            if (q < cnt) { item = it; tile = t0 + q; return true; }
-            q -= cnt;
-            it += gridDim.x;
-        }
-        return false;
-    };
     // thread 0's bookkeeping of issued / observed operations (for the bounded drain on abort)
     int n_load[kStages] = {0, 0}, n_wait[kStages] = {0, 0};
     int n_s_issued = 0, n_s_done = 0, n_phi_issued = 0;
@@ -206,12 +217,24 @@ __global__ void __launch_bounds__(256, 1)
             if (tid < R) a.z_part[(static_cast<size_t>(bh) * a.nsplit + split) * R + tid] = 0.f;
             continue;
         }
+        if (g.a_stride && bh % g.Hh != h_loaded) {
+            // Another head's projection.  Its first phi product was held back (below), and every earlier
+            // phi product has completed (each was waited for at its tile's start), so the A^T slot is
+            // free; all threads are past the previous item's closing barrier.
+            h_loaded = bh % g.Hh;
+            build_at(h_loaded);
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0 && !*abort_flag && !issue_phi(q)) fail();
+        }
         float zacc[RH];
 #pragma unroll
         for (int c = 0; c < RH; ++c) zacc[c] = 0.f;
         for (int tile = t0; tile < t1; ++tile, ++q) {
             const int s = q % kStages;
-            // phi_q was issued by thread 0 (at the end of the previous tile, or before the loop); its
+            // phi_q was issued by thread 0 (at the end of the previous tile, before the loop, or after a
+            // change of head's projection at the item start); its
             // completion also means every earlier S product has finished with the psi buffer
             const bool ok = mbar_wait(bar_phi, n_phi & 1, tmo, abort_flag);
             if (__syncthreads_or(!ok)) {
@@ -282,8 +305,9 @@ __global__ void __launch_bounds__(256, 1)
                 umma_commit(bar_s);
                 ++n_s_issued;
                 bool good = true;
-                // the next tile's phi product goes in right behind (its k tile is already loading)
-                if (q + 1 < q_total) good = issue_phi(q + 1);
+                // the next tile's phi product goes in right behind (its k tile is already loading),
+                // unless it needs another head's projection: then it is issued once that is staged
+                if (q + 1 < q_total && (!g.a_stride || head_of_tile(q + 1) == h_loaded)) good = issue_phi(q + 1);
                 // stage s is free once this S product is done: refill it with the tile two ahead
                 if (good && mbar_wait(bar_s, n_s_done & 1, tmo, abort_flag)) {
                     ++n_s_done;

@@ -407,7 +407,8 @@ __global__ void __launch_bounds__(256) lowrank_partial_kernel(const __nv_bfloat1
     const int per = (ntiles + nsplit - 1) / nsplit;
     const int t0 = split * per, t1 = min(ntiles, t0 + per);
 
-    for (int e = tid; e < D * R; e += 256) As[e] = __bfloat162float(A[e]);
+    const __nv_bfloat16* Ah = A + static_cast<size_t>(h) * g.a_stride;  // this head's key projection
+    for (int e = tid; e < D * R; e += 256) As[e] = __bfloat162float(Ah[e]);
     const int e_own = tid % D, cg = tid / D;
     float acc[NA];
 #pragma unroll
@@ -515,11 +516,12 @@ __device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
 // Fixed-order sum of the split-L partials -> S [R][D] and z [R] per head.  With images requested
 // (head_dim 128) it also writes, per head and 64-feature chunk, the S operand image of the attention
 // epilogue's readout product (K columns S_hi | S_lo | S_hi, bf16 split so that hi + lo = S to ~2^-16),
-// and (blocks of head 0) the A^T operand image of its feature product.
+// and the A^T operand image of its feature product from the query projection A: one image written by
+// the blocks of head 0 when A is shared (a_stride 0), else one per head, by the blocks of batch 0.
 __global__ void lowrank_reduce_kernel(const float* __restrict__ s_part, const float* __restrict__ z_part, int RD,
                                       int R, int D, int nsplit, float* __restrict__ S, float* __restrict__ z,
                                       const __nv_bfloat16* __restrict__ A, uint8_t* __restrict__ at_img,
-                                      uint8_t* __restrict__ sb_img) {
+                                      uint8_t* __restrict__ sb_img, int Hh, int a_stride) {
     const int bh = blockIdx.y;
     const int o = blockIdx.x * blockDim.x + threadIdx.x;
     if (o < RD) {
@@ -537,10 +539,11 @@ __global__ void lowrank_reduce_kernel(const float* __restrict__ s_part, const fl
             *reinterpret_cast<uint16_t*>(img + sw128_offset(e, rc + cc, D)) = lo;
             *reinterpret_cast<uint16_t*>(img + sw128_offset(e, 2 * rc + cc, D)) = hi;
         }
-        if (at_img && bh == 0) {  // element (c, d) of A^T = A[d][c]
+        if (at_img && (a_stride == 0 ? bh == 0 : bh < Hh)) {  // element (c, d) of A^T = A[d][c]
             const int c = o / D, d = o % D;
-            *reinterpret_cast<uint16_t*>(at_img + sw128_offset(c, d, R)) =
-                *reinterpret_cast<const uint16_t*>(A + static_cast<size_t>(d) * R + c);
+            const size_t hd = a_stride == 0 ? 0 : static_cast<size_t>(bh);  // bh = head when b = 0
+            *reinterpret_cast<uint16_t*>(at_img + hd * R * 256 + sw128_offset(c, d, R)) =
+                *reinterpret_cast<const uint16_t*>(A + hd * a_stride + static_cast<size_t>(d) * R + c);
         }
     } else if (o < RD + R) {
         const int c = o - RD;
@@ -556,7 +559,8 @@ cudaError_t launch_lowrank_reduce(const float* s_part, const float* z_part, cons
                                   cudaStream_t st) {
     const int RD = g.R * g.D;
     dim3 grid((RD + g.R + 255) / 256, g.BH());
-    lowrank_reduce_kernel<<<grid, 256, 0, st>>>(s_part, z_part, RD, g.R, g.D, nsplit, S, z, A, at_img, sb_img);
+    lowrank_reduce_kernel<<<grid, 256, 0, st>>>(s_part, z_part, RD, g.R, g.D, nsplit, S, z, A, at_img, sb_img, g.Hh,
+                                                g.a_stride);
     return cudaGetLastError();
 }
 

@@ -20,11 +20,12 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DE
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
 DEBUG_UNSATISFIED_WAIT = 1
-ABI_VERSION = 2
+ABI_VERSION = 3
 ACT_RELU, ACT_SILU, ACT_IDENTITY, ACT_TANH = 0, 1, 2, 3
 
 # Every symbol include/slra.h declares.
 EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_validate", "slra_keep_count",
+           "slra_projection_elems",
            "slra_workspace_layout", "slra_attn_fwd", "slra_host_io_bytes", "slra_attn_fwd_host",
            "slra_select_blocks", "slra_lowrank_summary", "slra_device_status", "slra_lowrank_summary_noalloc")
 
@@ -43,7 +44,8 @@ class _Problem(ctypes.Structure):
                 ("pos_offset", ctypes.c_int64 * 3), ("rope_split", ctypes.c_int64 * 3),
                 ("wait_timeout_ns", ctypes.c_uint64), ("debug_flags", ctypes.c_uint32),
                 ("stage_events", ctypes.c_void_p * 7), ("activation", ctypes.c_int32),
-                ("lowrank_norope", ctypes.c_int32)]
+                ("lowrank_norope", ctypes.c_int32), ("proj_separate", ctypes.c_int32),
+                ("proj_per_head", ctypes.c_int32)]
 
 
 class _Layout(ctypes.Structure):
@@ -75,6 +77,8 @@ def lib():
         L.slra_validate.argtypes = [PP]
         L.slra_keep_count.restype = ctypes.c_int64
         L.slra_keep_count.argtypes = [PP]
+        L.slra_projection_elems.restype = ctypes.c_int64
+        L.slra_projection_elems.argtypes = [PP]
         L.slra_workspace_layout.argtypes = [PP, ctypes.POINTER(_Layout)]
         L.slra_attn_fwd.argtypes = [PP, P, P, P, P, P, P, S, P]
         L.slra_host_io_bytes.restype = S
@@ -122,6 +126,8 @@ class Problem:
     stage_events: tuple = (None,) * 7  # raw cudaEvent_t handles (ints) or None, see slra_problem
     activation: int = 0                # ACT_* map of the low-rank features
     lowrank_norope: int = 0            # 1: no RoPE in the low-rank branch
+    proj_separate: int = 0             # 1: separate query / key projections Pq, Pk
+    proj_per_head: int = 0             # 1: one projection (pair) per head
 
     @property
     def L(self) -> int:
@@ -146,7 +152,17 @@ class Problem:
             p.stage_events[i] = e
         p.activation = int(self.activation)
         p.lowrank_norope = int(self.lowrank_norope)
+        p.proj_separate = int(self.proj_separate)
+        p.proj_per_head = int(self.proj_per_head)
         return p
+
+    @property
+    def projection_shape(self) -> tuple:
+        """Shape of the projection argument A: [D, rank] by default, else
+        [1 + proj_separate, proj_per_head ? heads : 1, D, rank] (query projections first)."""
+        if not self.proj_separate and not self.proj_per_head:
+            return (self.head_dim, self.rank)
+        return (1 + int(self.proj_separate), self.heads if self.proj_per_head else 1, self.head_dim, self.rank)
 
 
 @dataclass
@@ -165,6 +181,10 @@ def validate(prob: Problem) -> int:
 
 def keep_count(prob: Problem) -> int:
     return int(lib().slra_keep_count(ctypes.byref(prob.c())))
+
+
+def projection_elems(prob: Problem) -> int:
+    return int(lib().slra_projection_elems(ctypes.byref(prob.c())))
 
 
 def layout(prob: Problem) -> Layout:
@@ -203,13 +223,13 @@ def _check_bf16(name, t, shape):
 
 
 def attn_fwd(prob: Problem, q, k, v, A, out=None, workspace=None, stream=None):
-    """Full forward pass.  q, k, v: CUDA bf16 [B, L, Hh, D]; A: CUDA bf16 [D, rank].
+    """Full forward pass.  q, k, v: CUDA bf16 [B, L, Hh, D]; A: CUDA bf16 of prob.projection_shape.
     Returns (out, workspace); out is fp32 or bf16 [B, L, Hh, D] as prob.out_dtype."""
     torch = _torch()
     shp = (prob.batch, prob.L, prob.heads, prob.head_dim)
     for n, t in (("q", q), ("k", k), ("v", v)):
         _check_bf16(n, t, shp)
-    _check_bf16("A", A, (prob.head_dim, prob.rank))
+    _check_bf16("A", A, prob.projection_shape)
     if out is None:
         out = torch.empty(shp, dtype=torch.float32 if prob.out_dtype == OUT_F32 else torch.bfloat16,
                           device=q.device)
@@ -226,6 +246,8 @@ def host_io_bytes(prob: Problem) -> int:
 
 def attn_fwd_host(prob: Problem, q_host, k_host, v_host, A_host, out_host, io, workspace, stream=None):
     """Forward pass on host buffers (pinned CPU tensors): copies in, computes, copies out, synchronizes."""
+    if A_host.numel() != projection_elems(prob):
+        raise ValueError(f"A_host: expected {projection_elems(prob)} elements, got {A_host.numel()}")
     _check(lib().slra_attn_fwd_host(ctypes.byref(prob.c()), _ptr(q_host), _ptr(k_host), _ptr(v_host),
                                     _ptr(A_host), _ptr(out_host), _ptr(io), io.numel(), _ptr(workspace),
                                     workspace.numel(), _stream_handle(stream)), "slra_attn_fwd_host")
@@ -241,6 +263,7 @@ def select_blocks(prob: Problem, q, k, v, workspace=None, stream=None):
 
 
 def lowrank_summary(prob: Problem, k, v, A, workspace=None, stream=None):
+    _check_bf16("A", A, prob.projection_shape)
     if workspace is None:
         workspace = alloc_workspace(prob, k.device)
     _check(lib().slra_lowrank_summary(ctypes.byref(prob.c()), _ptr(k), _ptr(v), _ptr(A), _ptr(workspace),
@@ -251,6 +274,7 @@ def lowrank_summary(prob: Problem, k, v, A, workspace=None, stream=None):
 def lowrank_summary_noalloc(prob: Problem, k, v, A, S, z, stream=None):
     """Low-rank summary into caller tensors S [B*Hh, rank, D] and z [B*Hh, rank] (fp32, CUDA) without
     any allocation: the library's fixed scratch array is used instead of a workspace."""
+    _check_bf16("A", A, prob.projection_shape)
     _check(lib().slra_lowrank_summary_noalloc(ctypes.byref(prob.c()), _ptr(k), _ptr(v), _ptr(A), _ptr(S), _ptr(z),
                                               _stream_handle(stream)), "slra_lowrank_summary_noalloc")
     return S, z

@@ -72,7 +72,8 @@ def compare(prob: slra.Problem, x: dict, gpu: dict, heads=None, qblocks=None, ch
         override = gpu["idx"].reshape(B, Hh, *gpu["idx"].shape[1:])
     out_o, per = oracle.forward(x, grid, prob.block, prob.keep_frac, prob.rank, offset=prob.pos_offset,
                                 heads=pairs, qblocks=qblocks, branches=prob.branches, idx_override=override,
-                                activation=prob.activation, lowrank_rope=not prob.lowrank_norope)
+                                activation=prob.activation, lowrank_rope=not prob.lowrank_norope,
+                                proj_separate=bool(prob.proj_separate), proj_per_head=bool(prob.proj_per_head))
     stats = {"label": label, "mask_rows_differing": 0, "mask_rows": 0}
     for (b, h) in pairs:
         r = per[(b, h)]

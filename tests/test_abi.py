@@ -4,6 +4,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 from sparse_rank_hybrid_b200 import build as B
@@ -35,7 +36,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_abi_version_and_status_strings():
-    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 2
+    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 3
     for s in range(0, 9):
         assert slra.status_string(s) and slra.status_string(s) != "unknown status"
     assert slra.status_string(99) == "unknown status"
@@ -61,11 +62,29 @@ def test_keep_count_and_layout(w, oracle_mod):
     ("T", 5000, slra.ERR_UNSUPPORTED),  # 5000*45*80 tokens -> more than 2048 blocks
     ("activation", 4, slra.ERR_INVALID_ARG), ("activation", -1, slra.ERR_INVALID_ARG),
     ("lowrank_norope", 2, slra.ERR_INVALID_ARG),
+    ("proj_separate", 2, slra.ERR_INVALID_ARG), ("proj_per_head", -1, slra.ERR_INVALID_ARG),
 ])
 def test_validation_rejects(field, value, status):
     p = slra.Problem.from_workload(W.WAN_14B)
     setattr(p, field, value)
     assert slra.validate(p) == status
+
+
+@pytest.mark.parametrize("separate,per_head", [(0, 0), (1, 0), (0, 1), (1, 1)])
+def test_projection_elems_and_layout(separate, per_head):
+    """The projection argument holds (1 + separate) x (per_head ? heads : 1) matrices of D x rank;
+    per-head projections give the workspace one readout image per head (head_dim 128), and the
+    intermediates keep their offsets."""
+    w = W.WAN_14B
+    p = slra.Problem.from_workload(w, proj_separate=separate, proj_per_head=per_head)
+    n = (1 + separate) * (w.heads if per_head else 1) * w.head_dim * w.rank
+    assert slra.projection_elems(p) == n == int(np.prod(p.projection_shape))
+    base = slra.layout(slra.Problem.from_workload(w))
+    lay = slra.layout(p)
+    assert lay.offsets == base.offsets
+    extra = (w.heads - 1) * w.rank * 256 if per_head else 0
+    assert base.total_bytes + extra <= lay.total_bytes <= base.total_bytes + extra + 256
+    assert slra.projection_elems(slra.Problem.from_workload(w, proj_separate=3)) == -1
 
 
 def test_validation_grid_limit():

@@ -125,6 +125,38 @@ def test_full_width_linear_baseline():
     _case(EDGE_128.with_(rank=128), "edge128-linear", lowrank_norope=1, transform=_identity_A)
 
 
+def _projections(w, separate, per_head):
+    """Replace A by separate (Pq, Pk) and/or per-head projections drawn for this workload."""
+    def t(x):
+        y = dict(x)
+        y["A"] = I.make_projections(w.seed + 5000, w.heads, w.head_dim, w.rank, bool(separate), bool(per_head))
+        return y
+    return t
+
+
+# 8 heads x 24 tiles of 128 tokens = 192 low-rank work items for 148 persistent CTAs, so CTAs take
+# items of two different heads and restage the key projection in between
+EDGE_PROJ = W.Workload("edge-proj-128", 1, 8, 128, 4, 24, 32, 32, 128, 0.1, 7300)
+
+
+@pytest.mark.parametrize("separate,per_head", [(1, 0), (0, 1), (1, 1)])
+def test_projection_variants(separate, per_head):
+    """Separate query / key projections (RoLA E.2's Pq, Pk) and per-head projections (RoPeSLR's
+    head-wise parameterization) on both readout paths, including persistent low-rank CTAs that
+    change head (and so projection) between work items."""
+    for w in (W.TINY, EDGE_128, EDGE_128_R64, EDGE_PROJ):
+        _case(w, f"{w.name}-proj-s{separate}-h{per_head}", proj_separate=separate, proj_per_head=per_head,
+              transform=_projections(w, separate, per_head))
+
+
+def test_projection_per_head_wan_1_3b():
+    """Separate per-head projections at the Wan2.1-1.3B shape (1536 low-rank work items over 148
+    CTAs), on sampled heads and query blocks."""
+    w = W.WAN_1_3B
+    _case(w, "wan1.3b-proj-s1-h1", heads=[(0, 3), (0, 10)], qblocks=_sample_blocks(w.nb, 9, n=2),
+          proj_separate=1, proj_per_head=1, transform=_projections(w, 1, 1))
+
+
 def test_shift_invariance_on_gpu():
     """Shifting all positions leaves the masks unchanged exactly (fp64 selection) and the outputs
     unchanged up to the fp16 rounding of the rotated operands, which differs between the two runs:
