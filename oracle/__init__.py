@@ -62,6 +62,7 @@ def _load():
         _lib.orc_features.argtypes = [P, I, I, P, I, ctypes.c_int, P]
         _lib.orc_summary.argtypes = [P, P, P, I, I, I, P, P]
         _lib.orc_lowrank_apply.argtypes = [P, P, P, P, I, I, P, I, P]
+        _lib.orc_gated_fusion.argtypes = [P, P, P, P, ctypes.c_double, I, P, I, P]
     return _lib
 
 
@@ -191,15 +192,29 @@ def lowrank_apply(psiq, phiq, S, z, rows=None) -> np.ndarray:
     return out
 
 
+def gated_fusion(o_s, o_lr, q, w, b: float, rows) -> np.ndarray:
+    """out_i = O_s,i + sigmoid(q_i . w + b) * O_lr,i * rms(O_s,i) / sqrt(mean(O_lr,i^2) + 1e-6) for the
+    given rows (RoLA 4.4's token-wise gate with the sparse output's RMS as scale reference; the
+    formula is this implementation's reading, see slra_oracle.c)."""
+    o_s, o_lr, q = (np.ascontiguousarray(a, dtype=np.float64) for a in (o_s, o_lr, q))
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    L, D = o_s.shape
+    rr = np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.zeros((L, D))
+    _load().orc_gated_fusion(_p(o_s), _p(o_lr), _p(q), _p(w), float(b), D, _p(rr), rr.size, _p(out))
+    return out
+
+
 def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, theta=1e4,
                  offset=(0, 0, 0), split=None, qblocks=None, branches=3, idx_override=None,
-                 activation=ACT_RELU, lowrank_rope=True, A_k=None):
+                 activation=ACT_RELU, lowrank_rope=True, A_k=None, gate=None):
     """Forward pass of one (batch, head): q, k, v fp64 [L, D]; A fp64 [D, R].
 
     `activation` picks the feature map's nonlinearity; `lowrank_rope=False` drops the truncated RoPE
     from the low-rank branch (psi = phi), the no-RoPE setting of RoLA's ablation (5.3).  `A_k`, when
     given, is a separate key projection Pk (RoLA E.2 lists Pq and Pk as the branch's parameters):
-    query features use A, key features use A_k.
+    query features use A, key features use A_k.  `gate=(w, b)` replaces the plain sum of the two
+    branches by the gated fusion of RoLA 4.4 (see gated_fusion; needs both branches).
 
     Returns a dict with out (rows of the computed query blocks; NaN elsewhere), the sparse and
     low-rank branch outputs, the rotated q/k, block means, scores, idx, tie flags, S and z.
@@ -240,19 +255,24 @@ def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, t
     if branches & 2:
         o_lr = lowrank_apply(psiq, phiq, S, z, rows)
         res["out_lowrank"] = o_lr
-        out[rows] += o_lr[rows]
+        if gate is None:
+            out[rows] += o_lr[rows]
+        else:
+            assert branches == 3, "the gated fusion combines both branches"
+            out[rows] = gated_fusion(res["out_sparse"], o_lr, q, gate[0], gate[1], rows)[rows]
     res["out"] = out
     return res
 
 
 def forward(inp: dict, grid, block: int, keep_frac: float, rank: int, *, theta=1e4, offset=(0, 0, 0),
             split=None, heads=None, qblocks=None, branches=3, idx_override=None, keep_intermediates=False,
-            activation=ACT_RELU, lowrank_rope=True, proj_separate=False, proj_per_head=False):
+            activation=ACT_RELU, lowrank_rope=True, proj_separate=False, proj_per_head=False, gate=None):
     """Full forward over all (batch, head) pairs of bf16 inputs q, k, v [B, L, Hh, D] and A [D, R].
 
     With `proj_separate` and/or `proj_per_head`, A holds [1 + separate][per_head ? Hh : 1][D][R]
     bf16 values: the query projection(s) first, then the key projection(s) (RoLA E.2's Pq, Pk;
-    RoPeSLR's head-wise low-rank parameterization); head h uses entry h of each.
+    RoPeSLR's head-wise low-rank parameterization); head h uses entry h of each.  `gate=(w, b)`: the
+    gated fusion of the branches (w fp64 [D] shared by all heads, b a scalar).
 
     heads: optional list of (b, h) to compute (default all).  qblocks: dict {(b, h): [alpha...]} or a
     list applied to every head (default all query blocks).  Returns per-(b, h) dicts of results plus
@@ -271,7 +291,7 @@ def forward(inp: dict, grid, block: int, keep_frac: float, rank: int, *, theta=1
                          Af[0, h if proj_per_head else 0], grid, block, keep_frac, rank, theta=theta,
                          offset=offset, split=split, qblocks=qb, branches=branches, idx_override=ov,
                          activation=activation, lowrank_rope=lowrank_rope,
-                         A_k=Af[-1, h if proj_per_head else 0])
+                         A_k=Af[-1, h if proj_per_head else 0], gate=gate)
         out[b, :, h, :] = r["out"]
         if not keep_intermediates:
             for key in ("qh", "kh", "phiq", "phik", "psiq", "psik", "out_sparse", "out_lowrank", "out"):

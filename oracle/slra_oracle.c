@@ -308,3 +308,31 @@ ORC_EXPORT void orc_lowrank_apply(const double* psiq, const double* phiq, const 
         }
     }
 }
+
+/*
+ * Gated fusion of the two branches (RoLA "4.4": a token-wise scalar gate combines the sparse and the
+ * global output, the sparse output's RMS is the scale reference, and a negative gate bias starts the
+ * module near the sparse-only output; "E.2" names the gate parameters Wg, bg).  The pages give no
+ * formula; the reading implemented here, for each query row i of one head:
+ *   g_i    = 1 / (1 + exp(-(q_i . w + b)))          q_i the raw (pre-RoPE) query, w = Wg [D], b = bg
+ *   rms(x) = sqrt(sum_e x[e]^2 / D)
+ *   out_i  = O_s,i + g_i * O_lr,i * rms(O_s,i) / sqrt(sum_e O_lr,i[e]^2 / D + 1e-6)
+ * i.e. the global output is brought to the sparse output's RMS and then gated.
+ */
+ORC_EXPORT void orc_gated_fusion(const double* os, const double* olr, const double* q, const double* w, double b,
+                                 int64_t D, const int64_t* rows, int64_t nrows, double* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < nrows; ++t) {
+        int64_t i = rows[t];
+        double logit = b;
+        for (int64_t e = 0; e < D; ++e) logit += q[i * D + e] * w[e];
+        double g = 1.0 / (1.0 + exp(-logit));
+        double ss = 0.0, sl = 0.0;
+        for (int64_t e = 0; e < D; ++e) {
+            ss += os[i * D + e] * os[i * D + e];
+            sl += olr[i * D + e] * olr[i * D + e];
+        }
+        double scale = sqrt(ss / (double)D) / sqrt(sl / (double)D + 1e-6);
+        for (int64_t e = 0; e < D; ++e) out[i * D + e] = os[i * D + e] + g * olr[i * D + e] * scale;
+    }
+}

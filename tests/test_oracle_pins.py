@@ -458,3 +458,63 @@ def test_projection_layout_per_head_and_separate(oracle_mod):
     both = run(np.stack([np.stack([x["A"], other]), np.stack([x["A"], other])]), proj_separate=True,
                proj_per_head=True)
     assert np.array_equal(both[:, :, 0], shared[:, :, 0]) and np.array_equal(both[:, :, 1], shared_o[:, :, 1])
+
+
+# ------------------------------------------------------------------------------------ gated fusion
+def _gated(oracle_mod, w_gate, b_gate, v_scale=1.0):
+    w = W.TINY
+    x = I.make_inputs(w)
+    dec = oracle_mod.decode_bf16
+    q, k, v = dec(x["q"][0, :, 0]), dec(x["k"][0, :, 0]), dec(x["v"][0, :, 0]) * v_scale
+    r = oracle_mod.head_forward(q, k, v, dec(x["A"]), (w.T, w.H, w.W), w.block, w.keep_frac, w.rank,
+                                gate=(np.asarray(w_gate, dtype=np.float64), b_gate))
+    return r, q
+
+
+def _rms(a):
+    return np.sqrt((a ** 2).mean(axis=1))
+
+
+def test_gate_closed_is_sparse_only(oracle_mod):
+    """A very negative gate bias closes the gate: the output is the sparse branch alone, the
+    module's starting point (RoLA 4.4)."""
+    r, _ = _gated(oracle_mod, np.zeros(64), -1e4)
+    assert np.array_equal(r["out"], r["out_sparse"])
+
+
+def test_gate_half_open_adds_half_the_sparse_rms(oracle_mod):
+    """w = 0, b = 0: the gate is 1/2 on every row, the added term points along the low-rank output
+    and its RMS is half the sparse output's (the scale reference), up to the 1e-6 in the normaliser."""
+    r, _ = _gated(oracle_mod, np.zeros(64), 0.0)
+    add = r["out"] - r["out_sparse"]
+    lr = r["out_lowrank"]
+    eps_f = _rms(lr) / np.sqrt(_rms(lr) ** 2 + 1e-6)
+    assert np.allclose(_rms(add), 0.5 * _rms(r["out_sparse"]) * eps_f, rtol=1e-10)
+    cos = (add * lr).sum(1) / (np.linalg.norm(add, axis=1) * np.linalg.norm(lr, axis=1))
+    assert np.allclose(cos, 1.0, atol=1e-12)
+
+
+def test_gate_reads_the_raw_query(oracle_mod):
+    """w = e_0, b = 0: the gate of row i, recovered from the RMS of the added term, is sigmoid(q_i[0])
+    of the raw (pre-RoPE) query; the rotated query would give another value on rows with t > 0."""
+    w_gate = np.zeros(64)
+    w_gate[0] = 1.0
+    r, q = _gated(oracle_mod, w_gate, 0.0)
+    lr = r["out_lowrank"]
+    unit = _rms(r["out_sparse"]) * _rms(lr) / np.sqrt(_rms(lr) ** 2 + 1e-6)
+    g = _rms(r["out"] - r["out_sparse"]) / unit
+    assert np.allclose(g, 1.0 / (1.0 + np.exp(-q[:, 0])), rtol=1e-9)
+    assert not np.allclose(g, 1.0 / (1.0 + np.exp(-r["qh"][:, 0])), rtol=1e-3)
+
+
+def test_gate_is_homogeneous_in_v(oracle_mod):
+    """Both branches are linear in v and the RMS ratio does not change when v is scaled, so scaling v
+    by 2 doubles the gated output, up to the 1e-6 in the RMS normaliser (here a relative effect of at
+    most 1e-6 / (2 mean(O_lr^2)) ~ 3e-5 on the added term).  A scale reference that is not of degree
+    one in v (say the mean square instead of the RMS) fails by a factor of 2."""
+    rng = np.random.default_rng(3)
+    w_gate = rng.standard_normal(64) / 8
+    r1, _ = _gated(oracle_mod, w_gate, -1.0)
+    r2, _ = _gated(oracle_mod, w_gate, -1.0, v_scale=2.0)
+    ref = 2.0 * r1["out"]
+    assert np.abs(r2["out"] - ref).max() <= 5e-5 * np.abs(ref).max()
