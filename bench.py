@@ -114,11 +114,22 @@ def identity_bits(D: int) -> np.ndarray:
     return a
 
 
-def variant_of(args) -> dict:
-    """Low-rank branch options of the run (the oracle's keyword names)."""
+GATE_BIAS = -2.0  # negative: the gated fusion starts near the sparse output (RoLA 4.4)
+
+
+def gate_weights(w) -> np.ndarray:
+    """Synthetic gate weights Wg ~ N(0, 1/head_dim), fp32, from the workload seed + 6000."""
+    rng = np.random.default_rng(w.seed + 6000)
+    return (rng.standard_normal(w.head_dim) / np.sqrt(w.head_dim)).astype(np.float32)
+
+
+def variant_of(args, w) -> dict:
+    """Low-rank branch and fusion options of the run (the oracle's keyword names)."""
     sep, ph = PROJS[args.proj]
+    gate = (gate_weights(w).astype(np.float64), GATE_BIAS) if args.fusion == "gated" else None
     return {"activation": ACTS[args.activation], "lowrank_rope": not args.lowrank_norope,
-            "branches": BRANCHES[args.branches], "proj_separate": bool(sep), "proj_per_head": bool(ph)}
+            "branches": BRANCHES[args.branches], "proj_separate": bool(sep), "proj_per_head": bool(ph),
+            "gate": gate}
 
 
 def make_run_inputs(args, w) -> dict:
@@ -185,7 +196,7 @@ def run_reference(args, w, rank, world):
     def step():
         t0 = time.perf_counter()
         _, per = oracle.forward(x, grid, w.block, w.keep_frac, w.rank, heads=[(0, 0)], qblocks=qbs,
-                                **variant_of(args))
+                                **variant_of(args, w))
         return time.perf_counter() - t0, per[(0, 0)]
 
     for _ in range(args.warmup):
@@ -211,7 +222,8 @@ def run_reference(args, w, rank, world):
             "config": {"workload": w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
                        "block": w.block, "keep_frac": w.keep_frac, "activation": args.activation,
                        "lowrank_rope": not args.lowrank_norope, "branches": args.branches,
-                       "linear_baseline": bool(args.linear_baseline), "projection": args.proj},
+                       "linear_baseline": bool(args.linear_baseline), "projection": args.proj,
+                       "fusion": args.fusion},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -239,11 +251,16 @@ def run_ours(args, w, rank, world, local_rank):
     for e in stage_ev:
         e.record()
     torch.cuda.synchronize()
-    var = variant_of(args)
+    var = variant_of(args, w)
     br = BRANCHES[args.branches]
+    gate_kw = {}
+    if args.fusion == "gated":
+        gate_kw = dict(fusion=slra.FUSION_GATED, gate_bias=GATE_BIAS,
+                       gate_w=torch.from_numpy(gate_weights(w)).to(dev))
     prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev), branches=br,
                                       activation=var["activation"], lowrank_norope=int(not var["lowrank_rope"]),
-                                      proj_separate=int(var["proj_separate"]), proj_per_head=int(var["proj_per_head"]))
+                                      proj_separate=int(var["proj_separate"]), proj_per_head=int(var["proj_per_head"]),
+                                      **gate_kw)
     A = torch.from_numpy(x["A"].view(np.int16)).view(torch.bfloat16).to(dev).reshape(prob.projection_shape)
     ws = slra.alloc_workspace(prob, dev)
     out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
@@ -339,7 +356,7 @@ def run_ours(args, w, rank, world, local_rank):
                    "parallelism": f"replica x{world} (independent problems, no collective)",
                    "activation": args.activation, "lowrank_rope": not args.lowrank_norope,
                    "branches": args.branches, "linear_baseline": bool(args.linear_baseline),
-                   "projection": args.proj},
+                   "projection": args.proj, "fusion": args.fusion},
         "flops_per_step": {"sparse_kept": f_sparse, "lowrank": f_lr, "scores": f_sc},
         "roofline": {"kernel": "attn_sm100_kernel", "bound": "tensor", "achieved": achieved, "peak": tf_sust,
                      "unit": "TFLOP/s", "frac": achieved / tf_sust, "traffic": traffic,
@@ -387,7 +404,11 @@ def main():
     ap.add_argument("--branches", default="both", choices=["both", "sparse", "lowrank"])
     ap.add_argument("--proj", default="shared", choices=list(PROJS),
                     help="query/key projection layout: one shared A, separate Pq/Pk, per head, or both")
+    ap.add_argument("--fusion", default="sum", choices=["sum", "gated"],
+                    help="combine the branches by their sum or by the token-wise gate (synthetic Wg, bg = -2)")
     args = ap.parse_args()
+    if args.fusion == "gated" and args.branches != "both":
+        ap.error("--fusion gated needs both branches")
     if args.linear_baseline and args.proj != "shared":
         ap.error("--linear-baseline uses A = I (one shared projection)")
     w = WL.by_name(args.workload)

@@ -27,7 +27,10 @@
  *               psi = phi with its first r coordinates rotated like RoPE (unless lowrank_norope)
  *   S = sum_j psi(k_j) v_j^T (r x D),  z = sum_j phi(k_j)   (all L keys, per head)
  *   O_lowrank_i = psi(q_i)^T S / (phi(q_i) . z + 1e-6)
- *   out         = O_sparse + O_lowrank
+ *   out         = O_sparse + O_lowrank   (or, with slra_problem.fusion = SLRA_FUSION_GATED, RoLA "4.4"'s
+ *                 token-wise gate: out_i = O_sparse,i + g_i O_lowrank,i rms(O_sparse,i) /
+ *                 sqrt(mean(O_lowrank,i^2) + 1e-6), g_i = sigmoid(q_i . Wg + bg) on the raw query; the
+ *                 pages print no formula, this is the library's reading of their description)
  *
  * Conventions for every entry point:
  *   - Device pointers unless stated otherwise.  The caller owns every buffer; nothing is retained
@@ -51,7 +54,7 @@
 extern "C" {
 #endif
 
-#define SLRA_ABI_VERSION 3
+#define SLRA_ABI_VERSION 4
 
 /* Exported symbols (the library is built with hidden visibility for everything else). */
 #if defined(__GNUC__)
@@ -92,6 +95,9 @@ enum { SLRA_DEBUG_UNSATISFIED_WAIT = 1 };
  * benchmark's map; SILU (u / (1 + e^-u)), IDENTITY and TANH are the alternatives RoLA's ablation
  * compares ("5.3", Table 6).  With IDENTITY or TANH the normaliser phi(q) . sum_j phi(k_j) + 1e-6 can
  * come close to zero; the library computes it as defined and does not guard it. */
+/* How the two branches are combined (slra_problem.fusion). */
+typedef enum slra_fusion { SLRA_FUSION_SUM = 0, SLRA_FUSION_GATED = 1 } slra_fusion;
+
 typedef enum slra_activation {
     SLRA_ACT_RELU = 0,
     SLRA_ACT_SILU = 1,
@@ -132,6 +138,11 @@ typedef enum slra_activation {
  *                           Both flags only change how the A argument is laid out:
  *                           bf16 [1 + proj_separate][proj_per_head ? heads : 1][D][rank], the query
  *                           projection(s) first; slra_projection_elems gives its element count.
+ *   fusion                  SLRA_FUSION_SUM (default): out = sparse + low-rank output;
+ *                           SLRA_FUSION_GATED: the gated fusion above (needs both branches).
+ *   gate_bias               bg of the gated fusion (a negative value starts near the sparse output).
+ *   gate_w                  Wg of the gated fusion: DEVICE pointer to fp32 [D], 16-B aligned, shared by
+ *                           all heads (also for slra_attn_fwd_host); NULL unless fusion is GATED.
  */
 typedef struct slra_problem {
     int64_t batch, heads, head_dim;
@@ -151,6 +162,9 @@ typedef struct slra_problem {
     int32_t lowrank_norope;
     int32_t proj_separate;
     int32_t proj_per_head;
+    int32_t fusion;
+    float gate_bias;
+    const void* gate_w;
 } slra_problem;
 
 /*

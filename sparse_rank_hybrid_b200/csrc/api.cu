@@ -52,6 +52,12 @@ slra_status derive(const slra_problem* p, Derived* d) {
     if (p->lowrank_norope != 0 && p->lowrank_norope != 1) return SLRA_ERR_INVALID_ARG;
     if (p->proj_separate != 0 && p->proj_separate != 1) return SLRA_ERR_INVALID_ARG;
     if (p->proj_per_head != 0 && p->proj_per_head != 1) return SLRA_ERR_INVALID_ARG;
+    if (p->fusion != SLRA_FUSION_SUM && p->fusion != SLRA_FUSION_GATED) return SLRA_ERR_INVALID_ARG;
+    if (p->fusion == SLRA_FUSION_GATED) {  // gate parameters given, both branches on
+        if (!p->gate_w || !std::isfinite(p->gate_bias)) return SLRA_ERR_INVALID_ARG;
+        if (p->branches != 0 && p->branches != SLRA_BRANCH_BOTH) return SLRA_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(p->gate_w) & 15u) != 0) return SLRA_ERR_ALIGNMENT;
+    }
     if (p->head_dim != 64 && p->head_dim != 128) return SLRA_ERR_UNSUPPORTED;
     if (p->block != 64 && p->block != 128) return SLRA_ERR_UNSUPPORTED;
     if (p->rank < 16 || p->rank > p->head_dim || p->rank % 16 != 0) return SLRA_ERR_UNSUPPORTED;
@@ -323,6 +329,9 @@ slra_status slra_problem_init(slra_problem* p, int64_t batch, int64_t heads, int
     p->lowrank_norope = 0;
     p->proj_separate = 0;
     p->proj_per_head = 0;
+    p->fusion = SLRA_FUSION_SUM;
+    p->gate_bias = 0.0f;
+    p->gate_w = nullptr;
     return SLRA_OK;
 }
 
@@ -407,6 +416,9 @@ slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, c
     a.at_img = w.at_img;
     a.sb_img = w.sb_img;
     a.lowrank = (branches & SLRA_BRANCH_LOWRANK) ? 1 : 0;
+    a.gated = p->fusion == SLRA_FUSION_GATED ? 1 : 0;
+    a.gate_b = p->gate_bias;
+    a.gate_w = static_cast<const float*>(p->gate_w);
     a.out = out;
     a.out_bf16 = p->out_dtype == SLRA_OUT_BF16 ? 1 : 0;
     a.status = w.status;

@@ -140,8 +140,8 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 
 }  // namespace
 
-// kDefault: relu features with the low-rank RoPE (the benchmark's configuration); the activation and
-// no-RoPE branches then fold away at compile time.
+// kDefault: relu features with the low-rank RoPE and the plain sum of the branches (the benchmark's
+// configuration); the activation, no-RoPE and gated-fusion branches then fold away at compile time.
 template <int D, int BLK, bool kDefault>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     using Lay = AttnLayout<D>;
     const int act = kDefault ? 0 : g.act;        // low-rank feature map
     const int norope = kDefault ? 0 : g.norope;  // 1: no rotation in the low-rank branch
+    const int gated = kDefault ? 0 : a.gated;    // 1: gated fusion of the branches instead of their sum
     constexpr int HW = BLK / 2;   // keys per thread: the two warps of a lane group split the key block
     constexpr int NC = HW / 32;   // 32-column TMEM loads per thread
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -485,6 +486,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_valid = (i_row < blk) && (n < g.L) && !aborted;
     float inv_l = (keep > 0 && l_run > 0.f) ? 1.f / l_run : 0.f;
     bool o_live = keep > 0;  // O holds the sparse branch (and, below, the low-rank readout)
+    // Gated fusion (RoLA 4.4, as read here): out = O_s + g O_lr rms(O_s) / sqrt(mean(O_lr^2) + 1e-6),
+    // g = sigmoid(q . Wg + bg) on the raw query.  The readout then goes to TMEM columns of its own
+    // (head_dim 128: S buffer 1, free once the last P.V has completed) or stays in registers (64).
+    float glogit = 0.f;   // q . Wg + bg of this row
+    bool lr_live = false;  // gated: the low-rank output of this row is available
+    const uint32_t tLr = tmem + 128;
     if constexpr (D == 128) {
         if (a.lowrank && !aborted) {
             // Low-rank readout on the tensor cores, accumulated straight into O (so out = O / l):
@@ -550,11 +557,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (c0 + i < R) den = fmaf(phi_act(__uint_as_float(v[i]), act), __ldg(zh + c0 + i), den);
                     }
                 }
+                float gpart = 0.f;
+                if (gated) {
+                    // Wg . q over this thread's half of the raw query row, read from the tile in X
+                    // (the tile's barrier has only one phase, long complete)
+                    volatile int no_abort = 0;
+                    mbar_wait(bar_eld, 0, tmo, &no_abort);
+                    const float* gw = a.gate_w + hf * 64;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 raw =
+                            *reinterpret_cast<const uint4*>(X + hf * 16384 + i_row * 128 + ((j ^ (i_row & 7)) << 4));
+                        const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float2 qf = __bfloat1622float2(q2[u]);
+                            gpart = fmaf(qf.x, __ldg(gw + 8 * j + 2 * u), gpart);
+                            gpart = fmaf(qf.y, __ldg(gw + 8 * j + 2 * u + 1), gpart);
+                        }
+                    }
+                    xch[256 + hf * 128 + i_row] = gpart;
+                }
                 xch[hf * 128 + i_row] = den;
                 group_sync();
                 den += xch[(hf ^ 1) * 128 + i_row];  // same total in both halves
+                if (gated) glogit = a.gate_b + (gpart + xch[256 + (hf ^ 1) * 128 + i_row]);
                 const float l_eff = keep > 0 ? l_run : 1.f;
-                const float scale = l_eff / (den + 1e-6f);
+                // summed into O (out = O / l): psi carries l; gated: the readout alone
+                const float scale = (gated ? 1.f : l_eff) / (den + 1e-6f);
                 const int n_tab = n < g.L ? n : g.L - 1;  // rows past the sequence: any valid table entry
                 const int axis_t = token_axis_pos(n_tab, 0, g.H, g.W), axis_h = token_axis_pos(n_tab, 1, g.H, g.W),
                           axis_w = token_axis_pos(n_tab, 2, g.H, g.W);
@@ -637,7 +667,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int kk = 0; kk < (3 * rc) / 16; ++kk) {
                                 const uint64_t ad = sdesc_sw128(smem_addr(X) + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
                                 const uint64_t bd = sdesc_sw128(smem_addr(Z) + (kk >> 2) * (D * 128) + (kk & 3) * 32, 16, 1024);
-                                umma_ss(tO, ad, bd, idesc_lr, (keep > 0 || ch > 0 || kk > 0) ? 1u : 0u);
+                                const bool acc = gated ? (ch > 0 || kk > 0) : (keep > 0 || ch > 0 || kk > 0);
+                                umma_ss(gated ? tLr : tO, ad, bd, idesc_lr, acc ? 1u : 0u);
                             }
                             umma_commit(bar_emm);
                             ++n_emm_issued;
@@ -653,8 +684,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         ++n_emm;
                         tc_fence_after();
-                        inv_l = 1.f / l_eff;
-                        o_live = true;
+                        if (gated) {
+                            lr_live = true;
+                        } else {
+                            inv_l = 1.f / l_eff;
+                            o_live = true;
+                        }
                     }
                 }
             }
@@ -688,6 +723,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const float2 qf = __bfloat1622float2(q2[u]);
+                            if (gated && c0 == 0) {  // Wg . q (both threads of the row compute all of it)
+                                glogit = fmaf(qf.x, __ldg(a.gate_w + d0 + 2 * u), glogit);
+                                glogit = fmaf(qf.y, __ldg(a.gate_w + d0 + 2 * u + 1), glogit);
+                            }
                             const float* a0 = As + (d0 + 2 * u) * g.R + c0;
                             const float* a1 = a0 + g.R;
 #pragma unroll
@@ -723,7 +762,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 inv_den = 1.f / (den + 1e-6f);
+                glogit += a.gate_b;
             }
+            lr_live = true;
         }
     }
     // ---- out = O / l (+ the CUDA-core readout for head_dim 64): each thread writes its half of its
@@ -732,22 +773,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      is skipped.
     const bool aborted2 = group_sync_or(*abort_flag != 0);  // every product that read the tile buffers has completed
     if (!aborted2) {
+        // this thread's 32-column group cc of O (and, gated with head_dim 128, of the readout)
+        auto load_group = [&](int cc, uint32_t (&o)[32], uint32_t (&lr)[32]) {
+            const int c = hf * (D / 64) + cc;
+            if (o_live) tmem_ld32(tO + lane_base + c * 32, o);
+            if (D == 128 && gated && lr_live) tmem_ld32(tLr + lane_base + c * 32, lr);
+            if (o_live || (D == 128 && gated && lr_live)) {
+                tmem_ld_wait(o);
+                reg_fence(lr);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (!o_live) o[i] = 0u;
+                if (D != 128 || !gated || !lr_live) lr[i] = 0u;
+            }
+        };
+        auto lr_value = [&](int cc, int i, const uint32_t (&lr)[32]) -> float {
+            if constexpr (D == 128) return __uint_as_float(lr[i]);
+            else return acc[cc * 32 + i] * inv_den;
+        };
+        float gfac = 0.f;  // gated: g * rms(O_s) / sqrt(mean(O_lr^2) + 1e-6) of this row
+        if (gated) {
+            float ss_s = 0.f, ss_l = 0.f;  // this thread's half of the two sums of squares
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc) {
+                uint32_t o[32], lr[32];
+                load_group(cc, o, lr);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float xs = __uint_as_float(o[i]) * inv_l, xl = lr_value(cc, i, lr);
+                    ss_s = fmaf(xs, xs, ss_s);
+                    ss_l = fmaf(xl, xl, ss_l);
+                }
+            }
+            xch[hf * 128 + i_row] = ss_s;
+            xch[256 + hf * 128 + i_row] = ss_l;
+            group_sync();
+            ss_s += xch[(hf ^ 1) * 128 + i_row];
+            ss_l += xch[256 + (hf ^ 1) * 128 + i_row];
+            const float gsig = 1.f / (1.f + expf(-glogit));
+            gfac = lr_live ? gsig * sqrtf(ss_s / D) / sqrtf(ss_l / D + 1e-6f) : 0.f;
+        }
 #pragma unroll
         for (int cc = 0; cc < D / 64; ++cc) {
             const int c = hf * (D / 64) + cc;  // 32-column group of O
-            uint32_t o[32];
-            if (o_live) {
-                tmem_ld32(tO + lane_base + c * 32, o);
-                tmem_ld_wait(o);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] = 0u;
-            }
+            uint32_t o[32], lr[32];
+            load_group(cc, o, lr);
             float r[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 float x = __uint_as_float(o[i]) * inv_l;
-                if constexpr (D != 128) x += acc[cc * 32 + i] * inv_den;
+                if (gated) {
+                    x = fmaf(gfac, lr_value(cc, i, lr), x);
+                } else {
+                    if constexpr (D != 128) x += acc[cc * 32 + i] * inv_den;
+                }
                 r[i] = x;
             }
             if (a.out_bf16) {  // boxes of 64 columns
@@ -824,8 +904,8 @@ cudaError_t launch_attn_v(const AttnMaps& m, const AttnArgs& a, const Geom& g, c
 }
 template <int D, int BLK>
 cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st) {
-    return (g.act == 0 && g.norope == 0) ? launch_attn_v<D, BLK, true>(m, a, g, st)
-                                         : launch_attn_v<D, BLK, false>(m, a, g, st);
+    return (g.act == 0 && g.norope == 0 && !a.gated) ? launch_attn_v<D, BLK, true>(m, a, g, st)
+                                                     : launch_attn_v<D, BLK, false>(m, a, g, st);
 }
 }  // namespace
 

@@ -106,6 +106,9 @@ struct AttnArgs {
     const uint8_t* at_img;  // A^T operand image (head_dim 128)
     const uint8_t* sb_img;  // S operand images (head_dim 128)
     int lowrank;  // add the low-rank readout
+    int gated;    // gated fusion of the branches instead of their sum (both branches on)
+    float gate_b;
+    const float* gate_w;  // [D]
     void* out;
     int out_bf16;
     int* status;

@@ -20,8 +20,9 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DE
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
 DEBUG_UNSATISFIED_WAIT = 1
-ABI_VERSION = 3
+ABI_VERSION = 4
 ACT_RELU, ACT_SILU, ACT_IDENTITY, ACT_TANH = 0, 1, 2, 3
+FUSION_SUM, FUSION_GATED = 0, 1
 
 # Every symbol include/slra.h declares.
 EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_validate", "slra_keep_count",
@@ -45,7 +46,8 @@ class _Problem(ctypes.Structure):
                 ("wait_timeout_ns", ctypes.c_uint64), ("debug_flags", ctypes.c_uint32),
                 ("stage_events", ctypes.c_void_p * 7), ("activation", ctypes.c_int32),
                 ("lowrank_norope", ctypes.c_int32), ("proj_separate", ctypes.c_int32),
-                ("proj_per_head", ctypes.c_int32)]
+                ("proj_per_head", ctypes.c_int32), ("fusion", ctypes.c_int32), ("gate_bias", ctypes.c_float),
+                ("gate_w", ctypes.c_void_p)]
 
 
 class _Layout(ctypes.Structure):
@@ -128,6 +130,9 @@ class Problem:
     lowrank_norope: int = 0            # 1: no RoPE in the low-rank branch
     proj_separate: int = 0             # 1: separate query / key projections Pq, Pk
     proj_per_head: int = 0             # 1: one projection (pair) per head
+    fusion: int = 0                    # FUSION_SUM or FUSION_GATED
+    gate_bias: float = 0.0             # bg of the gated fusion
+    gate_w: object = None              # Wg of the gated fusion: CUDA fp32 tensor [head_dim] (or None)
 
     @property
     def L(self) -> int:
@@ -154,6 +159,14 @@ class Problem:
         p.lowrank_norope = int(self.lowrank_norope)
         p.proj_separate = int(self.proj_separate)
         p.proj_per_head = int(self.proj_per_head)
+        p.fusion = int(self.fusion)
+        p.gate_bias = float(self.gate_bias)
+        if self.gate_w is not None:
+            t = self.gate_w
+            torch = _torch()
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (self.head_dim,):
+                raise ValueError(f"gate_w: expected a contiguous CUDA fp32 tensor of shape ({self.head_dim},)")
+            p.gate_w = int(t.data_ptr())
         return p
 
     @property

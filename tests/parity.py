@@ -62,6 +62,14 @@ def mask_ok(idx_gpu: np.ndarray, s_orc: np.ndarray, idx_orc: np.ndarray, tie_orc
     return True, diff
 
 
+def _gate_of(prob: slra.Problem):
+    """The oracle's gate argument for a gated problem: (Wg as fp64, bg rounded to fp32 as the library
+    receives it), else None."""
+    if prob.fusion != slra.FUSION_GATED:
+        return None
+    return prob.gate_w.detach().cpu().numpy().astype(np.float64), float(np.float32(prob.gate_bias))
+
+
 def compare(prob: slra.Problem, x: dict, gpu: dict, heads=None, qblocks=None, check_masks=True, label=""):
     """Run the oracle on (a sample of) the problem and compare.  Returns a dict of error stats."""
     grid = (prob.T, prob.H, prob.W)
@@ -73,7 +81,8 @@ def compare(prob: slra.Problem, x: dict, gpu: dict, heads=None, qblocks=None, ch
     out_o, per = oracle.forward(x, grid, prob.block, prob.keep_frac, prob.rank, offset=prob.pos_offset,
                                 heads=pairs, qblocks=qblocks, branches=prob.branches, idx_override=override,
                                 activation=prob.activation, lowrank_rope=not prob.lowrank_norope,
-                                proj_separate=bool(prob.proj_separate), proj_per_head=bool(prob.proj_per_head))
+                                proj_separate=bool(prob.proj_separate), proj_per_head=bool(prob.proj_per_head),
+                                gate=_gate_of(prob))
     stats = {"label": label, "mask_rows_differing": 0, "mask_rows": 0}
     for (b, h) in pairs:
         r = per[(b, h)]

@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_abi_version_and_status_strings():
-    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 3
+    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 4
     for s in range(0, 9):
         assert slra.status_string(s) and slra.status_string(s) != "unknown status"
     assert slra.status_string(99) == "unknown status"
@@ -63,6 +63,7 @@ def test_keep_count_and_layout(w, oracle_mod):
     ("activation", 4, slra.ERR_INVALID_ARG), ("activation", -1, slra.ERR_INVALID_ARG),
     ("lowrank_norope", 2, slra.ERR_INVALID_ARG),
     ("proj_separate", 2, slra.ERR_INVALID_ARG), ("proj_per_head", -1, slra.ERR_INVALID_ARG),
+    ("fusion", 2, slra.ERR_INVALID_ARG), ("fusion", slra.FUSION_GATED, slra.ERR_INVALID_ARG),  # no gate_w
 ])
 def test_validation_rejects(field, value, status):
     p = slra.Problem.from_workload(W.WAN_14B)
@@ -85,6 +86,20 @@ def test_projection_elems_and_layout(separate, per_head):
     extra = (w.heads - 1) * w.rank * 256 if per_head else 0
     assert base.total_bytes + extra <= lay.total_bytes <= base.total_bytes + extra + 256
     assert slra.projection_elems(slra.Problem.from_workload(w, proj_separate=3)) == -1
+
+
+@pytest.mark.parametrize("gate_w,branches,bias,status", [
+    (4096, 3, -2.0, slra.OK), (4096, 0, 0.5, slra.OK), (4100, 3, -2.0, slra.ERR_ALIGNMENT),
+    (4096, 1, -2.0, slra.ERR_INVALID_ARG), (4096, 2, -2.0, slra.ERR_INVALID_ARG),
+    (4096, 3, float("nan"), slra.ERR_INVALID_ARG), (4096, 3, float("inf"), slra.ERR_INVALID_ARG),
+])
+def test_gated_fusion_validation(gate_w, branches, bias, status):
+    """The gated fusion needs its weight vector (16-B aligned device pointer; validation never
+    dereferences it), a finite bias and both branches."""
+    import ctypes
+    p = slra.Problem.from_workload(W.TINY).c()
+    p.fusion, p.gate_w, p.branches, p.gate_bias = slra.FUSION_GATED, gate_w, branches, bias
+    assert slra.lib().slra_validate(ctypes.byref(p)) == status
 
 
 def test_validation_grid_limit():

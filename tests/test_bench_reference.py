@@ -20,7 +20,8 @@ def _run(extra, env_extra=None):
     return [l for l in r.stdout.splitlines() if l.startswith("{")]
 
 
-@pytest.mark.parametrize("extra", [[], ["--proj", "separate-per-head"], ["--activation", "silu", "--lowrank-norope"]])
+@pytest.mark.parametrize("extra", [[], ["--proj", "separate-per-head"], ["--activation", "silu", "--lowrank-norope"],
+                                   ["--fusion", "gated"]])
 def test_reference_arm_line(extra):
     lines = _run(extra)
     assert len(lines) == 1

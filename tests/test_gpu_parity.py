@@ -157,6 +157,31 @@ def test_projection_per_head_wan_1_3b():
           proj_separate=1, proj_per_head=1, transform=_projections(w, 1, 1))
 
 
+def _gate(w, bias, seed=77):
+    """Gated-fusion options: Wg ~ N(0, 1/D) in fp32 (seeded), the given bias."""
+    import torch
+    rng = np.random.default_rng(seed)
+    gw = (rng.standard_normal(w.head_dim) / np.sqrt(w.head_dim)).astype(np.float32)
+    return dict(fusion=slra.FUSION_GATED, gate_bias=bias, gate_w=torch.from_numpy(gw).cuda())
+
+
+@pytest.mark.parametrize("bias", [-2.0, 0.5, -30.0])
+def test_gated_fusion(bias):
+    """The gated fusion of the branches (RoLA 4.4 as read here) on both readout paths: a typical
+    negative bias, an open gate, and a closed one (the output is then the sparse branch's)."""
+    for w in (W.TINY, EDGE_128, EDGE_128_R64):
+        _case(w, f"{w.name}-gated{bias}", **_gate(w, bias))
+
+
+def test_gated_fusion_with_other_options():
+    """Gated fusion together with separate per-head projections and SiLU features, and at the
+    Wan2.1-1.3B shape on sampled heads and query blocks."""
+    _case(EDGE_PROJ, "edge-proj-gated-silu", proj_separate=1, proj_per_head=1, activation=slra.ACT_SILU,
+          transform=lambda x: _nonneg(_projections(EDGE_PROJ, 1, 1)(x)), **_gate(EDGE_PROJ, -1.0))
+    w = W.WAN_1_3B
+    _case(w, "wan1.3b-gated", heads=[(0, 2)], qblocks=_sample_blocks(w.nb, 13, n=2), **_gate(w, -2.0))
+
+
 def test_shift_invariance_on_gpu():
     """Shifting all positions leaves the masks unchanged exactly (fp64 selection) and the outputs
     unchanged up to the fp16 rounding of the rotated operands, which differs between the two runs:
