@@ -207,13 +207,17 @@ def gated_fusion(o_s, o_lr, q, w, b: float, rows) -> np.ndarray:
 
 def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, theta=1e4,
                  offset=(0, 0, 0), split=None, qblocks=None, branches=3, idx_override=None,
-                 activation=ACT_RELU, lowrank_rope=True, A_k=None, gate=None):
+                 activation=ACT_RELU, lowrank_rope=True, A_k=None, gate=None, rope_inside=False):
     """Forward pass of one (batch, head): q, k, v fp64 [L, D]; A fp64 [D, R].
 
     `activation` picks the feature map's nonlinearity; `lowrank_rope=False` drops the truncated RoPE
     from the low-rank branch (psi = phi), the no-RoPE setting of RoLA's ablation (5.3).  `A_k`, when
     given, is a separate key projection Pk (RoLA E.2 lists Pq and Pk as the branch's parameters):
-    query features use A, key features use A_k.  `gate=(w, b)` replaces the plain sum of the two
+    query features use A, key features use A_k.  `rope_inside=True` applies the truncated RoPE to the
+    projected features BEFORE the activation, psi = act(R_r(p) x A), the ordering RoLA's ablation
+    compares against (5.1 Table 2, 5.3, B.3); numerator and normaliser then both use psi (there is no
+    unrotated feature left to normalise with), so the summary stays linear but loses the relative
+    property.  `gate=(w, b)` replaces the plain sum of the two
     branches by the gated fusion of RoLA 4.4 (see gated_fusion; needs both branches).
 
     Returns a dict with out (rows of the computed query blocks; NaN elsewhere), the sparse and
@@ -243,13 +247,22 @@ def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, t
         o_s = sparse_attn(qh, kh, v, block, use_idx, qb)
         res["out_sparse"] = o_s
         out[rows] += o_s[rows]
-    phiq = features(q, A, activation)
-    phik = features(k, A if A_k is None else A_k, activation)
-    if lowrank_rope:
-        psiq = rope_rows(phiq, grid, R // 2, theta, offset, split, schedule_dim=D)
-        psik = rope_rows(phik, grid, R // 2, theta, offset, split, schedule_dim=D)
+    if rope_inside:
+        assert lowrank_rope, "RoPE inside the activation needs the low-rank RoPE"
+        Ak = A if A_k is None else A_k
+        yq = rope_rows(features(q, A, ACT_IDENTITY), grid, R // 2, theta, offset, split, schedule_dim=D)
+        yk = rope_rows(features(k, Ak, ACT_IDENTITY), grid, R // 2, theta, offset, split, schedule_dim=D)
+        eye = np.eye(R)  # act(y I) = act(y) exactly in fp64
+        psiq, psik = features(yq, eye, activation), features(yk, eye, activation)
+        phiq, phik = psiq, psik
     else:
-        psiq, psik = phiq.copy(), phik.copy()
+        phiq = features(q, A, activation)
+        phik = features(k, A if A_k is None else A_k, activation)
+        if lowrank_rope:
+            psiq = rope_rows(phiq, grid, R // 2, theta, offset, split, schedule_dim=D)
+            psik = rope_rows(phik, grid, R // 2, theta, offset, split, schedule_dim=D)
+        else:
+            psiq, psik = phiq.copy(), phik.copy()
     S, z = summary(psik, phik, v)
     res.update(S=S, z=z, phiq=phiq, phik=phik, psiq=psiq, psik=psik)
     if branches & 2:
@@ -266,7 +279,8 @@ def head_forward(q, k, v, A, grid, block: int, keep_frac: float, rank: int, *, t
 
 def forward(inp: dict, grid, block: int, keep_frac: float, rank: int, *, theta=1e4, offset=(0, 0, 0),
             split=None, heads=None, qblocks=None, branches=3, idx_override=None, keep_intermediates=False,
-            activation=ACT_RELU, lowrank_rope=True, proj_separate=False, proj_per_head=False, gate=None):
+            activation=ACT_RELU, lowrank_rope=True, proj_separate=False, proj_per_head=False, gate=None,
+            rope_inside=False):
     """Full forward over all (batch, head) pairs of bf16 inputs q, k, v [B, L, Hh, D] and A [D, R].
 
     With `proj_separate` and/or `proj_per_head`, A holds [1 + separate][per_head ? Hh : 1][D][R]
@@ -291,7 +305,7 @@ def forward(inp: dict, grid, block: int, keep_frac: float, rank: int, *, theta=1
                          Af[0, h if proj_per_head else 0], grid, block, keep_frac, rank, theta=theta,
                          offset=offset, split=split, qblocks=qb, branches=branches, idx_override=ov,
                          activation=activation, lowrank_rope=lowrank_rope,
-                         A_k=Af[-1, h if proj_per_head else 0], gate=gate)
+                         A_k=Af[-1, h if proj_per_head else 0], gate=gate, rope_inside=rope_inside)
         out[b, :, h, :] = r["out"]
         if not keep_intermediates:
             for key in ("qh", "kh", "phiq", "phik", "psiq", "psik", "out_sparse", "out_lowrank", "out"):

@@ -518,3 +518,50 @@ def test_gate_is_homogeneous_in_v(oracle_mod):
     r2, _ = _gated(oracle_mod, w_gate, -1.0, v_scale=2.0)
     ref = 2.0 * r1["out"]
     assert np.abs(r2["out"] - ref).max() <= 5e-5 * np.abs(ref).max()
+
+
+# ----------------------------------------------------------------------- RoPE inside the activation
+def _inside(oracle_mod, act=0, offset=(0, 0, 0), **kw):
+    w = W.TINY
+    x = I.make_inputs(w)
+    dec = oracle_mod.decode_bf16
+    q, k, v = dec(x["q"][0, :, 1]), dec(x["k"][0, :, 1]), dec(x["v"][0, :, 1])
+    A = dec(x["A"])
+    r = oracle_mod.head_forward(q, k, v, A, (w.T, w.H, w.W), w.block, w.keep_frac, w.rank, branches=2,
+                                activation=act, offset=offset, **kw)
+    return r, (q, k, v, A, w)
+
+
+def test_rope_inside_written_out(oracle_mod):
+    """RoPE inside the activation (RoLA 5.3 / B.3 ordering): psi = relu(R_r(p) (x A)) with the rotation
+    done here by complex multiplication, and out = psi_q (psi_k^T v) / (psi_q . sum_j psi_k + 1e-6),
+    both sides using the rotated-then-activated features."""
+    r, (q, k, v, A, w) = _inside(oracle_mod, rope_inside=True)
+    axis, omega = oracle_mod.rope_pairs(w.head_dim)
+    pos = brute.grid_positions((w.T, w.H, w.W))
+    pq = np.maximum(brute.rope_complex(q @ A, pos, axis, omega, w.rank // 2), 0)
+    pk = np.maximum(brute.rope_complex(k @ A, pos, axis, omega, w.rank // 2), 0)
+    ref = (pq @ (pk.T @ v)) / (pq @ pk.sum(0) + 1e-6)[:, None]
+    assert np.allclose(r["out_lowrank"], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_rope_inside_identity_map_shares_the_numerator(oracle_mod):
+    """With the identity map the rotation and the activation commute, so the inside and outside
+    orderings give the same psi; only the normaliser differs (inside: rotated features)."""
+    ri, _ = _inside(oracle_mod, act=2, rope_inside=True)
+    ro, _ = _inside(oracle_mod, act=2)
+    assert np.allclose(ri["psiq"], ro["psiq"], rtol=0, atol=1e-13)
+    assert np.array_equal(ri["phiq"], ri["psiq"]) and not np.allclose(ri["phiq"], ro["phiq"], rtol=1e-3)
+
+
+def test_rope_inside_is_not_shift_invariant(oracle_mod):
+    """RoLA Table 2's contrast on synthetic features: shifting every position by a constant leaves the
+    outside-activation branch unchanged (relative property) but changes the inside-activation one
+    (absolute position leaks through the nonlinearity); without RoPE nothing changes."""
+    def resid(**kw):
+        a, _ = _inside(oracle_mod, **kw)
+        b, _ = _inside(oracle_mod, offset=(2, 3, 5), **kw)
+        return np.linalg.norm(a["out_lowrank"] - b["out_lowrank"]) / np.linalg.norm(a["out_lowrank"])
+    assert resid() < 1e-12
+    assert resid(lowrank_rope=False) == 0.0
+    assert resid(rope_inside=True) > 1e-2
