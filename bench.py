@@ -129,7 +129,7 @@ def variant_of(args, w) -> dict:
     gate = (gate_weights(w).astype(np.float64), GATE_BIAS) if args.fusion == "gated" else None
     return {"activation": ACTS[args.activation], "lowrank_rope": not args.lowrank_norope,
             "branches": BRANCHES[args.branches], "proj_separate": bool(sep), "proj_per_head": bool(ph),
-            "gate": gate}
+            "gate": gate, "rope_inside": bool(args.rope_inside)}
 
 
 def make_run_inputs(args, w) -> dict:
@@ -223,7 +223,7 @@ def run_reference(args, w, rank, world):
                        "block": w.block, "keep_frac": w.keep_frac, "activation": args.activation,
                        "lowrank_rope": not args.lowrank_norope, "branches": args.branches,
                        "linear_baseline": bool(args.linear_baseline), "projection": args.proj,
-                       "fusion": args.fusion},
+                       "fusion": args.fusion, "rope_inside": bool(args.rope_inside)},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -260,7 +260,7 @@ def run_ours(args, w, rank, world, local_rank):
     prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev), branches=br,
                                       activation=var["activation"], lowrank_norope=int(not var["lowrank_rope"]),
                                       proj_separate=int(var["proj_separate"]), proj_per_head=int(var["proj_per_head"]),
-                                      **gate_kw)
+                                      lowrank_rope_inside=int(args.rope_inside), **gate_kw)
     A = torch.from_numpy(x["A"].view(np.int16)).view(torch.bfloat16).to(dev).reshape(prob.projection_shape)
     ws = slra.alloc_workspace(prob, dev)
     out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
@@ -356,7 +356,7 @@ def run_ours(args, w, rank, world, local_rank):
                    "parallelism": f"replica x{world} (independent problems, no collective)",
                    "activation": args.activation, "lowrank_rope": not args.lowrank_norope,
                    "branches": args.branches, "linear_baseline": bool(args.linear_baseline),
-                   "projection": args.proj, "fusion": args.fusion},
+                   "projection": args.proj, "fusion": args.fusion, "rope_inside": bool(args.rope_inside)},
         "flops_per_step": {"sparse_kept": f_sparse, "lowrank": f_lr, "scores": f_sc},
         "roofline": {"kernel": "attn_sm100_kernel", "bound": "tensor", "achieved": achieved, "peak": tf_sust,
                      "unit": "TFLOP/s", "frac": achieved / tf_sust, "traffic": traffic,
@@ -406,7 +406,11 @@ def main():
                     help="query/key projection layout: one shared A, separate Pq/Pk, per head, or both")
     ap.add_argument("--fusion", default="sum", choices=["sum", "gated"],
                     help="combine the branches by their sum or by the token-wise gate (synthetic Wg, bg = -2)")
+    ap.add_argument("--rope-inside", action="store_true",
+                    help="low-rank RoPE before the activation (the ordering RoLA's ablation compares against)")
     args = ap.parse_args()
+    if args.rope_inside and (args.lowrank_norope or args.linear_baseline):
+        ap.error("--rope-inside needs the low-rank RoPE")
     if args.fusion == "gated" and args.branches != "both":
         ap.error("--fusion gated needs both branches")
     if args.linear_baseline and args.proj != "shared":

@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define SLRA_ABI_VERSION 4
+#define SLRA_ABI_VERSION 5
 
 /* Exported symbols (the library is built with hidden visibility for everything else). */
 #if defined(__GNUC__)
@@ -143,6 +143,11 @@ typedef enum slra_activation {
  *   gate_bias               bg of the gated fusion (a negative value starts near the sparse output).
  *   gate_w                  Wg of the gated fusion: DEVICE pointer to fp32 [D], 16-B aligned, shared by
  *                           all heads (also for slra_attn_fwd_host); NULL unless fusion is GATED.
+ *   lowrank_rope_inside     0 (default); 1: the truncated RoPE is applied to the projected features
+ *                           BEFORE the activation, psi = act(R_r(p) x P), and the normaliser uses psi
+ *                           too: the ordering RoLA's ablation compares against ("5.1" Table 2, "5.3",
+ *                           "B.3"); the summary stays linear but loses the relative property.  Not
+ *                           with lowrank_norope.
  */
 typedef struct slra_problem {
     int64_t batch, heads, head_dim;
@@ -165,6 +170,7 @@ typedef struct slra_problem {
     int32_t fusion;
     float gate_bias;
     const void* gate_w;
+    int32_t lowrank_rope_inside;
 } slra_problem;
 
 /*

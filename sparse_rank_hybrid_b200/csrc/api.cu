@@ -50,6 +50,8 @@ slra_status derive(const slra_problem* p, Derived* d) {
     if (p->branches < 0 || p->branches > 3) return SLRA_ERR_INVALID_ARG;
     if (p->activation < SLRA_ACT_RELU || p->activation > SLRA_ACT_TANH) return SLRA_ERR_INVALID_ARG;
     if (p->lowrank_norope != 0 && p->lowrank_norope != 1) return SLRA_ERR_INVALID_ARG;
+    if (p->lowrank_rope_inside != 0 && p->lowrank_rope_inside != 1) return SLRA_ERR_INVALID_ARG;
+    if (p->lowrank_rope_inside && p->lowrank_norope) return SLRA_ERR_INVALID_ARG;
     if (p->proj_separate != 0 && p->proj_separate != 1) return SLRA_ERR_INVALID_ARG;
     if (p->proj_per_head != 0 && p->proj_per_head != 1) return SLRA_ERR_INVALID_ARG;
     if (p->fusion != SLRA_FUSION_SUM && p->fusion != SLRA_FUSION_GATED) return SLRA_ERR_INVALID_ARG;
@@ -90,6 +92,7 @@ slra_status derive(const slra_problem* p, Derived* d) {
     g.act = static_cast<int>(p->activation);
     g.norope = static_cast<int>(p->lowrank_norope);
     g.a_stride = p->proj_per_head ? g.D * g.R : 0;
+    g.inside = static_cast<int>(p->lowrank_rope_inside);
     // projection argument: [1 + separate][per_head ? Hh : 1][D][R], query projection(s) first
     const size_t one_side = static_cast<size_t>(p->proj_per_head ? p->heads : 1) * p->head_dim * p->rank;
     d->a_elems = one_side * (p->proj_separate ? 2 : 1);
@@ -332,6 +335,7 @@ slra_status slra_problem_init(slra_problem* p, int64_t batch, int64_t heads, int
     p->fusion = SLRA_FUSION_SUM;
     p->gate_bias = 0.0f;
     p->gate_w = nullptr;
+    p->lowrank_rope_inside = 0;
     return SLRA_OK;
 }
 

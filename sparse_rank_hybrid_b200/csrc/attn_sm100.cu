@@ -97,6 +97,12 @@ __device__ __forceinline__ bool group_sync_or(bool pred) {
     return r != 0;
 }
 
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[16]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]));
+}
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
     asm volatile(""
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
@@ -151,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int act = kDefault ? 0 : g.act;        // low-rank feature map
     const int norope = kDefault ? 0 : g.norope;  // 1: no rotation in the low-rank branch
     const int gated = kDefault ? 0 : a.gated;    // 1: gated fusion of the branches instead of their sum
+    const int inside = kDefault ? 0 : g.inside;  // 1: the low-rank RoPE before the activation
     constexpr int HW = BLK / 2;   // keys per thread: the two warps of a lane group split the key block
     constexpr int NC = HW / 32;   // 32-column TMEM loads per thread
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -543,18 +550,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bulk_load(Z, sb_head, sb_bytes(0), bar_ez);
                     ++n_ez_issued;
                 }
-                // phi . z over all R features (unrotated features in the denominator)
+                const int n_tab = n < g.L ? n : g.L - 1;  // rows past the sequence: any valid table entry
+                const int axis_t = token_axis_pos(n_tab, 0, g.H, g.W), axis_h = token_axis_pos(n_tab, 1, g.H, g.W),
+                          axis_w = token_axis_pos(n_tab, 2, g.H, g.W);
+                // This thread's 16 rotation pairs of a chunk: features [16hf, 16hf + 16) and
+                // [32 + 16hf, 48 + 16hf) (so both warps of a lane group have work when rc <= 32).
+                auto feat = [&](int t) { return t < 8 ? 16 * hf + 2 * t : 32 + 16 * hf + 2 * (t - 8); };
+                // phi . z over all R features: the unrotated features (RoPE outside the activation), or
+                // with the RoPE inside, the rotated-then-activated ones over this thread's pairs
                 const float* zh = a.z + static_cast<size_t>(bh) * R;
                 float den = 0.f;
+                if (!inside) {
 #pragma unroll
-                for (int c0 = hf * 32; c0 < 128; c0 += 64) {
-                    if (c0 < R) {
-                        uint32_t v[32];
-                        tmem_ld32(tPhi + lane_base + c0, v);
-                        tmem_ld_wait(v);
+                    for (int c0 = hf * 32; c0 < 128; c0 += 64) {
+                        if (c0 < R) {
+                            uint32_t v[32];
+                            tmem_ld32(tPhi + lane_base + c0, v);
+                            tmem_ld_wait(v);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (c0 + i < R) den = fmaf(phi_act(__uint_as_float(v[i]), act), __ldg(zh + c0 + i), den);
+                            for (int i = 0; i < 32; ++i)
+                                if (c0 + i < R) den = fmaf(phi_act(__uint_as_float(v[i]), act), __ldg(zh + c0 + i), den);
+                        }
+                    }
+                } else {
+                    for (int ch = 0; ch < nch; ++ch) {
+                        const int rc = min(64, R - 64 * ch);
+                        uint32_t va[16], vb[16];
+                        tmem_ld16(tPhi + lane_base + 64 * ch + 16 * hf, va);
+                        tmem_ld16(tPhi + lane_base + 64 * ch + 32 + 16 * hf, vb);
+                        tmem_ld_wait(va);
+                        reg_fence(vb);
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) {
+                            const int f = feat(t);
+                            if (f < rc) {
+                                const int2 pi = a.pair_info[32 * ch + f / 2];
+                                const int ap = pi.x == 0 ? axis_t : (pi.x == 1 ? axis_h : axis_w);
+                                const double2 cs = __ldg(a.tab + pi.y + ap);
+                                const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+                                const float u0 = __uint_as_float(t < 8 ? va[2 * t] : vb[2 * (t - 8)]);
+                                const float u1 = __uint_as_float(t < 8 ? va[2 * t + 1] : vb[2 * (t - 8) + 1]);
+                                den = fmaf(phi_act(u0 * cf - u1 * sf, act), __ldg(zh + 64 * ch + f), den);
+                                den = fmaf(phi_act(u0 * sf + u1 * cf, act), __ldg(zh + 64 * ch + f + 1), den);
+                            }
+                        }
                     }
                 }
                 float gpart = 0.f;
@@ -585,9 +624,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float l_eff = keep > 0 ? l_run : 1.f;
                 // summed into O (out = O / l): psi carries l; gated: the readout alone
                 const float scale = (gated ? 1.f : l_eff) / (den + 1e-6f);
-                const int n_tab = n < g.L ? n : g.L - 1;  // rows past the sequence: any valid table entry
-                const int axis_t = token_axis_pos(n_tab, 0, g.H, g.W), axis_h = token_axis_pos(n_tab, 1, g.H, g.W),
-                          axis_w = token_axis_pos(n_tab, 2, g.H, g.W);
                 for (int ch = 0; ch < nch && ok; ++ch) {
                     const int rc = min(64, R - 64 * ch);
                     if (ch > 0) {  // the previous chunk's product must have finished with X and Z
@@ -605,12 +641,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ++n_ez_issued;
                         }
                     }
-                    // This thread's 16 rotation pairs of the chunk: features [16hf, 16hf + 16) and
-                    // [32 + 16hf, 48 + 16hf) (so both warps of a lane group have work when rc <= 32).
-                    // Their (cos, sin) loads are all issued before any is used; the pair table holds all
-                    // D/2 rotary pairs, so pairs past the rank are still valid entries (their results are
-                    // not stored).  The pair -> (axis, table offset) map comes from the launch parameters.
-                    auto feat = [&](int t) { return t < 8 ? 16 * hf + 2 * t : 32 + 16 * hf + 2 * (t - 8); };
+                    // This thread's 16 rotation pairs of the chunk (feat above).  Their (cos, sin) loads
+                    // are all issued before any is used; the pair table holds all D/2 rotary pairs, so
+                    // pairs past the rank are still valid entries (their results are not stored).  The
+                    // pair -> (axis, table offset) map comes from the launch parameters.
                     float2 rot[16];
                     // the second eight lie past the rank when rc <= 32; no rotation without the low-rank RoPE
                     const int nrot = norope ? 0 : (rc > 32 ? 16 : 8);
@@ -632,9 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld16(tPhi + lane_base + 64 * ch + 16 * hf, va);
                     tmem_ld16(tPhi + lane_base + 64 * ch + 32 + 16 * hf, vb);
                     tmem_ld_wait(va);
-                    asm volatile("" : "+r"(vb[0]), "+r"(vb[1]), "+r"(vb[2]), "+r"(vb[3]), "+r"(vb[4]), "+r"(vb[5]),
-                                 "+r"(vb[6]), "+r"(vb[7]), "+r"(vb[8]), "+r"(vb[9]), "+r"(vb[10]), "+r"(vb[11]),
-                                 "+r"(vb[12]), "+r"(vb[13]), "+r"(vb[14]), "+r"(vb[15]));
+                    reg_fence(vb);
 #pragma unroll
                     for (int t = 0; t < 16; ++t) {
                         const int f = feat(t);
@@ -642,10 +674,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (f < rc) {
                             const uint32_t u0 = t < 8 ? va[2 * t] : vb[2 * (t - 8)];
                             const uint32_t u1 = t < 8 ? va[2 * t + 1] : vb[2 * (t - 8) + 1];
-                            const float x0 = phi_act(__uint_as_float(u0), act);
-                            const float x1 = phi_act(__uint_as_float(u1), act);
+                            // outside: activation, then rotation; inside: rotation, then activation
+                            const float x0 = inside ? __uint_as_float(u0) : phi_act(__uint_as_float(u0), act);
+                            const float x1 = inside ? __uint_as_float(u1) : phi_act(__uint_as_float(u1), act);
                             const float cf = norope ? 1.f : rot[t].x, sf = norope ? 0.f : rot[t].y;
-                            const float y0 = (x0 * cf - x1 * sf) * scale, y1 = (x0 * sf + x1 * cf) * scale;
+                            float r0 = x0 * cf - x1 * sf, r1 = x0 * sf + x1 * cf;
+                            if (inside) {
+                                r0 = phi_act(r0, act);
+                                r1 = phi_act(r1, act);
+                            }
+                            const float y0 = r0 * scale, y1 = r1 * scale;
                             const __nv_bfloat162 hi = __floats2bfloat162_rn(y0, y1);
                             const float2 hf2 = __bfloat1622float2(hi);
                             const __nv_bfloat162 lo = __floats2bfloat162_rn(y0 - hf2.x, y1 - hf2.y);
@@ -733,10 +771,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int c = 0; c < 16; ++c) phi[c] = fmaf(qf.y, a1[c], fmaf(qf.x, a0[c], phi[c]));
                         }
                     }
+                    // outside: activation (the normaliser's features), then rotation; inside: rotation,
+                    // then activation, and the normaliser uses the result
+                    if (!inside) {
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        phi[c] = phi_act(phi[c], act);
-                        den = fmaf(phi[c], __ldg(zh + c0 + c), den);
+                        for (int c = 0; c < 16; ++c) {
+                            phi[c] = phi_act(phi[c], act);
+                            den = fmaf(phi[c], __ldg(zh + c0 + c), den);
+                        }
                     }
 #pragma unroll
                     for (int pp = 0; pp < 8; ++pp) {
@@ -747,6 +789,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float x0 = phi[2 * pp], x1 = phi[2 * pp + 1];
                         phi[2 * pp] = x0 * cf - x1 * sf;
                         phi[2 * pp + 1] = x0 * sf + x1 * cf;
+                    }
+                    if (inside) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            phi[c] = phi_act(phi[c], act);
+                            den = fmaf(phi[c], __ldg(zh + c0 + c), den);
+                        }
                     }
 #pragma unroll 4
                     for (int c = 0; c < 16; ++c) {
@@ -904,8 +953,8 @@ cudaError_t launch_attn_v(const AttnMaps& m, const AttnArgs& a, const Geom& g, c
 }
 template <int D, int BLK>
 cudaError_t launch_attn_t(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st) {
-    return (g.act == 0 && g.norope == 0 && !a.gated) ? launch_attn_v<D, BLK, true>(m, a, g, st)
-                                                     : launch_attn_v<D, BLK, false>(m, a, g, st);
+    return (g.act == 0 && g.norope == 0 && g.inside == 0 && !a.gated) ? launch_attn_v<D, BLK, true>(m, a, g, st)
+                                                                      : launch_attn_v<D, BLK, false>(m, a, g, st);
 }
 }  // namespace
 

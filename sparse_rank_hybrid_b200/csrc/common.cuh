@@ -21,6 +21,7 @@ struct Geom {
     int act;     // SLRA_ACT_* of the low-rank feature map
     int norope;  // 1: no rotation in the low-rank branch (psi = phi)
     int a_stride;  // elements between consecutive heads' projections (D * R when per head, else 0)
+    int inside;    // 1: the low-rank RoPE before the activation (psi = act(R x A), normaliser on psi)
     __host__ __device__ int BH() const { return B * Hh; }
 };
 

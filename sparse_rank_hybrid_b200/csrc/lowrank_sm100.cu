@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(256, 1)
     const LrLayout lay = lr_layout(R);
     const int act = kDefault ? 0 : g.act;
     const int norope = kDefault ? 0 : g.norope;
+    const int inside = kDefault ? 0 : g.inside;  // RoPE before the activation; z then sums psi
     constexpr int RP = R <= 64 ? 64 : 128;
     constexpr int RH = R / 2;           // features per thread: two threads share a token row
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -277,12 +278,19 @@ __global__ void __launch_bounds__(256, 1)
                 const int pp = p0 + u;
                 if (pp >= RH / 2) break;
                 const int p = half * (RH / 2) + pp;  // global rotary pair
-                float x0 = real ? phi_act(__uint_as_float(raw[2 * pp]), act) : 0.f;
-                float x1 = real ? phi_act(__uint_as_float(raw[2 * pp + 1]), act) : 0.f;
+                const float u0 = real ? __uint_as_float(raw[2 * pp]) : 0.f;
+                const float u1 = real ? __uint_as_float(raw[2 * pp + 1]) : 0.f;
+                float x0 = inside ? u0 : phi_act(u0, act), x1 = inside ? u1 : phi_act(u1, act);
+                const float cf = static_cast<float>(cs[u].x), sf = static_cast<float>(cs[u].y);
+                float y0 = x0 * cf - x1 * sf, y1 = x0 * sf + x1 * cf;
+                if (inside) {  // rotate, then the activation; the normaliser sums these features
+                    y0 = phi_act(y0, act);
+                    y1 = phi_act(y1, act);
+                    x0 = y0;
+                    x1 = y1;
+                }
                 zacc[2 * pp] += x0;
                 zacc[2 * pp + 1] += x1;
-                const float cf = static_cast<float>(cs[u].x), sf = static_cast<float>(cs[u].y);
-                const float y0 = x0 * cf - x1 * sf, y1 = x0 * sf + x1 * cf;
                 const __nv_bfloat162 hi = __floats2bfloat162_rn(y0, y1);
                 const float2 hf = __bfloat1622float2(hi);
                 const __nv_bfloat162 lo = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
@@ -405,8 +413,8 @@ static cudaError_t lr_tc_launch_v(const CUtensorMap& tk, const CUtensorMap& tv, 
 template <int R>
 static cudaError_t lr_tc_launch(const CUtensorMap& tk, const CUtensorMap& tv, const LrArgs& a, const Geom& g,
                                 cudaStream_t st) {
-    return (g.act == 0 && g.norope == 0) ? lr_tc_launch_v<R, true>(tk, tv, a, g, st)
-                                         : lr_tc_launch_v<R, false>(tk, tv, a, g, st);
+    return (g.act == 0 && g.norope == 0 && g.inside == 0) ? lr_tc_launch_v<R, true>(tk, tv, a, g, st)
+                                                         : lr_tc_launch_v<R, false>(tk, tv, a, g, st);
 }
 
 cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,

@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(256) lowrank_partial_kernel(const __nv_bfloat1
             float a = 0.f;
 #pragma unroll 16
             for (int d = 0; d < D; ++d) a = fmaf(kr[d], As[d * R + c], a);
-            ph[tt * (R + 1) + c] = phi_act(a, g.act);
+            ph[tt * (R + 1) + c] = g.inside ? a : phi_act(a, g.act);  // inside: activation after the rotation
         }
         __syncthreads();
         for (int o = tid; o < kLrTile * (R / 2); o += 256) {
@@ -451,8 +451,13 @@ __global__ void __launch_bounds__(256) lowrank_partial_kernel(const __nv_bfloat1
                 c = static_cast<float>(cs.x);
                 s = static_cast<float>(cs.y);
             }
-            ps[tt * R + 2 * p] = x0 * c - x1 * s;
-            ps[tt * R + 2 * p + 1] = x0 * s + x1 * c;
+            float y0 = x0 * c - x1 * s, y1 = x0 * s + x1 * c;
+            if (g.inside) {
+                y0 = phi_act(y0, g.act);
+                y1 = phi_act(y1, g.act);
+            }
+            ps[tt * R + 2 * p] = y0;
+            ps[tt * R + 2 * p + 1] = y1;
         }
         __syncthreads();
 #pragma unroll 4
@@ -462,8 +467,8 @@ __global__ void __launch_bounds__(256) lowrank_partial_kernel(const __nv_bfloat1
 #pragma unroll
             for (int i = 0; i < NA; ++i) acc[i] = fmaf(pr[G * i], vv, acc[i]);
         }
-        if (tid < R)
-            for (int tt = 0; tt < kLrTile; ++tt) zacc += ph[tt * (R + 1) + tid];
+        if (tid < R)  // z sums the unrotated features, or psi when the RoPE is inside the activation
+            for (int tt = 0; tt < kLrTile; ++tt) zacc += g.inside ? ps[tt * R + tid] : ph[tt * (R + 1) + tid];
     }
     float* sp = s_part + (static_cast<size_t>(bh) * nsplit + split) * R * D;
 #pragma unroll

@@ -20,7 +20,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DE
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
 DEBUG_UNSATISFIED_WAIT = 1
-ABI_VERSION = 4
+ABI_VERSION = 5
 ACT_RELU, ACT_SILU, ACT_IDENTITY, ACT_TANH = 0, 1, 2, 3
 FUSION_SUM, FUSION_GATED = 0, 1
 
@@ -47,7 +47,7 @@ class _Problem(ctypes.Structure):
                 ("stage_events", ctypes.c_void_p * 7), ("activation", ctypes.c_int32),
                 ("lowrank_norope", ctypes.c_int32), ("proj_separate", ctypes.c_int32),
                 ("proj_per_head", ctypes.c_int32), ("fusion", ctypes.c_int32), ("gate_bias", ctypes.c_float),
-                ("gate_w", ctypes.c_void_p)]
+                ("gate_w", ctypes.c_void_p), ("lowrank_rope_inside", ctypes.c_int32)]
 
 
 class _Layout(ctypes.Structure):
@@ -133,6 +133,7 @@ class Problem:
     fusion: int = 0                    # FUSION_SUM or FUSION_GATED
     gate_bias: float = 0.0             # bg of the gated fusion
     gate_w: object = None              # Wg of the gated fusion: CUDA fp32 tensor [head_dim] (or None)
+    lowrank_rope_inside: int = 0       # 1: the low-rank RoPE before the activation
 
     @property
     def L(self) -> int:
@@ -161,6 +162,7 @@ class Problem:
         p.proj_per_head = int(self.proj_per_head)
         p.fusion = int(self.fusion)
         p.gate_bias = float(self.gate_bias)
+        p.lowrank_rope_inside = int(self.lowrank_rope_inside)
         if self.gate_w is not None:
             t = self.gate_w
             torch = _torch()

@@ -82,7 +82,7 @@ def compare(prob: slra.Problem, x: dict, gpu: dict, heads=None, qblocks=None, ch
                                 heads=pairs, qblocks=qblocks, branches=prob.branches, idx_override=override,
                                 activation=prob.activation, lowrank_rope=not prob.lowrank_norope,
                                 proj_separate=bool(prob.proj_separate), proj_per_head=bool(prob.proj_per_head),
-                                gate=_gate_of(prob))
+                                gate=_gate_of(prob), rope_inside=bool(prob.lowrank_rope_inside))
     stats = {"label": label, "mask_rows_differing": 0, "mask_rows": 0}
     for (b, h) in pairs:
         r = per[(b, h)]

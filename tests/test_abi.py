@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_abi_version_and_status_strings():
-    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 4
+    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 5
     for s in range(0, 9):
         assert slra.status_string(s) and slra.status_string(s) != "unknown status"
     assert slra.status_string(99) == "unknown status"
@@ -64,6 +64,7 @@ def test_keep_count_and_layout(w, oracle_mod):
     ("lowrank_norope", 2, slra.ERR_INVALID_ARG),
     ("proj_separate", 2, slra.ERR_INVALID_ARG), ("proj_per_head", -1, slra.ERR_INVALID_ARG),
     ("fusion", 2, slra.ERR_INVALID_ARG), ("fusion", slra.FUSION_GATED, slra.ERR_INVALID_ARG),  # no gate_w
+    ("lowrank_rope_inside", 2, slra.ERR_INVALID_ARG),
 ])
 def test_validation_rejects(field, value, status):
     p = slra.Problem.from_workload(W.WAN_14B)
@@ -100,6 +101,13 @@ def test_gated_fusion_validation(gate_w, branches, bias, status):
     p = slra.Problem.from_workload(W.TINY).c()
     p.fusion, p.gate_w, p.branches, p.gate_bias = slra.FUSION_GATED, gate_w, branches, bias
     assert slra.lib().slra_validate(ctypes.byref(p)) == status
+
+
+def test_rope_inside_excludes_norope():
+    p = slra.Problem.from_workload(W.TINY, lowrank_rope_inside=1)
+    assert slra.validate(p) == slra.OK
+    p.lowrank_norope = 1
+    assert slra.validate(p) == slra.ERR_INVALID_ARG
 
 
 def test_validation_grid_limit():

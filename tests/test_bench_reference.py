@@ -21,7 +21,7 @@ def _run(extra, env_extra=None):
 
 
 @pytest.mark.parametrize("extra", [[], ["--proj", "separate-per-head"], ["--activation", "silu", "--lowrank-norope"],
-                                   ["--fusion", "gated"]])
+                                   ["--fusion", "gated"], ["--rope-inside"]])
 def test_reference_arm_line(extra):
     lines = _run(extra)
     assert len(lines) == 1

@@ -182,6 +182,31 @@ def test_gated_fusion_with_other_options():
     _case(w, "wan1.3b-gated", heads=[(0, 2)], qblocks=_sample_blocks(w.nb, 13, n=2), **_gate(w, -2.0))
 
 
+def test_rope_inside_activation():
+    """The truncated RoPE before the activation (the ordering RoLA's ablation compares against), on
+    both readout paths, with persistent summary CTAs changing head, and with SiLU."""
+    for w in (W.TINY, EDGE_128, EDGE_128_R64, EDGE_PROJ):
+        _case(w, f"{w.name}-inside", lowrank_rope_inside=1)
+    _case(EDGE_128, "edge128-inside-silu", lowrank_rope_inside=1, activation=slra.ACT_SILU, transform=_nonneg)
+
+
+def test_shift_residual_by_rope_ordering():
+    """RoLA Table 2's shift residual on synthetic inputs, measured on the GPU path's low-rank branch:
+    ||O_lr(p + c) - O_lr(p)|| / ||O_lr(p)|| for a constant shift c.  RoPE outside the activation:
+    unchanged up to fp32 rounding of the shifted angles; without RoPE: bit-identical; inside the
+    activation: a change of order one (absolute position leaks through the nonlinearity)."""
+    w = EDGE_128
+    x = I.make_inputs(w)
+    res = {}
+    for name, kw in (("outside", {}), ("none", {"lowrank_norope": 1}), ("inside", {"lowrank_rope_inside": 1})):
+        a = parity.run_gpu(slra.Problem.from_workload(w, branches=slra.BRANCH_LOWRANK, **kw), x)["out"]
+        b = parity.run_gpu(slra.Problem.from_workload(w, branches=slra.BRANCH_LOWRANK, pos_offset=(2, 3, 5), **kw),
+                           x)["out"]
+        res[name] = float(np.linalg.norm(a - b) / np.linalg.norm(a))
+    _log({"label": "shift-residual-edge128", **res})
+    assert res["outside"] < 1e-4 and res["none"] == 0.0 and res["inside"] > 1e-2
+
+
 def test_shift_invariance_on_gpu():
     """Shifting all positions leaves the masks unchanged exactly (fp64 selection) and the outputs
     unchanged up to the fp16 rounding of the rotated operands, which differs between the two runs:
