@@ -230,11 +230,20 @@ SLRA_API slra_status slra_attn_fwd(const slra_problem* p, const void* q, const v
 
 /*
  * The same forward pass on HOST buffers: copies q, k, v and A (slra_projection_elems(p) elements)
- * from host memory into `io` (a device buffer of at least slra_host_io_bytes(p) bytes), runs
- * slra_attn_fwd and copies `out` back to host memory, all on `stream`, then synchronizes the stream.
- * Host buffers should be pinned for speed.
+ * from host memory into `io` (a device buffer of at least slra_host_io_bytes(p) bytes), computes, and
+ * copies `out` back to host memory, then synchronizes `stream`.  Host buffers should be pinned.
+ * Heads are independent, so the call splits the problem into groups of heads (about eight per batch
+ * element) and pipelines them: the upload of one group, the compute of the previous one (on `stream`)
+ * and the download of the one before that overlap, on two copy streams of the library's own (created
+ * on first use, one pair per device) and two device slots carved from `io` and the workspace.  When
+ * two slots do not fit (or there is a single group) it copies everything in, computes and copies
+ * out, all on `stream`.  The device status word of `workspace` holds the OR of all groups' status.
+ * Calls on the same device are serialized inside the library; stage_events are not recorded.
  */
 SLRA_API size_t slra_host_io_bytes(const slra_problem* p);
+/* Number of head groups slra_attn_fwd_host will pipeline for p with the given buffer sizes (1: no
+ * pipelining), or -1 if p is invalid.  No GPU access. */
+SLRA_API int64_t slra_host_pipeline_groups(const slra_problem* p, size_t io_bytes, size_t workspace_bytes);
 SLRA_API slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const void* k_host,
                                const void* v_host, const void* A_host, void* out_host, void* io,
                                size_t io_bytes, void* workspace, size_t workspace_bytes, slra_stream_t stream);

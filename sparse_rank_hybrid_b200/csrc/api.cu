@@ -2,6 +2,7 @@
 // descriptors and the launch sequence of the hybrid attention forward.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -289,6 +290,158 @@ size_t qkv_bytes(const Derived& d) {
     return static_cast<size_t>(d.g.B) * d.g.L * d.g.Hh * d.g.D * 2;
 }
 
+// ------------------------------------------------------------------ host entry point, pipelined
+// Over PCIe the host entry point's copies (q, k, v in, out back) take several times the compute.
+// Heads are independent, so the call runs groups of heads as independent sub-problems, with the
+// upload of one group, the compute of the previous one and the download of the one before that in
+// flight together: two device slots used in turn, copies on two streams of their own (one per
+// direction), compute on the caller's stream, ordered by events.
+constexpr int kMaxPipeDevices = 64;
+struct HostPipe {
+    std::mutex mu;  // one pipelined call per device at a time: the streams and events are shared
+    bool ready = false;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, in[2] = {}, done[2] = {}, out[2] = {};
+};
+HostPipe g_pipes[kMaxPipeDevices];
+
+slra_status pipe_init(HostPipe& hp) {
+    if (hp.ready) return SLRA_OK;
+    const unsigned ef = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.start, ef) != cudaSuccess)
+        return SLRA_ERR_CUDA;
+    for (int i = 0; i < 2; ++i)
+        if (cudaEventCreateWithFlags(&hp.in[i], ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.done[i], ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.out[i], ef) != cudaSuccess)
+            return SLRA_ERR_CUDA;
+    hp.ready = true;
+    return SLRA_OK;
+}
+
+// The pipelined call's device status: each group's status word ORed into the caller's.
+__global__ void status_or_kernel(int* acc, const int* src) {
+    const int v = *src;
+    if (v) atomicOr(acc, v);
+}
+
+// Heads per group: about eight groups per batch element.
+int pipe_group_heads(int Hh) { return (Hh + 7) / 8; }
+
+// Number of head groups the host entry point pipelines (1: none) for these buffer sizes.
+int pipe_groups(const slra_problem* p, const Derived& d, size_t io_bytes, size_t ws_bytes) {
+    const Geom& g = d.g;
+    const int hg = pipe_group_heads(g.Hh);
+    const int G = g.B * ((g.Hh + hg - 1) / hg);
+    if (G < 2) return 1;
+    slra_problem pg = *p;
+    pg.batch = 1;
+    pg.heads = hg;
+    Derived dg;
+    if (derive(&pg, &dg) != SLRA_OK) return 1;
+    const size_t osz = p->out_dtype == SLRA_OUT_F32 ? 4 : 2;
+    const size_t in_g = align_up(static_cast<size_t>(g.L) * hg * g.D * 2, 256);
+    const size_t out_g = align_up(static_cast<size_t>(g.L) * hg * g.D * osz, 256);
+    const size_t a_full = align_up(d.a_elems * 2, 256);
+    const size_t a_g = p->proj_per_head ? align_up((p->proj_separate ? 2 : 1) * static_cast<size_t>(hg) * g.D * g.R * 2, 256) : 0;
+    const size_t slot_io = 3 * in_g + out_g + a_g, slot_ws = align_up(dg.lay.total_bytes, 256);
+    return (a_full + 2 * slot_io > io_bytes || 256 + 2 * slot_ws > ws_bytes) ? 1 : G;
+}
+
+// Runs the host entry point as pipelined head groups.  *used = false (nothing launched) when there
+// is a single group or the two slots do not fit the caller's io buffer and workspace.
+slra_status host_fwd_pipelined(const slra_problem* p, const Derived& d, const void* q_host, const void* k_host,
+                               const void* v_host, const void* A_host, void* out_host, uint8_t* io, size_t io_bytes,
+                               uint8_t* ws, size_t ws_bytes, cudaStream_t st, bool* used) {
+    *used = false;
+    const Geom& g = d.g;
+    const int hg = pipe_group_heads(g.Hh);
+    const int per_b = (g.Hh + hg - 1) / hg;
+    const int G = g.B * per_b;
+    if (pipe_groups(p, d, io_bytes, ws_bytes) < 2) return SLRA_OK;
+    slra_problem pg = *p;
+    pg.batch = 1;
+    pg.heads = hg;
+    for (auto& e : pg.stage_events) e = nullptr;  // the sub-calls time nothing
+    Derived dg;
+    if (derive(&pg, &dg) != SLRA_OK) return SLRA_OK;
+    const size_t osz = p->out_dtype == SLRA_OUT_F32 ? 4 : 2;
+    const size_t row_in = static_cast<size_t>(g.D) * 2, row_out = static_cast<size_t>(g.D) * osz;
+    const size_t in_g = align_up(static_cast<size_t>(g.L) * hg * row_in, 256);
+    const size_t out_g = align_up(static_cast<size_t>(g.L) * hg * row_out, 256);
+    const size_t a_full = align_up(d.a_elems * 2, 256);
+    const size_t side = static_cast<size_t>(g.D) * g.R;  // elements of one head's projection
+    const size_t a_g = p->proj_per_head ? align_up((p->proj_separate ? 2 : 1) * hg * side * 2, 256) : 0;
+    const size_t slot_io = 3 * in_g + out_g + a_g, slot_ws = align_up(dg.lay.total_bytes, 256);
+
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxPipeDevices) return SLRA_ERR_NO_DEVICE;
+    HostPipe& hp = g_pipes[dev];
+    std::lock_guard<std::mutex> lock(hp.mu);
+    slra_status s = pipe_init(hp);
+    if (s != SLRA_OK) return s;
+    *used = true;
+    auto fail = [&](slra_status why) {  // let nothing in flight outlive the call
+        cudaStreamSynchronize(hp.h2d);
+        cudaStreamSynchronize(hp.d2h);
+        cudaStreamSynchronize(st);
+        cudaGetLastError();
+        return why;
+    };
+    uint8_t* dA = io;
+    int* acc = reinterpret_cast<int*>(ws);  // the caller's status word (offset 0, as for slra_attn_fwd)
+    if (cudaEventRecord(hp.start, st) != cudaSuccess || cudaStreamWaitEvent(hp.h2d, hp.start, 0) != cudaSuccess ||
+        cudaMemsetAsync(acc, 0, sizeof(int), st) != cudaSuccess ||
+        cudaMemcpyAsync(dA, A_host, d.a_elems * 2, cudaMemcpyHostToDevice, hp.h2d) != cudaSuccess)
+        return fail(SLRA_ERR_CUDA);
+    for (int gi = 0; gi < G; ++gi) {
+        const int sl = gi & 1;
+        const int b = gi / per_b, h0 = (gi % per_b) * hg, hn = std::min(hg, g.Hh - h0);
+        uint8_t* base = io + a_full + sl * slot_io;
+        uint8_t *sq = base, *sk = base + in_g, *sv = base + 2 * in_g, *so = base + 3 * in_g, *sa = so + out_g;
+        uint8_t* sws = ws + 256 + sl * slot_ws;
+        const size_t off = (static_cast<size_t>(b) * g.L * g.Hh + h0);  // first row element offset / D
+        // upload, once the slot's previous group has finished reading its inputs
+        if (gi >= 2 && cudaStreamWaitEvent(hp.h2d, hp.done[sl], 0) != cudaSuccess) return fail(SLRA_ERR_CUDA);
+        const void* srcs[3] = {q_host, k_host, v_host};
+        uint8_t* dsts[3] = {sq, sk, sv};
+        for (int t = 0; t < 3; ++t)
+            if (cudaMemcpy2DAsync(dsts[t], hn * row_in, static_cast<const uint8_t*>(srcs[t]) + off * row_in,
+                                  g.Hh * row_in, hn * row_in, g.L, cudaMemcpyHostToDevice, hp.h2d) != cudaSuccess)
+                return fail(SLRA_ERR_CUDA);
+        if (cudaEventRecord(hp.in[sl], hp.h2d) != cudaSuccess) return fail(SLRA_ERR_CUDA);
+        // compute, once the inputs are in and the slot's previous output has been downloaded
+        if (cudaStreamWaitEvent(st, hp.in[sl], 0) != cudaSuccess ||
+            (gi >= 2 && cudaStreamWaitEvent(st, hp.out[sl], 0) != cudaSuccess))
+            return fail(SLRA_ERR_CUDA);
+        const void* Ag = dA;
+        if (p->proj_per_head) {  // this group's heads of each side, contiguous
+            for (int sd = 0; sd < (p->proj_separate ? 2 : 1); ++sd)
+                if (cudaMemcpyAsync(sa + sd * hn * side * 2, dA + (sd * g.Hh + h0) * side * 2, hn * side * 2,
+                                    cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+                    return fail(SLRA_ERR_CUDA);
+            Ag = sa;
+        }
+        slra_problem pgi = pg;
+        pgi.heads = hn;
+        s = slra_attn_fwd(&pgi, sq, sk, sv, Ag, so, sws, slot_ws, reinterpret_cast<slra_stream_t>(st));
+        if (s != SLRA_OK) return fail(s);
+        status_or_kernel<<<1, 1, 0, st>>>(acc, reinterpret_cast<const int*>(sws));
+        if (cudaGetLastError() != cudaSuccess || cudaEventRecord(hp.done[sl], st) != cudaSuccess)
+            return fail(SLRA_ERR_CUDA);
+        // download into the group's strided place in the host output
+        if (cudaStreamWaitEvent(hp.d2h, hp.done[sl], 0) != cudaSuccess ||
+            cudaMemcpy2DAsync(static_cast<uint8_t*>(out_host) + off * row_out, g.Hh * row_out, so, hn * row_out,
+                              hn * row_out, g.L, cudaMemcpyDeviceToHost, hp.d2h) != cudaSuccess ||
+            cudaEventRecord(hp.out[sl], hp.d2h) != cudaSuccess)
+            return fail(SLRA_ERR_CUDA);
+    }
+    if (cudaStreamWaitEvent(st, hp.out[(G - 1) & 1], 0) != cudaSuccess) return fail(SLRA_ERR_CUDA);
+    return cuda_status(cudaStreamSynchronize(st));
+}
+
 }  // namespace
 
 extern "C" {
@@ -441,6 +594,12 @@ size_t slra_host_io_bytes(const slra_problem* p) {
     return 3 * in_b + a_b + out_b;
 }
 
+int64_t slra_host_pipeline_groups(const slra_problem* p, size_t io_bytes, size_t workspace_bytes) {
+    Derived d;
+    if (derive(p, &d) != SLRA_OK) return -1;
+    return pipe_groups(p, d, io_bytes, workspace_bytes);
+}
+
 slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const void* k_host, const void* v_host,
                                const void* A_host, void* out_host, void* io, size_t io_bytes, void* workspace,
                                size_t workspace_bytes, slra_stream_t stream) {
@@ -449,7 +608,14 @@ slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const 
     if (s != SLRA_OK) return s;
     if (!q_host || !k_host || !v_host || !A_host || !out_host || !io) return SLRA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(io) & 255u) != 0 || io_bytes < slra_host_io_bytes(p)) return SLRA_ERR_WORKSPACE;
+    if ((s = check_ws(d, workspace, workspace_bytes)) != SLRA_OK) return s;
+    if ((s = check_device()) != SLRA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    bool used = false;
+    s = host_fwd_pipelined(p, d, q_host, k_host, v_host, A_host, out_host, static_cast<uint8_t*>(io), io_bytes,
+                           static_cast<uint8_t*>(workspace), workspace_bytes, st, &used);
+    if (used || s != SLRA_OK) return s;
+    // one group (or too little room for two slots): copy in, compute, copy out
     const size_t raw = qkv_bytes(d);
     const size_t in_b = align_up(raw, 256);
     const size_t a_raw = d.a_elems * 2;

@@ -27,7 +27,8 @@ FUSION_SUM, FUSION_GATED = 0, 1
 # Every symbol include/slra.h declares.
 EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_validate", "slra_keep_count",
            "slra_projection_elems",
-           "slra_workspace_layout", "slra_attn_fwd", "slra_host_io_bytes", "slra_attn_fwd_host",
+           "slra_workspace_layout", "slra_attn_fwd", "slra_host_io_bytes", "slra_host_pipeline_groups",
+           "slra_attn_fwd_host",
            "slra_select_blocks", "slra_lowrank_summary", "slra_device_status", "slra_lowrank_summary_noalloc")
 
 
@@ -85,6 +86,8 @@ def lib():
         L.slra_attn_fwd.argtypes = [PP, P, P, P, P, P, P, S, P]
         L.slra_host_io_bytes.restype = S
         L.slra_host_io_bytes.argtypes = [PP]
+        L.slra_host_pipeline_groups.restype = ctypes.c_int64
+        L.slra_host_pipeline_groups.argtypes = [PP, S, S]
         L.slra_attn_fwd_host.argtypes = [PP, P, P, P, P, P, P, S, P, S, P]
         L.slra_select_blocks.argtypes = [PP, P, P, P, P, S, P]
         L.slra_lowrank_summary.argtypes = [PP, P, P, P, P, S, P]
@@ -257,6 +260,11 @@ def attn_fwd(prob: Problem, q, k, v, A, out=None, workspace=None, stream=None):
 
 def host_io_bytes(prob: Problem) -> int:
     return int(lib().slra_host_io_bytes(ctypes.byref(prob.c())))
+
+
+def host_pipeline_groups(prob: Problem, io_bytes: int, workspace_bytes: int) -> int:
+    """Head groups the host entry point pipelines for these buffer sizes (1: none)."""
+    return int(lib().slra_host_pipeline_groups(ctypes.byref(prob.c()), io_bytes, workspace_bytes))
 
 
 def attn_fwd_host(prob: Problem, q_host, k_host, v_host, A_host, out_host, io, workspace, stream=None):

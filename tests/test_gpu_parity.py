@@ -248,6 +248,50 @@ def test_host_entry_point_matches_device():
     assert np.array_equal(out.numpy().astype(np.float64), dev)
 
 
+def _host_out(p, x):
+    import torch
+    host = {n: torch.from_numpy(np.ascontiguousarray(x[n]).view(np.int16)).view(torch.bfloat16).pin_memory()
+            for n in ("q", "k", "v", "A")}
+    dt = torch.float32 if p.out_dtype == slra.OUT_F32 else torch.bfloat16
+    out = torch.empty((p.batch, p.L, p.heads, p.head_dim), dtype=dt).pin_memory()
+    io = torch.empty(slra.host_io_bytes(p), dtype=torch.uint8, device="cuda")
+    ws = slra.alloc_workspace(p)
+    assert slra.host_pipeline_groups(p, io.numel(), ws.numel()) > 1  # the pipelined path is the one tested
+    slra.attn_fwd_host(p, host["q"], host["k"], host["v"], host["A"], out, io, ws)
+    st = slra.device_status(ws)
+    assert st == slra.OK, slra.status_string(st)
+    return out.float().numpy().astype(np.float64)
+
+
+EDGE_B2 = W.Workload("edge-b2-128", 2, 5, 128, 2, 9, 11, 32, 64, 0.25, 7410)
+
+
+@pytest.mark.parametrize("case", ["plain", "options", "batch2", "bf16"])
+def test_host_entry_point_pipelined(case):
+    """The host entry point's pipelined head groups (uploads, compute and downloads overlapped) give
+    the device entry point's output: the same kernels per head, only the low-rank summary's split of
+    the sequence can differ with the group size (fp32 order), hence a relative bound instead of
+    equality; and the result is within the oracle tolerance."""
+    w, kw, tf = EDGE_PROJ, {}, None
+    if case == "options":
+        kw = dict(proj_separate=1, proj_per_head=1, activation=slra.ACT_SILU, **_gate(EDGE_PROJ, -1.0))
+        tf = lambda x: _nonneg(_projections(EDGE_PROJ, 1, 1)(x))
+    elif case == "batch2":
+        w = EDGE_B2
+    elif case == "bf16":
+        kw = dict(out_dtype=slra.OUT_BF16)
+    p = slra.Problem.from_workload(w, **kw)
+    x = I.make_inputs(w)
+    if tf is not None:
+        x = tf(x)
+    dev = parity.run_gpu(p, x)
+    host = _host_out(p, x)
+    assert np.abs(host - dev["out"]).max() <= 1e-5 * np.abs(dev["out"]).max() + (4e-3 if case == "bf16" else 0.0)
+    if case != "bf16":
+        dev["out"] = host
+        _log(parity.compare(p, x, dev, label=f"host-pipelined-{case}"))
+
+
 def test_range_error_reported():
     """An input too large for the fp16 operands is reported through the device status word."""
     import torch
