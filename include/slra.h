@@ -232,7 +232,7 @@ SLRA_API slra_status slra_attn_fwd(const slra_problem* p, const void* q, const v
  * The same forward pass on HOST buffers: copies q, k, v and A (slra_projection_elems(p) elements)
  * from host memory into `io` (a device buffer of at least slra_host_io_bytes(p) bytes), computes, and
  * copies `out` back to host memory, then synchronizes `stream`.  Host buffers should be pinned.
- * Heads are independent, so the call splits the problem into groups of heads (about eight per batch
+ * Heads are independent, so the call splits the problem into groups of heads (about sixteen per batch
  * element) and pipelines them: the upload of one group, the compute of the previous one (on `stream`)
  * and the download of the one before that overlap, on two copy streams of the library's own (created
  * on first use, one pair per device) and two device slots carved from `io` and the workspace.  When

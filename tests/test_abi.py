@@ -111,14 +111,14 @@ def test_rope_inside_excludes_norope():
 
 
 def test_host_pipeline_plan():
-    """The host entry point pipelines about eight head groups per batch element when two group slots
+    """The host entry point pipelines about sixteen head groups per batch element when two group slots
     fit the buffers it is given, and falls back to one group otherwise (no GPU needed)."""
     def groups(w, io=None, ws=None, **kw):
         p = slra.Problem.from_workload(w, **kw)
         return slra.host_pipeline_groups(p, slra.host_io_bytes(p) if io is None else io,
                                          slra.layout(p).total_bytes if ws is None else ws)
-    assert groups(W.WAN_14B) == 8 and groups(W.WAN_1_3B) == 6
-    assert groups(W.WAN_14B, proj_separate=1, proj_per_head=1) == 8
+    assert groups(W.WAN_14B) == 14 and groups(W.WAN_1_3B) == 12   # 40 heads in groups of 3; 12 of 1
+    assert groups(W.WAN_14B, proj_separate=1, proj_per_head=1) == 14
     assert groups(W.TINY) == 1                      # two one-head slots need more than the 2-head workspace
     assert groups(W.WAN_14B, io=1 << 20) == 1 and groups(W.WAN_14B, ws=1 << 20) == 1
     bad = slra.Problem.from_workload(W.WAN_14B.with_(rank=24))
