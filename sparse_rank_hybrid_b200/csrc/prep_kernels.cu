@@ -108,6 +108,13 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
         return;
     }
     const uint32_t c16 = quad & 7, sl = quad >> 3;  // 16-byte chunk within its slab, slab
+    // (cos, sin) of this thread's pairs at the last position used: a thread's tokens are G apart, so the
+    // temporal position rarely changes within a block and the height one only every W tokens; only
+    // the pairs whose position moved are reloaded
+    double2 cs_c[4];
+    int pos_c[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) pos_c[u] = -1;
     for (int i = grp; i < blk; i += G) {
         const int n = n0 + i;
         const size_t dst = (static_cast<size_t>(bh) * g.Lp + n) * D + 8 * quad;
@@ -116,7 +123,7 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
             const uint4 qr = *reinterpret_cast<const uint4*>(smem + 0 * NS * slab + off);
             const uint4 kr = *reinterpret_cast<const uint4*>(smem + 1 * NS * slab + off);
             const uint4 vr = *reinterpret_cast<const uint4*>(smem + 2 * NS * slab + off);
-            const int pos3[3] = {n / HW, (n / g.W) % g.H, n % g.W};
+            const int pt = n / HW, ph = (n / g.W) % g.H, pw = n % g.W;
             const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qr);
             const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
             const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vr);
@@ -127,7 +134,12 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
             float m = 0.f;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const double2 cs = __ldg(tab + toff[u] + pos3[axis[u]]);
+                const int pos = axis[u] == 0 ? pt : (axis[u] == 1 ? ph : pw);
+                if (pos != pos_c[u]) {
+                    cs_c[u] = __ldg(tab + toff[u] + pos);
+                    pos_c[u] = pos;
+                }
+                const double2 cs = cs_c[u];
                 const float2 qf = __bfloat1622float2(q2[u]);
                 const float2 kf = __bfloat1622float2(k2[u]);
                 const float2 vf = __bfloat1622float2(v2[u]);
