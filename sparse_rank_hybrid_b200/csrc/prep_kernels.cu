@@ -267,21 +267,33 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
     const double* qb = qbar + static_cast<size_t>(bh) * nb * D;
     const double* kb = kbar + static_cast<size_t>(bh) * nb * D;
 
-    // A fragments: row l/4 of the 8 query blocks, dims 4*kk + l%4 for the D/4 k-steps
+    // The D/4 k-steps take the dims in pairs: k-steps 2m and 2m+1 give lane l dims 8m + 2(l%4) and
+    // 8m + 2(l%4) + 1, so each lane loads both with one 16-byte load and the four lanes of a row read 64
+    // contiguous bytes (any order of the dims gives the same dot product up to fp64 rounding).
+    // A fragments: row l/4 of the 8 query blocks.
     double af[D / 4];
     {
         const int ar = a0 + (lane >> 2);
+        const double2* arow = reinterpret_cast<const double2*>(qb + static_cast<size_t>(ar < nb ? ar : 0) * D) + (lane & 3);
 #pragma unroll
-        for (int kk = 0; kk < D / 4; ++kk)
-            af[kk] = ar < nb ? __ldg(qb + static_cast<size_t>(ar) * D + 4 * kk + (lane & 3)) : 0.0;
+        for (int m = 0; m < D / 8; ++m) {
+            const double2 a2 = ar < nb ? __ldg(arow + 4 * m) : make_double2(0.0, 0.0);
+            af[2 * m] = a2.x;
+            af[2 * m + 1] = a2.y;
+        }
     }
     const int ntile = (nb + 7) / 8;
     for (int t = warp; t < ntile; t += 8) {
-        const int key = 8 * t + (lane >> 2);  // B fragment: key l/4 of the tile, dims 4*kk + l%4
-        const double* kr = kb + static_cast<size_t>(key < nb ? key : nb - 1) * D + (lane & 3);
+        const int key = 8 * t + (lane >> 2);  // B fragment: key l/4 of the tile, the same dims as A
+        const double2* kr =
+            reinterpret_cast<const double2*>(kb + static_cast<size_t>(key < nb ? key : nb - 1) * D) + (lane & 3);
         double d0 = 0.0, d1 = 0.0;
 #pragma unroll
-        for (int kk = 0; kk < D / 4; ++kk) dmma_8x8x4(d0, d1, af[kk], __ldg(kr + 4 * kk));
+        for (int m = 0; m < D / 8; ++m) {
+            const double2 b2 = __ldg(kr + 4 * m);
+            dmma_8x8x4(d0, d1, af[2 * m], b2.x);
+            dmma_8x8x4(d0, d1, af[2 * m + 1], b2.y);
+        }
         const int r = lane >> 2, c = 8 * t + 2 * (lane & 3);
         if (c < nb) scores[r * nb + c] = d0;
         if (c + 1 < nb) scores[r * nb + c + 1] = d1;
