@@ -207,6 +207,28 @@ def test_shift_residual_by_rope_ordering():
     assert res["outside"] < 1e-4 and res["none"] == 0.0 and res["inside"] > 1e-2
 
 
+def test_exact_ties_keep_the_lower_blocks():
+    """Key blocks whose keys are all zero have block means of exactly zero, so their scores tie exactly
+    (+0 for every query block, whose mean has components of both signs); the selection keeps the
+    lowest-indexed of the tied blocks, the oracle's rule.  Here the cut falls inside the tied group,
+    so every row is tie-flagged and the kept lists must equal the oracle's bit for bit anyway."""
+    w = W.TINY.with_(name="ties", T=4, H=16, W=16, heads=2, block=64, keep_frac=0.5)  # 16 blocks, keep 8
+    x = I.make_inputs(w)
+    k = x["k"].copy()
+    k[:, 2 * 64:14 * 64] = 0  # blocks 2..13: zero keys
+    x = dict(x, k=k)
+    p = slra.Problem.from_workload(w)
+    gpu = parity.run_gpu(p, x)
+    import oracle
+    _, per = oracle.forward(x, (w.T, w.H, w.W), w.block, w.keep_frac, w.rank, branches=1, qblocks=[0])
+    for (b, h), r in per.items():
+        bh = b * w.heads + h
+        assert r["tie"].any()
+        assert np.array_equal(gpu["idx"][bh], r["idx"]), (bh, gpu["idx"][bh], r["idx"])
+        assert np.array_equal(gpu["tie"][bh].astype(bool), r["tie"].astype(bool))
+    parity.compare(p, x, gpu, label="exact-ties")
+
+
 def test_shift_invariance_on_gpu():
     """Shifting all positions leaves the masks unchanged exactly (fp64 selection) and the outputs
     unchanged up to the fp16 rounding of the rotated operands, which differs between the two runs:
