@@ -12,6 +12,14 @@
 
 using namespace slra;
 
+namespace slra {
+// The pipelined host call's device status: each group's status word ORed into the caller's.
+__global__ void status_or_kernel(int* acc, const int* src) {
+    const int v = *src;
+    if (v) atomicOr(acc, v);
+}
+}  // namespace slra
+
 namespace {
 
 constexpr int64_t kMaxBlocks = 2048;  // selection keeps a row of scores in shared memory
@@ -321,62 +329,60 @@ slra_status pipe_init(HostPipe& hp) {
     return SLRA_OK;
 }
 
-// The pipelined call's device status: each group's status word ORed into the caller's.
-__global__ void status_or_kernel(int* acc, const int* src) {
-    const int v = *src;
-    if (v) atomicOr(acc, v);
-}
-
 // Heads per group: about sixteen groups per batch element (at Wan2.1-14B, 14 groups of 3 heads: 47.6 ms
 // per call, against 49.8 with 8 groups and 58.3 with 4; the first upload and the last download are
 // what smaller groups shorten).
 int pipe_group_heads(int Hh) { return (Hh + 15) / 16; }
 
-// Number of head groups the host entry point pipelines (1: none) for these buffer sizes.
-int pipe_groups(const slra_problem* p, const Derived& d, size_t io_bytes, size_t ws_bytes) {
+// How the host entry point splits a problem: groups of hg heads (the last of a batch element may be
+// smaller), each a sub-problem with batch 1, run through two device slots.
+struct PipePlan {
+    int hg, per_b, G;      // heads per group, groups per batch element, groups
+    slra_problem sub;      // a full group's sub-problem (stage events cleared)
+    size_t row_in, row_out;  // bytes of one head row of the inputs / of the output
+    size_t in_g, out_g;    // bytes of one input tensor / of the output of a group in a slot
+    size_t a_full, a_g;    // the whole projection argument; a group's per-head projections (or 0)
+    size_t side;           // elements of one head's projection
+    size_t slot_io, slot_ws;  // one slot in the io buffer and in the workspace
+};
+
+// Fills *pl; returns the number of groups (1: no pipelining, because there is a single group or two
+// slots do not fit the buffers).
+int plan_pipeline(const slra_problem* p, const Derived& d, size_t io_bytes, size_t ws_bytes, PipePlan* pl) {
     const Geom& g = d.g;
-    const int hg = pipe_group_heads(g.Hh);
-    const int G = g.B * ((g.Hh + hg - 1) / hg);
-    if (G < 2) return 1;
-    slra_problem pg = *p;
-    pg.batch = 1;
-    pg.heads = hg;
+    pl->hg = pipe_group_heads(g.Hh);
+    pl->per_b = (g.Hh + pl->hg - 1) / pl->hg;
+    pl->G = g.B * pl->per_b;
+    if (pl->G < 2) return 1;
+    pl->sub = *p;
+    pl->sub.batch = 1;
+    pl->sub.heads = pl->hg;
+    for (auto& e : pl->sub.stage_events) e = nullptr;  // the sub-calls time nothing
     Derived dg;
-    if (derive(&pg, &dg) != SLRA_OK) return 1;
+    if (derive(&pl->sub, &dg) != SLRA_OK) return 1;
     const size_t osz = p->out_dtype == SLRA_OUT_F32 ? 4 : 2;
-    const size_t in_g = align_up(static_cast<size_t>(g.L) * hg * g.D * 2, 256);
-    const size_t out_g = align_up(static_cast<size_t>(g.L) * hg * g.D * osz, 256);
-    const size_t a_full = align_up(d.a_elems * 2, 256);
-    const size_t a_g = p->proj_per_head ? align_up((p->proj_separate ? 2 : 1) * static_cast<size_t>(hg) * g.D * g.R * 2, 256) : 0;
-    const size_t slot_io = 3 * in_g + out_g + a_g, slot_ws = align_up(dg.lay.total_bytes, 256);
-    return (a_full + 2 * slot_io > io_bytes || 256 + 2 * slot_ws > ws_bytes) ? 1 : G;
+    pl->row_in = static_cast<size_t>(g.D) * 2;
+    pl->row_out = static_cast<size_t>(g.D) * osz;
+    pl->in_g = align_up(static_cast<size_t>(g.L) * pl->hg * pl->row_in, 256);
+    pl->out_g = align_up(static_cast<size_t>(g.L) * pl->hg * pl->row_out, 256);
+    pl->a_full = align_up(d.a_elems * 2, 256);
+    pl->side = static_cast<size_t>(g.D) * g.R;
+    pl->a_g = p->proj_per_head ? align_up((p->proj_separate ? 2 : 1) * pl->hg * pl->side * 2, 256) : 0;
+    pl->slot_io = 3 * pl->in_g + pl->out_g + pl->a_g;
+    pl->slot_ws = align_up(dg.lay.total_bytes, 256);
+    if (pl->a_full + 2 * pl->slot_io > io_bytes || 256 + 2 * pl->slot_ws > ws_bytes) return 1;
+    return pl->G;
 }
 
-// Runs the host entry point as pipelined head groups.  *used = false (nothing launched) when there
-// is a single group or the two slots do not fit the caller's io buffer and workspace.
+// Runs the host entry point as pipelined head groups.  *used = false (nothing launched) when the plan
+// has a single group.
 slra_status host_fwd_pipelined(const slra_problem* p, const Derived& d, const void* q_host, const void* k_host,
                                const void* v_host, const void* A_host, void* out_host, uint8_t* io, size_t io_bytes,
                                uint8_t* ws, size_t ws_bytes, cudaStream_t st, bool* used) {
     *used = false;
     const Geom& g = d.g;
-    const int hg = pipe_group_heads(g.Hh);
-    const int per_b = (g.Hh + hg - 1) / hg;
-    const int G = g.B * per_b;
-    if (pipe_groups(p, d, io_bytes, ws_bytes) < 2) return SLRA_OK;
-    slra_problem pg = *p;
-    pg.batch = 1;
-    pg.heads = hg;
-    for (auto& e : pg.stage_events) e = nullptr;  // the sub-calls time nothing
-    Derived dg;
-    if (derive(&pg, &dg) != SLRA_OK) return SLRA_OK;
-    const size_t osz = p->out_dtype == SLRA_OUT_F32 ? 4 : 2;
-    const size_t row_in = static_cast<size_t>(g.D) * 2, row_out = static_cast<size_t>(g.D) * osz;
-    const size_t in_g = align_up(static_cast<size_t>(g.L) * hg * row_in, 256);
-    const size_t out_g = align_up(static_cast<size_t>(g.L) * hg * row_out, 256);
-    const size_t a_full = align_up(d.a_elems * 2, 256);
-    const size_t side = static_cast<size_t>(g.D) * g.R;  // elements of one head's projection
-    const size_t a_g = p->proj_per_head ? align_up((p->proj_separate ? 2 : 1) * hg * side * 2, 256) : 0;
-    const size_t slot_io = 3 * in_g + out_g + a_g, slot_ws = align_up(dg.lay.total_bytes, 256);
+    PipePlan pl;
+    if (plan_pipeline(p, d, io_bytes, ws_bytes, &pl) < 2) return SLRA_OK;
 
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxPipeDevices) return SLRA_ERR_NO_DEVICE;
@@ -393,6 +399,9 @@ slra_status host_fwd_pipelined(const slra_problem* p, const Derived& d, const vo
         return why;
     };
     uint8_t* dA = io;
+    const int hg = pl.hg, per_b = pl.per_b, G = pl.G;
+    const size_t row_in = pl.row_in, row_out = pl.row_out, in_g = pl.in_g, out_g = pl.out_g, side = pl.side;
+    const size_t slot_io = pl.slot_io, slot_ws = pl.slot_ws;
     int* acc = reinterpret_cast<int*>(ws);  // the caller's status word (offset 0, as for slra_attn_fwd)
     if (cudaEventRecord(hp.start, st) != cudaSuccess || cudaStreamWaitEvent(hp.h2d, hp.start, 0) != cudaSuccess ||
         cudaMemsetAsync(acc, 0, sizeof(int), st) != cudaSuccess ||
@@ -401,7 +410,7 @@ slra_status host_fwd_pipelined(const slra_problem* p, const Derived& d, const vo
     for (int gi = 0; gi < G; ++gi) {
         const int sl = gi & 1;
         const int b = gi / per_b, h0 = (gi % per_b) * hg, hn = std::min(hg, g.Hh - h0);
-        uint8_t* base = io + a_full + sl * slot_io;
+        uint8_t* base = io + pl.a_full + sl * slot_io;
         uint8_t *sq = base, *sk = base + in_g, *sv = base + 2 * in_g, *so = base + 3 * in_g, *sa = so + out_g;
         uint8_t* sws = ws + 256 + sl * slot_ws;
         const size_t off = (static_cast<size_t>(b) * g.L * g.Hh + h0);  // first row element offset / D
@@ -426,11 +435,11 @@ slra_status host_fwd_pipelined(const slra_problem* p, const Derived& d, const vo
                     return fail(SLRA_ERR_CUDA);
             Ag = sa;
         }
-        slra_problem pgi = pg;
+        slra_problem pgi = pl.sub;
         pgi.heads = hn;
         s = slra_attn_fwd(&pgi, sq, sk, sv, Ag, so, sws, slot_ws, reinterpret_cast<slra_stream_t>(st));
         if (s != SLRA_OK) return fail(s);
-        status_or_kernel<<<1, 1, 0, st>>>(acc, reinterpret_cast<const int*>(sws));
+        slra::status_or_kernel<<<1, 1, 0, st>>>(acc, reinterpret_cast<const int*>(sws));
         if (cudaGetLastError() != cudaSuccess || cudaEventRecord(hp.done[sl], st) != cudaSuccess)
             return fail(SLRA_ERR_CUDA);
         // download into the group's strided place in the host output
@@ -599,7 +608,8 @@ size_t slra_host_io_bytes(const slra_problem* p) {
 int64_t slra_host_pipeline_groups(const slra_problem* p, size_t io_bytes, size_t workspace_bytes) {
     Derived d;
     if (derive(p, &d) != SLRA_OK) return -1;
-    return pipe_groups(p, d, io_bytes, workspace_bytes);
+    PipePlan pl;
+    return plan_pipeline(p, d, io_bytes, workspace_bytes, &pl);
 }
 
 slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const void* k_host, const void* v_host,
