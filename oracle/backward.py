@@ -1,0 +1,100 @@
+"""fp64 CPU oracle for the gradients of the hybrid attention forward (one batch element, one head).
+
+TEST INFRASTRUCTURE ONLY, like the rest of `oracle/`: the library never imports it.
+
+The backward pass is defined as the derivative of the forward pass, so the plainest correct statement
+of it is the forward written with differentiable fp64 PyTorch CPU operations and differentiated by
+autograd.  The block selection is piecewise constant in q and k (it only picks which key blocks each
+query block attends to), so it is taken from the C oracle's forward and held fixed: gradients flow
+through the attention over the kept blocks and through the low-rank branch, not through the choice of
+blocks.
+
+The restatement follows the forward's steps (RoLA "3 Preliminary" 3D RoPE, "4.1" block-sparse softmax
+attention plus the low-rank branch, "4.2"/"4.3" rank-truncated RoPE outside the relu feature map,
+"B.1" the query-independent summary):
+  q^, k^ = RoPE(q), RoPE(k)                      (pairs (2j, 2j+1), the C oracle's own cos/sin)
+  O_s    = softmax(q^ k^T / sqrt(D) over the kept key blocks of each query block) v
+  phi    = relu(x A);  psi = phi with its first r coordinates rotated by the truncated RoPE
+  S      = sum_j psi(k_j) v_j^T,  z = sum_j phi(k_j)
+  O_lr   = psi(q) S / (phi(q) . z + 1e-6)
+  out    = O_s + O_lr
+The cos/sin of every (token, pair) come from the C oracle's rotation of unit vectors, so both
+restatements use the same tables; `tests/test_oracle_pins.py` pins this forward to the C oracle's and
+its gradients to finite differences and to torch's dense attention backward.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from . import block_means, block_scores, keep_count, rope_rows, topk
+
+
+def rope_cos_sin(grid, D: int, theta: float = 1e4, offset=(0, 0, 0), split=None) -> np.ndarray:
+    """[L, D/2, 2] (cos, sin) of every token and rotary pair of a D-wide head: the C oracle's rotation
+    applied to the unit vector of each pair's first coordinate."""
+    T, H, W = grid
+    L = T * H * W
+    e = np.zeros((L, D))
+    e[:, 0::2] = 1.0
+    y = rope_rows(e, grid, D // 2, theta, offset, split)
+    return np.stack([y[:, 0::2], y[:, 1::2]], axis=-1)
+
+
+def _rotate(x: torch.Tensor, cs: torch.Tensor, npairs: int) -> torch.Tensor:
+    """Rotate pairs (2j, 2j+1), j < npairs, of every row of x by the angles whose cos/sin are cs."""
+    x0, x1 = x[:, 0:2 * npairs:2], x[:, 1:2 * npairs:2]
+    c, s = cs[:, :npairs, 0], cs[:, :npairs, 1]
+    y = x.clone()
+    y[:, 0:2 * npairs:2] = x0 * c - x1 * s
+    y[:, 1:2 * npairs:2] = x0 * s + x1 * c
+    return y
+
+
+def block_mask(idx: np.ndarray, L: int, block: int) -> torch.Tensor:
+    """[L, L] bool: query i may attend key j iff j's block is kept for i's block."""
+    nb = idx.shape[0]
+    kept = np.zeros((nb, nb), dtype=bool)
+    for a in range(nb):
+        kept[a, idx[a]] = True
+    bl = np.arange(L) // block
+    return torch.from_numpy(kept[bl][:, bl])
+
+
+def forward_torch(q, k, v, A, cs, mask, rank: int, branches: int = 3) -> torch.Tensor:
+    """The forward of one head in differentiable fp64 torch (see the module docstring)."""
+    L, D = q.shape
+    out = torch.zeros_like(v)
+    if branches & 1:
+        qh, kh = _rotate(q, cs, D // 2), _rotate(k, cs, D // 2)
+        s = (qh @ kh.T) / math.sqrt(D)
+        s = s.masked_fill(~mask, float("-inf"))
+        out = out + torch.softmax(s, dim=1) @ v
+    if branches & 2:
+        phq, phk = torch.relu(q @ A), torch.relu(k @ A)
+        psq, psk = _rotate(phq, cs, rank // 2), _rotate(phk, cs, rank // 2)
+        S, z = psk.T @ v, phk.sum(0)
+        out = out + (psq @ S) / (phq @ z + 1e-6)[:, None]
+    return out
+
+
+def head_backward(q, k, v, A, dout, grid, block: int, keep_frac: float, rank: int, *, theta=1e4,
+                  offset=(0, 0, 0), split=None, branches: int = 3, idx=None):
+    """Gradients of sum(dout * out) with respect to q, k, v [L, D] and A [D, R] (all fp64 numpy), the
+    block selection held at the forward's (or `idx`).  Returns dict(dq, dk, dv, dA, out, idx)."""
+    L, D = q.shape
+    if idx is None:
+        qh = rope_rows(q, grid, D // 2, theta, offset, split)
+        kh = rope_rows(k, grid, D // 2, theta, offset, split)
+        s = block_scores(block_means(qh, block), block_means(kh, block))
+        idx, _ = topk(s, keep_count(keep_frac, s.shape[0]))
+    cs = torch.from_numpy(rope_cos_sin(grid, D, theta, offset, split))
+    mask = block_mask(np.asarray(idx), L, block)
+    tq, tk, tv, tA = (torch.tensor(np.asarray(a, dtype=np.float64), requires_grad=True) for a in (q, k, v, A))
+    out = forward_torch(tq, tk, tv, tA, cs, mask, rank, branches)
+    dq, dk, dv, dA = torch.autograd.grad(out, (tq, tk, tv, tA), torch.from_numpy(np.asarray(dout, dtype=np.float64)),
+                                         allow_unused=True)
+    z = lambda g, ref: np.zeros_like(np.asarray(ref, dtype=np.float64)) if g is None else g.numpy()
+    return dict(dq=z(dq, q), dk=z(dk, k), dv=z(dv, v), dA=z(dA, A), out=out.detach().numpy(), idx=np.asarray(idx))

@@ -565,3 +565,79 @@ def test_rope_inside_is_not_shift_invariant(oracle_mod):
     assert resid() < 1e-12
     assert resid(lowrank_rope=False) == 0.0
     assert resid(rope_inside=True) > 1e-2
+
+
+# ---------------------------------------------------------------------------------------- backward
+def _bw_case(oracle_mod, keep_frac=0.5, seed=9):
+    w = W.TINY.with_(keep_frac=keep_frac)
+    x = I.make_inputs(w)
+    dec = oracle_mod.decode_bf16
+    q, k, v = dec(x["q"][0, :, 0]), dec(x["k"][0, :, 0]), dec(x["v"][0, :, 0])
+    A = dec(x["A"])
+    dout = np.random.default_rng(seed).standard_normal(q.shape)
+    return w, q, k, v, A, dout
+
+
+def test_backward_restatement_matches_forward(oracle_mod):
+    """The differentiable fp64 torch restatement of the forward gives the C oracle's output."""
+    from oracle import backward as B
+    w, q, k, v, A, dout = _bw_case(oracle_mod)
+    g = B.head_backward(q, k, v, A, dout, (w.T, w.H, w.W), w.block, w.keep_frac, w.rank)
+    r = oracle_mod.head_forward(q, k, v, A, (w.T, w.H, w.W), w.block, w.keep_frac, w.rank)
+    assert np.array_equal(g["idx"], r["idx"])
+    assert np.allclose(g["out"], r["out"], rtol=1e-12, atol=1e-12)
+
+
+def test_backward_matches_finite_differences(oracle_mod):
+    """<grad, d> equals the central difference of sum(dout * out) along random directions d of q, k, v
+    and A, the forward evaluated by the C oracle with the selection held fixed (both branches; the
+    relu kinks are not crossed at this step size)."""
+    from oracle import backward as B
+    w, q, k, v, A, dout = _bw_case(oracle_mod)
+    grid = (w.T, w.H, w.W)
+    g = B.head_backward(q, k, v, A, dout, grid, w.block, w.keep_frac, w.rank)
+    rng = np.random.default_rng(4)
+    h = 1e-6
+
+    def f(qq, kk, vv, AA):
+        r = oracle_mod.head_forward(qq, kk, vv, AA, grid, w.block, w.keep_frac, w.rank, idx_override=g["idx"])
+        return float((dout * r["out"]).sum())
+
+    for name, arr in (("q", q), ("k", k), ("v", v), ("A", A)):
+        d = rng.standard_normal(arr.shape)
+        args = dict(qq=q, kk=k, vv=v, AA=A)
+        key = {"q": "qq", "k": "kk", "v": "vv", "A": "AA"}[name]
+        plus, minus = dict(args), dict(args)
+        plus[key], minus[key] = arr + h * d, arr - h * d
+        fd = (f(**plus) - f(**minus)) / (2 * h)
+        an = float((g["d" + name] * d).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_backward_dense_sparse_branch_matches_sdpa(oracle_mod):
+    """keep = 1, sparse branch only: the gradients equal torch's fp64 scaled-dot-product-attention
+    backward on the rotated q, k, rotated back to the raw inputs (R(p)^T)."""
+    import torch
+    from oracle import backward as B
+    w, q, k, v, A, dout = _bw_case(oracle_mod, keep_frac=1.0)
+    grid = (w.T, w.H, w.W)
+    g = B.head_backward(q, k, v, A, dout, grid, w.block, 1.0, w.rank, branches=1)
+    qh = torch.tensor(oracle_mod.rope_rows(q, grid, w.head_dim // 2), requires_grad=True)
+    kh = torch.tensor(oracle_mod.rope_rows(k, grid, w.head_dim // 2), requires_grad=True)
+    vv = torch.tensor(v, requires_grad=True)
+    o = torch.nn.functional.scaled_dot_product_attention(qh[None, None], kh[None, None], vv[None, None])[0, 0]
+    dqh, dkh, dv = torch.autograd.grad(o, (qh, kh, vv), torch.from_numpy(dout))
+    cs = B.rope_cos_sin(grid, w.head_dim)
+
+    def unrotate(y):  # R(p)^T y: rotate each pair by the negative angle
+        y = y.numpy()
+        x = y.copy()
+        c, s = cs[:, :, 0], cs[:, :, 1]
+        x[:, 0::2] = y[:, 0::2] * c + y[:, 1::2] * s
+        x[:, 1::2] = -y[:, 0::2] * s + y[:, 1::2] * c
+        return x
+
+    assert np.allclose(g["dq"], unrotate(dqh), rtol=1e-10, atol=1e-12)
+    assert np.allclose(g["dk"], unrotate(dkh), rtol=1e-10, atol=1e-12)
+    assert np.allclose(g["dv"], dv.numpy(), rtol=1e-10, atol=1e-12)
+    assert not g["dA"].any()
