@@ -65,9 +65,9 @@ struct AttnLayout {
 // mbarrier indices
 enum : int {
     kBarQ = 0,
-    kBarKFull = 1,    // +slot
+    kBarKFull = 1,    // +slot: k_0, k_1 landed (the first two S)
     kBarKEmpty = 3,   // +slot: S that read the slot has completed
-    kBarVFull = 5,    // +slot
+    kBarVFull = 5,    // +slot: v_j and, when there is one, k_{j+2} landed (block j's two products)
     kBarVEmpty = 7,   // +slot: P.V that read the slot has completed
     kBarSFull = 9,    // +buffer: S_j in TMEM
     kBarPFull = 12,   // +buffer: P_j in TMEM (one arrival per softmax thread)
@@ -254,22 +254,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 load_tile(bars + kBarKFull + 1, kslot(1), &tm_k, row0 + __ldg(my_idx + 1) * blk, blk);
                 nk = 2;
             }
+            // Block j's products read v_j (P.V_j) and k_{j+2} (S_{j+2}): both copies land on one
+            // barrier per slot, so the MMA warp checks one barrier for them instead of two.  v_j's
+            // bytes are registered without an arrival; the arrival comes with k_{j+2}'s bytes, or
+            // alone when there is no k_{j+2}.
+            auto add_tile = [&](uint64_t* bar, uint8_t* dst, const CUtensorMap* tm, int row, int rows, bool arrive) {
+                if (arrive) mbar_expect_tx(bar, static_cast<uint32_t>(rows) * D * 2);
+                else mbar_add_tx(bar, static_cast<uint32_t>(rows) * D * 2);
+#pragma unroll
+                for (int sl = 0; sl < D / 64; ++sl) tma_load_2d(dst + sl * (rows * 128), tm, bar, sl * 64, row);
+            };
             for (int j = 0; j < keep && ok; ++j) {
                 const int s = j & 1;
+                const bool has_k = j + 2 < keep;
                 // v_j into slot s once P.V_{j-2} (the slot's previous reader) has completed
                 if (j >= 2 && !mbar_wait(bars + kBarVEmpty + s, ((j - 2) >> 1) & 1, tmo, abort_flag)) {
                     ok = false;
                     break;
                 }
-                load_tile(bars + kBarVFull + s, vslot(s), &tm_v, row0 + __ldg(my_idx + j) * blk, blk);
+                add_tile(bars + kBarVFull + s, vslot(s), &tm_v, row0 + __ldg(my_idx + j) * blk, blk, !has_k);
                 ++nv;
                 // k_{j+2} into slot s once S_j has completed
-                if (j + 2 < keep) {
+                if (has_k) {
                     if (!mbar_wait(bars + kBarKEmpty + s, (j >> 1) & 1, tmo, abort_flag)) {
+                        mbar_arrive(bars + kBarVFull + s);  // complete the phase v_j's bytes are on
                         ok = false;
                         break;
                     }
-                    load_tile(bars + kBarKFull + s, kslot(s), &tm_k, row0 + __ldg(my_idx + j + 2) * blk, blk);
+                    add_tile(bars + kBarVFull + s, kslot(s), &tm_k, row0 + __ldg(my_idx + j + 2) * blk, blk, true);
                     ++nk;
                 }
             }
@@ -279,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 volatile int no_abort = 0;
                 const uint64_t drain = 10000000ull;
                 mbar_wait(bar_q, 0, drain, &no_abort);
-                for (int n = nk - 2 < 0 ? 0 : nk - 2; n < nk; ++n)
-                    mbar_wait(bars + kBarKFull + (n & 1), (n >> 1) & 1, drain, &no_abort);
+                for (int n = 0; n < (nk < 2 ? nk : 2); ++n)  // k_0, k_1 (later k tiles ride with the v tiles)
+                    mbar_wait(bars + kBarKFull + n, 0, drain, &no_abort);
                 for (int n = nv - 2 < 0 ? 0 : nv - 2; n < nv; ++n)
                     mbar_wait(bars + kBarVFull + (n & 1), (n >> 1) & 1, drain, &no_abort);
             }
@@ -335,8 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // from this thread: products run in order)
                 const bool has_s = j + 2 < keep;
                 if (!mbar_wait(bars + kBarPFull + j % kNumS, (j / kNumS) & 1, tmo, abort_flag) ||
-                    !mbar_wait(bars + kBarVFull + (j & 1), (j >> 1) & 1, tmo, abort_flag) ||
-                    (has_s && !mbar_wait(bars + kBarKFull + (j & 1), ((j + 2) >> 1) & 1, tmo, abort_flag))) {
+                    !mbar_wait(bars + kBarVFull + (j & 1), (j >> 1) & 1, tmo, abort_flag)) {  // v_j, k_{j+2}
                     ok = false;
                     break;
                 }
