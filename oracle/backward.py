@@ -18,6 +18,10 @@ attention plus the low-rank branch, "4.2"/"4.3" rank-truncated RoPE outside the 
   S      = sum_j psi(k_j) v_j^T,  z = sum_j phi(k_j)
   O_lr   = psi(q) S / (phi(q) . z + 1e-6)
   out    = O_s + O_lr
+The options of the forward are restated too: the feature map (relu, SiLU, identity, tanh), the
+low-rank RoPE outside the activation, absent or inside it (psi = act(R x A), normaliser on psi), a
+separate key projection, and the gated fusion of the two outputs.
+
 The cos/sin of every (token, pair) come from the C oracle's rotation of unit vectors, so both
 restatements use the same tables; `tests/test_oracle_pins.py` pins this forward to the C oracle's and
 its gradients to finite differences and to torch's dense attention backward.
@@ -29,7 +33,7 @@ import math
 import numpy as np
 import torch
 
-from . import block_means, block_scores, keep_count, rope_rows, topk
+from . import ACT_IDENTITY, ACT_RELU, ACT_SILU, block_means, block_scores, keep_count, rope_rows, topk
 
 
 def rope_cos_sin(grid, D: int, theta: float = 1e4, offset=(0, 0, 0), split=None) -> np.ndarray:
@@ -63,27 +67,57 @@ def block_mask(idx: np.ndarray, L: int, block: int) -> torch.Tensor:
     return torch.from_numpy(kept[bl][:, bl])
 
 
-def forward_torch(q, k, v, A, cs, mask, rank: int, branches: int = 3) -> torch.Tensor:
-    """The forward of one head in differentiable fp64 torch (see the module docstring)."""
+def _act(u: torch.Tensor, act: int) -> torch.Tensor:
+    if act == ACT_RELU:
+        return torch.relu(u)
+    if act == ACT_SILU:
+        return u / (1.0 + torch.exp(-u))
+    if act == ACT_IDENTITY:
+        return u
+    return torch.tanh(u)
+
+
+def forward_torch(q, k, v, A, cs, mask, rank: int, branches: int = 3, *, activation: int = ACT_RELU,
+                  rope: str = "outside", A_k=None, gate=None) -> torch.Tensor:
+    """The forward of one head in differentiable fp64 torch (see the module docstring).  rope is
+    "outside", "none" or "inside"; A_k a separate key projection; gate = (w, b) tensors."""
     L, D = q.shape
-    out = torch.zeros_like(v)
+    o_s = torch.zeros_like(v)
     if branches & 1:
         qh, kh = _rotate(q, cs, D // 2), _rotate(k, cs, D // 2)
         s = (qh @ kh.T) / math.sqrt(D)
         s = s.masked_fill(~mask, float("-inf"))
-        out = out + torch.softmax(s, dim=1) @ v
-    if branches & 2:
-        phq, phk = torch.relu(q @ A), torch.relu(k @ A)
-        psq, psk = _rotate(phq, cs, rank // 2), _rotate(phk, cs, rank // 2)
-        S, z = psk.T @ v, phk.sum(0)
-        out = out + (psq @ S) / (phq @ z + 1e-6)[:, None]
-    return out
+        o_s = torch.softmax(s, dim=1) @ v
+    if not branches & 2:
+        return o_s
+    Ak = A if A_k is None else A_k
+    if rope == "inside":
+        psq = _act(_rotate(q @ A, cs, rank // 2), activation)
+        psk = _act(_rotate(k @ Ak, cs, rank // 2), activation)
+        phq, phk = psq, psk
+    else:
+        phq, phk = _act(q @ A, activation), _act(k @ Ak, activation)
+        if rope == "outside":
+            psq, psk = _rotate(phq, cs, rank // 2), _rotate(phk, cs, rank // 2)
+        else:
+            psq, psk = phq, phk
+    S, z = psk.T @ v, phk.sum(0)
+    o_lr = (psq @ S) / (phq @ z + 1e-6)[:, None]
+    if gate is None:
+        return o_s + o_lr
+    w, b = gate
+    g = torch.sigmoid(q @ w + b)[:, None]
+    rms_s = torch.sqrt((o_s * o_s).mean(1, keepdim=True))
+    rms_l = torch.sqrt((o_lr * o_lr).mean(1, keepdim=True) + 1e-6)
+    return o_s + g * o_lr * rms_s / rms_l
 
 
 def head_backward(q, k, v, A, dout, grid, block: int, keep_frac: float, rank: int, *, theta=1e4,
-                  offset=(0, 0, 0), split=None, branches: int = 3, idx=None):
-    """Gradients of sum(dout * out) with respect to q, k, v [L, D] and A [D, R] (all fp64 numpy), the
-    block selection held at the forward's (or `idx`).  Returns dict(dq, dk, dv, dA, out, idx)."""
+                  offset=(0, 0, 0), split=None, branches: int = 3, idx=None, activation: int = ACT_RELU,
+                  rope: str = "outside", A_k=None, gate=None):
+    """Gradients of sum(dout * out) with respect to q, k, v [L, D], A [D, R] and (when given) the key
+    projection A_k and the gate weights and bias (all fp64 numpy), the block selection held at the
+    forward's (or `idx`).  Returns dict(dq, dk, dv, dA, [dA_k], [dgate_w, dgate_b], out, idx)."""
     L, D = q.shape
     if idx is None:
         qh = rope_rows(q, grid, D // 2, theta, offset, split)
@@ -92,9 +126,25 @@ def head_backward(q, k, v, A, dout, grid, block: int, keep_frac: float, rank: in
         idx, _ = topk(s, keep_count(keep_frac, s.shape[0]))
     cs = torch.from_numpy(rope_cos_sin(grid, D, theta, offset, split))
     mask = block_mask(np.asarray(idx), L, block)
-    tq, tk, tv, tA = (torch.tensor(np.asarray(a, dtype=np.float64), requires_grad=True) for a in (q, k, v, A))
-    out = forward_torch(tq, tk, tv, tA, cs, mask, rank, branches)
-    dq, dk, dv, dA = torch.autograd.grad(out, (tq, tk, tv, tA), torch.from_numpy(np.asarray(dout, dtype=np.float64)),
-                                         allow_unused=True)
+    leaf = lambda a: torch.tensor(np.asarray(a, dtype=np.float64), requires_grad=True)
+    tq, tk, tv, tA = (leaf(a) for a in (q, k, v, A))
+    extra, names = [], []
+    tAk = None
+    if A_k is not None:
+        tAk = leaf(A_k)
+        extra.append(tAk)
+        names.append("dA_k")
+    tgate = None
+    if gate is not None:
+        tgate = (leaf(gate[0]), leaf(float(gate[1])))
+        extra += list(tgate)
+        names += ["dgate_w", "dgate_b"]
+    out = forward_torch(tq, tk, tv, tA, cs, mask, rank, branches, activation=activation, rope=rope, A_k=tAk,
+                        gate=tgate)
+    grads = torch.autograd.grad(out, [tq, tk, tv, tA] + extra,
+                                torch.from_numpy(np.asarray(dout, dtype=np.float64)), allow_unused=True)
+    refs = [q, k, v, A] + [a.detach().numpy() for a in extra]
     z = lambda g, ref: np.zeros_like(np.asarray(ref, dtype=np.float64)) if g is None else g.numpy()
-    return dict(dq=z(dq, q), dk=z(dk, k), dv=z(dv, v), dA=z(dA, A), out=out.detach().numpy(), idx=np.asarray(idx))
+    res = dict(zip(["dq", "dk", "dv", "dA"] + names, (z(g, r) for g, r in zip(grads, refs))))
+    res.update(out=out.detach().numpy(), idx=np.asarray(idx))
+    return res

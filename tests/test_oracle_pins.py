@@ -641,3 +641,60 @@ def test_backward_dense_sparse_branch_matches_sdpa(oracle_mod):
     assert np.allclose(g["dk"], unrotate(dkh), rtol=1e-10, atol=1e-12)
     assert np.allclose(g["dv"], dv.numpy(), rtol=1e-10, atol=1e-12)
     assert not g["dA"].any()
+
+
+_BW_OPTIONS = [
+    dict(activation=1, rope="inside", separate=True, gate=True),    # SiLU, RoPE inside, Pq != Pk, gated
+    dict(activation=2, rope="none", separate=False, gate=False),    # identity map, no low-rank RoPE
+    dict(activation=3, rope="outside", separate=True, gate=True),   # tanh, Pq != Pk, gated
+]
+
+
+def _bw_options_case(oracle_mod, opt):
+    w, q, k, v, A, dout = _bw_case(oracle_mod)
+    q, k, A = np.abs(q), np.abs(k), np.abs(A)   # non-negative features keep the normaliser conditioned
+    rng = np.random.default_rng(21)
+    Ak = np.abs(rng.standard_normal(A.shape)) / 8 if opt["separate"] else None
+    gate = (rng.standard_normal(w.head_dim) / 8, -0.5) if opt["gate"] else None
+    fwd = dict(activation=opt["activation"], lowrank_rope=opt["rope"] != "none", rope_inside=opt["rope"] == "inside",
+               A_k=Ak, gate=gate)
+    bwd = dict(activation=opt["activation"], rope=opt["rope"], A_k=Ak, gate=gate)
+    return w, q, k, v, A, dout, Ak, gate, fwd, bwd
+
+
+@pytest.mark.parametrize("opt", _BW_OPTIONS, ids=lambda o: f"act{o['activation']}-{o['rope']}-sep{o['separate']}-gate{o['gate']}")
+def test_backward_options_restatement_and_finite_differences(oracle_mod, opt):
+    """With the forward's options (feature map, RoPE ordering, separate key projection, gated fusion)
+    the torch restatement reproduces the C oracle's forward, and its gradients -- including those of
+    the key projection and of the gate's weights and bias -- match central differences of the C
+    forward."""
+    from oracle import backward as B
+    w, q, k, v, A, dout, Ak, gate, fwd, bwd = _bw_options_case(oracle_mod, opt)
+    grid = (w.T, w.H, w.W)
+    g = B.head_backward(q, k, v, A, dout, grid, w.block, w.keep_frac, w.rank, **bwd)
+    r = oracle_mod.head_forward(q, k, v, A, grid, w.block, w.keep_frac, w.rank, **fwd)
+    assert np.allclose(g["out"], r["out"], rtol=1e-11, atol=1e-12)
+
+    def f(qq=q, kk=k, vv=v, AA=A, AAk=Ak, gw=None, gb=None):
+        kw = dict(fwd)
+        kw["A_k"] = AAk
+        if gate is not None:
+            kw["gate"] = (gate[0] if gw is None else gw, gate[1] if gb is None else gb)
+        rr = oracle_mod.head_forward(qq, kk, vv, AA, grid, w.block, w.keep_frac, w.rank, idx_override=g["idx"], **kw)
+        return float((dout * rr["out"]).sum())
+
+    rng = np.random.default_rng(5)
+    h = 1e-6
+    cases = [("dq", "qq", q), ("dk", "kk", k), ("dv", "vv", v), ("dA", "AA", A)]
+    if Ak is not None:
+        cases.append(("dA_k", "AAk", Ak))
+    if gate is not None:
+        cases.append(("dgate_w", "gw", gate[0]))
+    for name, key, arr in cases:
+        d = rng.standard_normal(np.shape(arr))
+        fd = (f(**{key: arr + h * d}) - f(**{key: arr - h * d})) / (2 * h)
+        an = float((g[name] * d).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+    if gate is not None:
+        fd = (f(gb=gate[1] + h) - f(gb=gate[1] - h)) / (2 * h)
+        assert abs(fd - float(g["dgate_b"])) <= 1e-6 * max(1.0, abs(fd)), ("dgate_b", fd, float(g["dgate_b"]))
