@@ -33,9 +33,11 @@
  *                 pages print no formula, this is the library's reading of their description)
  *
  * Conventions for every entry point:
- *   - Device pointers unless stated otherwise.  The caller owns every buffer; nothing is retained
- *     after a call returns.  Calls are asynchronous on `stream` (NULL = the legacy default stream)
- *     and never synchronize, except slra_device_status and slra_attn_fwd_host.
+ *   - Device pointers unless stated otherwise.  The caller owns every buffer; nothing the caller
+ *     passes is retained after a call returns (the library itself keeps, per device, the two copy
+ *     streams and a few events slra_attn_fwd_host creates on first use, and the fixed scratch array
+ *     of slra_lowrank_summary_noalloc).  Calls are asynchronous on `stream` (NULL = the legacy default
+ *     stream) and never synchronize, except slra_device_status and slra_attn_fwd_host.
  *   - All arguments are validated before anything is launched; an invalid call returns a status and
  *     launches nothing.  Launch failures return SLRA_ERR_CUDA.
  *   - Problems detected on the device (an input too large for the fp16 operands, a bounded wait that
