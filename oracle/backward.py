@@ -148,3 +148,77 @@ def head_backward(q, k, v, A, dout, grid, block: int, keep_frac: float, rank: in
     res = dict(zip(["dq", "dk", "dv", "dA"] + names, (z(g, r) for g, r in zip(grads, refs))))
     res.update(out=out.detach().numpy(), idx=np.asarray(idx))
     return res
+
+
+def _unrotate(y: np.ndarray, cs: np.ndarray, npairs: int) -> np.ndarray:
+    """R(p)^T y: rotate pairs (2j, 2j+1), j < npairs, back by their angles."""
+    x = y.copy()
+    c, s = cs[:, :npairs, 0], cs[:, :npairs, 1]
+    y0, y1 = y[:, 0:2 * npairs:2], y[:, 1:2 * npairs:2]
+    x[:, 0:2 * npairs:2] = y0 * c + y1 * s
+    x[:, 1:2 * npairs:2] = -y0 * s + y1 * c
+    return x
+
+
+def _rot_np(x: np.ndarray, cs: np.ndarray, npairs: int) -> np.ndarray:
+    y = x.copy()
+    c, s = cs[:, :npairs, 0], cs[:, :npairs, 1]
+    x0, x1 = x[:, 0:2 * npairs:2], x[:, 1:2 * npairs:2]
+    y[:, 0:2 * npairs:2] = x0 * c - x1 * s
+    y[:, 1:2 * npairs:2] = x0 * s + x1 * c
+    return y
+
+
+def head_backward_steps(q, k, v, A, dout, grid, block: int, rank: int, idx, *, theta=1e4, offset=(0, 0, 0),
+                        split=None):
+    """The same gradients as head_backward (relu features, RoPE outside, one shared projection, plain
+    sum), written as the explicit steps a kernel takes, in fp64 numpy:
+
+    sparse branch (per query row i over its allowed keys j):
+      s_ij = q^_i . k^_j / sqrt(D),  lse_i = log sum_j exp(s_ij),  P_ij = exp(s_ij - lse_i)
+      Delta_i = dO_i . O_s,i,  dP_ij = dO_i . v_j,  dS_ij = P_ij (dP_ij - Delta_i)
+      dq^_i = sum_j dS_ij k^_j / sqrt(D),  dk^_j = sum_i dS_ij q^_i / sqrt(D),  dv_j += sum_i P_ij dO_i
+      dq += R(p_i)^T dq^_i,  dk += R(p_j)^T dk^_j
+    low-rank branch (u = x A, phi = relu(u), psi = R_r phi, den_i = phi_q,i . z + 1e-6):
+      dpsi_q,i = S dO_i / den_i,  dden_i = -(dO_i . O_lr,i) / den_i,  dphi_q,i = R_r^T dpsi_q,i + dden_i z
+      dS = sum_i psi_q,i dO_i^T / den_i,  dz = sum_i dden_i phi_q,i
+      dpsi_k,j = dS v_j,  dv_j += dS^T psi_k,j,  dphi_k,j = R_r^T dpsi_k,j + dz
+      du = dphi * [u > 0],  dq += du_q A^T,  dk += du_k A^T,  dA = q^T du_q + k^T du_k
+    Returns dict(dq, dk, dv, dA)."""
+    q, k, v, A, dout = (np.asarray(a, dtype=np.float64) for a in (q, k, v, A, dout))
+    L, D = q.shape
+    cs = rope_cos_sin(grid, D, theta, offset, split)
+    mask = block_mask(np.asarray(idx), L, block).numpy()
+    # sparse branch
+    qh, kh = _rot_np(q, cs, D // 2), _rot_np(k, cs, D // 2)
+    s = np.where(mask, qh @ kh.T / math.sqrt(D), -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    lse = m + np.log(np.exp(s - m).sum(axis=1, keepdims=True))
+    P = np.exp(s - lse)
+    o_s = P @ v
+    delta = (dout * o_s).sum(axis=1, keepdims=True)
+    dS = P * (dout @ v.T - delta)
+    dqh, dkh = dS @ kh / math.sqrt(D), dS.T @ qh / math.sqrt(D)
+    dv = P.T @ dout
+    dq, dk = _unrotate(dqh, cs, D // 2), _unrotate(dkh, cs, D // 2)
+    # low-rank branch
+    r2 = rank // 2
+    uq, uk = q @ A, k @ A
+    phq, phk = np.maximum(uq, 0.0), np.maximum(uk, 0.0)
+    psq, psk = _rot_np(phq, cs, r2), _rot_np(phk, cs, r2)
+    Sm, z = psk.T @ v, phk.sum(axis=0)
+    den = phq @ z + 1e-6
+    o_lr = (psq @ Sm) / den[:, None]
+    dpsq = (dout @ Sm.T) / den[:, None]
+    dden = -(dout * o_lr).sum(axis=1) / den
+    dphq = _unrotate(dpsq, cs, r2) + dden[:, None] * z[None, :]
+    dSm = psq.T @ (dout / den[:, None])
+    dz = dden @ phq
+    dpsk = v @ dSm.T
+    dv = dv + psk @ dSm
+    dphk = _unrotate(dpsk, cs, r2) + dz[None, :]
+    duq, duk = dphq * (uq > 0), dphk * (uk > 0)
+    dq = dq + duq @ A.T
+    dk = dk + duk @ A.T
+    dA = q.T @ duq + k.T @ duk
+    return dict(dq=dq, dk=dk, dv=dv, dA=dA)

@@ -698,3 +698,17 @@ def test_backward_options_restatement_and_finite_differences(oracle_mod, opt):
     if gate is not None:
         fd = (f(gb=gate[1] + h) - f(gb=gate[1] - h)) / (2 * h)
         assert abs(fd - float(g["dgate_b"])) <= 1e-6 * max(1.0, abs(fd)), ("dgate_b", fd, float(g["dgate_b"]))
+
+
+def test_backward_steps_match_autograd(oracle_mod):
+    """The explicit gradient steps (flash-style sparse backward with lse and Delta; the low-rank chain
+    through the summary, the normaliser, R_r^T, the relu mask and A^T) give autograd's gradients: the
+    derivation the GPU backward is to follow."""
+    from oracle import backward as B
+    for keep in (0.5, 1.0):
+        w, q, k, v, A, dout = _bw_case(oracle_mod, keep_frac=keep)
+        grid = (w.T, w.H, w.W)
+        g = B.head_backward(q, k, v, A, dout, grid, w.block, keep, w.rank)
+        m = B.head_backward_steps(q, k, v, A, dout, grid, w.block, w.rank, g["idx"])
+        for name in ("dq", "dk", "dv", "dA"):
+            assert np.allclose(m[name], g[name], rtol=1e-10, atol=1e-12), name
