@@ -23,6 +23,75 @@ def _rows(path):
         return [l.split() for l in f if l.strip() and not l.startswith("#")]
 
 
+# ------------------------------------------------------------------------------------ bf16 inputs
+def _bf16_golden():
+    """(bits, value) pairs of tests/golden/bf16_decode.txt (written by hand from the bf16 format)."""
+    bits, vals = [], []
+    for h, v in _rows(os.path.join(GOLD, "bf16_decode.txt")):
+        bits.append(int(h, 16))
+        vals.append(-0.0 if v == "neg0" else float(v))
+    return np.array(bits, dtype=np.uint16), np.array(vals, dtype=np.float64)
+
+
+def _same_values(a, b):
+    """Equal as IEEE values, including the sign of zero and NaN in the same places."""
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    nan = np.isnan(a)
+    return bool(np.array_equal(nan, np.isnan(b)) and np.array_equal(a[~nan], b[~nan]) and
+                np.array_equal(np.signbit(a[~nan]), np.signbit(b[~nan])))
+
+
+def _bf16_by_fields(bits):
+    """The bf16 definition written out: sign, 8-bit exponent (bias 127), 7-bit fraction, subnormals,
+    infinities and NaN (independent of any reinterpretation of memory)."""
+    out = []
+    for b in np.asarray(bits, dtype=np.uint16).ravel().tolist():
+        s, e, f = b >> 15, (b >> 7) & 0xFF, b & 0x7F
+        if e == 0xFF:
+            x = math.nan if f else math.inf
+        elif e == 0:
+            x = math.ldexp(f / 128.0, -126)
+        else:
+            x = math.ldexp(1.0 + f / 128.0, e - 127)
+        out.append(-x if s else x)
+    return np.array(out, dtype=np.float64).reshape(np.shape(bits))
+
+
+def test_decode_bf16_golden_table(oracle_mod):
+    """orc_decode_bf16 (the entry of every bf16 input into the oracle) returns the exact value of each
+    pattern of a hand-written table: signed zeros, +-1, powers of two, the largest finite value, the
+    smallest normal, subnormals, infinities and NaN."""
+    bits, vals = _bf16_golden()
+    assert _same_values(oracle_mod.decode_bf16(bits), vals)
+    assert _same_values(_bf16_by_fields(bits), vals)
+
+
+def test_decode_bf16_all_patterns_and_generator_bits(oracle_mod):
+    """All 65,536 patterns against the field-by-field definition and against torch's own bf16 -> fp64
+    conversion; then the seeded generator's actual q, k, v and A bits against numpy's reinterpretation
+    of the pattern as the upper half of an fp32."""
+    torch = pytest.importorskip("torch")
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle_mod.decode_bf16(allb)
+    assert _same_values(got, _bf16_by_fields(allb))
+    assert _same_values(got, torch.from_numpy(allb.view(np.int16)).view(torch.bfloat16).double().numpy())
+    x = I.make_inputs(W.TINY)
+    for n in ("q", "k", "v", "A"):
+        ref = (x[n].astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+        assert _same_values(oracle_mod.decode_bf16(x[n]), ref), n
+
+
+def test_decode_bf16_pins_reject_planted_mistakes(oracle_mod):
+    """Plausible decoder mistakes, planted in CPU decoders written here, fail the golden table:
+    shifting by 15 instead of 16, dropping the sign bit, and reading the pattern as fp16."""
+    bits, vals = _bf16_golden()
+    shift15 = (bits.astype(np.uint32) << np.uint32(15)).view(np.float32).astype(np.float64)
+    unsigned = oracle_mod.decode_bf16(bits & np.uint16(0x7FFF))
+    as_fp16 = bits.view(np.float16).astype(np.float64)
+    for bad in (shift15, unsigned, as_fp16):
+        assert not _same_values(bad, vals)
+
+
 # ----------------------------------------------------------------------------------------- RoPE
 def test_rope_split_golden(oracle_mod):
     """Pairs per axis match the Wan 44/42/42 split (D=128) and the same rule at D=64."""
