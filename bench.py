@@ -231,6 +231,92 @@ def run_reference(args, w, rank, world):
 
 
 # ---------------------------------------------------------------------------------- GPU arm
+def _problem(args, w, slra, dev, torch, stage_ev):
+    """The run's problem description and its seeded inputs on the device."""
+    x = make_run_inputs(args, w)
+    q, k, v = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v"))
+    var = variant_of(args, w)
+    gate_kw = {}
+    if args.fusion == "gated":
+        gate_kw = dict(fusion=slra.FUSION_GATED, gate_bias=GATE_BIAS,
+                       gate_w=torch.from_numpy(gate_weights(w)).to(dev))
+    prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev),
+                                      branches=BRANCHES[args.branches], activation=var["activation"],
+                                      lowrank_norope=int(not var["lowrank_rope"]),
+                                      proj_separate=int(var["proj_separate"]), proj_per_head=int(var["proj_per_head"]),
+                                      lowrank_rope_inside=int(args.rope_inside), **gate_kw)
+    A = torch.from_numpy(x["A"].view(np.int16)).view(torch.bfloat16).to(dev).reshape(prob.projection_shape)
+    return x, var, prob, (q, k, v, A)
+
+
+def _work(w, prob, ws, slra, br):
+    """Algorithmic FLOPs of one call, counted exactly from the selected masks: (total, sparse kept,
+    low-rank, scores, attention kernel's own = kept + the fused readout's q A and psi S, keep)."""
+    BH = w.batch * w.heads
+    if br & 1:
+        idx = slra.ws_view(prob, ws, "idx").cpu().numpy()
+        f_sparse = F.sparse_flops(idx, w.L, w.block, w.head_dim)
+        f_sc = F.score_flops(w.nb, w.head_dim, BH)
+        keep_blocks = int(idx.shape[-1])
+    else:
+        f_sparse = f_sc = 0.0
+        keep_blocks = 0
+    f_lr = F.lowrank_flops(w.L, w.rank, w.head_dim, BH) if br & 2 else 0.0
+    f_attn = f_sparse + (4.0 * w.L * w.rank * w.head_dim * BH if br & 2 else 0.0)
+    return f_sparse + f_lr + f_sc, f_sparse, f_lr, f_sc, f_attn, keep_blocks
+
+
+STAGES = ("rope_table", "rope_pool", "select", "lowrank_partial", "lowrank_reduce", "attention")
+
+
+def _timed_calls(slra, torch, prob, tensors, out, ws, stage_ev, steps, warmup, flush, stream, barrier=lambda: None):
+    """Warm up, then time `steps` calls with CUDA events on the launching stream, the L2 flushed before
+    each.  Returns (per-call ms list, per-stage ms lists)."""
+    q, k, v, A = tensors
+    for _ in range(max(3, warmup)):
+        slra.attn_fwd(prob, q, k, v, A, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    status = slra.device_status(ws)
+    if status != slra.OK:
+        raise RuntimeError(f"device status after warm-up: {slra.status_string(status)}")
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    stage_ms = []
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        step_ev[i][0].record(stream)
+        slra.attn_fwd(prob, q, k, v, A, out=out, workspace=ws)
+        step_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        stage_ms.append([stage_ev[j].elapsed_time(stage_ev[j + 1]) for j in range(6)])
+    barrier()
+    torch.cuda.synchronize()
+    status = slra.device_status(ws)
+    if status != slra.OK:
+        raise RuntimeError(f"device status after timing: {slra.status_string(status)}")
+    return [a.elapsed_time(b) for a, b in step_ev], stage_ms
+
+
+def _rooflines(w, f_sparse, f_attn, attn_ms, ms_per_step):
+    """The attention kernel's roofline (its algorithmic FLOPs per launch / its event time, against the
+    measured burst bf16 peak: the kernel is timed alone inside a step of a few ms) and the whole call's
+    (max(kept FLOPs / tensor peak, minimum bytes / HBM bandwidth) against ms per call)."""
+    hbm, tf_burst, tf_sust, src = peaks()
+    achieved = f_attn / (attn_ms * 1e-3) / 1e12
+    bytes_min = F.io_bytes(w.batch, w.L, w.heads, w.head_dim, w.rank, 4)
+    t_roof = max(f_sparse / (tf_burst * 1e12), bytes_min / (hbm * 1e9))
+    t_roof_sust = max(f_sparse / (tf_sust * 1e12), bytes_min / (hbm * 1e9))
+    roof = {"kernel": "attn_sm100_kernel", "bound": "tensor", "achieved": achieved, "peak": tf_burst,
+            "unit": "TFLOP/s", "frac": achieved / tf_burst,
+            "peak_source": f"{src} burst bf16 (same rate as f16)", "attn_ms": attn_ms,
+            "peak_sustained": tf_sust, "frac_of_sustained": achieved / tf_sust}
+    call = {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_per_step,
+            "frac_of_sustained": t_roof_sust * 1e3 / ms_per_step,
+            "note": "max(kept FLOPs / burst tensor peak, min bytes / HBM peak) vs ms_per_step"}
+    return roof, call
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -245,23 +331,12 @@ def run_ours(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     base_w = w
     w = replicas.replica_workload(base_w, rank)  # each rank: its own independent problem
-    x = make_run_inputs(args, w)
-    q, k, v = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v"))
     stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
     for e in stage_ev:
         e.record()
     torch.cuda.synchronize()
-    var = variant_of(args, w)
+    x, var, prob, tensors = _problem(args, w, slra, dev, torch, stage_ev)
     br = BRANCHES[args.branches]
-    gate_kw = {}
-    if args.fusion == "gated":
-        gate_kw = dict(fusion=slra.FUSION_GATED, gate_bias=GATE_BIAS,
-                       gate_w=torch.from_numpy(gate_weights(w)).to(dev))
-    prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in stage_ev), branches=br,
-                                      activation=var["activation"], lowrank_norope=int(not var["lowrank_rope"]),
-                                      proj_separate=int(var["proj_separate"]), proj_per_head=int(var["proj_per_head"]),
-                                      lowrank_rope_inside=int(args.rope_inside), **gate_kw)
-    A = torch.from_numpy(x["A"].view(np.int16)).view(torch.bfloat16).to(dev).reshape(prob.projection_shape)
     ws = slra.alloc_workspace(prob, dev)
     out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
@@ -271,51 +346,21 @@ def run_ours(args, w, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    for _ in range(max(3, args.warmup)):
-        slra.attn_fwd(prob, q, k, v, A, out=out, workspace=ws)
+    q, k, v, A = tensors
+    slra.attn_fwd(prob, q, k, v, A, out=out, workspace=ws)
     torch.cuda.synchronize()
-    status = slra.device_status(ws)
-    if status != slra.OK:
-        raise RuntimeError(f"device status after warm-up: {slra.status_string(status)}")
-    BH = w.batch * w.heads
-    if br & 1:
-        idx = slra.ws_view(prob, ws, "idx").cpu().numpy()
-        f_sparse = F.sparse_flops(idx, w.L, w.block, w.head_dim)
-        f_sc = F.score_flops(w.nb, w.head_dim, BH)
-        keep_blocks = int(idx.shape[-1])
-    else:
-        f_sparse = f_sc = 0.0
-        keep_blocks = 0
-    f_lr = F.lowrank_flops(w.L, w.rank, w.head_dim, BH) if br & 2 else 0.0
-    f_total = f_sparse + f_lr + f_sc
-    # attention kernel's own algorithmic work: kept products + the fused readout (q A and psi S)
-    f_attn = f_sparse + (4.0 * w.L * w.rank * w.head_dim * BH if br & 2 else 0.0)
+    f_total, f_sparse, f_lr, f_sc, f_attn, keep_blocks = _work(w, prob, ws, slra, br)
 
-    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    stage_ms = []
     clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
-    barrier()
-    torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
-    for i in range(args.steps):
-        flush.zero_()
-        step_ev[i][0].record(stream)
-        slra.attn_fwd(prob, q, k, v, A, out=out, workspace=ws)
-        step_ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        stage_ms.append([stage_ev[i].elapsed_time(stage_ev[i + 1]) for i in range(6)])
-    barrier()
-    torch.cuda.synchronize()
+    step_ms, stage_ms = _timed_calls(slra, torch, prob, tensors, out, ws, stage_ev, args.steps, args.warmup, flush,
+                                     stream, barrier)
     clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in step_ev]
     tot_ms = replicas.max_over_ranks(sum(step_ms), dev)
     ms_per_step = tot_ms / args.steps
     job_flops = replicas.sum_over_ranks(f_total, dev)
-    status = slra.device_status(ws)
-    if status != slra.OK:
-        raise RuntimeError(f"device status after timing: {slra.status_string(status)}")
 
     # ---- end to end through the host entry point (pinned host buffers, copies inside the timing)
     host = {n: torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v", "A")}
@@ -337,13 +382,9 @@ def run_ours(args, w, rank, world, local_rank):
 
     if rank != 0:
         return
-    hbm, tf_burst, tf_sust, src = peaks()
     stage_avg = [statistics.mean(x[i] for x in stage_ms) for i in range(6)]
-    attn_avg = stage_avg[5]
-    achieved = f_attn / (attn_avg * 1e-3) / 1e12
-    traffic = load_traffic(w.name)
-    bytes_min = F.io_bytes(w.batch, w.L, w.heads, w.head_dim, w.rank, 4)
-    t_roof = max(f_sparse / (tf_sust * 1e12), bytes_min / (hbm * 1e9))
+    roof, call_roof = _rooflines(w, f_sparse, f_attn, stage_avg[5], ms_per_step)
+    roof["traffic"] = load_traffic(w.name)
     cpu_v, cpu_desc, cpu_threads, _ = oracle_sample(w, x, var)  # rank 0 runs the workload itself
     line = {
         "metric": METRIC, "value": replicas.job_throughput(job_flops, ms_per_step), "unit": "TFLOP/s",
@@ -358,21 +399,59 @@ def run_ours(args, w, rank, world, local_rank):
                    "branches": args.branches, "linear_baseline": bool(args.linear_baseline),
                    "projection": args.proj, "fusion": args.fusion, "rope_inside": bool(args.rope_inside)},
         "flops_per_step": {"sparse_kept": f_sparse, "lowrank": f_lr, "scores": f_sc},
-        "roofline": {"kernel": "attn_sm100_kernel", "bound": "tensor", "achieved": achieved, "peak": tf_sust,
-                     "unit": "TFLOP/s", "frac": achieved / tf_sust, "traffic": traffic,
-                     "peak_source": f"{src} sustained bf16 (same rate as f16)", "attn_ms": attn_avg},
-        "call_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_per_step,
-                          "note": "max(kept FLOPs / sustained tensor peak, min bytes / HBM peak) vs ms_per_step"},
+        "roofline": roof,
+        "call_roofline": call_roof,
         "e2e": {"value": replicas.job_throughput(job_flops, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "kernel_ms": dict(zip(("rope_table", "rope_pool", "select", "lowrank_partial", "lowrank_reduce",
-                               "attention"), (round(x, 4) for x in stage_avg))),
+        "kernel_ms": dict(zip(STAGES, (round(x, 4) for x in stage_avg))),
         "gpu_launches": 6 * args.steps,
         "clocks": clk,
         "cpu_baseline": {"value": cpu_v, "unit": "TFLOP/s", "cores": cpu_threads, "kind": "oracle",
                          "sample": cpu_desc},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_sweep(args):
+    """The keep x rank sweep at the Wan2.1-1.3B shape on one GPU: per point, ms per call, effective
+    TFLOP/s, the attention kernel's share of the call and its burst-peak roofline fraction, and the
+    call's roofline fraction.  One JSON line per point (not the benchmark contract line)."""
+    import torch
+    from sparse_rank_hybrid_b200 import build as B
+    from sparse_rank_hybrid_b200 import slra
+
+    B.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+    for e in stage_ev:
+        e.record()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0 if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                          int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[0]))
+    clocks.start()
+    for w in WL.sweep():
+        _, _, prob, tensors = _problem(args, w, slra, dev, torch, stage_ev)
+        ws = slra.alloc_workspace(prob, dev)
+        out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
+        q, k, v, A = tensors
+        slra.attn_fwd(prob, q, k, v, A, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        f_total, f_sparse, f_lr, f_sc, f_attn, keep_blocks = _work(w, prob, ws, slra, 3)
+        step_ms, stage_ms = _timed_calls(slra, torch, prob, tensors, out, ws, stage_ev, args.steps, args.warmup,
+                                         flush, stream)
+        ms = statistics.mean(step_ms)
+        stage_avg = [statistics.mean(x[i] for x in stage_ms) for i in range(6)]
+        roof, call_roof = _rooflines(w, f_sparse, f_attn, stage_avg[5], ms)
+        print(json.dumps({"sweep_point": w.name, "keep_frac": w.keep_frac, "keep_blocks": keep_blocks,
+                          "rank": w.rank, "ms_per_call": ms, "tflops": f_total / (ms * 1e-3) / 1e12,
+                          "attn_ms": stage_avg[5], "attn_share": stage_avg[5] / ms,
+                          "attn_frac_burst": roof["frac"], "call_frac_burst": call_roof["frac"],
+                          "kernel_ms": dict(zip(STAGES, (round(x, 4) for x in stage_avg)))}), flush=True)
+        del ws, out, tensors, q, k, v, A
+    print(json.dumps({"sweep_clocks": clocks.stop()}), flush=True)
 
 
 def load_traffic(workload: str):
@@ -406,6 +485,8 @@ def main():
                     help="query/key projection layout: one shared A, separate Pq/Pk, per head, or both")
     ap.add_argument("--fusion", default="sum", choices=["sum", "gated"],
                     help="combine the branches by their sum or by the token-wise gate (synthetic Wg, bg = -2)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the 20 keep x rank points at the Wan2.1-1.3B shape (one JSON line each)")
     ap.add_argument("--rope-inside", action="store_true",
                     help="low-rank RoPE before the activation (the ordering RoLA's ablation compares against)")
     args = ap.parse_args()
@@ -425,6 +506,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, w, rank, world)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
     if world > 1:
         import datetime

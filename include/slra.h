@@ -88,9 +88,10 @@ typedef enum slra_out_dtype { SLRA_OUT_F32 = 0, SLRA_OUT_BF16 = 1 } slra_out_dty
 enum { SLRA_BRANCH_SPARSE = 1, SLRA_BRANCH_LOWRANK = 2, SLRA_BRANCH_BOTH = 3 };
 
 /* Test hooks (slra_problem.debug_flags).  SLRA_DEBUG_UNSATISFIED_WAIT makes every CTA of the attention
- * kernel first wait on a barrier that nothing signals, so the bounded-wait path (timeout recorded in
- * the status word, the CTA returns without issuing work) can be exercised without faulting or hanging
- * the GPU.  Use a small wait_timeout_ns with it. */
+ * kernel and of the tensor-core low-rank summary kernel (head_dim 128) first wait on a barrier that
+ * nothing signals, so the bounded-wait path (timeout recorded in the status word, the CTA returns
+ * without issuing work) can be exercised without faulting or hanging the GPU.  Use a small
+ * wait_timeout_ns with it. */
 enum { SLRA_DEBUG_UNSATISFIED_WAIT = 1 };
 
 /* Nonlinearity of the low-rank feature map phi = act(x A) (slra_problem.activation).  RELU is the
@@ -295,14 +296,29 @@ SLRA_API slra_status slra_device_status(void* workspace, slra_stream_t stream, i
  * before anything is launched.  The call performs no cudaMalloc, cudaFree or other allocation.
  *
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current) and caches it; make that first call before any stream capture.  All calls
- * share the one array: every scratch byte a call reads it has first written itself, so nothing left
- * by an earlier call is used, but calls that overlap on the GPU (on different streams, or from
- * different host threads without ordering) race on the array and must be serialized by the caller.
+ * that device current) and caches it for the life of the process; make that first call before any
+ * stream capture, and do not keep using the entry point after a cudaDeviceReset of that device (the
+ * cached address would then be stale).  All calls share the one array, which keeps the last call's
+ * contents.  Each call first clears the array's status word (an asynchronous memset on `stream`);
+ * every other scratch byte a call reads it has first written itself, so nothing left by an earlier
+ * call is used.  Calls that overlap on the GPU (on different streams, or from different host threads
+ * without ordering) race on the array and must be serialized by the caller.
+ *
+ * Problems detected on the device (a bounded wait inside the summary kernel that ran out) are
+ * recorded in the array's status word: read them with slra_noalloc_device_status.  After a timeout
+ * S and z are unspecified.
  */
 #define SLRA_NOALLOC_SCRATCH_BYTES (16u << 20)
 SLRA_API slra_status slra_lowrank_summary_noalloc(const slra_problem* p, const void* k, const void* v,
                                                   const void* A, float* S, float* z, slra_stream_t stream);
+
+/*
+ * Device status of slra_lowrank_summary_noalloc on the current device: synchronize `stream`, then
+ * read and clear the status word of the fixed scratch array.  *status receives SLRA_OK or
+ * SLRA_ERR_DEVICE_TIMEOUT (the calls since the last no-allocation call began).  Allocates nothing.
+ * Like the entry point itself, this has no counterpart in the method's sources.
+ */
+SLRA_API slra_status slra_noalloc_device_status(slra_stream_t stream, int32_t* status);
 
 #ifdef __cplusplus
 }

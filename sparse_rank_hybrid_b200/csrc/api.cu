@@ -239,6 +239,8 @@ unsigned long long timeout_of(const slra_problem* p) {
     return p->wait_timeout_ns ? p->wait_timeout_ns : 2000000000ull;
 }
 
+int debug_wait_of(const slra_problem* p) { return (p->debug_flags & SLRA_DEBUG_UNSATISFIED_WAIT) ? 1 : 0; }
+
 
 // Tables + RoPE/pooling + selection.
 slra_status run_select(const slra_problem* p, const Derived& d, const Ptrs& w, const void* q, const void* k,
@@ -261,12 +263,13 @@ slra_status run_select(const slra_problem* p, const Derived& d, const Ptrs& w, c
 // whole projection argument; the kernels get the key projection(s).
 cudaError_t lowrank_partial(const Derived& d, const void* k, const void* v, const void* A, const double2* tab,
                             const int2* pairs, int nsplit, float* s_part, float* z_part, int* status,
-                            unsigned long long timeout_ns, cudaStream_t st) {
+                            unsigned long long timeout_ns, int debug_wait, cudaStream_t st) {
     const auto* kb = static_cast<const __nv_bfloat16*>(k);
     const auto* vb = static_cast<const __nv_bfloat16*>(v);
     const auto* Ab = static_cast<const __nv_bfloat16*>(A) + d.ak_off;  // the key projection(s)
     if (d.g.D == 128)
-        return launch_lowrank_tc(kb, vb, Ab, tab, d.meta, d.g, nsplit, s_part, z_part, status, timeout_ns, st);
+        return launch_lowrank_tc(kb, vb, Ab, tab, d.meta, d.g, nsplit, s_part, z_part, status, timeout_ns, debug_wait,
+                                 st);
     return launch_lowrank_partial(kb, vb, Ab, tab, pairs, d.g, nsplit, s_part, z_part, st);
 }
 
@@ -274,7 +277,7 @@ slra_status run_lowrank(const slra_problem* p, const Derived& d, const Ptrs& w, 
                         const void* A, cudaStream_t st) {
     const Geom& g = d.g;
     cudaError_t e = lowrank_partial(d, k, v, A, w.tab, w.pairs, d.nsplit, w.s_part, w.z_part, w.status,
-                                    timeout_of(p), st);
+                                    timeout_of(p), debug_wait_of(p), st);
     if (e != cudaSuccess) return SLRA_ERR_CUDA;
     slra_status s = mark(p, 4, st);
     if (s != SLRA_OK) return s;
@@ -690,14 +693,15 @@ slra_status slra_device_status(void* workspace, slra_stream_t stream, int32_t* s
 }  // extern "C"
 
 // ------------------------------------------------------------------------------------------------
-// Allocation-free low-rank summary.  Its scratch (rotary tables + split-L partial sums) is this
-// file-scope device array; host code must not pass the array's name to a kernel (on the host it is
-// only a stand-in), so its device address is looked up once per device and cached.
+// Allocation-free low-rank summary.  Its scratch (status word, rotary tables, split-L partial sums) is
+// this file-scope device array; host code must not pass the array's name to a kernel (on the host it
+// is only a stand-in), so its device address is looked up once per device and cached.
 namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SLRA_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
+constexpr size_t kNoallocStatusBytes = 256;  // the status word, at the start of the scratch
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
@@ -721,12 +725,9 @@ slra_status scratch_address(void** out) {
     return SLRA_OK;
 }
 
-// A status word for the kernels' bounded waits, placed after the partial sums inside the scratch.
-int* noalloc_status(uint8_t* base, size_t tab_bytes, const Geom& g, int nsplit) {
-    const size_t s_bytes = align_up(static_cast<size_t>(g.BH()) * nsplit * g.R * g.D * sizeof(float), 256);
-    const size_t z_bytes = align_up(static_cast<size_t>(g.BH()) * nsplit * g.R * sizeof(float), 256);
-    return reinterpret_cast<int*>(base + tab_bytes + s_bytes + z_bytes);
-}
+// Tokens per step of the partial-sum kernel: 128-token tiles on the tensor cores (head_dim 128), 32 on
+// the CUDA cores; a split covers ceil(tiles / nsplit) consecutive steps.
+int64_t lowrank_steps(const Geom& g) { return g.D == 128 ? (g.L + 127) / 128 : (g.L + 31) / 32; }
 
 }  // namespace
 
@@ -738,29 +739,51 @@ extern "C" slra_status slra_lowrank_summary_noalloc(const slra_problem* p, const
     if (!k || !v || !A || !S || !z) return SLRA_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(v) || !aligned16(A) || !aligned16(S) || !aligned16(z)) return SLRA_ERR_ALIGNMENT;
     const Geom& g = d.g;
-    // scratch: [cos/sin table | pair info] [partial S] [partial z], each 256-B aligned
+    // scratch: [status word] [cos/sin table | pair info] [partial S] [partial z], each 256-B aligned
     const size_t tab_bytes = align_up(sizeof(double2) * static_cast<size_t>(d.table_entries) + sizeof(int2) * kMaxPairs, 256);
+    const size_t fixed = kNoallocStatusBytes + tab_bytes;
     const size_t per_split = static_cast<size_t>(g.BH()) * g.R * (g.D + 1) * sizeof(float) + 512;
-    if (tab_bytes + per_split > SLRA_NOALLOC_SCRATCH_BYTES) return SLRA_ERR_SCRATCH_LIMIT;
-    int nsplit = d.nsplit;
-    const size_t fit = (SLRA_NOALLOC_SCRATCH_BYTES - tab_bytes) / per_split;
-    if (static_cast<size_t>(nsplit) > fit) nsplit = static_cast<int>(fit);
+    if (fixed + per_split > SLRA_NOALLOC_SCRATCH_BYTES) return SLRA_ERR_SCRATCH_LIMIT;
+    int64_t nsplit = d.nsplit;
+    const int64_t fit = static_cast<int64_t>((SLRA_NOALLOC_SCRATCH_BYTES - fixed) / per_split);
+    if (nsplit > fit) nsplit = fit;
+    // with fewer splits, re-balance so that no split is left without a step: ceil(steps / per split)
+    const int64_t steps = lowrank_steps(g);
+    const int64_t per = (steps + nsplit - 1) / nsplit;
+    nsplit = (steps + per - 1) / per;
     if ((s = check_device()) != SLRA_OK) return s;
     void* scratch = nullptr;
     if ((s = scratch_address(&scratch)) != SLRA_OK) return s;
     uint8_t* base = static_cast<uint8_t*>(scratch);
-    double2* tab = reinterpret_cast<double2*>(base);
-    int2* pairs = reinterpret_cast<int2*>(base + sizeof(double2) * d.table_entries);
-    float* s_part = reinterpret_cast<float*>(base + tab_bytes);
+    int* status = reinterpret_cast<int*>(base);
+    double2* tab = reinterpret_cast<double2*>(base + kNoallocStatusBytes);
+    int2* pairs = reinterpret_cast<int2*>(base + kNoallocStatusBytes + sizeof(double2) * d.table_entries);
+    float* s_part = reinterpret_cast<float*>(base + fixed);
     float* z_part = reinterpret_cast<float*>(
-        base + tab_bytes + align_up(static_cast<size_t>(g.BH()) * nsplit * g.R * g.D * sizeof(float), 256));
+        base + fixed + align_up(static_cast<size_t>(g.BH()) * nsplit * g.R * g.D * sizeof(float), 256));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // Every kernel below writes all the scratch it later reads (the whole table, every partial slot of
-    // every split), so nothing needs clearing between calls.
+    // The status word starts each call at zero (an async memset allocates nothing).  The kernels below
+    // write all the other scratch they later read (the whole table, every partial slot of every split),
+    // unless a bounded wait runs out: the status word then reports the timeout and S, z are unspecified.
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return SLRA_ERR_CUDA;
     if (launch_rope_table(tab, pairs, d.meta, d.table_entries, st) != cudaSuccess) return SLRA_ERR_CUDA;
-    // the device status word of this entry point is the scratch's first word after the partial sums
-    if (lowrank_partial(d, k, v, A, tab, pairs, nsplit, s_part, z_part, noalloc_status(base, tab_bytes, g, nsplit),
-                        timeout_of(p), st) != cudaSuccess)
+    if (lowrank_partial(d, k, v, A, tab, pairs, static_cast<int>(nsplit), s_part, z_part, status, timeout_of(p),
+                        debug_wait_of(p), st) != cudaSuccess)
         return SLRA_ERR_CUDA;
-    return cuda_status(launch_lowrank_reduce(s_part, z_part, g, nsplit, S, z, nullptr, nullptr, nullptr, st));
+    return cuda_status(launch_lowrank_reduce(s_part, z_part, g, static_cast<int>(nsplit), S, z, nullptr, nullptr,
+                                             nullptr, st));
+}
+
+extern "C" slra_status slra_noalloc_device_status(slra_stream_t stream, int32_t* status) {
+    if (!status) return SLRA_ERR_INVALID_ARG;
+    slra_status s = check_device();
+    if (s != SLRA_OK) return s;
+    void* scratch = nullptr;
+    if ((s = scratch_address(&scratch)) != SLRA_OK) return s;
+    int v = 0;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SLRA_ERR_CUDA;
+    if (cudaMemcpy(&v, scratch, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return SLRA_ERR_CUDA;
+    if (cudaMemset(scratch, 0, sizeof v) != cudaSuccess) return SLRA_ERR_CUDA;
+    *status = (v & kDevTimeout) ? SLRA_ERR_DEVICE_TIMEOUT : ((v & kDevRange) ? SLRA_ERR_RANGE : SLRA_OK);
+    return SLRA_OK;
 }

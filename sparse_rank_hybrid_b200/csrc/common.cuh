@@ -70,7 +70,8 @@ cudaError_t launch_lowrank_partial(const __nv_bfloat16* k, const __nv_bfloat16* 
 // Tensor-core low-rank partial sums (head_dim 128), see lowrank_sm100.cu.
 cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,
                               const double2* tab, const RopeMeta& meta, const Geom& g, int nsplit, float* s_part,
-                              float* z_part, int* status, unsigned long long timeout_ns, cudaStream_t st);
+                              float* z_part, int* status, unsigned long long timeout_ns, int debug_unsatisfied_wait,
+                              cudaStream_t st);
 int lowrank_nsplit(const Geom& g);
 bool make_map_headmajor(CUtensorMap* m, const void* base, uint64_t rows, int D, int box_rows);
 bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int D, int box_tokens);

@@ -72,6 +72,7 @@ struct LrArgs {
     int tiles_per_split;
     int* status;
     unsigned long long timeout_ns;
+    int debug_unsatisfied_wait;  // test hook: wait on a barrier nothing signals before any work
 };
 
 // kDefault: relu features with the RoPE (the benchmark's configuration); the activation and no-RoPE
@@ -92,6 +93,7 @@ __global__ void __launch_bounds__(256, 1)
     uint64_t* bar_kv = bars;         // [kStages]: k and v tile of a stage landed
     uint64_t* bar_phi = bars + 2;    // phi MMA done (covers every earlier MMA)
     uint64_t* bar_s = bars + 3;      // S MMA done (covers every earlier MMA)
+    uint64_t* bar_debug = bars + 4;  // test hook: nothing arrives here
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + lay.off_misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + lay.off_misc + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -100,7 +102,7 @@ __global__ void __launch_bounds__(256, 1)
     const uint64_t tmo = a.timeout_ns;
 
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -197,7 +199,11 @@ __global__ void __launch_bounds__(256, 1)
         ++n_phi_issued;
         return true;
     };
-    if (tid == 0) {
+    // Test hook: a wait on a barrier that nothing arrives at runs out, records a timeout and raises the
+    // abort flag before any copy or product has been issued; every thread then leaves the item loop.
+    if (a.debug_unsatisfied_wait && tid == 0 && !mbar_wait(bar_debug, 0, tmo, abort_flag)) fail();
+    __syncthreads();
+    if (tid == 0 && !*abort_flag) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
         issue_load(0);
@@ -212,7 +218,7 @@ __global__ void __launch_bounds__(256, 1)
     for (int item = blockIdx.x; item < n_items && !aborted; item += gridDim.x) {
         const int bh = item / a.nsplit, split = item % a.nsplit;
         const int t0 = split * a.tiles_per_split, t1 = min(ntiles, t0 + a.tiles_per_split);
-        if (t1 <= t0) {  // empty split (never produced by the host plan): contributes zeros
+        if (t1 <= t0) {  // empty split (the host plans avoid them): contributes zeros
             float* sp0 = a.s_part + (static_cast<size_t>(bh) * a.nsplit + split) * R * kD;
             for (int e = tid; e < R * kD; e += 256) sp0[e] = 0.f;
             if (tid < R) a.z_part[(static_cast<size_t>(bh) * a.nsplit + split) * R + tid] = 0.f;
@@ -419,7 +425,8 @@ static cudaError_t lr_tc_launch(const CUtensorMap& tk, const CUtensorMap& tv, co
 
 cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,
                               const double2* tab, const RopeMeta& meta, const Geom& g, int nsplit, float* s_part,
-                              float* z_part, int* status, unsigned long long timeout_ns, cudaStream_t st) {
+                              float* z_part, int* status, unsigned long long timeout_ns, int debug_unsatisfied_wait,
+                              cudaStream_t st) {
     CUtensorMap tk, tv;
     if (!make_map_tokens(&tk, k, g.B, g.L, g.Hh, g.D, kTok) || !make_map_tokens(&tv, v, g.B, g.L, g.Hh, g.D, kTok))
         return cudaErrorInvalidValue;
@@ -434,6 +441,7 @@ cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, co
     a.tiles_per_split = lowrank_tc_tiles_per_split(g, nsplit);
     a.status = status;
     a.timeout_ns = timeout_ns;
+    a.debug_unsatisfied_wait = debug_unsatisfied_wait;
     switch (g.R) {
         case 16: return lr_tc_launch<16>(tk, tv, a, g, st);
         case 32: return lr_tc_launch<32>(tk, tv, a, g, st);

@@ -29,7 +29,8 @@ EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_
            "slra_projection_elems",
            "slra_workspace_layout", "slra_attn_fwd", "slra_host_io_bytes", "slra_host_pipeline_groups",
            "slra_attn_fwd_host",
-           "slra_select_blocks", "slra_lowrank_summary", "slra_device_status", "slra_lowrank_summary_noalloc")
+           "slra_select_blocks", "slra_lowrank_summary", "slra_device_status", "slra_lowrank_summary_noalloc",
+           "slra_noalloc_device_status")
 
 
 class SlraError(RuntimeError):
@@ -93,9 +94,10 @@ def lib():
         L.slra_lowrank_summary.argtypes = [PP, P, P, P, P, S, P]
         L.slra_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.slra_lowrank_summary_noalloc.argtypes = [PP, P, P, P, P, P, P]
+        L.slra_noalloc_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
         for name in ("slra_problem_init", "slra_validate", "slra_workspace_layout", "slra_attn_fwd",
                      "slra_attn_fwd_host", "slra_select_blocks", "slra_lowrank_summary", "slra_device_status",
-                     "slra_lowrank_summary_noalloc"):
+                     "slra_lowrank_summary_noalloc", "slra_noalloc_device_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -301,6 +303,13 @@ def lowrank_summary_noalloc(prob: Problem, k, v, A, S, z, stream=None):
     _check(lib().slra_lowrank_summary_noalloc(ctypes.byref(prob.c()), _ptr(k), _ptr(v), _ptr(A), _ptr(S), _ptr(z),
                                               _stream_handle(stream)), "slra_lowrank_summary_noalloc")
     return S, z
+
+
+def noalloc_device_status(stream=None) -> int:
+    """Read and clear the device status of the no-allocation summary on the current device."""
+    st = ctypes.c_int32(-1)
+    _check(lib().slra_noalloc_device_status(_stream_handle(stream), ctypes.byref(st)), "slra_noalloc_device_status")
+    return int(st.value)
 
 
 def device_status(workspace, stream=None) -> int:

@@ -70,8 +70,11 @@ def _gate_of(prob: slra.Problem):
     return prob.gate_w.detach().cpu().numpy().astype(np.float64), float(np.float32(prob.gate_bias))
 
 
-def compare(prob: slra.Problem, x: dict, gpu: dict, heads=None, qblocks=None, check_masks=True, label=""):
-    """Run the oracle on (a sample of) the problem and compare.  Returns a dict of error stats."""
+def compare(prob: slra.Problem, x: dict, gpu: dict, heads=None, qblocks=None, check_masks=True, label="",
+            max_abs: float = MAX_ABS):
+    """Run the oracle on (a sample of) the problem and compare.  Returns a dict of error stats.
+    `max_abs` replaces the absolute bound for inputs whose v is scaled by s (the output scales with v,
+    so the same accuracy is 1e-2 * s there); the mean relative bound never changes."""
     grid = (prob.T, prob.H, prob.W)
     B, Hh = prob.batch, prob.heads
     pairs = [(b, h) for b in range(B) for h in range(Hh)] if heads is None else heads
@@ -111,6 +114,6 @@ def compare(prob: slra.Problem, x: dict, gpu: dict, heads=None, qblocks=None, ch
     stats["max_abs"] = float(err.max())
     stats["mean_rel"] = float(err.sum() / np.abs(o).sum())
     stats["n_compared"] = int(sel.sum())
-    assert stats["max_abs"] <= MAX_ABS, f"{label}: max abs error {stats['max_abs']:.3g}"
+    assert stats["max_abs"] <= max_abs, f"{label}: max abs error {stats['max_abs']:.3g}"
     assert stats["mean_rel"] <= MEAN_REL, f"{label}: mean rel error {stats['mean_rel']:.3g}"
     return stats

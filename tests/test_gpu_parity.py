@@ -318,6 +318,43 @@ def test_host_entry_point_pipelined(case):
         _log(parity.compare(p, x, dev, label=f"host-pipelined-{case}"))
 
 
+def _rescaled(x, seed, q=1.0, k=1.0, v=1.0, q_uniform=None):
+    """Inputs with q, k, v multiplied by the given factors and re-rounded to bf16 (RNE); q_uniform = c
+    draws q uniform in [-c, c] instead (seeded), so |q| stays below c and a rotated pair below c*sqrt(2)."""
+    y = dict(x)
+    for n, f in (("q", q), ("k", k), ("v", v)):
+        if f != 1.0:
+            y[n] = I.f32_to_bf16_bits(I.bf16_bits_to_f32(x[n]) * np.float32(f))
+    if q_uniform is not None:
+        rng = np.random.default_rng(seed)
+        y["q"] = I.f32_to_bf16_bits(rng.uniform(-q_uniform, q_uniform, x["q"].shape).astype(np.float32))
+    return y
+
+
+# (label, factors, absolute-bound multiplier): inputs far from unit scale, where the fp16 operands of
+# the attention kernel could lose range or precision.  q near 45,000 with k near 1e-4 keeps the logits
+# of order one while the rotated queries come within 3% of fp16's largest finite value (65,504).
+SCALE_CASES = [
+    ("qkv-1e-3", dict(q=1e-3, k=1e-3, v=1e-3), 1.0),
+    ("qkv-1e-5", dict(q=1e-5, k=1e-5, v=1e-5), 1.0),
+    ("v-1e-4", dict(v=1e-4), 1.0),
+    ("v-300", dict(v=300.0), 300.0),
+    ("q-near-fp16-max", dict(k=1e-4, q_uniform=45000.0), 1.0),
+]
+
+
+@pytest.mark.parametrize("label,factors,abs_mult", SCALE_CASES, ids=[c[0] for c in SCALE_CASES])
+@pytest.mark.parametrize("D", [64, 128])
+def test_input_scales(label, factors, abs_mult, D):
+    """Element-by-element parity far from unit scale (RoLA 4.1 defines the method on the model's
+    activations, which are not normalised), on both head dims; the device status must stay clean."""
+    w = W.Workload(f"scale-{label}-{D}", 1, 2, D, 3, 10, 13, 32 if D == 128 else 16, 64, 0.3, 7500 + D)
+    x = _rescaled(I.make_custom(w.seed, 1, (w.T, w.H, w.W), w.heads, D, w.rank), w.seed + 1, **factors)
+    p = slra.Problem.from_workload(w)
+    gpu = parity.run_gpu(p, x)
+    _log(parity.compare(p, x, gpu, label=f"scale-{label}-{D}", max_abs=parity.MAX_ABS * abs_mult))
+
+
 def test_range_error_reported():
     """An input too large for the fp16 operands is reported through the device status word."""
     import torch

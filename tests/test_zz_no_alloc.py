@@ -5,7 +5,9 @@ framework that owns all device memory through its own pool, an execute hook that
 a serving loop that cannot afford cudaMalloc's device-wide synchronization).  It keeps its scratch
 in one fixed array inside the library, so this test checks that two calls in a row, on different
 problem sizes, each reproduce slra_lowrank_summary within the summary tolerance, i.e. that nothing a
-previous call left in the shared array leaks into the next result.
+previous call left in the shared array leaks into the next result, and that a bounded wait that
+runs out inside the summary kernel is reported through slra_noalloc_device_status instead of
+passing silently.
 
 This file is collected last so that a failure here cannot hide another test's result.
 """
@@ -75,3 +77,28 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     with pytest.raises(slra.SlraError) as e:
         slra.lowrank_summary_noalloc(p, k, k, A, S, z)
     assert e.value.status == slra.ERR_SCRATCH_LIMIT
+
+
+# head_dim 128 (the tensor-core summary kernel, whose waits are bounded), L = 390 with a ragged tile
+EDGE_128 = W.Workload("noalloc-edge-128", 1, 2, 128, 3, 10, 13, 32, 128, 0.3, 7160)
+
+
+def test_noalloc_reports_a_timeout_and_recovers():
+    """The test hook makes every summary CTA wait on a barrier nothing signals; the wait runs out after
+    1 ms, the kernel records a timeout and returns, and the call's status reader reports it (once: it
+    clears the word).  The next call starts from a cleared status word and matches the workspace entry
+    point again."""
+    import torch
+    w = EDGE_128
+    x = I.make_inputs(w)
+    k, v, A = _gpu(x["k"]), _gpu(x["v"]), _gpu(x["A"])
+    BH = w.batch * w.heads
+    S = torch.zeros((BH, w.rank, w.head_dim), dtype=torch.float32, device="cuda")
+    z = torch.zeros((BH, w.rank), dtype=torch.float32, device="cuda")
+    p_hang = slra.Problem.from_workload(w, debug_flags=slra.DEBUG_UNSATISFIED_WAIT, wait_timeout_ns=1_000_000)
+    slra.lowrank_summary_noalloc(p_hang, k, v, A, S, z)
+    assert slra.noalloc_device_status() == slra.ERR_DEVICE_TIMEOUT
+    assert slra.noalloc_device_status() == slra.OK
+    S2, z2, S_ref, z_ref = _both(w)
+    assert slra.noalloc_device_status() == slra.OK
+    assert _rel(S2, S_ref) < SUMMARY_REL and _rel(z2, z_ref) < SUMMARY_REL
