@@ -44,7 +44,16 @@
  *     ran out) are recorded in a status word inside the workspace and reported by
  *     slra_device_status.
  *   - A workspace may be used by one call at a time (calls on one stream are ordered; calls on
- *     different streams need different workspaces).
+ *     different streams need different workspaces).  Where an entry point takes a workspace, NULL
+ *     means the library allocates one with cudaMallocAsync on `stream` (the current device's memory
+ *     pool) and frees it with cudaFreeAsync after its launches, both stream-ordered; the call's device
+ *     status then goes to slra_get_device_status instead.  Raising the release threshold of the
+ *     device's default pool (cudaMemPoolAttrReleaseThreshold) keeps that memory between calls.
+ *   - q, k, v and out are [B][L][Hh][D] with the D elements of a row contiguous; their batch, token and
+ *     head strides (in elements) are free (e.g. q, k, v as views of one fused QKV buffer), contiguous
+ *     token-major by default.  Input strides must be positive multiples of 8 elements (16 bytes of
+ *     bf16), output strides multiples of 16 bytes of the output type, all below 2^36, and distinct
+ *     output rows may not overlap.
  */
 #ifndef SLRA_H
 #define SLRA_H
@@ -56,7 +65,7 @@
 extern "C" {
 #endif
 
-#define SLRA_ABI_VERSION 5
+#define SLRA_ABI_VERSION 6
 
 /* Exported symbols (the library is built with hidden visibility for everything else). */
 #if defined(__GNUC__)
@@ -83,6 +92,28 @@ typedef enum slra_status {
 } slra_status;
 
 typedef enum slra_out_dtype { SLRA_OUT_F32 = 0, SLRA_OUT_BF16 = 1 } slra_out_dtype;
+
+/* Element type of a tensor descriptor. */
+typedef enum slra_dtype { SLRA_DTYPE_BF16 = 0, SLRA_DTYPE_F32 = 1 } slra_dtype;
+
+/*
+ * A [B][L][Hh][D] device tensor (batch, token, head, head dimension): `data` points at element
+ * (0, 0, 0, 0); element (b, n, h, d) sits at data + b*sB + n*sL + h*sH + d (strides in elements; all
+ * three zero = contiguous, i.e. sH = D, sL = Hh*D, sB = L*Hh*D).  The library only reads the inputs.
+ */
+typedef struct slra_tensor {
+    void* data;
+    int32_t dtype;  /* slra_dtype */
+    int64_t B, L, Hh, D;
+    int64_t sB, sL, sH;
+} slra_tensor;
+
+/* A [D][R] row-major device matrix: the low-rank projection A shared by queries, keys and heads. */
+typedef struct slra_mat {
+    const void* data;
+    int32_t dtype;  /* slra_dtype: bf16 */
+    int64_t D, R;
+} slra_mat;
 
 /* Which branches contribute to `out` (default both). */
 enum { SLRA_BRANCH_SPARSE = 1, SLRA_BRANCH_LOWRANK = 2, SLRA_BRANCH_BOTH = 3 };
@@ -151,6 +182,9 @@ typedef enum slra_activation {
  *                           too: the ordering RoLA's ablation compares against ("5.1" Table 2, "5.3",
  *                           "B.3"); the summary stays linear but loses the relative property.  Not
  *                           with lowrank_norope.
+ *   q_strides, k_strides,   (sB, sL, sH) element strides of q, k, v and out (see the conventions at the
+ *   v_strides, out_strides  top); all zero (default) = contiguous [B][L][Hh][D].  slra_attn_fwd_host
+ *                           takes contiguous host buffers only.
  */
 typedef struct slra_problem {
     int64_t batch, heads, head_dim;
@@ -174,6 +208,7 @@ typedef struct slra_problem {
     float gate_bias;
     const void* gate_w;
     int32_t lowrank_rope_inside;
+    int64_t q_strides[3], k_strides[3], v_strides[3], out_strides[3];
 } slra_problem;
 
 /*
@@ -218,18 +253,74 @@ SLRA_API int64_t slra_projection_elems(const slra_problem* p);
 SLRA_API slra_status slra_workspace_layout(const slra_problem* p, slra_ws_layout* layout);
 
 /*
- * Full forward pass (RoLA "4.1" sparse + low-rank hybrid; all steps listed at the top of this file).
- *   q, k, v    bf16 [B][L][Hh][D] contiguous (token-major), 16-B aligned.
+ * Workspace bytes of a forward call with these sizes (the same value slra_workspace_layout gives for a
+ * problem with the default options); 0 if the sizes are invalid.  No GPU access.
+ */
+SLRA_API size_t slra_workspace_bytes(int64_t batch, int64_t heads, int64_t head_dim, int64_t T, int64_t H,
+                                     int64_t W, int64_t block, float keep_frac, int64_t rank);
+
+/*
+ * Full forward pass, all steps listed at the top of this file (RoLA "4.1": block-sparse softmax
+ * branch over the top-k key blocks by block-mean-pooled post-RoPE scores, plus the low-rank branch
+ * with the rank-truncated RoPE outside the relu feature map, "4.2", "4.3"; the two outputs summed).
+ *   q, k, v    bf16 descriptors of equal shape [B][L][Hh][D], L = T*H*W; any strides per the
+ *              conventions above (e.g. three views of one fused QKV projection output).
+ *   A          bf16 [D][rank] projection shared by queries, keys and heads.
+ *   T, H, W    latent grid (row-major t, h, w); block in {64, 128}; keep_frac in (0, 1] (widened to
+ *              double: k = clamp(floor(keep_frac * nb + 0.5), 1, nb)); rank a multiple of 16, <= D.
+ *   out        fp32 or bf16 descriptor of the same shape; may not overlap q, k, v or A.
+ * The library allocates its workspace on `stream` (see the conventions) and leaves the device status
+ * to slra_get_device_status.  Asynchronous; the default options of slra_problem apply.
+ */
+SLRA_API slra_status slra_attn_fwd(const slra_tensor* q, const slra_tensor* k, const slra_tensor* v,
+                                   const slra_mat* A, int T, int H, int W, int block, float keep_frac, int rank,
+                                   slra_tensor* out, slra_stream_t stream);
+
+/*
+ * The forward pass with every option of the problem struct: feature map, RoPE ordering, projection layouts,
+ * gated fusion, branches, strides, timing events, test hooks.
+ *   q, k, v    bf16 [B][L][Hh][D] device tensors, 16-B aligned, strides from p (contiguous by default).
  *   A          bf16 projection(s), contiguous, 16-B aligned: [D][rank] shared by q, k and all heads by
  *              default; [1 + proj_separate][proj_per_head ? Hh : 1][D][rank] in general (query
- *              projections first, then key projections).
- *   out        [B][L][Hh][D] contiguous, fp32 or bf16 as p->out_dtype; must not alias q, k, v.
- *   workspace  device buffer of at least layout.total_bytes bytes, 256-B aligned.
+ *              projections first, then key projections).  May be NULL when the low-rank branch is off.
+ *   out        [B][L][Hh][D], fp32 or bf16 as p->out_dtype, strides from p; must not overlap the
+ *              inputs or the workspace.
+ *   workspace  device buffer of at least layout.total_bytes bytes, 256-B aligned, or NULL (allocated
+ *              by the library, see the conventions).
  * Launches 6 kernels on `stream` (tables, RoPE + pooling, selection, low-rank partial sums and their
  * reduction, attention with the fused low-rank readout) and returns without synchronizing.
  */
-SLRA_API slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
-                          void* out, void* workspace, size_t workspace_bytes, slra_stream_t stream);
+SLRA_API slra_status slra_attn_fwd_ex(const slra_problem* p, const void* q, const void* k, const void* v,
+                                      const void* A, void* out, void* workspace, size_t workspace_bytes,
+                                      slra_stream_t stream);
+
+/*
+ * The sparse branch alone (RoLA "4.1": softmax attention of each query block over its top-k key blocks,
+ * selected by block-mean-pooled post-RoPE scores): out = O_sparse.  Arguments as slra_attn_fwd; the
+ * workspace holds slra_workspace_bytes(B, Hh, D, T, H, W, block, keep_frac, 16) bytes (the branch has no
+ * rank; 16 sizes the unused low-rank sections) or is NULL.
+ */
+SLRA_API slra_status slra_sparse_fwd(const slra_tensor* q, const slra_tensor* k, const slra_tensor* v, int T,
+                                     int H, int W, int block, float keep_frac, slra_tensor* out, void* workspace,
+                                     size_t workspace_bytes, slra_stream_t stream);
+
+/*
+ * The low-rank branch alone (RoLA "4.1", "4.2", "4.3", "B.1"): out = psi(q)^T S / (phi(q) . z + 1e-6)
+ * with S = sum_j psi(k_j) v_j^T and z = sum_j phi(k_j) over all L keys.  Arguments as slra_attn_fwd;
+ * S (fp32 [B*Hh][rank][D]) and z (fp32 [B*Hh][rank]) receive the summary when not NULL (16-B aligned).
+ * The workspace holds slra_workspace_bytes(B, Hh, D, T, H, W, 128, 1e-4f, rank) bytes (the branch does
+ * not select blocks; these values size the unused sections) or is NULL.
+ */
+SLRA_API slra_status slra_lowrank_fwd(const slra_tensor* q, const slra_tensor* k, const slra_tensor* v,
+                                      const slra_mat* A, int T, int H, int W, int rank, slra_tensor* out, float* S,
+                                      float* z, void* workspace, size_t workspace_bytes, slra_stream_t stream);
+
+/*
+ * Device status of the calls whose workspace the library allocated (slra_attn_fwd, and the others when
+ * given a NULL workspace) on the current device: synchronize `stream`, then read and clear the word
+ * their status words were ORed into.  *status receives SLRA_OK, SLRA_ERR_DEVICE_TIMEOUT or SLRA_ERR_RANGE.
+ */
+SLRA_API slra_status slra_get_device_status(slra_stream_t stream, int32_t* status);
 
 /*
  * The same forward pass on HOST buffers: copies q, k, v and A (slra_projection_elems(p) elements)
@@ -253,14 +344,14 @@ SLRA_API slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_hos
 
 /*
  * Block selection only (3D RoPE, block means, scores, top-k): fills the qh/kh/vh, qbar/kbar, idx and
- * tie sections of the workspace.  Same argument rules as slra_attn_fwd.
+ * tie sections of the workspace.  Same argument rules as slra_attn_fwd_ex (the workspace is required).
  */
 SLRA_API slra_status slra_select_blocks(const slra_problem* p, const void* q, const void* k, const void* v,
                                void* workspace, size_t workspace_bytes, slra_stream_t stream);
 
 /*
  * Low-rank summary only (RoLA "4.1", "B.1"): fills the S and z sections of the workspace from raw k,
- * v and A.  Same argument rules as slra_attn_fwd.
+ * v and A.  Same argument rules as slra_attn_fwd_ex (the workspace is required).
  */
 SLRA_API slra_status slra_lowrank_summary(const slra_problem* p, const void* k, const void* v, const void* A,
                                  void* workspace, size_t workspace_bytes, slra_stream_t stream);
@@ -282,8 +373,8 @@ SLRA_API slra_status slra_device_status(void* workspace, slra_stream_t stream, i
  * allocations, plugin-style execute hooks that must not allocate, and latency-critical serving loops
  * where cudaMalloc/cudaFree would synchronize the device and stall other streams.
  *
- *   k, v     bf16 [B][L][Hh][D] contiguous, 16-B aligned (device).
- *   A        bf16 projection(s) laid out as for slra_attn_fwd, 16-B aligned (device); the summary
+ *   k, v     bf16 [B][L][Hh][D], 16-B aligned (device), strides from p (contiguous by default).
+ *   A        bf16 projection(s) laid out as for slra_attn_fwd_ex, 16-B aligned (device); the summary
  *            uses the key projection(s).
  *   S        fp32 [B*Hh][rank][D] output (device, 16-B aligned).
  *   z        fp32 [B*Hh][rank]    output (device, 16-B aligned).

@@ -18,11 +18,23 @@ __global__ void status_or_kernel(int* acc, const int* src) {
     const int v = *src;
     if (v) atomicOr(acc, v);
 }
+
+// Device status of the calls whose workspace the library allocated (and freed) itself: their status
+// words are ORed here before the workspace goes back to the pool (slra_get_device_status reads it).
+__device__ int g_call_status;
+__global__ void status_or_global_kernel(const int* src) {
+    const int v = *src;
+    if (v) atomicOr(&g_call_status, v);
+}
 }  // namespace slra
 
 namespace {
 
 constexpr int64_t kMaxBlocks = 2048;  // selection keeps a row of scores in shared memory
+// The branch entry points size their workspace with the parameters the branch does not use set to these.
+constexpr int kSparseOnlyRank = 16;
+constexpr int kLowrankOnlyBlock = 128;
+constexpr float kLowrankOnlyKeep = 1e-4f;  // one kept block per query block (up to 2048 blocks)
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -36,6 +48,44 @@ bool default_split(int64_t D, const int64_t* s, int64_t out[3]) {
     }
     if (s[0] < 0 || s[1] < 0 || s[2] < 0 || s[0] + s[1] + s[2] != c) return false;
     out[0] = s[0]; out[1] = s[1]; out[2] = s[2];
+    return true;
+}
+
+// Element strides (batch, token, head) of a [B][L][Hh][D] tensor: all zero means contiguous
+// (token-major); otherwise positive multiples of `align` elements (16-byte TMA strides), below 2^36.
+bool strides_of(const int64_t s[3], int64_t L, int64_t Hh, int64_t D, int64_t align, Strides* out) {
+    if (s[0] == 0 && s[1] == 0 && s[2] == 0) {
+        out->h = D;
+        out->l = Hh * D;
+        out->b = L * Hh * D;
+        return true;
+    }
+    for (int i = 0; i < 3; ++i)
+        if (s[i] <= 0 || s[i] % align != 0 || s[i] >= (int64_t(1) << 36)) return false;
+    out->b = s[0];
+    out->l = s[1];
+    out->h = s[2];
+    return true;
+}
+
+// Elements from a tensor's first element to one past its last.
+int64_t extent_elems(const Strides& st, int64_t B, int64_t L, int64_t Hh, int64_t D) {
+    return (B - 1) * st.b + (L - 1) * st.l + (Hh - 1) * st.h + D;
+}
+
+// True when distinct (batch, token, head) rows of D elements never share an element: taking the
+// dimensions by increasing stride, each stride clears everything the smaller ones span.
+bool rows_disjoint(const Strides& st, int64_t B, int64_t L, int64_t Hh, int64_t D) {
+    int64_t s[3] = {st.b, st.l, st.h}, n[3] = {B, L, Hh};
+    for (int i = 0; i < 3; ++i)
+        for (int j = i + 1; j < 3; ++j)
+            if (s[j] < s[i]) { std::swap(s[i], s[j]); std::swap(n[i], n[j]); }
+    int64_t span = D;
+    for (int i = 0; i < 3; ++i) {
+        if (n[i] == 1) continue;
+        if (s[i] < span) return false;
+        span += s[i] * (n[i] - 1);
+    }
     return true;
 }
 
@@ -102,6 +152,14 @@ slra_status derive(const slra_problem* p, Derived* d) {
     g.norope = static_cast<int>(p->lowrank_norope);
     g.a_stride = p->proj_per_head ? g.D * g.R : 0;
     g.inside = static_cast<int>(p->lowrank_rope_inside);
+    // element strides: inputs in 16-byte units of bf16; out in 16-byte units of its type, rows disjoint
+    const int64_t out_align = p->out_dtype == SLRA_OUT_F32 ? 4 : 8;
+    if (!strides_of(p->q_strides, L, p->heads, p->head_dim, 8, &g.sq) ||
+        !strides_of(p->k_strides, L, p->heads, p->head_dim, 8, &g.sk) ||
+        !strides_of(p->v_strides, L, p->heads, p->head_dim, 8, &g.sv) ||
+        !strides_of(p->out_strides, L, p->heads, p->head_dim, out_align, &g.so) ||
+        !rows_disjoint(g.so, p->batch, L, p->heads, p->head_dim))
+        return SLRA_ERR_INVALID_ARG;
     // projection argument: [1 + separate][per_head ? Hh : 1][D][R], query projection(s) first
     const size_t one_side = static_cast<size_t>(p->proj_per_head ? p->heads : 1) * p->head_dim * p->rank;
     d->a_elems = one_side * (p->proj_separate ? 2 : 1);
@@ -247,8 +305,9 @@ slra_status run_select(const slra_problem* p, const Derived& d, const Ptrs& w, c
                        const void* v, cudaStream_t st) {
     const Geom& g = d.g;
     CUtensorMap mq, mk, mv;  // token-major inputs, boxes of 64 columns x one key block of tokens
-    if (!make_map_tokens(&mq, q, g.B, g.L, g.Hh, g.D, g.block) || !make_map_tokens(&mk, k, g.B, g.L, g.Hh, g.D, g.block) ||
-        !make_map_tokens(&mv, v, g.B, g.L, g.Hh, g.D, g.block))
+    if (!make_map_tokens(&mq, q, g.B, g.L, g.Hh, g.D, g.sq, g.block) ||
+        !make_map_tokens(&mk, k, g.B, g.L, g.Hh, g.D, g.sk, g.block) ||
+        !make_map_tokens(&mv, v, g.B, g.L, g.Hh, g.D, g.sv, g.block))
         return SLRA_ERR_CUDA;
     cudaError_t e = launch_rope_pool(mq, mk, mv, w.tab, w.pairs, g, w.qh, w.kh, w.vh, w.qbar, w.kbar, w.status,
                                      timeout_of(p), st);
@@ -299,6 +358,66 @@ slra_status begin(const slra_problem* p, const Derived& d, const Ptrs& w, cudaSt
 
 size_t qkv_bytes(const Derived& d) {
     return static_cast<size_t>(d.g.B) * d.g.L * d.g.Hh * d.g.D * 2;
+}
+
+// Bytes a [B][L][Hh][D] tensor with strides st spans (es bytes per element).
+size_t span_bytes(const Geom& g, const Strides& st, size_t es) {
+    return static_cast<size_t>(extent_elems(st, g.B, g.L, g.Hh, g.D)) * es;
+}
+
+bool contiguous_io(const slra_problem* p) {
+    for (int i = 0; i < 3; ++i)
+        if (p->q_strides[i] || p->k_strides[i] || p->v_strides[i] || p->out_strides[i]) return false;
+    return true;
+}
+
+// The forward pass on a caller's (or the library's) workspace; arguments already validated by derive.
+slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, const void* k, const void* v,
+                     const void* A, void* out, void* workspace, cudaStream_t st);
+
+// Runs body(workspace) on the caller's workspace, or, when that is NULL, on one the library allocates
+// with cudaMallocAsync on `st` (the device's current memory pool) and frees with cudaFreeAsync after the
+// launches, both stream-ordered; that call's device status word is ORed into g_call_status first.
+template <class Body>
+slra_status with_workspace(const Derived& d, void* workspace, size_t workspace_bytes, cudaStream_t st, Body&& body) {
+    if (workspace) {
+        slra_status s = check_ws(d, workspace, workspace_bytes);
+        return s != SLRA_OK ? s : body(workspace);
+    }
+    void* raw = nullptr;
+    if (cudaMallocAsync(&raw, d.lay.total_bytes + 256, st) != cudaSuccess) {
+        cudaGetLastError();
+        return SLRA_ERR_CUDA;
+    }
+    void* ws = reinterpret_cast<void*>(align_up(reinterpret_cast<uintptr_t>(raw), 256));
+    slra_status s = body(ws);
+    if (s == SLRA_OK) {
+        slra::status_or_global_kernel<<<1, 1, 0, st>>>(reinterpret_cast<const int*>(static_cast<uint8_t*>(ws) +
+                                                                                    d.lay.status));
+        if (cudaGetLastError() != cudaSuccess) s = SLRA_ERR_CUDA;
+    }
+    if (cudaFreeAsync(raw, st) != cudaSuccess) {
+        cudaGetLastError();
+        if (s == SLRA_OK) s = SLRA_ERR_CUDA;
+    }
+    return s;
+}
+
+// Shared validation of the device entry points' tensor arguments.  A may be NULL when the low-rank
+// branch is off.
+slra_status check_fwd_args(const slra_problem* p, const Derived& d, const void* q, const void* k, const void* v,
+                           const void* A, const void* out, const void* workspace, size_t workspace_bytes) {
+    const int branches = p->branches == 0 ? SLRA_BRANCH_BOTH : p->branches;
+    if (!q || !k || !v || !out || ((branches & SLRA_BRANCH_LOWRANK) && !A)) return SLRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (A && !aligned16(A)) || !aligned16(out))
+        return SLRA_ERR_ALIGNMENT;
+    const Geom& g = d.g;
+    const size_t out_b = span_bytes(g, g.so, p->out_dtype == SLRA_OUT_F32 ? 4 : 2);
+    if (overlaps(out, out_b, q, span_bytes(g, g.sq, 2)) || overlaps(out, out_b, k, span_bytes(g, g.sk, 2)) ||
+        overlaps(out, out_b, v, span_bytes(g, g.sv, 2)) || (A && overlaps(out, out_b, A, d.a_elems * 2)) ||
+        (workspace && overlaps(out, out_b, workspace, workspace_bytes)))
+        return SLRA_ERR_INVALID_ARG;
+    return SLRA_OK;
 }
 
 // ------------------------------------------------------------------ host entry point, pipelined
@@ -440,7 +559,7 @@ slra_status host_fwd_pipelined(const slra_problem* p, const Derived& d, const vo
         }
         slra_problem pgi = pl.sub;
         pgi.heads = hn;
-        s = slra_attn_fwd(&pgi, sq, sk, sv, Ag, so, sws, slot_ws, reinterpret_cast<slra_stream_t>(st));
+        s = slra_attn_fwd_ex(&pgi, sq, sk, sv, Ag, so, sws, slot_ws, reinterpret_cast<slra_stream_t>(st));
         if (s != SLRA_OK) return fail(s);
         slra::status_or_kernel<<<1, 1, 0, st>>>(acc, reinterpret_cast<const int*>(sws));
         if (cudaGetLastError() != cudaSuccess || cudaEventRecord(hp.done[sl], st) != cudaSuccess)
@@ -454,6 +573,86 @@ slra_status host_fwd_pipelined(const slra_problem* p, const Derived& d, const vo
     }
     if (cudaStreamWaitEvent(st, hp.out[(G - 1) & 1], 0) != cudaSuccess) return fail(SLRA_ERR_CUDA);
     return cuda_status(cudaStreamSynchronize(st));
+}
+
+slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, const void* k, const void* v,
+                     const void* A, void* out, void* workspace, cudaStream_t st) {
+    slra_status s;
+    const Ptrs w = carve(workspace, d);
+    const int branches = p->branches == 0 ? SLRA_BRANCH_BOTH : p->branches;
+    const Geom& g = d.g;
+
+    AttnMaps maps;
+    const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
+    if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) || !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
+        !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
+        !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, g.sq, 128) ||
+        !make_map_out(&maps.out, out, g.B, g.L, g.Hh, g.D, g.so, p->out_dtype == SLRA_OUT_F32))
+        return SLRA_ERR_CUDA;
+
+    if ((s = begin(p, d, w, st)) != SLRA_OK) return s;
+    // a branch that is off still records its stage boundaries, so its stages time as zero
+    if (branches & SLRA_BRANCH_SPARSE) {
+        if ((s = run_select(p, d, w, q, k, v, st)) != SLRA_OK) return s;
+    } else if ((s = mark(p, 2, st)) != SLRA_OK || (s = mark(p, 3, st)) != SLRA_OK) {
+        return s;
+    }
+    if (branches & SLRA_BRANCH_LOWRANK) {
+        if ((s = run_lowrank(p, d, w, k, v, A, st)) != SLRA_OK) return s;
+    } else if ((s = mark(p, 4, st)) != SLRA_OK || (s = mark(p, 5, st)) != SLRA_OK) {
+        return s;
+    }
+
+    AttnArgs a;
+    a.qh = w.qh;
+    a.kh = w.kh;
+    a.vh = w.vh;
+    a.idx = w.idx;
+    a.keep = (branches & SLRA_BRANCH_SPARSE) ? g.keep : 0;
+    a.q_raw = static_cast<const __nv_bfloat16*>(q);
+    a.A = static_cast<const __nv_bfloat16*>(A);  // query projection(s); NULL when the low-rank branch is off
+    a.S = w.S;
+    a.z = w.z;
+    a.tab = w.tab;
+    a.pairs = w.pairs;
+    for (int e = 0; e < kMaxPairs; ++e)
+        a.pair_info[e] = e < d.meta.npairs ? make_int2(d.meta.axis[e], d.meta.tab_off[e]) : make_int2(0, 0);
+    a.at_img = w.at_img;
+    a.sb_img = w.sb_img;
+    a.lowrank = (branches & SLRA_BRANCH_LOWRANK) ? 1 : 0;
+    a.gated = p->fusion == SLRA_FUSION_GATED ? 1 : 0;
+    a.gate_b = p->gate_bias;
+    a.gate_w = static_cast<const float*>(p->gate_w);
+    a.out = out;
+    a.out_bf16 = p->out_dtype == SLRA_OUT_BF16 ? 1 : 0;
+    a.status = w.status;
+    a.timeout_ns = timeout_of(p);
+    a.debug_unsatisfied_wait = debug_wait_of(p);
+    if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
+    return mark(p, 6, st);
+}
+
+// A problem description from the tensor descriptors of the descriptor-style entry points.
+slra_status problem_from(const slra_tensor* q, const slra_tensor* k, const slra_tensor* v, const slra_tensor* out,
+                         int T, int H, int W, int block, float keep_frac, int rank, slra_problem* p) {
+    if (!q || !k || !v || !out) return SLRA_ERR_INVALID_ARG;
+    for (const slra_tensor* t : {q, k, v})
+        if (t->dtype != SLRA_DTYPE_BF16 || t->B != q->B || t->L != q->L || t->Hh != q->Hh || t->D != q->D)
+            return SLRA_ERR_INVALID_ARG;
+    if (out->dtype != SLRA_DTYPE_F32 && out->dtype != SLRA_DTYPE_BF16) return SLRA_ERR_INVALID_ARG;
+    if (out->B != q->B || out->L != q->L || out->Hh != q->Hh || out->D != q->D) return SLRA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(T) * H * W != q->L) return SLRA_ERR_INVALID_ARG;
+    slra_status s = slra_problem_init(p, q->B, q->Hh, q->D, T, H, W, block, static_cast<double>(keep_frac), rank);
+    if (s != SLRA_OK) return s;
+    p->out_dtype = out->dtype == SLRA_DTYPE_F32 ? SLRA_OUT_F32 : SLRA_OUT_BF16;
+    const slra_tensor* ts[4] = {q, k, v, out};
+    int64_t* dst[4] = {p->q_strides, p->k_strides, p->v_strides, p->out_strides};
+    for (int i = 0; i < 4; ++i) {
+        dst[i][0] = ts[i]->sB;
+        dst[i][1] = ts[i]->sL;
+        dst[i][2] = ts[i]->sH;
+    }
+    return SLRA_OK;
 }
 
 }  // namespace
@@ -530,73 +729,17 @@ slra_status slra_workspace_layout(const slra_problem* p, slra_ws_layout* layout)
     return SLRA_OK;
 }
 
-slra_status slra_attn_fwd(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
-                          void* out, void* workspace, size_t workspace_bytes, slra_stream_t stream) {
+slra_status slra_attn_fwd_ex(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
+                             void* out, void* workspace, size_t workspace_bytes, slra_stream_t stream) {
     Derived d;
     slra_status s = derive(p, &d);
     if (s != SLRA_OK) return s;
-    if (!q || !k || !v || !A || !out) return SLRA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(A) || !aligned16(out)) return SLRA_ERR_ALIGNMENT;
-    if ((s = check_ws(d, workspace, workspace_bytes)) != SLRA_OK) return s;
-    const size_t in_b = qkv_bytes(d);
-    const size_t out_b = in_b / 2 * (p->out_dtype == SLRA_OUT_F32 ? 4 : 2);
-    if (overlaps(out, out_b, q, in_b) || overlaps(out, out_b, k, in_b) || overlaps(out, out_b, v, in_b) ||
-        overlaps(out, out_b, A, d.a_elems * 2) || overlaps(out, out_b, workspace, workspace_bytes))
-        return SLRA_ERR_INVALID_ARG;
+    if ((s = check_fwd_args(p, d, q, k, v, A, out, workspace, workspace_bytes)) != SLRA_OK) return s;
+    if (workspace && (s = check_ws(d, workspace, workspace_bytes)) != SLRA_OK) return s;  // before the device
     if ((s = check_device()) != SLRA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const Ptrs w = carve(workspace, d);
-    const int branches = p->branches == 0 ? SLRA_BRANCH_BOTH : p->branches;
-    const Geom& g = d.g;
-
-    AttnMaps maps;
-    const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
-    if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) || !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
-        !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
-        !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, 128) ||
-        !make_map_out(&maps.out, out, g.B, g.L, g.Hh, g.D, p->out_dtype == SLRA_OUT_F32))
-        return SLRA_ERR_CUDA;
-
-    if ((s = begin(p, d, w, st)) != SLRA_OK) return s;
-    // a branch that is off still records its stage boundaries, so its stages time as zero
-    if (branches & SLRA_BRANCH_SPARSE) {
-        if ((s = run_select(p, d, w, q, k, v, st)) != SLRA_OK) return s;
-    } else if ((s = mark(p, 2, st)) != SLRA_OK || (s = mark(p, 3, st)) != SLRA_OK) {
-        return s;
-    }
-    if (branches & SLRA_BRANCH_LOWRANK) {
-        if ((s = run_lowrank(p, d, w, k, v, A, st)) != SLRA_OK) return s;
-    } else if ((s = mark(p, 4, st)) != SLRA_OK || (s = mark(p, 5, st)) != SLRA_OK) {
-        return s;
-    }
-
-    AttnArgs a;
-    a.qh = w.qh;
-    a.kh = w.kh;
-    a.vh = w.vh;
-    a.idx = w.idx;
-    a.keep = (branches & SLRA_BRANCH_SPARSE) ? g.keep : 0;
-    a.q_raw = static_cast<const __nv_bfloat16*>(q);
-    a.A = static_cast<const __nv_bfloat16*>(A);  // query projection(s)
-    a.S = w.S;
-    a.z = w.z;
-    a.tab = w.tab;
-    a.pairs = w.pairs;
-    for (int e = 0; e < kMaxPairs; ++e)
-        a.pair_info[e] = e < d.meta.npairs ? make_int2(d.meta.axis[e], d.meta.tab_off[e]) : make_int2(0, 0);
-    a.at_img = w.at_img;
-    a.sb_img = w.sb_img;
-    a.lowrank = (branches & SLRA_BRANCH_LOWRANK) ? 1 : 0;
-    a.gated = p->fusion == SLRA_FUSION_GATED ? 1 : 0;
-    a.gate_b = p->gate_bias;
-    a.gate_w = static_cast<const float*>(p->gate_w);
-    a.out = out;
-    a.out_bf16 = p->out_dtype == SLRA_OUT_BF16 ? 1 : 0;
-    a.status = w.status;
-    a.timeout_ns = p->wait_timeout_ns ? p->wait_timeout_ns : 2000000000ull;
-    a.debug_unsatisfied_wait = (p->debug_flags & SLRA_DEBUG_UNSATISFIED_WAIT) ? 1 : 0;
-    if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
-    return mark(p, 6, st);
+    return with_workspace(d, workspace, workspace_bytes, st,
+                          [&](void* ws) { return fwd_impl(p, d, q, k, v, A, out, ws, st); });
 }
 
 size_t slra_host_io_bytes(const slra_problem* p) {
@@ -622,6 +765,7 @@ slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const 
     slra_status s = derive(p, &d);
     if (s != SLRA_OK) return s;
     if (!q_host || !k_host || !v_host || !A_host || !out_host || !io) return SLRA_ERR_INVALID_ARG;
+    if (!contiguous_io(p)) return SLRA_ERR_INVALID_ARG;  // host buffers are contiguous [B][L][Hh][D]
     if ((reinterpret_cast<uintptr_t>(io) & 255u) != 0 || io_bytes < slra_host_io_bytes(p)) return SLRA_ERR_WORKSPACE;
     if ((s = check_ws(d, workspace, workspace_bytes)) != SLRA_OK) return s;
     if ((s = check_device()) != SLRA_OK) return s;
@@ -643,7 +787,7 @@ slra_status slra_attn_fwd_host(const slra_problem* p, const void* q_host, const 
         cudaMemcpyAsync(dv, v_host, raw, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(dA, A_host, a_raw, cudaMemcpyHostToDevice, st) != cudaSuccess)
         return SLRA_ERR_CUDA;
-    s = slra_attn_fwd(p, dq, dk, dv, dA, dout, workspace, workspace_bytes, stream);
+    s = slra_attn_fwd_ex(p, dq, dk, dv, dA, dout, workspace, workspace_bytes, stream);
     if (s != SLRA_OK) return s;
     if (cudaMemcpyAsync(out_host, dout, out_raw, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SLRA_ERR_CUDA;
     return cuda_status(cudaStreamSynchronize(st));
@@ -686,6 +830,80 @@ slra_status slra_device_status(void* workspace, slra_stream_t stream, int32_t* s
     if (cudaStreamSynchronize(st) != cudaSuccess) return SLRA_ERR_CUDA;
     if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return SLRA_ERR_CUDA;
     if (cudaMemset(workspace, 0, sizeof v) != cudaSuccess) return SLRA_ERR_CUDA;
+    *status = (v & kDevTimeout) ? SLRA_ERR_DEVICE_TIMEOUT : ((v & kDevRange) ? SLRA_ERR_RANGE : SLRA_OK);
+    return SLRA_OK;
+}
+
+size_t slra_workspace_bytes(int64_t batch, int64_t heads, int64_t head_dim, int64_t T, int64_t H, int64_t W,
+                            int64_t block, float keep_frac, int64_t rank) {
+    slra_problem p;
+    if (slra_problem_init(&p, batch, heads, head_dim, T, H, W, block, static_cast<double>(keep_frac), rank) != SLRA_OK)
+        return 0;
+    Derived d;
+    return derive(&p, &d) == SLRA_OK ? d.lay.total_bytes : 0;
+}
+
+slra_status slra_attn_fwd(const slra_tensor* q, const slra_tensor* k, const slra_tensor* v, const slra_mat* A,
+                          int T, int H, int W, int block, float keep_frac, int rank, slra_tensor* out,
+                          slra_stream_t stream) {
+    slra_problem p;
+    slra_status s = problem_from(q, k, v, out, T, H, W, block, keep_frac, rank, &p);
+    if (s != SLRA_OK) return s;
+    if (!A || !A->data || A->dtype != SLRA_DTYPE_BF16 || A->D != q->D || A->R != rank) return SLRA_ERR_INVALID_ARG;
+    return slra_attn_fwd_ex(&p, q->data, k->data, v->data, A->data, out->data, nullptr, 0, stream);
+}
+
+slra_status slra_sparse_fwd(const slra_tensor* q, const slra_tensor* k, const slra_tensor* v, int T, int H, int W,
+                            int block, float keep_frac, slra_tensor* out, void* workspace, size_t workspace_bytes,
+                            slra_stream_t stream) {
+    slra_problem p;
+    slra_status s = problem_from(q, k, v, out, T, H, W, block, keep_frac, kSparseOnlyRank, &p);
+    if (s != SLRA_OK) return s;
+    p.branches = SLRA_BRANCH_SPARSE;
+    return slra_attn_fwd_ex(&p, q->data, k->data, v->data, nullptr, out->data, workspace, workspace_bytes, stream);
+}
+
+slra_status slra_lowrank_fwd(const slra_tensor* q, const slra_tensor* k, const slra_tensor* v, const slra_mat* A,
+                             int T, int H, int W, int rank, slra_tensor* out, float* S, float* z, void* workspace,
+                             size_t workspace_bytes, slra_stream_t stream) {
+    slra_problem p;
+    slra_status s = problem_from(q, k, v, out, T, H, W, kLowrankOnlyBlock, kLowrankOnlyKeep, rank, &p);
+    if (s != SLRA_OK) return s;
+    if (!A || !A->data || A->dtype != SLRA_DTYPE_BF16 || A->D != q->D || A->R != rank) return SLRA_ERR_INVALID_ARG;
+    if ((S && !aligned16(S)) || (z && !aligned16(z))) return SLRA_ERR_ALIGNMENT;
+    p.branches = SLRA_BRANCH_LOWRANK;
+    Derived d;
+    if ((s = derive(&p, &d)) != SLRA_OK) return s;
+    if ((s = check_fwd_args(&p, d, q->data, k->data, v->data, A->data, out->data, workspace, workspace_bytes)) !=
+        SLRA_OK)
+        return s;
+    if (workspace && (s = check_ws(d, workspace, workspace_bytes)) != SLRA_OK) return s;
+    if ((s = check_device()) != SLRA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t s_bytes = static_cast<size_t>(d.g.BH()) * d.g.R * d.g.D * 4, z_bytes = static_cast<size_t>(d.g.BH()) * d.g.R * 4;
+    return with_workspace(d, workspace, workspace_bytes, st, [&](void* ws) {
+        slra_status r = fwd_impl(&p, d, q->data, k->data, v->data, A->data, out->data, ws, st);
+        if (r != SLRA_OK) return r;
+        const uint8_t* b = static_cast<const uint8_t*>(ws);
+        if ((S && cudaMemcpyAsync(S, b + d.lay.S, s_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess) ||
+            (z && cudaMemcpyAsync(z, b + d.lay.z, z_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess))
+            return SLRA_ERR_CUDA;
+        return SLRA_OK;
+    });
+}
+
+slra_status slra_get_device_status(slra_stream_t stream, int32_t* status) {
+    if (!status) return SLRA_ERR_INVALID_ARG;
+    slra_status s = check_device();
+    if (s != SLRA_OK) return s;
+    int v = 0;
+    const int zero = 0;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&v, slra::g_call_status, sizeof v) != cudaSuccess ||
+        cudaMemcpyToSymbol(slra::g_call_status, &zero, sizeof zero) != cudaSuccess) {
+        cudaGetLastError();
+        return SLRA_ERR_CUDA;
+    }
     *status = (v & kDevTimeout) ? SLRA_ERR_DEVICE_TIMEOUT : ((v & kDevRange) ? SLRA_ERR_RANGE : SLRA_OK);
     return SLRA_OK;
 }

@@ -758,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = tid; e < D * g.R; e += kSoftThreads) As[e] = __bfloat162float(Ah[e]);
             group_sync();
             if (row_valid) {
-                const __nv_bfloat16* qrow = a.q_raw + ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D;
+                const __nv_bfloat16* qrow = a.q_raw + g.sq.row(b, n, h);
                 const float* Sh = a.S + static_cast<size_t>(bh) * g.R * D + hf * DH;
                 const float* zh = a.z + static_cast<size_t>(bh) * g.R;
                 float den = 0.f;

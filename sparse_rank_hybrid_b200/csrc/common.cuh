@@ -15,6 +15,12 @@ constexpr int kMaxPairs = 64;  // head_dim <= 128
 constexpr int kDevTimeout = 1;
 constexpr int kDevRange = 2;
 
+// Element strides (batch, token, head) of a [B][L][Hh][D] tensor whose D elements are contiguous.
+struct Strides {
+    long long b, l, h;
+    __host__ __device__ long long row(int bi, int n, int hi) const { return bi * b + n * l + hi * h; }
+};
+
 // Sizes of one call.  L = T*H*W; Lp = nb*block (rows of the padded head-major buffers).
 struct Geom {
     int B, Hh, D, T, H, W, L, block, nb, keep, R, Lp;
@@ -22,6 +28,7 @@ struct Geom {
     int norope;  // 1: no rotation in the low-rank branch (psi = phi)
     int a_stride;  // elements between consecutive heads' projections (D * R when per head, else 0)
     int inside;    // 1: the low-rank RoPE before the activation (psi = act(R x A), normaliser on psi)
+    Strides sq, sk, sv, so;  // element strides of q, k, v and out
     __host__ __device__ int BH() const { return B * Hh; }
 };
 
@@ -74,8 +81,8 @@ cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, co
                               cudaStream_t st);
 int lowrank_nsplit(const Geom& g);
 bool make_map_headmajor(CUtensorMap* m, const void* base, uint64_t rows, int D, int box_rows);
-bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int D, int box_tokens);
-bool make_map_out(CUtensorMap* m, void* base, int B, int L, int Hh, int D, bool f32);
+bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int D, const Strides& st, int box_tokens);
+bool make_map_out(CUtensorMap* m, void* base, int B, int L, int Hh, int D, const Strides& st, bool f32);
 cudaError_t launch_lowrank_reduce(const float* s_part, const float* z_part, const Geom& g, int nsplit, float* S,
                                   float* z, const __nv_bfloat16* A, uint8_t* at_img, uint8_t* sb_img, cudaStream_t st);
 

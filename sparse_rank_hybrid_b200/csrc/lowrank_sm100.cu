@@ -428,7 +428,8 @@ cudaError_t launch_lowrank_tc(const __nv_bfloat16* k, const __nv_bfloat16* v, co
                               float* z_part, int* status, unsigned long long timeout_ns, int debug_unsatisfied_wait,
                               cudaStream_t st) {
     CUtensorMap tk, tv;
-    if (!make_map_tokens(&tk, k, g.B, g.L, g.Hh, g.D, kTok) || !make_map_tokens(&tv, v, g.B, g.L, g.Hh, g.D, kTok))
+    if (!make_map_tokens(&tk, k, g.B, g.L, g.Hh, g.D, g.sk, kTok) ||
+        !make_map_tokens(&tv, v, g.B, g.L, g.Hh, g.D, g.sv, kTok))
         return cudaErrorInvalidValue;
     LrArgs a;
     a.A = A;

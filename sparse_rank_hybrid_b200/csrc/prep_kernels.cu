@@ -447,9 +447,8 @@ __global__ void __launch_bounds__(256) lowrank_partial_kernel(const __nv_bfloat1
             const int n = n0 + tt;
             float2 kf = make_float2(0.f, 0.f), vf = make_float2(0.f, 0.f);
             if (n < g.L) {
-                const size_t src = ((static_cast<size_t>(b) * g.L + n) * g.Hh + h) * D + 2 * dp;
-                kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + src));
-                vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + src));
+                kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + g.sk.row(b, n, h) + 2 * dp));
+                vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + g.sv.row(b, n, h) + 2 * dp));
             }
             ks[tt * (D + 1) + 2 * dp] = kf.x; ks[tt * (D + 1) + 2 * dp + 1] = kf.y;
             vs[tt * D + 2 * dp] = vf.x; vs[tt * D + 2 * dp + 1] = vf.y;

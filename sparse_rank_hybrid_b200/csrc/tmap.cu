@@ -41,15 +41,17 @@ bool make_map_headmajor(CUtensorMap* m, const void* base, uint64_t rows, int D, 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 4D bf16 map over a token-major [B][L][Hh][D] input: coordinates (d, head, token, batch), box
-// 64 x 1 x box_tokens x 1, 128-B swizzle; tokens past L read as zero.
-bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int D, int box_tokens) {
+// 4D bf16 map over a [B][L][Hh][D] input with element strides st (D contiguous; token-major when
+// contiguous): coordinates (d, head, token, batch), box 64 x 1 x box_tokens x 1, 128-B swizzle; tokens
+// past L read as zero.
+bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int D, const Strides& st,
+                     int box_tokens) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hh), static_cast<cuuint64_t>(L),
                           static_cast<cuuint64_t>(B)};
-    cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hh) * D * 2,
-                             static_cast<cuuint64_t>(L) * Hh * D * 2};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.h) * 2, static_cast<cuuint64_t>(st.l) * 2,
+                             static_cast<cuuint64_t>(st.b) * 2};
     cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_tokens), 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -57,16 +59,17 @@ bool make_map_tokens(CUtensorMap* m, const void* base, int B, int L, int Hh, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 4D map over the output [B][L][Hh][D] for 64-token TMA stores of 128-byte column boxes (32 fp32 or 64
-// bf16 columns), 128-B swizzle on the shared-memory side; tokens past L are not written.
-bool make_map_out(CUtensorMap* m, void* base, int B, int L, int Hh, int D, bool f32) {
+// 4D map over the output [B][L][Hh][D] (element strides st, D contiguous) for 64-token TMA stores of
+// 128-byte column boxes (32 fp32 or 64 bf16 columns), 128-B swizzle on the shared-memory side; tokens
+// past L are not written.
+bool make_map_out(CUtensorMap* m, void* base, int B, int L, int Hh, int D, const Strides& st, bool f32) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t es = f32 ? 4 : 2;
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hh), static_cast<cuuint64_t>(L),
                           static_cast<cuuint64_t>(B)};
-    cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * es, static_cast<cuuint64_t>(Hh) * D * es,
-                             static_cast<cuuint64_t>(L) * Hh * D * es};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.h) * es, static_cast<cuuint64_t>(st.l) * es,
+                             static_cast<cuuint64_t>(st.b) * es};
     cuuint32_t box[4] = {f32 ? 32u : 64u, 1, 64, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides,

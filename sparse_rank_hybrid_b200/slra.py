@@ -20,14 +20,16 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DE
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
 DEBUG_UNSATISFIED_WAIT = 1
-ABI_VERSION = 5
+ABI_VERSION = 6
+DTYPE_BF16, DTYPE_F32 = 0, 1
 ACT_RELU, ACT_SILU, ACT_IDENTITY, ACT_TANH = 0, 1, 2, 3
 FUSION_SUM, FUSION_GATED = 0, 1
 
 # Every symbol include/slra.h declares.
 EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_validate", "slra_keep_count",
-           "slra_projection_elems",
-           "slra_workspace_layout", "slra_attn_fwd", "slra_host_io_bytes", "slra_host_pipeline_groups",
+           "slra_projection_elems", "slra_workspace_bytes", "slra_attn_fwd", "slra_attn_fwd_ex", "slra_sparse_fwd",
+           "slra_lowrank_fwd", "slra_get_device_status",
+           "slra_workspace_layout", "slra_host_io_bytes", "slra_host_pipeline_groups",
            "slra_attn_fwd_host",
            "slra_select_blocks", "slra_lowrank_summary", "slra_device_status", "slra_lowrank_summary_noalloc",
            "slra_noalloc_device_status")
@@ -49,7 +51,19 @@ class _Problem(ctypes.Structure):
                 ("stage_events", ctypes.c_void_p * 7), ("activation", ctypes.c_int32),
                 ("lowrank_norope", ctypes.c_int32), ("proj_separate", ctypes.c_int32),
                 ("proj_per_head", ctypes.c_int32), ("fusion", ctypes.c_int32), ("gate_bias", ctypes.c_float),
-                ("gate_w", ctypes.c_void_p), ("lowrank_rope_inside", ctypes.c_int32)]
+                ("gate_w", ctypes.c_void_p), ("lowrank_rope_inside", ctypes.c_int32),
+                ("q_strides", ctypes.c_int64 * 3), ("k_strides", ctypes.c_int64 * 3),
+                ("v_strides", ctypes.c_int64 * 3), ("out_strides", ctypes.c_int64 * 3)]
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("B", ctypes.c_int64), ("L", ctypes.c_int64),
+                ("Hh", ctypes.c_int64), ("D", ctypes.c_int64), ("sB", ctypes.c_int64), ("sL", ctypes.c_int64),
+                ("sH", ctypes.c_int64)]
+
+
+class _Mat(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("D", ctypes.c_int64), ("R", ctypes.c_int64)]
 
 
 class _Layout(ctypes.Structure):
@@ -84,7 +98,14 @@ def lib():
         L.slra_projection_elems.restype = ctypes.c_int64
         L.slra_projection_elems.argtypes = [PP]
         L.slra_workspace_layout.argtypes = [PP, ctypes.POINTER(_Layout)]
-        L.slra_attn_fwd.argtypes = [PP, P, P, P, P, P, P, S, P]
+        L.slra_attn_fwd_ex.argtypes = [PP, P, P, P, P, P, P, S, P]
+        PT, PM, I64, C = ctypes.POINTER(_Tensor), ctypes.POINTER(_Mat), ctypes.c_int64, ctypes.c_int
+        L.slra_workspace_bytes.restype = S
+        L.slra_workspace_bytes.argtypes = [I64] * 7 + [ctypes.c_float, I64]
+        L.slra_attn_fwd.argtypes = [PT, PT, PT, PM, C, C, C, C, ctypes.c_float, C, PT, P]
+        L.slra_sparse_fwd.argtypes = [PT, PT, PT, C, C, C, C, ctypes.c_float, PT, P, S, P]
+        L.slra_lowrank_fwd.argtypes = [PT, PT, PT, PM, C, C, C, C, PT, P, P, P, S, P]
+        L.slra_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
         L.slra_host_io_bytes.restype = S
         L.slra_host_io_bytes.argtypes = [PP]
         L.slra_host_pipeline_groups.restype = ctypes.c_int64
@@ -96,6 +117,7 @@ def lib():
         L.slra_lowrank_summary_noalloc.argtypes = [PP, P, P, P, P, P, P]
         L.slra_noalloc_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
         for name in ("slra_problem_init", "slra_validate", "slra_workspace_layout", "slra_attn_fwd",
+                     "slra_attn_fwd_ex", "slra_sparse_fwd", "slra_lowrank_fwd", "slra_get_device_status",
                      "slra_attn_fwd_host", "slra_select_blocks", "slra_lowrank_summary", "slra_device_status",
                      "slra_lowrank_summary_noalloc", "slra_noalloc_device_status"):
             getattr(L, name).restype = ctypes.c_int
@@ -139,6 +161,10 @@ class Problem:
     gate_bias: float = 0.0             # bg of the gated fusion
     gate_w: object = None              # Wg of the gated fusion: CUDA fp32 tensor [head_dim] (or None)
     lowrank_rope_inside: int = 0       # 1: the low-rank RoPE before the activation
+    q_strides: tuple = (0, 0, 0)       # (sB, sL, sH) element strides; all 0 = contiguous [B, L, Hh, D]
+    k_strides: tuple = (0, 0, 0)
+    v_strides: tuple = (0, 0, 0)
+    out_strides: tuple = (0, 0, 0)
 
     @property
     def L(self) -> int:
@@ -168,6 +194,8 @@ class Problem:
         p.fusion = int(self.fusion)
         p.gate_bias = float(self.gate_bias)
         p.lowrank_rope_inside = int(self.lowrank_rope_inside)
+        for name in ("q_strides", "k_strides", "v_strides", "out_strides"):
+            getattr(p, name)[:] = [int(x) for x in getattr(self, name)]
         if self.gate_w is not None:
             t = self.gate_w
             torch = _torch()
@@ -242,22 +270,94 @@ def _check_bf16(name, t, shape):
                          f"{t.dtype} {tuple(t.shape)} on {t.device}")
 
 
-def attn_fwd(prob: Problem, q, k, v, A, out=None, workspace=None, stream=None):
-    """Full forward pass.  q, k, v: CUDA bf16 [B, L, Hh, D]; A: CUDA bf16 of prob.projection_shape.
-    Returns (out, workspace); out is fp32 or bf16 [B, L, Hh, D] as prob.out_dtype."""
+def _row_strides(name, t, shape, dtype):
+    """(sB, sL, sH) element strides of a [B, L, Hh, D] CUDA tensor whose last dimension is contiguous;
+    (0, 0, 0) when the whole tensor is contiguous."""
+    if t.dtype != dtype or not t.is_cuda or tuple(t.shape) != tuple(shape) or t.stride(3) != 1:
+        raise ValueError(f"{name}: expected a CUDA {dtype} tensor of shape {tuple(shape)} with a contiguous last "
+                         f"dimension, got {t.dtype} {tuple(t.shape)} strides {t.stride()} on {t.device}")
+    return (0, 0, 0) if t.is_contiguous() else (t.stride(0), t.stride(1), t.stride(2))
+
+
+def attn_fwd(prob: Problem, q, k, v, A, out=None, workspace=None, stream=None, alloc_workspace_in_library=False):
+    """Full forward pass through slra_attn_fwd_ex.  q, k, v: CUDA bf16 [B, L, Hh, D] with a contiguous
+    last dimension (any other strides, e.g. views of a fused QKV tensor); A: CUDA bf16 of
+    prob.projection_shape.  Returns (out, workspace); out is fp32 or bf16 [B, L, Hh, D] as
+    prob.out_dtype (a given out may be strided too).  alloc_workspace_in_library=True passes a NULL
+    workspace (the library allocates it on the stream) and returns None for it."""
+    import dataclasses
     torch = _torch()
     shp = (prob.batch, prob.L, prob.heads, prob.head_dim)
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _check_bf16(n, t, shp)
-    _check_bf16("A", A, prob.projection_shape)
+    odt = torch.float32 if prob.out_dtype == OUT_F32 else torch.bfloat16
     if out is None:
-        out = torch.empty(shp, dtype=torch.float32 if prob.out_dtype == OUT_F32 else torch.bfloat16,
-                          device=q.device)
-    if workspace is None:
-        workspace = alloc_workspace(prob, q.device)
-    _check(lib().slra_attn_fwd(ctypes.byref(prob.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(A), _ptr(out),
-                               _ptr(workspace), workspace.numel(), _stream_handle(stream)), "slra_attn_fwd")
+        out = torch.empty(shp, dtype=odt, device=q.device)
+    strides = {f"{n}_strides": _row_strides(n, t, shp, dt) for n, t, dt in
+               (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16), ("out", out, odt))}
+    if prob.branches & BRANCH_LOWRANK or A is not None:
+        _check_bf16("A", A, prob.projection_shape)
+    p = dataclasses.replace(prob, **strides)
+    if workspace is None and not alloc_workspace_in_library:
+        workspace = alloc_workspace(p, q.device)
+    ws_ptr, ws_n = (0, 0) if workspace is None else (_ptr(workspace), workspace.numel())
+    _check(lib().slra_attn_fwd_ex(ctypes.byref(p.c()), _ptr(q), _ptr(k), _ptr(v), 0 if A is None else _ptr(A),
+                                  _ptr(out), ws_ptr or None, ws_n, _stream_handle(stream)), "slra_attn_fwd_ex")
     return out, workspace
+
+
+def _tensor(t, dtype_code) -> _Tensor:
+    """Descriptor of a [B, L, Hh, D] CUDA tensor (strides in elements; the last dimension contiguous)."""
+    if t.dim() != 4 or t.stride(3) != 1 or not t.is_cuda:
+        raise ValueError("expected a CUDA [B, L, Hh, D] tensor with a contiguous last dimension")
+    return _Tensor(_ptr(t), dtype_code, *t.shape, t.stride(0), t.stride(1), t.stride(2))
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    return {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[t.dtype]
+
+
+def workspace_bytes(batch, heads, head_dim, T, H, W, block, keep_frac, rank) -> int:
+    return int(lib().slra_workspace_bytes(batch, heads, head_dim, T, H, W, block, float(keep_frac), rank))
+
+
+def attn_fwd_tensors(q, k, v, A, T, H, W, block, keep_frac, rank, out, stream=None):
+    """slra_attn_fwd: the forward pass from tensor descriptors (strides taken from the tensors), the
+    workspace allocated by the library on the stream."""
+    a = _Mat(_ptr(A), DTYPE_BF16 if A.dtype == _torch().bfloat16 else DTYPE_F32, A.shape[0], A.shape[1])
+    tq, tk, tv, to = (_tensor(t, _dtype_code(t)) for t in (q, k, v, out))
+    _check(lib().slra_attn_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), ctypes.byref(a), T, H, W,
+                               block, float(keep_frac), rank, ctypes.byref(to), _stream_handle(stream)),
+           "slra_attn_fwd")
+    return out
+
+
+def sparse_fwd(q, k, v, T, H, W, block, keep_frac, out, workspace=None, stream=None):
+    """slra_sparse_fwd: the sparse branch alone into out (workspace None = allocated by the library)."""
+    tq, tk, tv, to = (_tensor(t, _dtype_code(t)) for t in (q, k, v, out))
+    ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel())
+    _check(lib().slra_sparse_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), T, H, W, block,
+                                 float(keep_frac), ctypes.byref(to), ws_ptr, ws_n, _stream_handle(stream)),
+           "slra_sparse_fwd")
+    return out
+
+
+def lowrank_fwd(q, k, v, A, T, H, W, rank, out, S=None, z=None, workspace=None, stream=None):
+    """slra_lowrank_fwd: the low-rank branch alone into out; S, z (fp32 CUDA) receive the summary."""
+    a = _Mat(_ptr(A), DTYPE_BF16, A.shape[0], A.shape[1])
+    tq, tk, tv, to = (_tensor(t, _dtype_code(t)) for t in (q, k, v, out))
+    ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel())
+    _check(lib().slra_lowrank_fwd(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), ctypes.byref(a), T, H, W,
+                                  rank, ctypes.byref(to), None if S is None else _ptr(S),
+                                  None if z is None else _ptr(z), ws_ptr, ws_n, _stream_handle(stream)),
+           "slra_lowrank_fwd")
+    return out
+
+
+def get_device_status(stream=None) -> int:
+    """Read and clear the device status of the calls whose workspace the library allocated."""
+    st = ctypes.c_int32(-1)
+    _check(lib().slra_get_device_status(_stream_handle(stream), ctypes.byref(st)), "slra_get_device_status")
+    return int(st.value)
 
 
 def host_io_bytes(prob: Problem) -> int:

@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_abi_version_and_status_strings():
-    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 5
+    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 6
     for s in range(0, 9):
         assert slra.status_string(s) and slra.status_string(s) != "unknown status"
     assert slra.status_string(99) == "unknown status"
@@ -145,6 +145,76 @@ def test_calls_without_device_fail_cleanly():
     import ctypes
     buf = ctypes.create_string_buffer(lay.total_bytes + 512)
     base = (ctypes.addressof(buf) + 255) // 256 * 256
-    s = slra.lib().slra_attn_fwd(ctypes.byref(p.c()), base, base, base, base, base + 256, base, lay.total_bytes,
-                                 None)
+    s = slra.lib().slra_attn_fwd_ex(ctypes.byref(p.c()), base, base, base, base, base + 256, base, lay.total_bytes,
+                                    None)
     assert s != slra.OK
+    # descriptor-style entry points: well-formed, disjoint host pointers reach the device check
+    n = W.TINY.batch * W.TINY.L * W.TINY.heads * W.TINY.head_dim
+    bufs = [ctypes.create_string_buffer(n * 4 + 256) for _ in range(4)]
+    ptrs = [(ctypes.addressof(b) + 255) // 256 * 256 for b in bufs]
+    t = [slra._Tensor(ptrs[i], slra.DTYPE_BF16, 1, W.TINY.L, W.TINY.heads, W.TINY.head_dim, 0, 0, 0) for i in range(3)]
+    o = slra._Tensor(ptrs[3], slra.DTYPE_F32, 1, W.TINY.L, W.TINY.heads, W.TINY.head_dim, 0, 0, 0)
+    a_buf = ctypes.create_string_buffer(64 * 16 * 2 + 256)
+    a = slra._Mat((ctypes.addressof(a_buf) + 255) // 256 * 256, slra.DTYPE_BF16, 64, 16)
+    args = (4, 8, 8)
+    assert slra.lib().slra_attn_fwd(*(ctypes.byref(x) for x in t), ctypes.byref(a), *args, 64, 0.5, 16,
+                                    ctypes.byref(o), None) == slra.ERR_NO_DEVICE
+    assert slra.lib().slra_sparse_fwd(*(ctypes.byref(x) for x in t), *args, 64, 0.5, ctypes.byref(o), None, 0,
+                                      None) == slra.ERR_NO_DEVICE
+    assert slra.lib().slra_lowrank_fwd(*(ctypes.byref(x) for x in t), ctypes.byref(a), *args, 16, ctypes.byref(o),
+                                       None, None, None, 0, None) == slra.ERR_NO_DEVICE
+    st = ctypes.c_int32(-1)
+    assert slra.lib().slra_get_device_status(None, ctypes.byref(st)) == slra.ERR_NO_DEVICE
+    # invalid descriptors are rejected before the device is looked at
+    bad_L = slra._Tensor(ptrs[0], slra.DTYPE_BF16, 1, W.TINY.L + 1, W.TINY.heads, W.TINY.head_dim, 0, 0, 0)
+    assert slra.lib().slra_attn_fwd(ctypes.byref(bad_L), ctypes.byref(t[1]), ctypes.byref(t[2]), ctypes.byref(a),
+                                    *args, 64, 0.5, 16, ctypes.byref(o), None) == slra.ERR_INVALID_ARG
+    f32_q = slra._Tensor(ptrs[0], slra.DTYPE_F32, 1, W.TINY.L, W.TINY.heads, W.TINY.head_dim, 0, 0, 0)
+    assert slra.lib().slra_attn_fwd(ctypes.byref(f32_q), ctypes.byref(t[1]), ctypes.byref(t[2]), ctypes.byref(a),
+                                    *args, 64, 0.5, 16, ctypes.byref(o), None) == slra.ERR_INVALID_ARG
+    a_rank = slra._Mat(a.data, slra.DTYPE_BF16, 64, 32)
+    assert slra.lib().slra_attn_fwd(*(ctypes.byref(x) for x in t), ctypes.byref(a_rank), *args, 64, 0.5, 16,
+                                    ctypes.byref(o), None) == slra.ERR_INVALID_ARG
+    alias = slra._Tensor(ptrs[0], slra.DTYPE_F32, 1, W.TINY.L, W.TINY.heads, W.TINY.head_dim, 0, 0, 0)
+    assert slra.lib().slra_attn_fwd(*(ctypes.byref(x) for x in t), ctypes.byref(a), *args, 64, 0.5, 16,
+                                    ctypes.byref(alias), None) == slra.ERR_INVALID_ARG
+
+
+def test_workspace_bytes_matches_layout():
+    for w in (W.TINY, W.WAN_1_3B, W.WAN_14B, W.HUNYUAN):
+        assert slra.workspace_bytes(w.batch, w.heads, w.head_dim, w.T, w.H, w.W, w.block, w.keep_frac, w.rank) == \
+            slra.layout(slra.Problem.from_workload(w)).total_bytes
+    assert slra.workspace_bytes(1, 2, 96, 4, 8, 8, 64, 0.5, 16) == 0  # head_dim 96 is not supported
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("q_strides", (0, 0, 0), slra.OK),
+    ("q_strides", None, slra.OK),                       # fused QKV: [B][L][3][Hh][D] views
+    ("k_strides", "headmajor", slra.OK),                # [B][Hh][L][D] input
+    ("v_strides", (8, 8, 8), slra.OK),                  # inputs may alias (read only)
+    ("q_strides", (0, 0, 4), slra.ERR_INVALID_ARG),     # not a multiple of 8 elements
+    ("q_strides", (0, 512, 64), slra.ERR_INVALID_ARG),  # zero stride with others set
+    ("out_strides", (0, 0, 0), slra.OK),
+    ("out_strides", "headmajor", slra.OK),
+    ("out_strides", "padded", slra.OK),                 # rows padded to 96 fp32
+    ("out_strides", (8, 8, 8), slra.ERR_INVALID_ARG),   # output rows overlap
+    ("out_strides", "shortrow", slra.ERR_INVALID_ARG),  # head stride below D: rows overlap
+])
+def test_stride_validation(field, value, status):
+    w = W.TINY
+    L, Hh, D = w.L, w.heads, w.head_dim
+    spec = {None: (L * 3 * Hh * D, 3 * Hh * D, D), "headmajor": (Hh * L * D, D, L * D),
+            "padded": (L * Hh * 96, Hh * 96, 96), "shortrow": (L * Hh * 32, Hh * 32, 32)}
+    p = slra.Problem.from_workload(w, **{field: spec.get(value, value) if not isinstance(value, tuple) else value})
+    assert slra.validate(p) == status
+
+
+def test_host_entry_point_rejects_strides():
+    import ctypes
+    p = slra.Problem.from_workload(W.TINY, q_strides=(W.TINY.L * 3 * 128, 3 * 128, 64))
+    assert slra.validate(p) == slra.OK
+    b = ctypes.create_string_buffer(1 << 20)
+    base = (ctypes.addressof(b) + 255) // 256 * 256
+    s = slra.lib().slra_attn_fwd_host(ctypes.byref(p.c()), base, base, base, base, base, base, 1 << 19, base,
+                                      1 << 19, None)
+    assert s == slra.ERR_INVALID_ARG
