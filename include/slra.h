@@ -316,6 +316,39 @@ SLRA_API slra_status slra_lowrank_fwd(const slra_tensor* q, const slra_tensor* k
                                       float* z, void* workspace, size_t workspace_bytes, slra_stream_t stream);
 
 /*
+ * Workspace bytes of slra_attn_bwd for p (the forward's layout followed by the backward's sections: the
+ * recomputed sparse output and its per-row log-sum-exp, an fp16 copy of dout, the inverted kept-block
+ * lists and the low-rank gradient partial sums); 0 if p is invalid or asks for an option the backward
+ * does not cover.  No GPU access.
+ */
+SLRA_API size_t slra_bwd_workspace_bytes(const slra_problem* p);
+
+/*
+ * Backward pass: the gradients of sum(dout * out) with respect to q, k, v and A, where out is the
+ * forward pass of slra_attn_fwd_ex on the same arguments (RoLA "4.5", "E.1", "E.2": the branch's
+ * parameters are trained jointly with the backbone).  The block selection is held at the forward's (it
+ * is piecewise constant in q and k).  Covered: relu features, the low-rank RoPE outside the activation,
+ * one shared projection, the plain sum, any branches mask; other options return SLRA_ERR_UNSUPPORTED.
+ *   q, k, v, A   as for slra_attn_fwd_ex (q, k, v may be strided per p).
+ *   dout         fp32 [B][L][Hh][D] contiguous: the gradient of the loss with respect to out.
+ *   dq, dk, dv   fp32 [B][L][Hh][D] contiguous outputs (p->out_strides must be zero).
+ *   dA           fp32 [D][rank] output (zero when the low-rank branch is off).
+ *   workspace    at least slra_bwd_workspace_bytes(p) bytes, 256-B aligned (the forward's sections are
+ *                refilled by the recompute and can be inspected afterwards).
+ * The sparse branch's gradients run on the tensor cores: a dQ kernel per query block (S = q^ k^T and
+ * dP = dO v^T in TMEM, dS = P (dP - rowsum(dO O_sparse)), dQ^ += dS k^) and a dK/dV kernel per key block
+ * over the query blocks that kept it (dV += P^T dO, dK^ += dS^T q^), with fp16 operands (dout must stay
+ * below 65504 in magnitude, else SLRA_ERR_RANGE is recorded) and fp32 accumulation; the low-rank chain
+ * runs as fp32 passes over the queries and the keys.  Deterministic.  stage_events are recorded at: [0]
+ * start, [1] after the recomputed forward, [2] after the dO copy and the inverted lists, [3] after the dQ
+ * kernel, [4] after the dK/dV kernel, [5] and [6] after the low-rank gradients.  Device problems go to
+ * the workspace's status word (slra_device_status).
+ */
+SLRA_API slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, const void* v,
+                                   const void* A, const float* dout, float* dq, float* dk, float* dv, float* dA,
+                                   void* workspace, size_t workspace_bytes, slra_stream_t stream);
+
+/*
  * Device status of the calls whose workspace the library allocated (slra_attn_fwd, and the others when
  * given a NULL workspace) on the current device: synchronize `stream`, then read and clear the word
  * their status words were ORed into.  *status receives SLRA_OK, SLRA_ERR_DEVICE_TIMEOUT or SLRA_ERR_RANGE.

@@ -628,8 +628,55 @@ slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, con
     a.status = w.status;
     a.timeout_ns = timeout_of(p);
     a.debug_unsatisfied_wait = debug_wait_of(p);
+    a.lse = nullptr;
     if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
     return mark(p, 6, st);
+}
+
+// ---------------------------------------------------------------- backward pass
+// Sections the backward adds after the forward's workspace layout (256-B aligned byte offsets).
+struct BwdLayout {
+    size_t lse, delta, os, doh, inv_cnt, inv, ds_part, dz_part, dS, dz, da_part, total;
+    int ns;  // splits of the low-rank gradient passes
+};
+
+BwdLayout bwd_layout(const Derived& d) {
+    const Geom& g = d.g;
+    BwdLayout b;
+    size_t o = d.lay.total_bytes;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align_up(o + bytes, 256);
+        return at;
+    };
+    const size_t rows = static_cast<size_t>(g.BH()) * g.Lp;
+    b.ns = lr_bwd_nsplit(g);
+    b.lse = take(rows * 4);
+    b.delta = take(rows * 4);
+    b.os = take(rows * g.D * 4);
+    b.doh = take(rows * g.D * 2);
+    b.inv_cnt = take(static_cast<size_t>(g.BH()) * g.nb * 4);
+    b.inv = take(static_cast<size_t>(g.BH()) * g.nb * g.nb * 4);
+    b.ds_part = take(static_cast<size_t>(g.BH()) * b.ns * g.R * g.D * 4);
+    b.dz_part = take(static_cast<size_t>(g.BH()) * b.ns * g.R * 4);
+    b.dS = take(static_cast<size_t>(g.BH()) * g.R * g.D * 4);
+    b.dz = take(static_cast<size_t>(g.BH()) * g.R * 4);
+    b.da_part = take(2 * static_cast<size_t>(g.BH()) * b.ns * g.D * g.R * 4);
+    b.total = o;
+    return b;
+}
+
+// The backward covers the default options: relu features, the low-rank RoPE outside the activation,
+// one shared projection and the plain sum; gradients are contiguous fp32 [B][L][Hh][D].
+slra_status check_bwd_problem(const slra_problem* p, Derived* d) {
+    slra_status s = derive(p, d);
+    if (s != SLRA_OK) return s;
+    if (p->activation != SLRA_ACT_RELU || p->lowrank_norope || p->lowrank_rope_inside || p->proj_separate ||
+        p->proj_per_head || p->fusion != SLRA_FUSION_SUM)
+        return SLRA_ERR_UNSUPPORTED;
+    for (int i = 0; i < 3; ++i)
+        if (p->out_strides[i]) return SLRA_ERR_INVALID_ARG;
+    return SLRA_OK;
 }
 
 // A problem description from the tensor descriptors of the descriptor-style entry points.
@@ -890,6 +937,151 @@ slra_status slra_lowrank_fwd(const slra_tensor* q, const slra_tensor* k, const s
             return SLRA_ERR_CUDA;
         return SLRA_OK;
     });
+}
+
+size_t slra_bwd_workspace_bytes(const slra_problem* p) {
+    Derived d;
+    return check_bwd_problem(p, &d) == SLRA_OK ? bwd_layout(d).total : 0;
+}
+
+slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
+                          const float* dout, float* dq, float* dk, float* dv, float* dA, void* workspace,
+                          size_t workspace_bytes, slra_stream_t stream) {
+    Derived d;
+    slra_status s = check_bwd_problem(p, &d);
+    if (s != SLRA_OK) return s;
+    const int branches = p->branches == 0 ? SLRA_BRANCH_BOTH : p->branches;
+    const bool lowrank = (branches & SLRA_BRANCH_LOWRANK) != 0, sparse = (branches & SLRA_BRANCH_SPARSE) != 0;
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || !dA || (lowrank && !A)) return SLRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (A && !aligned16(A)) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dA))
+        return SLRA_ERR_ALIGNMENT;
+    const Geom& g = d.g;
+    const BwdLayout bl = bwd_layout(d);
+    const size_t gb = qkv_bytes(d) * 2, ab = static_cast<size_t>(g.D) * g.R * 4;  // fp32 gradient bytes
+    const void* outs[4] = {dq, dk, dv, dA};
+    const size_t out_n[4] = {gb, gb, gb, ab};
+    const void* ins[5] = {q, k, v, A, dout};
+    const size_t in_n[5] = {span_bytes(g, g.sq, 2), span_bytes(g, g.sk, 2), span_bytes(g, g.sv, 2), d.a_elems * 2, gb};
+    for (int i = 0; i < 4; ++i) {
+        for (int j = 0; j < 5; ++j)
+            if (ins[j] && overlaps(outs[i], out_n[i], ins[j], in_n[j])) return SLRA_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 4; ++j)
+            if (overlaps(outs[i], out_n[i], outs[j], out_n[j])) return SLRA_ERR_INVALID_ARG;
+        if (workspace && overlaps(outs[i], out_n[i], workspace, workspace_bytes)) return SLRA_ERR_INVALID_ARG;
+    }
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < bl.total)
+        return SLRA_ERR_WORKSPACE;
+    if ((s = check_device()) != SLRA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const Ptrs w = carve(workspace, d);
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    float* lse = reinterpret_cast<float*>(base + bl.lse);
+    float* delta = reinterpret_cast<float*>(base + bl.delta);
+    float* os = reinterpret_cast<float*>(base + bl.os);
+    __half* doh = reinterpret_cast<__half*>(base + bl.doh);
+    int32_t* inv_cnt = reinterpret_cast<int32_t*>(base + bl.inv_cnt);
+    int32_t* inv = reinterpret_cast<int32_t*>(base + bl.inv);
+    // the recompute runs the forward's stages without recording the caller's events
+    slra_problem pr = *p;
+    for (auto& e : pr.stage_events) e = nullptr;
+
+    if ((s = mark(p, 0, st)) != SLRA_OK) return s;
+    if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return SLRA_ERR_CUDA;
+    if ((s = cuda_status(launch_rope_table(w.tab, w.pairs, d.meta, d.table_entries, st))) != SLRA_OK) return s;
+    if (sparse && (s = run_select(&pr, d, w, q, k, v, st)) != SLRA_OK) return s;
+    if (lowrank && (s = run_lowrank(&pr, d, w, k, v, A, st)) != SLRA_OK) return s;
+    if (sparse) {
+        // the sparse forward again, writing its output O_s (head-major fp32) and each row's lse
+        AttnMaps maps;
+        const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
+        const Strides os_st{static_cast<long long>(g.Hh) * g.Lp * g.D, g.D, static_cast<long long>(g.Lp) * g.D};
+        if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) ||
+            !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
+            !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
+            !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, g.sq, 128) ||
+            !make_map_out(&maps.out, os, g.B, g.L, g.Hh, g.D, os_st, true))
+            return SLRA_ERR_CUDA;
+        AttnArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.qh = w.qh;
+        a.kh = w.kh;
+        a.vh = w.vh;
+        a.idx = w.idx;
+        a.keep = g.keep;
+        a.q_raw = static_cast<const __nv_bfloat16*>(q);
+        a.tab = w.tab;
+        a.pairs = w.pairs;
+        a.lowrank = 0;
+        a.out = os;
+        a.status = w.status;
+        a.timeout_ns = timeout_of(p);
+        a.lse = lse;
+        if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
+    }
+    if ((s = mark(p, 1, st)) != SLRA_OK) return s;
+    if (sparse) {
+        if ((s = cuda_status(launch_bwd_prep(dout, os, g, doh, delta, w.status, st))) != SLRA_OK) return s;
+        if ((s = cuda_status(launch_bwd_invert(w.idx, g, inv, inv_cnt, st))) != SLRA_OK) return s;
+        if ((s = mark(p, 2, st)) != SLRA_OK) return s;
+        BwdMaps m;
+        const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
+        if (!make_map_headmajor(&m.q128, w.qh, rows, g.D, 128) || !make_map_headmajor(&m.do128, doh, rows, g.D, 128) ||
+            !make_map_headmajor(&m.kb, w.kh, rows, g.D, g.block) || !make_map_headmajor(&m.vb, w.vh, rows, g.D, g.block) ||
+            !make_map_headmajor(&m.k128, w.kh, rows, g.D, 128) || !make_map_headmajor(&m.v128, w.vh, rows, g.D, 128) ||
+            !make_map_headmajor(&m.qb, w.qh, rows, g.D, g.block) || !make_map_headmajor(&m.dob, doh, rows, g.D, g.block))
+            return SLRA_ERR_CUDA;
+        m.between = static_cast<cudaEvent_t>(p->stage_events[3]);
+        BwdArgs ba;
+        ba.idx = w.idx;
+        ba.keep = g.keep;
+        ba.inv = inv;
+        ba.inv_cnt = inv_cnt;
+        ba.lse = lse;
+        ba.delta = delta;
+        ba.tab = w.tab;
+        for (int e = 0; e < kMaxPairs; ++e)
+            ba.pair_info[e] = e < d.meta.npairs ? make_int2(d.meta.axis[e], d.meta.tab_off[e]) : make_int2(0, 0);
+        ba.dq = dq;
+        ba.dk = dk;
+        ba.dv = dv;
+        ba.status = w.status;
+        ba.timeout_ns = timeout_of(p);
+        if ((s = cuda_status(launch_bwd_sparse(m, ba, g, st))) != SLRA_OK) return s;
+    } else {
+        if (cudaMemsetAsync(dq, 0, gb, st) != cudaSuccess || cudaMemsetAsync(dk, 0, gb, st) != cudaSuccess ||
+            cudaMemsetAsync(dv, 0, gb, st) != cudaSuccess)
+            return SLRA_ERR_CUDA;
+        if ((s = mark(p, 2, st)) != SLRA_OK || (s = mark(p, 3, st)) != SLRA_OK) return s;
+    }
+    if ((s = mark(p, 4, st)) != SLRA_OK) return s;
+    if (lowrank) {
+        LrBwdArgs l;
+        l.q = static_cast<const __nv_bfloat16*>(q);
+        l.k = static_cast<const __nv_bfloat16*>(k);
+        l.v = static_cast<const __nv_bfloat16*>(v);
+        l.A = static_cast<const __nv_bfloat16*>(A);
+        l.dout = dout;
+        l.S = w.S;
+        l.z = w.z;
+        l.tab = w.tab;
+        l.pairs = w.pairs;
+        l.dq = dq;
+        l.dk = dk;
+        l.dv = dv;
+        l.dA = dA;
+        l.ds_part = reinterpret_cast<float*>(base + bl.ds_part);
+        l.dz_part = reinterpret_cast<float*>(base + bl.dz_part);
+        l.da_part = reinterpret_cast<float*>(base + bl.da_part);
+        l.dS = reinterpret_cast<float*>(base + bl.dS);
+        l.dz = reinterpret_cast<float*>(base + bl.dz);
+        l.nsplit = bl.ns;
+        if ((s = cuda_status(launch_lr_bwd(l, g, st))) != SLRA_OK) return s;
+    } else if (cudaMemsetAsync(dA, 0, ab, st) != cudaSuccess) {
+        return SLRA_ERR_CUDA;
+    }
+    if ((s = mark(p, 5, st)) != SLRA_OK) return s;
+    return mark(p, 6, st);
 }
 
 slra_status slra_get_device_status(slra_stream_t stream, int32_t* status) {

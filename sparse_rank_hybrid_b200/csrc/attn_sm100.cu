@@ -97,21 +97,6 @@ __device__ __forceinline__ bool group_sync_or(bool pred) {
     return r != 0;
 }
 
-__device__ __forceinline__ void reg_fence(uint32_t (&r)[16]) {
-    asm volatile(""
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                   "+r"(r[15]));
-}
-__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
-    asm volatile(""
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
-                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
-                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -232,6 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     float l_run = 0.f;
+    // m_run is the row's running max (identical in both halves); l_run sums this half's keys only.
+    float m_run = 0.f;
     if (warp == kWarpLoad) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0 && keep > 0 && !*abort_flag) {
@@ -383,8 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // only be the last one visited.
         const int last_valid = keep > 0 ? min(blk, g.L - __ldg(my_idx + keep - 1) * blk) : blk;
         const int key0 = hf * HW;  // first key of this thread's half of the block
-        // m_run is the row's running max (identical in both halves); l_run sums this half's keys only.
-        float m_run = 0.f;
         for (int j = 0; j < keep; ++j) {
             const int sb = j % kNumS;
             const uint32_t tSj = tmem + sb * 128;
@@ -494,6 +479,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     xch[hf * 128 + i_row] = l_run;
     group_sync();
     l_run += xch[(hf ^ 1) * 128 + i_row];
+    // the softmax's log-sum-exp per row (log2 units), for a backward pass; rows past L get +inf so that
+    // their probabilities recompute as zero
+    if (a.lse != nullptr && hf == 0 && i_row < blk && keep > 0) {
+        const int n_row = alpha * blk + i_row;
+        a.lse[static_cast<size_t>(bh) * g.Lp + n_row] =
+            n_row < g.L ? m_run + log2f(l_run) : INFINITY;
+    }
     // The producer and MMA warps may raise the abort flag at any time, so every decision that picks a
     // path through the group barriers is taken from one reduction.
     const bool aborted = group_sync_or(*abort_flag != 0);  // also: the exchange buffer is reused below

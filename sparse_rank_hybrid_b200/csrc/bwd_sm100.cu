@@ -1,0 +1,995 @@
+// Backward pass of the hybrid attention (relu features, RoPE outside the activation, one shared
+// projection A, plain sum of the branches): gradients of sum(dO * out) with respect to q, k, v and A,
+// the block selection held at the forward's (it is piecewise constant in q and k).
+//
+// Method: the derivative of the forward of RoLA "4.1" (block-sparse softmax attention over the kept
+// key blocks plus the low-rank branch), "4.2"/"4.3" (truncated RoPE outside the relu feature map) and
+// "B.1" (one query-independent summary per head); RoLA "4.5" and "E.1"/"E.2" train the branch's
+// parameters jointly with the backbone, which needs these gradients.
+//
+// Sparse branch (per query row i over its allowed keys j; lse and O_s from the forward):
+//   P_ij = 2^(s_ij log2(e)/sqrt(D) - lse_i),  Delta_i = dO_i . O_s,i,  dP_ij = dO_i . v_j,
+//   dS_ij = P_ij (dP_ij - Delta_i),  dq^_i = sum_j dS_ij k^_j / sqrt(D),  dk^_j = sum_i dS_ij q^_i / sqrt(D),
+//   dv_j = sum_i P_ij dO_i,  dq = R(p)^T dq^,  dk = R(p)^T dk^.
+//   bwd_dq_kernel      one CTA per (query block, head): S = q^ k^T and dP = dO v^T per kept key block
+//                      into TMEM, the softmax warps form dS (fp16) over S's columns, dQ^ += dS k^ is
+//                      accumulated in TMEM (tcgen05.mma kind::f16, operands fp16 in shared memory by TMA).
+//   bwd_dkdv_kernel    one CTA per (key block, head), over the query blocks that kept it (inverted
+//                      lists, ascending): S^T = k^ q^T and dP^T = v dO^T into TMEM, P^T and dS^T (fp16)
+//                      over their columns, dV += P^T dO and dK^ += dS^T q^ accumulated in TMEM.  Each
+//                      output row is owned by one CTA: no atomics, deterministic.
+// Low-rank branch (u = x A, phi = relu(u), psi = R_r phi, den_i = phi_q,i . z + 1e-6):
+//   G_i = S dO_i,  dpsi_q,i = G_i / den_i,  dden_i = -(psi_q,i . G_i) / den_i^2,
+//   dphi_q,i = R_r^T dpsi_q,i + dden_i z,  dS = sum_i psi_q,i dO_i^T / den_i,  dz = sum_i dden_i phi_q,i,
+//   dpsi_k,j = dS v_j,  dv_j += dS^T psi_k,j,  dphi_k,j = R_r^T dpsi_k,j + dz,
+//   du = dphi * [u > 0],  dq += du_q A^T,  dk += du_k A^T,  dA = q^T du_q + k^T du_k.
+//   bwd_lr_q_kernel / bwd_lr_k_kernel   CUDA-core fp32 passes over token tiles (split-L partial sums of
+//                      dS, dz and dA, summed in a fixed order).
+//
+// All waits are bounded (see sm100.cuh); a wait that runs out records a timeout in the status word and
+// the CTA drains what it issued and returns.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace slra {
+
+namespace {
+
+constexpr int kBwdMathThreads = 256;  // 8 warps: two per TMEM lane group, each half of the key columns
+constexpr int kBwdThreads = 288;      // + one issuing warp (TMA and tcgen05.mma from its lane 0)
+constexpr int kBwdIssueWarp = 8;
+
+
+__device__ __forceinline__ uint32_t pack_half2_lohi(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// TMEM column (32-bit) of the packed fp16 pair holding keys (columns) 2i, 2i+1 of a 16-key k-step kk,
+// when each half of the threads writes its HW keys packed at the start of its own column range
+// [h*HW, h*HW + HW/2): k-step kk covers keys [16kk, 16kk + 16) of half h = 16kk / HW.
+template <int HW>
+__device__ __forceinline__ uint32_t packed_col(int kk) {
+    const int h = (16 * kk) / HW;
+    return static_cast<uint32_t>(h * HW + (16 * kk - h * HW) / 2);
+}
+
+}  // namespace
+
+
+// Rotate the pairs of this thread's D/2 columns back by R(p)^T and store them (fp32) into a token-major
+// row; `vals` are the 32-bit TMEM words of columns [hf*D/2, hf*D/2 + D/2) of the row, already scaled.
+template <int D>
+__device__ __forceinline__ void store_row_unrotated(float* dst_row, const float* vals, int hf, int n,
+                                                    const BwdArgs& a, const Geom& g, bool rotate) {
+    const int pt = n / (g.H * g.W), ph = (n / g.W) % g.H, pw = n % g.W;
+#pragma unroll
+    for (int t = 0; t < D / 8; ++t) {  // 4 columns (2 pairs) per float4
+        float4 o;
+        float* ov = reinterpret_cast<float*>(&o);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int c = 4 * t + 2 * u;           // column within the half
+            const int pair = (hf * (D / 2) + c) / 2;
+            const float y0 = vals[c], y1 = vals[c + 1];
+            if (rotate) {
+                const int2 pi = a.pair_info[pair];
+                const int pos = pi.x == 0 ? pt : (pi.x == 1 ? ph : pw);
+                const double2 cs = __ldg(a.tab + pi.y + pos);
+                const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+                ov[2 * u] = cf * y0 + sf * y1;       // R^T: rotate back by the pair's angle
+                ov[2 * u + 1] = -sf * y0 + cf * y1;
+            } else {
+                ov[2 * u] = y0;
+                ov[2 * u + 1] = y1;
+            }
+        }
+        *reinterpret_cast<float4*>(dst_row + hf * (D / 2) + 4 * t) = o;
+    }
+}
+
+// ------------------------------------------------------------------------------------------ dQ
+template <int D>
+struct DqLayout {
+    static constexpr int kTile = 128 * D * 2;  // fp16 [128 rows][D] in 64-column slabs
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffDo = kTile;
+    static constexpr int kOffK = 2 * kTile;  // slots s at kOffK + s * kTile
+    static constexpr int kOffV = 4 * kTile;
+    static constexpr int kOffBar = 6 * kTile;
+    static constexpr int kOffMisc = kOffBar + 128;
+    static constexpr int kBytes = kOffMisc + 64;
+};
+
+enum : int { kDqBarQdo = 0, kDqBarKvFull = 1, kDqBarKvEmpty = 3, kDqBarSp = 5, kDqBarDs = 6, kDqBarFinal = 7,
+             kDqBarDrain = 8, kDqNumBars = 9 };
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, BwdArgs a,
+                  Geom g) {
+    using Lay = DqLayout<D>;
+    constexpr int HW = BLK / 2;  // key columns per thread
+    constexpr int NC = HW / 32;
+    constexpr int kSteps = D / 16, kKeySteps = BLK / 16;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int alpha = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int keep = a.keep;
+    const int32_t* my_idx = a.idx + (static_cast<size_t>(bh) * g.nb + alpha) * keep;
+    const int row0 = bh * g.Lp;
+    const uint64_t tmo = a.timeout_ns;
+
+    if (tid == 0) {
+        for (int i = 0; i < kDqNumBars; ++i) mbar_init(bars + i, i == kDqBarDs ? kBwdMathThreads : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
+    auto fail = [&]() {
+        *abort_flag = 1;
+        atomicOr(a.status, kDevTimeout);
+    };
+
+    if (warp == kBwdIssueWarp) {
+        // ------------------------------------------------------------ TMA + tcgen05.mma issuer
+        if (lane == 0 && keep > 0) {
+            auto kslot = [&](int s) { return smem + Lay::kOffK + s * Lay::kTile; };
+            auto vslot = [&](int s) { return smem + Lay::kOffV + s * Lay::kTile; };
+            auto load_rows = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int row, int rows) {
+#pragma unroll
+                for (int sl = 0; sl < D / 64; ++sl) tma_load_2d(dst + sl * (rows * 128), tm, bar, sl * 64, row);
+            };
+            auto load_kv = [&](int j) {
+                const int s = j & 1;
+                mbar_expect_tx(bars + kDqBarKvFull + s, 2u * BLK * D * 2);
+                const int r = row0 + __ldg(my_idx + j) * BLK;
+                load_rows(kslot(s), &tm_k, bars + kDqBarKvFull + s, r, BLK);
+                load_rows(vslot(s), &tm_v, bars + kDqBarKvFull + s, r, BLK);
+            };
+            mbar_expect_tx(bars + kDqBarQdo, 2u * 128 * D * 2);
+            load_rows(smem + Lay::kOffQ, &tm_q, bars + kDqBarQdo, row0 + alpha * BLK, 128);
+            load_rows(smem + Lay::kOffDo, &tm_do, bars + kDqBarQdo, row0 + alpha * BLK, 128);
+            int n_loaded = 0;
+            for (; n_loaded < 2 && n_loaded < keep; ++n_loaded) load_kv(n_loaded);
+            const uint32_t idesc_s = idesc_f16_f32(128, BLK, false, false);
+            const uint32_t idesc_q = idesc_f16_f32(128, D, false, true);
+            const uint32_t q_addr = smem_addr(smem + Lay::kOffQ), do_addr = smem_addr(smem + Lay::kOffDo);
+            // S_j = q^ k^T_j and dP_j = dO v^T_j, both K-major over the head dimension
+            auto issue_sp = [&](int j) {
+                const int s = j & 1;
+                const uint32_t k_addr = smem_addr(kslot(s)), v_addr = smem_addr(vslot(s));
+#pragma unroll
+                for (int kk = 0; kk < kSteps; ++kk) {
+                    const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * (BLK * 128) + (kk & 3) * 32;
+                    umma_ss(tS, sdesc_sw128(q_addr + ao, 16, 1024), sdesc_sw128(k_addr + bo, 16, 1024), idesc_s,
+                            kk > 0 ? 1u : 0u);
+                    umma_ss(tP, sdesc_sw128(do_addr + ao, 16, 1024), sdesc_sw128(v_addr + bo, 16, 1024), idesc_s,
+                            kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bars + kDqBarSp);
+            };
+            bool ok = mbar_wait(bars + kDqBarQdo, 0, tmo, abort_flag) && mbar_wait(bars + kDqBarKvFull, 0, tmo, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_sp(0);
+            }
+            for (int j = 0; j < keep && ok; ++j) {
+                const int s = j & 1;
+                // dQ^ += dS_j k^_j: A = dS_j (fp16, packed over S_j's columns), B = k^_j MN-major
+                if (!mbar_wait(bars + kDqBarDs, j & 1, tmo, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t k_addr = smem_addr(kslot(s));
+#pragma unroll
+                for (int kk = 0; kk < kKeySteps; ++kk)
+                    umma_ts(tQ, tS + packed_col<HW>(kk), sdesc_sw128(k_addr + kk * 2048, BLK * 128, 1024), idesc_q,
+                            (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(bars + kDqBarKvEmpty + s);
+                if (j + 1 < keep) {  // S_{j+1} overwrites dS_j: issued after the product that reads it
+                    if (!mbar_wait(bars + kDqBarKvFull + ((j + 1) & 1), ((j + 1) >> 1) & 1, tmo, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_sp(j + 1);
+                }
+                if (j + 2 < keep) {  // slot s is free once dQ_j (and so dP_j) has read it
+                    if (!mbar_wait(bars + kDqBarKvEmpty + s, (j >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+                    load_kv(j + 2);
+                    ++n_loaded;
+                }
+            }
+            if (ok) umma_commit(bars + kDqBarFinal);
+            else fail();
+            // drain: every product issued here and every copy have landed before the CTA leaves
+            umma_commit(bars + kDqBarDrain);
+            volatile int no_abort = 0;
+            mbar_wait(bars + kDqBarDrain, 0, 10000000ull, &no_abort);
+            if (!ok) {
+                mbar_wait(bars + kDqBarQdo, 0, 10000000ull, &no_abort);
+                for (int t = n_loaded - 2 < 0 ? 0 : n_loaded - 2; t < n_loaded; ++t)
+                    mbar_wait(bars + kDqBarKvFull + (t & 1), (t >> 1) & 1, 10000000ull, &no_abort);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax-gradient warps
+        const int lg = warp & 3, hf = warp >> 2;
+        const int i_row = lg * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(lg * 32) << 16;
+        const int n = alpha * BLK + i_row;
+        const bool row_real = i_row < BLK && n < g.L;
+        // rows that are not this block's (block 64: the tile's second half) or past L recompute as P = 0
+        const float lse_i = row_real ? __ldg(a.lse + static_cast<size_t>(row0) + n) : INFINITY;
+        const float delta_i = row_real ? __ldg(a.delta + static_cast<size_t>(row0) + n) : 0.f;
+        const float c2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+        const int key0 = hf * HW;
+        const int last_valid = keep > 0 ? min(BLK, g.L - __ldg(my_idx + keep - 1) * BLK) : BLK;
+        bool ok = true;
+        for (int j = 0; j < keep; ++j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bars + kDqBarSp, j & 1, tmo, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sr[NC][32], pr[NC][32];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                tmem_ld32(tS + lane_base + key0 + c * 32, sr[c]);
+                tmem_ld32(tP + lane_base + key0 + c * 32, pr[c]);
+            }
+            tmem_ld_wait(sr[0]);
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                reg_fence(sr[c]);
+                reg_fence(pr[c]);
+            }
+            const bool masked = (j == keep - 1) && last_valid < BLK;
+#pragma unroll
+            for (int c16 = 0; c16 < HW / 32; ++c16) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    float d2[2];
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int e = c16 * 32 + 2 * u + e2;  // key within this half
+                        const float s = __uint_as_float(sr[e >> 5][e & 31]);
+                        const float dp = __uint_as_float(pr[e >> 5][e & 31]);
+                        float p = ex2_approx(fmaf(s, c2, -lse_i));
+                        if (masked && key0 + e >= last_valid) p = 0.f;
+                        d2[e2] = p * (dp - delta_i);
+                    }
+                    pk[u] = pack_half2_lohi(d2[0], d2[1]);
+                }
+                tmem_st16(tS + lane_base + key0 + c16 * 16, pk);  // packed over this half's own columns
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bars + kDqBarDs);
+        }
+        // ---- epilogue: dq = R(p)^T dQ^ / sqrt(D), token-major fp32
+        if (keep > 0) {
+            const bool done = ok && __all_sync(0xffffffffu, mbar_wait(bars + kDqBarFinal, 0, tmo, abort_flag));
+            if (done) {
+                tc_fence_after();
+                float vals[D / 2];
+                const float inv_sqrt_d = 1.f / sqrtf(static_cast<float>(D));
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tQ + lane_base + hf * (D / 2) + c * 32, r);
+                    tmem_ld_wait(r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) vals[c * 32 + i] = __uint_as_float(r[i]) * inv_sqrt_d;
+                }
+                if (row_real)
+                    store_row_unrotated<D>(a.dq + g.so.row(b, n, h), vals, hf, n, a, g, true);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------------------- dK, dV
+template <int D, int BLK>
+struct DkvLayout {
+    static constexpr int kTile = 128 * D * 2;   // key-side tiles: 128 rows (the MMA's M)
+    static constexpr int kQTile = BLK * D * 2;  // query-side tiles: one query block
+    static constexpr int kOffK = 0;
+    static constexpr int kOffV = kTile;
+    static constexpr int kOffQ = 2 * kTile;               // slots s at kOffQ + s * kQTile
+    static constexpr int kOffDo = kOffQ + 2 * kQTile;     // slots s at kOffDo + s * kQTile
+    static constexpr int kOffLse = kOffDo + 2 * kQTile;   // slots s: [BLK] fp32 lse then [BLK] fp32 delta
+    static constexpr int kOffBar = kOffLse + 2 * 2 * BLK * 4;
+    static constexpr int kOffMisc = kOffBar + 128;
+    static constexpr int kBytes = kOffMisc + 64;
+};
+
+enum : int { kKvBarKv = 0, kKvBarQFull = 1, kKvBarQEmpty = 3, kKvBarSp = 5, kKvBarP = 6, kKvBarFinal = 7,
+             kKvBarDrain = 8, kKvNumBars = 9 };
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do, BwdArgs a,
+                    Geom g) {
+    using Lay = DkvLayout<D, BLK>;
+    constexpr int HW = BLK / 2;  // query columns per thread
+    constexpr int NC = HW / 32;
+    constexpr int kSteps = D / 16, kQSteps = BLK / 16;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int beta = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int row0 = bh * g.Lp;
+    const int cnt = __ldg(a.inv_cnt + static_cast<size_t>(bh) * g.nb + beta);
+    const int32_t* my_inv = a.inv + (static_cast<size_t>(bh) * g.nb + beta) * g.nb;
+    const uint64_t tmo = a.timeout_ns;
+
+    if (tid == 0) {
+        for (int i = 0; i < kKvNumBars; ++i) mbar_init(bars + i, i == kKvBarP ? kBwdMathThreads : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 384;
+    auto fail = [&]() {
+        *abort_flag = 1;
+        atomicOr(a.status, kDevTimeout);
+    };
+    auto qslot = [&](int s) { return smem + Lay::kOffQ + s * Lay::kQTile; };
+    auto doslot = [&](int s) { return smem + Lay::kOffDo + s * Lay::kQTile; };
+    auto lseslot = [&](int s) { return reinterpret_cast<float*>(smem + Lay::kOffLse + s * 2 * BLK * 4); };
+
+    if (warp == kBwdIssueWarp) {
+        // ------------------------------------------------------------ TMA + tcgen05.mma issuer
+        if (lane == 0 && cnt > 0) {
+            auto load_rows = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int row, int rows) {
+#pragma unroll
+                for (int sl = 0; sl < D / 64; ++sl) tma_load_2d(dst + sl * (rows * 128), tm, bar, sl * 64, row);
+            };
+            auto load_q = [&](int t) {
+                const int s = t & 1;
+                uint64_t* bar = bars + kKvBarQFull + s;
+                mbar_expect_tx(bar, 2u * BLK * D * 2 + 2u * BLK * 4);
+                const int qb = __ldg(my_inv + t);
+                load_rows(qslot(s), &tm_q, bar, row0 + qb * BLK, BLK);
+                load_rows(doslot(s), &tm_do, bar, row0 + qb * BLK, BLK);
+                bulk_load(lseslot(s), a.lse + static_cast<size_t>(row0) + qb * BLK, BLK * 4, bar);
+                bulk_load(lseslot(s) + BLK, a.delta + static_cast<size_t>(row0) + qb * BLK, BLK * 4, bar);
+            };
+            mbar_expect_tx(bars + kKvBarKv, 2u * 128 * D * 2);
+            load_rows(smem + Lay::kOffK, &tm_k, bars + kKvBarKv, row0 + beta * BLK, 128);
+            load_rows(smem + Lay::kOffV, &tm_v, bars + kKvBarKv, row0 + beta * BLK, 128);
+            int n_loaded = 0;
+            for (; n_loaded < 2 && n_loaded < cnt; ++n_loaded) load_q(n_loaded);
+            const uint32_t idesc_s = idesc_f16_f32(128, BLK, false, false);
+            const uint32_t idesc_o = idesc_f16_f32(128, D, false, true);
+            const uint32_t k_addr = smem_addr(smem + Lay::kOffK), v_addr = smem_addr(smem + Lay::kOffV);
+            // S^T_t = k^ q^T_t and dP^T_t = v dO^T_t (K-major over the head dimension)
+            auto issue_sp = [&](int t) {
+                const int s = t & 1;
+                const uint32_t q_addr = smem_addr(qslot(s)), do_addr = smem_addr(doslot(s));
+#pragma unroll
+                for (int kk = 0; kk < kSteps; ++kk) {
+                    const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * (BLK * 128) + (kk & 3) * 32;
+                    umma_ss(tS, sdesc_sw128(k_addr + ao, 16, 1024), sdesc_sw128(q_addr + bo, 16, 1024), idesc_s,
+                            kk > 0 ? 1u : 0u);
+                    umma_ss(tP, sdesc_sw128(v_addr + ao, 16, 1024), sdesc_sw128(do_addr + bo, 16, 1024), idesc_s,
+                            kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bars + kKvBarSp);
+            };
+            bool ok = mbar_wait(bars + kKvBarKv, 0, tmo, abort_flag) && mbar_wait(bars + kKvBarQFull, 0, tmo, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_sp(0);
+            }
+            for (int t = 0; t < cnt && ok; ++t) {
+                const int s = t & 1;
+                if (!mbar_wait(bars + kKvBarP, t & 1, tmo, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                // dV += P^T dO_t and dK^ += dS^T q^_t (A from TMEM, B MN-major over the query rows)
+                const uint32_t q_addr = smem_addr(qslot(s)), do_addr = smem_addr(doslot(s));
+#pragma unroll
+                for (int kk = 0; kk < kQSteps; ++kk) {
+                    const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+                    umma_ts(tV, tS + packed_col<HW>(kk), sdesc_sw128(do_addr + kk * 2048, BLK * 128, 1024), idesc_o, acc);
+                    umma_ts(tK, tP + packed_col<HW>(kk), sdesc_sw128(q_addr + kk * 2048, BLK * 128, 1024), idesc_o, acc);
+                }
+                umma_commit(bars + kKvBarQEmpty + s);
+                if (t + 1 < cnt) {
+                    if (!mbar_wait(bars + kKvBarQFull + ((t + 1) & 1), ((t + 1) >> 1) & 1, tmo, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_sp(t + 1);
+                }
+                if (t + 2 < cnt) {
+                    if (!mbar_wait(bars + kKvBarQEmpty + s, (t >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
+                    load_q(t + 2);
+                    ++n_loaded;
+                }
+            }
+            if (ok) umma_commit(bars + kKvBarFinal);
+            else fail();
+            umma_commit(bars + kKvBarDrain);
+            volatile int no_abort = 0;
+            mbar_wait(bars + kKvBarDrain, 0, 10000000ull, &no_abort);
+            if (!ok) {
+                mbar_wait(bars + kKvBarKv, 0, 10000000ull, &no_abort);
+                for (int t = n_loaded - 2 < 0 ? 0 : n_loaded - 2; t < n_loaded; ++t)
+                    mbar_wait(bars + kKvBarQFull + (t & 1), (t >> 1) & 1, 10000000ull, &no_abort);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax-gradient warps (rows = keys)
+        const int lg = warp & 3, hf = warp >> 2;
+        const int j_row = lg * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(lg * 32) << 16;
+        const int n = beta * BLK + j_row;
+        const bool row_real = j_row < BLK && n < g.L;
+        const float c2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+        const int q0 = hf * HW;  // first query column of this thread's half
+        bool ok = true;
+        for (int t = 0; t < cnt; ++t) {
+            const int s = t & 1;
+            // the query block's lse and delta arrived with its tiles (same barrier phase)
+            ok = __all_sync(0xffffffffu, mbar_wait(bars + kKvBarQFull + s, (t >> 1) & 1, tmo, abort_flag) &&
+                                             mbar_wait(bars + kKvBarSp, t & 1, tmo, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const float* lse_s = lseslot(s);
+            const float* del_s = lse_s + BLK;
+            uint32_t sr[NC][32], pr[NC][32];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                tmem_ld32(tS + lane_base + q0 + c * 32, sr[c]);
+                tmem_ld32(tP + lane_base + q0 + c * 32, pr[c]);
+            }
+            tmem_ld_wait(sr[0]);
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                reg_fence(sr[c]);
+                reg_fence(pr[c]);
+            }
+#pragma unroll
+            for (int c16 = 0; c16 < HW / 32; ++c16) {
+                uint32_t pk[16], dk16[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    float pp[2], dd[2];
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int e = c16 * 32 + 2 * u + e2;  // query column within this half
+                        const float sv = __uint_as_float(sr[e >> 5][e & 31]);
+                        const float dp = __uint_as_float(pr[e >> 5][e & 31]);
+                        const float p = ex2_approx(fmaf(sv, c2, -lse_s[q0 + e]));  // +inf lse: p = 0
+                        pp[e2] = p;
+                        dd[e2] = p * (dp - del_s[q0 + e]);
+                    }
+                    pk[u] = pack_half2_lohi(pp[0], pp[1]);
+                    dk16[u] = pack_half2_lohi(dd[0], dd[1]);
+                }
+                tmem_st16(tS + lane_base + q0 + c16 * 16, pk);
+                tmem_st16(tP + lane_base + q0 + c16 * 16, dk16);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bars + kKvBarP);
+        }
+        // ---- epilogue: dv = sum P^T dO, dk = R(p)^T dK^ / sqrt(D); key blocks nobody kept get zeros
+        const bool done = cnt == 0 || (ok && __all_sync(0xffffffffu, mbar_wait(bars + kKvBarFinal, 0, tmo, abort_flag)));
+        if (done) {
+            if (cnt > 0) tc_fence_after();
+            const float inv_sqrt_d = 1.f / sqrtf(static_cast<float>(D));
+            float vals[D / 2];
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {  // 0: dv, 1: dk
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t r[32];
+                    if (cnt > 0) {
+                        tmem_ld32((which ? tK : tV) + lane_base + hf * (D / 2) + c * 32, r);
+                        tmem_ld_wait(r);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        vals[c * 32 + i] = cnt > 0 ? __uint_as_float(r[i]) * (which ? inv_sqrt_d : 1.f) : 0.f;
+                }
+                if (row_real)
+                    store_row_unrotated<D>((which ? a.dk : a.dv) + g.so.row(b, n, h), vals, hf, n, a, g, which == 1);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------------------------ preparation
+// dO (fp32, token-major) -> fp16 head-major copy for the tensor cores (rows past L zero), and
+// Delta_i = dO_i . O_s,i (O_s head-major fp32 from the recomputed sparse forward).  One warp per row.
+__global__ void bwd_prep_kernel(const float* __restrict__ dout, const float* __restrict__ os, Geom g,
+                                __half* __restrict__ doh, float* __restrict__ delta, int* status) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const long long rows = static_cast<long long>(g.BH()) * g.Lp;
+    if (warp >= rows) return;
+    const int bh = static_cast<int>(warp / g.Lp), n = static_cast<int>(warp % g.Lp);
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int per = g.D / 32;  // elements per lane: 2 or 4
+    float dsum = 0.f;
+    bool bad = false;
+    __half* dst = doh + static_cast<size_t>(warp) * g.D + lane * per;
+    if (n < g.L) {
+        const float* src = dout + g.so.row(b, n, h) + lane * per;
+        const float* o = os + static_cast<size_t>(warp) * g.D + lane * per;
+        for (int e = 0; e < per; e += 2) {
+            const float2 x = *reinterpret_cast<const float2*>(src + e);
+            const float2 y = *reinterpret_cast<const float2*>(o + e);
+            dsum = fmaf(x.x, y.x, fmaf(x.y, y.y, dsum));
+            bad |= !(fmaxf(fabsf(x.x), fabsf(x.y)) < 65504.f);
+            *reinterpret_cast<__half2*>(dst + e) = __floats2half2_rn(x.x, x.y);
+        }
+    } else {
+        for (int e = 0; e < per; e += 2) *reinterpret_cast<__half2*>(dst + e) = __floats2half2_rn(0.f, 0.f);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+    if (lane == 0) delta[warp] = dsum;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, kDevRange);
+}
+
+// Inverted kept-block lists: for key block beta of head bh, the query blocks whose kept list holds
+// it, ascending (one CTA of 128 threads per (beta, bh); each thread tests query blocks by binary search
+// in their ascending kept lists; an ordered compaction writes them).
+__global__ void bwd_invert_kernel(const int32_t* __restrict__ idx, Geom g, int32_t* __restrict__ inv,
+                                  int32_t* __restrict__ inv_cnt) {
+    __shared__ int warp_tot[4];
+    const int beta = blockIdx.x, bh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int32_t* ib = idx + static_cast<size_t>(bh) * g.nb * g.keep;
+    int32_t* out = inv + (static_cast<size_t>(bh) * g.nb + beta) * g.nb;
+    int written = 0;
+    for (int base = 0; base < g.nb; base += 128) {
+        const int al = base + tid;
+        bool hit = false;
+        if (al < g.nb) {
+            const int32_t* row = ib + static_cast<size_t>(al) * g.keep;
+            int lo = 0, hi = g.keep - 1;
+            while (lo <= hi) {
+                const int mid = (lo + hi) >> 1;
+                const int x = __ldg(row + mid);
+                if (x == beta) { hit = true; break; }
+                if (x < beta) lo = mid + 1;
+                else hi = mid - 1;
+            }
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (lane == 0) warp_tot[warp] = __popc(m);
+        __syncthreads();
+        int before = written;
+        for (int w = 0; w < warp; ++w) before += warp_tot[w];
+        if (hit) out[before + __popc(m & ((1u << lane) - 1u))] = al;
+        written += warp_tot[0] + warp_tot[1] + warp_tot[2] + warp_tot[3];
+        __syncthreads();
+    }
+    if (tid == 0) inv_cnt[static_cast<size_t>(bh) * g.nb + beta] = written;
+}
+
+// ------------------------------------------------------------------------------------ low-rank
+// Token tile of the CUDA-core passes: 32 tokens (16 when rank > 64, so shared memory fits).
+template <int R>
+struct LrTile {
+    static constexpr int T = R <= 64 ? 32 : 16;
+};
+
+// Pass over the queries: per token u = q A, phi, psi, den, G = S dO; dpsi, dden, dphi, du; split-L
+// partial sums of dS = sum psi dO^T / den, dz = sum dden phi and dA_q = q^T du; dq += du A^T.
+template <int D, int R>
+__global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __restrict__ q,
+                                                       const float* __restrict__ dout,
+                                                       const __nv_bfloat16* __restrict__ A,
+                                                       const float* __restrict__ S, const float* __restrict__ z,
+                                                       const double2* __restrict__ tab,
+                                                       const int2* __restrict__ pairs, Geom g, int nsplit,
+                                                       float* __restrict__ dq, float* __restrict__ ds_part,
+                                                       float* __restrict__ dz_part, float* __restrict__ da_part) {
+    constexpr int TT = LrTile<R>::T;
+    extern __shared__ __align__(16) float smf[];
+    float* As = smf;                    // [D][R]
+    float* Ss = As + D * R;             // [R][D]
+    float* zs = Ss + R * D;             // [R]
+    float* xs = zs + R;                 // [TT][D+1] q
+    float* gs = xs + TT * (D + 1);      // [TT][D+1] dO
+    float* us = gs + TT * (D + 1);      // [TT][R+1] u
+    float* Gs = us + TT * (R + 1);      // [TT][R+1] G = S dO
+    float* ws = Gs + TT * (R + 1);      // [TT][R] psi / den
+    float* dus = ws + TT * R;           // [TT][R+1] du
+    float* phs = dus + TT * (R + 1);    // [TT][R] phi
+    float* dens = phs + TT * R;         // [TT] den
+    float* ddens = dens + TT;           // [TT] dden
+    constexpr int G = 256 / D;          // row groups of the D-wide accumulations
+    constexpr int NA = R / G;
+    const int tid = threadIdx.x;
+    const int split = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int ntiles = (g.L + TT - 1) / TT;
+    const int per = (ntiles + nsplit - 1) / nsplit;
+    const int t0 = split * per, t1 = min(ntiles, t0 + per);
+    for (int e = tid; e < D * R; e += 256) As[e] = __bfloat162float(A[e]);
+    for (int e = tid; e < R * D; e += 256) Ss[e] = S[static_cast<size_t>(bh) * R * D + e];
+    if (tid < R) zs[tid] = z[static_cast<size_t>(bh) * R + tid];
+    const int e_own = tid % D, cg = tid / D;
+    float acc_s[NA], acc_a[NA];  // dS[c][e_own], dA[e_own][c] for c = cg + G i
+#pragma unroll
+    for (int i = 0; i < NA; ++i) acc_s[i] = acc_a[i] = 0.f;
+    float acc_z = 0.f;
+    for (int tile = t0; tile < t1; ++tile) {
+        const int n0 = tile * TT;
+        __syncthreads();
+        for (int e = tid; e < TT * (D / 2); e += 256) {
+            const int tt = e / (D / 2), dp = e % (D / 2);
+            const int n = n0 + tt;
+            float2 xf = make_float2(0.f, 0.f), gf = make_float2(0.f, 0.f);
+            if (n < g.L) {
+                xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + g.sq.row(b, n, h) + 2 * dp));
+                gf = *reinterpret_cast<const float2*>(dout + g.so.row(b, n, h) + 2 * dp);
+            }
+            xs[tt * (D + 1) + 2 * dp] = xf.x; xs[tt * (D + 1) + 2 * dp + 1] = xf.y;
+            gs[tt * (D + 1) + 2 * dp] = gf.x; gs[tt * (D + 1) + 2 * dp + 1] = gf.y;
+        }
+        __syncthreads();
+        // u = q A and G = S dO, thread per (token, feature)
+        for (int o = tid; o < TT * R; o += 256) {
+            const int tt = o / R, c = o % R;
+            const float* xr = xs + tt * (D + 1);
+            const float* gr = gs + tt * (D + 1);
+            float u = 0.f, gg = 0.f;
+#pragma unroll 8
+            for (int d = 0; d < D; ++d) {
+                u = fmaf(xr[d], As[d * R + c], u);
+                gg = fmaf(Ss[c * D + d], gr[d], gg);
+            }
+            us[tt * (R + 1) + c] = u;
+            Gs[tt * (R + 1) + c] = gg;
+            phs[tt * R + c] = fmaxf(u, 0.f);
+        }
+        __syncthreads();
+        // per token: den = phi . z + 1e-6, dden = -(psi . G) / den^2 (one warp per token)
+        {
+            const int warp = tid >> 5, lane = tid & 31;
+            for (int tt = warp; tt < TT; tt += 8) {
+                const int n = n0 + tt;
+                const int nt = n < g.L ? n : 0;
+                float dz_ = 0.f, dot = 0.f;
+                for (int p = lane; p < R / 2; p += 32) {
+                    const float x0 = phs[tt * R + 2 * p], x1 = phs[tt * R + 2 * p + 1];
+                    const int2 pi = pairs[p];
+                    const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
+                    const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+                    const float y0 = x0 * cf - x1 * sf, y1 = x0 * sf + x1 * cf;
+                    dz_ = fmaf(x0, zs[2 * p], fmaf(x1, zs[2 * p + 1], dz_));
+                    dot = fmaf(y0, Gs[tt * (R + 1) + 2 * p], fmaf(y1, Gs[tt * (R + 1) + 2 * p + 1], dot));
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    dz_ += __shfl_xor_sync(0xffffffffu, dz_, o);
+                    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                }
+                if (lane == 0) {
+                    const float den = dz_ + 1e-6f;
+                    dens[tt] = den;
+                    ddens[tt] = n < g.L ? -dot / (den * den) : 0.f;
+                }
+            }
+        }
+        __syncthreads();
+        // per (token, pair): psi / den, dphi = R^T (G / den) + dden z, du = dphi [u > 0]
+        for (int o = tid; o < TT * (R / 2); o += 256) {
+            const int tt = o / (R / 2), p = o % (R / 2);
+            const int n = n0 + tt;
+            const int nt = n < g.L ? n : 0;
+            const int2 pi = pairs[p];
+            const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
+            const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+            const float den = dens[tt], dd = ddens[tt];
+            const float x0 = phs[tt * R + 2 * p], x1 = phs[tt * R + 2 * p + 1];
+            const float y0 = x0 * cf - x1 * sf, y1 = x0 * sf + x1 * cf;
+            ws[tt * R + 2 * p] = n < g.L ? y0 / den : 0.f;
+            ws[tt * R + 2 * p + 1] = n < g.L ? y1 / den : 0.f;
+            const float g0 = Gs[tt * (R + 1) + 2 * p] / den, g1 = Gs[tt * (R + 1) + 2 * p + 1] / den;
+            const float dph0 = cf * g0 + sf * g1 + dd * zs[2 * p];
+            const float dph1 = -sf * g0 + cf * g1 + dd * zs[2 * p + 1];
+            const bool live = n < g.L;
+            dus[tt * (R + 1) + 2 * p] = (live && us[tt * (R + 1) + 2 * p] > 0.f) ? dph0 : 0.f;
+            dus[tt * (R + 1) + 2 * p + 1] = (live && us[tt * (R + 1) + 2 * p + 1] > 0.f) ? dph1 : 0.f;
+        }
+        __syncthreads();
+        // partial sums: dS[c][e] += sum_t w[t][c] dO[t][e]; dA[d][c] += sum_t q[t][d] du[t][c]; dz
+#pragma unroll 4
+        for (int tt = 0; tt < TT; ++tt) {
+            const float go = gs[tt * (D + 1) + e_own], xo = xs[tt * (D + 1) + e_own];
+#pragma unroll
+            for (int i = 0; i < NA; ++i) {
+                acc_s[i] = fmaf(ws[tt * R + cg + G * i], go, acc_s[i]);
+                acc_a[i] = fmaf(xo, dus[tt * (R + 1) + cg + G * i], acc_a[i]);
+            }
+        }
+        if (tid < R)
+            for (int tt = 0; tt < TT; ++tt) acc_z = fmaf(ddens[tt], phs[tt * R + tid], acc_z);
+        // dq += du A^T, thread per (token, dim)
+        for (int o = tid; o < TT * D; o += 256) {
+            const int tt = o / D, d = o % D;
+            const int n = n0 + tt;
+            if (n >= g.L) continue;
+            float s = 0.f;
+#pragma unroll 8
+            for (int c = 0; c < R; ++c) s = fmaf(dus[tt * (R + 1) + c], As[d * R + c], s);
+            dq[g.so.row(b, n, h) + d] += s;
+        }
+    }
+    const size_t slot = static_cast<size_t>(bh) * nsplit + split;
+#pragma unroll
+    for (int i = 0; i < NA; ++i) {
+        ds_part[slot * R * D + (cg + G * i) * D + e_own] = acc_s[i];
+        da_part[slot * D * R + e_own * R + cg + G * i] = acc_a[i];
+    }
+    if (tid < R) dz_part[slot * R + tid] = acc_z;
+}
+
+// Pass over the keys: per token u = k A, phi, psi; dpsi = dS v; dv += dS^T psi; dphi = R^T dpsi + dz;
+// du; dk += du A^T; split-L partial sums of dA_k = k^T du.
+template <int D, int R>
+__global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __restrict__ k,
+                                                       const __nv_bfloat16* __restrict__ v,
+                                                       const __nv_bfloat16* __restrict__ A,
+                                                       const float* __restrict__ dS, const float* __restrict__ dz,
+                                                       const double2* __restrict__ tab,
+                                                       const int2* __restrict__ pairs, Geom g, int nsplit,
+                                                       float* __restrict__ dk, float* __restrict__ dv,
+                                                       float* __restrict__ da_part) {
+    constexpr int TT = LrTile<R>::T;
+    extern __shared__ __align__(16) float smf[];
+    float* As = smf;                    // [D][R]
+    float* Ss = As + D * R;             // [R][D] dS
+    float* zs = Ss + R * D;             // [R] dz
+    float* xs = zs + R;                 // [TT][D+1] k
+    float* vs = xs + TT * (D + 1);      // [TT][D+1] v
+    float* us = vs + TT * (D + 1);      // [TT][R+1] u
+    float* ps = us + TT * (R + 1);      // [TT][R+1] dpsi, then du
+    float* psis = ps + TT * (R + 1);    // [TT][R+1] psi
+    constexpr int G = 256 / D;
+    constexpr int NA = R / G;
+    const int tid = threadIdx.x;
+    const int split = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int ntiles = (g.L + TT - 1) / TT;
+    const int per = (ntiles + nsplit - 1) / nsplit;
+    const int t0 = split * per, t1 = min(ntiles, t0 + per);
+    for (int e = tid; e < D * R; e += 256) As[e] = __bfloat162float(A[e]);
+    for (int e = tid; e < R * D; e += 256) Ss[e] = dS[static_cast<size_t>(bh) * R * D + e];
+    if (tid < R) zs[tid] = dz[static_cast<size_t>(bh) * R + tid];
+    const int e_own = tid % D, cg = tid / D;
+    float acc_a[NA];
+#pragma unroll
+    for (int i = 0; i < NA; ++i) acc_a[i] = 0.f;
+    for (int tile = t0; tile < t1; ++tile) {
+        const int n0 = tile * TT;
+        __syncthreads();
+        for (int e = tid; e < TT * (D / 2); e += 256) {
+            const int tt = e / (D / 2), dp = e % (D / 2);
+            const int n = n0 + tt;
+            float2 xf = make_float2(0.f, 0.f), vf = make_float2(0.f, 0.f);
+            if (n < g.L) {
+                xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + g.sk.row(b, n, h) + 2 * dp));
+                vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + g.sv.row(b, n, h) + 2 * dp));
+            }
+            xs[tt * (D + 1) + 2 * dp] = xf.x; xs[tt * (D + 1) + 2 * dp + 1] = xf.y;
+            vs[tt * (D + 1) + 2 * dp] = vf.x; vs[tt * (D + 1) + 2 * dp + 1] = vf.y;
+        }
+        __syncthreads();
+        // u = k A and dpsi = dS v, thread per (token, feature)
+        for (int o = tid; o < TT * R; o += 256) {
+            const int tt = o / R, c = o % R;
+            const float* xr = xs + tt * (D + 1);
+            const float* vr = vs + tt * (D + 1);
+            float u = 0.f, dp = 0.f;
+#pragma unroll 8
+            for (int d = 0; d < D; ++d) {
+                u = fmaf(xr[d], As[d * R + c], u);
+                dp = fmaf(Ss[c * D + d], vr[d], dp);
+            }
+            us[tt * (R + 1) + c] = u;
+            ps[tt * (R + 1) + c] = dp;
+        }
+        __syncthreads();
+        // per (token, pair): psi = R phi; du = (R^T dpsi + dz) [u > 0] (written over dpsi)
+        for (int o = tid; o < TT * (R / 2); o += 256) {
+            const int tt = o / (R / 2), p = o % (R / 2);
+            const int n = n0 + tt;
+            const int nt = n < g.L ? n : 0;
+            const int2 pi = pairs[p];
+            const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
+            const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+            const float u0 = us[tt * (R + 1) + 2 * p], u1 = us[tt * (R + 1) + 2 * p + 1];
+            const float x0 = fmaxf(u0, 0.f), x1 = fmaxf(u1, 0.f);
+            psis[tt * (R + 1) + 2 * p] = x0 * cf - x1 * sf;
+            psis[tt * (R + 1) + 2 * p + 1] = x0 * sf + x1 * cf;
+            const float d0 = ps[tt * (R + 1) + 2 * p], d1 = ps[tt * (R + 1) + 2 * p + 1];
+            const float dph0 = cf * d0 + sf * d1 + zs[2 * p];
+            const float dph1 = -sf * d0 + cf * d1 + zs[2 * p + 1];
+            const bool live = n < g.L;
+            ps[tt * (R + 1) + 2 * p] = (live && u0 > 0.f) ? dph0 : 0.f;
+            ps[tt * (R + 1) + 2 * p + 1] = (live && u1 > 0.f) ? dph1 : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int tt = 0; tt < TT; ++tt) {
+            const float xo = xs[tt * (D + 1) + e_own];
+#pragma unroll
+            for (int i = 0; i < NA; ++i) acc_a[i] = fmaf(xo, ps[tt * (R + 1) + cg + G * i], acc_a[i]);
+        }
+        // dv += dS^T psi and dk += du A^T, thread per (token, dim)
+        for (int o = tid; o < TT * D; o += 256) {
+            const int tt = o / D, d = o % D;
+            const int n = n0 + tt;
+            if (n >= g.L) continue;
+            float sv = 0.f, sk = 0.f;
+#pragma unroll 8
+            for (int c = 0; c < R; ++c) {
+                sv = fmaf(Ss[c * D + d], psis[tt * (R + 1) + c], sv);
+                sk = fmaf(ps[tt * (R + 1) + c], As[d * R + c], sk);
+            }
+            const long long r = g.so.row(b, n, h) + d;
+            dv[r] += sv;
+            dk[r] += sk;
+        }
+    }
+    const size_t slot = static_cast<size_t>(bh) * nsplit + split;
+#pragma unroll
+    for (int i = 0; i < NA; ++i) da_part[slot * D * R + e_own * R + cg + G * i] = acc_a[i];
+}
+
+// dA = sum over both passes, all heads and all splits of the partials, in a fixed order.
+__global__ void bwd_da_reduce_kernel(const float* __restrict__ da_part, int nslots, int DR, float* __restrict__ dA) {
+    const int o = blockIdx.x * blockDim.x + threadIdx.x;
+    if (o >= DR) return;
+    float s = 0.f;
+    for (int i = 0; i < nslots; ++i) s += da_part[static_cast<size_t>(i) * DR + o];
+    dA[o] = s;
+}
+
+// ------------------------------------------------------------------------------------ launchers
+size_t lr_bwd_smem(int D, int R, bool qpass) {
+    const int TT = R <= 64 ? 32 : 16;
+    if (qpass)
+        return sizeof(float) * (2 * D * R + R + 2 * TT * (D + 1) + 3 * TT * (R + 1) + 2 * TT * R + 2 * TT);
+    return sizeof(float) * (2 * D * R + R + 2 * TT * (D + 1) + 3 * TT * (R + 1));
+}
+
+int lr_bwd_nsplit(const Geom& g) {
+    const int TT = g.R <= 64 ? 32 : 16;
+    const long long ntiles = (g.L + TT - 1) / TT;
+    long long ns = (2 * 148 + g.BH() - 1) / g.BH();
+    ns = ns < 1 ? 1 : (ns > ntiles ? ntiles : ns);
+    return static_cast<int>(ns);
+}
+
+namespace {
+template <int D, int BLK>
+cudaError_t launch_bwd_sparse_t(const BwdMaps& m, const BwdArgs& a, const Geom& g, cudaStream_t st) {
+    const size_t sq = DqLayout<D>::kBytes + 1024, skv = DkvLayout<D, BLK>::kBytes + 1024;
+    cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sq);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)skv);
+    if (e != cudaSuccess) return e;
+    bwd_dq_kernel<D, BLK><<<dim3(g.nb, g.BH()), kBwdThreads, sq, st>>>(m.q128, m.do128, m.kb, m.vb, a, g);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (m.between) cudaEventRecord(m.between, st);
+    bwd_dkdv_kernel<D, BLK><<<dim3(g.nb, g.BH()), kBwdThreads, skv, st>>>(m.k128, m.v128, m.qb, m.dob, a, g);
+    return cudaGetLastError();
+}
+
+template <int D, int R>
+cudaError_t launch_lr_bwd_t(const LrBwdArgs& l, const Geom& g, cudaStream_t st) {
+    const int ns = l.nsplit;
+    const size_t smq = lr_bwd_smem(D, R, true), smk = lr_bwd_smem(D, R, false);
+    cudaError_t e = cudaFuncSetAttribute(bwd_lr_q_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_lr_k_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk);
+    if (e != cudaSuccess) return e;
+    bwd_lr_q_kernel<D, R><<<dim3(ns, g.BH()), 256, smq, st>>>(l.q, l.dout, l.A, l.S, l.z, l.tab, l.pairs, g, ns, l.dq,
+                                                              l.ds_part, l.dz_part, l.da_part);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_lowrank_reduce(l.ds_part, l.dz_part, g, ns, l.dS, l.dz, nullptr, nullptr, nullptr, st)) !=
+        cudaSuccess)
+        return e;
+    bwd_lr_k_kernel<D, R><<<dim3(ns, g.BH()), 256, smk, st>>>(l.k, l.v, l.A, l.dS, l.dz, l.tab, l.pairs, g, ns, l.dk,
+                                                              l.dv, l.da_part + static_cast<size_t>(g.BH()) * ns * D * R);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int DR = D * R;
+    bwd_da_reduce_kernel<<<(DR + 255) / 256, 256, 0, st>>>(l.da_part, 2 * g.BH() * ns, DR, l.dA);
+    return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_bwd_prep(const float* dout, const float* os, const Geom& g, __half* doh, float* delta, int* status,
+                            cudaStream_t st) {
+    const long long rows = static_cast<long long>(g.BH()) * g.Lp;
+    const long long blocks = (rows * 32 + 255) / 256;
+    bwd_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(dout, os, g, doh, delta, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_invert(const int32_t* idx, const Geom& g, int32_t* inv, int32_t* inv_cnt, cudaStream_t st) {
+    bwd_invert_kernel<<<dim3(g.nb, g.BH()), 128, 0, st>>>(idx, g, inv, inv_cnt);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_sparse(const BwdMaps& m, const BwdArgs& a, const Geom& g, cudaStream_t st) {
+    if (g.D == 128) return g.block == 128 ? launch_bwd_sparse_t<128, 128>(m, a, g, st) : launch_bwd_sparse_t<128, 64>(m, a, g, st);
+    return g.block == 128 ? launch_bwd_sparse_t<64, 128>(m, a, g, st) : launch_bwd_sparse_t<64, 64>(m, a, g, st);
+}
+
+cudaError_t launch_lr_bwd(const LrBwdArgs& l, const Geom& g, cudaStream_t st) {
+    if (g.D == 128) {
+        switch (g.R) {
+            case 16: return launch_lr_bwd_t<128, 16>(l, g, st);
+            case 32: return launch_lr_bwd_t<128, 32>(l, g, st);
+            case 48: return launch_lr_bwd_t<128, 48>(l, g, st);
+            case 64: return launch_lr_bwd_t<128, 64>(l, g, st);
+            case 80: return launch_lr_bwd_t<128, 80>(l, g, st);
+            case 96: return launch_lr_bwd_t<128, 96>(l, g, st);
+            case 112: return launch_lr_bwd_t<128, 112>(l, g, st);
+            case 128: return launch_lr_bwd_t<128, 128>(l, g, st);
+        }
+    } else if (g.D == 64) {
+        switch (g.R) {
+            case 16: return launch_lr_bwd_t<64, 16>(l, g, st);
+            case 32: return launch_lr_bwd_t<64, 32>(l, g, st);
+            case 48: return launch_lr_bwd_t<64, 48>(l, g, st);
+            case 64: return launch_lr_bwd_t<64, 64>(l, g, st);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace slra

@@ -123,8 +123,50 @@ struct AttnArgs {
     int* status;
     unsigned long long timeout_ns;
     int debug_unsatisfied_wait;  // test hook: wait on a barrier nothing signals before any work
+    float* lse;  // optional fp32 [B*Hh][Lp]: per query row m + log2(l) of the sparse softmax in the kernel's
+                 // log2 units (P_ij = 2^(s_ij log2(e) / sqrt(D) - lse_i)); +inf for rows past L
 };
 cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st);
 size_t attn_smem_bytes(const Geom& g);
+
+// ---- backward pass (bwd_sm100.cu) --------------------------------------------------------------
+struct BwdArgs {
+    const int32_t* idx;      // [BH][nb][keep] kept key blocks per query block, ascending
+    int keep;
+    const int32_t* inv;      // [BH][nb][nb] query blocks that kept each key block, ascending
+    const int32_t* inv_cnt;  // [BH][nb]
+    const float* lse;        // [BH][Lp] (log2 units; +inf for rows past L)
+    const float* delta;      // [BH][Lp] dO . O_sparse per row
+    const double2* tab;      // rotary cos/sin table
+    int2 pair_info[kMaxPairs];
+    float* dq;  // token-major fp32 [B][L][Hh][D] (strides g.so)
+    float* dk;
+    float* dv;
+    int* status;
+    unsigned long long timeout_ns;
+};
+// fp16 head-major maps (128-B swizzle): 128-row boxes for the tiles that are an MMA's M side, block-row
+// boxes for the others; `between` (optional) is recorded between the dQ and the dK/dV kernels.
+struct BwdMaps {
+    CUtensorMap q128, do128, kb, vb;  // dQ kernel
+    CUtensorMap k128, v128, qb, dob;  // dK/dV kernel
+    cudaEvent_t between;
+};
+struct LrBwdArgs {
+    const __nv_bfloat16 *q, *k, *v, *A;
+    const float* dout;
+    const float *S, *z;
+    const double2* tab;
+    const int2* pairs;
+    float *dq, *dk, *dv, *dA;
+    float *ds_part, *dz_part, *da_part, *dS, *dz;
+    int nsplit;
+};
+cudaError_t launch_bwd_prep(const float* dout, const float* os, const Geom& g, __half* doh, float* delta, int* status,
+                            cudaStream_t st);
+cudaError_t launch_bwd_invert(const int32_t* idx, const Geom& g, int32_t* inv, int32_t* inv_cnt, cudaStream_t st);
+cudaError_t launch_bwd_sparse(const BwdMaps& m, const BwdArgs& a, const Geom& g, cudaStream_t st);
+cudaError_t launch_lr_bwd(const LrBwdArgs& l, const Geom& g, cudaStream_t st);
+int lr_bwd_nsplit(const Geom& g);
 
 }  // namespace slra

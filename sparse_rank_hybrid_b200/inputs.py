@@ -71,3 +71,9 @@ def make_projections(seed: int, heads: int, D: int, R: int, separate: bool, per_
     rng = np.random.Generator(np.random.PCG64(seed))
     shape = (2 if separate else 1, heads if per_head else 1, D, R)
     return f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32) * np.float32(1.0 / np.sqrt(D)))
+
+
+def make_dout(seed: int, B: int, L: int, heads: int, D: int, scale: float = 1.0) -> np.ndarray:
+    """A seeded upstream gradient dout ~ N(0, scale^2), fp32 [B, L, heads, D], for the backward pass."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return rng.standard_normal((B, L, heads, D), dtype=np.float32) * np.float32(scale)

@@ -28,7 +28,7 @@ FUSION_SUM, FUSION_GATED = 0, 1
 # Every symbol include/slra.h declares.
 EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_validate", "slra_keep_count",
            "slra_projection_elems", "slra_workspace_bytes", "slra_attn_fwd", "slra_attn_fwd_ex", "slra_sparse_fwd",
-           "slra_lowrank_fwd", "slra_get_device_status",
+           "slra_lowrank_fwd", "slra_get_device_status", "slra_bwd_workspace_bytes", "slra_attn_bwd",
            "slra_workspace_layout", "slra_host_io_bytes", "slra_host_pipeline_groups",
            "slra_attn_fwd_host",
            "slra_select_blocks", "slra_lowrank_summary", "slra_device_status", "slra_lowrank_summary_noalloc",
@@ -106,6 +106,9 @@ def lib():
         L.slra_sparse_fwd.argtypes = [PT, PT, PT, C, C, C, C, ctypes.c_float, PT, P, S, P]
         L.slra_lowrank_fwd.argtypes = [PT, PT, PT, PM, C, C, C, C, PT, P, P, P, S, P]
         L.slra_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
+        L.slra_bwd_workspace_bytes.restype = S
+        L.slra_bwd_workspace_bytes.argtypes = [PP]
+        L.slra_attn_bwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, S, P]
         L.slra_host_io_bytes.restype = S
         L.slra_host_io_bytes.argtypes = [PP]
         L.slra_host_pipeline_groups.restype = ctypes.c_int64
@@ -118,6 +121,7 @@ def lib():
         L.slra_noalloc_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
         for name in ("slra_problem_init", "slra_validate", "slra_workspace_layout", "slra_attn_fwd",
                      "slra_attn_fwd_ex", "slra_sparse_fwd", "slra_lowrank_fwd", "slra_get_device_status",
+                     "slra_attn_bwd",
                      "slra_attn_fwd_host", "slra_select_blocks", "slra_lowrank_summary", "slra_device_status",
                      "slra_lowrank_summary_noalloc", "slra_noalloc_device_status"):
             getattr(L, name).restype = ctypes.c_int
@@ -351,6 +355,38 @@ def lowrank_fwd(q, k, v, A, T, H, W, rank, out, S=None, z=None, workspace=None, 
                                   None if z is None else _ptr(z), ws_ptr, ws_n, _stream_handle(stream)),
            "slra_lowrank_fwd")
     return out
+
+
+def bwd_workspace_bytes(prob: Problem) -> int:
+    return int(lib().slra_bwd_workspace_bytes(ctypes.byref(prob.c())))
+
+
+def attn_bwd(prob: Problem, q, k, v, A, dout, grads=None, workspace=None, stream=None):
+    """Backward pass (slra_attn_bwd): gradients of sum(dout * out) for q, k, v (fp32 [B, L, Hh, D]) and A
+    (fp32 [D, rank]).  dout: contiguous CUDA fp32 [B, L, Hh, D].  q, k, v may be strided views.
+    Returns (dq, dk, dv, dA, workspace)."""
+    import dataclasses
+    torch = _torch()
+    shp = (prob.batch, prob.L, prob.heads, prob.head_dim)
+    strides = {f"{n}_strides": _row_strides(n, t, shp, torch.bfloat16) for n, t in (("q", q), ("k", k), ("v", v))}
+    p = dataclasses.replace(prob, **strides)
+    if dout.dtype != torch.float32 or not dout.is_cuda or not dout.is_contiguous() or tuple(dout.shape) != shp:
+        raise ValueError(f"dout: expected a contiguous CUDA fp32 tensor of shape {shp}")
+    if A is not None:
+        _check_bf16("A", A, prob.projection_shape)
+    if grads is None:
+        grads = tuple(torch.empty(shp, dtype=torch.float32, device=q.device) for _ in range(3)) + \
+            (torch.empty((prob.head_dim, prob.rank), dtype=torch.float32, device=q.device),)
+    dq, dk, dv, dA = grads
+    if workspace is None:
+        n = bwd_workspace_bytes(p)
+        if n == 0:
+            raise SlraError(ERR_UNSUPPORTED, "slra_bwd_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    _check(lib().slra_attn_bwd(ctypes.byref(p.c()), _ptr(q), _ptr(k), _ptr(v), None if A is None else _ptr(A),
+                               _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dA), _ptr(workspace),
+                               workspace.numel(), _stream_handle(stream)), "slra_attn_bwd")
+    return dq, dk, dv, dA, workspace
 
 
 def get_device_status(stream=None) -> int:

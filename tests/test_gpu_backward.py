@@ -1,0 +1,149 @@
+"""GPU parity of the backward pass (slra_attn_bwd) against the fp64 oracle's gradients.
+
+The oracle is oracle/backward.py's head_backward: the forward restated in differentiable fp64 torch and
+differentiated by autograd, pinned on the CPU to finite differences of the C oracle, to torch's dense
+attention backward and to the explicit gradient steps.  Both sides use the same block selection (the
+GPU's, read back from the workspace; the selection is piecewise constant, so gradients do not flow
+through it).  dA is the sum over all heads and batch elements of the per-head gradients (A is shared).
+
+Tolerance, derived from the arithmetic: the gradients go through fp16 operands (q^, k^, v, dO, P, dS;
+2^-12 relative rounding each, the inputs exact in bf16) with fp32 accumulation, the same class of error
+as the forward, whose mean relative error is ~3e-4 against a 2e-3 bound.  So every gradient tensor must
+have mean relative error sum|g - g*| / sum|g*| <= 2e-3, and max-abs error <= 1e-2 * max|g*| (the
+forward's absolute 1e-2 bound, scaled to the gradient's own magnitude, which grows with L and dout).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from sparse_rank_hybrid_b200 import inputs as I
+from sparse_rank_hybrid_b200 import slra
+from sparse_rank_hybrid_b200 import workloads as W
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+MEAN_REL = 2e-3
+MAX_ABS_REL = 1e-2
+REPORT = os.environ.get("SLRA_PARITY_REPORT")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_rank_hybrid_b200 import build
+    build.build()
+    import oracle
+    oracle.build()
+
+
+def _gpu_bwd(w, x, dout, **kw):
+    import torch
+    p = slra.Problem.from_workload(w, **kw)
+    q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
+    g = torch.from_numpy(dout).cuda()
+    dq, dk, dv, dA, ws = slra.attn_bwd(p, q, k, v, A, g)
+    assert slra.device_status(ws) == slra.OK
+    idx = slra.ws_view(p, ws, "idx").cpu().numpy() if p.branches & slra.BRANCH_SPARSE else None
+    return p, [t.cpu().numpy().astype(np.float64) for t in (dq, dk, dv, dA)], idx
+
+
+def _oracle_bwd(w, x, dout, idx, branches):
+    import oracle
+    from oracle import backward as OB
+    B, L, Hh, D = x["q"].shape
+    R = w.rank
+    A = oracle.decode_bf16(x["A"]).reshape(D, R)
+    grid = (w.T, w.H, w.W)
+    ref = [np.zeros((B, L, Hh, D)) for _ in range(3)] + [np.zeros((D, R))]
+    for b in range(B):
+        for h in range(Hh):
+            hidx = None if idx is None else idx[b * Hh + h]
+            if hidx is None:  # low-rank only: any selection (unused)
+                hidx = np.zeros((w.nb, 1), dtype=np.int32)
+            r = OB.head_backward(oracle.decode_bf16(x["q"][b, :, h]), oracle.decode_bf16(x["k"][b, :, h]),
+                                 oracle.decode_bf16(x["v"][b, :, h]), A, dout[b, :, h].astype(np.float64), grid,
+                                 w.block, w.keep_frac, R, branches=branches, idx=hidx)
+            ref[0][b, :, h] = r["dq"]
+            ref[1][b, :, h] = r["dk"]
+            ref[2][b, :, h] = r["dv"]
+            ref[3] += r["dA"]
+    return ref
+
+
+def _compare(label, got, ref):
+    stats = {"label": label}
+    for name, g, r in zip(("dq", "dk", "dv", "dA"), got, ref):
+        assert np.all(np.isfinite(g)), f"{label}: non-finite {name}"
+        err = np.abs(g - r)
+        scale = np.abs(r).max()
+        mean_rel = err.sum() / max(np.abs(r).sum(), 1e-300)
+        stats[name] = {"max_abs": float(err.max()), "max_ref": float(scale), "mean_rel": float(mean_rel)}
+        if scale == 0.0:
+            assert err.max() == 0.0, f"{label}: {name} should be zero"
+            continue
+        assert err.max() <= MAX_ABS_REL * scale, f"{label}: {name} max abs {err.max():.3g} vs max {scale:.3g}"
+        assert mean_rel <= MEAN_REL, f"{label}: {name} mean rel {mean_rel:.3g}"
+    if REPORT:
+        with open(REPORT, "a") as f:
+            f.write(json.dumps(stats) + "\n")
+    return stats
+
+
+def _case(w, label, branches=slra.BRANCH_BOTH, dout_scale=1.0):
+    x = I.make_inputs(w)
+    dout = I.make_dout(w.seed + 9000, w.batch, w.L, w.heads, w.head_dim, dout_scale)
+    p, got, idx = _gpu_bwd(w, x, dout, branches=branches)
+    ref = _oracle_bwd(w, x, dout, idx, branches)
+    return _compare(label, got, ref)
+
+
+EDGE_128 = W.Workload("bwd-edge-128", 1, 2, 128, 3, 10, 13, 32, 128, 0.3, 7160)         # L = 390, ragged
+EDGE_128_B64 = W.Workload("bwd-edge-128-b64", 1, 2, 128, 2, 9, 11, 64, 64, 0.25, 7192)  # block 64, r = 64
+EDGE_B2 = W.Workload("bwd-edge-b2", 2, 3, 128, 2, 9, 11, 32, 64, 0.25, 7410)            # batch 2
+DENSE = W.Workload("bwd-dense", 1, 2, 128, 4, 12, 16, 32, 128, 1.0, 7700)               # keep all
+MEDIUM = W.Workload("bwd-medium", 1, 2, 128, 4, 24, 32, 32, 128, 0.1, 7800)             # L = 3072
+
+
+@pytest.mark.parametrize("w", [W.TINY, EDGE_128, EDGE_128_B64, EDGE_B2, DENSE, MEDIUM], ids=lambda w: w.name)
+def test_backward_matches_oracle(w):
+    _case(w, w.name)
+
+
+@pytest.mark.parametrize("branches", [slra.BRANCH_SPARSE, slra.BRANCH_LOWRANK])
+@pytest.mark.parametrize("w", [W.TINY, EDGE_128], ids=lambda w: w.name)
+def test_backward_single_branch(w, branches):
+    _case(w, f"{w.name}-branches{branches}", branches=branches)
+
+
+def test_backward_deterministic_and_strided_inputs():
+    """Two calls give the same bits, and q, k, v as views of one fused QKV buffer give the same bits."""
+    import torch
+    w = EDGE_128
+    x = I.make_inputs(w)
+    dout = torch.from_numpy(I.make_dout(1, w.batch, w.L, w.heads, w.head_dim)).cuda()
+    p = slra.Problem.from_workload(w)
+    q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
+    a = slra.attn_bwd(p, q, k, v, A, dout)[:4]
+    b = slra.attn_bwd(p, q, k, v, A, dout)[:4]
+    qkv = torch.stack([q, k, v], dim=2).contiguous()
+    c = slra.attn_bwd(p, qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2], A, dout)[:4]
+    for ta, tb, tc in zip(a, b, c):
+        assert torch.equal(ta, tb) and torch.equal(ta, tc)
+
+
+def test_backward_dout_range_reported():
+    """A gradient too large for the fp16 operand copy is reported through the status word."""
+    import torch
+    w = W.TINY
+    x = I.make_inputs(w)
+    d = I.make_dout(2, w.batch, w.L, w.heads, w.head_dim)
+    d[0, 3, 1, 5] = 1e6
+    p = slra.Problem.from_workload(w)
+    q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
+    ws = slra.attn_bwd(p, q, k, v, A, torch.from_numpy(d).cuda())[4]
+    assert slra.device_status(ws) == slra.ERR_RANGE
