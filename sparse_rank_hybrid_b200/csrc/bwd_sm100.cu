@@ -244,7 +244,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool ok = true;
         for (int j = 0; j < keep; ++j) {
             ok = __all_sync(0xffffffffu, mbar_wait(bars + kDqBarSp, j & 1, tmo, abort_flag));
-            if (!ok) break;
+            if (!ok) {
+                if (lane == 0) fail();
+                break;
+            }
             tc_fence_after();
             uint32_t sr[NC][32], pr[NC][32];
 #pragma unroll
@@ -471,7 +474,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // the query block's lse and delta arrived with its tiles (same barrier phase)
             ok = __all_sync(0xffffffffu, mbar_wait(bars + kKvBarQFull + s, (t >> 1) & 1, tmo, abort_flag) &&
                                              mbar_wait(bars + kKvBarSp, t & 1, tmo, abort_flag));
-            if (!ok) break;
+            if (!ok) {
+                if (lane == 0) fail();
+                break;
+            }
             tc_fence_after();
             const float* lse_s = lseslot(s);
             const float* del_s = lse_s + BLK;
