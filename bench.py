@@ -412,6 +412,73 @@ def run_ours(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_backward(args, w):
+    """The backward pass (slra_attn_bwd) at the workload's shape on one GPU: ms per call, per-stage
+    times, and the sparse gradient kernels' throughput against the algorithmic count (five products per
+    kept (query block, key block) pair: S, dP, dQ, dK, dV = 2.5x the forward's kept FLOPs; the kernels
+    recompute S and dP once more, which is not counted).  One JSON line (not the benchmark contract)."""
+    import torch
+    from sparse_rank_hybrid_b200 import build as B
+    from sparse_rank_hybrid_b200 import slra
+
+    B.build()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+    for e in ev:
+        e.record()
+    torch.cuda.synchronize()
+    x = I.make_inputs(w)
+    q, k, v, A = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v", "A"))
+    dout = torch.from_numpy(I.make_dout(w.seed + 9000, w.batch, w.L, w.heads, w.head_dim)).to(dev)
+    prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in ev))
+    grads = tuple(torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
+                  for _ in range(3)) + (torch.empty((w.head_dim, w.rank), dtype=torch.float32, device=dev),)
+    ws = torch.empty(slra.bwd_workspace_bytes(prob), dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        slra.attn_bwd(prob, q, k, v, A, dout, grads=grads, workspace=ws)
+    torch.cuda.synchronize()
+    if slra.device_status(ws) != slra.OK:
+        raise RuntimeError("device status after warm-up")
+    f_total, f_sparse, f_lr, f_sc, f_attn, keep_blocks = _work(w, prob, ws, slra, 3)
+    clocks = ClockSampler(0 if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                          int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[0]))
+    clocks.start()
+    time.sleep(0.3)
+    tot, stages = [], []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        slra.attn_bwd(prob, q, k, v, A, dout, grads=grads, workspace=ws)
+        b.record(stream)
+        torch.cuda.synchronize()
+        tot.append(a.elapsed_time(b))
+        stages.append([ev[i].elapsed_time(ev[i + 1]) for i in range(6)])
+    clk = clocks.stop()
+    if slra.device_status(ws) != slra.OK:
+        raise RuntimeError("device status after timing")
+    st = [statistics.mean(s_[i] for s_ in stages) for i in range(6)]
+    ms = statistics.mean(tot)
+    _, tf_burst, tf_sust, src = peaks()
+    f_bwd_sparse = 2.5 * f_sparse
+    f_lr_bwd = 2.0 * F.lowrank_flops(w.L, w.rank, w.head_dim, w.batch * w.heads)  # ~2x the forward's chain
+    sparse_ms = st[2] + st[3]
+    line = {"backward": w.name, "ms_per_call": ms, "keep_blocks": keep_blocks,
+            "stage_ms": dict(zip(("recompute_forward", "dout_copy_and_lists", "dq_kernel", "dkdv_kernel",
+                                  "lowrank_grad", "-"), (round(x_, 4) for x_ in st))),
+            "sparse_bwd": {"algorithmic_flops": f_bwd_sparse, "ms": sparse_ms,
+                           "achieved_tflops": f_bwd_sparse / (sparse_ms * 1e-3) / 1e12,
+                           "frac_of_burst": f_bwd_sparse / (sparse_ms * 1e-3) / 1e12 / tf_burst,
+                           "peak": tf_burst, "peak_source": f"{src} burst bf16 (same rate as f16)"},
+            "lowrank_bwd_flops": f_lr_bwd,
+            "whole_call_tflops": (f_bwd_sparse + f_lr_bwd) / (ms * 1e-3) / 1e12,
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def run_sweep(args):
     """The keep x rank sweep at the Wan2.1-1.3B shape on one GPU: per point, ms per call, effective
     TFLOP/s, the attention kernel's share of the call and its burst-peak roofline fraction, and the
@@ -485,6 +552,8 @@ def main():
                     help="query/key projection layout: one shared A, separate Pq/Pk, per head, or both")
     ap.add_argument("--fusion", default="sum", choices=["sum", "gated"],
                     help="combine the branches by their sum or by the token-wise gate (synthetic Wg, bg = -2)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (slra_attn_bwd) at the workload's shape (one JSON line)")
     ap.add_argument("--sweep", action="store_true",
                     help="time the 20 keep x rank points at the Wan2.1-1.3B shape (one JSON line each)")
     ap.add_argument("--rope-inside", action="store_true",
@@ -509,6 +578,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args)
+        return
+    if args.backward:
+        run_backward(args, w)
         return
     if world > 1:
         import datetime

@@ -86,7 +86,9 @@ typedef enum slra_status {
     SLRA_ERR_WORKSPACE = 4,       /* workspace NULL, misaligned (256 B) or smaller than required         */
     SLRA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or a kernel launch failed                */
     SLRA_ERR_DEVICE_TIMEOUT = 6,  /* (device status) a bounded wait inside a kernel ran out              */
-    SLRA_ERR_RANGE = 7,           /* (device status) |value| >= 65504 after RoPE: does not fit fp16      */
+    SLRA_ERR_RANGE = 7,           /* (device status) a value does not fit the fp16 operands: |value| >=
+                                     65504 after RoPE, or a block of q^, k^ or v whose nonzero values all
+                                     lie below fp16's smallest normal 2^-14 (relative precision lost)     */
     SLRA_ERR_NO_DEVICE = 8,       /* no sm_100 device is current                                         */
     SLRA_ERR_SCRATCH_LIMIT = 9    /* slra_lowrank_summary_noalloc: problem exceeds its fixed scratch area */
 } slra_status;

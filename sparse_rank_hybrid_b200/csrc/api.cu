@@ -717,7 +717,7 @@ const char* slra_status_string(int s) {
         case SLRA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case SLRA_ERR_CUDA: return "CUDA call or kernel launch failed";
         case SLRA_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel ran out";
-        case SLRA_ERR_RANGE: return "input value out of fp16 range after RoPE";
+        case SLRA_ERR_RANGE: return "input values outside the fp16 operands' range after RoPE (overflow, or a block below 2^-14)";
         case SLRA_ERR_NO_DEVICE: return "no sm_100 device is current";
         case SLRA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the fixed no-allocation area holds";
         default: return "unknown status";

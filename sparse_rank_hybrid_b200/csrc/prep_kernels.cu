@@ -113,6 +113,9 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
     // the pairs whose position moved are reloaded
     double2 cs_c[4];
     int pos_c[4];
+    // largest |q^|, |k^|, |v| this thread wrote: a block whose nonzero values all lie below fp16's
+    // smallest normal (2^-14) has lost relative precision in the fp16 operands and is reported
+    float mq = 0.f, mk = 0.f, mv = 0.f;
 #pragma unroll
     for (int u = 0; u < 4; ++u) pos_c[u] = -1;
     for (int i = grp; i < blk; i += G) {
@@ -150,8 +153,10 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
                 sq[u][0] += qy0; sq[u][1] += qy1; sk[u][0] += ky0; sk[u][1] += ky1;
                 const float a0 = static_cast<float>(qy0), a1 = static_cast<float>(qy1);
                 const float c0 = static_cast<float>(ky0), c1 = static_cast<float>(ky1);
-                m = fmaxf(m, fmaxf(fmaxf(fabsf(a0), fabsf(a1)), fmaxf(fmaxf(fabsf(c0), fabsf(c1)),
-                                                                     fmaxf(fabsf(vf.x), fabsf(vf.y)))));
+                mq = fmaxf(mq, fmaxf(fabsf(a0), fabsf(a1)));
+                mk = fmaxf(mk, fmaxf(fabsf(c0), fabsf(c1)));
+                mv = fmaxf(mv, fmaxf(fabsf(vf.x), fabsf(vf.y)));
+                m = fmaxf(m, fmaxf(fmaxf(mq, mk), mv));
                 const __half2 hq = __floats2half2_rn(a0, a1), hk = __floats2half2_rn(c0, c1),
                               hv = __floats2half2_rn(vf.x, vf.y);
                 qo2[u] = *reinterpret_cast<const uint32_t*>(&hq);
@@ -169,7 +174,20 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
             *reinterpret_cast<uint4*>(vh + dst) = z4;
         }
     }
+    // block maxima of |q^|, |k^|, |v| (non-negative floats order like their bit patterns)
+    __shared__ unsigned int blk_max[3];
+    if (threadIdx.x < 3) blk_max[threadIdx.x] = 0u;
     __syncthreads();  // the tiles are consumed; the reduction reuses their space
+    {
+        const unsigned int wq = __reduce_max_sync(0xffffffffu, __float_as_uint(mq));
+        const unsigned int wk = __reduce_max_sync(0xffffffffu, __float_as_uint(mk));
+        const unsigned int wv = __reduce_max_sync(0xffffffffu, __float_as_uint(mv));
+        if ((threadIdx.x & 31) == 0) {
+            atomicMax(&blk_max[0], wq);
+            atomicMax(&blk_max[1], wk);
+            atomicMax(&blk_max[2], wv);
+        }
+    }
     double* red = reinterpret_cast<double*>(smem);  // [G][q0,q1,k0,k1][D/2]
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -194,6 +212,13 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
         kbar[o] = c0 / cnt; kbar[o + 1] = c1 / cnt;
     }
     if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, kDevRange);
+    if (threadIdx.x == 0) {
+        constexpr float kMinNormalF16 = 6.103515625e-05f;  // 2^-14
+        for (int t = 0; t < 3; ++t) {
+            const float mx = __uint_as_float(blk_max[t]);
+            if (mx > 0.f && mx < kMinNormalF16) atomicOr(status, kDevRange);
+        }
+    }
 }
 
 // The q, k, v tiles, or the block-sum exchange that later reuses them ([256/(D/8)][4][D/2] fp64 =

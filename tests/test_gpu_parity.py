@@ -244,6 +244,7 @@ def test_shift_invariance_on_gpu():
     g0, g1 = parity.run_gpu(p0, x), parity.run_gpu(p1, x)
     assert np.array_equal(g0["idx"], g1["idx"])
     d = np.abs(g0["out"] - g1["out"])
+    _log({"label": "shift-gpu-vs-gpu", "max_abs": float(d.max()), "mean_rel": float(d.sum() / np.abs(g0["out"]).sum())})
     assert d.max() <= parity.MAX_ABS and d.sum() / np.abs(g0["out"]).sum() <= parity.MEAN_REL
     parity.compare(p1, x, g1, label="tiny-shifted")
 
@@ -336,7 +337,7 @@ def _rescaled(x, seed, q=1.0, k=1.0, v=1.0, q_uniform=None):
 # of order one while the rotated queries come within 3% of fp16's largest finite value (65,504).
 SCALE_CASES = [
     ("qkv-1e-3", dict(q=1e-3, k=1e-3, v=1e-3), 1.0),
-    ("qkv-1e-5", dict(q=1e-5, k=1e-5, v=1e-5), 1.0),
+    ("qkv-1e-5", dict(q=1e-5, k=1e-5, v=1e-5), 1.0),  # below fp16's normal range: reported (see below)
     ("v-1e-4", dict(v=1e-4), 1.0),
     ("v-300", dict(v=300.0), 300.0),
     ("q-near-fp16-max", dict(k=1e-4, q_uniform=45000.0), 1.0),
@@ -351,7 +352,10 @@ def test_input_scales(label, factors, abs_mult, D):
     w = W.Workload(f"scale-{label}-{D}", 1, 2, D, 3, 10, 13, 32 if D == 128 else 16, 64, 0.3, 7500 + D)
     x = _rescaled(I.make_custom(w.seed, 1, (w.T, w.H, w.W), w.heads, D, w.rank), w.seed + 1, **factors)
     p = slra.Problem.from_workload(w)
-    gpu = parity.run_gpu(p, x)
+    # blocks whose values all sit below fp16's smallest normal (2^-14) are reported as a range problem
+    # (the fp16 copies keep only absolute precision there); the result is still compared
+    expect = slra.ERR_RANGE if label == "qkv-1e-5" else slra.OK
+    gpu = parity.run_gpu(p, x, expect_status=expect)
     _log(parity.compare(p, x, gpu, label=f"scale-{label}-{D}", max_abs=parity.MAX_ABS * abs_mult))
 
 
