@@ -640,9 +640,11 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
                                                        float* __restrict__ dz_part, float* __restrict__ da_part) {
     constexpr int TT = LrTile<R>::T;
     extern __shared__ __align__(16) float smf[];
-    float* As = smf;                    // [D][R]
-    float* Ss = As + D * R;             // [R][D]
-    float* zs = Ss + R * D;             // [R]
+    // A and S padded by one column: the loops below read them with consecutive lanes walking either
+    // index, and the padding keeps both walks free of shared-memory bank conflicts
+    float* As = smf;                    // [D][R+1]
+    float* Ss = As + D * (R + 1);       // [R][D+1]
+    float* zs = Ss + R * (D + 1);       // [R]
     float* xs = zs + R;                 // [TT][D+1] q
     float* gs = xs + TT * (D + 1);      // [TT][D+1] dO
     float* us = gs + TT * (D + 1);      // [TT][R+1] u
@@ -660,8 +662,8 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
     const int ntiles = (g.L + TT - 1) / TT;
     const int per = (ntiles + nsplit - 1) / nsplit;
     const int t0 = split * per, t1 = min(ntiles, t0 + per);
-    for (int e = tid; e < D * R; e += 256) As[e] = __bfloat162float(A[e]);
-    for (int e = tid; e < R * D; e += 256) Ss[e] = S[static_cast<size_t>(bh) * R * D + e];
+    for (int e = tid; e < D * R; e += 256) As[(e / R) * (R + 1) + e % R] = __bfloat162float(A[e]);
+    for (int e = tid; e < R * D; e += 256) Ss[(e / D) * (D + 1) + e % D] = S[static_cast<size_t>(bh) * R * D + e];
     if (tid < R) zs[tid] = z[static_cast<size_t>(bh) * R + tid];
     const int e_own = tid % D, cg = tid / D;
     float acc_s[NA], acc_a[NA];  // dS[c][e_own], dA[e_own][c] for c = cg + G i
@@ -691,8 +693,8 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
             float u = 0.f, gg = 0.f;
 #pragma unroll 8
             for (int d = 0; d < D; ++d) {
-                u = fmaf(xr[d], As[d * R + c], u);
-                gg = fmaf(Ss[c * D + d], gr[d], gg);
+                u = fmaf(xr[d], As[d * (R + 1) + c], u);
+                gg = fmaf(Ss[c * (D + 1) + d], gr[d], gg);
             }
             us[tt * (R + 1) + c] = u;
             Gs[tt * (R + 1) + c] = gg;
@@ -768,7 +770,7 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
             if (n >= g.L) continue;
             float s = 0.f;
 #pragma unroll 8
-            for (int c = 0; c < R; ++c) s = fmaf(dus[tt * (R + 1) + c], As[d * R + c], s);
+            for (int c = 0; c < R; ++c) s = fmaf(dus[tt * (R + 1) + c], As[d * (R + 1) + c], s);
             dq[g.so.row(b, n, h) + d] += s;
         }
     }
@@ -794,9 +796,9 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
                                                        float* __restrict__ da_part) {
     constexpr int TT = LrTile<R>::T;
     extern __shared__ __align__(16) float smf[];
-    float* As = smf;                    // [D][R]
-    float* Ss = As + D * R;             // [R][D] dS
-    float* zs = Ss + R * D;             // [R] dz
+    float* As = smf;                    // [D][R+1] (padded as in the query pass)
+    float* Ss = As + D * (R + 1);       // [R][D+1] dS
+    float* zs = Ss + R * (D + 1);       // [R] dz
     float* xs = zs + R;                 // [TT][D+1] k
     float* vs = xs + TT * (D + 1);      // [TT][D+1] v
     float* us = vs + TT * (D + 1);      // [TT][R+1] u
@@ -810,8 +812,8 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
     const int ntiles = (g.L + TT - 1) / TT;
     const int per = (ntiles + nsplit - 1) / nsplit;
     const int t0 = split * per, t1 = min(ntiles, t0 + per);
-    for (int e = tid; e < D * R; e += 256) As[e] = __bfloat162float(A[e]);
-    for (int e = tid; e < R * D; e += 256) Ss[e] = dS[static_cast<size_t>(bh) * R * D + e];
+    for (int e = tid; e < D * R; e += 256) As[(e / R) * (R + 1) + e % R] = __bfloat162float(A[e]);
+    for (int e = tid; e < R * D; e += 256) Ss[(e / D) * (D + 1) + e % D] = dS[static_cast<size_t>(bh) * R * D + e];
     if (tid < R) zs[tid] = dz[static_cast<size_t>(bh) * R + tid];
     const int e_own = tid % D, cg = tid / D;
     float acc_a[NA];
@@ -840,8 +842,8 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
             float u = 0.f, dp = 0.f;
 #pragma unroll 8
             for (int d = 0; d < D; ++d) {
-                u = fmaf(xr[d], As[d * R + c], u);
-                dp = fmaf(Ss[c * D + d], vr[d], dp);
+                u = fmaf(xr[d], As[d * (R + 1) + c], u);
+                dp = fmaf(Ss[c * (D + 1) + d], vr[d], dp);
             }
             us[tt * (R + 1) + c] = u;
             ps[tt * (R + 1) + c] = dp;
@@ -881,8 +883,8 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
             float sv = 0.f, sk = 0.f;
 #pragma unroll 8
             for (int c = 0; c < R; ++c) {
-                sv = fmaf(Ss[c * D + d], psis[tt * (R + 1) + c], sv);
-                sk = fmaf(ps[tt * (R + 1) + c], As[d * R + c], sk);
+                sv = fmaf(Ss[c * (D + 1) + d], psis[tt * (R + 1) + c], sv);
+                sk = fmaf(ps[tt * (R + 1) + c], As[d * (R + 1) + c], sk);
             }
             const long long r = g.so.row(b, n, h) + d;
             dv[r] += sv;
@@ -906,9 +908,9 @@ __global__ void bwd_da_reduce_kernel(const float* __restrict__ da_part, int nslo
 // ------------------------------------------------------------------------------------ launchers
 size_t lr_bwd_smem(int D, int R, bool qpass) {
     const int TT = R <= 64 ? 32 : 16;
-    if (qpass)
-        return sizeof(float) * (2 * D * R + R + 2 * TT * (D + 1) + 3 * TT * (R + 1) + 2 * TT * R + 2 * TT);
-    return sizeof(float) * (2 * D * R + R + 2 * TT * (D + 1) + 3 * TT * (R + 1));
+    const int mats = D * (R + 1) + R * (D + 1);  // padded A and S (or dS)
+    if (qpass) return sizeof(float) * (mats + R + 2 * TT * (D + 1) + 3 * TT * (R + 1) + 2 * TT * R + 2 * TT);
+    return sizeof(float) * (mats + R + 2 * TT * (D + 1) + 3 * TT * (R + 1));
 }
 
 int lr_bwd_nsplit(const Geom& g) {
