@@ -222,3 +222,70 @@ def head_backward_steps(q, k, v, A, dout, grid, block: int, rank: int, idx, *, t
     dk = dk + duk @ A.T
     dA = q.T @ duq + k.T @ duk
     return dict(dq=dq, dk=dk, dv=dv, dA=dA)
+
+
+def head_backward_sampled(q, k, v, A, dout, grid, block: int, rank: int, idx, qblocks, kblocks, *, theta=1e4,
+                          offset=(0, 0, 0), split=None):
+    """The gradients of head_backward_steps (relu features, RoPE outside, one shared projection, plain
+    sum) evaluated only where asked: dq on the rows of the query blocks `qblocks`, dk and dv on the rows
+    of the key blocks `kblocks`, and dA in full.  The sparse terms of a query row involve only its own
+    kept key blocks; those of a key row involve only the query blocks that kept its block (each with its
+    own softmax over its own kept set); the low-rank terms need the global sums S, z, dS, dz, which are
+    O(L r D).  So a full-size head is affordable in fp64.  Returns dict(dq={alpha: [rows, D]},
+    dk={beta: [rows, D]}, dv={beta: [rows, D]}, dA)."""
+    q, k, v, A, dout = (np.asarray(a, dtype=np.float64) for a in (q, k, v, A, dout))
+    L, D = q.shape
+    nb = idx.shape[0]
+    cs = rope_cos_sin(grid, D, theta, offset, split)
+    sc = 1.0 / math.sqrt(D)
+    qh, kh = _rot_np(q, cs, D // 2), _rot_np(k, cs, D // 2)
+    rows = lambda a: np.arange(a * block, min(L, (a + 1) * block))
+    keys = lambda a: np.concatenate([rows(b) for b in idx[a]])
+
+    def softmax_block(a):
+        """P, dS over the kept keys of query block a (rows of a x kept keys), and those keys."""
+        r, kk = rows(a), keys(a)
+        s = qh[r] @ kh[kk].T * sc
+        s = s - s.max(axis=1, keepdims=True)
+        P = np.exp(s)
+        P /= P.sum(axis=1, keepdims=True)
+        o_s = P @ v[kk]
+        delta = (dout[r] * o_s).sum(axis=1, keepdims=True)
+        dS = P * (dout[r] @ v[kk].T - delta)
+        return r, kk, P, dS
+
+    # low-rank branch: global sums
+    r2 = rank // 2
+    uq, uk = q @ A, k @ A
+    phq, phk = np.maximum(uq, 0.0), np.maximum(uk, 0.0)
+    psq, psk = _rot_np(phq, cs, r2), _rot_np(phk, cs, r2)
+    Sm, z = psk.T @ v, phk.sum(axis=0)
+    den = phq @ z + 1e-6
+    G = dout @ Sm.T
+    dden = -(psq * G).sum(axis=1) / den ** 2
+    dphq = _unrotate(G / den[:, None], cs, r2) + dden[:, None] * z[None, :]
+    dSm = psq.T @ (dout / den[:, None])
+    dz = dden @ phq
+    dphk = _unrotate(v @ dSm.T, cs, r2) + dz[None, :]
+    duq, duk = dphq * (uq > 0), dphk * (uk > 0)
+    dA = q.T @ duq + k.T @ duk
+    out = dict(dq={}, dk={}, dv={}, dA=dA)
+    for a in qblocks:
+        r, kk, P, dS = softmax_block(a)
+        dqh = dS @ kh[kk] * sc
+        out["dq"][a] = _unrotate(dqh, cs[r], D // 2) + duq[r] @ A.T
+    for b in kblocks:
+        kr = rows(b)
+        dkh = np.zeros((kr.size, D))
+        dvs = np.zeros((kr.size, D))
+        for a in range(nb):
+            if b not in idx[a]:
+                continue
+            r, kk, P, dS = softmax_block(a)
+            pos = np.searchsorted(kk, kr) if np.all(np.diff(kk) > 0) else None
+            sel = pos if pos is not None else np.array([np.where(kk == j)[0][0] for j in kr])
+            dvs += P[:, sel].T @ dout[r]
+            dkh += dS[:, sel].T @ qh[r] * sc
+        out["dk"][b] = _unrotate(dkh, cs[kr], D // 2) + duk[kr] @ A.T
+        out["dv"][b] = dvs + psk[kr] @ dSm
+    return out

@@ -147,3 +147,38 @@ def test_backward_dout_range_reported():
     q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
     ws = slra.attn_bwd(p, q, k, v, A, torch.from_numpy(d).cuda())[4]
     assert slra.device_status(ws) == slra.ERR_RANGE
+
+
+def test_backward_wan_1_3b_sampled():
+    """The full Wan2.1-1.3B shape (32,760 tokens, 12 heads, keep 26/256): the GPU backward of the whole
+    problem, compared on a sampled head's dq over sampled query blocks (first, last = ragged, random) and
+    dk, dv over sampled key blocks (first, last, and the most-kept one), and dA (all heads) against the
+    oracle's sampled gradients (head_backward_sampled, the explicit steps restricted to those rows)."""
+    import oracle
+    from oracle import backward as OB
+    w = W.WAN_1_3B
+    x = I.make_inputs(w)
+    dout = I.make_dout(w.seed + 9000, w.batch, w.L, w.heads, w.head_dim)
+    p, got, idx = _gpu_bwd(w, x, dout)
+    D, R, Hh = w.head_dim, w.rank, w.heads
+    A = oracle.decode_bf16(x["A"]).reshape(D, R)
+    grid = (w.T, w.H, w.W)
+    h = 5
+    rng = np.random.default_rng(13)
+    qbs = sorted({0, w.nb - 1, *rng.choice(w.nb, 2, replace=False).tolist()})
+    counts = np.bincount(idx[h].ravel(), minlength=w.nb)
+    kbs = sorted({0, w.nb - 1, int(counts.argmax())})
+    dA_ref = np.zeros((D, R))
+    for hh in range(Hh):
+        r = OB.head_backward_sampled(oracle.decode_bf16(x["q"][0, :, hh]), oracle.decode_bf16(x["k"][0, :, hh]),
+                                     oracle.decode_bf16(x["v"][0, :, hh]), A, dout[0, :, hh].astype(np.float64),
+                                     grid, w.block, R, idx[hh], qbs if hh == h else [], kbs if hh == h else [])
+        dA_ref += r["dA"]
+        if hh == h:
+            smp = r
+    rows = lambda a: slice(a * w.block, min(w.L, (a + 1) * w.block))
+    got_s = [np.concatenate([got[0][0, rows(a), h] for a in qbs]), np.concatenate([got[1][0, rows(b), h] for b in kbs]),
+             np.concatenate([got[2][0, rows(b), h] for b in kbs]), got[3]]
+    ref_s = [np.concatenate([smp["dq"][a] for a in qbs]), np.concatenate([smp["dk"][b] for b in kbs]),
+             np.concatenate([smp["dv"][b] for b in kbs]), dA_ref]
+    _compare("wan1.3b-sampled", got_s, ref_s)

@@ -781,3 +781,31 @@ def test_backward_steps_match_autograd(oracle_mod):
         m = B.head_backward_steps(q, k, v, A, dout, grid, w.block, w.rank, g["idx"])
         for name in ("dq", "dk", "dv", "dA"):
             assert np.allclose(m[name], g[name], rtol=1e-10, atol=1e-12), name
+
+
+def test_backward_sampled_equals_full_steps(oracle_mod):
+    """head_backward_sampled (the gradients evaluated only on chosen query / key blocks, plus dA, for
+    full-size heads) equals head_backward_steps on every block of a small ragged case, for a subset of
+    blocks, and for empty subsets (dA alone); a key block that no query block kept gets only its
+    low-rank gradient."""
+    from oracle import backward as OB
+    rng = np.random.default_rng(31)
+    grid, D, R, block = (3, 5, 7), 32, 16, 16  # L = 105: a ragged last block of 9 tokens
+    L = 105
+    q, k, v = (rng.standard_normal((L, D)) for _ in range(3))
+    A = rng.standard_normal((D, R)) / np.sqrt(D)
+    dout = rng.standard_normal((L, D))
+    qh, kh = oracle_mod.rope_rows(q, grid, D // 2), oracle_mod.rope_rows(k, grid, D // 2)
+    s = oracle_mod.block_scores(oracle_mod.block_means(qh, block), oracle_mod.block_means(kh, block))
+    nb = s.shape[0]
+    idx, _ = oracle_mod.topk(s, 2)
+    full = OB.head_backward_steps(q, k, v, A, dout, grid, block, R, idx)
+    rows = lambda a: slice(a * block, min(L, (a + 1) * block))
+    for qbs, kbs in ((range(nb), range(nb)), ([0, nb - 1], [3, nb - 1]), ([], [])):
+        smp = OB.head_backward_sampled(q, k, v, A, dout, grid, block, R, idx, qbs, kbs)
+        assert np.allclose(smp["dA"], full["dA"], rtol=1e-12, atol=1e-12)
+        for a in qbs:
+            assert np.allclose(smp["dq"][a], full["dq"][rows(a)], rtol=1e-12, atol=1e-12)
+        for b in kbs:
+            assert np.allclose(smp["dk"][b], full["dk"][rows(b)], rtol=1e-12, atol=1e-12)
+            assert np.allclose(smp["dv"][b], full["dv"][rows(b)], rtol=1e-12, atol=1e-12)
