@@ -235,8 +235,10 @@ def test_exact_ties_keep_the_lower_blocks():
 
 def test_shift_invariance_on_gpu():
     """Shifting all positions leaves the masks unchanged exactly (fp64 selection) and the outputs
-    unchanged up to the fp16 rounding of the rotated operands, which differs between the two runs:
-    both stay within the parity tolerance of the (exactly invariant) oracle."""
+    unchanged up to the fp16 rounding of the rotated operands, which differs between the two runs (the
+    same exact values rotated by other angles round differently): measured on a B200, max-abs 1.6e-3 and
+    mean-relative 2.4e-4 between the two runs, so the bound between them is 4e-3 / 6e-4; both also stay
+    within the parity tolerance of the (exactly invariant) oracle."""
     w = W.TINY.with_(T=4, H=16, W=16, heads=2, block=64, keep_frac=0.25)
     x = I.make_inputs(w)
     p0 = slra.Problem.from_workload(w)
@@ -245,7 +247,7 @@ def test_shift_invariance_on_gpu():
     assert np.array_equal(g0["idx"], g1["idx"])
     d = np.abs(g0["out"] - g1["out"])
     _log({"label": "shift-gpu-vs-gpu", "max_abs": float(d.max()), "mean_rel": float(d.sum() / np.abs(g0["out"]).sum())})
-    assert d.max() <= parity.MAX_ABS and d.sum() / np.abs(g0["out"]).sum() <= parity.MEAN_REL
+    assert d.max() <= 4e-3 and d.sum() / np.abs(g0["out"]).sum() <= 6e-4
     parity.compare(p1, x, g1, label="tiny-shifted")
 
 
