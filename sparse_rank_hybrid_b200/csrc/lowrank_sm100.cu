@@ -26,11 +26,21 @@ namespace {
 constexpr int kD = 128;
 constexpr int kTok = 128;                      // tokens per tile
 constexpr int kTileBytes = kTok * kD * 2;      // 32 KB (two 64-column slabs of 16 KB)
-constexpr int kStages = 2;
+// k/v stages per CTA: rank <= 48 uses one stage (about 110 KB of shared memory) and 256 TMEM columns,
+// so two CTAs share an SM and hide each other's latencies; larger ranks use two stages, one CTA per SM
+// (rank 64's single-stage layout, 114 KB, would not fit twice).  TMEM: phi at column 0 (R columns), S^T
+// at column 128 (2 RP columns).
+template <int R>
+struct LrCfg {
+    static constexpr int kStages = R <= 48 ? 1 : 2;
+    static constexpr int kTmemCols = R <= 64 ? 256 : 512;
+    static constexpr int kCtasPerSm = R <= 48 ? 2 : 1;
+};
+constexpr int kMaxStages = 2;
 
 struct LrLayout {
     int rp;           // padded psi width per half (64 or 128)
-    int off_k[kStages], off_v[kStages];
+    int off_k[kMaxStages], off_v[kMaxStages];
     int off_at;       // A^T [r][128] bf16, K-major swizzled
     int off_psi;      // [128 tokens][2*rp] bf16, 64-column slabs
     int off_zred;     // [8 warps][R/2] fp32
@@ -39,11 +49,12 @@ struct LrLayout {
     int bytes;
 };
 
-__host__ __device__ inline LrLayout lr_layout(int R) {
+__host__ __device__ inline LrLayout lr_layout(int R, int stages) {
     LrLayout l;
     l.rp = R <= 64 ? 64 : 128;
     int o = 0;
-    for (int s = 0; s < kStages; ++s) { l.off_k[s] = o; o += kTileBytes; l.off_v[s] = o; o += kTileBytes; }
+    for (int s = 0; s < kMaxStages; ++s) l.off_k[s] = l.off_v[s] = 0;
+    for (int s = 0; s < stages; ++s) { l.off_k[s] = o; o += kTileBytes; l.off_v[s] = o; o += kTileBytes; }
     l.off_at = o;
     o += ((R * 256 + 1023) / 1024) * 1024;
     l.off_psi = o;
@@ -78,10 +89,11 @@ struct LrArgs {
 // kDefault: relu features with the RoPE (the benchmark's configuration); the activation and no-RoPE
 // branches then fold away at compile time.
 template <int R, bool kDefault>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, LrCfg<R>::kCtasPerSm)
     lowrank_sm100_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          LrArgs a, Geom g) {
-    const LrLayout lay = lr_layout(R);
+    constexpr int kStages = LrCfg<R>::kStages;
+    const LrLayout lay = lr_layout(R, kStages);
     const int act = kDefault ? 0 : g.act;
     const int norope = kDefault ? 0 : g.norope;
     const int inside = kDefault ? 0 : g.inside;  // RoPE before the activation; z then sums psi
@@ -107,7 +119,7 @@ __global__ void __launch_bounds__(256, 1)
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, LrCfg<R>::kTmemCols);
         tmem_relinquish();
     }
     const int ntiles = (g.L + kTok - 1) / kTok;
@@ -160,7 +172,7 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t at_addr = smem_addr(smem + lay.off_at), psi_addr = smem_addr(smem + lay.off_psi);
 
     // thread 0's bookkeeping of issued / observed operations (for the bounded drain on abort)
-    int n_load[kStages] = {0, 0}, n_wait[kStages] = {0, 0};
+    int n_load[kMaxStages] = {0, 0}, n_wait[kMaxStages] = {0, 0};
     int n_s_issued = 0, n_s_done = 0, n_phi_issued = 0;
     int q_total = 0;  // tiles this CTA will process
     {
@@ -206,8 +218,7 @@ __global__ void __launch_bounds__(256, 1)
     if (tid == 0 && !*abort_flag) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
-        issue_load(0);
-        issue_load(1);
+        for (int st = 0; st < kStages; ++st) issue_load(st);
         if (q_total > 0 && !issue_phi(0)) fail();
     }
 
@@ -319,15 +330,29 @@ __global__ void __launch_bounds__(256, 1)
                 umma_commit(bar_s);
                 ++n_s_issued;
                 bool good = true;
-                // the next tile's phi product goes in right behind (its k tile is already loading),
-                // unless it needs another head's projection: then it is issued once that is staged
-                if (q + 1 < q_total && (!g.a_stride || head_of_tile(q + 1) == h_loaded)) good = issue_phi(q + 1);
-                // stage s is free once this S product is done: refill it with the tile two ahead
-                if (good && mbar_wait(bar_s, n_s_done & 1, tmo, abort_flag)) {
-                    ++n_s_done;
-                    issue_load(q + kStages);
+                const bool next_phi = q + 1 < q_total && (!g.a_stride || head_of_tile(q + 1) == h_loaded);
+                if constexpr (kStages > 1) {
+                    // the next tile's phi product goes in right behind (its k tile is already loading),
+                    // unless it needs another head's projection: then it is issued once that is staged
+                    if (next_phi) good = issue_phi(q + 1);
+                    // stage s is free once this S product is done: refill it with the tile two ahead
+                    if (good && mbar_wait(bar_s, n_s_done & 1, tmo, abort_flag)) {
+                        ++n_s_done;
+                        issue_load(q + kStages);
+                    } else {
+                        fail();
+                    }
                 } else {
-                    fail();
+                    // one stage: the next tile loads once this S product is done with v, then its phi
+                    // product follows (the other CTA on the SM works meanwhile)
+                    if (mbar_wait(bar_s, n_s_done & 1, tmo, abort_flag)) {
+                        ++n_s_done;
+                        issue_load(q + 1);
+                        if (next_phi) good = issue_phi(q + 1);
+                        if (!good) fail();
+                    } else {
+                        fail();
+                    }
                 }
             }
             ++n_s;
@@ -389,7 +414,7 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, LrCfg<R>::kTmemCols);
     }
 }
 
@@ -405,7 +430,7 @@ int lowrank_tc_tiles_per_split(const Geom& g, int nsplit) {
 template <int R, bool kDefault>
 static cudaError_t lr_tc_launch_v(const CUtensorMap& tk, const CUtensorMap& tv, const LrArgs& a, const Geom& g,
                                   cudaStream_t st) {
-    const size_t sm = static_cast<size_t>(lr_layout(R).bytes) + 1024;
+    const size_t sm = static_cast<size_t>(lr_layout(R, LrCfg<R>::kStages).bytes) + 1024;
     cudaError_t e = cudaFuncSetAttribute(lowrank_sm100_kernel<R, kDefault>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
@@ -413,7 +438,8 @@ static cudaError_t lr_tc_launch_v(const CUtensorMap& tk, const CUtensorMap& tv, 
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int items = g.BH() * a.nsplit;
-    lowrank_sm100_kernel<R, kDefault><<<items < sms ? items : sms, 256, sm, st>>>(tk, tv, a, g);
+    const int slots = sms * LrCfg<R>::kCtasPerSm;
+    lowrank_sm100_kernel<R, kDefault><<<items < slots ? items : slots, 256, sm, st>>>(tk, tv, a, g);
     return cudaGetLastError();
 }
 template <int R>
