@@ -896,6 +896,333 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
     for (int i = 0; i < NA; ++i) da_part[slot * D * R + e_own * R + cg + G * i] = acc_a[i];
 }
 
+// ---- register-tiled passes for rank <= 64 (32-token tiles): lane = token of the tile; each warp owns
+// FC = R/8 consecutive features (for the products over the head dimension) or D/8 consecutive dims (for
+// the products over the features), so A, S and dS are read as warp-wide broadcast vectors and the
+// per-token operands as conflict-free gathers (rows padded to D+1 / R+1), and a token's rotation pairs
+// stay inside one thread.
+template <int N>
+__device__ __forceinline__ void ld_bcast(float (&dst)[N], const float* src) {  // 8-B aligned, N even
+#pragma unroll
+    for (int i = 0; i < N; i += 2) {
+        const float2 v = *reinterpret_cast<const float2*>(src + i);
+        dst[i] = v.x;
+        dst[i + 1] = v.y;
+    }
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16* __restrict__ q,
+                                                             const float* __restrict__ dout,
+                                                             const __nv_bfloat16* __restrict__ A,
+                                                             const float* __restrict__ S, const float* __restrict__ z,
+                                                             const double2* __restrict__ tab,
+                                                             const int2* __restrict__ pairs, Geom g, int nsplit,
+                                                             float* __restrict__ dq, float* __restrict__ ds_part,
+                                                             float* __restrict__ dz_part, float* __restrict__ da_part) {
+    constexpr int TT = 32, FC = R / 8, DC = D / 8;
+    static_assert(R <= 64 && FC % 2 == 0, "rank 16..64");
+    extern __shared__ __align__(16) float smf[];
+    float* Au = smf;                   // [D][R]   A
+    float* At = Au + D * R;            // [R][D]   A^T
+    float* St = At + R * D;            // [D][R]   S^T
+    float* zs = St + D * R;            // [R]
+    float* xs = zs + R;                // [TT][D+1] q
+    float* gs = xs + TT * (D + 1);     // [TT][D+1] dO
+    float* ws = gs + TT * (D + 1);     // [TT][R]   psi / den
+    float* dus = ws + TT * R;          // [TT][R+1] du
+    float* phs = dus + TT * (R + 1);   // [TT][R]   phi
+    float* red = phs + TT * R;         // [8][2][TT] per-warp partial dots
+    float* dd = red + 8 * 2 * TT;      // [TT] dden
+    constexpr int G = 256 / D;
+    constexpr int NA = R / G;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int split = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int ntiles = (g.L + TT - 1) / TT;
+    const int per = (ntiles + nsplit - 1) / nsplit;
+    const int t0 = split * per, t1 = min(ntiles, t0 + per);
+    for (int e = tid; e < D * R; e += 256) {
+        const float a = __bfloat162float(A[e]);
+        Au[e] = a;
+        At[(e % R) * D + e / R] = a;
+    }
+    for (int e = tid; e < R * D; e += 256) St[(e % D) * R + e / D] = S[static_cast<size_t>(bh) * R * D + e];
+    if (tid < R) zs[tid] = z[static_cast<size_t>(bh) * R + tid];
+    const int e_own = tid % D, cg = tid / D;
+    float acc_s[NA], acc_a[NA];
+#pragma unroll
+    for (int i = 0; i < NA; ++i) acc_s[i] = acc_a[i] = 0.f;
+    float acc_z = 0.f;
+    const int c0 = warp * FC, d0 = warp * DC;
+    for (int tile = t0; tile < t1; ++tile) {
+        const int n0 = tile * TT;
+        __syncthreads();
+        for (int e = tid; e < TT * (D / 2); e += 256) {
+            const int tt = e / (D / 2), dp = e % (D / 2);
+            const int n = n0 + tt;
+            float2 xf = make_float2(0.f, 0.f), gf = make_float2(0.f, 0.f);
+            if (n < g.L) {
+                xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + g.sq.row(b, n, h) + 2 * dp));
+                gf = *reinterpret_cast<const float2*>(dout + g.so.row(b, n, h) + 2 * dp);
+            }
+            xs[tt * (D + 1) + 2 * dp] = xf.x; xs[tt * (D + 1) + 2 * dp + 1] = xf.y;
+            gs[tt * (D + 1) + 2 * dp] = gf.x; gs[tt * (D + 1) + 2 * dp + 1] = gf.y;
+        }
+        __syncthreads();
+        // u = q A and G = S dO for token `lane`, features [c0, c0 + FC)
+        float u[FC], gg[FC];
+#pragma unroll
+        for (int f = 0; f < FC; ++f) u[f] = gg[f] = 0.f;
+        const float* xr = xs + lane * (D + 1);
+        const float* gr = gs + lane * (D + 1);
+#pragma unroll 4
+        for (int d = 0; d < D; ++d) {
+            float av[FC], sv[FC];
+            ld_bcast(av, Au + d * R + c0);
+            ld_bcast(sv, St + d * R + c0);
+            const float x = xr[d], go = gr[d];
+#pragma unroll
+            for (int f = 0; f < FC; ++f) {
+                u[f] = fmaf(x, av[f], u[f]);
+                gg[f] = fmaf(sv[f], go, gg[f]);
+            }
+        }
+        // phi, psi, partial den = phi . z and psi . G over this warp's features
+        const int n = n0 + lane;
+        const bool live = n < g.L;
+        const int nt = live ? n : 0;
+        float phi[FC], psi[FC], cf[FC / 2], sf[FC / 2];
+        float den_p = 0.f, dot_p = 0.f;
+#pragma unroll
+        for (int pp = 0; pp < FC / 2; ++pp) {
+            const int p = c0 / 2 + pp;
+            const int2 pi = pairs[p];
+            const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
+            cf[pp] = static_cast<float>(cs.x);
+            sf[pp] = static_cast<float>(cs.y);
+            const float x0 = fmaxf(u[2 * pp], 0.f), x1 = fmaxf(u[2 * pp + 1], 0.f);
+            phi[2 * pp] = x0;
+            phi[2 * pp + 1] = x1;
+            psi[2 * pp] = x0 * cf[pp] - x1 * sf[pp];
+            psi[2 * pp + 1] = x0 * sf[pp] + x1 * cf[pp];
+            den_p = fmaf(x0, zs[c0 + 2 * pp], fmaf(x1, zs[c0 + 2 * pp + 1], den_p));
+            dot_p = fmaf(psi[2 * pp], gg[2 * pp], fmaf(psi[2 * pp + 1], gg[2 * pp + 1], dot_p));
+        }
+        red[(warp * 2 + 0) * TT + lane] = den_p;
+        red[(warp * 2 + 1) * TT + lane] = dot_p;
+        __syncthreads();
+        float den = 1e-6f, dot = 0.f;
+        {
+            float dsum = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                dsum += red[(w * 2 + 0) * TT + lane];
+                dot += red[(w * 2 + 1) * TT + lane];
+            }
+            den += dsum;
+        }
+        const float dden = live ? -dot / (den * den) : 0.f;
+        if (warp == 0) dd[lane] = dden;
+        // psi / den for dS, du = (R^T (G / den) + dden z) [u > 0] for dq and dA, phi for dz
+#pragma unroll
+        for (int pp = 0; pp < FC / 2; ++pp) {
+            const int c = c0 + 2 * pp;
+            const float g0 = gg[2 * pp] / den, g1 = gg[2 * pp + 1] / den;
+            const float dph0 = cf[pp] * g0 + sf[pp] * g1 + dden * zs[c];
+            const float dph1 = -sf[pp] * g0 + cf[pp] * g1 + dden * zs[c + 1];
+            ws[lane * R + c] = live ? psi[2 * pp] / den : 0.f;
+            ws[lane * R + c + 1] = live ? psi[2 * pp + 1] / den : 0.f;
+            dus[lane * (R + 1) + c] = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
+            dus[lane * (R + 1) + c + 1] = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
+            phs[lane * R + c] = phi[2 * pp];
+            phs[lane * R + c + 1] = phi[2 * pp + 1];
+        }
+        __syncthreads();
+        // partial sums: dS[c][e] += sum_t w[t][c] dO[t][e]; dA[d][c] += sum_t q[t][d] du[t][c]; dz
+#pragma unroll 4
+        for (int tt = 0; tt < TT; ++tt) {
+            const float go = gs[tt * (D + 1) + e_own], xo = xs[tt * (D + 1) + e_own];
+#pragma unroll
+            for (int i = 0; i < NA; ++i) {
+                acc_s[i] = fmaf(ws[tt * R + cg + G * i], go, acc_s[i]);
+                acc_a[i] = fmaf(xo, dus[tt * (R + 1) + cg + G * i], acc_a[i]);
+            }
+        }
+        if (tid < R)
+            for (int tt = 0; tt < TT; ++tt) acc_z = fmaf(dd[tt], phs[tt * R + tid], acc_z);
+        // dq += du A^T for token `lane`, dims [d0, d0 + DC)
+        if (live) {
+            float o[DC];
+#pragma unroll
+            for (int i = 0; i < DC; ++i) o[i] = 0.f;
+            const float* dur = dus + lane * (R + 1);
+#pragma unroll 4
+            for (int c = 0; c < R; ++c) {
+                float av[DC];
+                ld_bcast(av, At + c * D + d0);
+                const float du = dur[c];
+#pragma unroll
+                for (int i = 0; i < DC; ++i) o[i] = fmaf(du, av[i], o[i]);
+            }
+            float* dst = dq + g.so.row(b, n, h) + d0;
+#pragma unroll
+            for (int i = 0; i < DC; i += 4) {
+                float4 v = *reinterpret_cast<float4*>(dst + i);
+                v.x += o[i]; v.y += o[i + 1]; v.z += o[i + 2]; v.w += o[i + 3];
+                *reinterpret_cast<float4*>(dst + i) = v;
+            }
+        }
+    }
+    const size_t slot = static_cast<size_t>(bh) * nsplit + split;
+#pragma unroll
+    for (int i = 0; i < NA; ++i) {
+        ds_part[slot * R * D + (cg + G * i) * D + e_own] = acc_s[i];
+        da_part[slot * D * R + e_own * R + cg + G * i] = acc_a[i];
+    }
+    if (tid < R) dz_part[slot * R + tid] = acc_z;
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16* __restrict__ k,
+                                                             const __nv_bfloat16* __restrict__ v,
+                                                             const __nv_bfloat16* __restrict__ A,
+                                                             const float* __restrict__ dS, const float* __restrict__ dz,
+                                                             const double2* __restrict__ tab,
+                                                             const int2* __restrict__ pairs, Geom g, int nsplit,
+                                                             float* __restrict__ dk, float* __restrict__ dv,
+                                                             float* __restrict__ da_part) {
+    constexpr int TT = 32, FC = R / 8, DC = D / 8;
+    static_assert(R <= 64 && FC % 2 == 0, "rank 16..64");
+    extern __shared__ __align__(16) float smf[];
+    float* Au = smf;                   // [D][R]   A
+    float* At = Au + D * R;            // [R][D]   A^T
+    float* dSt = At + R * D;           // [D][R]   dS^T
+    float* dSs = dSt + D * R;          // [R][D]   dS
+    float* zs = dSs + R * D;           // [R]      dz
+    float* xs = zs + R;                // [TT][D+1] k
+    float* vs = xs + TT * (D + 1);     // [TT][D+1] v
+    float* psis = vs + TT * (D + 1);   // [TT][R+1] psi
+    float* dus = psis + TT * (R + 1);  // [TT][R+1] du
+    constexpr int G = 256 / D;
+    constexpr int NA = R / G;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int split = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int ntiles = (g.L + TT - 1) / TT;
+    const int per = (ntiles + nsplit - 1) / nsplit;
+    const int t0 = split * per, t1 = min(ntiles, t0 + per);
+    for (int e = tid; e < D * R; e += 256) {
+        const float a = __bfloat162float(A[e]);
+        Au[e] = a;
+        At[(e % R) * D + e / R] = a;
+    }
+    for (int e = tid; e < R * D; e += 256) {
+        const float x = dS[static_cast<size_t>(bh) * R * D + e];
+        dSs[e] = x;
+        dSt[(e % D) * R + e / D] = x;
+    }
+    if (tid < R) zs[tid] = dz[static_cast<size_t>(bh) * R + tid];
+    const int e_own = tid % D, cg = tid / D;
+    float acc_a[NA];
+#pragma unroll
+    for (int i = 0; i < NA; ++i) acc_a[i] = 0.f;
+    const int c0 = warp * FC, d0 = warp * DC;
+    for (int tile = t0; tile < t1; ++tile) {
+        const int n0 = tile * TT;
+        __syncthreads();
+        for (int e = tid; e < TT * (D / 2); e += 256) {
+            const int tt = e / (D / 2), dp = e % (D / 2);
+            const int n = n0 + tt;
+            float2 xf = make_float2(0.f, 0.f), vf = make_float2(0.f, 0.f);
+            if (n < g.L) {
+                xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + g.sk.row(b, n, h) + 2 * dp));
+                vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + g.sv.row(b, n, h) + 2 * dp));
+            }
+            xs[tt * (D + 1) + 2 * dp] = xf.x; xs[tt * (D + 1) + 2 * dp + 1] = xf.y;
+            vs[tt * (D + 1) + 2 * dp] = vf.x; vs[tt * (D + 1) + 2 * dp + 1] = vf.y;
+        }
+        __syncthreads();
+        // u = k A and dpsi = dS v for token `lane`, features [c0, c0 + FC)
+        float u[FC], dp[FC];
+#pragma unroll
+        for (int f = 0; f < FC; ++f) u[f] = dp[f] = 0.f;
+        const float* xr = xs + lane * (D + 1);
+        const float* vr = vs + lane * (D + 1);
+#pragma unroll 4
+        for (int d = 0; d < D; ++d) {
+            float av[FC], sv[FC];
+            ld_bcast(av, Au + d * R + c0);
+            ld_bcast(sv, dSt + d * R + c0);
+            const float x = xr[d], vo = vr[d];
+#pragma unroll
+            for (int f = 0; f < FC; ++f) {
+                u[f] = fmaf(x, av[f], u[f]);
+                dp[f] = fmaf(sv[f], vo, dp[f]);
+            }
+        }
+        const int n = n0 + lane;
+        const bool live = n < g.L;
+        const int nt = live ? n : 0;
+        // psi = R phi; du = (R^T dpsi + dz) [u > 0]
+#pragma unroll
+        for (int pp = 0; pp < FC / 2; ++pp) {
+            const int c = c0 + 2 * pp;
+            const int2 pi = pairs[c / 2];
+            const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
+            const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+            const float x0 = fmaxf(u[2 * pp], 0.f), x1 = fmaxf(u[2 * pp + 1], 0.f);
+            psis[lane * (R + 1) + c] = x0 * cf - x1 * sf;
+            psis[lane * (R + 1) + c + 1] = x0 * sf + x1 * cf;
+            const float d0_ = dp[2 * pp], d1_ = dp[2 * pp + 1];
+            const float dph0 = cf * d0_ + sf * d1_ + zs[c];
+            const float dph1 = -sf * d0_ + cf * d1_ + zs[c + 1];
+            dus[lane * (R + 1) + c] = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
+            dus[lane * (R + 1) + c + 1] = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int tt = 0; tt < TT; ++tt) {
+            const float xo = xs[tt * (D + 1) + e_own];
+#pragma unroll
+            for (int i = 0; i < NA; ++i) acc_a[i] = fmaf(xo, dus[tt * (R + 1) + cg + G * i], acc_a[i]);
+        }
+        // dv += dS^T psi and dk += du A^T for token `lane`, dims [d0, d0 + DC)
+        if (live) {
+            float ov[DC], ok[DC];
+#pragma unroll
+            for (int i = 0; i < DC; ++i) ov[i] = ok[i] = 0.f;
+            const float* pr = psis + lane * (R + 1);
+            const float* dur = dus + lane * (R + 1);
+#pragma unroll 2
+            for (int c = 0; c < R; ++c) {
+                float sv[DC], av[DC];
+                ld_bcast(sv, dSs + c * D + d0);
+                ld_bcast(av, At + c * D + d0);
+                const float ps = pr[c], du = dur[c];
+#pragma unroll
+                for (int i = 0; i < DC; ++i) {
+                    ov[i] = fmaf(ps, sv[i], ov[i]);
+                    ok[i] = fmaf(du, av[i], ok[i]);
+                }
+            }
+            const long long r = g.so.row(b, n, h) + d0;
+#pragma unroll
+            for (int i = 0; i < DC; i += 4) {
+                float4 x = *reinterpret_cast<float4*>(dv + r + i);
+                x.x += ov[i]; x.y += ov[i + 1]; x.z += ov[i + 2]; x.w += ov[i + 3];
+                *reinterpret_cast<float4*>(dv + r + i) = x;
+                float4 y = *reinterpret_cast<float4*>(dk + r + i);
+                y.x += ok[i]; y.y += ok[i + 1]; y.z += ok[i + 2]; y.w += ok[i + 3];
+                *reinterpret_cast<float4*>(dk + r + i) = y;
+            }
+        }
+    }
+    const size_t slot = static_cast<size_t>(bh) * nsplit + split;
+#pragma unroll
+    for (int i = 0; i < NA; ++i) da_part[slot * D * R + e_own * R + cg + G * i] = acc_a[i];
+}
+
 // dA = sum over both passes, all heads and all splits of the partials, in a fixed order.
 __global__ void bwd_da_reduce_kernel(const float* __restrict__ da_part, int nslots, int DR, float* __restrict__ dA) {
     const int o = blockIdx.x * blockDim.x + threadIdx.x;
@@ -911,6 +1238,13 @@ size_t lr_bwd_smem(int D, int R, bool qpass) {
     const int mats = D * (R + 1) + R * (D + 1);  // padded A and S (or dS)
     if (qpass) return sizeof(float) * (mats + R + 2 * TT * (D + 1) + 3 * TT * (R + 1) + 2 * TT * R + 2 * TT);
     return sizeof(float) * (mats + R + 2 * TT * (D + 1) + 3 * TT * (R + 1));
+}
+
+size_t lr_bwd_tiled_smem(int D, int R, bool qpass) {
+    const int TT = 32;
+    if (qpass)  // A, A^T, S^T; z; q, dO tiles; psi/den, du, phi; dot partials, dden
+        return sizeof(float) * (3 * D * R + R + 2 * TT * (D + 1) + TT * R + TT * (R + 1) + TT * R + 16 * TT + TT);
+    return sizeof(float) * (4 * D * R + R + 2 * TT * (D + 1) + 2 * TT * (R + 1));  // A, A^T, dS^T, dS; dz; k, v; psi, du
 }
 
 int lr_bwd_nsplit(const Geom& g) {
@@ -939,19 +1273,23 @@ cudaError_t launch_bwd_sparse_t(const BwdMaps& m, const BwdArgs& a, const Geom& 
 template <int D, int R>
 cudaError_t launch_lr_bwd_t(const LrBwdArgs& l, const Geom& g, cudaStream_t st) {
     const int ns = l.nsplit;
-    const size_t smq = lr_bwd_smem(D, R, true), smk = lr_bwd_smem(D, R, false);
-    cudaError_t e = cudaFuncSetAttribute(bwd_lr_q_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq);
+    constexpr bool kTiled = R <= 64;  // the register-tiled passes (32-token tiles)
+    const size_t smq = kTiled ? lr_bwd_tiled_smem(D, R, true) : lr_bwd_smem(D, R, true);
+    const size_t smk = kTiled ? lr_bwd_tiled_smem(D, R, false) : lr_bwd_smem(D, R, false);
+    auto qk = kTiled ? bwd_lr_q_tiled_kernel<D, (R <= 64 ? R : 64)> : bwd_lr_q_kernel<D, R>;
+    auto kk = kTiled ? bwd_lr_k_tiled_kernel<D, (R <= 64 ? R : 64)> : bwd_lr_k_kernel<D, R>;
+    cudaError_t e = cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_lr_k_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk);
+    e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk);
     if (e != cudaSuccess) return e;
-    bwd_lr_q_kernel<D, R><<<dim3(ns, g.BH()), 256, smq, st>>>(l.q, l.dout, l.A, l.S, l.z, l.tab, l.pairs, g, ns, l.dq,
-                                                              l.ds_part, l.dz_part, l.da_part);
+    qk<<<dim3(ns, g.BH()), 256, smq, st>>>(l.q, l.dout, l.A, l.S, l.z, l.tab, l.pairs, g, ns, l.dq, l.ds_part,
+                                           l.dz_part, l.da_part);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_lowrank_reduce(l.ds_part, l.dz_part, g, ns, l.dS, l.dz, nullptr, nullptr, nullptr, st)) !=
         cudaSuccess)
         return e;
-    bwd_lr_k_kernel<D, R><<<dim3(ns, g.BH()), 256, smk, st>>>(l.k, l.v, l.A, l.dS, l.dz, l.tab, l.pairs, g, ns, l.dk,
-                                                              l.dv, l.da_part + static_cast<size_t>(g.BH()) * ns * D * R);
+    kk<<<dim3(ns, g.BH()), 256, smk, st>>>(l.k, l.v, l.A, l.dS, l.dz, l.tab, l.pairs, g, ns, l.dk, l.dv,
+                                           l.da_part + static_cast<size_t>(g.BH()) * ns * D * R);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int DR = D * R;
     bwd_da_reduce_kernel<<<(DR + 255) / 256, 256, 0, st>>>(l.da_part, 2 * g.BH() * ns, DR, l.dA);
