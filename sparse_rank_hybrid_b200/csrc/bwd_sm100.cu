@@ -36,8 +36,7 @@ namespace slra {
 namespace {
 
 constexpr int kBwdMathThreads = 256;  // 8 warps: two per TMEM lane group, each half of the key columns
-constexpr int kBwdThreads = 288;      // + one issuing warp (TMA and tcgen05.mma from its lane 0)
-constexpr int kBwdIssueWarp = 8;
+constexpr int kBwdIssueWarp = 8;      // + the tcgen05.mma issuing warp (lane 0) and a TMA producer warp
 
 
 __device__ __forceinline__ uint32_t pack_half2_lohi(float lo, float hi) {
@@ -90,23 +89,32 @@ __device__ __forceinline__ void store_row_unrotated(float* dst_row, const float*
 }
 
 // ------------------------------------------------------------------------------------------ dQ
+// Warps 0-7 math (rows = queries), warp 8 issues the products, warp 9 loads the tiles.
+// TMEM (512 columns): S | dP buffer 0 | dP buffer 1 | dQ^.  Each math thread writes its packed dS_j over
+// its own half of dP_j's columns (already in its registers), so the S columns are free as soon as the
+// math warps have loaded S_j and dP_j: S_{j+1} and dP_{j+1} (into the other dP buffer) are computed
+// while the math warps work on block j, and dQ^ += dS_j k^_j follows when they are done.  k^ tiles stay
+// until their dQ product (three slots), v tiles until their dP product (two slots).
 template <int D>
 struct DqLayout {
     static constexpr int kTile = 128 * D * 2;  // fp16 [128 rows][D] in 64-column slabs
     static constexpr int kOffQ = 0;
     static constexpr int kOffDo = kTile;
-    static constexpr int kOffK = 2 * kTile;  // slots s at kOffK + s * kTile
-    static constexpr int kOffV = 4 * kTile;
-    static constexpr int kOffBar = 6 * kTile;
-    static constexpr int kOffMisc = kOffBar + 128;
+    static constexpr int kOffK = 2 * kTile;  // slots s < 3 at kOffK + s * kTile
+    static constexpr int kOffV = 5 * kTile;  // slots s < 2 at kOffV + s * kTile
+    static constexpr int kOffBar = 7 * kTile;
+    static constexpr int kOffMisc = kOffBar + 256;
     static constexpr int kBytes = kOffMisc + 64;
 };
 
-enum : int { kDqBarQdo = 0, kDqBarKvFull = 1, kDqBarKvEmpty = 3, kDqBarSp = 5, kDqBarDs = 6, kDqBarFinal = 7,
-             kDqBarDrain = 8, kDqNumBars = 9 };
+enum : int { kDqBarQdo = 0, kDqBarKFull = 1, kDqBarKEmpty = 4, kDqBarVFull = 7, kDqBarVEmpty = 9,
+             kDqBarSp = 11, kDqBarLd = 12, kDqBarDs = 13 /* +2 */, kDqBarFinal = 15, kDqBarDrain = 16,
+             kDqNumBars = 17 };
+constexpr int kBwdProdWarp = 9;
+constexpr int kBwdThreads2 = 320;
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads2, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, BwdArgs a,
                   Geom g) {
@@ -128,7 +136,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t tmo = a.timeout_ns;
 
     if (tid == 0) {
-        for (int i = 0; i < kDqNumBars; ++i) mbar_init(bars + i, i == kDqBarDs ? kBwdMathThreads : 1);
+        for (int i = 0; i < kDqNumBars; ++i)
+            mbar_init(bars + i, (i == kDqBarLd || i == kDqBarDs || i == kDqBarDs + 1) ? kBwdMathThreads : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -140,92 +149,109 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
+    const uint32_t tS = tmem, tQ = tmem + 384;
+    auto tP = [&](int j) { return tmem + 128 + (j & 1) * 128; };
     auto fail = [&]() {
         *abort_flag = 1;
         atomicOr(a.status, kDevTimeout);
     };
+    auto kslot = [&](int j) { return smem + Lay::kOffK + (j % 3) * Lay::kTile; };
+    auto vslot = [&](int j) { return smem + Lay::kOffV + (j & 1) * Lay::kTile; };
 
-    if (warp == kBwdIssueWarp) {
-        // ------------------------------------------------------------ TMA + tcgen05.mma issuer
+    if (warp == kBwdProdWarp) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0 && keep > 0) {
-            auto kslot = [&](int s) { return smem + Lay::kOffK + s * Lay::kTile; };
-            auto vslot = [&](int s) { return smem + Lay::kOffV + s * Lay::kTile; };
             auto load_rows = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int row, int rows) {
 #pragma unroll
                 for (int sl = 0; sl < D / 64; ++sl) tma_load_2d(dst + sl * (rows * 128), tm, bar, sl * 64, row);
             };
-            auto load_kv = [&](int j) {
-                const int s = j & 1;
-                mbar_expect_tx(bars + kDqBarKvFull + s, 2u * BLK * D * 2);
-                const int r = row0 + __ldg(my_idx + j) * BLK;
-                load_rows(kslot(s), &tm_k, bars + kDqBarKvFull + s, r, BLK);
-                load_rows(vslot(s), &tm_v, bars + kDqBarKvFull + s, r, BLK);
-            };
             mbar_expect_tx(bars + kDqBarQdo, 2u * 128 * D * 2);
             load_rows(smem + Lay::kOffQ, &tm_q, bars + kDqBarQdo, row0 + alpha * BLK, 128);
             load_rows(smem + Lay::kOffDo, &tm_do, bars + kDqBarQdo, row0 + alpha * BLK, 128);
-            int n_loaded = 0;
-            for (; n_loaded < 2 && n_loaded < keep; ++n_loaded) load_kv(n_loaded);
+            int nk = 0, nv = 0;
+            bool ok = true;
+            for (int j = 0; j < keep && ok; ++j) {
+                const int r = row0 + __ldg(my_idx + j) * BLK;
+                // k^_j into slot j % 3 once dQ_{j-3} has read it; v_j into slot j % 2 once dP_{j-2} has
+                if (j >= 3 && !mbar_wait(bars + kDqBarKEmpty + j % 3, ((j - 3) / 3) & 1, tmo, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                mbar_expect_tx(bars + kDqBarKFull + j % 3, static_cast<uint32_t>(BLK) * D * 2);
+                load_rows(kslot(j), &tm_k, bars + kDqBarKFull + j % 3, r, BLK);
+                ++nk;
+                if (j >= 2 && !mbar_wait(bars + kDqBarVEmpty + (j & 1), ((j - 2) >> 1) & 1, tmo, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                mbar_expect_tx(bars + kDqBarVFull + (j & 1), static_cast<uint32_t>(BLK) * D * 2);
+                load_rows(vslot(j), &tm_v, bars + kDqBarVFull + (j & 1), r, BLK);
+                ++nv;
+            }
+            if (!ok) {
+                fail();
+                volatile int no_abort = 0;  // let every issued copy land (bounded)
+                mbar_wait(bars + kDqBarQdo, 0, 10000000ull, &no_abort);
+                for (int t = nk - 3 < 0 ? 0 : nk - 3; t < nk; ++t)
+                    mbar_wait(bars + kDqBarKFull + t % 3, (t / 3) & 1, 10000000ull, &no_abort);
+                for (int t = nv - 2 < 0 ? 0 : nv - 2; t < nv; ++t)
+                    mbar_wait(bars + kDqBarVFull + (t & 1), (t >> 1) & 1, 10000000ull, &no_abort);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kBwdIssueWarp) {
+        // ------------------------------------------------------------ tcgen05.mma issuer
+        if (lane == 0 && keep > 0) {
             const uint32_t idesc_s = idesc_f16_f32(128, BLK, false, false);
             const uint32_t idesc_q = idesc_f16_f32(128, D, false, true);
             const uint32_t q_addr = smem_addr(smem + Lay::kOffQ), do_addr = smem_addr(smem + Lay::kOffDo);
-            // S_j = q^ k^T_j and dP_j = dO v^T_j, both K-major over the head dimension
-            auto issue_sp = [&](int j) {
-                const int s = j & 1;
-                const uint32_t k_addr = smem_addr(kslot(s)), v_addr = smem_addr(vslot(s));
+            // S_j = q^ k^T_j and dP_j = dO v^T_j (K-major over the head dimension)
+            auto issue_sp = [&](int j) -> bool {
+                if (!mbar_wait(bars + kDqBarKFull + j % 3, (j / 3) & 1, tmo, abort_flag) ||
+                    !mbar_wait(bars + kDqBarVFull + (j & 1), (j >> 1) & 1, tmo, abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t k_addr = smem_addr(kslot(j)), v_addr = smem_addr(vslot(j));
 #pragma unroll
                 for (int kk = 0; kk < kSteps; ++kk) {
                     const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
                     const uint32_t bo = (kk >> 2) * (BLK * 128) + (kk & 3) * 32;
                     umma_ss(tS, sdesc_sw128(q_addr + ao, 16, 1024), sdesc_sw128(k_addr + bo, 16, 1024), idesc_s,
                             kk > 0 ? 1u : 0u);
-                    umma_ss(tP, sdesc_sw128(do_addr + ao, 16, 1024), sdesc_sw128(v_addr + bo, 16, 1024), idesc_s,
+                    umma_ss(tP(j), sdesc_sw128(do_addr + ao, 16, 1024), sdesc_sw128(v_addr + bo, 16, 1024), idesc_s,
                             kk > 0 ? 1u : 0u);
                 }
+                umma_commit(bars + kDqBarVEmpty + (j & 1));
                 umma_commit(bars + kDqBarSp);
+                return true;
             };
-            bool ok = mbar_wait(bars + kDqBarQdo, 0, tmo, abort_flag) && mbar_wait(bars + kDqBarKvFull, 0, tmo, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                issue_sp(0);
-            }
+            bool ok = mbar_wait(bars + kDqBarQdo, 0, tmo, abort_flag) && issue_sp(0);
             for (int j = 0; j < keep && ok; ++j) {
-                const int s = j & 1;
-                // dQ^ += dS_j k^_j: A = dS_j (fp16, packed over S_j's columns), B = k^_j MN-major
-                if (!mbar_wait(bars + kDqBarDs, j & 1, tmo, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t k_addr = smem_addr(kslot(s));
-#pragma unroll
-                for (int kk = 0; kk < kKeySteps; ++kk)
-                    umma_ts(tQ, tS + packed_col<HW>(kk), sdesc_sw128(k_addr + kk * 2048, BLK * 128, 1024), idesc_q,
-                            (j > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(bars + kDqBarKvEmpty + s);
-                if (j + 1 < keep) {  // S_{j+1} overwrites dS_j: issued after the product that reads it
-                    if (!mbar_wait(bars + kDqBarKvFull + ((j + 1) & 1), ((j + 1) >> 1) & 1, tmo, abort_flag)) {
+                // S_{j+1} and dP_{j+1} once the math warps hold S_j and dP_j in registers
+                if (j + 1 < keep) {
+                    if (!mbar_wait(bars + kDqBarLd, j & 1, tmo, abort_flag) || !issue_sp(j + 1)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    issue_sp(j + 1);
                 }
-                if (j + 2 < keep) {  // slot s is free once dQ_j (and so dP_j) has read it
-                    if (!mbar_wait(bars + kDqBarKvEmpty + s, (j >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
-                    load_kv(j + 2);
-                    ++n_loaded;
+                // dQ^ += dS_j k^_j: A = dS_j packed over dP_j's columns, B = k^_j MN-major
+                if (!mbar_wait(bars + kDqBarDs + (j & 1), (j >> 1) & 1, tmo, abort_flag)) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                const uint32_t k_addr = smem_addr(kslot(j));
+#pragma unroll
+                for (int kk = 0; kk < kKeySteps; ++kk)
+                    umma_ts(tQ, tP(j) + packed_col<HW>(kk), sdesc_sw128(k_addr + kk * 2048, BLK * 128, 1024),
+                            idesc_q, (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(bars + kDqBarKEmpty + j % 3);
             }
             if (ok) umma_commit(bars + kDqBarFinal);
             else fail();
-            // drain: every product issued here and every copy have landed before the CTA leaves
-            umma_commit(bars + kDqBarDrain);
+            umma_commit(bars + kDqBarDrain);  // drain: every product issued here lands before the CTA leaves
             volatile int no_abort = 0;
             mbar_wait(bars + kDqBarDrain, 0, 10000000ull, &no_abort);
-            if (!ok) {
-                mbar_wait(bars + kDqBarQdo, 0, 10000000ull, &no_abort);
-                for (int t = n_loaded - 2 < 0 ? 0 : n_loaded - 2; t < n_loaded; ++t)
-                    mbar_wait(bars + kDqBarKvFull + (t & 1), (t >> 1) & 1, 10000000ull, &no_abort);
-            }
         }
         __syncwarp();
     } else {
@@ -253,7 +279,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int c = 0; c < NC; ++c) {
                 tmem_ld32(tS + lane_base + key0 + c * 32, sr[c]);
-                tmem_ld32(tP + lane_base + key0 + c * 32, pr[c]);
+                tmem_ld32(tP(j) + lane_base + key0 + c * 32, pr[c]);
             }
             tmem_ld_wait(sr[0]);
 #pragma unroll
@@ -261,6 +287,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 reg_fence(sr[c]);
                 reg_fence(pr[c]);
             }
+            tc_fence_before();
+            mbar_arrive(bars + kDqBarLd);  // S_j and dP_j are in registers: S may be overwritten
             const bool masked = (j == keep - 1) && last_valid < BLK;
 #pragma unroll
             for (int c16 = 0; c16 < HW / 32; ++c16) {
@@ -271,19 +299,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
                         const int e = c16 * 32 + 2 * u + e2;  // key within this half
-                        const float s = __uint_as_float(sr[e >> 5][e & 31]);
+                        const float sv = __uint_as_float(sr[e >> 5][e & 31]);
                         const float dp = __uint_as_float(pr[e >> 5][e & 31]);
-                        float p = ex2_approx(fmaf(s, c2, -lse_i));
+                        float p = ex2_approx(fmaf(sv, c2, -lse_i));
                         if (masked && key0 + e >= last_valid) p = 0.f;
                         d2[e2] = p * (dp - delta_i);
                     }
                     pk[u] = pack_half2_lohi(d2[0], d2[1]);
                 }
-                tmem_st16(tS + lane_base + key0 + c16 * 16, pk);  // packed over this half's own columns
+                tmem_st16(tP(j) + lane_base + key0 + c16 * 16, pk);  // packed over this half's dP columns
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(bars + kDqBarDs);
+            mbar_arrive(bars + kDqBarDs + (j & 1));
         }
         // ---- epilogue: dq = R(p)^T dQ^ / sqrt(D), token-major fp32
         if (keep > 0) {
@@ -314,6 +342,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------- dK, dV
+// Warps 0-7 math (rows = keys), warp 8 issues the products, warp 9 loads the query-side tiles.
+// TMEM: S^T | dP^T | dV | dK^.  Each math thread writes its packed P^T and dS^T over its own half of
+// dP^T's columns (P^T in the first quarter of the block's columns, dS^T in the second), so the S^T
+// columns are free once S^T_t and dP^T_t are in registers and S^T_{t+1} is computed during the math of
+// block t; dP^T_{t+1} follows the dV and dK products that read block t's packed operands.
 template <int D, int BLK>
 struct DkvLayout {
     static constexpr int kTile = 128 * D * 2;   // key-side tiles: 128 rows (the MMA's M)
@@ -324,15 +357,15 @@ struct DkvLayout {
     static constexpr int kOffDo = kOffQ + 2 * kQTile;     // slots s at kOffDo + s * kQTile
     static constexpr int kOffLse = kOffDo + 2 * kQTile;   // slots s: [BLK] fp32 lse then [BLK] fp32 delta
     static constexpr int kOffBar = kOffLse + 2 * 2 * BLK * 4;
-    static constexpr int kOffMisc = kOffBar + 128;
+    static constexpr int kOffMisc = kOffBar + 256;
     static constexpr int kBytes = kOffMisc + 64;
 };
 
-enum : int { kKvBarKv = 0, kKvBarQFull = 1, kKvBarQEmpty = 3, kKvBarSp = 5, kKvBarP = 6, kKvBarFinal = 7,
-             kKvBarDrain = 8, kKvNumBars = 9 };
+enum : int { kKvBarKv = 0, kKvBarQFull = 1, kKvBarQEmpty = 3, kKvBarS = 5, kKvBarP = 6, kKvBarLd = 7,
+             kKvBarDs = 8 /* +2 */, kKvBarFinal = 10, kKvBarDrain = 11, kKvNumBars = 12 };
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads2, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do, BwdArgs a,
                     Geom g) {
@@ -354,7 +387,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t tmo = a.timeout_ns;
 
     if (tid == 0) {
-        for (int i = 0; i < kKvNumBars; ++i) mbar_init(bars + i, i == kKvBarP ? kBwdMathThreads : 1);
+        for (int i = 0; i < kKvNumBars; ++i)
+            mbar_init(bars + i, (i == kKvBarLd || i == kKvBarDs || i == kKvBarDs + 1) ? kBwdMathThreads : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -375,15 +409,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto doslot = [&](int s) { return smem + Lay::kOffDo + s * Lay::kQTile; };
     auto lseslot = [&](int s) { return reinterpret_cast<float*>(smem + Lay::kOffLse + s * 2 * BLK * 4); };
 
-    if (warp == kBwdIssueWarp) {
-        // ------------------------------------------------------------ TMA + tcgen05.mma issuer
+    if (warp == kBwdProdWarp) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0 && cnt > 0) {
             auto load_rows = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int row, int rows) {
 #pragma unroll
                 for (int sl = 0; sl < D / 64; ++sl) tma_load_2d(dst + sl * (rows * 128), tm, bar, sl * 64, row);
             };
-            auto load_q = [&](int t) {
+            mbar_expect_tx(bars + kKvBarKv, 2u * 128 * D * 2);
+            load_rows(smem + Lay::kOffK, &tm_k, bars + kKvBarKv, row0 + beta * BLK, 128);
+            load_rows(smem + Lay::kOffV, &tm_v, bars + kKvBarKv, row0 + beta * BLK, 128);
+            int nq = 0;
+            bool ok = true;
+            for (int t = 0; t < cnt; ++t) {
                 const int s = t & 1;
+                // slot s once the dV and dK products of block t-2 (its last readers) have completed
+                if (t >= 2 && !mbar_wait(bars + kKvBarQEmpty + s, ((t - 2) >> 1) & 1, tmo, abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 uint64_t* bar = bars + kKvBarQFull + s;
                 mbar_expect_tx(bar, 2u * BLK * D * 2 + 2u * BLK * 4);
                 const int qb = __ldg(my_inv + t);
@@ -391,72 +435,81 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 load_rows(doslot(s), &tm_do, bar, row0 + qb * BLK, BLK);
                 bulk_load(lseslot(s), a.lse + static_cast<size_t>(row0) + qb * BLK, BLK * 4, bar);
                 bulk_load(lseslot(s) + BLK, a.delta + static_cast<size_t>(row0) + qb * BLK, BLK * 4, bar);
-            };
-            mbar_expect_tx(bars + kKvBarKv, 2u * 128 * D * 2);
-            load_rows(smem + Lay::kOffK, &tm_k, bars + kKvBarKv, row0 + beta * BLK, 128);
-            load_rows(smem + Lay::kOffV, &tm_v, bars + kKvBarKv, row0 + beta * BLK, 128);
-            int n_loaded = 0;
-            for (; n_loaded < 2 && n_loaded < cnt; ++n_loaded) load_q(n_loaded);
+                ++nq;
+            }
+            if (!ok) {
+                fail();
+                volatile int no_abort = 0;
+                mbar_wait(bars + kKvBarKv, 0, 10000000ull, &no_abort);
+                for (int t = nq - 2 < 0 ? 0 : nq - 2; t < nq; ++t)
+                    mbar_wait(bars + kKvBarQFull + (t & 1), (t >> 1) & 1, 10000000ull, &no_abort);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kBwdIssueWarp) {
+        // ------------------------------------------------------------ tcgen05.mma issuer
+        if (lane == 0 && cnt > 0) {
             const uint32_t idesc_s = idesc_f16_f32(128, BLK, false, false);
             const uint32_t idesc_o = idesc_f16_f32(128, D, false, true);
             const uint32_t k_addr = smem_addr(smem + Lay::kOffK), v_addr = smem_addr(smem + Lay::kOffV);
-            // S^T_t = k^ q^T_t and dP^T_t = v dO^T_t (K-major over the head dimension)
-            auto issue_sp = [&](int t) {
-                const int s = t & 1;
-                const uint32_t q_addr = smem_addr(qslot(s)), do_addr = smem_addr(doslot(s));
+            auto issue_s = [&](int t) {  // S^T_t = k^ q^T_t
+                const uint32_t q_addr = smem_addr(qslot(t & 1));
 #pragma unroll
-                for (int kk = 0; kk < kSteps; ++kk) {
-                    const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-                    const uint32_t bo = (kk >> 2) * (BLK * 128) + (kk & 3) * 32;
-                    umma_ss(tS, sdesc_sw128(k_addr + ao, 16, 1024), sdesc_sw128(q_addr + bo, 16, 1024), idesc_s,
+                for (int kk = 0; kk < kSteps; ++kk)
+                    umma_ss(tS, sdesc_sw128(k_addr + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
+                            sdesc_sw128(q_addr + (kk >> 2) * (BLK * 128) + (kk & 3) * 32, 16, 1024), idesc_s,
                             kk > 0 ? 1u : 0u);
-                    umma_ss(tP, sdesc_sw128(v_addr + ao, 16, 1024), sdesc_sw128(do_addr + bo, 16, 1024), idesc_s,
+                umma_commit(bars + kKvBarS);
+            };
+            auto issue_p = [&](int t) {  // dP^T_t = v dO^T_t
+                const uint32_t do_addr = smem_addr(doslot(t & 1));
+#pragma unroll
+                for (int kk = 0; kk < kSteps; ++kk)
+                    umma_ss(tP, sdesc_sw128(v_addr + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
+                            sdesc_sw128(do_addr + (kk >> 2) * (BLK * 128) + (kk & 3) * 32, 16, 1024), idesc_s,
                             kk > 0 ? 1u : 0u);
-                }
-                umma_commit(bars + kKvBarSp);
+                umma_commit(bars + kKvBarP);
             };
             bool ok = mbar_wait(bars + kKvBarKv, 0, tmo, abort_flag) && mbar_wait(bars + kKvBarQFull, 0, tmo, abort_flag);
             if (ok) {
                 tc_fence_after();
-                issue_sp(0);
+                issue_s(0);
+                issue_p(0);
             }
             for (int t = 0; t < cnt && ok; ++t) {
                 const int s = t & 1;
-                if (!mbar_wait(bars + kKvBarP, t & 1, tmo, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                // dV += P^T dO_t and dK^ += dS^T q^_t (A from TMEM, B MN-major over the query rows)
-                const uint32_t q_addr = smem_addr(qslot(s)), do_addr = smem_addr(doslot(s));
-#pragma unroll
-                for (int kk = 0; kk < kQSteps; ++kk) {
-                    const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts(tV, tS + packed_col<HW>(kk), sdesc_sw128(do_addr + kk * 2048, BLK * 128, 1024), idesc_o, acc);
-                    umma_ts(tK, tP + packed_col<HW>(kk), sdesc_sw128(q_addr + kk * 2048, BLK * 128, 1024), idesc_o, acc);
-                }
-                umma_commit(bars + kKvBarQEmpty + s);
+                // S^T_{t+1} once the math warps hold S^T_t and dP^T_t in registers
                 if (t + 1 < cnt) {
-                    if (!mbar_wait(bars + kKvBarQFull + ((t + 1) & 1), ((t + 1) >> 1) & 1, tmo, abort_flag)) {
+                    if (!mbar_wait(bars + kKvBarLd, t & 1, tmo, abort_flag) ||
+                        !mbar_wait(bars + kKvBarQFull + ((t + 1) & 1), ((t + 1) >> 1) & 1, tmo, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    issue_sp(t + 1);
+                    issue_s(t + 1);
                 }
-                if (t + 2 < cnt) {
-                    if (!mbar_wait(bars + kKvBarQEmpty + s, (t >> 1) & 1, tmo, abort_flag)) { ok = false; break; }
-                    load_q(t + 2);
-                    ++n_loaded;
+                if (!mbar_wait(bars + kKvBarDs + s, (t >> 1) & 1, tmo, abort_flag)) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                // dV += P^T dO_t and dK^ += dS^T q^_t (A packed over dP^T's columns, B MN-major)
+                const uint32_t q_addr = smem_addr(qslot(s)), do_addr = smem_addr(doslot(s));
+#pragma unroll
+                for (int kk = 0; kk < kQSteps; ++kk) {
+                    const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+                    const uint32_t col = packed_col<HW>(kk);
+                    umma_ts(tV, tP + col, sdesc_sw128(do_addr + kk * 2048, BLK * 128, 1024), idesc_o, acc);
+                    umma_ts(tK, tP + col + HW / 2, sdesc_sw128(q_addr + kk * 2048, BLK * 128, 1024), idesc_o, acc);
+                }
+                umma_commit(bars + kKvBarQEmpty + s);
+                if (t + 1 < cnt) issue_p(t + 1);  // after the products that read dP^T's columns
             }
             if (ok) umma_commit(bars + kKvBarFinal);
             else fail();
             umma_commit(bars + kKvBarDrain);
             volatile int no_abort = 0;
             mbar_wait(bars + kKvBarDrain, 0, 10000000ull, &no_abort);
-            if (!ok) {
-                mbar_wait(bars + kKvBarKv, 0, 10000000ull, &no_abort);
-                for (int t = n_loaded - 2 < 0 ? 0 : n_loaded - 2; t < n_loaded; ++t)
-                    mbar_wait(bars + kKvBarQFull + (t & 1), (t >> 1) & 1, 10000000ull, &no_abort);
-            }
         }
         __syncwarp();
     } else {
@@ -473,7 +526,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int s = t & 1;
             // the query block's lse and delta arrived with its tiles (same barrier phase)
             ok = __all_sync(0xffffffffu, mbar_wait(bars + kKvBarQFull + s, (t >> 1) & 1, tmo, abort_flag) &&
-                                             mbar_wait(bars + kKvBarSp, t & 1, tmo, abort_flag));
+                                             mbar_wait(bars + kKvBarS, t & 1, tmo, abort_flag) &&
+                                             mbar_wait(bars + kKvBarP, t & 1, tmo, abort_flag));
             if (!ok) {
                 if (lane == 0) fail();
                 break;
@@ -493,6 +547,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 reg_fence(sr[c]);
                 reg_fence(pr[c]);
             }
+            tc_fence_before();
+            mbar_arrive(bars + kKvBarLd);  // S^T_t and dP^T_t are in registers: S^T may be overwritten
 #pragma unroll
             for (int c16 = 0; c16 < HW / 32; ++c16) {
                 uint32_t pk[16], dk16[16];
@@ -511,12 +567,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     pk[u] = pack_half2_lohi(pp[0], pp[1]);
                     dk16[u] = pack_half2_lohi(dd[0], dd[1]);
                 }
-                tmem_st16(tS + lane_base + q0 + c16 * 16, pk);
-                tmem_st16(tP + lane_base + q0 + c16 * 16, dk16);
+                tmem_st16(tP + lane_base + q0 + c16 * 16, pk);            // P^T: first quarter of the half
+                tmem_st16(tP + lane_base + q0 + HW / 2 + c16 * 16, dk16);  // dS^T: second quarter
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(bars + kKvBarP);
+            mbar_arrive(bars + kKvBarDs + s);
         }
         // ---- epilogue: dv = sum P^T dO, dk = R(p)^T dK^ / sqrt(D); key blocks nobody kept get zeros
         const bool done = cnt == 0 || (ok && __all_sync(0xffffffffu, mbar_wait(bars + kKvBarFinal, 0, tmo, abort_flag)));
@@ -1263,10 +1319,10 @@ cudaError_t launch_bwd_sparse_t(const BwdMaps& m, const BwdArgs& a, const Geom& 
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)skv);
     if (e != cudaSuccess) return e;
-    bwd_dq_kernel<D, BLK><<<dim3(g.nb, g.BH()), kBwdThreads, sq, st>>>(m.q128, m.do128, m.kb, m.vb, a, g);
+    bwd_dq_kernel<D, BLK><<<dim3(g.nb, g.BH()), kBwdThreads2, sq, st>>>(m.q128, m.do128, m.kb, m.vb, a, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (m.between) cudaEventRecord(m.between, st);
-    bwd_dkdv_kernel<D, BLK><<<dim3(g.nb, g.BH()), kBwdThreads, skv, st>>>(m.k128, m.v128, m.qb, m.dob, a, g);
+    bwd_dkdv_kernel<D, BLK><<<dim3(g.nb, g.BH()), kBwdThreads2, skv, st>>>(m.k128, m.v128, m.qb, m.dob, a, g);
     return cudaGetLastError();
 }
 
