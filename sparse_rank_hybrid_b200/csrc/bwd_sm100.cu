@@ -957,13 +957,26 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
 // the products over the features), so A, S and dS are read as warp-wide broadcast vectors and the
 // per-token operands as conflict-free gathers (rows padded to D+1 / R+1), and a token's rotation pairs
 // stay inside one thread.
+// N consecutive floats from shared memory: 16-byte loads when N is a multiple of 4 (src 16-B aligned),
+// else 8-byte loads (src 8-B aligned, N even).
 template <int N>
-__device__ __forceinline__ void ld_bcast(float (&dst)[N], const float* src) {  // 8-B aligned, N even
+__device__ __forceinline__ void ld_bcast(float (&dst)[N], const float* src) {
+    if constexpr (N % 4 == 0) {
 #pragma unroll
-    for (int i = 0; i < N; i += 2) {
-        const float2 v = *reinterpret_cast<const float2*>(src + i);
-        dst[i] = v.x;
-        dst[i + 1] = v.y;
+        for (int i = 0; i < N; i += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src + i);
+            dst[i] = v.x;
+            dst[i + 1] = v.y;
+            dst[i + 2] = v.z;
+            dst[i + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; i += 2) {
+            const float2 v = *reinterpret_cast<const float2*>(src + i);
+            dst[i] = v.x;
+            dst[i + 1] = v.y;
+        }
     }
 }
 
@@ -990,6 +1003,7 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
     float* phs = dus + TT * (R + 1);   // [TT][R]   phi
     float* red = phs + TT * R;         // [8][2][TT] per-warp partial dots
     float* dd = red + 8 * 2 * TT;      // [TT] dden
+    float* duc = dd + TT;              // [TT][R]   du, unpadded (vector reads in the partial sums)
     constexpr int G = 256 / D;
     constexpr int NA = R / G;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1005,6 +1019,7 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
     }
     for (int e = tid; e < R * D; e += 256) St[(e % D) * R + e / D] = S[static_cast<size_t>(bh) * R * D + e];
     if (tid < R) zs[tid] = z[static_cast<size_t>(bh) * R + tid];
+    // partial sums: thread (e_own, cg) owns features [cg * NA, cg * NA + NA) of column e_own
     const int e_own = tid % D, cg = tid / D;
     float acc_s[NA], acc_a[NA];
 #pragma unroll
@@ -1089,20 +1104,27 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
             const float dph1 = -sf[pp] * g0 + cf[pp] * g1 + dden * zs[c + 1];
             ws[lane * R + c] = live ? psi[2 * pp] / den : 0.f;
             ws[lane * R + c + 1] = live ? psi[2 * pp + 1] / den : 0.f;
-            dus[lane * (R + 1) + c] = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
-            dus[lane * (R + 1) + c + 1] = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
+            const float du0 = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
+            const float du1 = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
+            dus[lane * (R + 1) + c] = du0;
+            dus[lane * (R + 1) + c + 1] = du1;
+            duc[lane * R + c] = du0;
+            duc[lane * R + c + 1] = du1;
             phs[lane * R + c] = phi[2 * pp];
             phs[lane * R + c + 1] = phi[2 * pp + 1];
         }
         __syncthreads();
         // partial sums: dS[c][e] += sum_t w[t][c] dO[t][e]; dA[d][c] += sum_t q[t][d] du[t][c]; dz
-#pragma unroll 4
+#pragma unroll 2
         for (int tt = 0; tt < TT; ++tt) {
             const float go = gs[tt * (D + 1) + e_own], xo = xs[tt * (D + 1) + e_own];
+            float wv[NA], uv[NA];
+            ld_bcast(wv, ws + tt * R + cg * NA);
+            ld_bcast(uv, duc + tt * R + cg * NA);
 #pragma unroll
             for (int i = 0; i < NA; ++i) {
-                acc_s[i] = fmaf(ws[tt * R + cg + G * i], go, acc_s[i]);
-                acc_a[i] = fmaf(xo, dus[tt * (R + 1) + cg + G * i], acc_a[i]);
+                acc_s[i] = fmaf(wv[i], go, acc_s[i]);
+                acc_a[i] = fmaf(xo, uv[i], acc_a[i]);
             }
         }
         if (tid < R)
@@ -1133,8 +1155,8 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
     const size_t slot = static_cast<size_t>(bh) * nsplit + split;
 #pragma unroll
     for (int i = 0; i < NA; ++i) {
-        ds_part[slot * R * D + (cg + G * i) * D + e_own] = acc_s[i];
-        da_part[slot * D * R + e_own * R + cg + G * i] = acc_a[i];
+        ds_part[slot * R * D + (cg * NA + i) * D + e_own] = acc_s[i];
+        da_part[slot * D * R + e_own * R + cg * NA + i] = acc_a[i];
     }
     if (tid < R) dz_part[slot * R + tid] = acc_z;
 }
@@ -1160,6 +1182,7 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
     float* vs = xs + TT * (D + 1);     // [TT][D+1] v
     float* psis = vs + TT * (D + 1);   // [TT][R+1] psi
     float* dus = psis + TT * (R + 1);  // [TT][R+1] du
+    float* duc = dus + TT * (R + 1);   // [TT][R]   du, unpadded (vector reads in the partial sums)
     constexpr int G = 256 / D;
     constexpr int NA = R / G;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1233,15 +1256,21 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
             const float d0_ = dp[2 * pp], d1_ = dp[2 * pp + 1];
             const float dph0 = cf * d0_ + sf * d1_ + zs[c];
             const float dph1 = -sf * d0_ + cf * d1_ + zs[c + 1];
-            dus[lane * (R + 1) + c] = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
-            dus[lane * (R + 1) + c + 1] = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
+            const float du0 = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
+            const float du1 = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
+            dus[lane * (R + 1) + c] = du0;
+            dus[lane * (R + 1) + c + 1] = du1;
+            duc[lane * R + c] = du0;
+            duc[lane * R + c + 1] = du1;
         }
         __syncthreads();
-#pragma unroll 4
+#pragma unroll 2
         for (int tt = 0; tt < TT; ++tt) {
             const float xo = xs[tt * (D + 1) + e_own];
+            float uv[NA];
+            ld_bcast(uv, duc + tt * R + cg * NA);
 #pragma unroll
-            for (int i = 0; i < NA; ++i) acc_a[i] = fmaf(xo, dus[tt * (R + 1) + cg + G * i], acc_a[i]);
+            for (int i = 0; i < NA; ++i) acc_a[i] = fmaf(xo, uv[i], acc_a[i]);
         }
         // dv += dS^T psi and dk += du A^T for token `lane`, dims [d0, d0 + DC)
         if (live) {
@@ -1276,7 +1305,7 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
     }
     const size_t slot = static_cast<size_t>(bh) * nsplit + split;
 #pragma unroll
-    for (int i = 0; i < NA; ++i) da_part[slot * D * R + e_own * R + cg + G * i] = acc_a[i];
+    for (int i = 0; i < NA; ++i) da_part[slot * D * R + e_own * R + cg * NA + i] = acc_a[i];
 }
 
 // dA = sum over both passes, all heads and all splits of the partials, in a fixed order.
@@ -1298,9 +1327,10 @@ size_t lr_bwd_smem(int D, int R, bool qpass) {
 
 size_t lr_bwd_tiled_smem(int D, int R, bool qpass) {
     const int TT = 32;
-    if (qpass)  // A, A^T, S^T; z; q, dO tiles; psi/den, du, phi; dot partials, dden
-        return sizeof(float) * (3 * D * R + R + 2 * TT * (D + 1) + TT * R + TT * (R + 1) + TT * R + 16 * TT + TT);
-    return sizeof(float) * (4 * D * R + R + 2 * TT * (D + 1) + 2 * TT * (R + 1));  // A, A^T, dS^T, dS; dz; k, v; psi, du
+    if (qpass)  // A, A^T, S^T; z; q, dO tiles; psi/den, du, phi; dot partials, dden; du unpadded
+        return sizeof(float) * (3 * D * R + R + 2 * TT * (D + 1) + TT * R + TT * (R + 1) + TT * R + 16 * TT + TT + TT * R);
+    // A, A^T, dS^T, dS; dz; k, v; psi, du; du unpadded
+    return sizeof(float) * (4 * D * R + R + 2 * TT * (D + 1) + 2 * TT * (R + 1) + TT * R);
 }
 
 int lr_bwd_nsplit(const Geom& g) {
