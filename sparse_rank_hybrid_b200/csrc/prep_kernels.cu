@@ -279,7 +279,7 @@ __device__ __forceinline__ void dmma_8x8x4(double& d0, double& d1, double a, dou
 // block indices in ascending order (ties at the threshold resolved to the lowest indices) and the tie
 // flag.
 template <int D>
-__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ qbar,
+__global__ void __launch_bounds__(256, 2) select_kernel(const double* __restrict__ qbar,
                                                      const double* __restrict__ kbar, Geom g,
                                                      int32_t* __restrict__ idx, uint8_t* __restrict__ tie) {
     extern __shared__ __align__(16) unsigned char sm_raw[];
@@ -312,13 +312,19 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
         const int key = 8 * t + (lane >> 2);  // B fragment: key l/4 of the tile, the same dims as A
         const double2* kr =
             reinterpret_cast<const double2*>(kb + static_cast<size_t>(key < nb ? key : nb - 1) * D) + (lane & 3);
-        double d0 = 0.0, d1 = 0.0;
+        // four independent accumulator chains over the k-steps (a single chain of D/4 dependent
+        // products is latency-bound), summed at the end
+        double d[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
 #pragma unroll
         for (int m = 0; m < D / 8; ++m) {
             const double2 b2 = __ldg(kr + 4 * m);
-            dmma_8x8x4(d0, d1, af[2 * m], b2.x);
-            dmma_8x8x4(d0, d1, af[2 * m + 1], b2.y);
+            double (&da)[2] = d[(2 * m) & 3];
+            double (&db)[2] = d[(2 * m + 1) & 3];
+            dmma_8x8x4(da[0], da[1], af[2 * m], b2.x);
+            dmma_8x8x4(db[0], db[1], af[2 * m + 1], b2.y);
         }
+        const double d0 = (d[0][0] + d[1][0]) + (d[2][0] + d[3][0]);
+        const double d1 = (d[0][1] + d[1][1]) + (d[2][1] + d[3][1]);
         const int r = lane >> 2, c = 8 * t + 2 * (lane & 3);
         if (c < nb) scores[r * nb + c] = d0;
         if (c + 1 < nb) scores[r * nb + c + 1] = d1;
