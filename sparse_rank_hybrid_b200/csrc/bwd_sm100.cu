@@ -57,11 +57,15 @@ __device__ __forceinline__ uint32_t packed_col(int kk) {
 }  // namespace
 
 
-// Rotate the pairs of this thread's D/2 columns back by R(p)^T and store them (fp32) into a token-major
-// row; `vals` are the 32-bit TMEM words of columns [hf*D/2, hf*D/2 + D/2) of the row, already scaled.
+// Rotate the pairs of this thread's D/2 columns back by R(p)^T and add them (fp32) to a token-major row
+// (which holds the low-rank branch's part, or zeros); `vals` are the 32-bit TMEM words of columns
+// [hf*D/2, hf*D/2 + D/2) of the row, already scaled.
 template <int D>
 __device__ __forceinline__ void store_row_unrotated(float* dst_row, const float* vals, int hf, int n,
                                                     const BwdArgs& a, const Geom& g, bool rotate) {
+    float4 prev[D / 8];
+#pragma unroll
+    for (int t = 0; t < D / 8; ++t) prev[t] = *reinterpret_cast<const float4*>(dst_row + hf * (D / 2) + 4 * t);
     const int pt = n / (g.H * g.W), ph = (n / g.W) % g.H, pw = n % g.W;
 #pragma unroll
     for (int t = 0; t < D / 8; ++t) {  // 4 columns (2 pairs) per float4
@@ -84,6 +88,10 @@ __device__ __forceinline__ void store_row_unrotated(float* dst_row, const float*
                 ov[2 * u + 1] = y1;
             }
         }
+        o.x += prev[t].x;
+        o.y += prev[t].y;
+        o.z += prev[t].z;
+        o.w += prev[t].w;
         *reinterpret_cast<float4*>(dst_row + hf * (D / 2) + 4 * t) = o;
     }
 }
@@ -827,7 +835,7 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
             float s = 0.f;
 #pragma unroll 8
             for (int c = 0; c < R; ++c) s = fmaf(dus[tt * (R + 1) + c], As[d * (R + 1) + c], s);
-            dq[g.so.row(b, n, h) + d] += s;
+            dq[g.so.row(b, n, h) + d] = s;
         }
     }
     const size_t slot = static_cast<size_t>(bh) * nsplit + split;
@@ -943,8 +951,8 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
                 sk = fmaf(ps[tt * (R + 1) + c], As[d * (R + 1) + c], sk);
             }
             const long long r = g.so.row(b, n, h) + d;
-            dv[r] += sv;
-            dk[r] += sk;
+            dv[r] = sv;
+            dk[r] = sk;
         }
     }
     const size_t slot = static_cast<size_t>(bh) * nsplit + split;
@@ -1026,21 +1034,55 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
     for (int i = 0; i < NA; ++i) acc_s[i] = acc_a[i] = 0.f;
     float acc_z = 0.f;
     const int c0 = warp * FC, d0 = warp * DC;
+    // the next tile's q and dO are loaded into registers while this tile is computed
+    constexpr int NL = TT * (D / 2) / 256;
+    __nv_bfloat162 pq[NL];
+    float2 pg[NL];
+    auto fetch = [&](int tile) {
+#pragma unroll
+        for (int l = 0; l < NL; ++l) {
+            const int e = tid + 256 * l, tt = e / (D / 2), dp = e % (D / 2);
+            const int n = tile * TT + tt;
+            if (tile < t1 && n < g.L) {
+                pq[l] = *reinterpret_cast<const __nv_bfloat162*>(q + g.sq.row(b, n, h) + 2 * dp);
+                pg[l] = *reinterpret_cast<const float2*>(dout + g.so.row(b, n, h) + 2 * dp);
+            } else {
+                pq[l] = __floats2bfloat162_rn(0.f, 0.f);
+                pg[l] = make_float2(0.f, 0.f);
+            }
+        }
+    };
+    fetch(t0);
     for (int tile = t0; tile < t1; ++tile) {
         const int n0 = tile * TT;
         __syncthreads();
-        for (int e = tid; e < TT * (D / 2); e += 256) {
-            const int tt = e / (D / 2), dp = e % (D / 2);
-            const int n = n0 + tt;
-            float2 xf = make_float2(0.f, 0.f), gf = make_float2(0.f, 0.f);
-            if (n < g.L) {
-                xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + g.sq.row(b, n, h) + 2 * dp));
-                gf = *reinterpret_cast<const float2*>(dout + g.so.row(b, n, h) + 2 * dp);
-            }
+#pragma unroll
+        for (int l = 0; l < NL; ++l) {
+            const int e = tid + 256 * l, tt = e / (D / 2), dp = e % (D / 2);
+            const float2 xf = __bfloat1622float2(pq[l]);
             xs[tt * (D + 1) + 2 * dp] = xf.x; xs[tt * (D + 1) + 2 * dp + 1] = xf.y;
-            gs[tt * (D + 1) + 2 * dp] = gf.x; gs[tt * (D + 1) + 2 * dp + 1] = gf.y;
+            gs[tt * (D + 1) + 2 * dp] = pg[l].x; gs[tt * (D + 1) + 2 * dp + 1] = pg[l].y;
         }
         __syncthreads();
+        fetch(tile + 1);
+        const int n = n0 + lane;
+        const bool live = n < g.L;
+        const int nt = live ? n : 0;
+        // this token's (cos, sin) of the warp's pairs, loaded before the products that hide their latency
+        float cf[FC / 2], sf[FC / 2];
+        {
+            double2 cs[FC / 2];
+#pragma unroll
+            for (int pp = 0; pp < FC / 2; ++pp) {
+                const int2 pi = __ldg(pairs + c0 / 2 + pp);
+                cs[pp] = __ldg(tab + pi.y + token_axis_pos(nt, pi.x, g.H, g.W));
+            }
+#pragma unroll
+            for (int pp = 0; pp < FC / 2; ++pp) {
+                cf[pp] = static_cast<float>(cs[pp].x);
+                sf[pp] = static_cast<float>(cs[pp].y);
+            }
+        }
         // u = q A and G = S dO for token `lane`, features [c0, c0 + FC)
         float u[FC], gg[FC];
 #pragma unroll
@@ -1060,18 +1102,10 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
             }
         }
         // phi, psi, partial den = phi . z and psi . G over this warp's features
-        const int n = n0 + lane;
-        const bool live = n < g.L;
-        const int nt = live ? n : 0;
-        float phi[FC], psi[FC], cf[FC / 2], sf[FC / 2];
+        float phi[FC], psi[FC];
         float den_p = 0.f, dot_p = 0.f;
 #pragma unroll
         for (int pp = 0; pp < FC / 2; ++pp) {
-            const int p = c0 / 2 + pp;
-            const int2 pi = pairs[p];
-            const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
-            cf[pp] = static_cast<float>(cs.x);
-            sf[pp] = static_cast<float>(cs.y);
             const float x0 = fmaxf(u[2 * pp], 0.f), x1 = fmaxf(u[2 * pp + 1], 0.f);
             phi[2 * pp] = x0;
             phi[2 * pp + 1] = x1;
@@ -1143,13 +1177,10 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
 #pragma unroll
                 for (int i = 0; i < DC; ++i) o[i] = fmaf(du, av[i], o[i]);
             }
-            float* dst = dq + g.so.row(b, n, h) + d0;
+            float* dst = dq + g.so.row(b, n, h) + d0;  // the sparse branch's dQ kernel adds its part later
 #pragma unroll
-            for (int i = 0; i < DC; i += 4) {
-                float4 v = *reinterpret_cast<float4*>(dst + i);
-                v.x += o[i]; v.y += o[i + 1]; v.z += o[i + 2]; v.w += o[i + 3];
-                *reinterpret_cast<float4*>(dst + i) = v;
-            }
+            for (int i = 0; i < DC; i += 4)
+                *reinterpret_cast<float4*>(dst + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
         }
     }
     const size_t slot = static_cast<size_t>(bh) * nsplit + split;
@@ -1207,21 +1238,52 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
 #pragma unroll
     for (int i = 0; i < NA; ++i) acc_a[i] = 0.f;
     const int c0 = warp * FC, d0 = warp * DC;
+    // the next tile's k and v are loaded into registers while this tile is computed
+    constexpr int NL = TT * (D / 2) / 256;
+    __nv_bfloat162 pk[NL], pv[NL];
+    auto fetch = [&](int tile) {
+#pragma unroll
+        for (int l = 0; l < NL; ++l) {
+            const int e = tid + 256 * l, tt = e / (D / 2), dp = e % (D / 2);
+            const int n = tile * TT + tt;
+            if (tile < t1 && n < g.L) {
+                pk[l] = *reinterpret_cast<const __nv_bfloat162*>(k + g.sk.row(b, n, h) + 2 * dp);
+                pv[l] = *reinterpret_cast<const __nv_bfloat162*>(v + g.sv.row(b, n, h) + 2 * dp);
+            } else {
+                pk[l] = pv[l] = __floats2bfloat162_rn(0.f, 0.f);
+            }
+        }
+    };
+    fetch(t0);
     for (int tile = t0; tile < t1; ++tile) {
         const int n0 = tile * TT;
         __syncthreads();
-        for (int e = tid; e < TT * (D / 2); e += 256) {
-            const int tt = e / (D / 2), dp = e % (D / 2);
-            const int n = n0 + tt;
-            float2 xf = make_float2(0.f, 0.f), vf = make_float2(0.f, 0.f);
-            if (n < g.L) {
-                xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + g.sk.row(b, n, h) + 2 * dp));
-                vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + g.sv.row(b, n, h) + 2 * dp));
-            }
+#pragma unroll
+        for (int l = 0; l < NL; ++l) {
+            const int e = tid + 256 * l, tt = e / (D / 2), dp = e % (D / 2);
+            const float2 xf = __bfloat1622float2(pk[l]), vf = __bfloat1622float2(pv[l]);
             xs[tt * (D + 1) + 2 * dp] = xf.x; xs[tt * (D + 1) + 2 * dp + 1] = xf.y;
             vs[tt * (D + 1) + 2 * dp] = vf.x; vs[tt * (D + 1) + 2 * dp + 1] = vf.y;
         }
         __syncthreads();
+        fetch(tile + 1);
+        const int n = n0 + lane;
+        const bool live = n < g.L;
+        const int nt = live ? n : 0;
+        float cfs[FC / 2], sfs[FC / 2];  // this token's (cos, sin) of the warp's pairs, loaded early
+        {
+            double2 cs[FC / 2];
+#pragma unroll
+            for (int pp = 0; pp < FC / 2; ++pp) {
+                const int2 pi = __ldg(pairs + c0 / 2 + pp);
+                cs[pp] = __ldg(tab + pi.y + token_axis_pos(nt, pi.x, g.H, g.W));
+            }
+#pragma unroll
+            for (int pp = 0; pp < FC / 2; ++pp) {
+                cfs[pp] = static_cast<float>(cs[pp].x);
+                sfs[pp] = static_cast<float>(cs[pp].y);
+            }
+        }
         // u = k A and dpsi = dS v for token `lane`, features [c0, c0 + FC)
         float u[FC], dp[FC];
 #pragma unroll
@@ -1240,16 +1302,11 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
                 dp[f] = fmaf(sv[f], vo, dp[f]);
             }
         }
-        const int n = n0 + lane;
-        const bool live = n < g.L;
-        const int nt = live ? n : 0;
         // psi = R phi; du = (R^T dpsi + dz) [u > 0]
 #pragma unroll
         for (int pp = 0; pp < FC / 2; ++pp) {
             const int c = c0 + 2 * pp;
-            const int2 pi = pairs[c / 2];
-            const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
-            const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+            const float cf = cfs[pp], sf = sfs[pp];
             const float x0 = fmaxf(u[2 * pp], 0.f), x1 = fmaxf(u[2 * pp + 1], 0.f);
             psis[lane * (R + 1) + c] = x0 * cf - x1 * sf;
             psis[lane * (R + 1) + c + 1] = x0 * sf + x1 * cf;
@@ -1291,15 +1348,11 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
                     ok[i] = fmaf(du, av[i], ok[i]);
                 }
             }
-            const long long r = g.so.row(b, n, h) + d0;
+            const long long r = g.so.row(b, n, h) + d0;  // the dK/dV kernel adds the sparse parts later
 #pragma unroll
             for (int i = 0; i < DC; i += 4) {
-                float4 x = *reinterpret_cast<float4*>(dv + r + i);
-                x.x += ov[i]; x.y += ov[i + 1]; x.z += ov[i + 2]; x.w += ov[i + 3];
-                *reinterpret_cast<float4*>(dv + r + i) = x;
-                float4 y = *reinterpret_cast<float4*>(dk + r + i);
-                y.x += ok[i]; y.y += ok[i + 1]; y.z += ok[i + 2]; y.w += ok[i + 3];
-                *reinterpret_cast<float4*>(dk + r + i) = y;
+                *reinterpret_cast<float4*>(dv + r + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
+                *reinterpret_cast<float4*>(dk + r + i) = make_float4(ok[i], ok[i + 1], ok[i + 2], ok[i + 3]);
             }
         }
     }
