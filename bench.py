@@ -358,6 +358,11 @@ def run_ours(args, w, rank, world, local_rank):
     step_ms, stage_ms = _timed_calls(slra, torch, prob, tensors, out, ws, stage_ev, args.steps, args.warmup, flush,
                                      stream, barrier)
     clk = clocks.stop()
+    # per-kernel times: a few more calls with the branches' preparation serialised (the timed calls
+    # overlap the low-rank preparation with RoPE + pooling and selection on a side stream)
+    import dataclasses
+    _, stage_serial = _timed_calls(slra, torch, dataclasses.replace(prob, debug_flags=slra.DEBUG_SERIAL_BRANCHES),
+                                   tensors, out, ws, stage_ev, 3, 3, flush, stream)
     tot_ms = replicas.max_over_ranks(sum(step_ms), dev)
     ms_per_step = tot_ms / args.steps
     job_flops = replicas.sum_over_ranks(f_total, dev)
@@ -383,6 +388,7 @@ def run_ours(args, w, rank, world, local_rank):
     if rank != 0:
         return
     stage_avg = [statistics.mean(x[i] for x in stage_ms) for i in range(6)]
+    serial_avg = [statistics.mean(x[i] for x in stage_serial) for i in range(6)]
     roof, call_roof = _rooflines(w, f_sparse, f_attn, stage_avg[5], ms_per_step)
     roof["traffic"] = load_traffic(w.name)
     cpu_v, cpu_desc, cpu_threads, _ = oracle_sample(w, x, var)  # rank 0 runs the workload itself
@@ -403,7 +409,11 @@ def run_ours(args, w, rank, world, local_rank):
         "call_roofline": call_roof,
         "e2e": {"value": replicas.job_throughput(job_flops, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "kernel_ms": dict(zip(STAGES, (round(x, 4) for x in stage_avg))),
+        "stage_ms": {"rope_table": round(stage_avg[0], 4),
+                     "preparation (rope_pool + select on the stream, low-rank summary on a side stream)":
+                         round(sum(stage_avg[1:5]), 4), "attention": round(stage_avg[5], 4)},
+        "kernel_ms": dict(zip(STAGES, (round(x, 4) for x in serial_avg))),
+        "kernel_ms_note": "each kernel alone: 3 extra calls with the preparation serialised",
         "gpu_launches": 6 * args.steps,
         "clocks": clk,
         "cpu_baseline": {"value": cpu_v, "unit": "TFLOP/s", "cores": cpu_threads, "kind": "oracle",
@@ -516,7 +526,7 @@ def run_sweep(args):
                           "rank": w.rank, "ms_per_call": ms, "tflops": f_total / (ms * 1e-3) / 1e12,
                           "attn_ms": stage_avg[5], "attn_share": stage_avg[5] / ms,
                           "attn_frac_burst": roof["frac"], "call_frac_burst": call_roof["frac"],
-                          "kernel_ms": dict(zip(STAGES, (round(x, 4) for x in stage_avg)))}), flush=True)
+                          "prep_ms": round(sum(stage_avg[1:5]), 4)}), flush=True)
         del ws, out, tensors, q, k, v, A
     print(json.dumps({"sweep_clocks": clocks.stop()}), flush=True)
 

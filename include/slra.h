@@ -35,7 +35,8 @@
  * Conventions for every entry point:
  *   - Device pointers unless stated otherwise.  The caller owns every buffer; nothing the caller
  *     passes is retained after a call returns (the library itself keeps, per device, the two copy
- *     streams and a few events slra_attn_fwd_host creates on first use, and the fixed scratch array
+ *     streams and a few events slra_attn_fwd_host creates on first use, the side stream and its two
+ *     events the forward uses to overlap the two branches' preparation, and the fixed scratch array
  *     of slra_lowrank_summary_noalloc).  Calls are asynchronous on `stream` (NULL = the legacy default
  *     stream) and never synchronize, except slra_device_status and slra_attn_fwd_host.
  *   - All arguments are validated before anything is launched; an invalid call returns a status and
@@ -125,7 +126,9 @@ enum { SLRA_BRANCH_SPARSE = 1, SLRA_BRANCH_LOWRANK = 2, SLRA_BRANCH_BOTH = 3 };
  * nothing signals, so the bounded-wait path (timeout recorded in the status word, the CTA returns
  * without issuing work) can be exercised without faulting or hanging the GPU.  Use a small
  * wait_timeout_ns with it. */
-enum { SLRA_DEBUG_UNSATISFIED_WAIT = 1 };
+enum { SLRA_DEBUG_UNSATISFIED_WAIT = 1, SLRA_DEBUG_SERIAL_BRANCHES = 2 };
+/* SLRA_DEBUG_SERIAL_BRANCHES: run the two branches' preparation one after the other on the calling
+ * stream instead of overlapping them (see slra_attn_fwd_ex), so stage_events time each kernel alone. */
 
 /* Nonlinearity of the low-rank feature map phi = act(x A) (slra_problem.activation).  RELU is the
  * benchmark's map; SILU (u / (1 + e^-u)), IDENTITY and TANH are the alternatives RoLA's ablation
@@ -156,12 +159,16 @@ typedef enum slra_activation {
  *   rope_split              rotary pairs per (t, h, w); all zero = default split described above.
  *   wait_timeout_ns         bound of every wait inside the kernels (default 2e9 ns = 2 s).
  *   debug_flags             SLRA_DEBUG_* test hooks (default 0).
- *   stage_events            optional cudaEvent_t handles (NULL entries are skipped), recorded on
- *                           `stream` between the library's launches so a caller can time each
- *                           kernel alone: [0] before the first launch, [1] after the rotary tables,
- *                           [2] after RoPE + pooling, [3] after block selection, [4] after the low-rank
- *                           partial sums, [5] after their reduction, [6] after the attention kernel
- *                           (the branch entry points record the boundaries of the stages they run).
+ *   stage_events            optional cudaEvent_t handles (NULL entries are skipped), recorded
+ *                           between the library's launches so a caller can time each stage: [0]
+ *                           before the first launch, [1] after the rotary tables, [2] after RoPE +
+ *                           pooling, [3] after block selection, [4] after the low-rank partial sums,
+ *                           [5] after their reduction, [6] after the attention kernel (the branch
+ *                           entry points record the boundaries of the stages they run).  With both
+ *                           branches on, the low-rank preparation runs on the library's side stream
+ *                           concurrently with RoPE + pooling and selection: [4] is recorded there and
+ *                           [5] on `stream` once both are done, so [5] -> [6] is the attention kernel
+ *                           alone (SLRA_DEBUG_SERIAL_BRANCHES serialises them for per-kernel times).
  *                           The caller creates and owns them.
  *   activation              SLRA_ACT_* map of the low-rank features (default SLRA_ACT_RELU).
  *   lowrank_norope          0 (default): the low-rank branch rotates the first r feature coordinates

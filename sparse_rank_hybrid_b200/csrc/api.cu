@@ -435,6 +435,30 @@ struct HostPipe {
 };
 HostPipe g_pipes[kMaxPipeDevices];
 
+// The low-rank branch's preparation (partial sums and their reduction, on raw k and v) does not depend
+// on the sparse branch's (RoPE + pooling, selection), so it runs on a side stream of the library's own
+// (one per device, with a fork and a join event, created on first use) while the calling stream runs
+// the other; the calling stream waits for it before the attention kernel.
+struct SideStream {
+    std::mutex mu;  // the fork/join events are shared by the calls on this device
+    bool ready = false;
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+SideStream g_side[kMaxPipeDevices];
+
+slra_status side_init(SideStream& ss) {
+    if (ss.ready) return SLRA_OK;
+    const unsigned ef = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, ef) != cudaSuccess || cudaEventCreateWithFlags(&ss.join, ef) != cudaSuccess) {
+        cudaGetLastError();
+        return SLRA_ERR_CUDA;
+    }
+    ss.ready = true;
+    return SLRA_OK;
+}
+
 slra_status pipe_init(HostPipe& hp) {
     if (hp.ready) return SLRA_OK;
     const unsigned ef = cudaEventDisableTiming;
@@ -591,16 +615,46 @@ slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, con
         return SLRA_ERR_CUDA;
 
     if ((s = begin(p, d, w, st)) != SLRA_OK) return s;
-    // a branch that is off still records its stage boundaries, so its stages time as zero
-    if (branches & SLRA_BRANCH_SPARSE) {
-        if ((s = run_select(p, d, w, q, k, v, st)) != SLRA_OK) return s;
-    } else if ((s = mark(p, 2, st)) != SLRA_OK || (s = mark(p, 3, st)) != SLRA_OK) {
-        return s;
-    }
-    if (branches & SLRA_BRANCH_LOWRANK) {
-        if ((s = run_lowrank(p, d, w, k, v, A, st)) != SLRA_OK) return s;
-    } else if ((s = mark(p, 4, st)) != SLRA_OK || (s = mark(p, 5, st)) != SLRA_OK) {
-        return s;
+    const bool overlap = branches == SLRA_BRANCH_BOTH && !(p->debug_flags & SLRA_DEBUG_SERIAL_BRANCHES);
+    if (overlap) {
+        int dev = -1;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxPipeDevices) {
+            cudaGetLastError();
+            return SLRA_ERR_NO_DEVICE;
+        }
+        SideStream& ss = g_side[dev];
+        std::lock_guard<std::mutex> lock(ss.mu);
+        if ((s = side_init(ss)) != SLRA_OK) return s;
+        if (cudaEventRecord(ss.fork, st) != cudaSuccess || cudaStreamWaitEvent(ss.s, ss.fork, 0) != cudaSuccess)
+            return SLRA_ERR_CUDA;
+        // the low-rank preparation on the side stream (stage events [4], [5] recorded there), the
+        // sparse one on the calling stream; the join is enqueued whatever happened, so nothing of this
+        // call is left running unordered
+        const slra_status s_lr = run_lowrank(p, d, w, k, v, A, ss.s);
+        const bool rec = cudaEventRecord(ss.join, ss.s) == cudaSuccess;
+        const slra_status s_sel = run_select(p, d, w, q, k, v, st);
+        const bool joined = rec && cudaStreamWaitEvent(st, ss.join, 0) == cudaSuccess;
+        if (!joined) {
+            cudaGetLastError();
+            cudaStreamSynchronize(ss.s);
+            return SLRA_ERR_CUDA;
+        }
+        if (s_lr != SLRA_OK) return s_lr;
+        if (s_sel != SLRA_OK) return s_sel;
+        // [5] again, on the calling stream: both preparations are done and the attention kernel starts
+        if ((s = mark(p, 5, st)) != SLRA_OK) return s;
+    } else {
+        // a branch that is off still records its stage boundaries, so its stages time as zero
+        if (branches & SLRA_BRANCH_SPARSE) {
+            if ((s = run_select(p, d, w, q, k, v, st)) != SLRA_OK) return s;
+        } else if ((s = mark(p, 2, st)) != SLRA_OK || (s = mark(p, 3, st)) != SLRA_OK) {
+            return s;
+        }
+        if (branches & SLRA_BRANCH_LOWRANK) {
+            if ((s = run_lowrank(p, d, w, k, v, A, st)) != SLRA_OK) return s;
+        } else if ((s = mark(p, 4, st)) != SLRA_OK || (s = mark(p, 5, st)) != SLRA_OK) {
+            return s;
+        }
     }
 
     AttnArgs a;

@@ -19,7 +19,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DE
     ERR_NO_DEVICE, ERR_SCRATCH_LIMIT = range(1, 10)
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
-DEBUG_UNSATISFIED_WAIT = 1
+DEBUG_UNSATISFIED_WAIT, DEBUG_SERIAL_BRANCHES = 1, 2
 ABI_VERSION = 6
 DTYPE_BF16, DTYPE_F32 = 0, 1
 ACT_RELU, ACT_SILU, ACT_IDENTITY, ACT_TANH = 0, 1, 2, 3

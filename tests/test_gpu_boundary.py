@@ -142,3 +142,37 @@ def test_null_workspace_reports_device_status():
     slra.attn_fwd_tensors(q, t["k"], t["v"], t["A"], w.T, w.H, w.W, w.block, w.keep_frac, w.rank, out)
     assert slra.get_device_status() == slra.ERR_RANGE
     assert slra.get_device_status() == slra.OK
+
+
+@pytest.mark.parametrize("w", [W.TINY, EDGE_128], ids=lambda w: w.name)
+def test_overlapped_preparation_equals_serial(w):
+    """With both branches on, the low-rank preparation runs on the library's side stream while the
+    calling stream runs RoPE + pooling and selection; the result equals the serialised order bit for bit
+    (the same kernels on the same bytes), also when two host threads call on two streams at once."""
+    import threading
+    import torch
+    _, t = _inputs(w)
+    ser, _, _ = _ex(w, t, debug_flags=slra.DEBUG_SERIAL_BRANCHES)
+    ovl, _, _ = _ex(w, t)
+    assert torch.equal(ser, ovl)
+    p = slra.Problem.from_workload(w)
+    outs, errs = [None, None], []
+
+    def run(i):
+        try:
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                o, ws = slra.attn_fwd(p, t["q"], t["k"], t["v"], t["A"], stream=s)
+                s.synchronize()
+                assert slra.device_status(ws, stream=s) == slra.OK
+                outs[i] = o
+        except Exception as e:  # noqa: BLE001
+            errs.append(e)
+
+    th = [threading.Thread(target=run, args=(i,)) for i in range(2)]
+    for x in th:
+        x.start()
+    for x in th:
+        x.join()
+    assert not errs, errs
+    assert torch.equal(outs[0], ser) and torch.equal(outs[1], ser)
