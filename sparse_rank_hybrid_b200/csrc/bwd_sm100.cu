@@ -57,6 +57,15 @@ __device__ __forceinline__ uint32_t packed_col(int kk) {
 }  // namespace
 
 
+// Bring this thread's half of a gradient row (D/2 fp32) towards L2 before the row is read back, so the
+// read in the epilogue overlaps the last products instead of following them.
+template <int D>
+__device__ __forceinline__ void prefetch_half_row(const float* row, int hf) {
+#pragma unroll
+    for (int o = 0; o < D / 2; o += 32)  // 128-byte lines
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(row + hf * (D / 2) + o));
+}
+
 // Rotate the pairs of this thread's D/2 columns back by R(p)^T and add them (fp32) to a token-major row
 // (which holds the low-rank branch's part, or zeros); `vals` are the 32-bit TMEM words of columns
 // [hf*D/2, hf*D/2 + D/2) of the row, already scaled.
@@ -321,8 +330,9 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
             tc_fence_before();
             mbar_arrive(bars + kDqBarDs + (j & 1));
         }
-        // ---- epilogue: dq = R(p)^T dQ^ / sqrt(D), token-major fp32
+        // ---- epilogue: dq += R(p)^T dQ^ / sqrt(D), token-major fp32
         if (keep > 0) {
+            if (ok && row_real) prefetch_half_row<D>(a.dq + g.so.row(b, n, h), hf);
             const bool done = ok && __all_sync(0xffffffffu, mbar_wait(bars + kDqBarFinal, 0, tmo, abort_flag));
             if (done) {
                 tc_fence_after();
@@ -582,7 +592,11 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
             tc_fence_before();
             mbar_arrive(bars + kKvBarDs + s);
         }
-        // ---- epilogue: dv = sum P^T dO, dk = R(p)^T dK^ / sqrt(D); key blocks nobody kept get zeros
+        // ---- epilogue: dv += sum P^T dO, dk += R(p)^T dK^ / sqrt(D); key blocks nobody kept add zeros
+        if (ok && row_real) {
+            prefetch_half_row<D>(a.dv + g.so.row(b, n, h), hf);
+            prefetch_half_row<D>(a.dk + g.so.row(b, n, h), hf);
+        }
         const bool done = cnt == 0 || (ok && __all_sync(0xffffffffu, mbar_wait(bars + kKvBarFinal, 0, tmo, abort_flag)));
         if (done) {
             if (cnt > 0) tc_fence_after();
