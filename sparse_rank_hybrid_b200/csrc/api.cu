@@ -1097,6 +1097,9 @@ slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, c
         l.dS = reinterpret_cast<float*>(base + bl.dS);
         l.dz = reinterpret_cast<float*>(base + bl.dz);
         l.nsplit = bl.ns;
+        l.meta = &d.meta;
+        l.status = w.status;
+        l.timeout_ns = timeout_of(p);
         if ((s = cuda_status(launch_lr_bwd(l, g, st))) != SLRA_OK) return s;
     } else if (cudaMemsetAsync(dA, 0, ab, st) != cudaSuccess || cudaMemsetAsync(dq, 0, gb, st) != cudaSuccess ||
                cudaMemsetAsync(dk, 0, gb, st) != cudaSuccess || cudaMemsetAsync(dv, 0, gb, st) != cudaSuccess) {

@@ -1401,6 +1401,7 @@ size_t lr_bwd_tiled_smem(int D, int R, bool qpass) {
 }
 
 int lr_bwd_nsplit(const Geom& g) {
+    if (lr_bwd_on_tensor_cores(g)) return lowrank_nsplit(g);  // 128-token tiles, about 8 items per CTA
     const int TT = g.R <= 64 ? 32 : 16;
     const long long ntiles = (g.L + TT - 1) / TT;
     long long ns = (2 * 148 + g.BH() - 1) / g.BH();
@@ -1469,6 +1470,13 @@ cudaError_t launch_bwd_sparse(const BwdMaps& m, const BwdArgs& a, const Geom& g,
 }
 
 cudaError_t launch_lr_bwd(const LrBwdArgs& l, const Geom& g, cudaStream_t st) {
+    if (lr_bwd_on_tensor_cores(g)) {
+        cudaError_t e = launch_lr_bwd_tc(l, g, st);
+        if (e != cudaSuccess) return e;
+        const int DR = g.D * g.R;
+        bwd_da_reduce_kernel<<<(DR + 255) / 256, 256, 0, st>>>(l.da_part, 2 * g.BH() * l.nsplit, DR, l.dA);
+        return cudaGetLastError();
+    }
     if (g.D == 128) {
         switch (g.R) {
             case 16: return launch_lr_bwd_t<128, 16>(l, g, st);

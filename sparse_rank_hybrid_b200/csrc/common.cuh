@@ -161,12 +161,18 @@ struct LrBwdArgs {
     float *dq, *dk, *dv, *dA;
     float *ds_part, *dz_part, *da_part, *dS, *dz;
     int nsplit;
+    const RopeMeta* meta;  // rotary schedule (tensor-core passes)
+    int* status;
+    unsigned long long timeout_ns;
 };
 cudaError_t launch_bwd_prep(const float* dout, const float* os, const Geom& g, __half* doh, float* delta, int* status,
                             cudaStream_t st);
 cudaError_t launch_bwd_invert(const int32_t* idx, const Geom& g, int32_t* inv, int32_t* inv_cnt, cudaStream_t st);
 cudaError_t launch_bwd_sparse(const BwdMaps& m, const BwdArgs& a, const Geom& g, cudaStream_t st);
 cudaError_t launch_lr_bwd(const LrBwdArgs& l, const Geom& g, cudaStream_t st);
+// Tensor-core low-rank gradient passes (head_dim 128, rank <= 48), see lr_bwd_sm100.cu.
+cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st);
+inline bool lr_bwd_on_tensor_cores(const Geom& g) { return g.D == 128 && g.R <= 48; }
 int lr_bwd_nsplit(const Geom& g);
 
 }  // namespace slra
