@@ -348,11 +348,11 @@ SLRA_API size_t slra_bwd_workspace_bytes(const slra_problem* p);
  * dP = dO v^T in TMEM, dS = P (dP - rowsum(dO O_sparse)), dQ^ += dS k^) and a dK/dV kernel per key block
  * over the query blocks that kept it (dV += P^T dO, dK^ += dS^T q^), with fp16 operands (dout must stay
  * below 65504 in magnitude, else SLRA_ERR_RANGE is recorded) and fp32 accumulation; the low-rank chain
- * runs first, as fp32 passes over the queries and the keys that store dq, dk, dv and dA, and the sparse
- * kernels add their parts.  Deterministic.  stage_events are recorded at: [0] start, [1] after the
- * recomputed forward, [2] after the low-rank gradients, [3] after the dO copy and the inverted lists,
- * [4] after the dQ kernel, [5] and [6] after the dK/dV kernel.  Device problems go to the workspace's
- * status word (slra_device_status).
+ * follows as a pass over the queries and one over the keys (on the tensor cores for head_dim 128 and
+ * rank <= 48, fp32 otherwise) that add their parts to dq, dk, dv and produce dA.  Deterministic.
+ * stage_events are recorded at: [0] start, [1] after the recomputed forward, [2] after the dO copy and
+ * the inverted lists, [3] after the dQ kernel, [4] after the dK/dV kernel, [5] and [6] after the
+ * low-rank gradients.  Device problems go to the workspace's status word (slra_device_status).
  */
 SLRA_API slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, const void* v,
                                    const void* A, const float* dout, float* dq, float* dk, float* dv, float* dA,

@@ -1074,8 +1074,41 @@ slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, c
         if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
     }
     if ((s = mark(p, 1, st)) != SLRA_OK) return s;
-    // The low-rank gradients go first and store dq, dk, dv (and dA); the sparse kernels then add their
-    // parts row by row.  Without the low-rank branch the gradients start from zero.
+    // The sparse kernels store dq, dk, dv; the low-rank gradients then add their parts (or store them
+    // when the sparse branch is off).
+    if (sparse) {
+        if ((s = cuda_status(launch_bwd_prep(dout, os, g, doh, delta, w.status, st))) != SLRA_OK) return s;
+        if ((s = cuda_status(launch_bwd_invert(w.idx, g, inv, inv_cnt, st))) != SLRA_OK) return s;
+        if ((s = mark(p, 2, st)) != SLRA_OK) return s;
+        BwdMaps m;
+        const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
+        if (!make_map_headmajor(&m.q128, w.qh, rows, g.D, 128) || !make_map_headmajor(&m.do128, doh, rows, g.D, 128) ||
+            !make_map_headmajor(&m.kb, w.kh, rows, g.D, g.block) || !make_map_headmajor(&m.vb, w.vh, rows, g.D, g.block) ||
+            !make_map_headmajor(&m.k128, w.kh, rows, g.D, 128) || !make_map_headmajor(&m.v128, w.vh, rows, g.D, 128) ||
+            !make_map_headmajor(&m.qb, w.qh, rows, g.D, g.block) || !make_map_headmajor(&m.dob, doh, rows, g.D, g.block))
+            return SLRA_ERR_CUDA;
+        m.between = static_cast<cudaEvent_t>(p->stage_events[3]);
+        BwdArgs ba;
+        ba.idx = w.idx;
+        ba.keep = g.keep;
+        ba.inv = inv;
+        ba.inv_cnt = inv_cnt;
+        ba.lse = lse;
+        ba.delta = delta;
+        ba.tab = w.tab;
+        for (int e = 0; e < kMaxPairs; ++e)
+            ba.pair_info[e] = e < d.meta.npairs ? make_int2(d.meta.axis[e], d.meta.tab_off[e]) : make_int2(0, 0);
+        ba.dq = dq;
+        ba.dk = dk;
+        ba.dv = dv;
+        ba.accumulate = 0;
+        ba.status = w.status;
+        ba.timeout_ns = timeout_of(p);
+        if ((s = cuda_status(launch_bwd_sparse(m, ba, g, st))) != SLRA_OK) return s;
+    } else if ((s = mark(p, 2, st)) != SLRA_OK || (s = mark(p, 3, st)) != SLRA_OK) {
+        return s;
+    }
+    if ((s = mark(p, 4, st)) != SLRA_OK) return s;
     if (lowrank) {
         LrBwdArgs l;
         l.q = static_cast<const __nv_bfloat16*>(q);
@@ -1100,42 +1133,10 @@ slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, c
         l.meta = &d.meta;
         l.status = w.status;
         l.timeout_ns = timeout_of(p);
+        l.accumulate = sparse ? 1 : 0;
         if ((s = cuda_status(launch_lr_bwd(l, g, st))) != SLRA_OK) return s;
-    } else if (cudaMemsetAsync(dA, 0, ab, st) != cudaSuccess || cudaMemsetAsync(dq, 0, gb, st) != cudaSuccess ||
-               cudaMemsetAsync(dk, 0, gb, st) != cudaSuccess || cudaMemsetAsync(dv, 0, gb, st) != cudaSuccess) {
+    } else if (cudaMemsetAsync(dA, 0, ab, st) != cudaSuccess) {
         return SLRA_ERR_CUDA;
-    }
-    if ((s = mark(p, 2, st)) != SLRA_OK) return s;
-    if (sparse) {
-        if ((s = cuda_status(launch_bwd_prep(dout, os, g, doh, delta, w.status, st))) != SLRA_OK) return s;
-        if ((s = cuda_status(launch_bwd_invert(w.idx, g, inv, inv_cnt, st))) != SLRA_OK) return s;
-        if ((s = mark(p, 3, st)) != SLRA_OK) return s;
-        BwdMaps m;
-        const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
-        if (!make_map_headmajor(&m.q128, w.qh, rows, g.D, 128) || !make_map_headmajor(&m.do128, doh, rows, g.D, 128) ||
-            !make_map_headmajor(&m.kb, w.kh, rows, g.D, g.block) || !make_map_headmajor(&m.vb, w.vh, rows, g.D, g.block) ||
-            !make_map_headmajor(&m.k128, w.kh, rows, g.D, 128) || !make_map_headmajor(&m.v128, w.vh, rows, g.D, 128) ||
-            !make_map_headmajor(&m.qb, w.qh, rows, g.D, g.block) || !make_map_headmajor(&m.dob, doh, rows, g.D, g.block))
-            return SLRA_ERR_CUDA;
-        m.between = static_cast<cudaEvent_t>(p->stage_events[4]);
-        BwdArgs ba;
-        ba.idx = w.idx;
-        ba.keep = g.keep;
-        ba.inv = inv;
-        ba.inv_cnt = inv_cnt;
-        ba.lse = lse;
-        ba.delta = delta;
-        ba.tab = w.tab;
-        for (int e = 0; e < kMaxPairs; ++e)
-            ba.pair_info[e] = e < d.meta.npairs ? make_int2(d.meta.axis[e], d.meta.tab_off[e]) : make_int2(0, 0);
-        ba.dq = dq;
-        ba.dk = dk;
-        ba.dv = dv;
-        ba.status = w.status;
-        ba.timeout_ns = timeout_of(p);
-        if ((s = cuda_status(launch_bwd_sparse(m, ba, g, st))) != SLRA_OK) return s;
-    } else if ((s = mark(p, 3, st)) != SLRA_OK || (s = mark(p, 4, st)) != SLRA_OK) {
-        return s;
     }
     if ((s = mark(p, 5, st)) != SLRA_OK) return s;
     return mark(p, 6, st);

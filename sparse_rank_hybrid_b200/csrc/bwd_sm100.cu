@@ -66,15 +66,17 @@ __device__ __forceinline__ void prefetch_half_row(const float* row, int hf) {
         asm volatile("prefetch.global.L2 [%0];" ::"l"(row + hf * (D / 2) + o));
 }
 
-// Rotate the pairs of this thread's D/2 columns back by R(p)^T and add them (fp32) to a token-major row
-// (which holds the low-rank branch's part, or zeros); `vals` are the 32-bit TMEM words of columns
-// [hf*D/2, hf*D/2 + D/2) of the row, already scaled.
+// Rotate the pairs of this thread's D/2 columns back by R(p)^T and store them (fp32) into a token-major
+// row, or add them to it when a.accumulate (the row then holds the low-rank branch's part); `vals` are
+// the 32-bit TMEM words of columns [hf*D/2, hf*D/2 + D/2) of the row, already scaled.
 template <int D>
 __device__ __forceinline__ void store_row_unrotated(float* dst_row, const float* vals, int hf, int n,
                                                     const BwdArgs& a, const Geom& g, bool rotate) {
     float4 prev[D / 8];
 #pragma unroll
-    for (int t = 0; t < D / 8; ++t) prev[t] = *reinterpret_cast<const float4*>(dst_row + hf * (D / 2) + 4 * t);
+    for (int t = 0; t < D / 8; ++t)
+        prev[t] = a.accumulate ? *reinterpret_cast<const float4*>(dst_row + hf * (D / 2) + 4 * t)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
     const int pt = n / (g.H * g.W), ph = (n / g.W) % g.H, pw = n % g.W;
 #pragma unroll
     for (int t = 0; t < D / 8; ++t) {  // 4 columns (2 pairs) per float4
@@ -332,7 +334,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
         }
         // ---- epilogue: dq += R(p)^T dQ^ / sqrt(D), token-major fp32
         if (keep > 0) {
-            if (ok && row_real) prefetch_half_row<D>(a.dq + g.so.row(b, n, h), hf);
+            if (ok && row_real && a.accumulate) prefetch_half_row<D>(a.dq + g.so.row(b, n, h), hf);
             const bool done = ok && __all_sync(0xffffffffu, mbar_wait(bars + kDqBarFinal, 0, tmo, abort_flag));
             if (done) {
                 tc_fence_after();
@@ -593,7 +595,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
             mbar_arrive(bars + kKvBarDs + s);
         }
         // ---- epilogue: dv += sum P^T dO, dk += R(p)^T dK^ / sqrt(D); key blocks nobody kept add zeros
-        if (ok && row_real) {
+        if (ok && row_real && a.accumulate) {
             prefetch_half_row<D>(a.dv + g.so.row(b, n, h), hf);
             prefetch_half_row<D>(a.dk + g.so.row(b, n, h), hf);
         }
@@ -715,7 +717,8 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
                                                        const double2* __restrict__ tab,
                                                        const int2* __restrict__ pairs, Geom g, int nsplit,
                                                        float* __restrict__ dq, float* __restrict__ ds_part,
-                                                       float* __restrict__ dz_part, float* __restrict__ da_part) {
+                                                       float* __restrict__ dz_part, float* __restrict__ da_part,
+                                                       int accumulate) {
     constexpr int TT = LrTile<R>::T;
     extern __shared__ __align__(16) float smf[];
     // A and S padded by one column: the loops below read them with consecutive lanes walking either
@@ -849,7 +852,8 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
             float s = 0.f;
 #pragma unroll 8
             for (int c = 0; c < R; ++c) s = fmaf(dus[tt * (R + 1) + c], As[d * (R + 1) + c], s);
-            dq[g.so.row(b, n, h) + d] = s;
+            float* dst = dq + g.so.row(b, n, h) + d;
+            *dst = accumulate ? *dst + s : s;
         }
     }
     const size_t slot = static_cast<size_t>(bh) * nsplit + split;
@@ -871,7 +875,7 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
                                                        const double2* __restrict__ tab,
                                                        const int2* __restrict__ pairs, Geom g, int nsplit,
                                                        float* __restrict__ dk, float* __restrict__ dv,
-                                                       float* __restrict__ da_part) {
+                                                       float* __restrict__ da_part, int accumulate) {
     constexpr int TT = LrTile<R>::T;
     extern __shared__ __align__(16) float smf[];
     float* As = smf;                    // [D][R+1] (padded as in the query pass)
@@ -965,8 +969,8 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
                 sk = fmaf(ps[tt * (R + 1) + c], As[d * (R + 1) + c], sk);
             }
             const long long r = g.so.row(b, n, h) + d;
-            dv[r] = sv;
-            dk[r] = sk;
+            dv[r] = accumulate ? dv[r] + sv : sv;
+            dk[r] = accumulate ? dk[r] + sk : sk;
         }
     }
     const size_t slot = static_cast<size_t>(bh) * nsplit + split;
@@ -1010,7 +1014,8 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
                                                              const double2* __restrict__ tab,
                                                              const int2* __restrict__ pairs, Geom g, int nsplit,
                                                              float* __restrict__ dq, float* __restrict__ ds_part,
-                                                             float* __restrict__ dz_part, float* __restrict__ da_part) {
+                                                             float* __restrict__ dz_part, float* __restrict__ da_part,
+                                                             int accumulate) {
     constexpr int TT = 32, FC = R / 8, DC = D / 8;
     static_assert(R <= 64 && FC % 2 == 0, "rank 16..64");
     extern __shared__ __align__(16) float smf[];
@@ -1191,10 +1196,16 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
 #pragma unroll
                 for (int i = 0; i < DC; ++i) o[i] = fmaf(du, av[i], o[i]);
             }
-            float* dst = dq + g.so.row(b, n, h) + d0;  // the sparse branch's dQ kernel adds its part later
+            float* dst = dq + g.so.row(b, n, h) + d0;
 #pragma unroll
-            for (int i = 0; i < DC; i += 4)
-                *reinterpret_cast<float4*>(dst + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+            for (int i = 0; i < DC; i += 4) {
+                float4 v = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+                if (accumulate) {  // the sparse part is there already
+                    const float4 p = *reinterpret_cast<const float4*>(dst + i);
+                    v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+                }
+                *reinterpret_cast<float4*>(dst + i) = v;
+            }
         }
     }
     const size_t slot = static_cast<size_t>(bh) * nsplit + split;
@@ -1214,7 +1225,7 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
                                                              const double2* __restrict__ tab,
                                                              const int2* __restrict__ pairs, Geom g, int nsplit,
                                                              float* __restrict__ dk, float* __restrict__ dv,
-                                                             float* __restrict__ da_part) {
+                                                             float* __restrict__ da_part, int accumulate) {
     constexpr int TT = 32, FC = R / 8, DC = D / 8;
     static_assert(R <= 64 && FC % 2 == 0, "rank 16..64");
     extern __shared__ __align__(16) float smf[];
@@ -1362,11 +1373,19 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
                     ok[i] = fmaf(du, av[i], ok[i]);
                 }
             }
-            const long long r = g.so.row(b, n, h) + d0;  // the dK/dV kernel adds the sparse parts later
+            const long long r = g.so.row(b, n, h) + d0;
 #pragma unroll
             for (int i = 0; i < DC; i += 4) {
-                *reinterpret_cast<float4*>(dv + r + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
-                *reinterpret_cast<float4*>(dk + r + i) = make_float4(ok[i], ok[i + 1], ok[i + 2], ok[i + 3]);
+                float4 x = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
+                float4 y = make_float4(ok[i], ok[i + 1], ok[i + 2], ok[i + 3]);
+                if (accumulate) {  // the sparse parts are there already
+                    const float4 px = *reinterpret_cast<const float4*>(dv + r + i);
+                    const float4 py = *reinterpret_cast<const float4*>(dk + r + i);
+                    x.x += px.x; x.y += px.y; x.z += px.z; x.w += px.w;
+                    y.x += py.x; y.y += py.y; y.z += py.z; y.w += py.w;
+                }
+                *reinterpret_cast<float4*>(dv + r + i) = x;
+                *reinterpret_cast<float4*>(dk + r + i) = y;
             }
         }
     }
@@ -1437,13 +1456,13 @@ cudaError_t launch_lr_bwd_t(const LrBwdArgs& l, const Geom& g, cudaStream_t st) 
     e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk);
     if (e != cudaSuccess) return e;
     qk<<<dim3(ns, g.BH()), 256, smq, st>>>(l.q, l.dout, l.A, l.S, l.z, l.tab, l.pairs, g, ns, l.dq, l.ds_part,
-                                           l.dz_part, l.da_part);
+                                           l.dz_part, l.da_part, l.accumulate);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_lowrank_reduce(l.ds_part, l.dz_part, g, ns, l.dS, l.dz, nullptr, nullptr, nullptr, st)) !=
         cudaSuccess)
         return e;
     kk<<<dim3(ns, g.BH()), 256, smk, st>>>(l.k, l.v, l.A, l.dS, l.dz, l.tab, l.pairs, g, ns, l.dk, l.dv,
-                                           l.da_part + static_cast<size_t>(g.BH()) * ns * D * R);
+                                           l.da_part + static_cast<size_t>(g.BH()) * ns * D * R, l.accumulate);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int DR = D * R;
     bwd_da_reduce_kernel<<<(DR + 255) / 256, 256, 0, st>>>(l.da_part, 2 * g.BH() * ns, DR, l.dA);

@@ -142,6 +142,7 @@ struct BwdArgs {
     float* dq;  // token-major fp32 [B][L][Hh][D] (strides g.so)
     float* dk;
     float* dv;
+    int accumulate;  // 1: add to the rows (the low-rank part is already there); 0: store them
     int* status;
     unsigned long long timeout_ns;
 };
@@ -164,6 +165,7 @@ struct LrBwdArgs {
     const RopeMeta* meta;  // rotary schedule (tensor-core passes)
     int* status;
     unsigned long long timeout_ns;
+    int accumulate;  // tensor-core passes: 1 adds dq, dk, dv to the rows (the sparse part is there)
 };
 cudaError_t launch_bwd_prep(const float* dout, const float* os, const Geom& g, __half* doh, float* delta, int* status,
                             cudaStream_t st);

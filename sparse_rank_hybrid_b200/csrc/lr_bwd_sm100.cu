@@ -74,6 +74,7 @@ struct LrTcBwdArgs {
     float* dz_part;  // [BH][nsplit][R]
     float* da_part;  // [BH][nsplit][D][R]
     int nsplit, tiles_per_split;
+    int accumulate;  // 1: add dq (dk, dv) to the rows; 0: store them
     int* status;
     unsigned long long timeout_ns;
 };
@@ -236,6 +237,16 @@ __global__ void __launch_bounds__(256, 1)
                     }
                 }
                 fence_async_smem();
+            }
+            // the rows this tile's outputs are added to, brought towards L2 while the tile is computed
+            if (a.accumulate && live) {
+                const size_t r0 = g.so.row(b, n, h) + half * 64;
+#pragma unroll
+                for (int which = 0; which < (kKey ? 2 : 1); ++which) {
+                    const float* rowp = (kKey ? (which ? a.dk : a.dv) : a.dq) + r0;
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(rowp));
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(rowp + 32));
+                }
             }
             // (cos, sin) of this row's pairs, loaded while the tile lands
             const int nt = live ? n : 0;
@@ -430,10 +441,15 @@ __global__ void __launch_bounds__(256, 1)
                     tmem_ld_wait(r);
                     if (live) {
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(dst + c0 + i) =
-                                make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
-                                            __uint_as_float(r[i + 3]));
+                        for (int i = 0; i < 32; i += 4) {
+                            float4 v = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                                   __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+                            if (a.accumulate) {
+                                const float4 p = *reinterpret_cast<const float4*>(dst + c0 + i);
+                                v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+                            }
+                            *reinterpret_cast<float4*>(dst + c0 + i) = v;
+                        }
                     }
                 }
             }
@@ -561,6 +577,7 @@ cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st)
     a.tiles_per_split = ((g.L + kTok - 1) / kTok + l.nsplit - 1) / l.nsplit;
     a.status = l.status;
     a.timeout_ns = l.timeout_ns;
+    a.accumulate = l.accumulate;
     switch (g.R) {
         case 16: return launch_lr_bwd_tc_r<16>(a, g, tq, tk, tv, l.dS, l.dz, st);
         case 32: return launch_lr_bwd_tc_r<32>(a, g, tq, tk, tv, l.dS, l.dz, st);
