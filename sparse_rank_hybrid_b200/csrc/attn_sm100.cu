@@ -66,12 +66,11 @@ struct AttnLayout {
 enum : int {
     kBarQ = 0,
     kBarKFull = 1,    // +slot: k_0, k_1 landed (the first two S)
-    kBarKEmpty = 3,   // +slot: S that read the slot has completed
+    kBarKvEmpty = 3,  // +slot: the products that read the slot's k and v tiles have completed
     kBarVFull = 5,    // +slot: v_j and, when there is one, k_{j+2} landed (block j's two products)
-    kBarVEmpty = 7,   // +slot: P.V that read the slot has completed
-    kBarSFull = 9,    // +buffer: S_j in TMEM
+    kBarSFull = 9,    // +buffer: S_j in TMEM (and every product issued before it completed)
     kBarPFull = 12,   // +buffer: P_j in TMEM (one arrival per softmax thread)
-    kBarODone = 15,   // +buffer: P.V_j (reading P from that buffer) has completed
+    kBarODone = 15,   // P.V_{keep-2} has completed (one phase)
     kBarEld = 18,     // epilogue: raw query tile + A^T image
     kBarEz = 19,      // epilogue: S image of each 64-feature chunk
     kBarEmm = 20,     // epilogue products
@@ -251,19 +250,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int sl = 0; sl < D / 64; ++sl) tma_load_2d(dst + sl * (rows * 128), tm, bar, sl * 64, row);
             };
+            // Slot s's k and v tiles are read by the products the MMA warp issues together (P.V_j with
+            // S_{j+2}), so one commit frees both: v_j and k_{j+2} go into slot s once P.V_{j-2} and S_j
+            // have completed (for j < 2: S_j alone, and v_j needs no wait).
             for (int j = 0; j < keep && ok; ++j) {
                 const int s = j & 1;
                 const bool has_k = j + 2 < keep;
-                // v_j into slot s once P.V_{j-2} (the slot's previous reader) has completed
-                if (j >= 2 && !mbar_wait(bars + kBarVEmpty + s, ((j - 2) >> 1) & 1, tmo, abort_flag)) {
+                if (j >= 2 && !mbar_wait(bars + kBarKvEmpty + s, (j >> 1) & 1, tmo, abort_flag)) {
                     ok = false;
                     break;
                 }
                 add_tile(bars + kBarVFull + s, vslot(s), &tm_v, row0 + __ldg(my_idx + j) * blk, blk, !has_k);
                 ++nv;
-                // k_{j+2} into slot s once S_j has completed
                 if (has_k) {
-                    if (!mbar_wait(bars + kBarKEmpty + s, (j >> 1) & 1, tmo, abort_flag)) {
+                    if (j < 2 && !mbar_wait(bars + kBarKvEmpty + s, 0, tmo, abort_flag)) {
                         mbar_arrive(bars + kBarVFull + s);  // complete the phase v_j's bytes are on
                         ok = false;
                         break;
@@ -305,17 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ko = static_cast<uint32_t>(((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4);
                 umma_ss(dst, dq + qo, dkj + ko, idesc_s, kk > 0 ? 1u : 0u);
             };
-            auto s_done = [&](int j) {
-                umma_commit(bars + kBarSFull + j % kNumS);
-                umma_commit(bars + kBarKEmpty + (j & 1));
-            };
             auto pv_step = [&](uint32_t p, uint64_t dvj, int kk, uint32_t acc) {  // k-step kk of O += P v
                 umma_ts(tO, p + kk * 8, dvj + static_cast<uint32_t>((kk * 2048) >> 4), idesc_o, acc);
-            };
-            auto pv_done = [&](int j) {
-                umma_commit(bars + kBarVEmpty + (j & 1));
-                umma_commit(bars + kBarODone + j % kNumS);
-                if (j == keep - 1) umma_commit(bars + kBarOFinal);
             };
             constexpr int kSSteps = D / 16, kPvSteps = BLK / 16;
             bool ok = mbar_wait(bar_q, 0, tmo, abort_flag);
@@ -326,7 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t dst = tmem + j * 128;
 #pragma unroll
                     for (int kk = 0; kk < kSSteps; ++kk) s_step(dst, j ? dk1 : dk0, kk);
-                    s_done(j);
+                    umma_commit(bars + kBarSFull + j);
+                    if (j + 2 < keep) umma_commit(bars + kBarKvEmpty + j);
                 }
             }
             for (int j = 0; j < keep && ok; ++j) {
@@ -352,8 +344,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int t = 0; t < kPvSteps; ++t) pv_step(pj, dvj, t, t > 0 ? 1u : acc0);
                 }
-                pv_done(j);
-                if (has_s) s_done(j + 2);
+                // Two commits per block: a commit tracks every product issued before it, so S_{j+2}'s
+                // also reports P.V_j (the softmax's rescale of O waits on it), and one frees both tiles
+                // of slot j & 1.  The last two P.V have no S beside them and barriers of their own.
+                if (has_s) {
+                    umma_commit(bars + kBarSFull + (j + 2) % kNumS);
+                    umma_commit(bars + kBarKvEmpty + (j & 1));
+                } else {
+                    umma_commit(bars + (j == keep - 1 ? kBarOFinal : kBarODone));
+                }
             }
             if (!ok) fail();
             // One more commit tracks every product this thread issued; waiting for it (bounded, whatever
@@ -419,10 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {  // warp-uniform: TMEM access is collective
                 // Both warps of the lane group see the same maxima, so they take the same branch; each
                 // rescales its half of O's columns once P.V_{j-1} has landed in O.
-                // (per-buffer barriers: when S_j has completed, P.V_{j-2} may or may not have, so one
-                // shared counter could be three phases from here)
-                const bool landed = __all_sync(0xffffffffu, mbar_wait(bars + kBarODone + (j - 1) % kNumS,
-                                                                      ((j - 1) / kNumS) & 1, tmo, abort_flag));
+                // P.V_{j-1} completes with S_{j+1} (issued together, one commit); the last two P.V have
+                // no S beside them, and P.V_{keep-2} has a barrier of its own.  S_{j+1}'s buffer has no
+                // later phase yet (that would need P_{j+2}).
+                const bool landed = __all_sync(
+                    0xffffffffu, j + 1 < keep
+                                     ? mbar_wait(bars + kBarSFull + (j + 1) % kNumS, ((j + 1) / kNumS) & 1, tmo, abort_flag)
+                                     : mbar_wait(bars + kBarODone, 0, tmo, abort_flag));
                 tc_fence_after();
                 const float m_new = fmaxf(m_run, mx);
                 const float alpha_r = ex2_approx(m_run - m_new);

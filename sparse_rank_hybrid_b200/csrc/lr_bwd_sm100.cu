@@ -420,6 +420,19 @@ __global__ void __launch_bounds__(256, 1)
                 umma_commit(bar_m2);
                 ++n_m2_issued;
             }
+            // The values the first output is added to, loaded while the products run (all 16 loads in
+            // flight at once); the key pass loads dk's after storing dv.
+            auto out_row = [&](int which) {
+                return (kKey ? (which ? a.dk : a.dv) : a.dq) + g.so.row(b, live ? n : 0, h) + half * 64;
+            };
+            float4 prev[16];
+            auto load_prev = [&](const float* rowp) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    prev[i] = (a.accumulate && live) ? *reinterpret_cast<const float4*>(rowp + 4 * i)
+                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+            };
+            load_prev(out_row(0));
             ok = mbar_wait(bar_m2, n_m2 & 1, tmo, abort_flag);
             if (__syncthreads_or(!ok)) {
                 if (tid == 0) fail();
@@ -433,7 +446,8 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
             for (int which = 0; which < (kKey ? 2 : 1); ++which) {
                 const uint32_t src = kKey ? (which ? tK : tV) : tO;
-                float* dst = (kKey ? (which ? a.dk : a.dv) : a.dq) + g.so.row(b, live ? n : 0, h) + half * 64;
+                float* dst = out_row(which);
+                if (which == 1) load_prev(dst);
 #pragma unroll
                 for (int c0 = 0; c0 < 64; c0 += 32) {
                     uint32_t r[32];
@@ -442,12 +456,9 @@ __global__ void __launch_bounds__(256, 1)
                     if (live) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 4) {
-                            float4 v = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                                                   __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-                            if (a.accumulate) {
-                                const float4 p = *reinterpret_cast<const float4*>(dst + c0 + i);
-                                v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
-                            }
+                            const float4 p = prev[(c0 + i) / 4];
+                            const float4 v = make_float4(__uint_as_float(r[i]) + p.x, __uint_as_float(r[i + 1]) + p.y,
+                                                         __uint_as_float(r[i + 2]) + p.z, __uint_as_float(r[i + 3]) + p.w);
                             *reinterpret_cast<float4*>(dst + c0 + i) = v;
                         }
                     }
