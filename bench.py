@@ -426,7 +426,8 @@ def run_backward(args, w):
     """The backward pass (slra_attn_bwd) at the workload's shape on one GPU: ms per call, per-stage
     times, and the sparse gradient kernels' throughput against the algorithmic count (five products per
     kept (query block, key block) pair: S, dP, dQ, dK, dV = 2.5x the forward's kept FLOPs; the kernels
-    recompute S and dP once more, which is not counted).  One JSON line (not the benchmark contract)."""
+    recompute S and dP once more, which is not counted); then a training step, the forward that keeps
+    its state followed by the backward from it.  One JSON line (not the benchmark contract)."""
     import torch
     from sparse_rank_hybrid_b200 import build as B
     from sparse_rank_hybrid_b200 import slra
@@ -467,10 +468,34 @@ def run_backward(args, w):
         torch.cuda.synchronize()
         tot.append(a.elapsed_time(b))
         stages.append([ev[i].elapsed_time(ev[i + 1]) for i in range(6)])
+    # A training step: the forward that keeps its state (slra_attn_fwd_train), then the backward from it
+    # (slra_attn_bwd_saved), with no recompute.
+    prob_f = slra.Problem.from_workload(w)
+    out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
+    for _ in range(max(3, args.warmup)):
+        slra.attn_fwd_train(prob_f, q, k, v, A, out=out, workspace=ws)
+        slra.attn_bwd_saved(prob, q, k, v, A, dout, ws, grads=grads)
+    torch.cuda.synchronize()
+    if slra.device_status(ws) != slra.OK:
+        raise RuntimeError("device status after the training-step warm-up")
+    t_fwd, t_bwd, st_saved = [], [], []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, m, b = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(stream)
+        slra.attn_fwd_train(prob_f, q, k, v, A, out=out, workspace=ws)
+        m.record(stream)
+        slra.attn_bwd_saved(prob, q, k, v, A, dout, ws, grads=grads)
+        b.record(stream)
+        torch.cuda.synchronize()
+        t_fwd.append(a.elapsed_time(m))
+        t_bwd.append(m.elapsed_time(b))
+        st_saved.append([ev[i].elapsed_time(ev[i + 1]) for i in range(6)])
     clk = clocks.stop()
     if slra.device_status(ws) != slra.OK:
         raise RuntimeError("device status after timing")
     st = [statistics.mean(s_[i] for s_ in stages) for i in range(6)]
+    sts = [statistics.mean(s_[i] for s_ in st_saved) for i in range(6)]
     ms = statistics.mean(tot)
     _, tf_burst, tf_sust, src = peaks()
     f_bwd_sparse = 2.5 * f_sparse
@@ -485,6 +510,11 @@ def run_backward(args, w):
                            "peak": tf_burst, "peak_source": f"{src} burst bf16 (same rate as f16)"},
             "lowrank_bwd_flops": f_lr_bwd,
             "whole_call_tflops": (f_bwd_sparse + f_lr_bwd) / (ms * 1e-3) / 1e12,
+            "train_step": {"ms": statistics.mean(t_fwd) + statistics.mean(t_bwd),
+                           "forward_train_ms": statistics.mean(t_fwd),
+                           "backward_saved_ms": statistics.mean(t_bwd),
+                           "backward_saved_stage_ms": dict(zip(("-", "dout_copy_and_lists", "dq_kernel", "dkdv_kernel",
+                                                                "lowrank_grad", "-"), (round(x_, 4) for x_ in sts)))},
             "clocks": clk}
     print(json.dumps(line), flush=True)
 

@@ -66,7 +66,7 @@
 extern "C" {
 #endif
 
-#define SLRA_ABI_VERSION 6
+#define SLRA_ABI_VERSION 7
 
 /* Exported symbols (the library is built with hidden visibility for everything else). */
 #if defined(__GNUC__)
@@ -357,6 +357,33 @@ SLRA_API size_t slra_bwd_workspace_bytes(const slra_problem* p);
 SLRA_API slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, const void* v,
                                    const void* A, const float* dout, float* dq, float* dk, float* dv, float* dA,
                                    void* workspace, size_t workspace_bytes, slra_stream_t stream);
+
+/*
+ * Forward pass for training: slra_attn_fwd_ex on the options slra_attn_bwd covers (same arguments;
+ * out contiguous), which also keeps in `workspace` what the backward would recompute: the tables, the
+ * block selection, the low-rank summary, the fp16 operand copies, each query row's log-sum-exp and
+ * the sparse branch's own output (stored by the attention kernel before the low-rank readout joins
+ * it).  out is bit for bit that of slra_attn_fwd_ex.
+ *   workspace    at least slra_bwd_workspace_bytes(p) bytes, 256-B aligned (NULL is rejected:
+ *                SLRA_ERR_WORKSPACE); its status word starts cleared, as for slra_attn_fwd_ex.
+ * Pass the same workspace, untouched, to slra_attn_bwd_saved.
+ */
+SLRA_API slra_status slra_attn_fwd_train(const slra_problem* p, const void* q, const void* k, const void* v,
+                                         const void* A, void* out, void* workspace, size_t workspace_bytes,
+                                         slra_stream_t stream);
+
+/*
+ * Backward pass from a forward kept by slra_attn_fwd_train: slra_attn_bwd without the recompute (the
+ * same problem and the same q, k, v, A as that forward; the workspace as it left it).  The gradients
+ * are bit for bit those of slra_attn_bwd.  The workspace's status word is not cleared: it holds what
+ * the forward and the backward recorded.  stage_events as for slra_attn_bwd, [1] right after [0].
+ * The library cannot tell a workspace of another problem or of other inputs: the gradients are then
+ * meaningless.
+ */
+SLRA_API slra_status slra_attn_bwd_saved(const slra_problem* p, const void* q, const void* k, const void* v,
+                                         const void* A, const float* dout, float* dq, float* dk, float* dv,
+                                         float* dA, void* workspace, size_t workspace_bytes,
+                                         slra_stream_t stream);
 
 /*
  * Device status of the calls whose workspace the library allocated (slra_attn_fwd, and the others when

@@ -372,8 +372,11 @@ bool contiguous_io(const slra_problem* p) {
 }
 
 // The forward pass on a caller's (or the library's) workspace; arguments already validated by derive.
+// `lse` and `os` (both NULL, or both set): also keep each row's lse and the sparse branch's own output
+// for a backward pass (head-major fp32, the backward workspace's sections).
 slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, const void* k, const void* v,
-                     const void* A, void* out, void* workspace, cudaStream_t st);
+                     const void* A, void* out, void* workspace, cudaStream_t st, float* lse = nullptr,
+                     float* os = nullptr);
 
 // Runs body(workspace) on the caller's workspace, or, when that is NULL, on one the library allocates
 // with cudaMallocAsync on `st` (the device's current memory pool) and frees with cudaFreeAsync after the
@@ -600,7 +603,7 @@ slra_status host_fwd_pipelined(const slra_problem* p, const Derived& d, const vo
 }
 
 slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, const void* k, const void* v,
-                     const void* A, void* out, void* workspace, cudaStream_t st) {
+                     const void* A, void* out, void* workspace, cudaStream_t st, float* lse, float* os) {
     slra_status s;
     const Ptrs w = carve(workspace, d);
     const int branches = p->branches == 0 ? SLRA_BRANCH_BOTH : p->branches;
@@ -613,6 +616,8 @@ slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, con
         !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, g.sq, 128) ||
         !make_map_out(&maps.out, out, g.B, g.L, g.Hh, g.D, g.so, p->out_dtype == SLRA_OUT_F32))
         return SLRA_ERR_CUDA;
+    std::memset(&maps.os, 0, sizeof maps.os);
+    if (os && !make_map_out(&maps.os, os, g.B, g.L, g.Hh, g.D, headmajor_strides(g), true)) return SLRA_ERR_CUDA;
 
     if ((s = begin(p, d, w, st)) != SLRA_OK) return s;
     const bool overlap = branches == SLRA_BRANCH_BOTH && !(p->debug_flags & SLRA_DEBUG_SERIAL_BRANCHES);
@@ -682,7 +687,8 @@ slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, con
     a.status = w.status;
     a.timeout_ns = timeout_of(p);
     a.debug_unsatisfied_wait = debug_wait_of(p);
-    a.lse = nullptr;
+    a.lse = lse;
+    a.os_save = os;
     if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
     return mark(p, 6, st);
 }
@@ -998,9 +1004,12 @@ size_t slra_bwd_workspace_bytes(const slra_problem* p) {
     return check_bwd_problem(p, &d) == SLRA_OK ? bwd_layout(d).total : 0;
 }
 
-slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
-                          const float* dout, float* dq, float* dk, float* dv, float* dA, void* workspace,
-                          size_t workspace_bytes, slra_stream_t stream) {
+namespace {
+// The backward pass.  saved: the workspace holds the state slra_attn_fwd_train left for this problem
+// and these inputs (tables, selection, summary, fp16 copies, lse, O_s), so nothing is recomputed.
+slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
+                     const float* dout, float* dq, float* dk, float* dv, float* dA, void* workspace,
+                     size_t workspace_bytes, slra_stream_t stream, bool saved) {
     Derived d;
     slra_status s = check_bwd_problem(p, &d);
     if (s != SLRA_OK) return s;
@@ -1041,21 +1050,23 @@ slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, c
     for (auto& e : pr.stage_events) e = nullptr;
 
     if ((s = mark(p, 0, st)) != SLRA_OK) return s;
-    if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return SLRA_ERR_CUDA;
-    if ((s = cuda_status(launch_rope_table(w.tab, w.pairs, d.meta, d.table_entries, st))) != SLRA_OK) return s;
-    if (sparse && (s = run_select(&pr, d, w, q, k, v, st)) != SLRA_OK) return s;
-    if (lowrank && (s = run_lowrank(&pr, d, w, k, v, A, st)) != SLRA_OK) return s;
-    if (sparse) {
+    // the saved forward's status word keeps whatever it recorded; a recompute starts a fresh one
+    if (!saved && cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return SLRA_ERR_CUDA;
+    if (!saved && (s = cuda_status(launch_rope_table(w.tab, w.pairs, d.meta, d.table_entries, st))) != SLRA_OK)
+        return s;
+    if (!saved && sparse && (s = run_select(&pr, d, w, q, k, v, st)) != SLRA_OK) return s;
+    if (!saved && lowrank && (s = run_lowrank(&pr, d, w, k, v, A, st)) != SLRA_OK) return s;
+    if (!saved && sparse) {
         // the sparse forward again, writing its output O_s (head-major fp32) and each row's lse
         AttnMaps maps;
         const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
-        const Strides os_st{static_cast<long long>(g.Hh) * g.Lp * g.D, g.D, static_cast<long long>(g.Lp) * g.D};
         if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) ||
             !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
             !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
             !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, g.sq, 128) ||
-            !make_map_out(&maps.out, os, g.B, g.L, g.Hh, g.D, os_st, true))
+            !make_map_out(&maps.out, os, g.B, g.L, g.Hh, g.D, headmajor_strides(g), true))
             return SLRA_ERR_CUDA;
+        std::memset(&maps.os, 0, sizeof maps.os);
         AttnArgs a;
         std::memset(&a, 0, sizeof a);
         a.qh = w.qh;
@@ -1071,6 +1082,7 @@ slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, c
         a.status = w.status;
         a.timeout_ns = timeout_of(p);
         a.lse = lse;
+        a.os_save = nullptr;
         if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
     }
     if ((s = mark(p, 1, st)) != SLRA_OK) return s;
@@ -1140,6 +1152,37 @@ slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, c
     }
     if ((s = mark(p, 5, st)) != SLRA_OK) return s;
     return mark(p, 6, st);
+}
+}  // namespace
+
+slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
+                          const float* dout, float* dq, float* dk, float* dv, float* dA, void* workspace,
+                          size_t workspace_bytes, slra_stream_t stream) {
+    return bwd_impl(p, q, k, v, A, dout, dq, dk, dv, dA, workspace, workspace_bytes, stream, false);
+}
+
+slra_status slra_attn_bwd_saved(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
+                                const float* dout, float* dq, float* dk, float* dv, float* dA, void* workspace,
+                                size_t workspace_bytes, slra_stream_t stream) {
+    return bwd_impl(p, q, k, v, A, dout, dq, dk, dv, dA, workspace, workspace_bytes, stream, true);
+}
+
+slra_status slra_attn_fwd_train(const slra_problem* p, const void* q, const void* k, const void* v, const void* A,
+                                void* out, void* workspace, size_t workspace_bytes, slra_stream_t stream) {
+    Derived d;
+    slra_status s = check_bwd_problem(p, &d);
+    if (s != SLRA_OK) return s;
+    if ((s = check_fwd_args(p, d, q, k, v, A, out, workspace, workspace_bytes)) != SLRA_OK) return s;
+    const BwdLayout bl = bwd_layout(d);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < bl.total)
+        return SLRA_ERR_WORKSPACE;
+    if ((s = check_device()) != SLRA_OK) return s;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    const int branches = p->branches == 0 ? SLRA_BRANCH_BOTH : p->branches;
+    const bool sparse = (branches & SLRA_BRANCH_SPARSE) != 0;
+    return fwd_impl(p, d, q, k, v, A, out, workspace, reinterpret_cast<cudaStream_t>(stream),
+                    sparse ? reinterpret_cast<float*>(base + bl.lse) : nullptr,
+                    sparse ? reinterpret_cast<float*>(base + bl.os) : nullptr);
 }
 
 slra_status slra_get_device_status(slra_stream_t stream, int32_t* status) {

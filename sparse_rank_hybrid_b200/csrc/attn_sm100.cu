@@ -136,7 +136,8 @@ template <int D, int BLK, bool kDefault>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qraw,
-                      const __grid_constant__ CUtensorMap tm_out, AttnArgs a, Geom g) {
+                      const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_os,
+                      AttnArgs a, Geom g) {
     using Lay = AttnLayout<D>;
     const int act = kDefault ? 0 : g.act;        // low-rank feature map
     const int norope = kDefault ? 0 : g.norope;  // 1: no rotation in the low-rank branch
@@ -492,6 +493,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     // path through the group barriers is taken from one reduction.
     const bool aborted = group_sync_or(*abort_flag != 0);  // also: the exchange buffer is reused below
     tc_fence_after();
+
+    // Kept for a backward pass: the sparse branch's own output O_s = O / l, read before the low-rank
+    // readout joins O.  It is staged in the v slots (free once the last P.V has completed; the readout
+    // uses the q tile and the k slots) as fp32 boxes of 32 columns and stored head-major; the stores'
+    // reads of the staging are waited for with the output's, or in the teardown.
+    bool os_committed = false;
+    if (a.os_save != nullptr && keep > 0 && !aborted) {
+        const float inv_l_s = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {
+            const int c = hf * (D / 64) + cc;  // 32-column group of O
+            uint32_t o[32];
+            tmem_ld32(tO + lane_base + c * 32, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t off = Lay::kOffV + c * 16384 + i_row * 128 + ((u ^ (i_row & 7)) << 4);
+                *reinterpret_cast<float4*>(smem + off) =
+                    make_float4(__uint_as_float(o[4 * u]) * inv_l_s, __uint_as_float(o[4 * u + 1]) * inv_l_s,
+                                __uint_as_float(o[4 * u + 2]) * inv_l_s, __uint_as_float(o[4 * u + 3]) * inv_l_s);
+            }
+        }
+        fence_async_smem();
+        group_sync();
+        if (tid == 0) {
+            for (int bx = 0; bx < D / 32; ++bx)
+                for (int rh = 0; rh * 64 < blk; ++rh) {
+                    if (alpha * blk + rh * 64 >= g.L) break;
+                    tma_store_4d(&tm_os, smem + Lay::kOffV + bx * 16384 + rh * 64 * 128, bx * 32, h,
+                                 alpha * blk + rh * 64, b);
+                }
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            os_committed = true;
+        }
+    }
 
     // ------------------------------------------------------------------ epilogue
     const int n = alpha * blk + i_row;
@@ -922,6 +958,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     // ------------------------------------------------------------------ teardown (softmax warps)
+    if (os_committed && aborted2) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     if (*abort_flag && tid == 0) {
         // Let the epilogue's copies and products still in flight land before the memory is released.
         // Each wait is bounded (10 ms) and ignores the abort flag.
@@ -953,7 +990,7 @@ cudaError_t launch_attn_v(const AttnMaps& m, const AttnArgs& a, const Geom& g, c
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
     if (e != cudaSuccess) return e;
     attn_sm100_kernel<D, BLK, kDefault><<<dim3(g.nb, g.BH()), kThreads, sm, st>>>(m.q, m.k, m.v, m.q_raw, m.out,
-                                                                                    a, g);
+                                                                                    m.os, a, g);
     return cudaGetLastError();
 }
 template <int D, int BLK>

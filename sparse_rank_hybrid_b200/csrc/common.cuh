@@ -32,6 +32,11 @@ struct Geom {
     __host__ __device__ int BH() const { return B * Hh; }
 };
 
+// Strides of a head-major [B][Hh][Lp][D] buffer addressed as [B][L][Hh][D] rows.
+inline Strides headmajor_strides(const Geom& g) {
+    return Strides{static_cast<long long>(g.Hh) * g.Lp * g.D, g.D, static_cast<long long>(g.Lp) * g.D};
+}
+
 // phi = act(u) for the low-rank feature map: relu (0), SiLU u / (1 + e^-u) (1), identity (2), tanh (3).
 // relu stays inline; the other maps go through one out-of-line function, so the fully unrolled feature
 // loops do not carry inlined copies of expf / tanhf (the choice is uniform over a launch).
@@ -91,6 +96,7 @@ struct AttnMaps {
     CUtensorMap q, k, v;
     CUtensorMap q_raw;  // 4D map over the raw bf16 queries [B][L][Hh][D], box 64 x 1 x 128 x 1
     CUtensorMap out;    // 4D map over out [B][L][Hh][D] (fp32: box 32 x 1 x 64 x 1; bf16: 64 x 1 x 64 x 1)
+    CUtensorMap os;     // with AttnArgs::os_save: fp32 map over the saved sparse output (head-major)
 };
 
 // Operand images for the tensor-core low-rank readout (head_dim 128), built by the reduction:
@@ -125,6 +131,8 @@ struct AttnArgs {
     int debug_unsatisfied_wait;  // test hook: wait on a barrier nothing signals before any work
     float* lse;  // optional fp32 [B*Hh][Lp]: per query row m + log2(l) of the sparse softmax in the kernel's
                  // log2 units (P_ij = 2^(s_ij log2(e) / sqrt(D) - lse_i)); +inf for rows past L
+    float* os_save;  // optional: the sparse branch's own output O_s = O / l, stored through AttnMaps::os
+                     // before the low-rank readout joins O (for a backward pass)
 };
 cudaError_t launch_attn(const AttnMaps& m, const AttnArgs& a, const Geom& g, cudaStream_t st);
 size_t attn_smem_bytes(const Geom& g);

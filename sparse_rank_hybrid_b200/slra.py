@@ -20,7 +20,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DE
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
 DEBUG_UNSATISFIED_WAIT, DEBUG_SERIAL_BRANCHES = 1, 2
-ABI_VERSION = 6
+ABI_VERSION = 7
 DTYPE_BF16, DTYPE_F32 = 0, 1
 ACT_RELU, ACT_SILU, ACT_IDENTITY, ACT_TANH = 0, 1, 2, 3
 FUSION_SUM, FUSION_GATED = 0, 1
@@ -32,7 +32,7 @@ EXPORTS = ("slra_abi_version", "slra_status_string", "slra_problem_init", "slra_
            "slra_workspace_layout", "slra_host_io_bytes", "slra_host_pipeline_groups",
            "slra_attn_fwd_host",
            "slra_select_blocks", "slra_lowrank_summary", "slra_device_status", "slra_lowrank_summary_noalloc",
-           "slra_noalloc_device_status")
+           "slra_noalloc_device_status", "slra_attn_fwd_train", "slra_attn_bwd_saved")
 
 
 class SlraError(RuntimeError):
@@ -109,6 +109,8 @@ def lib():
         L.slra_bwd_workspace_bytes.restype = S
         L.slra_bwd_workspace_bytes.argtypes = [PP]
         L.slra_attn_bwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, S, P]
+        L.slra_attn_bwd_saved.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, S, P]
+        L.slra_attn_fwd_train.argtypes = [PP, P, P, P, P, P, P, S, P]
         L.slra_host_io_bytes.restype = S
         L.slra_host_io_bytes.argtypes = [PP]
         L.slra_host_pipeline_groups.restype = ctypes.c_int64
@@ -121,7 +123,7 @@ def lib():
         L.slra_noalloc_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
         for name in ("slra_problem_init", "slra_validate", "slra_workspace_layout", "slra_attn_fwd",
                      "slra_attn_fwd_ex", "slra_sparse_fwd", "slra_lowrank_fwd", "slra_get_device_status",
-                     "slra_attn_bwd",
+                     "slra_attn_bwd", "slra_attn_bwd_saved", "slra_attn_fwd_train",
                      "slra_attn_fwd_host", "slra_select_blocks", "slra_lowrank_summary", "slra_device_status",
                      "slra_lowrank_summary_noalloc", "slra_noalloc_device_status"):
             getattr(L, name).restype = ctypes.c_int
@@ -361,7 +363,36 @@ def bwd_workspace_bytes(prob: Problem) -> int:
     return int(lib().slra_bwd_workspace_bytes(ctypes.byref(prob.c())))
 
 
-def attn_bwd(prob: Problem, q, k, v, A, dout, grads=None, workspace=None, stream=None):
+def attn_fwd_train(prob: Problem, q, k, v, A, out=None, workspace=None, stream=None):
+    """Forward pass for training (slra_attn_fwd_train): out as attn_fwd gives it, and the workspace
+    (backward-sized, allocated when None) keeps what attn_bwd_saved needs.  Returns (out, workspace)."""
+    import dataclasses
+    torch = _torch()
+    shp = (prob.batch, prob.L, prob.heads, prob.head_dim)
+    strides = {f"{n}_strides": _row_strides(n, t, shp, torch.bfloat16) for n, t in (("q", q), ("k", k), ("v", v))}
+    p = dataclasses.replace(prob, **strides)
+    if A is not None:
+        _check_bf16("A", A, prob.projection_shape)
+    if out is None:
+        out = torch.empty(shp, dtype=torch.float32 if prob.out_dtype == OUT_F32 else torch.bfloat16, device=q.device)
+    if workspace is None:
+        n = bwd_workspace_bytes(p)
+        if n == 0:
+            raise SlraError(ERR_UNSUPPORTED, "slra_bwd_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    _check(lib().slra_attn_fwd_train(ctypes.byref(p.c()), _ptr(q), _ptr(k), _ptr(v), None if A is None else _ptr(A),
+                                     _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream)),
+           "slra_attn_fwd_train")
+    return out, workspace
+
+
+def attn_bwd_saved(prob: Problem, q, k, v, A, dout, workspace, grads=None, stream=None):
+    """Backward pass from attn_fwd_train's workspace (slra_attn_bwd_saved): as attn_bwd, without the
+    recompute.  Returns (dq, dk, dv, dA, workspace)."""
+    return attn_bwd(prob, q, k, v, A, dout, grads=grads, workspace=workspace, stream=stream, _saved=True)
+
+
+def attn_bwd(prob: Problem, q, k, v, A, dout, grads=None, workspace=None, stream=None, _saved=False):
     """Backward pass (slra_attn_bwd): gradients of sum(dout * out) for q, k, v (fp32 [B, L, Hh, D]) and A
     (fp32 [D, rank]).  dout: contiguous CUDA fp32 [B, L, Hh, D].  q, k, v may be strided views.
     Returns (dq, dk, dv, dA, workspace)."""
@@ -383,9 +414,10 @@ def attn_bwd(prob: Problem, q, k, v, A, dout, grads=None, workspace=None, stream
         if n == 0:
             raise SlraError(ERR_UNSUPPORTED, "slra_bwd_workspace_bytes")
         workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
-    _check(lib().slra_attn_bwd(ctypes.byref(p.c()), _ptr(q), _ptr(k), _ptr(v), None if A is None else _ptr(A),
-                               _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dA), _ptr(workspace),
-                               workspace.numel(), _stream_handle(stream)), "slra_attn_bwd")
+    fn = "slra_attn_bwd_saved" if _saved else "slra_attn_bwd"
+    _check(getattr(lib(), fn)(ctypes.byref(p.c()), _ptr(q), _ptr(k), _ptr(v), None if A is None else _ptr(A),
+                              _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dA), _ptr(workspace),
+                              workspace.numel(), _stream_handle(stream)), fn)
     return dq, dk, dv, dA, workspace
 
 

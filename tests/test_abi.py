@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_abi_version_and_status_strings():
-    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 6
+    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 7
     for s in range(0, 9):
         assert slra.status_string(s) and slra.status_string(s) != "unknown status"
     assert slra.status_string(99) == "unknown status"
@@ -218,3 +218,40 @@ def test_host_entry_point_rejects_strides():
     s = slra.lib().slra_attn_fwd_host(ctypes.byref(p.c()), base, base, base, base, base, base, 1 << 19, base,
                                       1 << 19, None)
     assert s == slra.ERR_INVALID_ARG
+
+
+def test_train_forward_and_saved_backward_validation():
+    """slra_attn_fwd_train wants a backward-sized workspace and the backward's options; both new entry
+    points check their arguments before looking for a device."""
+    import ctypes
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("has a GPU")
+    p = slra.Problem.from_workload(W.TINY)
+    n = W.TINY.batch * W.TINY.L * W.TINY.heads * W.TINY.head_dim
+    bufs = [ctypes.create_string_buffer(n * 4 + 256) for _ in range(9)]
+    q, k, v, A, out, dout, dq, dk, dv = [(ctypes.addressof(b) + 255) // 256 * 256 for b in bufs]
+    dA_buf = ctypes.create_string_buffer(64 * 16 * 4 + 256)
+    dA = (ctypes.addressof(dA_buf) + 255) // 256 * 256
+    fwd_b = slra.layout(p).total_bytes
+    bwd_b = slra.bwd_workspace_bytes(p)
+    assert bwd_b > fwd_b
+    ws_buf = ctypes.create_string_buffer(bwd_b + 256)
+    ws = (ctypes.addressof(ws_buf) + 255) // 256 * 256
+    L = slra.lib()
+    pc = p.c()
+    # a forward-sized workspace is too small for the kept state; NULL is not allowed
+    assert L.slra_attn_fwd_train(ctypes.byref(pc), q, k, v, A, out, ws, fwd_b, None) == slra.ERR_WORKSPACE
+    assert L.slra_attn_fwd_train(ctypes.byref(pc), q, k, v, A, out, None, 0, None) == slra.ERR_WORKSPACE
+    assert L.slra_attn_fwd_train(ctypes.byref(pc), q, k, v, A, out, ws + 16, bwd_b, None) == slra.ERR_WORKSPACE
+    assert L.slra_attn_fwd_train(ctypes.byref(pc), q, k, v, A, out, ws, bwd_b, None) == slra.ERR_NO_DEVICE
+    # options the backward does not cover are refused by the training forward too
+    ps = slra.Problem.from_workload(W.TINY)
+    ps.activation = slra.ACT_SILU
+    assert L.slra_attn_fwd_train(ctypes.byref(ps.c()), q, k, v, A, out, ws, bwd_b, None) == slra.ERR_UNSUPPORTED
+    # the saved backward: same checks as slra_attn_bwd
+    args = (q, k, v, A, dout, dq, dk, dv, dA)
+    assert L.slra_attn_bwd_saved(ctypes.byref(pc), *args, ws, bwd_b - 256, None) == slra.ERR_WORKSPACE
+    assert L.slra_attn_bwd_saved(ctypes.byref(pc), *args, ws, bwd_b, None) == slra.ERR_NO_DEVICE
+    assert L.slra_attn_bwd_saved(ctypes.byref(pc), q, k, v, A, dout, dq, dq, dv, dA, ws, bwd_b,
+                                 None) == slra.ERR_INVALID_ARG

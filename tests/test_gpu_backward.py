@@ -182,3 +182,34 @@ def test_backward_wan_1_3b_sampled():
     ref_s = [np.concatenate([smp["dq"][a] for a in qbs]), np.concatenate([smp["dk"][b] for b in kbs]),
              np.concatenate([smp["dv"][b] for b in kbs]), dA_ref]
     _compare("wan1.3b-sampled", got_s, ref_s)
+
+
+def _saved_vs_recompute(w, branches=slra.BRANCH_BOTH):
+    """slra_attn_fwd_train gives slra_attn_fwd_ex's output bit for bit, and slra_attn_bwd_saved on its
+    workspace gives slra_attn_bwd's gradients bit for bit (the saved O_s and lse are the ones the
+    recompute writes: same kernel, same arithmetic)."""
+    import torch
+    x = I.make_inputs(w)
+    dout = torch.from_numpy(I.make_dout(w.seed + 9100, w.batch, w.L, w.heads, w.head_dim)).cuda()
+    p = slra.Problem.from_workload(w, branches=branches)
+    q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
+    out_ref, ws_f = slra.attn_fwd(p, q, k, v, A)
+    assert slra.device_status(ws_f) == slra.OK
+    out_t, ws = slra.attn_fwd_train(p, q, k, v, A)
+    assert slra.device_status(ws) == slra.OK
+    assert torch.equal(out_t, out_ref)
+    ref = slra.attn_bwd(p, q, k, v, A, dout)[:4]
+    got = slra.attn_bwd_saved(p, q, k, v, A, dout, ws)[:4]
+    assert slra.device_status(ws) == slra.OK
+    for name, a, b in zip(("dq", "dk", "dv", "dA"), got, ref):
+        assert torch.equal(a, b), f"{w.name}: {name} differs from the recomputing backward"
+
+
+@pytest.mark.parametrize("w", [W.TINY, EDGE_128, EDGE_128_B64, EDGE_B2, W.WAN_1_3B], ids=lambda w: w.name)
+def test_saved_forward_backward_equals_recompute(w):
+    _saved_vs_recompute(w)
+
+
+@pytest.mark.parametrize("branches", [slra.BRANCH_SPARSE, slra.BRANCH_LOWRANK])
+def test_saved_forward_backward_single_branch(branches):
+    _saved_vs_recompute(EDGE_128, branches)
