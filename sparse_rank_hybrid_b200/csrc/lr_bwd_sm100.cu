@@ -131,6 +131,7 @@ __device__ __forceinline__ void build_dk_image(uint8_t* hi_img, uint8_t* lo_img,
 template <int R, bool kKey>
 __global__ void __launch_bounds__(256, 1)
     lr_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
+                        const __grid_constant__ CUtensorMap tm_o0, const __grid_constant__ CUtensorMap tm_o1,
                         LrTcBwdArgs a, Geom g) {
     using Lay = LbLayout<R>;
     constexpr int RH = R / 2;  // features per thread
@@ -420,19 +421,6 @@ __global__ void __launch_bounds__(256, 1)
                 umma_commit(bar_m2);
                 ++n_m2_issued;
             }
-            // The values the first output is added to, loaded while the products run (all 16 loads in
-            // flight at once); the key pass loads dk's after storing dv.
-            auto out_row = [&](int which) {
-                return (kKey ? (which ? a.dk : a.dv) : a.dq) + g.so.row(b, live ? n : 0, h) + half * 64;
-            };
-            float4 prev[16];
-            auto load_prev = [&](const float* rowp) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    prev[i] = (a.accumulate && live) ? *reinterpret_cast<const float4*>(rowp + 4 * i)
-                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-            };
-            load_prev(out_row(0));
             ok = mbar_wait(bar_m2, n_m2 & 1, tmo, abort_flag);
             if (__syncthreads_or(!ok)) {
                 if (tid == 0) fail();
@@ -441,28 +429,44 @@ __global__ void __launch_bounds__(256, 1)
             }
             ++n_m2;
             tc_fence_after();
-            // ---- outputs of the tile: this thread's 64 columns of the row (query pass: dq; key: dv, dk).
-            // The TMEM loads are warp-collective, so every lane takes them; rows past L store nothing.
+            // ---- outputs of the tile: this thread's 64 columns of the row (query pass: dq; key: dv, dk),
+            // staged as fp32 boxes of 32 columns (128-B swizzled, the output map's layout) in tile buffers
+            // the products are done with (dq, dv: w and du; dk: the k and v tiles), then stored by the
+            // TMA engine, or with `accumulate` added to the rows in memory (one add per element, in L2).
+            // The TMEM loads are warp-collective, so every lane takes them; the maps clip rows past L.
 #pragma unroll
             for (int which = 0; which < (kKey ? 2 : 1); ++which) {
                 const uint32_t src = kKey ? (which ? tK : tV) : tO;
-                float* dst = out_row(which);
-                if (which == 1) load_prev(dst);
+                uint8_t* stg = smem + (which ? Lay::kOffX : Lay::kOffW);
 #pragma unroll
                 for (int c0 = 0; c0 < 64; c0 += 32) {
                     uint32_t r[32];
                     tmem_ld32(src + lane_base + half * 64 + c0, r);
                     tmem_ld_wait(r);
-                    if (live) {
+                    uint8_t* box = stg + (half * 2 + c0 / 32) * 16384 + row * 128;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4) {
-                            const float4 p = prev[(c0 + i) / 4];
-                            const float4 v = make_float4(__uint_as_float(r[i]) + p.x, __uint_as_float(r[i + 1]) + p.y,
-                                                         __uint_as_float(r[i + 2]) + p.z, __uint_as_float(r[i + 3]) + p.w);
-                            *reinterpret_cast<float4*>(dst + c0 + i) = v;
-                        }
-                    }
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<float4*>(box + ((u ^ (row & 7)) << 4)) =
+                            make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                                        __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
                 }
+            }
+            fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+#pragma unroll
+                for (int which = 0; which < (kKey ? 2 : 1); ++which) {
+                    const CUtensorMap* map = which ? &tm_o1 : &tm_o0;
+                    const uint8_t* stg = smem + (which ? Lay::kOffX : Lay::kOffW);
+                    for (int bx = 0; bx < 4; ++bx)
+                        for (int rh = 0; rh < 2; ++rh) {
+                            const int n0 = tile * kTok + rh * 64;
+                            if (n0 >= g.L) break;
+                            if (a.accumulate) tma_reduce_add_4d(map, stg + bx * 16384 + rh * 8192, bx * 32, h, n0, b);
+                            else tma_store_4d(map, stg + bx * 16384 + rh * 8192, bx * 32, h, n0, b);
+                        }
+                }
+                tma_store_commit_and_wait();  // the next tile's loads and operands reuse the staging
             }
             tc_fence_before();
             __syncthreads();  // the next tile overwrites the staged operands and the token-row TMEM
@@ -534,7 +538,8 @@ __global__ void __launch_bounds__(256, 1)
 namespace {
 template <int R>
 cudaError_t launch_lr_bwd_tc_r(const LrTcBwdArgs& a, const Geom& g, const CUtensorMap& tq, const CUtensorMap& tk,
-                               const CUtensorMap& tv, float* dS, float* dz, cudaStream_t st) {
+                               const CUtensorMap& tv, const CUtensorMap& tdq, const CUtensorMap& tdk,
+                               const CUtensorMap& tdv, float* dS, float* dz, cudaStream_t st) {
     const size_t sm = static_cast<size_t>(LbLayout<R>::kBytes) + 1024;
     cudaError_t e = cudaFuncSetAttribute(lr_bwd_sm100_kernel<R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
@@ -545,7 +550,7 @@ cudaError_t launch_lr_bwd_tc_r(const LrTcBwdArgs& a, const Geom& g, const CUtens
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int items = g.BH() * a.nsplit;
     const int grid = items < sms ? items : sms;
-    lr_bwd_sm100_kernel<R, false><<<grid, 256, sm, st>>>(tq, tq, a, g);
+    lr_bwd_sm100_kernel<R, false><<<grid, 256, sm, st>>>(tq, tq, tdq, tdq, a, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_lowrank_reduce(a.ds_part, a.dz_part, g, a.nsplit, dS, dz, nullptr, nullptr, nullptr, st)) !=
         cudaSuccess)
@@ -554,7 +559,7 @@ cudaError_t launch_lr_bwd_tc_r(const LrTcBwdArgs& a, const Geom& g, const CUtens
     ak.dS = dS;
     ak.dz = dz;
     ak.da_part = a.da_part + static_cast<size_t>(g.BH()) * a.nsplit * kD * R;
-    lr_bwd_sm100_kernel<R, true><<<grid, 256, sm, st>>>(tk, tv, ak, g);
+    lr_bwd_sm100_kernel<R, true><<<grid, 256, sm, st>>>(tk, tv, tdv, tdk, ak, g);
     return cudaGetLastError();
 }
 }  // namespace
@@ -563,10 +568,13 @@ cudaError_t launch_lr_bwd_tc_r(const LrTcBwdArgs& a, const Geom& g, const CUtens
 // pass.  The dA partials of both passes are left for the caller's fixed-order reduction.
 cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st) {
     const RopeMeta& meta = *l.meta;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tdq, tdk, tdv;
     if (!make_map_tokens(&tq, l.q, g.B, g.L, g.Hh, g.D, g.sq, kTok) ||
         !make_map_tokens(&tk, l.k, g.B, g.L, g.Hh, g.D, g.sk, kTok) ||
-        !make_map_tokens(&tv, l.v, g.B, g.L, g.Hh, g.D, g.sv, kTok))
+        !make_map_tokens(&tv, l.v, g.B, g.L, g.Hh, g.D, g.sv, kTok) ||
+        !make_map_out(&tdq, l.dq, g.B, g.L, g.Hh, g.D, g.so, true) ||
+        !make_map_out(&tdk, l.dk, g.B, g.L, g.Hh, g.D, g.so, true) ||
+        !make_map_out(&tdv, l.dv, g.B, g.L, g.Hh, g.D, g.so, true))
         return cudaErrorInvalidValue;
     LrTcBwdArgs a;
     a.dout = l.dout;
@@ -590,9 +598,9 @@ cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st)
     a.timeout_ns = l.timeout_ns;
     a.accumulate = l.accumulate;
     switch (g.R) {
-        case 16: return launch_lr_bwd_tc_r<16>(a, g, tq, tk, tv, l.dS, l.dz, st);
-        case 32: return launch_lr_bwd_tc_r<32>(a, g, tq, tk, tv, l.dS, l.dz, st);
-        case 48: return launch_lr_bwd_tc_r<48>(a, g, tq, tk, tv, l.dS, l.dz, st);
+        case 16: return launch_lr_bwd_tc_r<16>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, st);
+        case 32: return launch_lr_bwd_tc_r<32>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, st);
+        case 48: return launch_lr_bwd_tc_r<48>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, st);
     }
     return cudaErrorInvalidValue;
 }
