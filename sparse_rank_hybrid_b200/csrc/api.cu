@@ -726,14 +726,12 @@ BwdLayout bwd_layout(const Derived& d) {
     return b;
 }
 
-// The backward covers the default options: relu features, the low-rank RoPE outside the activation,
-// one shared projection and the plain sum; gradients are contiguous fp32 [B][L][Hh][D].
+// The backward covers every feature map, RoPE ordering and projection layout with the plain sum of the
+// branches (not the gated fusion); gradients are contiguous fp32 [B][L][Hh][D].
 slra_status check_bwd_problem(const slra_problem* p, Derived* d) {
     slra_status s = derive(p, d);
     if (s != SLRA_OK) return s;
-    if (p->activation != SLRA_ACT_RELU || p->lowrank_norope || p->lowrank_rope_inside || p->proj_separate ||
-        p->proj_per_head || p->fusion != SLRA_FUSION_SUM)
-        return SLRA_ERR_UNSUPPORTED;
+    if (p->fusion != SLRA_FUSION_SUM) return SLRA_ERR_UNSUPPORTED;
     for (int i = 0; i < 3; ++i)
         if (p->out_strides[i]) return SLRA_ERR_INVALID_ARG;
     return SLRA_OK;
@@ -1021,7 +1019,7 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
         return SLRA_ERR_ALIGNMENT;
     const Geom& g = d.g;
     const BwdLayout bl = bwd_layout(d);
-    const size_t gb = qkv_bytes(d) * 2, ab = static_cast<size_t>(g.D) * g.R * 4;  // fp32 gradient bytes
+    const size_t gb = qkv_bytes(d) * 2, ab = d.a_elems * 4;  // fp32 gradient bytes
     const void* outs[4] = {dq, dk, dv, dA};
     const size_t out_n[4] = {gb, gb, gb, ab};
     const void* ins[5] = {q, k, v, A, dout};
@@ -1127,6 +1125,8 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
         l.k = static_cast<const __nv_bfloat16*>(k);
         l.v = static_cast<const __nv_bfloat16*>(v);
         l.A = static_cast<const __nv_bfloat16*>(A);
+        l.proj_separate = p->proj_separate ? 1 : 0;
+        l.proj_per_head = p->proj_per_head ? 1 : 0;
         l.dout = dout;
         l.S = w.S;
         l.z = w.z;

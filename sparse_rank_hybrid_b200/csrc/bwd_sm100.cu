@@ -707,8 +707,9 @@ struct LrTile {
     static constexpr int T = R <= 64 ? 32 : 16;
 };
 
-// Pass over the queries: per token u = q A, phi, psi, den, G = S dO; dpsi, dden, dphi, du; split-L
-// partial sums of dS = sum psi dO^T / den, dz = sum dden phi and dA_q = q^T du; dq += du A^T.
+// Pass over the queries: per token u = q A, psi and the normaliser feature nf (lr_pair_fwd), den = nf . z,
+// G = S dO; dpsi = G / den, dden, du (lr_pair_bwd); split-L partial sums of dS = sum psi dO^T / den,
+// dz = sum dden nf and dA_q = q^T du; dq += du A^T.  A: this pass's projection (head h at h * a_stride).
 template <int D, int R>
 __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __restrict__ q,
                                                        const float* __restrict__ dout,
@@ -743,9 +744,22 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
     const int ntiles = (g.L + TT - 1) / TT;
     const int per = (ntiles + nsplit - 1) / nsplit;
     const int t0 = split * per, t1 = min(ntiles, t0 + per);
-    for (int e = tid; e < D * R; e += 256) As[(e / R) * (R + 1) + e % R] = __bfloat162float(A[e]);
+    const __nv_bfloat16* Ah = A + static_cast<size_t>(h) * g.a_stride;
+    for (int e = tid; e < D * R; e += 256) As[(e / R) * (R + 1) + e % R] = __bfloat162float(Ah[e]);
     for (int e = tid; e < R * D; e += 256) Ss[(e / D) * (D + 1) + e % D] = S[static_cast<size_t>(bh) * R * D + e];
     if (tid < R) zs[tid] = z[static_cast<size_t>(bh) * R + tid];
+    // (cos, sin) of pair p at token n; no rotation without the low-rank RoPE
+    auto rot = [&](int p, int n, float& cf, float& sf) {
+        if (g.norope) {
+            cf = 1.f;
+            sf = 0.f;
+            return;
+        }
+        const int2 pi = pairs[p];
+        const double2 cs = tab[pi.y + token_axis_pos(n, pi.x, g.H, g.W)];
+        cf = static_cast<float>(cs.x);
+        sf = static_cast<float>(cs.y);
+    };
     const int e_own = tid % D, cg = tid / D;
     float acc_s[NA], acc_a[NA];  // dS[c][e_own], dA[e_own][c] for c = cg + G i
 #pragma unroll
@@ -779,10 +793,9 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
             }
             us[tt * (R + 1) + c] = u;
             Gs[tt * (R + 1) + c] = gg;
-            phs[tt * R + c] = fmaxf(u, 0.f);
         }
         __syncthreads();
-        // per token: den = phi . z + 1e-6, dden = -(psi . G) / den^2 (one warp per token)
+        // per token: den = nf . z + 1e-6, dden = -(psi . G) / den^2 (one warp per token); nf kept for dz
         {
             const int warp = tid >> 5, lane = tid & 31;
             for (int tt = warp; tt < TT; tt += 8) {
@@ -790,13 +803,14 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
                 const int nt = n < g.L ? n : 0;
                 float dz_ = 0.f, dot = 0.f;
                 for (int p = lane; p < R / 2; p += 32) {
-                    const float x0 = phs[tt * R + 2 * p], x1 = phs[tt * R + 2 * p + 1];
-                    const int2 pi = pairs[p];
-                    const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
-                    const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
-                    const float y0 = x0 * cf - x1 * sf, y1 = x0 * sf + x1 * cf;
-                    dz_ = fmaf(x0, zs[2 * p], fmaf(x1, zs[2 * p + 1], dz_));
-                    dot = fmaf(y0, Gs[tt * (R + 1) + 2 * p], fmaf(y1, Gs[tt * (R + 1) + 2 * p + 1], dot));
+                    float cf, sf;
+                    rot(p, nt, cf, sf);
+                    const LrPair P = lr_pair_fwd(us[tt * (R + 1) + 2 * p], us[tt * (R + 1) + 2 * p + 1], cf, sf,
+                                                 g.act, g.inside);
+                    phs[tt * R + 2 * p] = P.nf0;
+                    phs[tt * R + 2 * p + 1] = P.nf1;
+                    dz_ = fmaf(P.nf0, zs[2 * p], fmaf(P.nf1, zs[2 * p + 1], dz_));
+                    dot = fmaf(P.psi0, Gs[tt * (R + 1) + 2 * p], fmaf(P.psi1, Gs[tt * (R + 1) + 2 * p + 1], dot));
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
@@ -811,25 +825,24 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
             }
         }
         __syncthreads();
-        // per (token, pair): psi / den, dphi = R^T (G / den) + dden z, du = dphi [u > 0]
+        // per (token, pair): psi / den; du from dpsi = G / den and dnf = dden z
         for (int o = tid; o < TT * (R / 2); o += 256) {
             const int tt = o / (R / 2), p = o % (R / 2);
             const int n = n0 + tt;
             const int nt = n < g.L ? n : 0;
-            const int2 pi = pairs[p];
-            const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
-            const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
+            float cf, sf;
+            rot(p, nt, cf, sf);
             const float den = dens[tt], dd = ddens[tt];
-            const float x0 = phs[tt * R + 2 * p], x1 = phs[tt * R + 2 * p + 1];
-            const float y0 = x0 * cf - x1 * sf, y1 = x0 * sf + x1 * cf;
-            ws[tt * R + 2 * p] = n < g.L ? y0 / den : 0.f;
-            ws[tt * R + 2 * p + 1] = n < g.L ? y1 / den : 0.f;
+            const LrPair P = lr_pair_fwd(us[tt * (R + 1) + 2 * p], us[tt * (R + 1) + 2 * p + 1], cf, sf, g.act,
+                                         g.inside);
+            ws[tt * R + 2 * p] = n < g.L ? P.psi0 / den : 0.f;
+            ws[tt * R + 2 * p + 1] = n < g.L ? P.psi1 / den : 0.f;
             const float g0 = Gs[tt * (R + 1) + 2 * p] / den, g1 = Gs[tt * (R + 1) + 2 * p + 1] / den;
-            const float dph0 = cf * g0 + sf * g1 + dd * zs[2 * p];
-            const float dph1 = -sf * g0 + cf * g1 + dd * zs[2 * p + 1];
+            float du0, du1;
+            lr_pair_bwd(P, g0, g1, dd * zs[2 * p], dd * zs[2 * p + 1], cf, sf, g.inside, du0, du1);
             const bool live = n < g.L;
-            dus[tt * (R + 1) + 2 * p] = (live && us[tt * (R + 1) + 2 * p] > 0.f) ? dph0 : 0.f;
-            dus[tt * (R + 1) + 2 * p + 1] = (live && us[tt * (R + 1) + 2 * p + 1] > 0.f) ? dph1 : 0.f;
+            dus[tt * (R + 1) + 2 * p] = live ? du0 : 0.f;
+            dus[tt * (R + 1) + 2 * p + 1] = live ? du1 : 0.f;
         }
         __syncthreads();
         // partial sums: dS[c][e] += sum_t w[t][c] dO[t][e]; dA[d][c] += sum_t q[t][d] du[t][c]; dz
@@ -865,8 +878,8 @@ __global__ void __launch_bounds__(256) bwd_lr_q_kernel(const __nv_bfloat16* __re
     if (tid < R) dz_part[slot * R + tid] = acc_z;
 }
 
-// Pass over the keys: per token u = k A, phi, psi; dpsi = dS v; dv += dS^T psi; dphi = R^T dpsi + dz;
-// du; dk += du A^T; split-L partial sums of dA_k = k^T du.
+// Pass over the keys: per token u = k A, psi (lr_pair_fwd); dpsi = dS v; dv += dS^T psi; du from dpsi and
+// dnf = dz (lr_pair_bwd); dk += du A^T; split-L partial sums of dA_k = k^T du.  A: the key projection.
 template <int D, int R>
 __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __restrict__ k,
                                                        const __nv_bfloat16* __restrict__ v,
@@ -894,7 +907,8 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
     const int ntiles = (g.L + TT - 1) / TT;
     const int per = (ntiles + nsplit - 1) / nsplit;
     const int t0 = split * per, t1 = min(ntiles, t0 + per);
-    for (int e = tid; e < D * R; e += 256) As[(e / R) * (R + 1) + e % R] = __bfloat162float(A[e]);
+    const __nv_bfloat16* Ah = A + static_cast<size_t>(h) * g.a_stride;
+    for (int e = tid; e < D * R; e += 256) As[(e / R) * (R + 1) + e % R] = __bfloat162float(Ah[e]);
     for (int e = tid; e < R * D; e += 256) Ss[(e / D) * (D + 1) + e % D] = dS[static_cast<size_t>(bh) * R * D + e];
     if (tid < R) zs[tid] = dz[static_cast<size_t>(bh) * R + tid];
     const int e_own = tid % D, cg = tid / D;
@@ -931,24 +945,28 @@ __global__ void __launch_bounds__(256) bwd_lr_k_kernel(const __nv_bfloat16* __re
             ps[tt * (R + 1) + c] = dp;
         }
         __syncthreads();
-        // per (token, pair): psi = R phi; du = (R^T dpsi + dz) [u > 0] (written over dpsi)
+        // per (token, pair): psi; du from dpsi and dnf = dz (written over dpsi)
         for (int o = tid; o < TT * (R / 2); o += 256) {
             const int tt = o / (R / 2), p = o % (R / 2);
             const int n = n0 + tt;
             const int nt = n < g.L ? n : 0;
-            const int2 pi = pairs[p];
-            const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
-            const float cf = static_cast<float>(cs.x), sf = static_cast<float>(cs.y);
-            const float u0 = us[tt * (R + 1) + 2 * p], u1 = us[tt * (R + 1) + 2 * p + 1];
-            const float x0 = fmaxf(u0, 0.f), x1 = fmaxf(u1, 0.f);
-            psis[tt * (R + 1) + 2 * p] = x0 * cf - x1 * sf;
-            psis[tt * (R + 1) + 2 * p + 1] = x0 * sf + x1 * cf;
-            const float d0 = ps[tt * (R + 1) + 2 * p], d1 = ps[tt * (R + 1) + 2 * p + 1];
-            const float dph0 = cf * d0 + sf * d1 + zs[2 * p];
-            const float dph1 = -sf * d0 + cf * d1 + zs[2 * p + 1];
+            float cf = 1.f, sf = 0.f;
+            if (!g.norope) {
+                const int2 pi = pairs[p];
+                const double2 cs = tab[pi.y + token_axis_pos(nt, pi.x, g.H, g.W)];
+                cf = static_cast<float>(cs.x);
+                sf = static_cast<float>(cs.y);
+            }
+            const LrPair P = lr_pair_fwd(us[tt * (R + 1) + 2 * p], us[tt * (R + 1) + 2 * p + 1], cf, sf, g.act,
+                                         g.inside);
+            psis[tt * (R + 1) + 2 * p] = P.psi0;
+            psis[tt * (R + 1) + 2 * p + 1] = P.psi1;
+            float du0, du1;
+            lr_pair_bwd(P, ps[tt * (R + 1) + 2 * p], ps[tt * (R + 1) + 2 * p + 1], zs[2 * p], zs[2 * p + 1], cf, sf,
+                        g.inside, du0, du1);
             const bool live = n < g.L;
-            ps[tt * (R + 1) + 2 * p] = (live && u0 > 0.f) ? dph0 : 0.f;
-            ps[tt * (R + 1) + 2 * p + 1] = (live && u1 > 0.f) ? dph1 : 0.f;
+            ps[tt * (R + 1) + 2 * p] = live ? du0 : 0.f;
+            ps[tt * (R + 1) + 2 * p + 1] = live ? du1 : 0.f;
         }
         __syncthreads();
 #pragma unroll 4
@@ -1039,8 +1057,9 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
     const int ntiles = (g.L + TT - 1) / TT;
     const int per = (ntiles + nsplit - 1) / nsplit;
     const int t0 = split * per, t1 = min(ntiles, t0 + per);
+    const __nv_bfloat16* Ah = A + static_cast<size_t>(h) * g.a_stride;
     for (int e = tid; e < D * R; e += 256) {
-        const float a = __bfloat162float(A[e]);
+        const float a = __bfloat162float(Ah[e]);
         Au[e] = a;
         At[(e % R) * D + e / R] = a;
     }
@@ -1094,7 +1113,7 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
 #pragma unroll
             for (int pp = 0; pp < FC / 2; ++pp) {
                 const int2 pi = __ldg(pairs + c0 / 2 + pp);
-                cs[pp] = __ldg(tab + pi.y + token_axis_pos(nt, pi.x, g.H, g.W));
+                cs[pp] = g.norope ? make_double2(1.0, 0.0) : __ldg(tab + pi.y + token_axis_pos(nt, pi.x, g.H, g.W));
             }
 #pragma unroll
             for (int pp = 0; pp < FC / 2; ++pp) {
@@ -1120,18 +1139,14 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
                 gg[f] = fmaf(sv[f], go, gg[f]);
             }
         }
-        // phi, psi, partial den = phi . z and psi . G over this warp's features
-        float phi[FC], psi[FC];
+        // psi and the normaliser feature nf, partial den = nf . z and psi . G over this warp's features
+        LrPair P[FC / 2];
         float den_p = 0.f, dot_p = 0.f;
 #pragma unroll
         for (int pp = 0; pp < FC / 2; ++pp) {
-            const float x0 = fmaxf(u[2 * pp], 0.f), x1 = fmaxf(u[2 * pp + 1], 0.f);
-            phi[2 * pp] = x0;
-            phi[2 * pp + 1] = x1;
-            psi[2 * pp] = x0 * cf[pp] - x1 * sf[pp];
-            psi[2 * pp + 1] = x0 * sf[pp] + x1 * cf[pp];
-            den_p = fmaf(x0, zs[c0 + 2 * pp], fmaf(x1, zs[c0 + 2 * pp + 1], den_p));
-            dot_p = fmaf(psi[2 * pp], gg[2 * pp], fmaf(psi[2 * pp + 1], gg[2 * pp + 1], dot_p));
+            P[pp] = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], g.act, g.inside);
+            den_p = fmaf(P[pp].nf0, zs[c0 + 2 * pp], fmaf(P[pp].nf1, zs[c0 + 2 * pp + 1], den_p));
+            dot_p = fmaf(P[pp].psi0, gg[2 * pp], fmaf(P[pp].psi1, gg[2 * pp + 1], dot_p));
         }
         red[(warp * 2 + 0) * TT + lane] = den_p;
         red[(warp * 2 + 1) * TT + lane] = dot_p;
@@ -1148,23 +1163,23 @@ __global__ void __launch_bounds__(256) bwd_lr_q_tiled_kernel(const __nv_bfloat16
         }
         const float dden = live ? -dot / (den * den) : 0.f;
         if (warp == 0) dd[lane] = dden;
-        // psi / den for dS, du = (R^T (G / den) + dden z) [u > 0] for dq and dA, phi for dz
+        // psi / den for dS; du from dpsi = G / den and dnf = dden z for dq and dA; nf for dz
 #pragma unroll
         for (int pp = 0; pp < FC / 2; ++pp) {
             const int c = c0 + 2 * pp;
             const float g0 = gg[2 * pp] / den, g1 = gg[2 * pp + 1] / den;
-            const float dph0 = cf[pp] * g0 + sf[pp] * g1 + dden * zs[c];
-            const float dph1 = -sf[pp] * g0 + cf[pp] * g1 + dden * zs[c + 1];
-            ws[lane * R + c] = live ? psi[2 * pp] / den : 0.f;
-            ws[lane * R + c + 1] = live ? psi[2 * pp + 1] / den : 0.f;
-            const float du0 = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
-            const float du1 = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
+            float du0, du1;
+            lr_pair_bwd(P[pp], g0, g1, dden * zs[c], dden * zs[c + 1], cf[pp], sf[pp], g.inside, du0, du1);
+            du0 = live ? du0 : 0.f;
+            du1 = live ? du1 : 0.f;
+            ws[lane * R + c] = live ? P[pp].psi0 / den : 0.f;
+            ws[lane * R + c + 1] = live ? P[pp].psi1 / den : 0.f;
             dus[lane * (R + 1) + c] = du0;
             dus[lane * (R + 1) + c + 1] = du1;
             duc[lane * R + c] = du0;
             duc[lane * R + c + 1] = du1;
-            phs[lane * R + c] = phi[2 * pp];
-            phs[lane * R + c + 1] = phi[2 * pp + 1];
+            phs[lane * R + c] = P[pp].nf0;
+            phs[lane * R + c + 1] = P[pp].nf1;
         }
         __syncthreads();
         // partial sums: dS[c][e] += sum_t w[t][c] dO[t][e]; dA[d][c] += sum_t q[t][d] du[t][c]; dz
@@ -1247,8 +1262,9 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
     const int ntiles = (g.L + TT - 1) / TT;
     const int per = (ntiles + nsplit - 1) / nsplit;
     const int t0 = split * per, t1 = min(ntiles, t0 + per);
+    const __nv_bfloat16* Ah = A + static_cast<size_t>(h) * g.a_stride;
     for (int e = tid; e < D * R; e += 256) {
-        const float a = __bfloat162float(A[e]);
+        const float a = __bfloat162float(Ah[e]);
         Au[e] = a;
         At[(e % R) * D + e / R] = a;
     }
@@ -1301,7 +1317,7 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
 #pragma unroll
             for (int pp = 0; pp < FC / 2; ++pp) {
                 const int2 pi = __ldg(pairs + c0 / 2 + pp);
-                cs[pp] = __ldg(tab + pi.y + token_axis_pos(nt, pi.x, g.H, g.W));
+                cs[pp] = g.norope ? make_double2(1.0, 0.0) : __ldg(tab + pi.y + token_axis_pos(nt, pi.x, g.H, g.W));
             }
 #pragma unroll
             for (int pp = 0; pp < FC / 2; ++pp) {
@@ -1327,19 +1343,18 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
                 dp[f] = fmaf(sv[f], vo, dp[f]);
             }
         }
-        // psi = R phi; du = (R^T dpsi + dz) [u > 0]
+        // psi; du from dpsi and dnf = dz
 #pragma unroll
         for (int pp = 0; pp < FC / 2; ++pp) {
             const int c = c0 + 2 * pp;
             const float cf = cfs[pp], sf = sfs[pp];
-            const float x0 = fmaxf(u[2 * pp], 0.f), x1 = fmaxf(u[2 * pp + 1], 0.f);
-            psis[lane * (R + 1) + c] = x0 * cf - x1 * sf;
-            psis[lane * (R + 1) + c + 1] = x0 * sf + x1 * cf;
-            const float d0_ = dp[2 * pp], d1_ = dp[2 * pp + 1];
-            const float dph0 = cf * d0_ + sf * d1_ + zs[c];
-            const float dph1 = -sf * d0_ + cf * d1_ + zs[c + 1];
-            const float du0 = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
-            const float du1 = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
+            const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf, sf, g.act, g.inside);
+            psis[lane * (R + 1) + c] = P.psi0;
+            psis[lane * (R + 1) + c + 1] = P.psi1;
+            float du0, du1;
+            lr_pair_bwd(P, dp[2 * pp], dp[2 * pp + 1], zs[c], zs[c + 1], cf, sf, g.inside, du0, du1);
+            du0 = live ? du0 : 0.f;
+            du1 = live ? du1 : 0.f;
             dus[lane * (R + 1) + c] = du0;
             dus[lane * (R + 1) + c + 1] = du1;
             duc[lane * R + c] = du0;
@@ -1394,14 +1409,37 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
     for (int i = 0; i < NA; ++i) da_part[slot * D * R + e_own * R + cg * NA + i] = acc_a[i];
 }
 
-// dA = sum over both passes, all heads and all splits of the partials, in a fixed order.
-__global__ void bwd_da_reduce_kernel(const float* __restrict__ da_part, int nslots, int DR, float* __restrict__ dA) {
+// dA [1 + sep][per_head ? Hh : 1][D][R] from the partials [2 passes][B * Hh][ns][D][R], in a fixed order
+// (pass, batch, head, split): each projection sums the passes that used it (the query pass for Pq, the
+// key pass for Pk, both when they are one matrix) over the heads that share it and every split.
+__global__ void bwd_da_reduce_kernel(const float* __restrict__ da_part, Geom g, int ns, int sep, int per_head,
+                                     float* __restrict__ dA) {
+    const int DR = g.D * g.R;
+    const int nh = per_head ? g.Hh : 1;
     const int o = blockIdx.x * blockDim.x + threadIdx.x;
-    if (o >= DR) return;
+    if (o >= (1 + sep) * nh * DR) return;
+    const int e = o % DR, hh = (o / DR) % nh, pj = o / (DR * nh);
     float s = 0.f;
-    for (int i = 0; i < nslots; ++i) s += da_part[static_cast<size_t>(i) * DR + o];
+    for (int pass = 0; pass < 2; ++pass) {
+        if (sep && pass != pj) continue;
+        for (int b = 0; b < g.B; ++b)
+            for (int h = 0; h < g.Hh; ++h) {
+                if (per_head && h != hh) continue;
+                const size_t slot0 = (static_cast<size_t>(pass) * g.BH() + b * g.Hh + h) * ns;
+                for (int sp = 0; sp < ns; ++sp) s += da_part[(slot0 + sp) * DR + e];
+            }
+    }
     dA[o] = s;
 }
+
+namespace {
+cudaError_t launch_da_reduce(const LrBwdArgs& l, const Geom& g, cudaStream_t st) {
+    const int n = (1 + l.proj_separate) * (l.proj_per_head ? g.Hh : 1) * g.D * g.R;
+    bwd_da_reduce_kernel<<<(n + 255) / 256, 256, 0, st>>>(l.da_part, g, l.nsplit, l.proj_separate, l.proj_per_head,
+                                                           l.dA);
+    return cudaGetLastError();
+}
+}  // namespace
 
 // ------------------------------------------------------------------------------------ launchers
 size_t lr_bwd_smem(int D, int R, bool qpass) {
@@ -1456,17 +1494,16 @@ cudaError_t launch_lr_bwd_t(const LrBwdArgs& l, const Geom& g, cudaStream_t st) 
     e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smk);
     if (e != cudaSuccess) return e;
     qk<<<dim3(ns, g.BH()), 256, smq, st>>>(l.q, l.dout, l.A, l.S, l.z, l.tab, l.pairs, g, ns, l.dq, l.ds_part,
-                                           l.dz_part, l.da_part, l.accumulate);
+                                           l.dz_part, l.da_part, l.accumulate);  // query projection(s)
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_lowrank_reduce(l.ds_part, l.dz_part, g, ns, l.dS, l.dz, nullptr, nullptr, nullptr, st)) !=
         cudaSuccess)
         return e;
-    kk<<<dim3(ns, g.BH()), 256, smk, st>>>(l.k, l.v, l.A, l.dS, l.dz, l.tab, l.pairs, g, ns, l.dk, l.dv,
-                                           l.da_part + static_cast<size_t>(g.BH()) * ns * D * R, l.accumulate);
+    kk<<<dim3(ns, g.BH()), 256, smk, st>>>(l.k, l.v, l.A + l.key_proj_offset(g), l.dS, l.dz, l.tab, l.pairs, g, ns,
+                                           l.dk, l.dv, l.da_part + static_cast<size_t>(g.BH()) * ns * D * R,
+                                           l.accumulate);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int DR = D * R;
-    bwd_da_reduce_kernel<<<(DR + 255) / 256, 256, 0, st>>>(l.da_part, 2 * g.BH() * ns, DR, l.dA);
-    return cudaGetLastError();
+    return launch_da_reduce(l, g, st);
 }
 }  // namespace
 
@@ -1492,9 +1529,7 @@ cudaError_t launch_lr_bwd(const LrBwdArgs& l, const Geom& g, cudaStream_t st) {
     if (lr_bwd_on_tensor_cores(g)) {
         cudaError_t e = launch_lr_bwd_tc(l, g, st);
         if (e != cudaSuccess) return e;
-        const int DR = g.D * g.R;
-        bwd_da_reduce_kernel<<<(DR + 255) / 256, 256, 0, st>>>(l.da_part, 2 * g.BH() * l.nsplit, DR, l.dA);
-        return cudaGetLastError();
+        return launch_da_reduce(l, g, st);
     }
     if (g.D == 128) {
         switch (g.R) {

@@ -51,6 +51,68 @@ __device__ __forceinline__ float phi_act(float u, int act) {
     return act == 0 ? fmaxf(u, 0.f) : phi_act_other(u, act);
 }
 
+// phi = act(u) and d phi / d u (the backward's feature maps; relu inline, the others out of line).
+static __device__ __noinline__ void phi_act_grad_other(float u, int act, float& y, float& dy) {
+    switch (act) {
+        case 1: {
+            const float sg = 1.0f / (1.0f + expf(-u));
+            y = u * sg;
+            dy = sg * (1.0f + u * (1.0f - sg));
+            return;
+        }
+        case 2: y = u; dy = 1.0f; return;
+        default: {
+            const float t = tanhf(u);
+            y = t;
+            dy = 1.0f - t * t;
+            return;
+        }
+    }
+}
+__device__ __forceinline__ void phi_act_grad(float u, int act, float& y, float& dy) {
+    if (act == 0) {
+        y = fmaxf(u, 0.f);
+        dy = u > 0.f ? 1.f : 0.f;
+    } else {
+        phi_act_grad_other(u, act, y, dy);
+    }
+}
+
+// One rotation pair (features 2p, 2p+1) of the low-rank branch, forward and backward, for every
+// ordering of the RoPE and the activation.  (c, s) is the pair's rotation ((1, 0) without the
+// low-rank RoPE).  RoPE outside the activation: phi = act(u), psi = R phi, normaliser feature nf = phi;
+// inside: r = R u, psi = act(r), nf = psi.  a0, a1: the activation's derivative at its input.
+struct LrPair {
+    float psi0, psi1, nf0, nf1, a0, a1;
+};
+__device__ __forceinline__ LrPair lr_pair_fwd(float u0, float u1, float c, float s, int act, int inside) {
+    LrPair p;
+    if (inside) {
+        phi_act_grad(u0 * c - u1 * s, act, p.psi0, p.a0);
+        phi_act_grad(u0 * s + u1 * c, act, p.psi1, p.a1);
+        p.nf0 = p.psi0;
+        p.nf1 = p.psi1;
+    } else {
+        phi_act_grad(u0, act, p.nf0, p.a0);
+        phi_act_grad(u1, act, p.nf1, p.a1);
+        p.psi0 = p.nf0 * c - p.nf1 * s;
+        p.psi1 = p.nf0 * s + p.nf1 * c;
+    }
+    return p;
+}
+// du = d loss / d u of the pair, from the gradients reaching psi (dpsi) and the normaliser feature (dnf).
+__device__ __forceinline__ void lr_pair_bwd(const LrPair& p, float dpsi0, float dpsi1, float dnf0, float dnf1,
+                                            float c, float s, int inside, float& du0, float& du1) {
+    if (inside) {  // d r = (dpsi + dnf) act'(r), du = R^T d r
+        const float dr0 = (dpsi0 + dnf0) * p.a0, dr1 = (dpsi1 + dnf1) * p.a1;
+        du0 = c * dr0 + s * dr1;
+        du1 = -s * dr0 + c * dr1;
+    } else {  // d phi = R^T dpsi + dnf, du = d phi act'(u)
+        du0 = (c * dpsi0 + s * dpsi1 + dnf0) * p.a0;
+        du1 = (-s * dpsi0 + c * dpsi1 + dnf1) * p.a1;
+    }
+}
+
 // 3D RoPE schedule: pair j rotates with the position along axis[j]; its cos/sin for position p
 // (0-based grid coordinate; the constant offset is folded into the table) is tab[tab_off[j] + p].
 struct RopeMeta {
@@ -162,7 +224,10 @@ struct BwdMaps {
     cudaEvent_t between;
 };
 struct LrBwdArgs {
+    // A: the projections as the forward takes them, [1 + proj_separate][proj_per_head ? Hh : 1][D][R]
+    // (per head: head h at A + h * g.a_stride; the key projection after the query projection(s))
     const __nv_bfloat16 *q, *k, *v, *A;
+    int proj_separate, proj_per_head;
     const float* dout;
     const float *S, *z;
     const double2* tab;
@@ -173,7 +238,11 @@ struct LrBwdArgs {
     const RopeMeta* meta;  // rotary schedule (tensor-core passes)
     int* status;
     unsigned long long timeout_ns;
-    int accumulate;  // tensor-core passes: 1 adds dq, dk, dv to the rows (the sparse part is there)
+    int accumulate;  // 1 adds dq, dk, dv to the rows (the sparse part is there); 0 stores them
+    // dA: [1 + proj_separate][proj_per_head ? Hh : 1][D][R], the partials reduced in a fixed order
+    long long key_proj_offset(const Geom& g) const {
+        return proj_separate ? static_cast<long long>(proj_per_head ? g.Hh : 1) * g.D * g.R : 0;
+    }
 };
 cudaError_t launch_bwd_prep(const float* dout, const float* os, const Geom& g, __half* doh, float* delta, int* status,
                             cudaStream_t st);

@@ -157,13 +157,6 @@ __global__ void __launch_bounds__(256, 1)
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    // A^T image [R][128] (B of x A) and A image [128][64] (B of du A^T), once: A is shared
-    for (int e = tid; e < kD * R; e += 256) {
-        const int d = e / R, c = e % R;
-        const uint16_t bits = *reinterpret_cast<const uint16_t*>(a.A + e);
-        *reinterpret_cast<uint16_t*>(smem + Lay::kOffAt + sw128_offset(c, d, R)) = bits;
-        *reinterpret_cast<uint16_t*>(smem + Lay::kOffAi + sw128_offset(d, c, kTok)) = bits;
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -189,9 +182,22 @@ __global__ void __launch_bounds__(256, 1)
     };
     const int ntiles = (g.L + kTok - 1) / kTok;
     const int n_items = g.BH() * a.nsplit;
+    int staged_head = -1;  // head whose projection the A images hold
     for (int item = blockIdx.x; item < n_items && !aborted; item += gridDim.x) {
         const int bh = item / a.nsplit, split = item % a.nsplit;
         const int b = bh / g.Hh, h = bh % g.Hh;
+        // A^T image [R][128] (B of x A) and A image [128][64] (B of du A^T) of this pass's projection:
+        // once when it is shared, again whenever the head changes when there is one per head
+        if (staged_head < 0 || (g.a_stride != 0 && h != staged_head)) {
+            const __nv_bfloat16* Ah = a.A + static_cast<size_t>(h) * g.a_stride;
+            for (int e = tid; e < kD * R; e += 256) {
+                const int d = e / R, c = e % R;
+                const uint16_t bits = *reinterpret_cast<const uint16_t*>(Ah + e);
+                *reinterpret_cast<uint16_t*>(smem + Lay::kOffAt + sw128_offset(c, d, R)) = bits;
+                *reinterpret_cast<uint16_t*>(smem + Lay::kOffAi + sw128_offset(d, c, kTok)) = bits;
+            }
+            staged_head = h;
+        }
         const int t0 = split * a.tiles_per_split, t1 = min(ntiles, t0 + a.tiles_per_split);
         // this head's S (query pass) or dS (key pass) images; every product of the previous item has
         // completed (each tile waits for its second products) and all threads are past its end
@@ -256,7 +262,8 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
             for (int pp = 0; pp < RH / 2; ++pp) {
                 const int2 pi = a.pair_info[half * (RH / 2) + pp];
-                const double2 cs = __ldg(a.tab + pi.y + (pi.x == 0 ? pos_t : (pi.x == 1 ? pos_h : pos_w)));
+                const double2 cs = g.norope ? make_double2(1.0, 0.0)
+                                            : __ldg(a.tab + pi.y + (pi.x == 0 ? pos_t : (pi.x == 1 ? pos_h : pos_w)));
                 cf[pp] = static_cast<float>(cs.x);
                 sf[pp] = static_cast<float>(cs.y);
             }
@@ -316,16 +323,16 @@ __global__ void __launch_bounds__(256, 1)
                     gv[c] = __uint_as_float(r2[c]);
                 }
             }
-            float psi[RH], du[RH], w[RH];
+            // psi, the normaliser feature nf and du per rotation pair (lr_pair_fwd / lr_pair_bwd: every
+            // feature map and RoPE ordering); the pair's forward is recomputed where it is needed again
+            float du[RH], w[RH];
             if constexpr (!kKey) {
                 float den_p = 0.f, dot_p = 0.f;
 #pragma unroll
                 for (int pp = 0; pp < RH / 2; ++pp) {
-                    const float x0 = fmaxf(u[2 * pp], 0.f), x1 = fmaxf(u[2 * pp + 1], 0.f);
-                    psi[2 * pp] = x0 * cf[pp] - x1 * sf[pp];
-                    psi[2 * pp + 1] = x0 * sf[pp] + x1 * cf[pp];
-                    den_p = fmaf(x0, zr[2 * pp], fmaf(x1, zr[2 * pp + 1], den_p));
-                    dot_p = fmaf(psi[2 * pp], gv[2 * pp], fmaf(psi[2 * pp + 1], gv[2 * pp + 1], dot_p));
+                    const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], g.act, g.inside);
+                    den_p = fmaf(P.nf0, zr[2 * pp], fmaf(P.nf1, zr[2 * pp + 1], den_p));
+                    dot_p = fmaf(P.psi0, gv[2 * pp], fmaf(P.psi1, gv[2 * pp + 1], dot_p));
                 }
                 xch[(0 * 2 + half) * 128 + row] = den_p;
                 xch[(1 * 2 + half) * 128 + row] = dot_p;
@@ -335,27 +342,28 @@ __global__ void __launch_bounds__(256, 1)
                 const float dden = live ? -dot / (den * den) : 0.f;
 #pragma unroll
                 for (int pp = 0; pp < RH / 2; ++pp) {
-                    const float g0 = gv[2 * pp] / den, g1 = gv[2 * pp + 1] / den;
-                    const float dph0 = cf[pp] * g0 + sf[pp] * g1 + dden * zr[2 * pp];
-                    const float dph1 = -sf[pp] * g0 + cf[pp] * g1 + dden * zr[2 * pp + 1];
-                    du[2 * pp] = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
-                    du[2 * pp + 1] = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
-                    w[2 * pp] = live ? psi[2 * pp] / den : 0.f;
-                    w[2 * pp + 1] = live ? psi[2 * pp + 1] / den : 0.f;
-                    dzacc[2 * pp] = fmaf(dden, fmaxf(u[2 * pp], 0.f), dzacc[2 * pp]);
-                    dzacc[2 * pp + 1] = fmaf(dden, fmaxf(u[2 * pp + 1], 0.f), dzacc[2 * pp + 1]);
+                    const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], g.act, g.inside);
+                    float du0, du1;
+                    lr_pair_bwd(P, gv[2 * pp] / den, gv[2 * pp + 1] / den, dden * zr[2 * pp], dden * zr[2 * pp + 1],
+                                cf[pp], sf[pp], g.inside, du0, du1);
+                    du[2 * pp] = live ? du0 : 0.f;
+                    du[2 * pp + 1] = live ? du1 : 0.f;
+                    w[2 * pp] = live ? P.psi0 / den : 0.f;
+                    w[2 * pp + 1] = live ? P.psi1 / den : 0.f;
+                    dzacc[2 * pp] = fmaf(dden, P.nf0, dzacc[2 * pp]);
+                    dzacc[2 * pp + 1] = fmaf(dden, P.nf1, dzacc[2 * pp + 1]);
                 }
             } else {
 #pragma unroll
                 for (int pp = 0; pp < RH / 2; ++pp) {
-                    const float x0 = fmaxf(u[2 * pp], 0.f), x1 = fmaxf(u[2 * pp + 1], 0.f);
-                    w[2 * pp] = live ? x0 * cf[pp] - x1 * sf[pp] : 0.f;  // psi, the A operand of dv
-                    w[2 * pp + 1] = live ? x0 * sf[pp] + x1 * cf[pp] : 0.f;
-                    const float d0 = gv[2 * pp], d1 = gv[2 * pp + 1];
-                    const float dph0 = cf[pp] * d0 + sf[pp] * d1 + zr[2 * pp];
-                    const float dph1 = -sf[pp] * d0 + cf[pp] * d1 + zr[2 * pp + 1];
-                    du[2 * pp] = (live && u[2 * pp] > 0.f) ? dph0 : 0.f;
-                    du[2 * pp + 1] = (live && u[2 * pp + 1] > 0.f) ? dph1 : 0.f;
+                    const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], g.act, g.inside);
+                    w[2 * pp] = live ? P.psi0 : 0.f;  // psi, the A operand of dv
+                    w[2 * pp + 1] = live ? P.psi1 : 0.f;
+                    float du0, du1;
+                    lr_pair_bwd(P, gv[2 * pp], gv[2 * pp + 1], zr[2 * pp], zr[2 * pp + 1], cf[pp], sf[pp], g.inside,
+                                du0, du1);
+                    du[2 * pp] = live ? du0 : 0.f;
+                    du[2 * pp + 1] = live ? du1 : 0.f;
                 }
             }
             // w (psi / den, or psi) and du as bf16 hi | lo operand tiles [128 tokens][hi 64 | lo 64]
@@ -539,7 +547,7 @@ namespace {
 template <int R>
 cudaError_t launch_lr_bwd_tc_r(const LrTcBwdArgs& a, const Geom& g, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const CUtensorMap& tdq, const CUtensorMap& tdk,
-                               const CUtensorMap& tdv, float* dS, float* dz, cudaStream_t st) {
+                               const CUtensorMap& tdv, float* dS, float* dz, long long key_off, cudaStream_t st) {
     const size_t sm = static_cast<size_t>(LbLayout<R>::kBytes) + 1024;
     cudaError_t e = cudaFuncSetAttribute(lr_bwd_sm100_kernel<R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
@@ -556,6 +564,7 @@ cudaError_t launch_lr_bwd_tc_r(const LrTcBwdArgs& a, const Geom& g, const CUtens
         cudaSuccess)
         return e;
     LrTcBwdArgs ak = a;
+    ak.A = a.A + key_off;  // the key projection
     ak.dS = dS;
     ak.dz = dz;
     ak.da_part = a.da_part + static_cast<size_t>(g.BH()) * a.nsplit * kD * R;
@@ -598,9 +607,9 @@ cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st)
     a.timeout_ns = l.timeout_ns;
     a.accumulate = l.accumulate;
     switch (g.R) {
-        case 16: return launch_lr_bwd_tc_r<16>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, st);
-        case 32: return launch_lr_bwd_tc_r<32>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, st);
-        case 48: return launch_lr_bwd_tc_r<48>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, st);
+        case 16: return launch_lr_bwd_tc_r<16>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, l.key_proj_offset(g), st);
+        case 32: return launch_lr_bwd_tc_r<32>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, l.key_proj_offset(g), st);
+        case 48: return launch_lr_bwd_tc_r<48>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, l.key_proj_offset(g), st);
     }
     return cudaErrorInvalidValue;
 }

@@ -393,9 +393,9 @@ def attn_bwd_saved(prob: Problem, q, k, v, A, dout, workspace, grads=None, strea
 
 
 def attn_bwd(prob: Problem, q, k, v, A, dout, grads=None, workspace=None, stream=None, _saved=False):
-    """Backward pass (slra_attn_bwd): gradients of sum(dout * out) for q, k, v (fp32 [B, L, Hh, D]) and A
-    (fp32 [D, rank]).  dout: contiguous CUDA fp32 [B, L, Hh, D].  q, k, v may be strided views.
-    Returns (dq, dk, dv, dA, workspace)."""
+    """Backward pass (slra_attn_bwd): gradients of sum(dout * out) for q, k, v (fp32 [B, L, Hh, D]) and the
+    projection(s) A (fp32, prob.projection_shape).  dout: contiguous CUDA fp32 [B, L, Hh, D].  q, k, v may be
+    strided views.  Returns (dq, dk, dv, dA, workspace)."""
     import dataclasses
     torch = _torch()
     shp = (prob.batch, prob.L, prob.heads, prob.head_dim)
@@ -407,7 +407,7 @@ def attn_bwd(prob: Problem, q, k, v, A, dout, grads=None, workspace=None, stream
         _check_bf16("A", A, prob.projection_shape)
     if grads is None:
         grads = tuple(torch.empty(shp, dtype=torch.float32, device=q.device) for _ in range(3)) + \
-            (torch.empty((prob.head_dim, prob.rank), dtype=torch.float32, device=q.device),)
+            (torch.empty(prob.projection_shape, dtype=torch.float32, device=q.device),)
     dq, dk, dv, dA = grads
     if workspace is None:
         n = bwd_workspace_bytes(p)

@@ -246,9 +246,15 @@ def test_train_forward_and_saved_backward_validation():
     assert L.slra_attn_fwd_train(ctypes.byref(pc), q, k, v, A, out, ws + 16, bwd_b, None) == slra.ERR_WORKSPACE
     assert L.slra_attn_fwd_train(ctypes.byref(pc), q, k, v, A, out, ws, bwd_b, None) == slra.ERR_NO_DEVICE
     # options the backward does not cover are refused by the training forward too
-    ps = slra.Problem.from_workload(W.TINY)
-    ps.activation = slra.ACT_SILU
-    assert L.slra_attn_fwd_train(ctypes.byref(ps.c()), q, k, v, A, out, ws, bwd_b, None) == slra.ERR_UNSUPPORTED
+    pg = slra.Problem.from_workload(W.TINY).c()
+    pg.fusion = slra.FUSION_GATED
+    pg.gate_w = dA  # an aligned pointer: the option is refused before anything is read
+    assert L.slra_attn_fwd_train(ctypes.byref(pg), q, k, v, A, out, ws, bwd_b, None) == slra.ERR_UNSUPPORTED
+    # the feature maps, RoPE orderings and projection layouts are covered: they reach the device check
+    for field, value in (("activation", slra.ACT_SILU), ("lowrank_rope_inside", 1), ("lowrank_norope", 1)):
+        po = slra.Problem.from_workload(W.TINY).c()
+        setattr(po, field, value)
+        assert L.slra_attn_fwd_train(ctypes.byref(po), q, k, v, A, out, ws, bwd_b, None) == slra.ERR_NO_DEVICE
     # the saved backward: same checks as slra_attn_bwd
     args = (q, k, v, A, dout, dq, dk, dv, dA)
     assert L.slra_attn_bwd_saved(ctypes.byref(pc), *args, ws, bwd_b - 256, None) == slra.ERR_WORKSPACE

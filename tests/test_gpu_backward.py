@@ -52,26 +52,35 @@ def _gpu_bwd(w, x, dout, **kw):
     return p, [t.cpu().numpy().astype(np.float64) for t in (dq, dk, dv, dA)], idx
 
 
-def _oracle_bwd(w, x, dout, idx, branches):
+def _oracle_bwd(w, x, dout, idx, branches, activation=slra.ACT_RELU, rope="outside", separate=0, per_head=0):
+    """The oracle's gradients head by head; dA in the projection argument's layout (query projections
+    first, then the key projections when separate; one per head when per head)."""
     import oracle
     from oracle import backward as OB
     B, L, Hh, D = x["q"].shape
     R = w.rank
-    A = oracle.decode_bf16(x["A"]).reshape(D, R)
+    nh = Hh if per_head else 1
+    P = oracle.decode_bf16(x["A"]).reshape(1 + separate, nh, D, R)
     grid = (w.T, w.H, w.W)
-    ref = [np.zeros((B, L, Hh, D)) for _ in range(3)] + [np.zeros((D, R))]
+    ref = [np.zeros((B, L, Hh, D)) for _ in range(3)] + [np.zeros((1 + separate, nh, D, R))]
     for b in range(B):
         for h in range(Hh):
             hidx = None if idx is None else idx[b * Hh + h]
             if hidx is None:  # low-rank only: any selection (unused)
                 hidx = np.zeros((w.nb, 1), dtype=np.int32)
+            hp = h if per_head else 0
             r = OB.head_backward(oracle.decode_bf16(x["q"][b, :, h]), oracle.decode_bf16(x["k"][b, :, h]),
-                                 oracle.decode_bf16(x["v"][b, :, h]), A, dout[b, :, h].astype(np.float64), grid,
-                                 w.block, w.keep_frac, R, branches=branches, idx=hidx)
+                                 oracle.decode_bf16(x["v"][b, :, h]), P[0, hp], dout[b, :, h].astype(np.float64),
+                                 grid, w.block, w.keep_frac, R, branches=branches, idx=hidx, activation=activation,
+                                 rope=rope, A_k=P[1, hp] if separate else None)
             ref[0][b, :, h] = r["dq"]
             ref[1][b, :, h] = r["dk"]
             ref[2][b, :, h] = r["dv"]
-            ref[3] += r["dA"]
+            ref[3][0, hp] += r["dA"]
+            if separate:
+                ref[3][1, hp] += r["dA_k"]
+    if not separate and not per_head:
+        ref[3] = ref[3].reshape(D, R)
     return ref
 
 
@@ -213,3 +222,84 @@ def test_saved_forward_backward_equals_recompute(w):
 @pytest.mark.parametrize("branches", [slra.BRANCH_SPARSE, slra.BRANCH_LOWRANK])
 def test_saved_forward_backward_single_branch(branches):
     _saved_vs_recompute(EDGE_128, branches)
+
+
+# ---- the forward's options (RoLA 5.3 Table 6 feature maps, the RoPE orderings of Table 2, separate and
+# per-head projections of App. E.2 / RoPeSLR's head-wise parameterization)
+
+R128 = W.Workload("bwd-r128", 1, 2, 128, 2, 9, 11, 128, 64, 0.25, 7500)    # rank 128: untiled fp32 passes
+EDGE_PROJ = W.Workload("bwd-proj-128", 1, 8, 128, 4, 24, 32, 32, 128, 0.1, 7300)  # CTAs change head
+
+
+def _nonneg(x):
+    """q, k and A with the bf16 sign bit cleared, so every feature x A >= 0 and the normaliser stays
+    away from zero for the maps whose features can be negative (as in the forward's tests)."""
+    y = dict(x)
+    for n in ("q", "k", "A"):
+        y[n] = np.bitwise_and(x[n], np.uint16(0x7FFF))
+    return y
+
+
+def _case_opts(w, label, activation=slra.ACT_RELU, rope="outside", separate=0, per_head=0,
+               branches=slra.BRANCH_BOTH, nonneg=False):
+    x = I.make_inputs(w)
+    if separate or per_head:
+        x["A"] = I.make_projections(w.seed + 5000, w.heads, w.head_dim, w.rank, bool(separate), bool(per_head))
+    if nonneg:
+        x = _nonneg(x)
+    dout = I.make_dout(w.seed + 9000, w.batch, w.L, w.heads, w.head_dim)
+    kw = dict(branches=branches, activation=activation, lowrank_norope=int(rope == "none"),
+              lowrank_rope_inside=int(rope == "inside"), proj_separate=separate, proj_per_head=per_head)
+    p, got, idx = _gpu_bwd(w, x, dout, **kw)
+    ref = _oracle_bwd(w, x, dout, idx, branches, activation, rope, separate, per_head)
+    return _compare(label, got, ref)
+
+
+@pytest.mark.parametrize("act", [slra.ACT_SILU, slra.ACT_IDENTITY, slra.ACT_TANH])
+@pytest.mark.parametrize("w", [W.TINY, EDGE_128, EDGE_128_B64, R128], ids=lambda w: w.name)
+def test_backward_activations(w, act):
+    """Each feature map on every low-rank gradient path: head_dim 64 and rank 64 (register-tiled fp32),
+    rank 32 (tensor cores), rank 128 (untiled fp32)."""
+    _case_opts(w, f"{w.name}-act{act}", activation=act, nonneg=True)
+
+
+@pytest.mark.parametrize("rope", ["none", "inside"])
+@pytest.mark.parametrize("w", [W.TINY, EDGE_128, EDGE_128_B64, R128], ids=lambda w: w.name)
+def test_backward_rope_orderings(w, rope):
+    """No low-rank RoPE, and the RoPE inside the activation (the normaliser on psi), on every path;
+    inside with SiLU on the tensor-core path."""
+    _case_opts(w, f"{w.name}-rope-{rope}", rope=rope)
+    if rope == "inside" and w is EDGE_128:
+        _case_opts(w, f"{w.name}-rope-inside-silu", rope=rope, activation=slra.ACT_SILU, nonneg=True)
+
+
+@pytest.mark.parametrize("separate,per_head", [(1, 0), (0, 1), (1, 1)])
+@pytest.mark.parametrize("w", [W.TINY, EDGE_128, EDGE_128_B64, R128, EDGE_PROJ], ids=lambda w: w.name)
+def test_backward_projections(w, separate, per_head):
+    """Separate query / key projections and per-head projections: dA per projection in the argument's
+    layout, on every path; 8 heads on the tensor-core path, where persistent CTAs restage the head's
+    projection between work items."""
+    _case_opts(w, f"{w.name}-proj-s{separate}-h{per_head}", separate=separate, per_head=per_head)
+
+
+def test_backward_r128_default():
+    _case_opts(R128, "bwd-r128")
+
+
+def test_saved_backward_with_options():
+    """The training pair with SiLU features and separate per-head projections: bit for bit the
+    recomputing backward."""
+    import torch
+    w = EDGE_PROJ
+    x = _nonneg(dict(I.make_inputs(w), A=I.make_projections(w.seed + 5000, w.heads, w.head_dim, w.rank, True, True)))
+    dout = torch.from_numpy(I.make_dout(w.seed + 9100, w.batch, w.L, w.heads, w.head_dim)).cuda()
+    p = slra.Problem.from_workload(w, activation=slra.ACT_SILU, proj_separate=1, proj_per_head=1)
+    q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
+    out_ref = slra.attn_fwd(p, q, k, v, A)[0]
+    out_t, ws = slra.attn_fwd_train(p, q, k, v, A)
+    assert torch.equal(out_t, out_ref)
+    ref = slra.attn_bwd(p, q, k, v, A, dout)[:4]
+    got = slra.attn_bwd_saved(p, q, k, v, A, dout, ws)[:4]
+    assert slra.device_status(ws) == slra.OK
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
