@@ -66,7 +66,7 @@
 extern "C" {
 #endif
 
-#define SLRA_ABI_VERSION 7
+#define SLRA_ABI_VERSION 8
 
 /* Exported symbols (the library is built with hidden visibility for everything else). */
 #if defined(__GNUC__)
@@ -218,6 +218,8 @@ typedef struct slra_problem {
     const void* gate_w;
     int32_t lowrank_rope_inside;
     int64_t q_strides[3], k_strides[3], v_strides[3], out_strides[3];
+    void* dgate_w;  /* backward, gated fusion: output fp32 [head_dim], d loss / d Wg (16-B aligned) */
+    void* dgate_b;  /* backward, gated fusion: output fp32 [1], d loss / d bg (4-B aligned) */
 } slra_problem;
 
 /*
@@ -336,12 +338,15 @@ SLRA_API size_t slra_bwd_workspace_bytes(const slra_problem* p);
  * Backward pass: the gradients of sum(dout * out) with respect to q, k, v and A, where out is the
  * forward pass of slra_attn_fwd_ex on the same arguments (RoLA "4.5", "E.1", "E.2": the branch's
  * parameters are trained jointly with the backbone).  The block selection is held at the forward's (it
- * is piecewise constant in q and k).  Covered: relu features, the low-rank RoPE outside the activation,
- * one shared projection, the plain sum, any branches mask; other options return SLRA_ERR_UNSUPPORTED.
+ * is piecewise constant in q and k).  Every option of the forward is covered: the feature maps, the
+ * RoPE orderings, separate and per-head projections (dA then has A's layout), any branches mask, and
+ * the gated fusion, whose parameter gradients go to p->dgate_w (fp32 [head_dim], 16-B aligned) and
+ * p->dgate_b (one fp32), both required then and disjoint from every other argument.
  *   q, k, v, A   as for slra_attn_fwd_ex (q, k, v may be strided per p).
  *   dout         fp32 [B][L][Hh][D] contiguous: the gradient of the loss with respect to out.
  *   dq, dk, dv   fp32 [B][L][Hh][D] contiguous outputs (p->out_strides must be zero).
- *   dA           fp32 [D][rank] output (zero when the low-rank branch is off).
+ *   dA           fp32 output in the projection argument's layout, slra_projection_elems(p) elements
+ *                (zero when the low-rank branch is off).
  *   workspace    at least slra_bwd_workspace_bytes(p) bytes, 256-B aligned (the forward's sections are
  *                refilled by the recompute and can be inspected afterwards).
  * The sparse branch's gradients run on the tensor cores: a dQ kernel per query block (S = q^ k^T and
@@ -349,21 +354,25 @@ SLRA_API size_t slra_bwd_workspace_bytes(const slra_problem* p);
  * over the query blocks that kept it (dV += P^T dO, dK^ += dS^T q^), with fp16 operands (dout must stay
  * below 65504 in magnitude, else SLRA_ERR_RANGE is recorded) and fp32 accumulation; the low-rank chain
  * follows as a pass over the queries and one over the keys (on the tensor cores for head_dim 128 and
- * rank <= 48, fp32 otherwise) that add their parts to dq, dk, dv and produce dA.  Deterministic.
+ * rank <= 48, fp32 otherwise) that add their parts to dq, dk, dv and produce dA.  With the gated fusion
+ * the low-rank branch's output is recomputed too, one pass per row splits dout into the two branches'
+ * gradients and the gate's, and a last pass adds the gate's part to dq and reduces dWg, dbg.
+ * Deterministic.
  * stage_events are recorded at: [0] start, [1] after the recomputed forward, [2] after the dO copy and
  * the inverted lists, [3] after the dQ kernel, [4] after the dK/dV kernel, [5] and [6] after the
- * low-rank gradients.  Device problems go to the workspace's status word (slra_device_status).
+ * low-rank (and gate) gradients.  Device problems go to the workspace's status word (slra_device_status).
  */
 SLRA_API slra_status slra_attn_bwd(const slra_problem* p, const void* q, const void* k, const void* v,
                                    const void* A, const float* dout, float* dq, float* dk, float* dv, float* dA,
                                    void* workspace, size_t workspace_bytes, slra_stream_t stream);
 
 /*
- * Forward pass for training: slra_attn_fwd_ex on the options slra_attn_bwd covers (same arguments;
- * out contiguous), which also keeps in `workspace` what the backward would recompute: the tables, the
- * block selection, the low-rank summary, the fp16 operand copies, each query row's log-sum-exp and
- * the sparse branch's own output (stored by the attention kernel before the low-rank readout joins
- * it).  out is bit for bit that of slra_attn_fwd_ex.
+ * Forward pass for training: slra_attn_fwd_ex with out contiguous (same arguments), which also keeps
+ * in `workspace` what the backward would recompute: the tables, the block selection, the low-rank
+ * summary and readout operands, the fp16 operand copies, each query row's log-sum-exp and the sparse
+ * branch's own output (stored by the attention kernel before the low-rank readout joins it).  out is
+ * bit for bit that of slra_attn_fwd_ex.  (With the gated fusion the backward still recomputes the
+ * low-rank branch's output alone, a pass without the sparse loop.)
  *   workspace    at least slra_bwd_workspace_bytes(p) bytes, 256-B aligned (NULL is rejected:
  *                SLRA_ERR_WORKSPACE); its status word starts cleared, as for slra_attn_fwd_ex.
  * Pass the same workspace, untouched, to slra_attn_bwd_saved.

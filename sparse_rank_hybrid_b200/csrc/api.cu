@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <utility>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -98,6 +99,7 @@ struct Derived {
     size_t at_img, sb_img;  // operand images of the tensor-core readout (offsets; head_dim 128 only)
     size_t a_elems;         // bf16 elements of the projection argument
     size_t ak_off;          // elements from its start to the key projection(s)
+    bool gated;             // gated fusion of the branches
 };
 
 slra_status derive(const slra_problem* p, Derived* d) {
@@ -164,6 +166,7 @@ slra_status derive(const slra_problem* p, Derived* d) {
     const size_t one_side = static_cast<size_t>(p->proj_per_head ? p->heads : 1) * p->head_dim * p->rank;
     d->a_elems = one_side * (p->proj_separate ? 2 : 1);
     d->ak_off = p->proj_separate ? one_side : 0;
+    d->gated = p->fusion == SLRA_FUSION_GATED;
 
     RopeMeta& m = d->meta;
     std::memset(&m, 0, sizeof m);
@@ -696,7 +699,9 @@ slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, con
 // ---------------------------------------------------------------- backward pass
 // Sections the backward adds after the forward's workspace layout (256-B aligned byte offsets).
 struct BwdLayout {
-    size_t lse, delta, os, doh, inv_cnt, inv, ds_part, dz_part, dS, dz, da_part, total;
+    size_t lse, delta, os, doh, inv_cnt, inv, ds_part, dz_part, dS, dz, da_part;
+    size_t olr, dolr, dlogit, gpart;  // gated fusion only (empty otherwise)
+    size_t total;
     int ns;  // splits of the low-rank gradient passes
 };
 
@@ -722,16 +727,19 @@ BwdLayout bwd_layout(const Derived& d) {
     b.dS = take(static_cast<size_t>(g.BH()) * g.R * g.D * 4);
     b.dz = take(static_cast<size_t>(g.BH()) * g.R * 4);
     b.da_part = take(2 * static_cast<size_t>(g.BH()) * b.ns * g.D * g.R * 4);
+    const bool gated = d.gated;
+    b.olr = take(gated ? rows * g.D * 4 : 0);
+    b.dolr = take(gated ? static_cast<size_t>(g.B) * g.L * g.Hh * g.D * 4 : 0);
+    b.dlogit = take(gated ? rows * 4 : 0);
+    b.gpart = take(gated ? static_cast<size_t>(kGateParts) * (g.D + 1) * 4 : 0);
     b.total = o;
     return b;
 }
 
-// The backward covers every feature map, RoPE ordering and projection layout with the plain sum of the
-// branches (not the gated fusion); gradients are contiguous fp32 [B][L][Hh][D].
+// The backward covers every option of the forward; gradients are contiguous fp32 [B][L][Hh][D].
 slra_status check_bwd_problem(const slra_problem* p, Derived* d) {
     slra_status s = derive(p, d);
     if (s != SLRA_OK) return s;
-    if (p->fusion != SLRA_FUSION_SUM) return SLRA_ERR_UNSUPPORTED;
     for (int i = 0; i < 3; ++i)
         if (p->out_strides[i]) return SLRA_ERR_INVALID_ARG;
     return SLRA_OK;
@@ -807,6 +815,8 @@ slra_status slra_problem_init(slra_problem* p, int64_t batch, int64_t heads, int
     p->gate_bias = 0.0f;
     p->gate_w = nullptr;
     p->lowrank_rope_inside = 0;
+    p->dgate_w = nullptr;
+    p->dgate_b = nullptr;
     return SLRA_OK;
 }
 
@@ -1031,6 +1041,24 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
             if (overlaps(outs[i], out_n[i], outs[j], out_n[j])) return SLRA_ERR_INVALID_ARG;
         if (workspace && overlaps(outs[i], out_n[i], workspace, workspace_bytes)) return SLRA_ERR_INVALID_ARG;
     }
+    // the gated fusion's parameter gradients: disjoint from every other argument
+    float* dgw = static_cast<float*>(p->dgate_w);
+    float* dgb = static_cast<float*>(p->dgate_b);
+    if (d.gated) {
+        if (!dgw || !dgb) return SLRA_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(dgw) & 15u) != 0 || (reinterpret_cast<uintptr_t>(dgb) & 3u) != 0)
+            return SLRA_ERR_ALIGNMENT;
+        const size_t gwb = static_cast<size_t>(g.D) * 4;
+        if (overlaps(dgw, gwb, dgb, 4)) return SLRA_ERR_INVALID_ARG;
+        for (const auto& [ptr, n] : {std::pair<const void*, size_t>{dgw, gwb}, {dgb, 4}}) {
+            for (int j = 0; j < 5; ++j)
+                if (ins[j] && overlaps(ptr, n, ins[j], in_n[j])) return SLRA_ERR_INVALID_ARG;
+            for (int j = 0; j < 4; ++j)
+                if (overlaps(ptr, n, outs[j], out_n[j])) return SLRA_ERR_INVALID_ARG;
+            if (overlaps(ptr, n, p->gate_w, gwb) || (workspace && overlaps(ptr, n, workspace, workspace_bytes)))
+                return SLRA_ERR_INVALID_ARG;
+        }
+    }
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < bl.total)
         return SLRA_ERR_WORKSPACE;
     if ((s = check_device()) != SLRA_OK) return s;
@@ -1083,11 +1111,56 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
         a.os_save = nullptr;
         if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
     }
+    float* olr = reinterpret_cast<float*>(base + bl.olr);
+    float* dolr = reinterpret_cast<float*>(base + bl.dolr);
+    float* dlogit = reinterpret_cast<float*>(base + bl.dlogit);
+    if (d.gated) {
+        // the low-rank branch's own output O_lr (head-major fp32): the attention kernel with the sparse
+        // branch off, the readout alone (both in the recompute and after a training forward)
+        AttnMaps maps;
+        const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
+        if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) ||
+            !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
+            !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
+            !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, g.sq, 128) ||
+            !make_map_out(&maps.out, olr, g.B, g.L, g.Hh, g.D, headmajor_strides(g), true))
+            return SLRA_ERR_CUDA;
+        std::memset(&maps.os, 0, sizeof maps.os);
+        AttnArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.qh = w.qh;
+        a.kh = w.kh;
+        a.vh = w.vh;
+        a.idx = w.idx;
+        a.keep = 0;
+        a.q_raw = static_cast<const __nv_bfloat16*>(q);
+        a.A = static_cast<const __nv_bfloat16*>(A);
+        a.S = w.S;
+        a.z = w.z;
+        a.tab = w.tab;
+        a.pairs = w.pairs;
+        for (int e = 0; e < kMaxPairs; ++e)
+            a.pair_info[e] = e < d.meta.npairs ? make_int2(d.meta.axis[e], d.meta.tab_off[e]) : make_int2(0, 0);
+        a.at_img = w.at_img;
+        a.sb_img = w.sb_img;
+        a.lowrank = 1;
+        a.out = olr;
+        a.status = w.status;
+        a.timeout_ns = timeout_of(p);
+        if ((s = cuda_status(launch_attn(maps, a, g, st))) != SLRA_OK) return s;
+    }
     if ((s = mark(p, 1, st)) != SLRA_OK) return s;
     // The sparse kernels store dq, dk, dv; the low-rank gradients then add their parts (or store them
     // when the sparse branch is off).
     if (sparse) {
-        if ((s = cuda_status(launch_bwd_prep(dout, os, g, doh, delta, w.status, st))) != SLRA_OK) return s;
+        // dO_s as the sparse branch sees it: dout itself, or through the gate (with dO_lr and dlogit)
+        if (d.gated)
+            s = cuda_status(launch_gate_prep(dout, os, olr, static_cast<const __nv_bfloat16*>(q),
+                                             static_cast<const float*>(p->gate_w), p->gate_bias, g, doh, delta, dolr,
+                                             dlogit, w.status, st));
+        else
+            s = cuda_status(launch_bwd_prep(dout, os, g, doh, delta, w.status, st));
+        if (s != SLRA_OK) return s;
         if ((s = cuda_status(launch_bwd_invert(w.idx, g, inv, inv_cnt, st))) != SLRA_OK) return s;
         if ((s = mark(p, 2, st)) != SLRA_OK) return s;
         BwdMaps m;
@@ -1127,7 +1200,7 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
         l.A = static_cast<const __nv_bfloat16*>(A);
         l.proj_separate = p->proj_separate ? 1 : 0;
         l.proj_per_head = p->proj_per_head ? 1 : 0;
-        l.dout = dout;
+        l.dout = d.gated ? dolr : dout;
         l.S = w.S;
         l.z = w.z;
         l.tab = w.tab;
@@ -1150,6 +1223,11 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
     } else if (cudaMemsetAsync(dA, 0, ab, st) != cudaSuccess) {
         return SLRA_ERR_CUDA;
     }
+    if (d.gated &&
+        (s = cuda_status(launch_gate_final(static_cast<const __nv_bfloat16*>(q), dlogit,
+                                           static_cast<const float*>(p->gate_w), g, dq,
+                                           reinterpret_cast<float*>(base + bl.gpart), dgw, dgb, st))) != SLRA_OK)
+        return s;
     if ((s = mark(p, 5, st)) != SLRA_OK) return s;
     return mark(p, 6, st);
 }

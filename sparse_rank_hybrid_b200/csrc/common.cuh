@@ -62,9 +62,11 @@ static __device__ __noinline__ void phi_act_grad_other(float u, int act, float& 
         }
         case 2: y = u; dy = 1.0f; return;
         default: {
-            const float t = tanhf(u);
-            y = t;
-            dy = 1.0f - t * t;
+            // 1 - tanh^2 = 4 e / (1 + e)^2 with e = exp(-2|u|): no cancellation where tanh saturates
+            // (1 - t * t in fp32 loses all digits of a derivative below ~1e-6)
+            const float e = expf(-2.0f * fabsf(u));
+            y = tanhf(u);
+            dy = 4.0f * e / ((1.0f + e) * (1.0f + e));
             return;
         }
     }
@@ -253,5 +255,16 @@ cudaError_t launch_lr_bwd(const LrBwdArgs& l, const Geom& g, cudaStream_t st);
 cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st);
 inline bool lr_bwd_on_tensor_cores(const Geom& g) { return g.D == 128 && g.R <= 48; }
 int lr_bwd_nsplit(const Geom& g);
+
+// ---- backward of the gated fusion (gate_bwd.cu) -------------------------------------------------
+constexpr int kGateParts = 296;  // CTAs (and partial sums) of the gate-parameter reduction
+// dO_s (fp16 head-major copy and Delta), dO_lr (fp32 token-major) and dlogit per row from dout, O_s and
+// O_lr (head-major fp32) and the raw queries.
+cudaError_t launch_gate_prep(const float* dout, const float* os, const float* olr, const __nv_bfloat16* q,
+                             const float* gate_w, float gate_b, const Geom& g, __half* doh, float* delta, float* dolr,
+                             float* dlogit, int* status, cudaStream_t st);
+// dq += dlogit Wg; dWg, dbg (part: kGateParts x (D + 1) floats of scratch).
+cudaError_t launch_gate_final(const __nv_bfloat16* q, const float* dlogit, const float* gate_w, const Geom& g,
+                              float* dq, float* part, float* dgw, float* dgb, cudaStream_t st);
 
 }  // namespace slra

@@ -1,0 +1,156 @@
+// Backward of the gated fusion of the two branches (RoLA 4.4, in the reading the forward implements):
+//   out = O_s + c O_lr,   c = g a / b,   a = sqrt(mean(O_s^2)),   b = sqrt(mean(O_lr^2) + 1e-6),
+//   g = sigmoid(q . Wg + bg) on the head's raw query row.
+// Per row, with t = dout . O_lr:
+//   dO_s   = dout + c t / (D a^2) O_s        (the a-term is absent when a = 0)
+//   dO_lr  = c dout - c t / (D b^2) O_lr
+//   dlogit = t (a / b) g (1 - g),   dq += dlogit Wg,   dWg = sum dlogit q,   dbg = sum dlogit.
+// The sparse gradient kernels then run on dO_s (through the fp16 copy and Delta = dO_s . O_s this prep
+// writes) and the low-rank passes on dO_lr.
+#include "common.cuh"
+
+namespace slra {
+
+namespace {
+
+// One warp per row (b, h, n) of the padded head-major grid: O_s and O_lr head-major fp32, dout and
+// dO_lr token-major fp32, the fp16 copy of dO_s head-major (rows past L zero).
+__global__ void bwd_gate_prep_kernel(const float* __restrict__ dout, const float* __restrict__ os,
+                                     const float* __restrict__ olr, const __nv_bfloat16* __restrict__ q,
+                                     const float* __restrict__ gate_w, float gate_b, Geom g,
+                                     __half* __restrict__ doh, float* __restrict__ delta, float* __restrict__ dolr,
+                                     float* __restrict__ dlogit, int* status) {
+    const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const long long rows = static_cast<long long>(g.BH()) * g.Lp;
+    if (warp >= rows) return;
+    const int bh = static_cast<int>(warp / g.Lp), n = static_cast<int>(warp % g.Lp);
+    const int b = bh / g.Hh, h = bh % g.Hh;
+    const int per = g.D / 32;  // elements per lane: 2 or 4
+    __half* dst = doh + static_cast<size_t>(warp) * g.D + lane * per;
+    if (n >= g.L) {
+        for (int e = 0; e < per; e += 2) *reinterpret_cast<__half2*>(dst + e) = __floats2half2_rn(0.f, 0.f);
+        if (lane == 0) {
+            delta[warp] = 0.f;
+            dlogit[warp] = 0.f;
+        }
+        return;
+    }
+    float x[4], s[4], l[4];
+    float ss_s = 0.f, ss_l = 0.f, t = 0.f, qw = 0.f;
+    const float* src = dout + g.so.row(b, n, h) + lane * per;
+    const float* so = os + static_cast<size_t>(warp) * g.D + lane * per;
+    const float* sl = olr + static_cast<size_t>(warp) * g.D + lane * per;
+    const __nv_bfloat16* sq = q + g.sq.row(b, n, h) + lane * per;
+    for (int e = 0; e < per; ++e) {
+        x[e] = src[e];
+        s[e] = so[e];
+        l[e] = sl[e];
+        ss_s = fmaf(s[e], s[e], ss_s);
+        ss_l = fmaf(l[e], l[e], ss_l);
+        t = fmaf(x[e], l[e], t);
+        qw = fmaf(__bfloat162float(sq[e]), __ldg(gate_w + lane * per + e), qw);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ss_s += __shfl_xor_sync(0xffffffffu, ss_s, o);
+        ss_l += __shfl_xor_sync(0xffffffffu, ss_l, o);
+        t += __shfl_xor_sync(0xffffffffu, t, o);
+        qw += __shfl_xor_sync(0xffffffffu, qw, o);
+    }
+    const float inv_d = 1.f / static_cast<float>(g.D);
+    const float a = sqrtf(ss_s * inv_d), bb = sqrtf(ss_l * inv_d + 1e-6f);
+    const float gg = 1.f / (1.f + expf(-(qw + gate_b)));
+    const float c = gg * a / bb;
+    const float ks = a > 0.f ? c * t * inv_d / (a * a) : 0.f;
+    const float kl = c * t * inv_d / (bb * bb);
+    float dsum = 0.f;
+    bool bad = false;
+    float* dl = dolr + g.so.row(b, n, h) + lane * per;
+    for (int e = 0; e < per; e += 2) {
+        const float d0 = fmaf(ks, s[e], x[e]), d1 = fmaf(ks, s[e + 1], x[e + 1]);
+        dsum = fmaf(d0, s[e], fmaf(d1, s[e + 1], dsum));
+        bad |= !(fmaxf(fabsf(d0), fabsf(d1)) < 65504.f);
+        *reinterpret_cast<__half2*>(dst + e) = __floats2half2_rn(d0, d1);
+        *reinterpret_cast<float2*>(dl + e) = make_float2(c * x[e] - kl * l[e], c * x[e + 1] - kl * l[e + 1]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+    if (lane == 0) {
+        delta[warp] = dsum;
+        dlogit[warp] = t * (a / bb) * gg * (1.f - gg);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, kDevRange);
+}
+
+// dq += dlogit Wg on every row, and per-CTA partial sums of dWg = sum dlogit q and dbg = sum dlogit
+// over a fixed range of rows, in a fixed order (thread = column of a row stream).
+__global__ void bwd_gate_final_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ dlogit,
+                                      const float* __restrict__ gate_w, Geom g, long long rows_per_cta,
+                                      float* __restrict__ dq, float* __restrict__ part) {
+    __shared__ float red[256 + 8];
+    const int tid = threadIdx.x, col = tid % g.D, rs = tid / g.D, nstream = blockDim.x / g.D;
+    const long long rows = static_cast<long long>(g.BH()) * g.L;
+    const long long r0 = blockIdx.x * rows_per_cta;
+    const long long r1 = r0 + rows_per_cta < rows ? r0 + rows_per_cta : rows;
+    const float wg = __ldg(gate_w + col);
+    float acc = 0.f, accb = 0.f;
+    for (long long r = r0 + rs; r < r1; r += nstream) {
+        const int bh = static_cast<int>(r / g.L), n = static_cast<int>(r % g.L);
+        const int b = bh / g.Hh, h = bh % g.Hh;
+        const float d = dlogit[static_cast<size_t>(bh) * g.Lp + n];
+        acc = fmaf(d, __bfloat162float(q[g.sq.row(b, n, h) + col]), acc);
+        accb += d;
+        float* o = dq + g.so.row(b, n, h) + col;
+        *o = fmaf(d, wg, *o);
+    }
+    red[tid] = acc;
+    if (col == 0) red[256 + rs] = accb;
+    __syncthreads();
+    float* mine = part + static_cast<size_t>(blockIdx.x) * (g.D + 1);
+    if (rs == 0) {
+        float s = 0.f;
+        for (int i = 0; i < nstream; ++i) s += red[i * g.D + col];
+        mine[col] = s;
+    }
+    if (tid == 0) {
+        float s = 0.f;
+        for (int i = 0; i < nstream; ++i) s += red[256 + i];
+        mine[g.D] = s;
+    }
+}
+
+__global__ void bwd_gate_reduce_kernel(const float* __restrict__ part, int nparts, int D, float* __restrict__ dgw,
+                                       float* __restrict__ dgb) {
+    const int o = threadIdx.x;
+    if (o > D) return;
+    float s = 0.f;
+    for (int i = 0; i < nparts; ++i) s += part[static_cast<size_t>(i) * (D + 1) + o];
+    if (o < D) dgw[o] = s;
+    else *dgb = s;
+}
+
+}  // namespace
+
+cudaError_t launch_gate_prep(const float* dout, const float* os, const float* olr, const __nv_bfloat16* q,
+                             const float* gate_w, float gate_b, const Geom& g, __half* doh, float* delta, float* dolr,
+                             float* dlogit, int* status, cudaStream_t st) {
+    const long long rows = static_cast<long long>(g.BH()) * g.Lp;
+    const long long blocks = (rows * 32 + 255) / 256;
+    bwd_gate_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(dout, os, olr, q, gate_w, gate_b, g, doh, delta,
+                                                                        dolr, dlogit, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gate_final(const __nv_bfloat16* q, const float* dlogit, const float* gate_w, const Geom& g,
+                              float* dq, float* part, float* dgw, float* dgb, cudaStream_t st) {
+    const long long rows = static_cast<long long>(g.BH()) * g.L;
+    const long long per = (rows + kGateParts - 1) / kGateParts;
+    bwd_gate_final_kernel<<<kGateParts, 256, 0, st>>>(q, dlogit, gate_w, g, per, dq, part);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bwd_gate_reduce_kernel<<<1, 256, 0, st>>>(part, kGateParts, g.D, dgw, dgb);
+    return cudaGetLastError();
+}
+
+}  // namespace slra

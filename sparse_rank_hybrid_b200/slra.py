@@ -20,7 +20,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_DE
 OUT_F32, OUT_BF16 = 0, 1
 BRANCH_SPARSE, BRANCH_LOWRANK, BRANCH_BOTH = 1, 2, 3
 DEBUG_UNSATISFIED_WAIT, DEBUG_SERIAL_BRANCHES = 1, 2
-ABI_VERSION = 7
+ABI_VERSION = 8
 DTYPE_BF16, DTYPE_F32 = 0, 1
 ACT_RELU, ACT_SILU, ACT_IDENTITY, ACT_TANH = 0, 1, 2, 3
 FUSION_SUM, FUSION_GATED = 0, 1
@@ -53,7 +53,8 @@ class _Problem(ctypes.Structure):
                 ("proj_per_head", ctypes.c_int32), ("fusion", ctypes.c_int32), ("gate_bias", ctypes.c_float),
                 ("gate_w", ctypes.c_void_p), ("lowrank_rope_inside", ctypes.c_int32),
                 ("q_strides", ctypes.c_int64 * 3), ("k_strides", ctypes.c_int64 * 3),
-                ("v_strides", ctypes.c_int64 * 3), ("out_strides", ctypes.c_int64 * 3)]
+                ("v_strides", ctypes.c_int64 * 3), ("out_strides", ctypes.c_int64 * 3),
+                ("dgate_w", ctypes.c_void_p), ("dgate_b", ctypes.c_void_p)]
 
 
 class _Tensor(ctypes.Structure):
@@ -171,6 +172,8 @@ class Problem:
     k_strides: tuple = (0, 0, 0)
     v_strides: tuple = (0, 0, 0)
     out_strides: tuple = (0, 0, 0)
+    dgate_w: object = None             # backward, gated: output CUDA fp32 tensor [head_dim] (d loss / d Wg)
+    dgate_b: object = None             # backward, gated: output CUDA fp32 tensor [1] (d loss / d bg)
 
     @property
     def L(self) -> int:
@@ -208,6 +211,13 @@ class Problem:
             if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (self.head_dim,):
                 raise ValueError(f"gate_w: expected a contiguous CUDA fp32 tensor of shape ({self.head_dim},)")
             p.gate_w = int(t.data_ptr())
+        for name, n in (("dgate_w", self.head_dim), ("dgate_b", 1)):
+            t = getattr(self, name)
+            if t is not None:
+                torch = _torch()
+                if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.numel() != n:
+                    raise ValueError(f"{name}: expected a contiguous CUDA fp32 tensor of {n} elements")
+                setattr(p, name, int(t.data_ptr()))
         return p
 
     @property
@@ -395,7 +405,8 @@ def attn_bwd_saved(prob: Problem, q, k, v, A, dout, workspace, grads=None, strea
 def attn_bwd(prob: Problem, q, k, v, A, dout, grads=None, workspace=None, stream=None, _saved=False):
     """Backward pass (slra_attn_bwd): gradients of sum(dout * out) for q, k, v (fp32 [B, L, Hh, D]) and the
     projection(s) A (fp32, prob.projection_shape).  dout: contiguous CUDA fp32 [B, L, Hh, D].  q, k, v may be
-    strided views.  Returns (dq, dk, dv, dA, workspace)."""
+    strided views.  With the gated fusion, prob.dgate_w and prob.dgate_b receive the gate parameters'
+    gradients.  Returns (dq, dk, dv, dA, workspace)."""
     import dataclasses
     torch = _torch()
     shp = (prob.batch, prob.L, prob.heads, prob.head_dim)

@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_abi_version_and_status_strings():
-    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 7
+    assert slra.lib().slra_abi_version() == slra.ABI_VERSION == 8
     for s in range(0, 9):
         assert slra.status_string(s) and slra.status_string(s) != "unknown status"
     assert slra.status_string(99) == "unknown status"
@@ -220,6 +220,10 @@ def test_host_entry_point_rejects_strides():
     assert s == slra.ERR_INVALID_ARG
 
 
+def args_g(*a):
+    return a
+
+
 def test_train_forward_and_saved_backward_validation():
     """slra_attn_fwd_train wants a backward-sized workspace and the backward's options; both new entry
     points check their arguments before looking for a device."""
@@ -246,10 +250,25 @@ def test_train_forward_and_saved_backward_validation():
     assert L.slra_attn_fwd_train(ctypes.byref(pc), q, k, v, A, out, ws + 16, bwd_b, None) == slra.ERR_WORKSPACE
     assert L.slra_attn_fwd_train(ctypes.byref(pc), q, k, v, A, out, ws, bwd_b, None) == slra.ERR_NO_DEVICE
     # options the backward does not cover are refused by the training forward too
+    # the gated fusion: covered too (its backward also wants the gate gradients' outputs)
     pg = slra.Problem.from_workload(W.TINY).c()
     pg.fusion = slra.FUSION_GATED
-    pg.gate_w = dA  # an aligned pointer: the option is refused before anything is read
-    assert L.slra_attn_fwd_train(ctypes.byref(pg), q, k, v, A, out, ws, bwd_b, None) == slra.ERR_UNSUPPORTED
+    pg.gate_w = dA
+    bwd_g = L.slra_bwd_workspace_bytes(ctypes.byref(pg))
+    assert bwd_g > bwd_b  # O_lr, dO_lr and the gate's partial sums
+    gbuf = ctypes.create_string_buffer(bwd_g + 256)
+    gws = (ctypes.addressof(gbuf) + 255) // 256 * 256
+    assert L.slra_attn_fwd_train(ctypes.byref(pg), q, k, v, A, out, gws, bwd_g, None) == slra.ERR_NO_DEVICE
+    assert L.slra_attn_bwd(ctypes.byref(pg), *args_g(q, k, v, A, dout, dq, dk, dv, dA), gws, bwd_g,
+                           None) == slra.ERR_INVALID_ARG  # no dgate_w / dgate_b
+    gw_buf = ctypes.create_string_buffer(64 * 4 + 256 + 16)
+    pg.dgate_w = (ctypes.addressof(gw_buf) + 255) // 256 * 256
+    pg.dgate_b = pg.dgate_w + 64 * 4
+    assert L.slra_attn_bwd(ctypes.byref(pg), *args_g(q, k, v, A, dout, dq, dk, dv, dA), gws, bwd_g,
+                           None) == slra.ERR_NO_DEVICE
+    pg.dgate_b = pg.dgate_w + 8  # overlaps dgate_w
+    assert L.slra_attn_bwd(ctypes.byref(pg), *args_g(q, k, v, A, dout, dq, dk, dv, dA), gws, bwd_g,
+                           None) == slra.ERR_INVALID_ARG
     # the feature maps, RoPE orderings and projection layouts are covered: they reach the device check
     for field, value in (("activation", slra.ACT_SILU), ("lowrank_rope_inside", 1), ("lowrank_norope", 1)):
         po = slra.Problem.from_workload(W.TINY).c()

@@ -303,3 +303,95 @@ def test_saved_backward_with_options():
     assert slra.device_status(ws) == slra.OK
     for a, b in zip(got, ref):
         assert torch.equal(a, b)
+
+
+# ---- the gated fusion (RoLA 4.4 as the forward reads it): gradients of q, k, v, A and of Wg, bg
+
+def _gate_params(w, bias, seed=77):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal(w.head_dim) / np.sqrt(w.head_dim)).astype(np.float32), float(bias)
+
+
+def _gated_case(w, label, bias, activation=slra.ACT_RELU, separate=0, per_head=0, nonneg=False):
+    import torch
+    import oracle
+    from oracle import backward as OB
+    x = I.make_inputs(w)
+    if separate or per_head:
+        x["A"] = I.make_projections(w.seed + 5000, w.heads, w.head_dim, w.rank, bool(separate), bool(per_head))
+    if nonneg:
+        x = _nonneg(x)
+    gw, gb = _gate_params(w, bias)
+    dout = I.make_dout(w.seed + 9000, w.batch, w.L, w.heads, w.head_dim)
+    dgw = torch.empty(w.head_dim, dtype=torch.float32, device="cuda")
+    dgb = torch.empty(1, dtype=torch.float32, device="cuda")
+    p = slra.Problem.from_workload(w, fusion=slra.FUSION_GATED, gate_bias=gb, gate_w=torch.from_numpy(gw).cuda(),
+                                   activation=activation, proj_separate=separate, proj_per_head=per_head,
+                                   dgate_w=dgw, dgate_b=dgb)
+    q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
+    dq, dk, dv, dA, ws = slra.attn_bwd(p, q, k, v, A, torch.from_numpy(dout).cuda())
+    assert slra.device_status(ws) == slra.OK
+    idx = slra.ws_view(p, ws, "idx").cpu().numpy()
+    got = [t.cpu().numpy().astype(np.float64) for t in (dq, dk, dv, dA)]
+    B, L, Hh, D = x["q"].shape
+    nh = Hh if per_head else 1
+    P = oracle.decode_bf16(x["A"]).reshape(1 + separate, nh, D, w.rank)
+    ref = [np.zeros((B, L, Hh, D)) for _ in range(3)] + [np.zeros((1 + separate, nh, D, w.rank))]
+    rgw, rgb = np.zeros(D), 0.0
+    for b in range(B):
+        for h in range(Hh):
+            hp = h if per_head else 0
+            r = OB.head_backward(oracle.decode_bf16(x["q"][b, :, h]), oracle.decode_bf16(x["k"][b, :, h]),
+                                 oracle.decode_bf16(x["v"][b, :, h]), P[0, hp], dout[b, :, h].astype(np.float64),
+                                 (w.T, w.H, w.W), w.block, w.keep_frac, w.rank, idx=idx[b * Hh + h],
+                                 activation=activation, A_k=P[1, hp] if separate else None,
+                                 gate=(gw.astype(np.float64), gb))
+            ref[0][b, :, h], ref[1][b, :, h], ref[2][b, :, h] = r["dq"], r["dk"], r["dv"]
+            ref[3][0, hp] += r["dA"]
+            if separate:
+                ref[3][1, hp] += r["dA_k"]
+            rgw += r["dgate_w"]
+            rgb += float(r["dgate_b"])
+    if not separate and not per_head:
+        ref[3] = ref[3].reshape(D, w.rank)
+    _compare(label, got, ref)
+    # [dWg, dbg] as one vector (compared under the first name of the report)
+    _compare(label + "-gate", [np.concatenate([dgw.cpu().numpy().astype(np.float64), dgb.cpu().numpy()])],
+             [np.concatenate([rgw, [rgb]])])
+    return p, (q, k, v, A), dout
+
+
+@pytest.mark.parametrize("bias", [-2.0, 0.5])
+@pytest.mark.parametrize("w", [W.TINY, EDGE_128, EDGE_128_B64], ids=lambda w: w.name)
+def test_backward_gated_fusion(w, bias):
+    """dq, dk, dv, dA and the gate's dWg, dbg on every low-rank path, a closed-ish and an open gate."""
+    _gated_case(w, f"{w.name}-gated{bias}", bias)
+
+
+def test_backward_gated_with_other_options():
+    """The gate together with SiLU features and separate per-head projections (8 heads, tensor cores)."""
+    _gated_case(EDGE_PROJ, "proj-gated-silu", -1.0, activation=slra.ACT_SILU, separate=1, per_head=1, nonneg=True)
+
+
+def test_saved_backward_gated():
+    """The training pair with the gated fusion: forward output and every gradient bit for bit those of
+    the forward and the recomputing backward."""
+    import torch
+    w = EDGE_128
+    x = I.make_inputs(w)
+    gw, gb = _gate_params(w, -1.0)
+    dout = torch.from_numpy(I.make_dout(w.seed + 9100, w.batch, w.L, w.heads, w.head_dim)).cuda()
+    g1 = (torch.empty(w.head_dim, device="cuda"), torch.empty(1, device="cuda"))
+    g2 = (torch.empty(w.head_dim, device="cuda"), torch.empty(1, device="cuda"))
+    kw = dict(fusion=slra.FUSION_GATED, gate_bias=gb, gate_w=torch.from_numpy(gw).cuda())
+    q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
+    p1 = slra.Problem.from_workload(w, dgate_w=g1[0], dgate_b=g1[1], **kw)
+    p2 = slra.Problem.from_workload(w, dgate_w=g2[0], dgate_b=g2[1], **kw)
+    out_ref = slra.attn_fwd(p1, q, k, v, A)[0]
+    out_t, ws = slra.attn_fwd_train(p2, q, k, v, A)
+    assert torch.equal(out_t, out_ref)
+    ref = slra.attn_bwd(p1, q, k, v, A, dout)[:4]
+    got = slra.attn_bwd_saved(p2, q, k, v, A, dout, ws)[:4]
+    assert slra.device_status(ws) == slra.OK
+    for a, b in zip(got + g2, ref + g1):
+        assert torch.equal(a, b)
