@@ -441,12 +441,15 @@ def run_backward(args, w):
     for e in ev:
         e.record()
     torch.cuda.synchronize()
-    x = I.make_inputs(w)
-    q, k, v, A = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v", "A"))
+    import dataclasses
+    # the run's options (feature map, RoPE ordering, projections, gated fusion) as for the forward
+    x, var, prob, (q, k, v, A) = _problem(args, w, slra, dev, torch, ev)
     dout = torch.from_numpy(I.make_dout(w.seed + 9000, w.batch, w.L, w.heads, w.head_dim)).to(dev)
-    prob = slra.Problem.from_workload(w, stage_events=tuple(e.cuda_event for e in ev))
+    if prob.fusion == slra.FUSION_GATED:
+        prob = dataclasses.replace(prob, dgate_w=torch.empty(w.head_dim, dtype=torch.float32, device=dev),
+                                   dgate_b=torch.empty(1, dtype=torch.float32, device=dev))
     grads = tuple(torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
-                  for _ in range(3)) + (torch.empty((w.head_dim, w.rank), dtype=torch.float32, device=dev),)
+                  for _ in range(3)) + (torch.empty(prob.projection_shape, dtype=torch.float32, device=dev),)
     ws = torch.empty(slra.bwd_workspace_bytes(prob), dtype=torch.uint8, device=dev)
     for _ in range(max(3, args.warmup)):
         slra.attn_bwd(prob, q, k, v, A, dout, grads=grads, workspace=ws)
@@ -470,7 +473,7 @@ def run_backward(args, w):
         stages.append([ev[i].elapsed_time(ev[i + 1]) for i in range(6)])
     # A training step: the forward that keeps its state (slra_attn_fwd_train), then the backward from it
     # (slra_attn_bwd_saved), with no recompute.
-    prob_f = slra.Problem.from_workload(w)
+    prob_f = dataclasses.replace(prob, stage_events=(None,) * 7)
     out = torch.empty((w.batch, w.L, w.heads, w.head_dim), dtype=torch.float32, device=dev)
     for _ in range(max(3, args.warmup)):
         slra.attn_fwd_train(prob_f, q, k, v, A, out=out, workspace=ws)
@@ -501,7 +504,9 @@ def run_backward(args, w):
     f_bwd_sparse = 2.5 * f_sparse
     f_lr_bwd = 2.0 * F.lowrank_flops(w.L, w.rank, w.head_dim, w.batch * w.heads)  # ~2x the forward's chain
     sparse_ms = st[2] + st[3]
-    line = {"backward": w.name, "ms_per_call": ms, "keep_blocks": keep_blocks,
+    line = {"backward": w.name, "options": {k_: (v_ if not isinstance(v_, tuple) else "gated")
+                                            for k_, v_ in var.items() if k_ != "gate" or v_ is not None},
+            "ms_per_call": ms, "keep_blocks": keep_blocks,
             "stage_ms": dict(zip(("recompute_forward", "dout_copy_and_lists", "dq_kernel", "dkdv_kernel",
                                   "lowrank_grad", "-"), (round(x_, 4) for x_ in st))),
             "sparse_bwd": {"algorithmic_flops": f_bwd_sparse, "ms": sparse_ms,
