@@ -257,7 +257,7 @@ inline bool lr_bwd_on_tensor_cores(const Geom& g) { return g.D == 128 && g.R <= 
 int lr_bwd_nsplit(const Geom& g);
 
 // ---- backward of the gated fusion (gate_bwd.cu) -------------------------------------------------
-constexpr int kGateParts = 296;  // CTAs (and partial sums) of the gate-parameter reduction
+constexpr int kGateParts = 148 * 8;  // CTAs (and partial sums) of the gate-parameter reduction
 // dO_s (fp16 head-major copy and Delta), dO_lr (fp32 token-major) and dlogit per row from dout, O_s and
 // O_lr (head-major fp32) and the raw queries.
 cudaError_t launch_gate_prep(const float* dout, const float* os, const float* olr, const __nv_bfloat16* q,

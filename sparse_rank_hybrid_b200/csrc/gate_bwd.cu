@@ -84,10 +84,14 @@ __global__ void bwd_gate_prep_kernel(const float* __restrict__ dout, const float
 }
 
 // dq += dlogit Wg on every row, and per-CTA partial sums of dWg = sum dlogit q and dbg = sum dlogit
-// over a fixed range of rows, in a fixed order (thread = column of a row stream).
-__global__ void bwd_gate_final_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ dlogit,
-                                      const float* __restrict__ gate_w, Geom g, long long rows_per_cta,
-                                      float* __restrict__ dq, float* __restrict__ part) {
+// over a fixed range of rows, in a fixed order (thread = column of a row stream; four rows of a stream
+// in flight at a time).
+__global__ void __launch_bounds__(256) bwd_gate_final_kernel(const __nv_bfloat16* __restrict__ q,
+                                                             const float* __restrict__ dlogit,
+                                                             const float* __restrict__ gate_w, Geom g,
+                                                             long long rows_per_cta, float* __restrict__ dq,
+                                                             float* __restrict__ part) {
+    constexpr int U = 4;
     __shared__ float red[256 + 8];
     const int tid = threadIdx.x, col = tid % g.D, rs = tid / g.D, nstream = blockDim.x / g.D;
     const long long rows = static_cast<long long>(g.BH()) * g.L;
@@ -95,14 +99,30 @@ __global__ void bwd_gate_final_kernel(const __nv_bfloat16* __restrict__ q, const
     const long long r1 = r0 + rows_per_cta < rows ? r0 + rows_per_cta : rows;
     const float wg = __ldg(gate_w + col);
     float acc = 0.f, accb = 0.f;
-    for (long long r = r0 + rs; r < r1; r += nstream) {
-        const int bh = static_cast<int>(r / g.L), n = static_cast<int>(r % g.L);
-        const int b = bh / g.Hh, h = bh % g.Hh;
-        const float d = dlogit[static_cast<size_t>(bh) * g.Lp + n];
-        acc = fmaf(d, __bfloat162float(q[g.sq.row(b, n, h) + col]), acc);
-        accb += d;
-        float* o = dq + g.so.row(b, n, h) + col;
-        *o = fmaf(d, wg, *o);
+    for (long long rb = r0 + rs; rb < r1; rb += U * nstream) {
+        float dl[U], qv[U], prev[U];
+        float* dst[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long r = rb + u * nstream;
+            dst[u] = nullptr;
+            dl[u] = qv[u] = prev[u] = 0.f;
+            if (r < r1) {
+                const int bh = static_cast<int>(r / g.L), n = static_cast<int>(r % g.L);
+                const int b = bh / g.Hh, h = bh % g.Hh;
+                dl[u] = dlogit[static_cast<size_t>(bh) * g.Lp + n];
+                qv[u] = __bfloat162float(q[g.sq.row(b, n, h) + col]);
+                dst[u] = dq + g.so.row(b, n, h) + col;
+                prev[u] = *dst[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (dst[u] == nullptr) continue;
+            acc = fmaf(dl[u], qv[u], acc);
+            accb += dl[u];
+            *dst[u] = fmaf(dl[u], wg, prev[u]);
+        }
     }
     red[tid] = acc;
     if (col == 0) red[256 + rs] = accb;

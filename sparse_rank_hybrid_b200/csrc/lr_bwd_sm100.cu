@@ -127,14 +127,16 @@ __device__ __forceinline__ void build_dk_image(uint8_t* hi_img, uint8_t* lo_img,
 
 }  // namespace
 
-// kKey = false: the query pass; true: the key pass.
-template <int R, bool kKey>
+// kKey = false: the query pass; true: the key pass.  kRelu: relu features with the RoPE outside the
+// activation (the other feature maps' out-of-line code then drops out at compile time).
+template <int R, bool kKey, bool kRelu>
 __global__ void __launch_bounds__(256, 1)
     lr_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
                         const __grid_constant__ CUtensorMap tm_o0, const __grid_constant__ CUtensorMap tm_o1,
                         LrTcBwdArgs a, Geom g) {
     using Lay = LbLayout<R>;
     constexpr int RH = R / 2;  // features per thread
+    const int act = kRelu ? 0 : g.act, inside = kRelu ? 0 : g.inside;
     static_assert(R % 16 == 0 && R <= 48, "rank 16..48 (rank 64's operands do not fit the shared memory)");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -226,6 +228,17 @@ __global__ void __launch_bounds__(256, 1)
                     if (kKey) tma_load_4d(smem + Lay::kOffY + x * kSlab, &tm_y, bar_ld, x * 64, h, tile * kTok, b);
                 }
                 ++n_ld_issued;
+                // the next tile's inputs towards L2 while this one is computed
+                if (tile + 1 < t1)
+                    for (int x = 0; x < 2; ++x) {
+                        tma_prefetch_l2_4d(&tm_x, x * 64, h, (tile + 1) * kTok, b);
+                        if (kKey) tma_prefetch_l2_4d(&tm_y, x * 64, h, (tile + 1) * kTok, b);
+                    }
+            }
+            if (!kKey && tile + 1 < t1 && n + kTok < g.L) {  // and the next tile's dO rows
+                const float* nxt = a.dout + g.so.row(b, n + kTok, h) + half * 64;
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt + 32));
             }
             if constexpr (!kKey) {
                 const float* src = a.dout + g.so.row(b, live ? n : 0, h) + half * 64;
@@ -330,7 +343,7 @@ __global__ void __launch_bounds__(256, 1)
                 float den_p = 0.f, dot_p = 0.f;
 #pragma unroll
                 for (int pp = 0; pp < RH / 2; ++pp) {
-                    const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], g.act, g.inside);
+                    const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], act, inside);
                     den_p = fmaf(P.nf0, zr[2 * pp], fmaf(P.nf1, zr[2 * pp + 1], den_p));
                     dot_p = fmaf(P.psi0, gv[2 * pp], fmaf(P.psi1, gv[2 * pp + 1], dot_p));
                 }
@@ -342,10 +355,10 @@ __global__ void __launch_bounds__(256, 1)
                 const float dden = live ? -dot / (den * den) : 0.f;
 #pragma unroll
                 for (int pp = 0; pp < RH / 2; ++pp) {
-                    const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], g.act, g.inside);
+                    const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], act, inside);
                     float du0, du1;
                     lr_pair_bwd(P, gv[2 * pp] / den, gv[2 * pp + 1] / den, dden * zr[2 * pp], dden * zr[2 * pp + 1],
-                                cf[pp], sf[pp], g.inside, du0, du1);
+                                cf[pp], sf[pp], inside, du0, du1);
                     du[2 * pp] = live ? du0 : 0.f;
                     du[2 * pp + 1] = live ? du1 : 0.f;
                     w[2 * pp] = live ? P.psi0 / den : 0.f;
@@ -356,11 +369,11 @@ __global__ void __launch_bounds__(256, 1)
             } else {
 #pragma unroll
                 for (int pp = 0; pp < RH / 2; ++pp) {
-                    const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], g.act, g.inside);
+                    const LrPair P = lr_pair_fwd(u[2 * pp], u[2 * pp + 1], cf[pp], sf[pp], act, inside);
                     w[2 * pp] = live ? P.psi0 : 0.f;  // psi, the A operand of dv
                     w[2 * pp + 1] = live ? P.psi1 : 0.f;
                     float du0, du1;
-                    lr_pair_bwd(P, gv[2 * pp], gv[2 * pp + 1], zr[2 * pp], zr[2 * pp + 1], cf[pp], sf[pp], g.inside,
+                    lr_pair_bwd(P, gv[2 * pp], gv[2 * pp + 1], zr[2 * pp], zr[2 * pp + 1], cf[pp], sf[pp], inside,
                                 du0, du1);
                     du[2 * pp] = live ? du0 : 0.f;
                     du[2 * pp + 1] = live ? du1 : 0.f;
@@ -544,21 +557,22 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 namespace {
-template <int R>
+template <int R, bool kRelu>
 cudaError_t launch_lr_bwd_tc_r(const LrTcBwdArgs& a, const Geom& g, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const CUtensorMap& tdq, const CUtensorMap& tdk,
                                const CUtensorMap& tdv, float* dS, float* dz, long long key_off, cudaStream_t st) {
     const size_t sm = static_cast<size_t>(LbLayout<R>::kBytes) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(lr_bwd_sm100_kernel<R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    cudaError_t e = cudaFuncSetAttribute(lr_bwd_sm100_kernel<R, false, kRelu>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(lr_bwd_sm100_kernel<R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    e = cudaFuncSetAttribute(lr_bwd_sm100_kernel<R, true, kRelu>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int items = g.BH() * a.nsplit;
     const int grid = items < sms ? items : sms;
-    lr_bwd_sm100_kernel<R, false><<<grid, 256, sm, st>>>(tq, tq, tdq, tdq, a, g);
+    lr_bwd_sm100_kernel<R, false, kRelu><<<grid, 256, sm, st>>>(tq, tq, tdq, tdq, a, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_lowrank_reduce(a.ds_part, a.dz_part, g, a.nsplit, dS, dz, nullptr, nullptr, nullptr, st)) !=
         cudaSuccess)
@@ -568,7 +582,7 @@ cudaError_t launch_lr_bwd_tc_r(const LrTcBwdArgs& a, const Geom& g, const CUtens
     ak.dS = dS;
     ak.dz = dz;
     ak.da_part = a.da_part + static_cast<size_t>(g.BH()) * a.nsplit * kD * R;
-    lr_bwd_sm100_kernel<R, true><<<grid, 256, sm, st>>>(tk, tv, tdv, tdk, ak, g);
+    lr_bwd_sm100_kernel<R, true, kRelu><<<grid, 256, sm, st>>>(tk, tv, tdv, tdk, ak, g);
     return cudaGetLastError();
 }
 }  // namespace
@@ -606,10 +620,18 @@ cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st)
     a.status = l.status;
     a.timeout_ns = l.timeout_ns;
     a.accumulate = l.accumulate;
+    const bool relu = g.act == 0 && !g.inside;
+    const long long koff = l.key_proj_offset(g);
     switch (g.R) {
-        case 16: return launch_lr_bwd_tc_r<16>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, l.key_proj_offset(g), st);
-        case 32: return launch_lr_bwd_tc_r<32>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, l.key_proj_offset(g), st);
-        case 48: return launch_lr_bwd_tc_r<48>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, l.key_proj_offset(g), st);
+        case 16:
+            return relu ? launch_lr_bwd_tc_r<16, true>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st)
+                        : launch_lr_bwd_tc_r<16, false>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st);
+        case 32:
+            return relu ? launch_lr_bwd_tc_r<32, true>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st)
+                        : launch_lr_bwd_tc_r<32, false>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st);
+        case 48:
+            return relu ? launch_lr_bwd_tc_r<48, true>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st)
+                        : launch_lr_bwd_tc_r<48, false>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st);
     }
     return cudaErrorInvalidValue;
 }
