@@ -1409,34 +1409,47 @@ __global__ void __launch_bounds__(256) bwd_lr_k_tiled_kernel(const __nv_bfloat16
     for (int i = 0; i < NA; ++i) da_part[slot * D * R + e_own * R + cg * NA + i] = acc_a[i];
 }
 
-// dA [1 + sep][per_head ? Hh : 1][D][R] from the partials [2 passes][B * Hh][ns][D][R], in a fixed order
-// (pass, batch, head, split): each projection sums the passes that used it (the query pass for Pq, the
-// key pass for Pk, both when they are one matrix) over the heads that share it and every split.
-__global__ void bwd_da_reduce_kernel(const float* __restrict__ da_part, Geom g, int ns, int sep, int per_head,
-                                     float* __restrict__ dA) {
+// dA [1 + sep][per_head ? Hh : 1][D][R] from the partials [2 passes][B * Hh][ns][D][R]: each projection
+// sums the passes that used it (the query pass for Pq, the key pass for Pk, both when they are one
+// matrix) over the heads that share it and every split.  A CTA takes 32 consecutive outputs; its 8 warps
+// each sum every 8th partial of the fixed (pass, batch, head, split) order, and the 8 sums are added in
+// warp order: deterministic, with 8 loads of 128 bytes in flight per output group.
+__global__ void __launch_bounds__(256) bwd_da_reduce_kernel(const float* __restrict__ da_part, Geom g, int ns,
+                                                            int sep, int per_head, float* __restrict__ dA) {
+    __shared__ float red[8][32];
     const int DR = g.D * g.R;
     const int nh = per_head ? g.Hh : 1;
-    const int o = blockIdx.x * blockDim.x + threadIdx.x;
-    if (o >= (1 + sep) * nh * DR) return;
-    const int e = o % DR, hh = (o / DR) % nh, pj = o / (DR * nh);
+    const int lo = threadIdx.x & 31, sl = threadIdx.x >> 5;
+    const int o = blockIdx.x * 32 + lo;
+    const int n_out = (1 + sep) * nh * DR;
     float s = 0.f;
-    for (int pass = 0; pass < 2; ++pass) {
-        if (sep && pass != pj) continue;
-        for (int b = 0; b < g.B; ++b)
-            for (int h = 0; h < g.Hh; ++h) {
-                if (per_head && h != hh) continue;
-                const size_t slot0 = (static_cast<size_t>(pass) * g.BH() + b * g.Hh + h) * ns;
-                for (int sp = 0; sp < ns; ++sp) s += da_part[(slot0 + sp) * DR + e];
-            }
+    if (o < n_out) {
+        const int e = o % DR, hh = (o / DR) % nh, pj = o / (DR * nh);
+        const int npass = sep ? 1 : 2, nheads = per_head ? 1 : g.Hh;
+        const int per_pass = g.B * nheads * ns, total = npass * per_pass;
+        for (int t = sl; t < total; t += 8) {
+            const int pass = sep ? pj : t / per_pass;
+            const int rem = t % per_pass;
+            const int b = rem / (nheads * ns), rem2 = rem % (nheads * ns);
+            const int h = per_head ? hh : rem2 / ns, sp = rem2 % ns;
+            s += da_part[((static_cast<size_t>(pass) * g.BH() + b * g.Hh + h) * ns + sp) * DR + e];
+        }
     }
-    dA[o] = s;
+    red[sl][lo] = s;
+    __syncthreads();
+    if (sl == 0 && o < n_out) {
+        float t = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t += red[i][lo];
+        dA[o] = t;
+    }
 }
 
 namespace {
 cudaError_t launch_da_reduce(const LrBwdArgs& l, const Geom& g, cudaStream_t st) {
     const int n = (1 + l.proj_separate) * (l.proj_per_head ? g.Hh : 1) * g.D * g.R;
-    bwd_da_reduce_kernel<<<(n + 255) / 256, 256, 0, st>>>(l.da_part, g, l.nsplit, l.proj_separate, l.proj_per_head,
-                                                           l.dA);
+    bwd_da_reduce_kernel<<<(n + 31) / 32, 256, 0, st>>>(l.da_part, g, l.nsplit, l.proj_separate, l.proj_per_head,
+                                                         l.dA);
     return cudaGetLastError();
 }
 }  // namespace

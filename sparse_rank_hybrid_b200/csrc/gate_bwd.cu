@@ -99,21 +99,28 @@ __global__ void __launch_bounds__(256) bwd_gate_final_kernel(const __nv_bfloat16
     const long long r1 = r0 + rows_per_cta < rows ? r0 + rows_per_cta : rows;
     const float wg = __ldg(gate_w + col);
     float acc = 0.f, accb = 0.f;
-    for (long long rb = r0 + rs; rb < r1; rb += U * nstream) {
+    // (head, token) of this thread's next row, advanced incrementally (no 64-bit division in the loop)
+    long long r = r0 + rs;
+    int bh = static_cast<int>(r / g.L), n = static_cast<int>(r % g.L);
+    while (r < r1) {
         float dl[U], qv[U], prev[U];
         float* dst[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const long long r = rb + u * nstream;
             dst[u] = nullptr;
             dl[u] = qv[u] = prev[u] = 0.f;
             if (r < r1) {
-                const int bh = static_cast<int>(r / g.L), n = static_cast<int>(r % g.L);
                 const int b = bh / g.Hh, h = bh % g.Hh;
                 dl[u] = dlogit[static_cast<size_t>(bh) * g.Lp + n];
                 qv[u] = __bfloat162float(q[g.sq.row(b, n, h) + col]);
                 dst[u] = dq + g.so.row(b, n, h) + col;
                 prev[u] = *dst[u];
+            }
+            r += nstream;
+            n += nstream;
+            while (n >= g.L) {
+                n -= g.L;
+                ++bh;
             }
         }
 #pragma unroll
