@@ -15,7 +15,8 @@ namespace {
 
 // One warp per row (b, h, n) of the padded head-major grid: O_s and O_lr head-major fp32, dout and
 // dO_lr token-major fp32, the fp16 copy of dO_s head-major (rows past L zero).
-__global__ void bwd_gate_prep_kernel(const float* __restrict__ dout, const float* __restrict__ os,
+template <int D>
+__global__ void __launch_bounds__(256) bwd_gate_prep_kernel(const float* __restrict__ dout, const float* __restrict__ os,
                                      const float* __restrict__ olr, const __nv_bfloat16* __restrict__ q,
                                      const float* __restrict__ gate_w, float gate_b, Geom g,
                                      __half* __restrict__ doh, float* __restrict__ delta, float* __restrict__ dolr,
@@ -26,8 +27,8 @@ __global__ void bwd_gate_prep_kernel(const float* __restrict__ dout, const float
     if (warp >= rows) return;
     const int bh = static_cast<int>(warp / g.Lp), n = static_cast<int>(warp % g.Lp);
     const int b = bh / g.Hh, h = bh % g.Hh;
-    const int per = g.D / 32;  // elements per lane: 2 or 4
-    __half* dst = doh + static_cast<size_t>(warp) * g.D + lane * per;
+    constexpr int per = D / 32;  // elements per lane: 2 or 4
+    __half* dst = doh + static_cast<size_t>(warp) * D + lane * per;
     if (n >= g.L) {
         for (int e = 0; e < per; e += 2) *reinterpret_cast<__half2*>(dst + e) = __floats2half2_rn(0.f, 0.f);
         if (lane == 0) {
@@ -36,20 +37,28 @@ __global__ void bwd_gate_prep_kernel(const float* __restrict__ dout, const float
         }
         return;
     }
-    float x[4], s[4], l[4];
+    float x[per], s[per], l[per], qf[per];
     float ss_s = 0.f, ss_l = 0.f, t = 0.f, qw = 0.f;
     const float* src = dout + g.so.row(b, n, h) + lane * per;
-    const float* so = os + static_cast<size_t>(warp) * g.D + lane * per;
-    const float* sl = olr + static_cast<size_t>(warp) * g.D + lane * per;
+    const float* so = os + static_cast<size_t>(warp) * D + lane * per;
+    const float* sl = olr + static_cast<size_t>(warp) * D + lane * per;
     const __nv_bfloat16* sq = q + g.sq.row(b, n, h) + lane * per;
+#pragma unroll
+    for (int e = 0; e < per; e += 2) {  // 8-byte loads (the rows are 16-byte aligned)
+        const float2 x2 = *reinterpret_cast<const float2*>(src + e), s2 = *reinterpret_cast<const float2*>(so + e),
+                     l2 = *reinterpret_cast<const float2*>(sl + e);
+        const float2 q2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sq + e));
+        x[e] = x2.x; x[e + 1] = x2.y;
+        s[e] = s2.x; s[e + 1] = s2.y;
+        l[e] = l2.x; l[e + 1] = l2.y;
+        qf[e] = q2.x; qf[e + 1] = q2.y;
+    }
+#pragma unroll
     for (int e = 0; e < per; ++e) {
-        x[e] = src[e];
-        s[e] = so[e];
-        l[e] = sl[e];
         ss_s = fmaf(s[e], s[e], ss_s);
         ss_l = fmaf(l[e], l[e], ss_l);
         t = fmaf(x[e], l[e], t);
-        qw = fmaf(__bfloat162float(sq[e]), __ldg(gate_w + lane * per + e), qw);
+        qw = fmaf(qf[e], __ldg(gate_w + lane * per + e), qw);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -58,7 +67,7 @@ __global__ void bwd_gate_prep_kernel(const float* __restrict__ dout, const float
         t += __shfl_xor_sync(0xffffffffu, t, o);
         qw += __shfl_xor_sync(0xffffffffu, qw, o);
     }
-    const float inv_d = 1.f / static_cast<float>(g.D);
+    const float inv_d = 1.f / static_cast<float>(D);
     const float a = sqrtf(ss_s * inv_d), bb = sqrtf(ss_l * inv_d + 1e-6f);
     const float gg = 1.f / (1.f + expf(-(qw + gate_b)));
     const float c = gg * a / bb;
@@ -67,6 +76,7 @@ __global__ void bwd_gate_prep_kernel(const float* __restrict__ dout, const float
     float dsum = 0.f;
     bool bad = false;
     float* dl = dolr + g.so.row(b, n, h) + lane * per;
+#pragma unroll
     for (int e = 0; e < per; e += 2) {
         const float d0 = fmaf(ks, s[e], x[e]), d1 = fmaf(ks, s[e + 1], x[e + 1]);
         dsum = fmaf(d0, s[e], fmaf(d1, s[e + 1], dsum));
@@ -84,40 +94,58 @@ __global__ void bwd_gate_prep_kernel(const float* __restrict__ dout, const float
 }
 
 // dq += dlogit Wg on every row, and per-CTA partial sums of dWg = sum dlogit q and dbg = sum dlogit
-// over a fixed range of rows, in a fixed order (thread = column of a row stream; four rows of a stream
-// in flight at a time).
+// over a fixed range of rows, in a fixed order.  A warp takes a row (each lane D/32 consecutive
+// columns, vector loads and stores), the CTA's 8 warps 8 rows at a time, four such steps in flight.
+template <int D>
 __global__ void __launch_bounds__(256) bwd_gate_final_kernel(const __nv_bfloat16* __restrict__ q,
                                                              const float* __restrict__ dlogit,
                                                              const float* __restrict__ gate_w, Geom g,
                                                              long long rows_per_cta, float* __restrict__ dq,
                                                              float* __restrict__ part) {
-    constexpr int U = 4;
-    __shared__ float red[256 + 8];
-    const int tid = threadIdx.x, col = tid % g.D, rs = tid / g.D, nstream = blockDim.x / g.D;
+    constexpr int P = D / 32, U = 4, NW = 8;
+    __shared__ float red[NW][D + 1];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const long long rows = static_cast<long long>(g.BH()) * g.L;
     const long long r0 = blockIdx.x * rows_per_cta;
     const long long r1 = r0 + rows_per_cta < rows ? r0 + rows_per_cta : rows;
-    const float wg = __ldg(gate_w + col);
-    float acc = 0.f, accb = 0.f;
-    // (head, token) of this thread's next row, advanced incrementally (no 64-bit division in the loop)
-    long long r = r0 + rs;
+    float wg[P], acc[P];
+#pragma unroll
+    for (int e = 0; e < P; ++e) {
+        wg[e] = __ldg(gate_w + lane * P + e);
+        acc[e] = 0.f;
+    }
+    float accb = 0.f;
+    // (head, token) of this warp's next row, advanced incrementally (no 64-bit division in the loop)
+    long long r = r0 + wid;
     int bh = static_cast<int>(r / g.L), n = static_cast<int>(r % g.L);
     while (r < r1) {
-        float dl[U], qv[U], prev[U];
+        float dl[U], qv[U][P], pv[U][P];
         float* dst[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             dst[u] = nullptr;
-            dl[u] = qv[u] = prev[u] = 0.f;
+            dl[u] = 0.f;
             if (r < r1) {
                 const int b = bh / g.Hh, h = bh % g.Hh;
                 dl[u] = dlogit[static_cast<size_t>(bh) * g.Lp + n];
-                qv[u] = __bfloat162float(q[g.sq.row(b, n, h) + col]);
-                dst[u] = dq + g.so.row(b, n, h) + col;
-                prev[u] = *dst[u];
+                const __nv_bfloat16* qs = q + g.sq.row(b, n, h) + lane * P;
+                dst[u] = dq + g.so.row(b, n, h) + lane * P;
+                if constexpr (P == 4) {
+                    const uint2 raw = *reinterpret_cast<const uint2*>(qs);
+                    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+                    const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+                    qv[u][0] = a0.x; qv[u][1] = a0.y; qv[u][2] = a1.x; qv[u][3] = a1.y;
+                    const float4 o = *reinterpret_cast<const float4*>(dst[u]);
+                    pv[u][0] = o.x; pv[u][1] = o.y; pv[u][2] = o.z; pv[u][3] = o.w;
+                } else {
+                    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qs));
+                    qv[u][0] = a0.x; qv[u][1] = a0.y;
+                    const float2 o = *reinterpret_cast<const float2*>(dst[u]);
+                    pv[u][0] = o.x; pv[u][1] = o.y;
+                }
             }
-            r += nstream;
-            n += nstream;
+            r += NW;
+            n += NW;
             while (n >= g.L) {
                 n -= g.L;
                 ++bh;
@@ -126,24 +154,28 @@ __global__ void __launch_bounds__(256) bwd_gate_final_kernel(const __nv_bfloat16
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (dst[u] == nullptr) continue;
-            acc = fmaf(dl[u], qv[u], acc);
+#pragma unroll
+            for (int e = 0; e < P; ++e) {
+                acc[e] = fmaf(dl[u], qv[u][e], acc[e]);
+                pv[u][e] = fmaf(dl[u], wg[e], pv[u][e]);
+            }
             accb += dl[u];
-            *dst[u] = fmaf(dl[u], wg, prev[u]);
+            if constexpr (P == 4)
+                *reinterpret_cast<float4*>(dst[u]) = make_float4(pv[u][0], pv[u][1], pv[u][2], pv[u][3]);
+            else
+                *reinterpret_cast<float2*>(dst[u]) = make_float2(pv[u][0], pv[u][1]);
         }
     }
-    red[tid] = acc;
-    if (col == 0) red[256 + rs] = accb;
+#pragma unroll
+    for (int e = 0; e < P; ++e) red[wid][lane * P + e] = acc[e];
+    if (lane == 0) red[wid][D] = accb;  // every lane of a warp sums the same dlogit values
     __syncthreads();
-    float* mine = part + static_cast<size_t>(blockIdx.x) * (g.D + 1);
-    if (rs == 0) {
-        float s = 0.f;
-        for (int i = 0; i < nstream; ++i) s += red[i * g.D + col];
-        mine[col] = s;
-    }
-    if (tid == 0) {
-        float s = 0.f;
-        for (int i = 0; i < nstream; ++i) s += red[256 + i];
-        mine[g.D] = s;
+    float* mine = part + static_cast<size_t>(blockIdx.x) * (D + 1);
+    for (int c = threadIdx.x; c <= D; c += blockDim.x) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) t += red[w][c];
+        mine[c] = t;
     }
 }
 
@@ -164,8 +196,12 @@ cudaError_t launch_gate_prep(const float* dout, const float* os, const float* ol
                              float* dlogit, int* status, cudaStream_t st) {
     const long long rows = static_cast<long long>(g.BH()) * g.Lp;
     const long long blocks = (rows * 32 + 255) / 256;
-    bwd_gate_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(dout, os, olr, q, gate_w, gate_b, g, doh, delta,
-                                                                        dolr, dlogit, status);
+    if (g.D == 128)
+        bwd_gate_prep_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(dout, os, olr, q, gate_w, gate_b, g,
+                                                                                 doh, delta, dolr, dlogit, status);
+    else
+        bwd_gate_prep_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(dout, os, olr, q, gate_w, gate_b, g,
+                                                                                doh, delta, dolr, dlogit, status);
     return cudaGetLastError();
 }
 
@@ -173,7 +209,8 @@ cudaError_t launch_gate_final(const __nv_bfloat16* q, const float* dlogit, const
                               float* dq, float* part, float* dgw, float* dgb, cudaStream_t st) {
     const long long rows = static_cast<long long>(g.BH()) * g.L;
     const long long per = (rows + kGateParts - 1) / kGateParts;
-    bwd_gate_final_kernel<<<kGateParts, 256, 0, st>>>(q, dlogit, gate_w, g, per, dq, part);
+    if (g.D == 128) bwd_gate_final_kernel<128><<<kGateParts, 256, 0, st>>>(q, dlogit, gate_w, g, per, dq, part);
+    else bwd_gate_final_kernel<64><<<kGateParts, 256, 0, st>>>(q, dlogit, gate_w, g, per, dq, part);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     bwd_gate_reduce_kernel<<<1, 256, 0, st>>>(part, kGateParts, g.D, dgw, dgb);
