@@ -327,10 +327,11 @@ SLRA_API slra_status slra_lowrank_fwd(const slra_tensor* q, const slra_tensor* k
                                       float* z, void* workspace, size_t workspace_bytes, slra_stream_t stream);
 
 /*
- * Workspace bytes of slra_attn_bwd for p (the forward's layout followed by the backward's sections: the
- * recomputed sparse output and its per-row log-sum-exp, an fp16 copy of dout, the inverted kept-block
- * lists and the low-rank gradient partial sums); 0 if p is invalid or asks for an option the backward
- * does not cover.  No GPU access.
+ * Workspace bytes of slra_attn_bwd, slra_attn_bwd_saved and slra_attn_fwd_train for p (the forward's
+ * layout followed by the backward's sections: the sparse output and its per-row log-sum-exp, an fp16
+ * copy of dout, the inverted kept-block lists and the low-rank gradient partial sums; with the gated
+ * fusion also the low-rank output, its gradient and the gate's per-row terms and partial sums); 0 if p
+ * is invalid.  No GPU access.
  */
 SLRA_API size_t slra_bwd_workspace_bytes(const slra_problem* p);
 
