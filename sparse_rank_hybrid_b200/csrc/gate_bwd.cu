@@ -179,14 +179,25 @@ __global__ void __launch_bounds__(256) bwd_gate_final_kernel(const __nv_bfloat16
     }
 }
 
-__global__ void bwd_gate_reduce_kernel(const float* __restrict__ part, int nparts, int D, float* __restrict__ dgw,
-                                       float* __restrict__ dgb) {
-    const int o = threadIdx.x;
-    if (o > D) return;
+// dWg, dbg from the kGateParts partials: a CTA takes 32 consecutive outputs, its 8 warps each sum
+// every 8th partial, and the 8 sums are added in warp order (deterministic).
+__global__ void __launch_bounds__(256) bwd_gate_reduce_kernel(const float* __restrict__ part, int nparts, int D,
+                                                              float* __restrict__ dgw, float* __restrict__ dgb) {
+    __shared__ float red[8][32];
+    const int lo = threadIdx.x & 31, sl = threadIdx.x >> 5;
+    const int o = blockIdx.x * 32 + lo;
     float s = 0.f;
-    for (int i = 0; i < nparts; ++i) s += part[static_cast<size_t>(i) * (D + 1) + o];
-    if (o < D) dgw[o] = s;
-    else *dgb = s;
+    if (o <= D)
+        for (int i = sl; i < nparts; i += 8) s += part[static_cast<size_t>(i) * (D + 1) + o];
+    red[sl][lo] = s;
+    __syncthreads();
+    if (sl == 0 && o <= D) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += red[w][lo];
+        if (o < D) dgw[o] = t;
+        else *dgb = t;
+    }
 }
 
 }  // namespace
@@ -213,7 +224,7 @@ cudaError_t launch_gate_final(const __nv_bfloat16* q, const float* dlogit, const
     else bwd_gate_final_kernel<64><<<kGateParts, 256, 0, st>>>(q, dlogit, gate_w, g, per, dq, part);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_gate_reduce_kernel<<<1, 256, 0, st>>>(part, kGateParts, g.D, dgw, dgb);
+    bwd_gate_reduce_kernel<<<(g.D + 1 + 31) / 32, 256, 0, st>>>(part, kGateParts, g.D, dgw, dgb);
     return cudaGetLastError();
 }
 
