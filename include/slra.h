@@ -355,7 +355,7 @@ SLRA_API size_t slra_bwd_workspace_bytes(const slra_problem* p);
  * over the query blocks that kept it (dV += P^T dO, dK^ += dS^T q^), with fp16 operands (dout must stay
  * below 65504 in magnitude, else SLRA_ERR_RANGE is recorded) and fp32 accumulation; the low-rank chain
  * follows as a pass over the queries and one over the keys (on the tensor cores for head_dim 128 and
- * rank <= 48, fp32 otherwise) that add their parts to dq, dk, dv and produce dA.  With the gated fusion
+ * rank <= 64, fp32 otherwise) that add their parts to dq, dk, dv and produce dA.  With the gated fusion
  * the low-rank branch's output is recomputed too, one pass per row splits dout into the two branches'
  * gradients and the gate's, and a last pass adds the gate's part to dq and reduces dWg, dbg.
  * Deterministic.

@@ -251,9 +251,9 @@ cudaError_t launch_bwd_prep(const float* dout, const float* os, const Geom& g, _
 cudaError_t launch_bwd_invert(const int32_t* idx, const Geom& g, int32_t* inv, int32_t* inv_cnt, cudaStream_t st);
 cudaError_t launch_bwd_sparse(const BwdMaps& m, const BwdArgs& a, const Geom& g, cudaStream_t st);
 cudaError_t launch_lr_bwd(const LrBwdArgs& l, const Geom& g, cudaStream_t st);
-// Tensor-core low-rank gradient passes (head_dim 128, rank <= 48), see lr_bwd_sm100.cu.
+// Tensor-core low-rank gradient passes (head_dim 128, rank <= 64), see lr_bwd_sm100.cu.
 cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st);
-inline bool lr_bwd_on_tensor_cores(const Geom& g) { return g.D == 128 && g.R <= 48; }
+inline bool lr_bwd_on_tensor_cores(const Geom& g) { return g.D == 128 && g.R <= 64; }
 int lr_bwd_nsplit(const Geom& g);
 
 // ---- backward of the gated fusion (gate_bwd.cu) -------------------------------------------------

@@ -1,4 +1,4 @@
-// Gradients of the low-rank branch on the sm_100a tensor cores (head_dim 128, rank <= 48): the
+// Gradients of the low-rank branch on the sm_100a tensor cores (head_dim 128, rank <= 64): the
 // derivative of RoLA "4.1"/"4.2"/"4.3"/"B.1"'s branch (phi = relu(x A), psi = R_r phi outside the
 // activation, S = sum psi_k v^T, z = sum phi_k, O_lr = psi_q S / (phi_q . z + 1e-6)).
 //
@@ -88,9 +88,8 @@ struct LbLayout {
     static constexpr int kOffX = 0;                                 // q or k tile
     static constexpr int kOffY = kTile;                             // query pass: dO hi; key pass: v
     static constexpr int kOffY2 = 2 * kTile;                        // query pass: dO lo; key pass: dS^T images
-    static constexpr int kOffAt = 3 * kTile;                        // A^T image (B of x A)
-    static constexpr int kOffAi = kOffAt + kAtImg;                  // A image [128][64] K-major (B of du A^T)
-    static constexpr int kOffSi = kOffAi + kSlab;                   // S or dS images hi, lo: [R][128] each
+    static constexpr int kOffAt = 3 * kTile;  // A^T image [R][128]: B of x A (K-major), B of du A^T (MN-major)
+    static constexpr int kOffSi = kOffAt + kAtImg;                  // S or dS images hi, lo: [R][128] each
     static constexpr int kOffW = kOffSi + 2 * kAtImg;               // [128][hi 64 | lo 64]: w or psi
     static constexpr int kOffDu = kOffW + kTile;                    // [128][hi 64 | lo 64]: du
     static constexpr int kOffXch = kOffDu + kTile;                  // [2][2][128] fp32 row partials
@@ -137,7 +136,7 @@ __global__ void __launch_bounds__(256, 1)
     using Lay = LbLayout<R>;
     constexpr int RH = R / 2;  // features per thread
     const int act = kRelu ? 0 : g.act, inside = kRelu ? 0 : g.inside;
-    static_assert(R % 16 == 0 && R <= 48, "rank 16..48 (rank 64's operands do not fit the shared memory)");
+    static_assert(R % 16 == 0 && R <= 64, "rank 16..64");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
@@ -171,11 +170,12 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t sx = smem_addr(smem + Lay::kOffX), sy = smem_addr(smem + Lay::kOffY),
                    sy2 = smem_addr(smem + Lay::kOffY2), sat = smem_addr(smem + Lay::kOffAt),
-                   sai = smem_addr(smem + Lay::kOffAi), ssi = smem_addr(smem + Lay::kOffSi),
+                   ssi = smem_addr(smem + Lay::kOffSi),
                    sw = smem_addr(smem + Lay::kOffW), sdu = smem_addr(smem + Lay::kOffDu);
     const uint32_t id_tok_r = idesc_bf16(128, R, false, false);     // [tokens x R], K = 128 dims
     const uint32_t id_acc = idesc_bf16(128, 2 * kRp, true, true);   // [dims x (hi|lo)], K = tokens
     const uint32_t id_tok_d = idesc_bf16(128, kD, false, false);    // [tokens x dims], K = features
+    const uint32_t id_tok_dt = idesc_bf16(128, kD, false, true);    // the same with B = A^T read MN-major
     int n_ld = 0, n_m1 = 0, n_m2 = 0, n_ld_issued = 0, n_m1_issued = 0, n_m2_issued = 0;
     bool aborted = false;
     auto fail = [&]() {
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(256, 1)
     for (int item = blockIdx.x; item < n_items && !aborted; item += gridDim.x) {
         const int bh = item / a.nsplit, split = item % a.nsplit;
         const int b = bh / g.Hh, h = bh % g.Hh;
-        // A^T image [R][128] (B of x A) and A image [128][64] (B of du A^T) of this pass's projection:
+        // A^T image [R][128] of this pass's projection (B of x A, and read MN-major the B of du A^T):
         // once when it is shared, again whenever the head changes when there is one per head
         if (staged_head < 0 || (g.a_stride != 0 && h != staged_head)) {
             const __nv_bfloat16* Ah = a.A + static_cast<size_t>(h) * g.a_stride;
@@ -196,7 +196,6 @@ __global__ void __launch_bounds__(256, 1)
                 const int d = e / R, c = e % R;
                 const uint16_t bits = *reinterpret_cast<const uint16_t*>(Ah + e);
                 *reinterpret_cast<uint16_t*>(smem + Lay::kOffAt + sw128_offset(c, d, R)) = bits;
-                *reinterpret_cast<uint16_t*>(smem + Lay::kOffAi + sw128_offset(d, c, kTok)) = bits;
             }
             staged_head = h;
         }
@@ -411,10 +410,10 @@ __global__ void __launch_bounds__(256, 1)
                     // dq = du A^T: du hi, then lo (K = R features)
 #pragma unroll
                     for (int kk = 0; kk < R / 16; ++kk)
-                        umma_ss(tO, kmaj(sdu, kk, kSlab), kmaj(sai, kk, kSlab), id_tok_d, kk > 0 ? 1u : 0u);
+                        umma_ss(tO, kmaj(sdu, kk, kSlab), mnmaj(sat, kk, R * 128), id_tok_dt, kk > 0 ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < R / 16; ++kk)
-                        umma_ss(tO, kmaj(sdu + kSlab, kk, kSlab), kmaj(sai, kk, kSlab), id_tok_d, 1u);
+                        umma_ss(tO, kmaj(sdu + kSlab, kk, kSlab), mnmaj(sat, kk, R * 128), id_tok_dt, 1u);
                 } else {
                     const uint32_t sdst = sy2;  // dS^T images hi, lo: [128][64] K-major each
                     // dv = psi dS: psi_hi dS_hi + psi_hi dS_lo + psi_lo dS_hi
@@ -430,10 +429,10 @@ __global__ void __launch_bounds__(256, 1)
                     // dk = du A^T
 #pragma unroll
                     for (int kk = 0; kk < R / 16; ++kk)
-                        umma_ss(tK, kmaj(sdu, kk, kSlab), kmaj(sai, kk, kSlab), id_tok_d, kk > 0 ? 1u : 0u);
+                        umma_ss(tK, kmaj(sdu, kk, kSlab), mnmaj(sat, kk, R * 128), id_tok_dt, kk > 0 ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < R / 16; ++kk)
-                        umma_ss(tK, kmaj(sdu + kSlab, kk, kSlab), kmaj(sai, kk, kSlab), id_tok_d, 1u);
+                        umma_ss(tK, kmaj(sdu + kSlab, kk, kSlab), mnmaj(sat, kk, R * 128), id_tok_dt, 1u);
                 }
                 // dA^T += x^T [du_hi | du_lo]
 #pragma unroll
@@ -587,7 +586,7 @@ cudaError_t launch_lr_bwd_tc_r(const LrTcBwdArgs& a, const Geom& g, const CUtens
 }
 }  // namespace
 
-// Tensor-core low-rank gradients (head_dim 128, rank <= 48): query pass, reduction of dS and dz, key
+// Tensor-core low-rank gradients (head_dim 128, rank <= 64): query pass, reduction of dS and dz, key
 // pass.  The dA partials of both passes are left for the caller's fixed-order reduction.
 cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st) {
     const RopeMeta& meta = *l.meta;
@@ -632,6 +631,9 @@ cudaError_t launch_lr_bwd_tc(const LrBwdArgs& l, const Geom& g, cudaStream_t st)
         case 48:
             return relu ? launch_lr_bwd_tc_r<48, true>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st)
                         : launch_lr_bwd_tc_r<48, false>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st);
+        case 64:
+            return relu ? launch_lr_bwd_tc_r<64, true>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st)
+                        : launch_lr_bwd_tc_r<64, false>(a, g, tq, tk, tv, tdq, tdk, tdv, l.dS, l.dz, koff, st);
     }
     return cudaErrorInvalidValue;
 }
