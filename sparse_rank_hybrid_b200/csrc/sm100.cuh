@@ -79,7 +79,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2D tiled load (no multicast): box at element coordinates (x, y) into shared memory, completion
+// 2D tiled load into this CTA only: box at element coordinates (x, y) into shared memory, completion
 // reported as transaction bytes on `bar`.  x * elemsize must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
     asm volatile(
@@ -89,7 +89,7 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-// 4D tiled load (no multicast), coordinates innermost first.
+// 4D tiled load into this CTA only, coordinates innermost first.
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
                                             int c3) {
     asm volatile(
@@ -116,7 +116,7 @@ __device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c
 }
 
 // 4D tiled reduce-add of a shared-memory box into global memory: each element is added to the one in
-// memory (in L2) by the TMA engine.  Same coordinate rules as tma_store_4d; no multicast.
+// memory (in L2) by the TMA engine.  Same coordinate rules as tma_store_4d.
 __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
                                                   int c3) {
     asm volatile("cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
@@ -131,7 +131,7 @@ __device__ __forceinline__ void tma_store_commit_and_wait() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
-// Plain bulk copy global -> shared (no multicast); both addresses 16-B aligned, bytes a multiple of 16.
+// Plain bulk copy global -> shared of this CTA; both addresses 16-B aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                      smem_addr(dst)),
