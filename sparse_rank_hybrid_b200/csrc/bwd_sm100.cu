@@ -35,8 +35,19 @@ namespace slra {
 
 namespace {
 
-constexpr int kBwdMathThreads = 256;  // 8 warps: two per TMEM lane group, each half of the key columns
-constexpr int kBwdIssueWarp = 8;      // + the tcgen05.mma issuing warp (lane 0) and a TMA producer warp
+// Warp roles of the dQ and dK/dV kernels for a block of BLK columns: NQ = BLK / 32 math warps per TMEM
+// lane group, each owning 32 of the block's columns (and D / NQ columns of the output rows), then the
+// tcgen05.mma issuing warp (lane 0) and a TMA producer warp.
+template <int BLK>
+struct BwdRoles {
+    static constexpr int NQ = BLK / 32;
+    static constexpr int kMathWarps = 4 * NQ;
+    static constexpr int kMathThreads = 32 * kMathWarps;
+    static constexpr int kIssueWarp = kMathWarps;
+    static constexpr int kProdWarp = kMathWarps + 1;
+    static constexpr int kThreads = kMathThreads + 64;
+    static constexpr int HW = 32;  // block columns per math thread
+};
 
 
 __device__ __forceinline__ uint32_t pack_half2_lohi(float lo, float hi) {
@@ -57,35 +68,56 @@ __device__ __forceinline__ uint32_t packed_col(int kk) {
 }  // namespace
 
 
-// Bring this thread's half of a gradient row (D/2 fp32) towards L2 before the row is read back, so the
+// Bring this thread's DW columns of a gradient row towards L2 before the row is read back, so the
 // read in the epilogue overlaps the last products instead of following them.
-template <int D>
-__device__ __forceinline__ void prefetch_half_row(const float* row, int hf) {
+template <int DW>
+__device__ __forceinline__ void prefetch_cols(const float* row_cols) {
 #pragma unroll
-    for (int o = 0; o < D / 2; o += 32)  // 128-byte lines
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(row + hf * (D / 2) + o));
+    for (int o = 0; o < DW; o += 32)  // 128-byte lines
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(row_cols + o));
 }
 
-// Rotate the pairs of this thread's D/2 columns back by R(p)^T and store them (fp32) into a token-major
-// row, or add them to it when a.accumulate (the row then holds the low-rank branch's part); `vals` are
-// the 32-bit TMEM words of columns [hf*D/2, hf*D/2 + D/2) of the row, already scaled.
-template <int D>
-__device__ __forceinline__ void store_row_unrotated(float* dst_row, const float* vals, int hf, int n,
-                                                    const BwdArgs& a, const Geom& g, bool rotate) {
-    float4 prev[D / 8];
+// This thread's DW consecutive TMEM columns of its lane from taddr (warp-collective loads), scaled.
+template <int DW>
+__device__ __forceinline__ void load_cols(uint32_t taddr, float* vals, float scale) {
+    if constexpr (DW >= 32) {
 #pragma unroll
-    for (int t = 0; t < D / 8; ++t)
-        prev[t] = a.accumulate ? *reinterpret_cast<const float4*>(dst_row + hf * (D / 2) + 4 * t)
+        for (int c = 0; c < DW / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c * 32, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) vals[c * 32 + i] = __uint_as_float(r[i]) * scale;
+        }
+    } else {
+        uint32_t r[16];
+        tmem_ld16(taddr, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) vals[i] = __uint_as_float(r[i]) * scale;
+    }
+}
+
+// Rotate the pairs of this thread's DW columns [c0, c0 + DW) back by R(p)^T and store them (fp32) into a
+// token-major row, or add them to it when a.accumulate (the row then holds the low-rank branch's part);
+// `vals` are the 32-bit TMEM words of those columns, already scaled.
+template <int DW>
+__device__ __forceinline__ void store_row_unrotated(float* dst_row, const float* vals, int c0, int n,
+                                                    const BwdArgs& a, const Geom& g, bool rotate) {
+    float4 prev[DW / 4];
+#pragma unroll
+    for (int t = 0; t < DW / 4; ++t)
+        prev[t] = a.accumulate ? *reinterpret_cast<const float4*>(dst_row + c0 + 4 * t)
                                : make_float4(0.f, 0.f, 0.f, 0.f);
     const int pt = n / (g.H * g.W), ph = (n / g.W) % g.H, pw = n % g.W;
 #pragma unroll
-    for (int t = 0; t < D / 8; ++t) {  // 4 columns (2 pairs) per float4
+    for (int t = 0; t < DW / 4; ++t) {  // 4 columns (2 pairs) per float4
         float4 o;
         float* ov = reinterpret_cast<float*>(&o);
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const int c = 4 * t + 2 * u;           // column within the half
-            const int pair = (hf * (D / 2) + c) / 2;
+            const int c = 4 * t + 2 * u;  // column within this thread's range
+            const int pair = (c0 + c) / 2;
             const float y0 = vals[c], y1 = vals[c + 1];
             if (rotate) {
                 const int2 pi = a.pair_info[pair];
@@ -103,14 +135,15 @@ __device__ __forceinline__ void store_row_unrotated(float* dst_row, const float*
         o.y += prev[t].y;
         o.z += prev[t].z;
         o.w += prev[t].w;
-        *reinterpret_cast<float4*>(dst_row + hf * (D / 2) + 4 * t) = o;
+        *reinterpret_cast<float4*>(dst_row + c0 + 4 * t) = o;
     }
 }
 
 // ------------------------------------------------------------------------------------------ dQ
-// Warps 0-7 math (rows = queries), warp 8 issues the products, warp 9 loads the tiles.
+// BwdRoles<BLK>: 4 * BLK / 32 math warps (rows = queries; each 32 key columns of a block), then the
+// warp that issues the products and the warp that loads the tiles.
 // TMEM (512 columns): S | dP buffer 0 | dP buffer 1 | dQ^.  Each math thread writes its packed dS_j over
-// its own half of dP_j's columns (already in its registers), so the S columns are free as soon as the
+// its own 32 of dP_j's columns (already in its registers), so the S columns are free as soon as the
 // math warps have loaded S_j and dP_j: S_{j+1} and dP_{j+1} (into the other dP buffer) are computed
 // while the math warps work on block j, and dQ^ += dS_j k^_j follows when they are done.  k^ tiles stay
 // until their dQ product (three slots), v tiles until their dP product (two slots).
@@ -129,17 +162,17 @@ struct DqLayout {
 enum : int { kDqBarQdo = 0, kDqBarKFull = 1, kDqBarKEmpty = 4, kDqBarVFull = 7, kDqBarVEmpty = 9,
              kDqBarSp = 11, kDqBarLd = 12, kDqBarDs = 13 /* +2 */, kDqBarFinal = 15, kDqBarDrain = 16,
              kDqNumBars = 17 };
-constexpr int kBwdProdWarp = 9;
-constexpr int kBwdThreads2 = 320;
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(kBwdThreads2, 1)
+__global__ void __launch_bounds__(BwdRoles<BLK>::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, BwdArgs a,
                   Geom g) {
     using Lay = DqLayout<D>;
-    constexpr int HW = BLK / 2;  // key columns per thread
+    using Roles = BwdRoles<BLK>;
+    constexpr int HW = Roles::HW;  // key columns per math thread
     constexpr int NC = HW / 32;
+    constexpr int DW = D / Roles::NQ;  // dQ columns per math thread in the epilogue
     constexpr int kSteps = D / 16, kKeySteps = BLK / 16;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -156,7 +189,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
 
     if (tid == 0) {
         for (int i = 0; i < kDqNumBars; ++i)
-            mbar_init(bars + i, (i == kDqBarLd || i == kDqBarDs || i == kDqBarDs + 1) ? kBwdMathThreads : 1);
+            mbar_init(bars + i, (i == kDqBarLd || i == kDqBarDs || i == kDqBarDs + 1) ? Roles::kMathThreads : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -177,7 +210,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
     auto kslot = [&](int j) { return smem + Lay::kOffK + (j % 3) * Lay::kTile; };
     auto vslot = [&](int j) { return smem + Lay::kOffV + (j & 1) * Lay::kTile; };
 
-    if (warp == kBwdProdWarp) {
+    if (warp == Roles::kProdWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && keep > 0) {
             auto load_rows = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int row, int rows) {
@@ -218,7 +251,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
             }
         }
         __syncwarp();
-    } else if (warp == kBwdIssueWarp) {
+    } else if (warp == Roles::kIssueWarp) {
         // ------------------------------------------------------------ tcgen05.mma issuer
         if (lane == 0 && keep > 0) {
             const uint32_t idesc_s = idesc_f16_f32(128, BLK, false, false);
@@ -334,22 +367,15 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
         }
         // ---- epilogue: dq += R(p)^T dQ^ / sqrt(D), token-major fp32
         if (keep > 0) {
-            if (ok && row_real && a.accumulate) prefetch_half_row<D>(a.dq + g.so.row(b, n, h), hf);
+            if (ok && row_real && a.accumulate) prefetch_cols<DW>(a.dq + g.so.row(b, n, h) + hf * DW);
             const bool done = ok && __all_sync(0xffffffffu, mbar_wait(bars + kDqBarFinal, 0, tmo, abort_flag));
             if (done) {
                 tc_fence_after();
-                float vals[D / 2];
+                float vals[DW];
                 const float inv_sqrt_d = 1.f / sqrtf(static_cast<float>(D));
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tQ + lane_base + hf * (D / 2) + c * 32, r);
-                    tmem_ld_wait(r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) vals[c * 32 + i] = __uint_as_float(r[i]) * inv_sqrt_d;
-                }
+                load_cols<DW>(tQ + lane_base + hf * DW, vals, inv_sqrt_d);
                 if (row_real)
-                    store_row_unrotated<D>(a.dq + g.so.row(b, n, h), vals, hf, n, a, g, true);
+                    store_row_unrotated<DW>(a.dq + g.so.row(b, n, h), vals, hf * DW, n, a, g, true);
             }
         }
     }
@@ -362,8 +388,9 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
 }
 
 // ---------------------------------------------------------------------------------------- dK, dV
-// Warps 0-7 math (rows = keys), warp 8 issues the products, warp 9 loads the query-side tiles.
-// TMEM: S^T | dP^T | dV | dK^.  Each math thread writes its packed P^T and dS^T over its own half of
+// BwdRoles<BLK> math warps (rows = keys; each 32 query columns of a block), then the warp that issues
+// the products and the warp that loads the query-side tiles.
+// TMEM: S^T | dP^T | dV | dK^.  Each math thread writes its packed P^T and dS^T over its own 32 of
 // dP^T's columns (P^T in the first quarter of the block's columns, dS^T in the second), so the S^T
 // columns are free once S^T_t and dP^T_t are in registers and S^T_{t+1} is computed during the math of
 // block t; dP^T_{t+1} follows the dV and dK products that read block t's packed operands.
@@ -385,13 +412,15 @@ enum : int { kKvBarKv = 0, kKvBarQFull = 1, kKvBarQEmpty = 3, kKvBarS = 5, kKvBa
              kKvBarDs = 8 /* +2 */, kKvBarFinal = 10, kKvBarDrain = 11, kKvNumBars = 12 };
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(kBwdThreads2, 1)
+__global__ void __launch_bounds__(BwdRoles<BLK>::kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do, BwdArgs a,
                     Geom g) {
     using Lay = DkvLayout<D, BLK>;
-    constexpr int HW = BLK / 2;  // query columns per thread
+    using Roles = BwdRoles<BLK>;
+    constexpr int HW = Roles::HW;  // query columns per math thread
     constexpr int NC = HW / 32;
+    constexpr int DW = D / Roles::NQ;  // dK, dV columns per math thread in the epilogue
     constexpr int kSteps = D / 16, kQSteps = BLK / 16;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -408,7 +437,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
 
     if (tid == 0) {
         for (int i = 0; i < kKvNumBars; ++i)
-            mbar_init(bars + i, (i == kKvBarLd || i == kKvBarDs || i == kKvBarDs + 1) ? kBwdMathThreads : 1);
+            mbar_init(bars + i, (i == kKvBarLd || i == kKvBarDs || i == kKvBarDs + 1) ? Roles::kMathThreads : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -429,7 +458,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
     auto doslot = [&](int s) { return smem + Lay::kOffDo + s * Lay::kQTile; };
     auto lseslot = [&](int s) { return reinterpret_cast<float*>(smem + Lay::kOffLse + s * 2 * BLK * 4); };
 
-    if (warp == kBwdProdWarp) {
+    if (warp == Roles::kProdWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && cnt > 0) {
             auto load_rows = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int row, int rows) {
@@ -466,7 +495,7 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
             }
         }
         __syncwarp();
-    } else if (warp == kBwdIssueWarp) {
+    } else if (warp == Roles::kIssueWarp) {
         // ------------------------------------------------------------ tcgen05.mma issuer
         if (lane == 0 && cnt > 0) {
             const uint32_t idesc_s = idesc_f16_f32(128, BLK, false, false);
@@ -596,29 +625,25 @@ __global__ void __launch_bounds__(kBwdThreads2, 1)
         }
         // ---- epilogue: dv += sum P^T dO, dk += R(p)^T dK^ / sqrt(D); key blocks nobody kept add zeros
         if (ok && row_real && a.accumulate) {
-            prefetch_half_row<D>(a.dv + g.so.row(b, n, h), hf);
-            prefetch_half_row<D>(a.dk + g.so.row(b, n, h), hf);
+            prefetch_cols<DW>(a.dv + g.so.row(b, n, h) + hf * DW);
+            prefetch_cols<DW>(a.dk + g.so.row(b, n, h) + hf * DW);
         }
         const bool done = cnt == 0 || (ok && __all_sync(0xffffffffu, mbar_wait(bars + kKvBarFinal, 0, tmo, abort_flag)));
         if (done) {
             if (cnt > 0) tc_fence_after();
             const float inv_sqrt_d = 1.f / sqrtf(static_cast<float>(D));
-            float vals[D / 2];
+            float vals[DW];
 #pragma unroll
             for (int which = 0; which < 2; ++which) {  // 0: dv, 1: dk
+                if (cnt > 0) {  // uniform over the CTA: the loads are warp-collective
+                    load_cols<DW>((which ? tK : tV) + lane_base + hf * DW, vals, which ? inv_sqrt_d : 1.f);
+                } else {
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
-                    uint32_t r[32];
-                    if (cnt > 0) {
-                        tmem_ld32((which ? tK : tV) + lane_base + hf * (D / 2) + c * 32, r);
-                        tmem_ld_wait(r);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        vals[c * 32 + i] = cnt > 0 ? __uint_as_float(r[i]) * (which ? inv_sqrt_d : 1.f) : 0.f;
+                    for (int i = 0; i < DW; ++i) vals[i] = 0.f;
                 }
                 if (row_real)
-                    store_row_unrotated<D>((which ? a.dk : a.dv) + g.so.row(b, n, h), vals, hf, n, a, g, which == 1);
+                    store_row_unrotated<DW>((which ? a.dk : a.dv) + g.so.row(b, n, h), vals, hf * DW, n, a, g,
+                                            which == 1);
             }
         }
     }
@@ -1487,10 +1512,11 @@ cudaError_t launch_bwd_sparse_t(const BwdMaps& m, const BwdArgs& a, const Geom& 
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)skv);
     if (e != cudaSuccess) return e;
-    bwd_dq_kernel<D, BLK><<<dim3(g.nb, g.BH()), kBwdThreads2, sq, st>>>(m.q128, m.do128, m.kb, m.vb, a, g);
+    bwd_dq_kernel<D, BLK><<<dim3(g.nb, g.BH()), BwdRoles<BLK>::kThreads, sq, st>>>(m.q128, m.do128, m.kb, m.vb, a, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (m.between) cudaEventRecord(m.between, st);
-    bwd_dkdv_kernel<D, BLK><<<dim3(g.nb, g.BH()), kBwdThreads2, skv, st>>>(m.k128, m.v128, m.qb, m.dob, a, g);
+    bwd_dkdv_kernel<D, BLK><<<dim3(g.nb, g.BH()), BwdRoles<BLK>::kThreads, skv, st>>>(m.k128, m.v128, m.qb, m.dob, a,
+                                                                                    g);
     return cudaGetLastError();
 }
 
