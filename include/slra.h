@@ -331,7 +331,7 @@ SLRA_API slra_status slra_lowrank_fwd(const slra_tensor* q, const slra_tensor* k
  * layout followed by the backward's sections: the sparse output and its per-row log-sum-exp, an fp16
  * copy of dout, the inverted kept-block lists and the low-rank gradient partial sums; with the gated
  * fusion also the low-rank output, its gradient and the gate's per-row terms and partial sums); 0 if p
- * is invalid.  No GPU access.
+ * is invalid or has output strides (the backward's gradients are contiguous).  No GPU access.
  */
 SLRA_API size_t slra_bwd_workspace_bytes(const slra_problem* p);
 

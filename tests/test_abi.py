@@ -280,3 +280,18 @@ def test_train_forward_and_saved_backward_validation():
     assert L.slra_attn_bwd_saved(ctypes.byref(pc), *args, ws, bwd_b, None) == slra.ERR_NO_DEVICE
     assert L.slra_attn_bwd_saved(ctypes.byref(pc), q, k, v, A, dout, dq, dq, dv, dA, ws, bwd_b,
                                  None) == slra.ERR_INVALID_ARG
+
+
+def test_backward_rejects_strided_outputs():
+    """The gradients are contiguous: a problem with output strides is refused by the backward entry
+    points (before any device access), while the forward accepts it."""
+    import ctypes
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("has a GPU")
+    p = slra.Problem.from_workload(W.TINY)
+    pc = p.c()
+    D, Hh = W.TINY.head_dim, W.TINY.heads
+    pc.out_strides[:] = [W.TINY.L * Hh * D * 2, Hh * D * 2, D]  # rows of a wider buffer
+    assert slra.lib().slra_bwd_workspace_bytes(ctypes.byref(pc)) == 0
+    assert slra.lib().slra_validate(ctypes.byref(pc)) == slra.OK

@@ -395,3 +395,27 @@ def test_saved_backward_gated():
     assert slra.device_status(ws) == slra.OK
     for a, b in zip(got + g2, ref + g1):
         assert torch.equal(a, b)
+
+
+def test_backward_gated_batch2():
+    """The gate's dWg and dbg sum over batch elements and heads: batch 2, three heads."""
+    _gated_case(EDGE_B2, "edge-b2-gated", -0.5)
+
+
+def test_saved_backward_bf16_output():
+    """The training forward with a bf16 output: the output bit for bit the forward's, the kept O_s and
+    lse (fp32 regardless of the output type) give the recomputing backward's gradients bit for bit."""
+    import torch
+    w = EDGE_128
+    x = I.make_inputs(w)
+    dout = torch.from_numpy(I.make_dout(w.seed + 9200, w.batch, w.L, w.heads, w.head_dim)).cuda()
+    p = slra.Problem.from_workload(w, out_dtype=slra.OUT_BF16)
+    q, k, v, A = (parity.to_gpu(x[n]) for n in ("q", "k", "v", "A"))
+    out_ref = slra.attn_fwd(p, q, k, v, A)[0]
+    out_t, ws = slra.attn_fwd_train(p, q, k, v, A)
+    assert out_t.dtype == torch.bfloat16 and torch.equal(out_t, out_ref)
+    ref = slra.attn_bwd(p, q, k, v, A, dout)[:4]
+    got = slra.attn_bwd_saved(p, q, k, v, A, dout, ws)[:4]
+    assert slra.device_status(ws) == slra.OK
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
