@@ -1,17 +1,21 @@
 // Gradients of the low-rank branch on the sm_100a tensor cores (head_dim 128, rank <= 64): the
-// derivative of RoLA "4.1"/"4.2"/"4.3"/"B.1"'s branch (phi = relu(x A), psi = R_r phi outside the
-// activation, S = sum psi_k v^T, z = sum phi_k, O_lr = psi_q S / (phi_q . z + 1e-6)).
+// derivative of RoLA "4.1"/"4.2"/"4.3"/"B.1"'s branch (default: phi = relu(x A), psi = R_r phi outside
+// the activation, S = sum psi_k v^T, z = sum phi_k, O_lr = psi_q S / (phi_q . z + 1e-6)), and of its
+// variants: the other feature maps, no low-rank RoPE, the RoPE inside the activation (psi = act(R_r x A),
+// the normaliser on psi), separate and per-head projections.  Per rotation pair, lr_pair_fwd /
+// lr_pair_bwd (common.cuh) give psi, the normaliser's feature nf and du for each of these.
 //
 // Persistent CTAs (one per SM, 256 threads: two per token row, each half of the features) walk work
 // items = (head, range of 128-token tiles), like the forward summary kernel.  Per tile:
 //   query pass  MMA  U = q A, G = dO S^T                                 (token rows in TMEM)
-//               threads (row = TMEM lane): phi, psi, den = phi . z + 1e-6, dden = -(psi . G) / den^2,
-//               dphi = R^T (G / den) + dden z, du = dphi [u > 0], w = psi / den; dz += dden phi
+//               threads (row = TMEM lane): psi, nf, den = nf . z + 1e-6, dden = -(psi . G) / den^2,
+//               du from dpsi = G / den and dnf = dden z, w = psi / den; dz += dden nf
 //               MMA  dS^T += dO^T [w_hi | w_lo],  dA^T += q^T [du_hi | du_lo]   (accumulated over the
-//                    item's tiles, d rows in TMEM),  dq = du A^T          (stored by the threads)
+//                    item's tiles, d rows in TMEM),  dq = du A^T
 //   key pass    MMA  U = k A, dpsi = v dS^T
-//               threads: phi, psi, du = (R^T dpsi + dz) [u > 0]
-//               MMA  dv = psi dS, dk = du A^T (stored), dA^T += k^T [du_hi | du_lo] (accumulated)
+//               threads: psi, du from dpsi and dnf = dz
+//               MMA  dv = psi dS, dk = du A^T, dA^T += k^T [du_hi | du_lo] (accumulated)
+// dq, dk, dv leave through shared memory and TMA: stored, or added to the sparse branch's rows.
 // Operands that are not exact in bf16 (dO, S, dS, w, du, psi) are split into bf16 hi + lo (x = hi + lo
 // to ~2^-16); products take hi*hi + hi*lo + lo*hi with fp32 accumulation.  The item's dS, dA and dz
 // partial sums go to split-L buffers that a fixed-order reduction sums.
