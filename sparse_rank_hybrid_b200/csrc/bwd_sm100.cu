@@ -1,6 +1,9 @@
-// Backward pass of the hybrid attention (relu features, RoPE outside the activation, one shared
-// projection A, plain sum of the branches): gradients of sum(dO * out) with respect to q, k, v and A,
-// the block selection held at the forward's (it is piecewise constant in q and k).
+// Backward pass of the hybrid attention: gradients of sum(dO * out) with respect to q, k, v and the
+// projection(s), the block selection held at the forward's (it is piecewise constant in q and k).  The
+// formulas below are the default options' (relu features, RoPE outside the activation, one shared
+// projection, plain sum); the feature maps and RoPE orderings go through lr_pair_fwd / lr_pair_bwd
+// (common.cuh), separate and per-head projections through the A offsets and the dA reduction, and the
+// gated fusion through gate_bwd.cu, which hands the two branches their own output gradients.
 //
 // Method: the derivative of the forward of RoLA "4.1" (block-sparse softmax attention over the kept
 // key blocks plus the low-rank branch), "4.2"/"4.3" (truncated RoPE outside the relu feature map) and
@@ -12,7 +15,7 @@
 //   dS_ij = P_ij (dP_ij - Delta_i),  dq^_i = sum_j dS_ij k^_j / sqrt(D),  dk^_j = sum_i dS_ij q^_i / sqrt(D),
 //   dv_j = sum_i P_ij dO_i,  dq = R(p)^T dq^,  dk = R(p)^T dk^.
 //   bwd_dq_kernel      one CTA per (query block, head): S = q^ k^T and dP = dO v^T per kept key block
-//                      into TMEM, the softmax warps form dS (fp16) over S's columns, dQ^ += dS k^ is
+//                      into TMEM, the math warps form dS (fp16) over dP's columns, dQ^ += dS k^ is
 //                      accumulated in TMEM (tcgen05.mma kind::f16, operands fp16 in shared memory by TMA).
 //   bwd_dkdv_kernel    one CTA per (key block, head), over the query blocks that kept it (inverted
 //                      lists, ascending): S^T = k^ q^T and dP^T = v dO^T into TMEM, P^T and dS^T (fp16)
@@ -23,8 +26,9 @@
 //   dphi_q,i = R_r^T dpsi_q,i + dden_i z,  dS = sum_i psi_q,i dO_i^T / den_i,  dz = sum_i dden_i phi_q,i,
 //   dpsi_k,j = dS v_j,  dv_j += dS^T psi_k,j,  dphi_k,j = R_r^T dpsi_k,j + dz,
 //   du = dphi * [u > 0],  dq += du_q A^T,  dk += du_k A^T,  dA = q^T du_q + k^T du_k.
-//   bwd_lr_q_kernel / bwd_lr_k_kernel   CUDA-core fp32 passes over token tiles (split-L partial sums of
-//                      dS, dz and dA, summed in a fixed order).
+//   lr_bwd_sm100_kernel (lr_bwd_sm100.cu)   the same on the tensor cores for head_dim 128, rank <= 64;
+//   bwd_lr_q_kernel / bwd_lr_k_kernel   CUDA-core fp32 passes over token tiles for the other shapes
+//                      (split-L partial sums of dS, dz and dA, summed in a fixed order).
 //
 // All waits are bounded (see sm100.cuh); a wait that runs out records a timeout in the status word and
 // the CTA drains what it issued and returns.
