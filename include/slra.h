@@ -88,8 +88,9 @@ typedef enum slra_status {
     SLRA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or a kernel launch failed                */
     SLRA_ERR_DEVICE_TIMEOUT = 6,  /* (device status) a bounded wait inside a kernel ran out              */
     SLRA_ERR_RANGE = 7,           /* (device status) a value does not fit the fp16 operands: |value| >=
-                                     65504 after RoPE, or a block of q^, k^ or v whose nonzero values all
-                                     lie below fp16's smallest normal 2^-14 (relative precision lost)     */
+                                     65504 after RoPE, or a block of q^, k^ or (where an fp16 copy of v
+                                     is made) v whose nonzero values all lie below fp16's smallest
+                                     normal 2^-14 (relative precision lost)                              */
     SLRA_ERR_NO_DEVICE = 8,       /* no sm_100 device is current                                         */
     SLRA_ERR_SCRATCH_LIMIT = 9    /* slra_lowrank_summary_noalloc: problem exceeds its fixed scratch area */
 } slra_status;
@@ -226,6 +227,8 @@ typedef struct slra_problem {
  * Where the intermediates live inside a workspace (byte offsets from its start; all 256-B aligned).
  * They are valid after a forward call and may be read for inspection:
  *   qh, kh, vh   fp16 [B*Hh][nb*block][D]  rotated q, k and fp16 copy of v, head-major, zero padded
+ *                                          (vh: written by slra_select_blocks, the training forward and
+ *                                          the backward; the inference forward reads v itself)
  *   qbar, kbar   fp64 [B*Hh][nb][D]        block means of qh, kh (computed in fp64)
  *   idx          int32 [B*Hh][nb][keep]    kept key blocks per query block, ascending
  *   tie          uint8 [B*Hh][nb]          1 where the k-th and (k+1)-th block scores are within

@@ -303,17 +303,17 @@ unsigned long long timeout_of(const slra_problem* p) {
 int debug_wait_of(const slra_problem* p) { return (p->debug_flags & SLRA_DEBUG_UNSATISFIED_WAIT) ? 1 : 0; }
 
 
-// Tables + RoPE/pooling + selection.
+// Tables + RoPE/pooling + selection; write_v: also the fp16 v copy the backward kernels read.
 slra_status run_select(const slra_problem* p, const Derived& d, const Ptrs& w, const void* q, const void* k,
-                       const void* v, cudaStream_t st) {
+                       const void* v, bool write_v, cudaStream_t st) {
     const Geom& g = d.g;
     CUtensorMap mq, mk, mv;  // token-major inputs, boxes of 64 columns x one key block of tokens
     if (!make_map_tokens(&mq, q, g.B, g.L, g.Hh, g.D, g.sq, g.block) ||
         !make_map_tokens(&mk, k, g.B, g.L, g.Hh, g.D, g.sk, g.block) ||
         !make_map_tokens(&mv, v, g.B, g.L, g.Hh, g.D, g.sv, g.block))
         return SLRA_ERR_CUDA;
-    cudaError_t e = launch_rope_pool(mq, mk, mv, w.tab, w.pairs, g, w.qh, w.kh, w.vh, w.qbar, w.kbar, w.status,
-                                     timeout_of(p), st);
+    cudaError_t e = launch_rope_pool(mq, mk, mv, w.tab, w.pairs, g, write_v, w.qh, w.kh, w.vh, w.qbar, w.kbar,
+                                     w.status, timeout_of(p), st);
     if (e != cudaSuccess) return SLRA_ERR_CUDA;
     slra_status s = mark(p, 2, st);
     if (s != SLRA_OK) return s;
@@ -615,7 +615,7 @@ slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, con
     AttnMaps maps;
     const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
     if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) || !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
-        !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
+        !make_map_tokens(&maps.v, v, g.B, g.L, g.Hh, g.D, g.sv, g.block) ||
         !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, g.sq, 128) ||
         !make_map_out(&maps.out, out, g.B, g.L, g.Hh, g.D, g.so, p->out_dtype == SLRA_OUT_F32))
         return SLRA_ERR_CUDA;
@@ -640,7 +640,7 @@ slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, con
         // call is left running unordered
         const slra_status s_lr = run_lowrank(p, d, w, k, v, A, ss.s);
         const bool rec = cudaEventRecord(ss.join, ss.s) == cudaSuccess;
-        const slra_status s_sel = run_select(p, d, w, q, k, v, st);
+        const slra_status s_sel = run_select(p, d, w, q, k, v, lse != nullptr, st);
         const bool joined = rec && cudaStreamWaitEvent(st, ss.join, 0) == cudaSuccess;
         if (!joined) {
             cudaGetLastError();
@@ -654,7 +654,7 @@ slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, con
     } else {
         // a branch that is off still records its stage boundaries, so its stages time as zero
         if (branches & SLRA_BRANCH_SPARSE) {
-            if ((s = run_select(p, d, w, q, k, v, st)) != SLRA_OK) return s;
+            if ((s = run_select(p, d, w, q, k, v, lse != nullptr, st)) != SLRA_OK) return s;
         } else if ((s = mark(p, 2, st)) != SLRA_OK || (s = mark(p, 3, st)) != SLRA_OK) {
             return s;
         }
@@ -920,7 +920,7 @@ slra_status slra_select_blocks(const slra_problem* p, const void* q, const void*
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const Ptrs w = carve(workspace, d);
     if ((s = begin(p, d, w, st)) != SLRA_OK) return s;
-    return run_select(p, d, w, q, k, v, st);
+    return run_select(p, d, w, q, k, v, true, st);
 }
 
 slra_status slra_lowrank_summary(const slra_problem* p, const void* k, const void* v, const void* A, void* workspace,
@@ -1080,7 +1080,7 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
     if (!saved && cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return SLRA_ERR_CUDA;
     if (!saved && (s = cuda_status(launch_rope_table(w.tab, w.pairs, d.meta, d.table_entries, st))) != SLRA_OK)
         return s;
-    if (!saved && sparse && (s = run_select(&pr, d, w, q, k, v, st)) != SLRA_OK) return s;
+    if (!saved && sparse && (s = run_select(&pr, d, w, q, k, v, true, st)) != SLRA_OK) return s;
     if (!saved && lowrank && (s = run_lowrank(&pr, d, w, k, v, A, st)) != SLRA_OK) return s;
     if (!saved && sparse) {
         // the sparse forward again, writing its output O_s (head-major fp32) and each row's lse
@@ -1088,7 +1088,7 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
         const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
         if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) ||
             !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
-            !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
+            !make_map_tokens(&maps.v, v, g.B, g.L, g.Hh, g.D, g.sv, g.block) ||
             !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, g.sq, 128) ||
             !make_map_out(&maps.out, os, g.B, g.L, g.Hh, g.D, headmajor_strides(g), true))
             return SLRA_ERR_CUDA;
@@ -1121,7 +1121,7 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
         const uint64_t rows = static_cast<uint64_t>(g.BH()) * g.Lp;
         if (!make_map_headmajor(&maps.q, w.qh, rows, g.D, 128) ||
             !make_map_headmajor(&maps.k, w.kh, rows, g.D, g.block) ||
-            !make_map_headmajor(&maps.v, w.vh, rows, g.D, g.block) ||
+            !make_map_tokens(&maps.v, v, g.B, g.L, g.Hh, g.D, g.sv, g.block) ||
             !make_map_tokens(&maps.q_raw, q, g.B, g.L, g.Hh, g.D, g.sq, 128) ||
             !make_map_out(&maps.out, olr, g.B, g.L, g.Hh, g.D, headmajor_strides(g), true))
             return SLRA_ERR_CUDA;

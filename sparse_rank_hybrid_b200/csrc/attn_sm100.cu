@@ -11,14 +11,15 @@
 //   warps 0-7  softmax: row i lives in TMEM lane i; warps w and w+4 both reach lanes 32(w%4).. and
 //              split the key block in halves, exchanging their row maxima (and at the end their row
 //              sums) through shared memory: row max, lazy rescale of O (only when the max grows by
-//              more than 2^8), P = 2^(s*log2e/sqrt(D) - m) rounded to fp16 and written back into the
+//              more than 2^8), P = 2^(s*log2e/sqrt(D) - m) rounded to bf16 and written back into the
 //              TMEM columns of that S buffer;
-//   warp 8     TMA producer: q^ tile, then k^ and v tiles into two slots each (fp16, 128-B swizzle),
-//              each slot refilled as soon as the product that read it has completed;
+//   warp 8     TMA producer: q^ tile, then k^ tiles (the fp16 head-major copies) and v tiles (bf16,
+//              straight from the caller's token-major v) into two slots each (128-B swizzle), each
+//              slot refilled as soon as the product that read it has completed;
 //   warp 9     MMA issuer: once the softmax has released P_j, O += P_j v_j (A operand P_j from TMEM,
-//              B = v tile MN-major) and S_{j+2} = q^ k^T_{j+2} into the S buffer P_{j-1} occupied
-//              (tcgen05.mma kind::f16, M=128, N=block, K=D, fp32 in TMEM), their k-steps issued
-//              alternately.
+//              B = v tile MN-major; bf16) and S_{j+2} = q^ k^T_{j+2} (fp16) into the S buffer P_{j-1}
+//              occupied (tcgen05.mma kind::f16, M=128, N=block, K=D, fp32 in TMEM), their k-steps
+//              issued alternately.
 // With three S buffers S_{j+1} is already in TMEM when the softmax finishes S_j, so a key block
 // costs about the longer of the softmax and the two products instead of their sum.  The two
 // products' k-steps are interleaved one by one: the tensor pipe runs a run of four or more
@@ -121,10 +122,10 @@ __device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) 
         : "f"(a0), "f"(a1));
 }
 
-// fp16x2 with lo in the low half (the lower key index sits in the lower 16 bits of a TMEM column).
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+// bf16x2 with lo in the low half (the lower key index sits in the lower 16 bits of a TMEM column).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
 
@@ -251,6 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int sl = 0; sl < D / 64; ++sl) tma_load_2d(dst + sl * (rows * 128), tm, bar, sl * 64, row);
             };
+            // v_j straight from the caller's token-major bf16 v (tokens past L read as zero)
+            auto add_vtile = [&](uint64_t* bar, uint8_t* dst, int j, bool arrive) {
+                if (arrive) mbar_expect_tx(bar, static_cast<uint32_t>(blk) * D * 2);
+                else mbar_add_tx(bar, static_cast<uint32_t>(blk) * D * 2);
+                const int n0 = __ldg(my_idx + j) * blk;
+#pragma unroll
+                for (int sl = 0; sl < D / 64; ++sl) tma_load_4d(dst + sl * (blk * 128), &tm_v, bar, sl * 64, h, n0, b);
+            };
             // Slot s's k and v tiles are read by the products the MMA warp issues together (P.V_j with
             // S_{j+2}), so one commit frees both: v_j and k_{j+2} go into slot s once P.V_{j-2} and S_j
             // have completed (for j < 2: S_j alone, and v_j needs no wait).
@@ -261,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                add_tile(bars + kBarVFull + s, vslot(s), &tm_v, row0 + __ldg(my_idx + j) * blk, blk, !has_k);
+                add_vtile(bars + kBarVFull + s, vslot(s), j, !has_k);
                 ++nv;
                 if (has_k) {
                     if (j < 2 && !mbar_wait(bars + kBarKvEmpty + s, 0, tmo, abort_flag)) {
@@ -290,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------------------- tcgen05.mma issuer
         if (lane == 0 && keep > 0 && !*abort_flag) {
             const uint32_t idesc_s = idesc_f16_f32(128, blk, false, false);
-            const uint32_t idesc_o = idesc_f16_f32(128, D, false, true);
+            const uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);  // P bf16 (TMEM), v bf16
             const uint32_t q_addr = smem_addr(smem + Lay::kOffQ);
             // Operand descriptors per slot, computed once; a k-step adds a compile-time offset to the
             // 14-bit address field (shared-memory addresses stay below 2^18, so it cannot carry out).
@@ -448,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float neg_m = -m_run;
             float sums[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};  // independent accumulators
-            // keys (2i, 2i+1) of this half -> packed fp16x2 TMEM column key0/2 + i, 16 columns at a time
+            // keys (2i, 2i+1) of this half -> packed bf16x2 TMEM column key0/2 + i, 16 columns at a time
 #pragma unroll
             for (int c16 = 0; c16 < NE / 32; ++c16) {
                 uint32_t pk[16];
@@ -460,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           neg_m, neg_m);
                     const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
                     fadd2(sums[u & 3][0], sums[u & 3][1], p0, p1);
-                    pk[u] = pack_half2(p0, p1);
+                    pk[u] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(tSj + lane_base + key0 / 2 + c16 * 16, pk);
             }

@@ -134,10 +134,11 @@ __host__ __device__ inline int token_axis_pos(int n, int axis, int H, int W) {
 
 // ---- launchers (defined in prep_kernels.cu and attn_sm100.cu) --------------------------------
 cudaError_t launch_rope_table(double2* tab, int2* pairs, const RopeMeta& meta, int entries, cudaStream_t st);
+// write_v: also the fp16 head-major v copy (for the backward kernels; the forward reads v itself).
 cudaError_t launch_rope_pool(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                             const double2* tab, const int2* pairs, const Geom& g, __half* qh, __half* kh,
-                             __half* vh, double* qbar, double* kbar, int* status, unsigned long long timeout_ns,
-                             cudaStream_t st);
+                             const double2* tab, const int2* pairs, const Geom& g, bool write_v, __half* qh,
+                             __half* kh, __half* vh, double* qbar, double* kbar, int* status,
+                             unsigned long long timeout_ns, cudaStream_t st);
 cudaError_t launch_select(const double* qbar, const double* kbar, const Geom& g, int32_t* idx, uint8_t* tie,
                           cudaStream_t st);
 cudaError_t launch_lowrank_partial(const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* A,

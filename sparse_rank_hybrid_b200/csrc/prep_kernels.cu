@@ -37,15 +37,16 @@ cudaError_t launch_rope_table(double2* tab, int2* pairs, const RopeMeta& meta, i
 }
 
 // ------------------------------------------------------------------------------ rope_pool
-// One CTA per (query/key block, batch*head), two CTAs per SM.  Thread 0 brings the block's q, k and v
-// rows of this head into shared memory with TMA (token-major 4D maps, 64-column boxes, 128-B swizzle;
-// tokens past L read as zero), so a whole block's 3 x block x 2D bytes are in flight at once.  Then
+// One CTA per (query/key block, batch*head), two CTAs per SM.  Thread 0 brings the block's q, k (and,
+// with kV, v) rows of this head into shared memory with TMA (token-major 4D maps, 64-column boxes,
+// 128-B swizzle; tokens past L read as zero), so a whole block's tiles are in flight at once.  The fp16
+// v copy is only made for the backward kernels (kV); the forward's attention kernel reads v itself.  Then
 // thread t owns four consecutive rotary pairs (8 elements, 16 bytes) j = 4*(t % (D/8)) .. +3 and walks
 // the block's tokens with stride 256/(D/8); each fp16 output access is one 16-byte store, and the D/8
 // threads of a token cover its row, so a block's rows go out as one contiguous stretch per tensor.
 // The rotation and the block sums are fp64 so the selection scores are exact to ~1e-15 relative (the
 // top-k decision is made on them); the fp16 copies come from the same values.
-template <int D>
+template <int D, bool kV>
 __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                            const __grid_constant__ CUtensorMap tm_k,
                                                            const __grid_constant__ CUtensorMap tm_v,
@@ -78,12 +79,12 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
     __syncthreads();
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&tm_q);
-        mbar_expect_tx(&bar, 3 * NS * slab);
+        mbar_expect_tx(&bar, (kV ? 3 : 2) * NS * slab);
 #pragma unroll
         for (int s = 0; s < NS; ++s) {
             tma_load_4d(smem + (0 * NS + s) * slab, &tm_q, &bar, 64 * s, h, n0, b);
             tma_load_4d(smem + (1 * NS + s) * slab, &tm_k, &bar, 64 * s, h, n0, b);
-            tma_load_4d(smem + (2 * NS + s) * slab, &tm_v, &bar, 64 * s, h, n0, b);
+            if (kV) tma_load_4d(smem + (2 * NS + s) * slab, &tm_v, &bar, 64 * s, h, n0, b);
         }
     }
     int axis[4], toff[4];
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
             const uint32_t off = sl * slab + i * 128 + ((c16 ^ (i & 7)) << 4);
             const uint4 qr = *reinterpret_cast<const uint4*>(smem + 0 * NS * slab + off);
             const uint4 kr = *reinterpret_cast<const uint4*>(smem + 1 * NS * slab + off);
-            const uint4 vr = *reinterpret_cast<const uint4*>(smem + 2 * NS * slab + off);
+            const uint4 vr = kV ? *reinterpret_cast<const uint4*>(smem + 2 * NS * slab + off) : make_uint4(0u, 0u, 0u, 0u);
             const int pt = n / HW, ph = (n / g.W) % g.H, pw = n % g.W;
             const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qr);
             const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
@@ -155,23 +156,23 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
                 const float c0 = static_cast<float>(ky0), c1 = static_cast<float>(ky1);
                 mq = fmaxf(mq, fmaxf(fabsf(a0), fabsf(a1)));
                 mk = fmaxf(mk, fmaxf(fabsf(c0), fabsf(c1)));
-                mv = fmaxf(mv, fmaxf(fabsf(vf.x), fabsf(vf.y)));
+                if (kV) mv = fmaxf(mv, fmaxf(fabsf(vf.x), fabsf(vf.y)));
                 m = fmaxf(m, fmaxf(fmaxf(mq, mk), mv));
                 const __half2 hq = __floats2half2_rn(a0, a1), hk = __floats2half2_rn(c0, c1),
                               hv = __floats2half2_rn(vf.x, vf.y);
                 qo2[u] = *reinterpret_cast<const uint32_t*>(&hq);
                 ko2[u] = *reinterpret_cast<const uint32_t*>(&hk);
-                vo2[u] = *reinterpret_cast<const uint32_t*>(&hv);
+                if (kV) vo2[u] = *reinterpret_cast<const uint32_t*>(&hv);
             }
             bad |= !(m <= 65504.0f);
             *reinterpret_cast<uint4*>(qh + dst) = qo;
             *reinterpret_cast<uint4*>(kh + dst) = ko;
-            *reinterpret_cast<uint4*>(vh + dst) = vo;
+            if (kV) *reinterpret_cast<uint4*>(vh + dst) = vo;
         } else {
             const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
             *reinterpret_cast<uint4*>(qh + dst) = z4;
             *reinterpret_cast<uint4*>(kh + dst) = z4;
-            *reinterpret_cast<uint4*>(vh + dst) = z4;
+            if (kV) *reinterpret_cast<uint4*>(vh + dst) = z4;
         }
     }
     // block maxima of |q^|, |k^|, |v| (non-negative floats order like their bit patterns)
@@ -229,25 +230,33 @@ size_t rope_pool_smem_bytes(const Geom& g) {
     return (tiles > red ? tiles : red) + 1024;
 }
 
-cudaError_t launch_rope_pool(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                             const double2* tab, const int2* pairs, const Geom& g, __half* qh, __half* kh,
-                             __half* vh, double* qbar, double* kbar, int* status, unsigned long long timeout_ns,
-                             cudaStream_t st) {
+template <int D, bool kV>
+static cudaError_t launch_rope_pool_t(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                      const double2* tab, const int2* pairs, const Geom& g, __half* qh, __half* kh,
+                                      __half* vh, double* qbar, double* kbar, int* status,
+                                      unsigned long long timeout_ns, cudaStream_t st) {
     dim3 grid(g.BH(), g.nb);
     const int sm = static_cast<int>(rope_pool_smem_bytes(g));
-    cudaError_t e;
-    if (g.D == 128) {
-        e = cudaFuncSetAttribute(rope_pool_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-        if (e != cudaSuccess) return e;
-        rope_pool_kernel<128><<<grid, 256, sm, st>>>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar, status,
-                                                     timeout_ns);
-    } else {
-        e = cudaFuncSetAttribute(rope_pool_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-        if (e != cudaSuccess) return e;
-        rope_pool_kernel<64><<<grid, 256, sm, st>>>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar, status,
-                                                    timeout_ns);
-    }
+    cudaError_t e = cudaFuncSetAttribute(rope_pool_kernel<D, kV>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    rope_pool_kernel<D, kV><<<grid, 256, sm, st>>>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar, status,
+                                                   timeout_ns);
     return cudaGetLastError();
+}
+
+cudaError_t launch_rope_pool(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                             const double2* tab, const int2* pairs, const Geom& g, bool write_v, __half* qh,
+                             __half* kh, __half* vh, double* qbar, double* kbar, int* status,
+                             unsigned long long timeout_ns, cudaStream_t st) {
+    if (g.D == 128)
+        return write_v ? launch_rope_pool_t<128, true>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar, status,
+                                                       timeout_ns, st)
+                       : launch_rope_pool_t<128, false>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar,
+                                                        status, timeout_ns, st);
+    return write_v ? launch_rope_pool_t<64, true>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar, status,
+                                                  timeout_ns, st)
+                   : launch_rope_pool_t<64, false>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar, status,
+                                                   timeout_ns, st);
 }
 
 // ------------------------------------------------------------------------------ select

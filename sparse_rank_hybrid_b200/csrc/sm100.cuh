@@ -148,10 +148,10 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int 
                                  ((((c >> 3) ^ (row & 7)) << 4) | ((c & 7) << 1)));
 }
 
-// Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulation, both K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(N) >> 3) << 17) |
-           ((static_cast<uint32_t>(M) >> 4) << 24);
+// Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulation, K-major unless stated.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major = false, bool b_mn_major = false) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((static_cast<uint32_t>(N) >> 3) << 17) | ((static_cast<uint32_t>(M) >> 4) << 24);
 }
 
 // ------------------------------------------------------------------------------- tcgen05 / TMEM
