@@ -395,7 +395,7 @@ def run_ours(args, w, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": replicas.job_throughput(job_flops, ms_per_step), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16 tensor-core operands, fp32 accumulate, fp64 selection",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16 (S = q^k^T) and bf16 (P.V) tensor-core operands, fp32 accumulate, fp64 selection",
         "data": "synthetic (seeded clustered-Gaussian bf16 q/k/v, A ~ N(0, 1/d_h)); inputs resident in HBM",
         "config": {"workload": base_w.name, "L": w.L, "heads": w.heads, "head_dim": w.head_dim, "rank": w.rank,
                    "block": w.block, "keep_frac": w.keep_frac, "keep_blocks": keep_blocks,
