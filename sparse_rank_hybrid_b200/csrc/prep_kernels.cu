@@ -37,17 +37,19 @@ cudaError_t launch_rope_table(double2* tab, int2* pairs, const RopeMeta& meta, i
 }
 
 // ------------------------------------------------------------------------------ rope_pool
-// One CTA per (query/key block, batch*head), two CTAs per SM.  Thread 0 brings the block's q, k (and,
-// with kV, v) rows of this head into shared memory with TMA (token-major 4D maps, 64-column boxes,
-// 128-B swizzle; tokens past L read as zero), so a whole block's tiles are in flight at once.  The fp16
-// v copy is only made for the backward kernels (kV); the forward's attention kernel reads v itself.  Then
-// thread t owns four consecutive rotary pairs (8 elements, 16 bytes) j = 4*(t % (D/8)) .. +3 and walks
-// the block's tokens with stride 256/(D/8); each fp16 output access is one 16-byte store, and the D/8
-// threads of a token cover its row, so a block's rows go out as one contiguous stretch per tensor.
-// The rotation and the block sums are fp64 so the selection scores are exact to ~1e-15 relative (the
-// top-k decision is made on them); the fp16 copies come from the same values.
-template <int D, bool kV>
-__global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
+// One CTA per (query/key block, batch*head): NTH = 256 threads and two CTAs per SM when the fp16 v copy
+// is made (kV), 128 threads and three CTAs per SM without it (the same shared memory then holds three
+// blocks in flight).  Thread 0 brings the block's q, k (and, with kV, v) rows of this head into shared
+// memory with TMA (token-major 4D maps, 64-column boxes, 128-B swizzle; tokens past L read as zero), so
+// a whole block's tiles are in flight at once.  The fp16 v copy is only made for the backward kernels;
+// the forward's attention kernel reads v itself.  Then thread t owns four consecutive rotary pairs (8
+// elements, 16 bytes) j = 4*(t % (D/8)) .. +3 and walks the block's tokens with stride NTH/(D/8); each
+// fp16 output access is one 16-byte store, and the D/8 threads of a token cover its row, so a block's
+// rows go out as one contiguous stretch per tensor.  The rotation and the block sums are fp64 so the
+// selection scores are exact to ~1e-15 relative (the top-k decision is made on them); the fp16 copies
+// come from the same values.
+template <int D, bool kV, int NTH>
+__global__ void __launch_bounds__(NTH, NTH == 256 ? 2 : 3) rope_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                            const __grid_constant__ CUtensorMap tm_k,
                                                            const __grid_constant__ CUtensorMap tm_v,
                                                            const double2* __restrict__ tab,
@@ -57,7 +59,7 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
                                                            double* __restrict__ kbar, int* status,
                                                            unsigned long long timeout_ns) {
     constexpr int Q4 = D / 8;          // threads per token row
-    constexpr int G = 256 / Q4;        // tokens in flight
+    constexpr int G = NTH / Q4;        // tokens in flight
     constexpr int NS = D / 64;         // 64-column slabs per row
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -222,11 +224,11 @@ __global__ void __launch_bounds__(256, 2) rope_pool_kernel(const __grid_constant
     }
 }
 
-// The q, k, v tiles, or the block-sum exchange that later reuses them ([256/(D/8)][4][D/2] fp64 =
-// 32 KB for any D), whichever is larger.
-size_t rope_pool_smem_bytes(const Geom& g) {
-    const size_t tiles = static_cast<size_t>(3) * g.block * g.D * 2;
-    const size_t red = static_cast<size_t>(256 / (g.D / 8)) * 4 * (g.D / 2) * 8;
+// The q, k (and v) tiles, or the block-sum exchange that later reuses them ([threads/(D/8)][4][D/2]
+// fp64 = threads/8 KB for any D), whichever is larger.
+size_t rope_pool_smem_bytes(const Geom& g, bool write_v, int threads) {
+    const size_t tiles = static_cast<size_t>(write_v ? 3 : 2) * g.block * g.D * 2;
+    const size_t red = static_cast<size_t>(threads / (g.D / 8)) * 4 * (g.D / 2) * 8;
     return (tiles > red ? tiles : red) + 1024;
 }
 
@@ -235,12 +237,14 @@ static cudaError_t launch_rope_pool_t(const CUtensorMap& tm_q, const CUtensorMap
                                       const double2* tab, const int2* pairs, const Geom& g, __half* qh, __half* kh,
                                       __half* vh, double* qbar, double* kbar, int* status,
                                       unsigned long long timeout_ns, cudaStream_t st) {
+    // without v: three CTAs of 128 threads per SM (more blocks in flight); with v: two of 256
+    constexpr int NTH = kV ? 256 : 128;
     dim3 grid(g.BH(), g.nb);
-    const int sm = static_cast<int>(rope_pool_smem_bytes(g));
-    cudaError_t e = cudaFuncSetAttribute(rope_pool_kernel<D, kV>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    const int sm = static_cast<int>(rope_pool_smem_bytes(g, kV, NTH));
+    cudaError_t e = cudaFuncSetAttribute(rope_pool_kernel<D, kV, NTH>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
-    rope_pool_kernel<D, kV><<<grid, 256, sm, st>>>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar, status,
-                                                   timeout_ns);
+    rope_pool_kernel<D, kV, NTH><<<grid, NTH, sm, st>>>(tm_q, tm_k, tm_v, tab, pairs, g, qh, kh, vh, qbar, kbar,
+                                                        status, timeout_ns);
     return cudaGetLastError();
 }
 
