@@ -668,7 +668,6 @@ slra_status fwd_impl(const slra_problem* p, const Derived& d, const void* q, con
     AttnArgs a;
     a.qh = w.qh;
     a.kh = w.kh;
-    a.vh = w.vh;
     a.idx = w.idx;
     a.keep = (branches & SLRA_BRANCH_SPARSE) ? g.keep : 0;
     a.q_raw = static_cast<const __nv_bfloat16*>(q);
@@ -1097,7 +1096,6 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
         std::memset(&a, 0, sizeof a);
         a.qh = w.qh;
         a.kh = w.kh;
-        a.vh = w.vh;
         a.idx = w.idx;
         a.keep = g.keep;
         a.q_raw = static_cast<const __nv_bfloat16*>(q);
@@ -1130,7 +1128,6 @@ slra_status bwd_impl(const slra_problem* p, const void* q, const void* k, const 
         std::memset(&a, 0, sizeof a);
         a.qh = w.qh;
         a.kh = w.kh;
-        a.vh = w.vh;
         a.idx = w.idx;
         a.keep = 0;
         a.q_raw = static_cast<const __nv_bfloat16*>(q);

@@ -171,9 +171,8 @@ struct AttnMaps {
 constexpr int kSbChunkBytes = 3 * 128 * 128;
 
 struct AttnArgs {
-    const __half* qh;   // head-major fp16 q^, k^, v rows [B*Hh][Lp][D]
-    const __half* kh;
-    const __half* vh;
+    const __half* qh;   // head-major fp16 q^, k^ rows [B*Hh][Lp][D] (read through the TMA maps; v tiles come
+    const __half* kh;   // from the caller's token-major v)
     const int32_t* idx;
     int keep;  // 0: no sparse branch
     const __nv_bfloat16* q_raw;
