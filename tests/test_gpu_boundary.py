@@ -9,6 +9,8 @@
     the latter also its S and z;
   - a NULL workspace (stream-ordered allocation inside the library) gives the caller-workspace output
     bit for bit and reports its device status through slra_get_device_status;
+  - the fp16 v copy in the workspace is written by the selection-only call and the training forward
+    (for the backward kernels) and left alone by the inference forward, which reads v itself;
 and the descriptor call is checked against the oracle once.  Inputs: the seeded generator.
 """
 import numpy as np
@@ -176,3 +178,32 @@ def test_overlapped_preparation_equals_serial(w):
         x.join()
     assert not errs, errs
     assert torch.equal(outs[0], ser) and torch.equal(outs[1], ser)
+
+
+@pytest.mark.parametrize("w", [W.TINY, EDGE_128], ids=lambda w: w.name)
+def test_v_copy_only_where_the_backward_reads_it(w):
+    """The inference forward reads v from the caller's tensor and leaves the workspace's fp16 v section
+    as it was; the selection-only call and the training forward write it (v in head-major order, rounded
+    to fp16, zero padded to whole blocks) for the backward kernels, as the header's workspace layout
+    states."""
+    import torch
+    _, t = _inputs(w)
+    p = slra.Problem.from_workload(w)
+    BH, Lp = w.batch * w.heads, w.nb * w.block
+    expect = torch.zeros((BH, Lp, w.head_dim), dtype=torch.float16, device="cuda")
+    expect[:, :w.L] = t["v"].permute(0, 2, 1, 3).reshape(BH, w.L, w.head_dim).half()
+
+    ws = slra.alloc_workspace(p)
+    slra.ws_view(p, ws, "vh").fill_(7.0)
+    slra.attn_fwd(p, t["q"], t["k"], t["v"], t["A"], workspace=ws)
+    assert slra.device_status(ws) == slra.OK
+    assert torch.all(slra.ws_view(p, ws, "vh") == 7.0)
+    slra.select_blocks(p, t["q"], t["k"], t["v"], workspace=ws)
+    assert slra.device_status(ws) == slra.OK
+    assert torch.equal(slra.ws_view(p, ws, "vh"), expect)
+
+    wst = torch.empty(slra.bwd_workspace_bytes(p), dtype=torch.uint8, device="cuda")
+    slra.ws_view(p, wst, "vh").fill_(7.0)
+    slra.attn_fwd_train(p, t["q"], t["k"], t["v"], t["A"], workspace=wst)
+    assert slra.device_status(wst) == slra.OK
+    assert torch.equal(slra.ws_view(p, wst, "vh"), expect)
